@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""MoE-layer forward throughput on B200 (tokens/s) and roofline fractions.
+
+    python bench.py [--gpus N --steps K --warmup W] [--config 2] [--alpha A]
+    python bench.py --impl reference ...      (the CPU oracle, timed on host cores)
+
+A step is one pass of the whole path (route, histogram/scan/permute, grouped
+SwiGLU, grouped down projection, combine) over one batch of T seeded synthetic
+tokens of the Mixtral-8x7B-shaped layer (T=512, H=4096, F=14336, E=8, top-2)
+unless --config says otherwise.  Inputs are resident in HBM; L2 is flushed
+(a 256 MiB write) between timed steps, outside the timed intervals.  Each step
+is timed with CUDA events on the stream the kernels run on, between every
+entry point, so the per-kernel times come from the same timed region.
+
+Multi-GPU: the path has no exchange step, so N GPUs run N independent
+replicas (one process per GPU, its own token batch); the only collectives are
+the barrier and the max-over-ranks of the elapsed time.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "MoE-layer fwd tokens/s at 1 B200; % of roofline (bf16 TC peak or HBM BW)"
+FLUSH_BYTES = 256 << 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--config", type=int, default=2)
+    p.add_argument("--alpha", type=float, default=None)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    p.add_argument("--ref-budget-s", type=float, default=150.0)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(args):
+    import synth
+    cfg = synth.CONFIGS[args.config]
+    if args.alpha is not None:
+        cfg = cfg.with_(alpha=args.alpha)
+    return cfg
+
+
+def config_json(cfg, extra=None):
+    d = {"workload": cfg.name + ("" if cfg.alpha in (0.0,) else "-alpha%g" % cfg.alpha), "T": cfg.T, "H": cfg.H,
+         "F": cfg.F, "E": cfg.E, "k": cfg.k, "C": cfg.C, "alpha": cfg.alpha, "seed": cfg.seed,
+         "l2": "flushed between timed steps (256 MiB write)"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def routing_stats(counts, C):
+    import numpy as np
+    n = np.asarray(counts, dtype=np.float64)
+    mean = n.mean()
+    gini = float(np.abs(n[:, None] - n[None, :]).sum() / (2 * len(n) ** 2 * mean)) if mean > 0 else 0.0
+    d = {"counts_min": int(n.min()), "counts_max": int(n.max()), "max_over_mean": float(n.max() / mean),
+         "gini": gini, "experts_touched": int((n > 0).sum())}
+    if C > 0:
+        d["overflow_frac"] = float(np.maximum(n - C, 0).sum() / n.sum())
+    return d
+
+
+def algorithmic_work(cfg, counts):
+    """Algorithmic bytes / FLOPs of each kernel from the actual routing.
+    Weights count once per touched expert; padded tile rows are not work."""
+    T, H, F, k = cfg.T, cfg.H, cfg.F, cfg.k
+    R = T * k
+    touched = sum(1 for c in counts if c > 0)
+    w = {}
+    w["swiglu_bytes"] = touched * 2 * H * F * 2 + R * H * 2 + R * F * 2
+    w["swiglu_flops"] = 2 * R * H * 2 * F
+    w["down_bytes"] = touched * F * H * 2 + R * F * 2 + R * H * 2
+    w["down_flops"] = 2 * R * F * H
+    w["route_bytes"] = T * H * 2 + H * cfg.E * 4 + T * cfg.E * 4 + T * k * 8
+    w["route_flops"] = 2 * T * H * cfg.E
+    w["permute_bytes"] = T * H * 2 + R * H * 2 + R * 4 * 4
+    w["combine_bytes"] = R * H * 2 + T * H * 2 + R * 8
+    w["layer_bytes"] = touched * 3 * H * F * 2 + 2 * T * H * 2 + H * cfg.E * 4
+    w["layer_flops"] = w["swiglu_flops"] + w["down_flops"] + w["route_flops"]
+    return w
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for_smi(torch, dev):
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return dev
+
+
+def cpu_baseline(cfg, L, budget_s):
+    """The CPU oracle as it stands, single-threaded, on the first S tokens of
+    the same batch (route, dispatch, experts, combine), S sized to the budget."""
+    import numpy as np
+
+    from oracle import Oracle
+    orc = Oracle()
+
+    def run(S):
+        x = L.x[:S]
+        t0 = time.perf_counter()
+        orc.forward(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, cfg.k, C=cfg.C, capped=cfg.C > 0)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    S = int(max(1, min(cfg.T, budget_s / max(t1, 1e-6))))
+    dt = run(S) if S > 1 else t1
+    return {"value": S / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d of the %d tokens of the same seeded batch through the whole oracle forward "
+                      "(single-threaded C, fp64 accumulation); %.1f s" % (S, cfg.T, dt)}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    from oracle import Oracle
+    cfg = workload(args)
+    L = synth.make_layer(cfg)
+    orc = Oracle()
+
+    def step(S):
+        t0 = time.perf_counter()
+        orc.forward(L.x[:S], L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, cfg.k, C=cfg.C, capped=cfg.C > 0)
+        return time.perf_counter() - t0
+
+    t1 = step(1)
+    per_step = args.ref_budget_s / max(1, args.steps + args.warmup)
+    S = int(max(1, min(cfg.T, per_step / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        step(S)
+    total = 0.0
+    for _ in range(args.steps):
+        total += step(S)
+    value = S * args.steps / total
+    sample = ("first %d of the %d tokens of the seeded batch per step through the whole oracle forward "
+              "(single-threaded C, fp64 accumulation)" % (S, cfg.T))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, {"tokens_per_step": S}),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import grouped_expert_gemm_router_b200 as moe
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    cfg = workload(args)
+    t0 = time.time()
+    L = synth.make_layer(cfg)
+    x_rank = synth.x_tokens(cfg, seed_offset=rank) if rank else L.x  # each replica its own tokens
+    log("rank %d: generated %s in %.1f s" % (rank, cfg.name, time.time() - t0))
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=cfg.C > 0)
+    b = moe.alloc_buffers(shape, dev)
+    b.update(x=dev_bf16(x_rank), w_router=torch.from_numpy(L.w_router).to(dev),
+             bias=None if L.bias is None else torch.from_numpy(L.bias).to(dev),
+             w_gate=dev_bf16(L.w_gate), w_up=dev_bf16(L.w_up), w_down=dev_bf16(L.w_down))
+    ws = b["ws"]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_events(ev):
+        ev[0].record(stream)
+        moe.moe_route(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"], ws, stream)
+        ev[1].record(stream)
+        moe.moe_permute(shape, b["x"], b["topk_idx"], b["expert_counts"], b["expert_offsets"], b["src_token"],
+                        b["dest_row"], b["x_perm"], ws, stream)
+        ev[2].record(stream)
+        moe.moe_grouped_swiglu(shape, b["x_perm"], b["w_gate"], b["w_up"], b["h"], ws, stream)
+        ev[3].record(stream)
+        moe.moe_grouped_down(shape, b["h"], b["w_down"], b["y"], ws, stream)
+        ev[4].record(stream)
+        moe.moe_combine(shape, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
+        ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # warm-up
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step_events(wev)
+    torch.cuda.synchronize(dev)
+    status = moe.moe_read_status(ws, stream)
+    if status & ~moe.MOE_DEV_NAN_LOGIT:
+        raise RuntimeError("device status %#x after warm-up" % status)
+
+    # timed region
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    sampler = ClockSampler(gpu_id_for_smi(torch, local))
+    barrier()
+    sampler.start()
+    time.sleep(0.15)  # let the sampler take its first reading
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        step_events(evs[i])
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(K)])  # ms
+    step_ms = seg.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = moe.moe_read_status(ws, stream)
+
+    counts = b["expert_counts"].cpu().numpy()
+    work = algorithmic_work(cfg, counts)
+    peaks, peak_src = load_peaks()
+    kmean = seg.mean(axis=0) * 1e-3  # s per launch
+    names = ["route", "permute", "grouped_swiglu", "grouped_down", "combine"]
+
+    # whole layer captured in a CUDA graph (same work; graph replays timed one by one)
+    graph_ms = None
+    try:
+        args_c = moe.forward_args(b)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+            moe.moe_forward(shape, b, ws, args=args_c)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(3):
+            flush.zero_()
+            g.replay()
+        for i in range(K):
+            flush.zero_()
+            gev[i][0].record(stream)
+            g.replay()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = float(np.mean([a.elapsed_time(c) for a, c in gev]))
+        del g
+    except Exception as e:  # reported, not fatal: the eager numbers stand
+        log("graph timing skipped: %r" % (e,))
+
+    # end to end: pinned host tokens in, layer, host result out, each step
+    x_host = torch.from_numpy(np.ascontiguousarray(x_rank).view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    args_e = moe.forward_args(b)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(-3, K):
+        flush.zero_()
+        if i >= 0:
+            eev[i][0].record(stream)
+        b["x"].copy_(x_host, non_blocking=True)
+        moe.moe_forward(shape, b, ws, stream, args=args_e)
+        out_host.copy_(b["out"], non_blocking=True)
+        if i >= 0:
+            eev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.sum([a.elapsed_time(c) for a, c in eev]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    result = None
+    if rank == 0:
+        tokens = cfg.T * K * world
+        value = tokens / (total_ms * 1e-3)
+        # dominant kernel: the fused gate+up SwiGLU grouped GEMM
+        t_sw = kmean[2]
+        t_hbm = work["swiglu_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = work["swiglu_flops"] / (peaks["bf16_tflops"] * 1e12)
+        if t_hbm >= t_tc:
+            achieved = work["swiglu_bytes"] / t_sw / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"]}
+        else:
+            achieved = work["swiglu_flops"] / t_sw / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"]}
+        roof.update({"traffic": None, "kernel": "k_grouped_gemm<0> (moe_grouped_swiglu)",
+                     "algorithmic_bytes": work["swiglu_bytes"], "algorithmic_flops": work["swiglu_flops"],
+                     "peak_source": peak_src})
+        layer_t = max(work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                      work["layer_flops"] / (peaks["bf16_tflops"] * 1e12))
+        kernels = {}
+        for nm, t in zip(names, kmean):
+            kernels[nm + "_us"] = t * 1e6
+        kernels["grouped_swiglu_GBps"] = work["swiglu_bytes"] / kmean[2] / 1e9
+        kernels["grouped_swiglu_TFLOPs"] = work["swiglu_flops"] / kmean[2] / 1e12
+        kernels["grouped_down_GBps"] = work["down_bytes"] / kmean[3] / 1e9
+        kernels["grouped_down_TFLOPs"] = work["down_flops"] / kmean[3] / 1e12
+        kernels["grouped_down_hbm_frac"] = work["down_bytes"] / kmean[3] / 1e9 / peaks["hbm_gbs"]
+        kernels["permute_GBps"] = work["permute_bytes"] / kmean[1] / 1e9
+        kernels["combine_GBps"] = work["combine_bytes"] / kmean[4] / 1e9
+        kernels["route_TFLOPs_fp32"] = work["route_flops"] / kmean[0] / 1e12
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu"}),
+            "roofline": roof,
+            "layer_roofline": {"frac": layer_t / (total_ms * 1e-3 / K), "roofline_us": layer_t * 1e6,
+                               "bound": "hbm" if work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
+                               >= work["layer_flops"] / (peaks["bf16_tflops"] * 1e12) else "tensor"},
+            "kernels": kernels,
+            "graph_ms_per_step": graph_ms,
+            "e2e": {"value": cfg.T * K * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+            "gpu_launches": 7 * K,
+            "clocks": clocks,
+            "routing": routing_stats(counts, cfg.C),
+            "device_status": status,
+            "wall_s_timed_region": wall,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(cfg, L, args.cpu_budget_s)
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

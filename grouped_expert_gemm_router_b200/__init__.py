@@ -1,0 +1,235 @@
+"""Python binding of the B200 MoE-layer forward library (include/moe.h).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libmoe_b200.so``.  Functions carry the C names; tensors are torch CUDA
+tensors (their ``data_ptr()`` is passed through), ``stream`` defaults to the
+current torch stream.  There is no fallback: if the library is missing or the
+device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_DEV_SCAN_TIMEOUT = 0x1
+MOE_DEV_GEMM_TIMEOUT = 0x2
+MOE_DEV_BAD_EXPERT = 0x4
+MOE_DEV_NAN_LOGIT = 0x8
+MOE_DEV_BAD_ROW = 0x10
+MOE_FLAG_CAPACITY = 0x1
+MOE_FLAG_LOGITS_IN = 0x2
+MOE_FLAG_TEST_STALL_SCAN = 0x40000000
+
+# Every symbol include/moe.h declares (the CPU tests check the library exports each).
+ABI_FUNCTIONS = (
+    "moe_permuted_rows", "moe_workspace_bytes", "moe_workspace_layout", "moe_workspace_init", "moe_route",
+    "moe_permute", "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward", "moe_read_status",
+    "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version",
+)
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("F", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("C", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+    def __repr__(self):
+        return "MoeShape(T=%d, H=%d, F=%d, E=%d, k=%d, C=%d, flags=%#x)" % (
+            self.T, self.H, self.F, self.E, self.k, self.C, self.flags)
+
+
+class MoeForwardArgs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "x", "w_router", "bias", "w_gate", "w_up", "w_down", "logits", "topk_idx", "topk_w", "expert_counts",
+        "expert_offsets", "src_token", "dest_row", "x_perm", "h", "y", "out")]
+
+
+class MoeWsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "total", "status", "num_tiles", "total_spill", "cap_cnt", "spill_cnt", "spill_off", "order",
+        "grp_tile_start", "tile_map")] + [("max_tiles", ctypes.c_int32), ("tile_rows", ctypes.c_int32)]
+
+
+class MoeError(RuntimeError):
+    pass
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and declare the C ABI.  Raises if the library is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise MoeError("CUDA library %s is missing: build it with "
+                       "`python -m grouped_expert_gemm_router_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, sp = ctypes.c_void_p, ctypes.POINTER(MoeShape)
+    st = ctypes.c_int
+    lib.moe_permuted_rows.argtypes = [sp]
+    lib.moe_permuted_rows.restype = ctypes.c_int64
+    lib.moe_workspace_bytes.argtypes = [sp]
+    lib.moe_workspace_bytes.restype = ctypes.c_size_t
+    lib.moe_workspace_layout.argtypes = [sp, ctypes.POINTER(MoeWsLayout)]
+    lib.moe_workspace_layout.restype = st
+    lib.moe_workspace_init.argtypes = [sp, vp, vp]
+    lib.moe_workspace_init.restype = st
+    lib.moe_route.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.moe_route.restype = st
+    lib.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.moe_permute.restype = st
+    lib.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp]
+    lib.moe_grouped_swiglu.restype = st
+    lib.moe_grouped_down.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.moe_grouped_down.restype = st
+    lib.moe_combine.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.moe_combine.restype = st
+    lib.moe_forward.argtypes = [sp, ctypes.POINTER(MoeForwardArgs), vp, vp]
+    lib.moe_forward.restype = st
+    lib.moe_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+    lib.moe_read_status.restype = st
+    lib.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.moe_set_wait_timeout_ns.restype = None
+    lib.moe_status_string.argtypes = [st]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_last_error_string.argtypes = []
+    lib.moe_last_error_string.restype = ctypes.c_char_p
+    lib.moe_version.argtypes = []
+    lib.moe_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def make_shape(T, H, F, E, k, C=0, capacity=False, logits_in=False, flags=0) -> MoeShape:
+    f = flags | (MOE_FLAG_CAPACITY if capacity else 0) | (MOE_FLAG_LOGITS_IN if logits_in else 0)
+    return MoeShape(T, H, F, E, k, C, f)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc, what):
+    if rc != MOE_OK:
+        lib = load_library()
+        raise MoeError("%s failed: %s (%s)" % (what, lib.moe_status_string(rc).decode(),
+                                               lib.moe_last_error_string().decode()))
+
+
+def moe_permuted_rows(shape: MoeShape) -> int:
+    return int(load_library().moe_permuted_rows(ctypes.byref(shape)))
+
+
+def moe_workspace_bytes(shape: MoeShape) -> int:
+    return int(load_library().moe_workspace_bytes(ctypes.byref(shape)))
+
+
+def moe_workspace_layout(shape: MoeShape) -> MoeWsLayout:
+    out = MoeWsLayout()
+    _check(load_library().moe_workspace_layout(ctypes.byref(shape), ctypes.byref(out)), "moe_workspace_layout")
+    return out
+
+
+def moe_workspace_init(shape, ws, stream=None):
+    _check(load_library().moe_workspace_init(ctypes.byref(shape), _ptr(ws), _stream(stream)), "moe_workspace_init")
+
+
+def moe_route(shape, x, w_router, bias, logits, topk_idx, topk_w, ws, stream=None):
+    _check(load_library().moe_route(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits),
+                                    _ptr(topk_idx), _ptr(topk_w), _ptr(ws), _stream(stream)), "moe_route")
+
+
+def moe_permute(shape, x, topk_idx, expert_counts, expert_offsets, src_token, dest_row, x_perm, ws, stream=None):
+    _check(load_library().moe_permute(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts),
+                                      _ptr(expert_offsets), _ptr(src_token), _ptr(dest_row), _ptr(x_perm),
+                                      _ptr(ws), _stream(stream)), "moe_permute")
+
+
+def moe_grouped_swiglu(shape, x_perm, w_gate, w_up, h, ws, stream=None):
+    _check(load_library().moe_grouped_swiglu(ctypes.byref(shape), _ptr(x_perm), _ptr(w_gate), _ptr(w_up), _ptr(h),
+                                             _ptr(ws), _stream(stream)), "moe_grouped_swiglu")
+
+
+def moe_grouped_down(shape, h, w_down, y, ws, stream=None):
+    _check(load_library().moe_grouped_down(ctypes.byref(shape), _ptr(h), _ptr(w_down), _ptr(y), _ptr(ws),
+                                           _stream(stream)), "moe_grouped_down")
+
+
+def moe_combine(shape, y, dest_row, topk_w, out, stream=None):
+    _check(load_library().moe_combine(ctypes.byref(shape), _ptr(y), _ptr(dest_row), _ptr(topk_w), _ptr(out),
+                                      _stream(stream)), "moe_combine")
+
+
+def forward_args(bufs: dict) -> MoeForwardArgs:
+    a = MoeForwardArgs()
+    for name, _ in MoeForwardArgs._fields_:
+        setattr(a, name, _ptr(bufs.get(name)))
+    return a
+
+
+def moe_forward(shape, bufs: dict, ws, stream=None, args: MoeForwardArgs | None = None):
+    """bufs: dict with the moe_forward_args field names -> tensors (or None)."""
+    a = args if args is not None else forward_args(bufs)
+    _check(load_library().moe_forward(ctypes.byref(shape), ctypes.byref(a), _ptr(ws), _stream(stream)), "moe_forward")
+
+
+def moe_read_status(ws, stream=None, clear=True) -> int:
+    v = ctypes.c_uint32(0)
+    _check(load_library().moe_read_status(_ptr(ws), _stream(stream), ctypes.byref(v), int(bool(clear))),
+           "moe_read_status")
+    return int(v.value)
+
+
+def moe_set_wait_timeout_ns(ns: int) -> None:
+    load_library().moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_version() -> int:
+    return int(load_library().moe_version())
+
+
+def alloc_buffers(shape: MoeShape, device="cuda"):
+    """Allocate (with torch) every intermediate/output buffer of moe_forward
+    and a zeroed workspace.  Returns a dict keyed like moe_forward_args plus
+    'ws'."""
+    import torch
+    T, H, F, E, k = shape.T, shape.H, shape.F, shape.E, shape.k
+    P = moe_permuted_rows(shape)
+    if P < 0:
+        raise MoeError("unsupported shape %r" % (shape,))
+    dev = torch.device(device)
+    b = dict(
+        logits=torch.empty((T, E), dtype=torch.float32, device=dev),
+        topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+        topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+        expert_counts=torch.empty((E,), dtype=torch.int32, device=dev),
+        expert_offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+        src_token=torch.empty((P,), dtype=torch.int32, device=dev),
+        dest_row=torch.empty((T * k,), dtype=torch.int32, device=dev),
+        x_perm=torch.empty((P, H), dtype=torch.bfloat16, device=dev),
+        h=torch.empty((P, F), dtype=torch.bfloat16, device=dev),
+        y=torch.empty((P, H), dtype=torch.bfloat16, device=dev),
+        out=torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+    )
+    ws = torch.empty((moe_workspace_bytes(shape) + 255) // 256 * 256, dtype=torch.uint8, device=dev)
+    moe_workspace_init(shape, ws)
+    b["ws"] = ws
+    return b

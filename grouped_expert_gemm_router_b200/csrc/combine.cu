@@ -1,0 +1,65 @@
+// Step 5: weighted unpermutation ("TritonMoE" verdict page, arXiv 2605.23911,
+// referee report summary):
+//   out[t] = bf16( sum_{j<k} topk_w[t,j] * y[dest_row[t*k+j]] )
+// summed in fp32 in slot order with each product and each sum rounded on its
+// own (no fused multiply-add), so that given the same y the result is
+// bit-identical to a plain sequential fp32 loop.
+//
+// HBM-bound gather: each thread owns 8 consecutive features (one 16-byte
+// vector) of one token, reads the k expert rows with 16-byte loads and writes
+// one 16-byte vector.  Grid: tokens x ceil(H/8 / 256) blocks of 256 threads.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4 &q, float (&v)[8]) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const int *__restrict__ dest_row,
+                                                 const float *__restrict__ w, uint4 *__restrict__ out, int k, int H8,
+                                                 int P) {
+    const int t = blockIdx.x;
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;
+    if (v >= H8) return;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const int r = __ldg(dest_row + (size_t)t * k + j);
+        if ((unsigned)r >= (unsigned)P) continue;  // only after an earlier device error
+        const float wj = __ldg(w + (size_t)t * k + j);
+        float yv[8];
+        unpack8(__ldg(y + (size_t)r * H8 + v), yv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, yv[i]));
+    }
+    uint4 o;
+    __nv_bfloat162 *ob = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ob[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    out[(size_t)t * H8 + v] = o;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
+                           cudaStream_t stream) {
+    const int H8 = s.H / 8;
+    const dim3 grid((unsigned)s.T, (unsigned)((H8 + 255) / 256));
+    const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, (s.flags & MOE_FLAG_CAPACITY) != 0);
+    k_combine<<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

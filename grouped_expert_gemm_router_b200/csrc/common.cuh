@@ -1,0 +1,258 @@
+// Shared definitions of the sm_100a MoE kernels: workspace layout, tile
+// descriptors, and thin inline-PTX wrappers for mbarrier, TMA (bulk tensor
+// copies) and the 5th-generation tensor cores (tcgen05 + tensor memory).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ tiling --
+constexpr int kScanChunk = 2048;     // routed pairs per histogram / rank block
+constexpr int kScanThreads = 256;
+constexpr int kMaxExperts = 256;
+constexpr int kTileRows = 256;       // largest UMMA N: permuted rows per GEMM tile
+constexpr int kPieceAlign = 16;      // rows of one B-operand TMA box
+
+// Scan look-back state: a 64-bit word per (block, expert): flag << 32 | value.
+constexpr uint32_t kFlagAggregate = 1u;
+constexpr uint32_t kFlagPrefix = 2u;
+
+// ---------------------------------------------------------------- workspace --
+// Byte offsets inside the caller's workspace.  The "reset" range (ticket +
+// look-back state) is zeroed by a memset node before every histogram launch;
+// the status word lives outside it and is sticky.
+struct WsLayout {
+    size_t status, num_tiles, total_spill;
+    size_t counts, offsets, cap_cnt, spill_cnt, spill_off, order, grp_tile_start;
+    size_t chunk_excl;            // int32[nchunks * E] exclusive per-block prefix
+    size_t reset_begin;           // start of the memset range
+    size_t ticket;                // uint32 dynamic block ticket
+    size_t scan_state;            // uint64[nchunks * E]
+    size_t reset_end;
+    size_t tile_map;              // int4[max_tiles]
+    size_t total;
+    int nchunks, max_tiles;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
+    if (!capped) return (int64_t)T * k;
+    return (int64_t)E * C + (int64_t)k * (T > C ? T - C : 0);
+}
+
+// Upper bound on the tiles the schedule builder emits.  Per expert, every
+// tile but the first holds only overflow rows and closes only when full, so
+// an expert needs at most 2 + spill/kTileRows tiles (uncapped: 1 +
+// n_e/kTileRows).  Summed: 2E + P/kTileRows.
+inline int max_tiles_for(int64_t P, int E) { return (int)(2 * (int64_t)E + P / kTileRows + 1); }
+
+inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
+    WsLayout L{};
+    const int64_t R = (int64_t)T * k;
+    const int64_t P = permuted_rows(T, E, k, C, capped);
+    L.nchunks = (int)((R + kScanChunk - 1) / kScanChunk);
+    L.max_tiles = max_tiles_for(P, E);
+    size_t o = 0;
+    L.status = o;
+    L.num_tiles = o + 4;
+    L.total_spill = o + 8;
+    o += 256;
+    auto arr = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.counts = arr(4 * (size_t)E);
+    L.offsets = arr(4 * (size_t)(E + 1));
+    L.cap_cnt = arr(4 * (size_t)E);
+    L.spill_cnt = arr(4 * (size_t)E);
+    L.spill_off = arr(4 * (size_t)(E + 1));
+    L.order = arr(4 * (size_t)E);
+    L.grp_tile_start = arr(4 * (size_t)(E + 1));
+    L.chunk_excl = arr(4 * (size_t)L.nchunks * E);
+    L.reset_begin = o;
+    L.ticket = o;
+    o += 256;
+    L.scan_state = arr(8 * (size_t)L.nchunks * E);
+    L.reset_end = o;
+    L.tile_map = arr(16 * (size_t)L.max_tiles);
+    L.total = o;
+    return L;
+}
+
+// Device-side view of the workspace (pointers resolved on the host).
+struct WsPtrs {
+    uint32_t *status;
+    int *num_tiles, *total_spill;
+    int *counts, *offsets, *cap_cnt, *spill_cnt, *spill_off, *order, *grp_tile_start;
+    int *chunk_excl;
+    uint32_t *ticket;
+    unsigned long long *scan_state;
+    int4 *tile_map;
+    int nchunks, max_tiles;
+};
+
+inline WsPtrs ws_ptrs(void *ws, const WsLayout &L) {
+    char *b = (char *)ws;
+    WsPtrs p;
+    p.status = (uint32_t *)(b + L.status);
+    p.num_tiles = (int *)(b + L.num_tiles);
+    p.total_spill = (int *)(b + L.total_spill);
+    p.counts = (int *)(b + L.counts);
+    p.offsets = (int *)(b + L.offsets);
+    p.cap_cnt = (int *)(b + L.cap_cnt);
+    p.spill_cnt = (int *)(b + L.spill_cnt);
+    p.spill_off = (int *)(b + L.spill_off);
+    p.order = (int *)(b + L.order);
+    p.grp_tile_start = (int *)(b + L.grp_tile_start);
+    p.chunk_excl = (int *)(b + L.chunk_excl);
+    p.ticket = (uint32_t *)(b + L.ticket);
+    p.scan_state = (unsigned long long *)(b + L.scan_state);
+    p.tile_map = (int4 *)(b + L.tile_map);
+    p.nchunks = L.nchunks;
+    p.max_tiles = L.max_tiles;
+    return p;
+}
+
+// ------------------------------------------------------------ device helpers --
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// ---- mbarrier ----
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase of parity `parity` to complete.  Gives up (returns
+// false) when *abort becomes non-zero or after timeout_ns; the clock is only
+// read once the wait has already spun for a while.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                                  volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t deadline = 0;
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((spin & 255u) == 0) {
+            if (*abort) return false;
+            const uint64_t now = globaltimer_ns();
+            if (deadline == 0) deadline = now + timeout_ns;
+            else if (now > deadline) return false;
+        }
+    }
+}
+
+// ---- TMA: 2-D tiled bulk tensor load into this CTA's shared memory ----
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---- tcgen05: tensor memory and the 5th-generation MMA ----
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Arrives once on `bar` when every tcgen05.mma issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 lanes x 32 bits, 16 consecutive columns: register i <- column (col + i)
+// of the lane this thread maps to (warp w reads lanes 32*(w%4) .. +31).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a tcgen05 operand laid out with the
+// 128-byte swizzle: bits 0-13 start address >> 4, 16-29 leading-dimension
+// byte offset >> 4, 32-45 stride-dimension byte offset >> 4, 46-47 version
+// (1 on sm_100), 61-63 layout (2 = SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+#endif  // __CUDACC__
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
+// 4-5 = 1), A and B bf16 (bits 7-9 and 10-12 = 1), A/B major-ness (bit 15 /
+// 16: 0 = K-major, 1 = MN-major), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+}  // namespace moe

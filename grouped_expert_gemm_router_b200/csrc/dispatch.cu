@@ -1,0 +1,380 @@
+// Steps 2-3: per-expert histogram, exclusive scan and stable permutation of
+// the routed (token, slot) pairs into expert-contiguous order ("TritonMoE"
+// verdict page, arXiv 2605.23911: tokens reordered onto experts), with the
+// optional capacity-plus-compacted-overflow layout ("Cap-and-Spill" critique,
+// juhe.plus, section "Cap-and-Spill"), and the device-built tile schedule of
+// the grouped GEMMs.
+//
+// k_hist_scan  one pass over topk_idx.  Each block takes a ticket (its block
+//              index in launch-independent order), histograms its chunk of
+//              2048 pairs in shared memory and resolves, per expert, the count
+//              of that expert in all earlier chunks by decoupled look-back
+//              over per-(chunk, expert) flag words.  The block holding the
+//              last chunk owns the totals and builds the per-expert offsets,
+//              the capacity/overflow offsets and the GEMM tile schedule, all
+//              on the device: nothing goes back to the host.
+// k_rank       each block re-reads its chunk and ranks every pair among the
+//              pairs of its expert (stable: earlier flat index = lower rank),
+//              using warp match masks and per-warp counts, and writes
+//              dest_row / src_token.
+// k_gather     x_perm[row] = x[src_token[row]] with 16-byte loads and stores,
+//              zero rows for unfilled capacity slots.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+struct ScanArgs {
+    const int *topk_idx;
+    int T, E, k, C, capped, R;
+    int stall_first_block;  // test hook: block 0 never publishes
+    unsigned long long timeout_ns;
+    int *counts_out;   // caller's expert_counts [E]
+    int *offsets_out;  // caller's expert_offsets [E+1]
+    WsPtrs ws;
+};
+
+__device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
+
+// Tiles of one expert: its row segments (uncapped: one; capacity layout:
+// capacity slots then overflow) are cut into pieces and packed into tiles of
+// at most kTileRows rows, each piece starting on a 16-row boundary of the
+// tile and at most two pieces per tile.  Emits if `out` is non-null; returns
+// the tile count.
+__device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_start, int seg1_len, int4 *out) {
+    int ntiles = 0, used = 0, np = 0;
+    int p_start[2] = {0, 0}, p_len[2] = {0, 0};
+    const int seg_start[2] = {seg0_start, seg1_start};
+    const int seg_len[2] = {seg0_len, seg1_len};
+    for (int s = 0; s < 2; ++s) {
+        int start = seg_start[s], len = seg_len[s];
+        while (len > 0) {
+            if (used == kTileRows || np == 2) {
+                if (out) out[ntiles] = make_int4(e, p_start[0], p_len[0] | (p_len[1] << 16), p_start[1]);
+                ++ntiles;
+                used = 0;
+                np = 0;
+                p_len[1] = 0;
+                p_start[1] = 0;
+            }
+            const int take = len < kTileRows - used ? len : kTileRows - used;
+            p_start[np] = start;
+            p_len[np] = take;
+            ++np;
+            used += round16(take);
+            start += take;
+            len -= take;
+        }
+    }
+    if (np > 0) {
+        if (out) out[ntiles] = make_int4(e, p_start[0], p_len[0] | (p_len[1] << 16), p_start[1]);
+        ++ntiles;
+    }
+    return ntiles;
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
+    __shared__ int hist[kMaxExperts];
+    __shared__ int s_scan[kMaxExperts + 1];
+    __shared__ int s_aux[kMaxExperts + 1];
+    __shared__ int s_chunk, s_bad, s_timeout;
+    const int tid = threadIdx.x, E = a.E;
+    if (tid == 0) {
+        s_chunk = (int)atomicAdd(a.ws.ticket, 1u);
+        s_bad = 0;
+        s_timeout = 0;
+    }
+    for (int e = tid; e < E; e += kScanThreads) hist[e] = 0;
+    __syncthreads();
+    const int chunk = s_chunk;
+    const int begin = chunk * kScanChunk;
+    const int end = min(a.R, begin + kScanChunk);
+    for (int i = begin + tid; i < end; i += kScanThreads) {
+        const int e = a.topk_idx[i];
+        if ((unsigned)e < (unsigned)E)
+            atomicAdd(&hist[e], 1);
+        else
+            s_bad = 1;
+    }
+    __syncthreads();
+    if (tid == 0 && s_bad) atomicOr(a.ws.status, MOE_DEV_BAD_EXPERT);
+
+    // Decoupled look-back, one thread per expert.
+    const bool last = (chunk == a.ws.nchunks - 1);
+    for (int e = tid; e < E; e += kScanThreads) {
+        const int agg = hist[e];
+        unsigned long long *mine = a.ws.scan_state + (size_t)chunk * E + e;
+        const bool publish = !(a.stall_first_block && chunk == 0);
+        int excl = 0;
+        if (chunk == 0) {
+            if (publish) st_release_u64(mine, ((unsigned long long)kFlagPrefix << 32) | (uint32_t)agg);
+        } else {
+            st_release_u64(mine, ((unsigned long long)kFlagAggregate << 32) | (uint32_t)agg);
+            int p = chunk - 1;
+            uint64_t deadline = 0;
+            uint32_t spins = 0;
+            while (p >= 0) {
+                const unsigned long long v = ld_acquire_u64(a.ws.scan_state + (size_t)p * E + e);
+                const uint32_t flag = (uint32_t)(v >> 32);
+                if (flag == 0u) {
+                    if ((++spins & 63u) == 0) {
+                        const uint64_t now = globaltimer_ns();
+                        if (deadline == 0) {
+                            deadline = now + a.timeout_ns;
+                        } else if (now > deadline) {
+                            s_timeout = 1;
+                            break;
+                        }
+                    }
+                    __nanosleep(64);
+                    continue;
+                }
+                excl += (int)(uint32_t)v;
+                if (flag == kFlagPrefix) break;
+                --p;
+            }
+            st_release_u64(mine, ((unsigned long long)kFlagPrefix << 32) | (uint32_t)(excl + agg));
+        }
+        a.ws.chunk_excl[(size_t)chunk * E + e] = excl;
+        if (last) hist[e] = excl + agg;  // totals
+    }
+    __syncthreads();
+    if (tid == 0 && s_timeout) atomicOr(a.ws.status, MOE_DEV_SCAN_TIMEOUT);
+    if (!last) return;
+
+    // ---- the block with the last chunk: offsets, capacity layout, schedule ----
+    const int C = a.C;
+    if (tid == 0) {
+        int run = 0, spill = 0;
+        for (int e = 0; e < E; ++e) {
+            s_scan[e] = run;
+            run += hist[e];
+            s_aux[e] = spill;
+            const int cap = a.capped ? min(hist[e], C) : hist[e];
+            spill += hist[e] - cap;
+        }
+        s_scan[E] = run;
+        s_aux[E] = spill;
+        *a.ws.total_spill = spill;
+    }
+    __syncthreads();
+    for (int e = tid; e <= E; e += kScanThreads) {
+        a.offsets_out[e] = s_scan[e];
+        a.ws.offsets[e] = s_scan[e];
+        a.ws.spill_off[e] = s_aux[e];
+        if (e < E) {
+            const int n = hist[e];
+            const int cap = a.capped ? min(n, C) : n;
+            a.counts_out[e] = n;
+            a.ws.counts[e] = n;
+            a.ws.cap_cnt[e] = cap;
+            a.ws.spill_cnt[e] = n - cap;
+        }
+    }
+    // Expert order: descending count, ties by index (largest work first).
+    __shared__ int s_rank[kMaxExperts];
+    __shared__ int s_order[kMaxExperts];
+    __shared__ int s_ntiles[kMaxExperts];
+    for (int e = tid; e < E; e += kScanThreads) {
+        const int n = hist[e];
+        int r = 0;
+        for (int f = 0; f < E; ++f) {
+            const int m = hist[f];
+            r += (m > n) || (m == n && f < e);
+        }
+        s_rank[e] = r;
+        s_order[r] = e;
+        a.ws.order[r] = e;
+        int nt = 0;
+        if (n > 0) {
+            if (a.capped) {
+                const int cap = min(n, C);
+                nt = pack_expert_tiles(e, e * C, cap, E * C + s_aux[e], n - cap, nullptr);
+            } else {
+                nt = pack_expert_tiles(e, s_scan[e], n, 0, 0, nullptr);
+            }
+        }
+        s_ntiles[e] = nt;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // First tile of each expert in schedule order; s_scan held the
+        // offsets, which are in global memory by now.
+        int run = 0;
+        for (int g = 0; g < E; ++g) {
+            s_scan[g] = run;
+            run += s_ntiles[s_order[g]];
+        }
+        s_scan[E] = run;
+        *a.ws.num_tiles = run;
+    }
+    __syncthreads();
+    for (int g = tid; g <= E; g += kScanThreads) a.ws.grp_tile_start[g] = s_scan[g];
+    for (int e = tid; e < E; e += kScanThreads) {
+        const int n = hist[e];
+        if (n == 0) continue;
+        int4 *dst = a.ws.tile_map + s_scan[s_rank[e]];
+        if (a.capped) {
+            const int cap = min(n, C);
+            pack_expert_tiles(e, e * C, cap, E * C + a.ws.spill_off[e], n - cap, dst);
+        } else {
+            pack_expert_tiles(e, a.ws.offsets[e], n, 0, 0, dst);
+        }
+    }
+}
+
+struct RankArgs {
+    const int *topk_idx;
+    int E, k, C, capped, R, P;
+    int *dest_row;
+    int *src_token;
+    WsPtrs ws;
+};
+
+__global__ void __launch_bounds__(kScanThreads) k_rank(RankArgs a) {
+    constexpr int W = kScanThreads / 32;
+    __shared__ int running[kMaxExperts];
+    __shared__ int wcnt[W][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, E = a.E;
+    const int chunk = blockIdx.x;
+    for (int e = tid; e < E; e += kScanThreads) {
+        running[e] = a.ws.chunk_excl[(size_t)chunk * E + e];
+        for (int w = 0; w < W; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    const int begin = chunk * kScanChunk, end = min(a.R, begin + kScanChunk);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = begin; base < end; base += kScanThreads) {
+        const int i = base + tid;
+        int e = -1;
+        if (i < end) {
+            e = a.topk_idx[i];
+            if ((unsigned)e >= (unsigned)E) e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int lrank = __popc(peers & lt_mask);
+        if (e >= 0 && lrank == 0) wcnt[warp][e] = __popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int r = running[e] + lrank;
+            for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+            int row;
+            if (!a.capped)
+                row = a.ws.offsets[e] + r;
+            else if (r < a.C)
+                row = e * a.C + r;
+            else
+                row = E * a.C + a.ws.spill_off[e] + (r - a.C);
+            if ((unsigned)row < (unsigned)a.P) {
+                a.dest_row[i] = row;
+                a.src_token[row] = i / a.k;
+            } else {
+                a.dest_row[i] = -1;
+                atomicOr(a.ws.status, MOE_DEV_BAD_ROW);
+            }
+        } else if (i < end) {
+            a.dest_row[i] = -1;
+        }
+        __syncthreads();
+        for (int f = tid; f < E; f += kScanThreads) {
+            int s = 0;
+            for (int w = 0; w < W; ++w) {
+                s += wcnt[w][f];
+                wcnt[w][f] = 0;
+            }
+            running[f] += s;
+        }
+        __syncthreads();
+    }
+}
+
+// One warp per permuted row; rows are [0, R) uncapped, or the E*C capacity
+// slots plus the used part of the overflow region.
+__global__ void __launch_bounds__(256) k_gather(const uint4 *__restrict__ x, const int *__restrict__ src_token,
+                                                uint4 *__restrict__ x_perm, int H8, int T, int P, int fixed_rows,
+                                                int cap_rows, const int *total_spill) {
+    int rows = fixed_rows >= 0 ? fixed_rows : cap_rows + *total_spill;
+    if (rows > P) rows = P;
+    const int lane = threadIdx.x & 31;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    for (int row = gw; row < rows; row += nw) {
+        const int t = src_token[row];
+        uint4 *dst = x_perm + (size_t)row * H8;
+        if ((unsigned)t < (unsigned)T) {
+            const uint4 *src = x + (size_t)t * H8;
+            int v = lane;
+            for (; v + 96 < H8; v += 128) {
+                const uint4 q0 = __ldg(src + v), q1 = __ldg(src + v + 32), q2 = __ldg(src + v + 64),
+                            q3 = __ldg(src + v + 96);
+                dst[v] = q0;
+                dst[v + 32] = q1;
+                dst[v + 64] = q2;
+                dst[v + 96] = q3;
+            }
+            for (; v < H8; v += 32) dst[v] = __ldg(src + v);
+        } else {
+            for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
+                           int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
+                           void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int R = s.T * s.k;
+    WsPtrs p = ws_ptrs(ws, L);
+    cudaError_t err = cudaMemsetAsync((char *)ws + L.reset_begin, 0, L.reset_end - L.reset_begin, stream);
+    if (err != cudaSuccess) return err;
+    if (capped) {
+        const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, true);
+        err = cudaMemsetAsync(src_token, 0xFF, sizeof(int32_t) * (size_t)P, stream);
+        if (err != cudaSuccess) return err;
+    }
+    ScanArgs sa;
+    sa.topk_idx = topk_idx;
+    sa.T = s.T;
+    sa.E = s.E;
+    sa.k = s.k;
+    sa.C = s.C;
+    sa.capped = capped;
+    sa.R = R;
+    sa.stall_first_block = (s.flags & MOE_FLAG_TEST_STALL_SCAN) ? 1 : 0;
+    sa.timeout_ns = timeout_ns;
+    sa.counts_out = counts;
+    sa.offsets_out = offsets;
+    sa.ws = p;
+    k_hist_scan<<<L.nchunks, kScanThreads, 0, stream>>>(sa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    RankArgs ra;
+    ra.topk_idx = topk_idx;
+    ra.E = s.E;
+    ra.k = s.k;
+    ra.C = s.C;
+    ra.capped = capped;
+    ra.R = R;
+    ra.P = (int)permuted_rows(s.T, s.E, s.k, s.C, capped);
+    ra.dest_row = dest_row;
+    ra.src_token = src_token;
+    ra.ws = p;
+    k_rank<<<L.nchunks, kScanThreads, 0, stream>>>(ra);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int H8 = s.H / 8;
+    const int fixed = capped ? -1 : R;
+    const int rows_hint = capped ? s.E * s.C + s.k * (s.T > s.C ? s.T - s.C : 0) : R;
+    int blocks = (rows_hint + 7) / 8;  // 8 warps per block, one row each
+    const int cap_blocks = num_sms * 8;
+    if (blocks > cap_blocks) blocks = cap_blocks;
+    if (blocks < 1) blocks = 1;
+    k_gather<<<blocks, 256, 0, stream>>>((const uint4 *)x, src_token, (uint4 *)x_perm, H8, s.T, ra.P, fixed,
+                                         s.E * s.C, p.total_spill);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

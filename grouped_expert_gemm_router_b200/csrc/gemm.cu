@@ -1,0 +1,409 @@
+// Step 4: grouped expert GEMMs on the sm_100a tensor cores.
+//   mode 0, fused gate+up SwiGLU ("TritonMoE" verdict page, arXiv 2605.23911,
+//           pith extraction key machinery: both projections from one load of
+//           each input tile, SiLU in registers, the two intermediates never
+//           written to global memory):
+//           h[r, f] = bf16( silu(x_perm[r] . Wg[e][:, f]) * (x_perm[r] . Wu[e][:, f]) )
+//   mode 1, down projection (same page, desk editor letter):
+//           y[r, c] = bf16( h[r] . Wd[e][:, c] )
+//
+// Design (B200 first, not the page's Triton kernel):
+// - Swap-AB.  The MMA computes D[feature, row] = W^T[feature, k] * X^T[k, row]:
+//   the expert weights are the M = 128 operand (MN-major, read straight from
+//   the [E, K, N] weight tensors) and up to 256 permuted rows of one expert
+//   are the N operand (K-major).  An expert with <= 256 routed rows therefore
+//   streams each weight tile from HBM exactly once, which is what the
+//   weight-streaming regime of small per-expert batches needs, and N is
+//   rounded only to 16 rows, not to a 128-row M tile.
+// - Two accumulators per work unit share every B tile: gate and up for the
+//   same 128 features (mode 0), or two adjacent 128-feature blocks (mode 1).
+//   They live in tensor memory at columns [0, N) and [256, 256 + N).
+// - Persistent, warp-specialised: warp 0 issues TMA loads into a 3-stage
+//   ring of shared-memory stages (mbarrier expect-tx), warp 1 issues
+//   tcgen05.mma from one thread and commits each stage back to the producer,
+//   warps 2-5 drain tensor memory with tcgen05.ld and write bf16 results.
+// - The schedule is the device-built tile map: work unit u -> (expert group
+//   in descending-count order, feature block, row tile), feature-block-major
+//   inside an expert so that the row tiles of one expert that share a weight
+//   tile run next to each other.  Nothing depends on the host knowing the
+//   routing, so the kernel is launched with one CTA per SM and can be
+//   captured in a CUDA graph.
+// - Every wait is bounded: on expiry the kernel records MOE_DEV_GEMM_TIMEOUT,
+//   tells the other roles to stop, lets in-flight copies and MMAs land, frees
+//   its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 3;
+constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 features (8 KiB)
+constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
+constexpr uint32_t kBBox = 16 * kBK * 2;       // TMA box: 16 rows x 64 K (2 KiB)
+constexpr uint32_t kBTile = kTileRows * kBK * 2;
+constexpr uint32_t kStage = 2 * kATile + kBTile;
+constexpr uint32_t kCtrlBytes = 2048;
+constexpr uint32_t kSmemBytes = kStages * kStage + 1024 + kCtrlBytes;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcc1Col = 256;
+
+struct GemmArgs {
+    const int4 *tile_map;
+    const int *grp_tile_start;
+    const int *num_tiles;
+    uint32_t *status;
+    __nv_bfloat16 *out;
+    int n_out;   // row length of `out`: F (mode 0) or H (mode 1)
+    int K;       // reduction length: H (mode 0) or F (mode 1)
+    int num_fb;  // feature blocks per row tile
+    int E;
+    int P;          // rows of the permuted buffers
+    int max_tiles;  // capacity of the tile map
+    unsigned long long timeout_ns;
+};
+
+struct Unit {
+    int e, fb, nacc, N, n0p, p0s, p0l, p1s, p1l;
+    bool valid;  // false only for a corrupt schedule: every role then skips the unit
+};
+
+template <int MODE>
+__device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, Unit &U) {
+    int lo = 0, hi = a.E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (gts[mid] * a.num_fb <= u)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int g0 = gts[lo], nt = gts[lo + 1] - g0;
+    U.valid = false;
+    U.N = 0;
+    if (nt <= 0 || g0 < 0) return;
+    const int local = u - g0 * a.num_fb;
+    U.fb = local / nt;
+    const int tile = g0 + local % nt;
+    if (tile >= a.max_tiles) return;
+    const int4 d = a.tile_map[tile];
+    U.e = d.x;
+    U.p0s = d.y;
+    U.p0l = d.z & 0xFFFF;
+    U.p1l = (d.z >> 16) & 0xFFFF;
+    U.p1s = d.w;
+    U.n0p = (U.p0l + 15) & ~15;
+    U.N = U.n0p + ((U.p1l + 15) & ~15);
+    U.nacc = (MODE == 0) ? 2 : ((U.fb * 256 + 128 < a.n_out) ? 2 : 1);
+    U.valid = (unsigned)U.e < (unsigned)a.E && U.N > 0 && U.N <= kTileRows && U.p0s >= 0 && U.p1s >= 0 &&
+              U.p0s + U.p0l <= a.P && U.p1s + U.p1l <= a.P && U.fb < a.num_fb;
+}
+
+__device__ __forceinline__ int unit_row(const Unit &U, int c) {
+    if (c < U.n0p) return c < U.p0l ? U.p0s + c : -1;
+    const int c1 = c - U.n0p;
+    return c1 < U.p1l ? U.p1s + c1 : -1;
+}
+
+__device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *status) {
+    *abort = 1;
+    atomicOr(status, MOE_DEV_GEMM_TIMEOUT);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // SW128 tiles need 1 KiB alignment
+    uint8_t *ctrl = smem + kStages * kStage;
+    uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);
+    uint64_t *empty = full + kStages;
+    uint64_t *tfull = empty + kStages;
+    uint64_t *tempty = tfull + 1;
+    uint64_t *mma_done = tempty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);  // E + 1 <= 257 ints
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = *a.num_tiles;
+    const int total = (ntiles < a.max_tiles ? ntiles : a.max_tiles) * a.num_fb;
+    if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
+
+    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 4);
+        mbar_init(mma_done, 1);
+        *s_abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmA1);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nk = a.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t ph = 0;
+            int issued_ph[kStages];
+            for (int s = 0; s < kStages; ++s) issued_ph[s] = -1;
+            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+                Unit U;
+                decode_unit<MODE>(u, s_gts, a, U);
+                if (!U.valid) {
+                    atomicOr(a.status, MOE_DEV_BAD_ROW);
+                    continue;
+                }
+                const int fx0 = MODE == 0 ? U.fb * 128 : U.fb * 256;
+                const int fx1 = MODE == 0 ? U.fb * 128 : U.fb * 256 + 128;
+                const int nb0 = (U.p0l + 15) >> 4, nb1 = (U.p1l + 15) >> 4;
+                const uint32_t bytes = (uint32_t)U.nacc * kATile + (uint32_t)(nb0 + nb1) * kBBox;
+                const int krow = U.e * a.K;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, a.timeout_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa0 = smem + stage * kStage;
+                    uint8_t *sa1 = sa0 + kATile;
+                    uint8_t *sb = sa1 + kATile;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    const int ky = krow + kb * kBK, kx = kb * kBK;
+                    tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
+                    tma_load_2d(sa0 + kABox, &tmA0, &full[stage], fx0 + 64, ky);
+                    if (U.nacc == 2) {
+                        tma_load_2d(sa1, &tmA1, &full[stage], fx1, ky);
+                        tma_load_2d(sa1 + kABox, &tmA1, &full[stage], fx1 + 64, ky);
+                    }
+                    for (int i = 0; i < nb0; ++i) tma_load_2d(sb + i * kBBox, &tmB, &full[stage], kx, U.p0s + 16 * i);
+                    for (int i = 0; i < nb1; ++i)
+                        tma_load_2d(sb + U.n0p * (kBK * 2) + i * kBBox, &tmB, &full[stage], kx, U.p1s + 16 * i);
+                    issued_ph[stage] = (int)ph;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    if (!*s_abort) raise_abort(s_abort, a.status);
+                    break;
+                }
+            }
+            // Every issued copy must land before the CTA may leave.
+            int never = 0;
+            for (int s = 0; s < kStages; ++s)
+                if (issued_ph[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)issued_ph[s], a.timeout_ns, &never);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ----
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t ph = 0, tph = 0;
+            const uint32_t base = smem_u32(smem);
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                Unit U;
+                decode_unit<MODE>(u, s_gts, a, U);
+                if (!U.valid) continue;
+                const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
+                if (!mbar_wait_bounded(tempty, tph ^ 1u, a.timeout_ns, s_abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], ph, a.timeout_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa0 = base + stage * kStage, sa1 = sa0 + kATile, sb = sa1 + kATile;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        // B: K-major, 16 K-elements (32 bytes) per MMA inside the 128-byte row.
+                        const uint64_t bdesc = sdesc_sw128(sb + kk * 32, 16, 1024);
+                        // A: MN-major, 16 K-rows (2 KiB) per MMA; the two 64-feature halves 8 KiB apart.
+                        const uint64_t a0desc = sdesc_sw128(sa0 + kk * 2048, kABox, 1024);
+                        const uint32_t accum = (kb | kk) ? 1u : 0u;
+                        tc_mma_bf16(tmem, a0desc, bdesc, idesc, accum);
+                        if (U.nacc == 2) {
+                            const uint64_t a1desc = sdesc_sw128(sa1 + kk * 2048, kABox, 1024);
+                            tc_mma_bf16(tmem + kAcc1Col, a1desc, bdesc, idesc, accum);
+                        }
+                    }
+                    tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+                    if (++stage == kStages) {
+                        stage = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(tfull);
+                tph ^= 1u;
+            }
+            if (!ok && !*s_abort) raise_abort(s_abort, a.status);
+            // All MMAs issued by this thread complete before tensor memory is freed.
+            int never = 0;
+            tc_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0, a.timeout_ns, &never);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- epilogue ----
+        const int q = warp & 3;           // tensor-memory lane quarter of this warp
+        const int L = q * 32 + lane;      // feature within a 128-feature accumulator
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+        uint32_t tph = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            Unit U;
+            decode_unit<MODE>(u, s_gts, a, U);
+            if (!U.valid) continue;
+            // The whole warp takes one decision, so the .sync.aligned loads
+            // below never run with part of the warp.
+            const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, tph, a.timeout_ns, s_abort));
+            if (!ready) {
+                if (lane == 0 && !*s_abort) raise_abort(s_abort, a.status);
+                break;
+            }
+            tc_fence_after();
+            const int f0 = MODE == 0 ? U.fb * 128 + L : U.fb * 256 + L;
+            for (int c0 = 0; c0 < U.N; c0 += 16) {
+                uint32_t r0[16], r1[16];
+                tmem_ld16(tq + (uint32_t)c0, r0);
+                if (U.nacc == 2) tmem_ld16(tq + kAcc1Col + (uint32_t)c0, r1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int row = unit_row(U, c0 + j);
+                    if (row < 0) continue;
+                    __nv_bfloat16 *dst = a.out + (size_t)row * a.n_out + f0;
+                    if (MODE == 0) {
+                        const float g = __uint_as_float(r0[j]), v = __uint_as_float(r1[j]);
+                        dst[0] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * v);
+                    } else {
+                        dst[0] = __float2bfloat16_rn(__uint_as_float(r0[j]));
+                        if (U.nacc == 2) dst[128] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);
+            tph ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with the 128-byte
+// swizzle; box = box_cols x box_rows (box_cols * 2 bytes must be 128).
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols,
+               uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// mode 0: act = x_perm [P,H], w0 = gate, w1 = up, out = h [P,F]
+// mode 1: act = h [P,F],      w0 = w1 = down,   out = y [P,H]
+cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
+                                void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                cudaStream_t stream) {
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
+    const int K = mode == 0 ? s.H : s.F;
+    const int n_out = mode == 0 ? s.F : s.H;
+    CUtensorMap tA0, tA1, tB;
+    if (!make_tmap(&tA0, w0, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
+        !make_tmap(&tA1, w1, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
+        !make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16))
+        return cudaErrorInvalidValue;
+    WsPtrs p = ws_ptrs(ws, L);
+    GemmArgs a;
+    a.tile_map = p.tile_map;
+    a.grp_tile_start = p.grp_tile_start;
+    a.num_tiles = p.num_tiles;
+    a.status = p.status;
+    a.out = (__nv_bfloat16 *)out;
+    a.n_out = n_out;
+    a.K = K;
+    a.num_fb = mode == 0 ? s.F / 128 : (s.H + 255) / 256;
+    a.E = s.E;
+    a.P = (int)P;
+    a.max_tiles = L.max_tiles;
+    a.timeout_ns = timeout_ns;
+    static bool attr_done[2] = {false, false};
+    cudaError_t err;
+    if (mode == 0) {
+        if (!attr_done[0]) {
+            err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (err != cudaSuccess) return err;
+            attr_done[0] = true;
+        }
+        k_grouped_gemm<0><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+    } else {
+        if (!attr_done[1]) {
+            err = cudaFuncSetAttribute(k_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (err != cudaSuccess) return err;
+            attr_done[1] = true;
+        }
+        k_grouped_gemm<1><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,250 @@
+// extern "C" entry points declared in include/moe.h: argument validation,
+// workspace carving and kernel launches.  No entry point allocates, frees or
+// synchronises except moe_read_status.
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
+                         int32_t *topk_idx, float *topk_w, uint32_t *status, int num_sms, cudaStream_t stream);
+cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
+                           int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
+                           void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
+cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
+                                void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                cudaStream_t stream);
+cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
+                           cudaStream_t stream);
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+std::atomic<uint64_t> g_timeout_ns{1000000000ull};
+thread_local char g_last_error[160] = "no error";
+
+constexpr uint32_t kKnownFlags = MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FLAG_TEST_STALL_SCAN;
+
+bool aligned(const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
+
+moe_status cuda_fail(cudaError_t e, const char *where) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+moe_status check_shape(const moe_shape *s) {
+    if (!s) return MOE_ERR_INVALID_ARG;
+    if (s->flags & ~kKnownFlags) return MOE_ERR_INVALID_ARG;
+    if (s->T < 1 || s->E < 1 || s->E > kMaxExperts || s->k < 1 || s->k > s->E || s->C < 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (s->H < 128 || s->H % 128 || s->H > 65536 || s->F < 128 || s->F % 128 || s->F > 65536)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    const bool capped = (s->flags & MOE_FLAG_CAPACITY) != 0;
+    const int64_t R = (int64_t)s->T * s->k;
+    const int64_t P = permuted_rows(s->T, s->E, s->k, s->C, capped);
+    if (R >= (1ll << 30) || P >= (1ll << 30) || (int64_t)s->E * s->C >= (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int64_t units = (int64_t)max_tiles_for(P, s->E) * (s->F / 128 > s->H / 256 + 1 ? s->F / 128 : s->H / 256 + 1);
+    if (units >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+WsLayout layout_of(const moe_shape *s) {
+    return ws_layout(s->T, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
+}
+
+// sm_100 check and SM count of the current device, cached per device.
+moe_status device_info(int *num_sms) {
+    static std::atomic<int> cache[64];  // 0 unknown, -1 not sm_100, else SM count
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    int v = (dev >= 0 && dev < 64) ? cache[dev].load() : 0;
+    if (v == 0) {
+        int major = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        v = (major == 10 && sms > 0) ? sms : -1;
+        if (dev >= 0 && dev < 64) cache[dev].store(v);
+    }
+    if (v < 0) {
+        std::snprintf(g_last_error, sizeof(g_last_error), "current device is not sm_100");
+        return MOE_ERR_DEVICE;
+    }
+    *num_sms = v;
+    return MOE_OK;
+}
+
+moe_status check_ws(void *ws) { return aligned(ws, 256) ? MOE_OK : MOE_ERR_WORKSPACE; }
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_permuted_rows(const moe_shape *s) {
+    if (check_shape(s) != MOE_OK) return -1;
+    return permuted_rows(s->T, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
+}
+
+size_t moe_workspace_bytes(const moe_shape *s) {
+    if (check_shape(s) != MOE_OK) return 0;
+    return layout_of(s).total;
+}
+
+moe_status moe_workspace_layout(const moe_shape *s, moe_ws_layout *out) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!out) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = layout_of(s);
+    out->total = L.total;
+    out->status = L.status;
+    out->num_tiles = L.num_tiles;
+    out->total_spill = L.total_spill;
+    out->cap_cnt = L.cap_cnt;
+    out->spill_cnt = L.spill_cnt;
+    out->spill_off = L.spill_off;
+    out->order = L.order;
+    out->grp_tile_start = L.grp_tile_start;
+    out->tile_map = L.tile_map;
+    out->max_tiles = L.max_tiles;
+    out->tile_rows = kTileRows;
+    return MOE_OK;
+}
+
+moe_status moe_workspace_init(const moe_shape *s, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    cudaError_t e = cudaMemsetAsync(ws, 0, layout_of(s).total, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
+}
+
+moe_status moe_route(const moe_shape *s, const void *x, const float *w_router, const float *bias, float *logits,
+                     int32_t *topk_idx, float *topk_w, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    const bool logits_in = (s->flags & MOE_FLAG_LOGITS_IN) != 0;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+    if (logits_in) {
+        if (!aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
+    } else {
+        if (!aligned(x, 16) || !aligned(w_router, 4)) return MOE_ERR_INVALID_ARG;
+        if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
+        if (logits && !aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    uint32_t *status = (uint32_t *)((char *)ws + L.status);
+    cudaError_t e = launch_route(*s, x, w_router, bias, logits, topk_idx, topk_w, status, sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
+}
+
+moe_status moe_permute(const moe_shape *s, const void *x, const int32_t *topk_idx, int32_t *expert_counts,
+                       int32_t *expert_offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, void *ws,
+                       void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_idx, 4) || !aligned(expert_counts, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(src_token, 4) || !aligned(dest_row, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_permute(*s, x, topk_idx, expert_counts, expert_offsets, src_token, dest_row, x_perm, L, ws,
+                                   g_timeout_ns.load(), sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_permute");
+}
+
+moe_status moe_grouped_swiglu(const moe_shape *s, const void *x_perm, const void *w_gate, const void *w_up, void *h,
+                              void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(x_perm, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(h, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_grouped_gemm(0, *s, x_perm, w_gate, w_up, h, L, ws, g_timeout_ns.load(), sms,
+                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_swiglu");
+}
+
+moe_status moe_grouped_down(const moe_shape *s, const void *h, const void *w_down, void *y, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(h, 16) || !aligned(w_down, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_grouped_gemm(1, *s, h, w_down, w_down, y, L, ws, g_timeout_ns.load(), sms,
+                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down");
+}
+
+moe_status moe_combine(const moe_shape *s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
+                       void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(dest_row, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e = launch_combine(*s, y, dest_row, topk_w, out, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine");
+}
+
+moe_status moe_forward(const moe_shape *s, const moe_forward_args *a, void *ws, void *stream) {
+    if (!a) return MOE_ERR_INVALID_ARG;
+    moe_status st = moe_route(s, a->x, a->w_router, a->bias, a->logits, a->topk_idx, a->topk_w, ws, stream);
+    if (st != MOE_OK) return st;
+    st = moe_permute(s, a->x, a->topk_idx, a->expert_counts, a->expert_offsets, a->src_token, a->dest_row, a->x_perm,
+                     ws, stream);
+    if (st != MOE_OK) return st;
+    st = moe_grouped_swiglu(s, a->x_perm, a->w_gate, a->w_up, a->h, ws, stream);
+    if (st != MOE_OK) return st;
+    st = moe_grouped_down(s, a->h, a->w_down, a->y, ws, stream);
+    if (st != MOE_OK) return st;
+    return moe_combine(s, a->y, a->dest_row, a->topk_w, a->out, stream);
+}
+
+moe_status moe_read_status(void *ws, void *stream, uint32_t *device_status, int clear) {
+    if (!aligned(ws, 256) || !device_status) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_read_status");
+    *device_status = v;
+    return MOE_OK;
+}
+
+void moe_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : 1); }
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_WORKSPACE: return "unusable workspace";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_error_string(void) { return g_last_error; }
+
+int32_t moe_version(void) { return 100; }
+
+}  // extern "C"

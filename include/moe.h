@@ -1,0 +1,214 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) MoE-layer forward dispatch library.
+ *
+ * The library computes, on one GPU, the five-step forward path of a
+ * Mixture-of-Experts layer described on the "TritonMoE" verdict page
+ * (pith.science, arXiv 2605.23911; referee report summary and pith summary):
+ * router scoring, permutation of the routed tokens onto experts, the grouped
+ * expert GEMMs (a fused gate+up SwiGLU projection, then the down projection)
+ * and a weighted unpermutation.  The optional capacity layout follows the
+ * "Cap-and-Spill" critique page (juhe.plus), section "Cap-and-Spill": C slots
+ * per expert plus a compacted overflow buffer sized for the largest possible
+ * overflow, so no routed token is ever dropped.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Ownership: the CALLER allocates and owns every buffer (inputs, outputs,
+ *   intermediates and the workspace `ws`).  The library never allocates,
+ *   frees or synchronises, except moe_read_status, which synchronises.
+ * - Memory: every data pointer is a DEVICE pointer on the current CUDA
+ *   device, 16-byte aligned; `ws` is 256-byte aligned.  bf16 tensors are
+ *   passed as `void *` holding IEEE bfloat16 values.  All matrices are dense
+ *   and row-major with the leading dimension equal to the row length.
+ * - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  Each
+ *   call only enqueues work on it and returns; every call is
+ *   stream-ordered, performs no host synchronisation and may be captured in
+ *   a CUDA graph.  Grid sizes depend only on the shape and the SM count,
+ *   never on the routing, so a captured graph stays valid for any input
+ *   values of the same shape.
+ * - Errors: a bad argument or an unsupported shape returns a non-zero
+ *   moe_status before anything is enqueued.  A failed launch returns
+ *   MOE_ERR_CUDA.  Faults found on the device (a bounded wait that expired,
+ *   an expert index out of range) are OR-ed into a sticky status word in
+ *   `ws`; read it with moe_read_status.  No kernel traps.
+ * - Workspace: size it with moe_workspace_bytes and zero it once after
+ *   allocating it (moe_workspace_init, or a plain memset); afterwards every
+ *   call keeps it consistent by itself.
+ * - Workspace coupling: moe_permute leaves the per-expert offsets and the
+ *   tile schedule of the grouped GEMMs in `ws`; moe_grouped_swiglu and
+ *   moe_grouped_down read them.  A workspace must not be used by two
+ *   streams at once.
+ *
+ * Supported shapes: T >= 1, H and F multiples of 128, 1 <= E <= 256,
+ * 1 <= k <= E, C >= 0, and the permuted row count below 2^31.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,       /* null/misaligned pointer, bad flag */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the supported set above */
+    MOE_ERR_WORKSPACE = 3,         /* workspace pointer unusable */
+    MOE_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
+    MOE_ERR_DEVICE = 5             /* current device is not sm_100 */
+} moe_status;
+
+/* Bits of the device status word (sticky until cleared by moe_read_status). */
+#define MOE_DEV_SCAN_TIMEOUT 0x1u  /* histogram look-back wait expired */
+#define MOE_DEV_GEMM_TIMEOUT 0x2u  /* a grouped-GEMM pipeline wait expired */
+#define MOE_DEV_BAD_EXPERT 0x4u    /* a routed expert index was outside [0, E) */
+#define MOE_DEV_NAN_LOGIT 0x8u     /* warning: a router logit was NaN */
+#define MOE_DEV_BAD_ROW 0x10u      /* a row index fell outside its buffer and the
+                                      access was skipped (follows another error) */
+
+/* moe_shape.flags */
+#define MOE_FLAG_CAPACITY 0x1u  /* capacity layout: C slots per expert + overflow */
+#define MOE_FLAG_LOGITS_IN 0x2u /* moe_route/moe_forward read the caller's fp32
+                                   logits instead of computing x * W_r + bias */
+#define MOE_FLAG_TEST_STALL_SCAN 0x40000000u /* test only: the first histogram
+                                   block never publishes, so its successor's
+                                   bounded wait expires and reports
+                                   MOE_DEV_SCAN_TIMEOUT */
+
+typedef struct {
+    int32_t T;      /* tokens */
+    int32_t H;      /* hidden size */
+    int32_t F;      /* expert FFN size */
+    int32_t E;      /* experts */
+    int32_t k;      /* experts per token */
+    int32_t C;      /* capacity slots per expert (used with MOE_FLAG_CAPACITY) */
+    uint32_t flags; /* MOE_FLAG_* */
+} moe_shape;
+
+/* Every pointer argument of the whole layer, for moe_forward. */
+typedef struct {
+    const void *x;         /* [T,H]   bf16 tokens */
+    const float *w_router; /* [H,E]   fp32 router weights (unused with LOGITS_IN) */
+    const float *bias;     /* [E]     fp32 additive logit bias, or NULL */
+    const void *w_gate;    /* [E,H,F] bf16 */
+    const void *w_up;      /* [E,H,F] bf16 */
+    const void *w_down;    /* [E,F,H] bf16 */
+    float *logits;         /* [T,E]   fp32 (input with LOGITS_IN, else output; may be NULL without LOGITS_IN) */
+    int32_t *topk_idx;     /* [T,k]   expert ids in rank order */
+    float *topk_w;         /* [T,k]   gate weights */
+    int32_t *expert_counts;  /* [E]   routed pairs per expert */
+    int32_t *expert_offsets; /* [E+1] exclusive prefix sum of expert_counts */
+    int32_t *src_token;    /* [P]     token of each permuted row, -1 = empty slot */
+    int32_t *dest_row;     /* [T*k]   permuted row of each routed pair */
+    void *x_perm;          /* [P,H]   bf16 permuted tokens */
+    void *h;               /* [P,F]   bf16 SwiGLU activations */
+    void *y;               /* [P,H]   bf16 expert outputs */
+    void *out;             /* [T,H]   bf16 layer output */
+} moe_forward_args;
+
+/* Byte offsets of the workspace sections a caller may inspect (tests do). */
+typedef struct {
+    size_t total;          /* bytes the workspace must hold */
+    size_t status;         /* uint32 sticky device status word */
+    size_t num_tiles;      /* int32 number of GEMM row tiles */
+    size_t total_spill;    /* int32 rows used in the overflow region */
+    size_t cap_cnt;        /* int32[E] min(n_e, C) (n_e when uncapped) */
+    size_t spill_cnt;      /* int32[E] n_e - cap_cnt[e] */
+    size_t spill_off;      /* int32[E+1] exclusive prefix sum of spill_cnt */
+    size_t order;          /* int32[E] experts by descending count, ties by index */
+    size_t grp_tile_start; /* int32[E+1] first tile of the g-th expert of `order` */
+    size_t tile_map;       /* int32[4*max_tiles] tiles: {e, row0, len0 | len1<<16, row1} */
+    int32_t max_tiles;     /* capacity of tile_map */
+    int32_t tile_rows;     /* largest number of rows one tile holds */
+} moe_ws_layout;
+
+/* Rows of the permuted buffers x_perm, h, y: T*k uncapped; with the capacity
+ * layout E*C + k*max(0, T-C) (the overflow is at most k*(T-C): it is largest
+ * when k experts take every token).  Returns -1 for an unsupported shape. */
+MOE_API int64_t moe_permuted_rows(const moe_shape *shape);
+
+/* Workspace bytes for `shape`, or 0 for an unsupported shape. */
+MOE_API size_t moe_workspace_bytes(const moe_shape *shape);
+
+/* Fills `layout` for `shape`; MOE_ERR_UNSUPPORTED_SHAPE if unsupported. */
+MOE_API moe_status moe_workspace_layout(const moe_shape *shape, moe_ws_layout *layout);
+
+/* Zero-fills `ws` (moe_workspace_bytes(shape) bytes) on `stream`.  Needed
+ * once per newly allocated workspace; clears the sticky status word too. */
+MOE_API moe_status moe_workspace_init(const moe_shape *shape, void *ws, void *stream);
+
+/* Step 1, router scoring ("TritonMoE" verdict page, referee report summary):
+ *   logits[t,e] = fp32(sum_h x[t,h] * w_router[h,e]) + bias[e]
+ *   topk_idx[t,:] = the k experts of largest logit, in rank order, equal
+ *                   logits to the lower index, NaN below every number;
+ *   topk_w[t,j]   = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected.
+ * With MOE_FLAG_LOGITS_IN, `logits` is read (w_router, bias unused).
+ * Otherwise `logits` may be NULL (not written). */
+MOE_API moe_status moe_route(const moe_shape *shape, const void *x, const float *w_router, const float *bias, float *logits,
+                     int32_t *topk_idx, float *topk_w, void *ws, void *stream);
+
+/* Steps 2-3, histogram + exclusive scan + stable permutation ("TritonMoE"
+ * verdict page: tokens reordered onto experts; "Cap-and-Spill" page for the
+ * capacity layout):
+ *   expert_counts[e]  = #{(t,j): topk_idx[t,j] == e}
+ *   expert_offsets    = exclusive prefix sum of expert_counts
+ *   the r-th pair of expert e in flat order t*k+j goes to row
+ *     uncapped:  expert_offsets[e] + r
+ *     capacity:  r < C ? e*C + r : E*C + spill_off[e] + (r - C)
+ *   dest_row[t*k+j] = its row; src_token[row] = t (-1 for an unfilled row);
+ *   x_perm[row] = x[src_token[row]] (zeros for unfilled capacity slots).
+ * Also leaves the grouped-GEMM tile schedule in `ws`. */
+MOE_API moe_status moe_permute(const moe_shape *shape, const void *x, const int32_t *topk_idx, int32_t *expert_counts,
+                       int32_t *expert_offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, void *ws,
+                       void *stream);
+
+/* Step 4a, fused gate+up SwiGLU over every filled permuted row r of expert e
+ * ("TritonMoE" verdict page, pith extraction key machinery):
+ *   h[r,f] = bf16( silu(x_perm[r] . w_gate[e][:,f]) * (x_perm[r] . w_up[e][:,f]) ),
+ *   silu(z) = z / (1 + exp(-z)), fp32 accumulation.  Rows not filled are
+ *   left unwritten.  Reads the tile schedule moe_permute left in `ws`. */
+MOE_API moe_status moe_grouped_swiglu(const moe_shape *shape, const void *x_perm, const void *w_gate, const void *w_up,
+                              void *h, void *ws, void *stream);
+
+/* Step 4b, down projection ("TritonMoE" verdict page, desk editor letter):
+ *   y[r,c] = bf16( h[r] . w_down[e][:,c] ), fp32 accumulation. */
+MOE_API moe_status moe_grouped_down(const moe_shape *shape, const void *h, const void *w_down, void *y, void *ws,
+                            void *stream);
+
+/* Step 5, weighted unpermutation ("TritonMoE" verdict page, referee report
+ * summary):  out[t] = bf16( sum_j topk_w[t,j] * y[dest_row[t*k+j]] ), the
+ * sum in fp32 in slot order j, products and sums rounded separately. */
+MOE_API moe_status moe_combine(const moe_shape *shape, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
+                       void *stream);
+
+/* The five steps in order on one stream (no host sync; graph-capturable). */
+MOE_API moe_status moe_forward(const moe_shape *shape, const moe_forward_args *args, void *ws, void *stream);
+
+/* Synchronises `stream`, copies the sticky device status word of `ws` to
+ * *device_status and, if clear != 0, resets it.  Not graph-capturable. */
+MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_status, int clear);
+
+/* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
+MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
+
+MOE_API const char *moe_status_string(moe_status status);
+
+/* Text of the last CUDA failure seen by this thread's calls ("no error" if none). */
+MOE_API const char *moe_last_error_string(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MOE_API int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

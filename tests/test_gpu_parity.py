@@ -1,0 +1,210 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element,
+on seeded inputs small enough for the whole oracle, spanning several GEMM
+tiles per expert with ragged tails, plus the edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import grouped_expert_gemm_router_b200 as moe
+import synth
+from gpu_util import (LOGIT_TOL, WEIGHT_TOL, DeviceLayer, assert_close_bf16, check_tile_schedule, host, run_steps,
+                      shape_of)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # two row tiles per expert (about 350 routed rows each) and ragged tails
+    "two_tiles_E4_k2": synth.LayerConfig("t", 700, 256, 384, 4, 2, seed=1),
+    # H = 384: the down projection ends on a single 128-feature accumulator
+    "skew_E8_k3_H384": synth.LayerConfig("t", 300, 384, 256, 8, 3, alpha=1.5, seed=2),
+    "capacity_E16_k4_C24": synth.LayerConfig("t", 200, 256, 256, 16, 4, C=24, alpha=1.0, seed=3),
+    "tiny_config": synth.CONFIGS[1],
+    "single_token": synth.LayerConfig("t", 1, 128, 128, 1, 1, seed=4),
+    "k_equals_E": synth.LayerConfig("t", 40, 128, 128, 4, 4, seed=5),
+    "E1_dense": synth.LayerConfig("t", 300, 128, 256, 1, 1, seed=6),
+    "many_experts_E256_k8": synth.LayerConfig("t", 96, 128, 128, 256, 8, alpha=0.5, seed=7),
+}
+
+
+def _oracle_full(orc, L, cfg, logits_gpu):
+    """Oracle routing from the GPU logits (same fp32 logits on both sides),
+    then the oracle's own dispatch, experts and combine."""
+    idx, w, _ = orc.topk_softmax(logits_gpu, cfg.k)
+    capped = cfg.C > 0
+    d = orc.dispatch(idx, cfg.E, C=cfg.C, capped=capped)
+    P = d["P"]
+    x_perm = np.zeros((P, cfg.H), np.uint16)
+    h = np.zeros((P, cfg.F), np.uint16)
+    y = np.zeros((P, cfg.H), np.uint16)
+    flat = idx.reshape(-1)
+    for i, r in enumerate(d["dest_row"]):
+        t, e = i // cfg.k, flat[i]
+        x_perm[r] = L.x[t]
+        h[r] = orc.swiglu_row(L.x[t], L.w_gate[e], L.w_up[e])
+        y[r] = orc.down_row(h[r], L.w_down[e])
+    out = orc.combine(y, d["dest_row"], w)
+    return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_parity(orc, name):
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    r = host(run_steps(dl, shape), shape)
+    assert r["status"] == 0, hex(r["status"])
+
+    # step 1: logits against the oracle's, then indices/weights given the GPU's logits
+    ref_logits = orc.router_logits(L.x, L.w_router, L.bias)
+    assert np.all(np.abs(r["logits"] - ref_logits) <= LOGIT_TOL * np.maximum(1.0, np.abs(ref_logits)))
+    o = _oracle_full(orc, L, cfg, r["logits"])
+    assert np.array_equal(r["topk_idx"], o["idx"])
+    assert np.max(np.abs(r["topk_w"] - o["w"])) <= WEIGHT_TOL
+
+    # steps 2-3: bit-exact counts, offsets, permutation, gathered rows, schedule
+    d = o["d"]
+    assert np.array_equal(r["expert_counts"], d["counts"])
+    assert np.array_equal(r["expert_offsets"], d["offsets"])
+    assert np.array_equal(r["dest_row"], d["dest_row"])
+    filled = d["src_token"] >= 0
+    assert np.array_equal(r["src_token"][filled], d["src_token"][filled])
+    if cfg.C > 0:
+        assert np.all(r["src_token"][~filled] == -1)
+        assert np.array_equal(r["cap_cnt"], d["cap_cnt"]) and np.array_equal(r["spill_cnt"], d["spill_cnt"])
+        assert np.array_equal(r["spill_off"], d["spill_off"])
+        assert r["total_spill"] == int(d["spill_cnt"].sum())
+    assert np.array_equal(r["x_perm"][filled], o["x_perm"][filled])
+    check_tile_schedule(r, shape, d["counts"], d["offsets"], d["spill_off"])
+
+    # step 4: GEMMs within the output tolerance, on every filled row
+    assert_close_bf16(r["h"][filled], o["h"][filled], "h")
+    assert_close_bf16(r["y"][filled], o["y"][filled], "y")
+    # step 5: combine is bit-exact given the same y; the layer within tolerance
+    same_y_out = orc.combine(r["y"], r["dest_row"], r["topk_w"])
+    assert np.array_equal(r["out"], same_y_out)
+    assert_close_bf16(r["out"], o["out"], "out")
+
+
+def test_forward_entry_point_matches_steps(orc):
+    cfg = CASES["skew_E8_k3_H384"]
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    a = host(run_steps(dl, shape), shape)
+    b = dl.bufs(shape)
+    moe.moe_forward(shape, b, b["ws"])
+    torch.cuda.synchronize()
+    f = host(b, shape)
+    for key in ("logits", "topk_idx", "topk_w", "dest_row", "h", "y", "out"):
+        assert np.array_equal(a[key], f[key]), key
+
+
+def test_logits_in_ties(orc):
+    """Integer-valued logits with many ties, given to the router directly:
+    indices must follow the lowest-index tie-break exactly."""
+    cfg = synth.LayerConfig("t", 257, 128, 128, 16, 5, seed=8)
+    L = synth.make_layer(cfg)
+    rng = np.random.default_rng(0)
+    logits = rng.integers(-2, 3, size=(cfg.T, cfg.E)).astype(np.float32)
+    logits[3, :] = np.nan
+    logits[4, 7] = np.nan
+    shape = shape_of(cfg, logits_in=True)
+    dl = DeviceLayer(L)
+    r = host(run_steps(dl, shape, logits=logits), shape)
+    idx, w, _ = orc.topk_softmax(logits, cfg.k)
+    assert np.array_equal(r["topk_idx"], idx)
+    ok = np.isfinite(w).all(axis=1)
+    assert np.max(np.abs(r["topk_w"][ok] - w[ok])) <= WEIGHT_TOL
+    assert r["status"] & moe.MOE_DEV_NAN_LOGIT
+
+
+def test_all_tokens_to_one_expert(orc):
+    """A dominant bias sends every token to expert 0 (n_0 = T, 3 row tiles)."""
+    cfg = synth.LayerConfig("t", 600, 128, 256, 8, 2, seed=9)
+    L = synth.make_layer(cfg)
+    L.bias = np.zeros(cfg.E, np.float32)
+    L.bias[0] = 1000.0
+    shape = shape_of(cfg)
+    r = host(run_steps(DeviceLayer(L), shape), shape)
+    assert r["expert_counts"][0] == cfg.T
+    o = _oracle_full(orc, L, cfg, r["logits"])
+    assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
+    assert_close_bf16(r["out"], o["out"], "out")
+
+
+@pytest.mark.parametrize("C", [0, 1, 7, 10_000])
+def test_capacity_equals_uncapped(orc, C):
+    """Capacity layout (C = 0: everything in the overflow; C >= max n_e:
+    nothing spills) gives the uncapped output bit for bit, with no drops."""
+    cfg = synth.LayerConfig("t", 150, 128, 256, 12, 3, alpha=1.2, seed=10)
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    su = shape_of(cfg)
+    sc = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=C, capacity=True)
+    u = host(run_steps(dl, su), su)
+    c = host(run_steps(dl, sc), sc)
+    assert u["status"] == 0 and c["status"] == 0
+    assert np.array_equal(u["out"], c["out"])
+    assert len(set(c["dest_row"].tolist())) == cfg.T * cfg.k
+    if C == 0:
+        assert np.array_equal(c["dest_row"], u["dest_row"])
+    if C >= cfg.T:
+        assert c["total_spill"] == 0
+
+
+def test_cuda_graph_replay_with_new_routing(orc):
+    """Capture the whole layer once; replay it on new tokens (new routing):
+    no routing-dependent host shape exists, so the replay stays exact."""
+    cfg = CASES["skew_E8_k3_H384"]
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    b = dl.bufs(shape)
+    args = moe.forward_args(b)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.moe_forward(shape, b, b["ws"], stream=s, args=args)  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_forward(shape, b, b["ws"], args=args)
+    for seed_offset in (11, 12):
+        x2 = synth.x_tokens(cfg, seed_offset)
+        b["x"].copy_(torch.from_numpy(x2.view(np.int16)).view(torch.bfloat16))
+        g.replay()
+        torch.cuda.synchronize()
+        r = host(b, shape)
+        L2 = synth.Layer(cfg, x2, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down)
+        o = _oracle_full(orc, L2, cfg, r["logits"])
+        assert np.array_equal(r["topk_idx"], o["idx"])
+        assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
+        assert_close_bf16(r["out"], o["out"], "out after replay")
+    del g
+
+
+def test_scan_wait_expires_and_reports(orc):
+    """A histogram block that never publishes makes its successor's bounded
+    wait run out: the kernel returns, the status word says so, and the
+    context stays usable."""
+    cfg = synth.LayerConfig("t", 2048, 128, 128, 8, 2, seed=13)  # 4096 pairs = 2 scan blocks
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    shape = shape_of(cfg, flags=moe.MOE_FLAG_TEST_STALL_SCAN)
+    b = dl.bufs(shape)
+    moe.moe_set_wait_timeout_ns(200_000_000)
+    try:
+        moe.moe_route(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"], b["ws"])
+        moe.moe_permute(shape, b["x"], b["topk_idx"], b["expert_counts"], b["expert_offsets"], b["src_token"],
+                        b["dest_row"], b["x_perm"], b["ws"])
+        st = moe.moe_read_status(b["ws"], clear=True)
+    finally:
+        moe.moe_set_wait_timeout_ns(1_000_000_000)
+    assert st & moe.MOE_DEV_SCAN_TIMEOUT
+    ok = shape_of(cfg)
+    r = host(run_steps(dl, ok), ok)
+    assert r["status"] == 0
+    o = _oracle_full(orc, L, cfg, r["logits"])
+    assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
