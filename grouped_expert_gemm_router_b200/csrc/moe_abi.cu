@@ -133,7 +133,7 @@ moe_status moe_route(const moe_shape *s, const void *x, const float *w_router, c
     if (logits_in) {
         if (!aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
     } else {
-        if (!aligned(x, 16) || !aligned(w_router, 4)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_ERR_INVALID_ARG;
         if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
         if (logits && !aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
     }

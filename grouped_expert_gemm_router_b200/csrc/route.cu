@@ -4,9 +4,10 @@
 // softmax over the k selected logits.
 //
 // One CTA of 8 warps owns a block of TB = 8*TW tokens and all E experts.  The
-// logits are a small fp32 GEMM: x and W_r are staged through shared memory in
-// chunks of 32 hidden units, and each lane accumulates TW tokens x EJ experts
-// in registers.  When E < 32 the spare lanes split the hidden dimension and
+// logits are a small fp32 GEMM: x and W_r stream through shared memory in
+// chunks of HC hidden units (HC chosen so a chunk of W_r is about 16-40 KiB)
+// with a 2-4 stage cp.async pipeline, so several chunks are in flight per
+// CTA; each lane accumulates TW tokens x EJ experts in registers.  When E < 32 the spare lanes split the hidden dimension and
 // are folded together with shuffles at the end.  The top-k then runs one warp
 // per token: each lane holds ceil(E/32) candidates as 64-bit keys
 // (orderable logit << 32 | ~expert) and k rounds of a warp-wide max pick the
@@ -19,7 +20,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kHC = 32;  // hidden units per staged chunk
 
 struct RouteArgs {
     const __nv_bfloat16 *x;
@@ -31,6 +31,9 @@ struct RouteArgs {
     uint32_t *status;
     int T, H, E, k;
     int logits_in;
+    int hc;           // hidden units per pipeline chunk (power of two dividing H, >= 64)
+    int stages;       // cp.async pipeline depth (2..4)
+    int stage_bytes;  // bytes of one stage (16-byte multiple)
 };
 
 // Monotone map of a float onto uint32 (larger float -> larger key); -0 is
@@ -54,81 +57,83 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 template <int TW>
 __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     constexpr int TB = 8 * TW;
-    // x chunk, transposed; rows padded by 4 floats so lanes reading different
-    // rows hit different banks while float4 reads stay 16-byte aligned.
-    __shared__ __align__(16) float xs[kHC][TB + 4];
-    // W_r chunk during the GEMM phase (dense [32][Wcols]), then the logits
-    // tile for the top-k.
-    __shared__ __align__(16) float pool[(kHC * kMaxExperts > TB * (kMaxExperts + 1)) ? kHC * kMaxExperts
-                                                                                       : TB * (kMaxExperts + 1)];
+    extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_nan;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * TB;
-    const int E = a.E, H = a.H;
+    const int E = a.E, H = a.H, HC = a.hc, S = a.stages;
     if (tid == 0) s_nan = 0;
-
-    float *wsm = pool;
-    float(*lg)[kMaxExperts + 1] = reinterpret_cast<float(*)[kMaxExperts + 1]>(pool);
+    // After the GEMM phase the pipeline buffers hold the logits tile.
+    float(*lg)[kMaxExperts + 1] = reinterpret_cast<float(*)[kMaxExperts + 1]>(smem);
 
     if (!a.logits_in) {
+        // Stage layout: x chunk [TB][HC] bf16, then the W_r chunk [HC][E] fp32.
+        const int xbytes = TB * HC * 2;
+        const int stage_bytes = a.stage_bytes;
+        const int nchunks = H / HC;
+        auto issue = [&](int c, int st) {
+            uint8_t *sx = smem + (size_t)st * stage_bytes;
+            float *sw = reinterpret_cast<float *>(sx + xbytes);
+            const int vpr = HC / 8;  // 16-byte vectors per token row
+            for (int i = tid; i < TB * vpr; i += 256) {
+                const int tok = i / vpr, v = i % vpr, t = t0 + tok;
+                void *dst = sx + ((size_t)tok * HC + v * 8) * 2;
+                if (t < a.T)
+                    cp_async16(dst, a.x + (size_t)t * H + (size_t)c * HC + v * 8);
+                else
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+            }
+            const float *src = a.w_router + (size_t)c * HC * E;  // rows c*HC .. +HC: contiguous
+            for (int i = tid; i < HC * E / 4; i += 256) cp_async16(sw + 4 * i, src + 4 * i);
+        };
         // Lane split: ES lanes across experts, HS = 32/ES lanes across hidden units.
         int ES = 1;
         while (ES < E && ES < 32) ES <<= 1;
         const int HS = 32 / ES;
         const int es = lane % ES, hs = lane / ES;
         const int EJ = (E + ES - 1) / ES;  // <= 8
-        // W chunk columns incl. zero padding.  With ES < 32 this is ES (EJ = 1),
-        // so lanes (hs, es) read word hs*ES + es of a 32-word window: no bank
-        // conflicts; with ES = 32 all lanes read one row.
-        const int Wcols = ES * EJ;
+        int ecol[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ecol[j] = min(es + ES * j, E - 1);  // reads past E are clamped and unused
         float acc[TW][8];
 #pragma unroll
         for (int i = 0; i < TW; ++i)
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
 
-        for (int h0 = 0; h0 < H; h0 += kHC) {
-            __syncthreads();
-            // x chunk: TB tokens x 32 hidden units, transposed into xs[h][token].
-            for (int i = tid; i < TB * (kHC / 2); i += 256) {
-                const int tok = i / (kHC / 2), hp = (i % (kHC / 2)) * 2;
-                const int t = t0 + tok;
-                float2 v = make_float2(0.f, 0.f);
-                if (t < a.T) {
-                    const __nv_bfloat162 b =
-                        *reinterpret_cast<const __nv_bfloat162 *>(a.x + (size_t)t * H + h0 + hp);
-                    v = __bfloat1622float2(b);
-                }
-                xs[hp][tok] = v.x;
-                xs[hp + 1][tok] = v.y;
-            }
-            // W_r chunk: rows h0..h0+31, E columns, zero-padded to Wcols.
-            for (int i = tid; i < kHC * Wcols; i += 256) {
-                const int hh = i / Wcols, e = i % Wcols;
-                wsm[hh * Wcols + e] = e < E ? a.w_router[(size_t)(h0 + hh) * E + e] : 0.0f;
-            }
-            __syncthreads();
-            for (int hh = hs; hh < kHC; hh += HS) {
-                float xv[TW];
-                if constexpr (TW == 4) {
-                    const float4 q = *reinterpret_cast<const float4 *>(&xs[hh][warp * 4]);
-                    xv[0] = q.x;
-                    xv[1] = q.y;
-                    xv[2] = q.z;
-                    xv[3] = q.w;
-                } else {
+        for (int s = 0; s < S - 1; ++s) {
+            if (s < nchunks) issue(s, s);
+            cp_async_commit();
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            if (c + S - 1 < nchunks) issue(c + S - 1, (c + S - 1) % S);
+            cp_async_commit();
+            cp_async_wait_pending(S - 1);  // this thread's copies of chunk c have landed
+            __syncthreads();               // ... and everyone else's
+            const uint8_t *sx = smem + (size_t)(c % S) * stage_bytes;
+            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx);
+            const float *wsm = reinterpret_cast<const float *>(sx + xbytes);
+            // Pairs of hidden units 2p, 2p+1; this lane takes p = hs, hs + HS, ...
+            for (int p = hs; p < HC / 2; p += HS) {
+                float2 xv[TW];
 #pragma unroll
-                    for (int i = 0; i < TW; ++i) xv[i] = xs[hh][warp * TW + i];
-                }
+                for (int i = 0; i < TW; ++i)
+                    xv[i] = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(warp * TW + i) * HC + 2 * p));
+                const float *w0 = wsm + (size_t)(2 * p) * E;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     if (j < EJ) {
-                        const float wv = wsm[hh * Wcols + es + ES * j];
+                        const float wa = w0[ecol[j]], wb = w0[E + ecol[j]];
 #pragma unroll
-                        for (int i = 0; i < TW; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+                        for (int i = 0; i < TW; ++i) {
+                            acc[i][j] = fmaf(xv[i].x, wa, acc[i][j]);
+                            acc[i][j] = fmaf(xv[i].y, wb, acc[i][j]);
+                        }
                     }
                 }
             }
+            __syncthreads();  // stage c % S may be refilled from here on
         }
         // Fold the hidden-unit split.
         for (int off = ES; off < 32; off <<= 1)
@@ -136,7 +141,6 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             for (int i = 0; i < TW; ++i)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
-        __syncthreads();  // everyone is done with wsm; pool becomes lg
         if (hs == 0) {
 #pragma unroll
             for (int i = 0; i < TW; ++i) {
@@ -216,6 +220,19 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
 
 }  // namespace
 
+template <int TW>
+cudaError_t launch_route_tw(const RouteArgs &a0, int smem_bytes, cudaStream_t stream) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(k_route<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const int TB = 8 * TW;
+    k_route<TW><<<(a0.T + TB - 1) / TB, 256, smem_bytes, stream>>>(a0);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
                          int32_t *topk_idx, float *topk_w, uint32_t *status, int num_sms, cudaStream_t stream) {
     RouteArgs a;
@@ -232,12 +249,22 @@ cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_route
     a.k = s.k;
     a.logits_in = (s.flags & MOE_FLAG_LOGITS_IN) ? 1 : 0;
     // Four tokens per warp when that still gives every SM a block.
-    if ((s.T + 31) / 32 >= num_sms) {
-        k_route<4><<<(s.T + 31) / 32, 256, 0, stream>>>(a);
-    } else {
-        k_route<1><<<(s.T + 7) / 8, 256, 0, stream>>>(a);
-    }
-    return cudaGetLastError();
+    const int TW = ((s.T + 31) / 32 >= num_sms) ? 4 : 1;
+    const int TB = 8 * TW;
+    // Chunk: the largest power of two dividing H with the stage <= 40 KiB, >= 64.
+    int hc = 1024;
+    while (hc > 64 && (s.H % hc != 0 || hc * (4 * s.E + 2 * TB) > 40 * 1024)) hc >>= 1;
+    const int stage_bytes = (int)align_up((size_t)TB * hc * 2, 16) + (int)align_up((size_t)hc * s.E * 4, 16);
+    int stages = (160 * 1024) / stage_bytes;
+    stages = stages < 2 ? 2 : (stages > 4 ? 4 : stages);
+    a.hc = hc;
+    a.stages = stages;
+    a.stage_bytes = stage_bytes;
+    int smem = stages * stage_bytes;
+    const int lg_bytes = TB * (kMaxExperts + 1) * 4;
+    if (a.logits_in || smem < lg_bytes) smem = smem > lg_bytes ? smem : lg_bytes;
+    if (a.logits_in) smem = lg_bytes;
+    return TW == 4 ? launch_route_tw<4>(a, smem, stream) : launch_route_tw<1>(a, smem, stream);
 }
 
 }  // namespace moe

@@ -17,7 +17,8 @@
  *   intermediates and the workspace `ws`).  The library never allocates,
  *   frees or synchronises, except moe_read_status, which synchronises.
  * - Memory: every data pointer is a DEVICE pointer on the current CUDA
- *   device, 16-byte aligned; `ws` is 256-byte aligned.  bf16 tensors are
+ *   device; bf16 tensors and w_router are 16-byte aligned, int32/fp32
+ *   vectors 4-byte aligned, `ws` 256-byte aligned.  bf16 tensors are
  *   passed as `void *` holding IEEE bfloat16 values.  All matrices are dense
  *   and row-major with the leading dimension equal to the row length.
  * - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  Each
