@@ -28,8 +28,9 @@ MOE_FLAG_TEST_STALL_SCAN = 0x40000000
 ABI_FUNCTIONS = (
     "moe_permuted_rows", "moe_workspace_bytes", "moe_workspace_layout", "moe_workspace_init", "moe_route",
     "moe_permute", "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward", "moe_read_status",
-    "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version",
+    "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version", "moe_permute_static",
 )
+MOE_STATIC_WS_BYTES = 1 << 20
 
 
 class MoeShape(ctypes.Structure):
@@ -101,6 +102,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_last_error_string.restype = ctypes.c_char_p
     lib.moe_version.argtypes = []
     lib.moe_version.restype = ctypes.c_int32
+    lib.moe_permute_static.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.moe_permute_static.restype = st
     _lib = lib
     return lib
 
@@ -161,6 +164,16 @@ def moe_permute(shape, x, topk_idx, expert_counts, expert_offsets, src_token, de
     _check(load_library().moe_permute(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts),
                                       _ptr(expert_offsets), _ptr(src_token), _ptr(dest_row), _ptr(x_perm),
                                       _ptr(ws), _stream(stream)), "moe_permute")
+
+
+def moe_permute_static(shape, x, topk_idx, expert_counts, expert_offsets, src_token, dest_row, x_perm, stream=None):
+    """moe_permute without a caller workspace, for callers that cannot
+    allocate device memory: the scratch is a fixed array inside the library
+    (MOE_STATIC_WS_BYTES).  Make the first call on a device before any stream
+    capture; calls that overlap on the GPU race on the shared array."""
+    _check(load_library().moe_permute_static(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts),
+                                             _ptr(expert_offsets), _ptr(src_token), _ptr(dest_row), _ptr(x_perm),
+                                             _stream(stream)), "moe_permute_static")
 
 
 def moe_grouped_swiglu(shape, x_perm, w_gate, w_up, h, ws, stream=None):

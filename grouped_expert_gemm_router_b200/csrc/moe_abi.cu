@@ -84,6 +84,13 @@ moe_status check_ws(void *ws) { return aligned(ws, 256) ? MOE_OK : MOE_ERR_WORKS
 
 }  // namespace
 
+// Shared with the other entry-point file of the library (static_ws.cu).
+moe_status moe_internal_check_shape(const moe_shape *s) { return check_shape(s); }
+moe_status moe_internal_device_info(int *num_sms) { return device_info(num_sms); }
+moe_status moe_internal_cuda_fail(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+void moe_internal_set_error(const char *msg) { std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+uint64_t moe_internal_timeout_ns() { return g_timeout_ns.load(); }
+
 extern "C" {
 
 int64_t moe_permuted_rows(const moe_shape *s) {

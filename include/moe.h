@@ -198,6 +198,33 @@ MOE_API moe_status moe_forward(const moe_shape *shape, const moe_forward_args *a
  * *device_status and, if clear != 0, resets it.  Not graph-capturable. */
 MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_status, int clear);
 
+/* Dispatch for callers that cannot allocate device memory.  (This entry
+ * point has no counterpart on the source pages; it is an interface
+ * convenience.)  Some callers cannot call cudaMalloc: code running while a
+ * stream is captured in global capture mode, where allocation calls are
+ * refused, or a plug-in whose host application owns every device
+ * allocation.  moe_permute_static computes exactly what moe_permute computes
+ * (same arguments, minus `ws`) but takes its scratch from an array of
+ * MOE_STATIC_WS_BYTES bytes compiled into the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   - It allocates nothing and calls no allocating routine.
+ *   - Shapes whose scratch (moe_workspace_bytes) exceeds MOE_STATIC_WS_BYTES
+ *     are rejected with MOE_ERR_WORKSPACE (see moe_last_error_string).
+ *   - The first call on each device (with that device current) looks up the
+ *     array's device address and zero-fills it on `stream`; make that first
+ *     call before any stream capture begins.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears what must start at zero.  Calls that overlap on the GPU
+ *     (other streams, other host threads) race on the array: order them.
+ *   - The GEMM schedule it builds stays inside the array, so the grouped GEMM
+ *     entry points still need the workspace form (moe_permute).  Device-side
+ *     faults are not reported through a status word: a pair that cannot be
+ *     placed gets dest_row = -1. */
+#define MOE_STATIC_WS_BYTES (1u << 20)
+MOE_API moe_status moe_permute_static(const moe_shape *shape, const void *x, const int32_t *topk_idx,
+                                      int32_t *expert_counts, int32_t *expert_offsets, int32_t *src_token,
+                                      int32_t *dest_row, void *x_perm, void *stream);
+
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
 
