@@ -8,7 +8,7 @@ A step is one pass of the whole path (route, histogram/scan/permute, grouped
 SwiGLU, grouped down projection, combine) over one batch of T seeded synthetic
 tokens of the Mixtral-8x7B-shaped layer (T=512, H=4096, F=14336, E=8, top-2)
 unless --config says otherwise.  Inputs are resident in HBM; L2 is flushed
-(a 256 MiB write) between timed steps, outside the timed intervals.  Each step
+(a 256 MiB write then a 256 MiB read) between timed steps, outside the timed intervals.  Each step
 is timed with CUDA events on the stream the kernels run on, between every
 entry point, so the per-kernel times come from the same timed region.
 
@@ -77,7 +77,7 @@ def workload(args):
 def config_json(cfg, extra=None):
     d = {"workload": cfg.name + ("" if cfg.alpha in (0.0,) else "-alpha%g" % cfg.alpha), "T": cfg.T, "H": cfg.H,
          "F": cfg.F, "E": cfg.E, "k": cfg.k, "C": cfg.C, "alpha": cfg.alpha, "seed": cfg.seed,
-         "l2": "flushed between timed steps (256 MiB write)"}
+         "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)"}
     if extra:
         d.update(extra)
     return d
@@ -259,8 +259,20 @@ def run_ours(args):
              bias=None if L.bias is None else torch.from_numpy(L.bias).to(dev),
              w_gate=dev_bf16(L.w_gate), w_up=dev_bf16(L.w_up), w_down=dev_bf16(L.w_down))
     ws = b["ws"]
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    class _Flush:
+        """Between timed steps: write 256 MiB (evicts everything), then read
+        another 256 MiB so the cache holds clean lines and the next step does
+        not pay for writing the first buffer back."""
+
+        def zero_(self):
+            flush_w.zero_()
+            flush_r.sum()
+
+    flush = _Flush()
 
     def step_events(ev):
         ev[0].record(stream)

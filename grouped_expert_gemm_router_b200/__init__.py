@@ -51,7 +51,8 @@ class MoeForwardArgs(ctypes.Structure):
 class MoeWsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total", "status", "num_tiles", "total_spill", "cap_cnt", "spill_cnt", "spill_off", "order",
-        "grp_tile_start", "tile_map")] + [("max_tiles", ctypes.c_int32), ("tile_rows", ctypes.c_int32)]
+        "grp_tile_start", "tile_map")] + [("max_tiles", ctypes.c_int32), ("tile_rows", ctypes.c_int32),
+                                          ("row_cap", ctypes.c_size_t)]
 
 
 class MoeError(RuntimeError):

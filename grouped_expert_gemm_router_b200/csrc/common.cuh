@@ -7,7 +7,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/moe.h"
+#include "moe.h"  // include/ is on the include path
 
 namespace moe {
 
@@ -15,7 +15,7 @@ namespace moe {
 constexpr int kScanChunk = 2048;     // routed pairs per histogram / rank block
 constexpr int kScanThreads = 256;
 constexpr int kMaxExperts = 256;
-constexpr int kTileRows = 256;       // largest UMMA N: permuted rows per GEMM tile
+constexpr int kTileRows = 256;       // largest UMMA N: most permuted rows a GEMM tile holds
 constexpr int kPieceAlign = 16;      // rows of one B-operand TMA box
 
 // Scan look-back state: a 64-bit word per (block, expert): flag << 32 | value.
@@ -27,7 +27,7 @@ constexpr uint32_t kFlagPrefix = 2u;
 // look-back state) is zeroed by a memset node before every histogram launch;
 // the status word lives outside it and is sticky.
 struct WsLayout {
-    size_t status, num_tiles, total_spill;
+    size_t status, num_tiles, total_spill, tile_rows;
     size_t counts, offsets, cap_cnt, spill_cnt, spill_off, order, grp_tile_start;
     size_t chunk_excl;            // int32[nchunks * E] exclusive per-block prefix
     size_t reset_begin;           // start of the memset range
@@ -46,10 +46,12 @@ inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
     return (int64_t)E * C + (int64_t)k * (T > C ? T - C : 0);
 }
 
-// Upper bound on the tiles the schedule builder emits.  Per expert, every
-// tile but the first holds only overflow rows and closes only when full, so
-// an expert needs at most 2 + spill/kTileRows tiles (uncapped: 1 +
-// n_e/kTileRows).  Summed: 2E + P/kTileRows.
+// Upper bound on the tiles the schedule builder emits.  Its row cap is either
+// below kTileRows, and then every expert fits one tile (<= E tiles), or equal
+// to kTileRows; then every tile of an expert but the first holds only
+// overflow rows and closes only when full, so an expert needs at most
+// 2 + spill/kTileRows tiles (uncapped: 1 + n_e/kTileRows).  Summed:
+// 2E + P/kTileRows.
 inline int max_tiles_for(int64_t P, int E) { return (int)(2 * (int64_t)E + P / kTileRows + 1); }
 
 inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
@@ -62,6 +64,7 @@ inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
     L.status = o;
     L.num_tiles = o + 4;
     L.total_spill = o + 8;
+    L.tile_rows = o + 12;
     o += 256;
     auto arr = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
     L.counts = arr(4 * (size_t)E);
@@ -85,7 +88,7 @@ inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
 // Device-side view of the workspace (pointers resolved on the host).
 struct WsPtrs {
     uint32_t *status;
-    int *num_tiles, *total_spill;
+    int *num_tiles, *total_spill, *tile_rows;
     int *counts, *offsets, *cap_cnt, *spill_cnt, *spill_off, *order, *grp_tile_start;
     int *chunk_excl;
     uint32_t *ticket;
@@ -100,6 +103,7 @@ inline WsPtrs ws_ptrs(void *ws, const WsLayout &L) {
     p.status = (uint32_t *)(b + L.status);
     p.num_tiles = (int *)(b + L.num_tiles);
     p.total_spill = (int *)(b + L.total_spill);
+    p.tile_rows = (int *)(b + L.tile_rows);
     p.counts = (int *)(b + L.counts);
     p.offsets = (int *)(b + L.offsets);
     p.cap_cnt = (int *)(b + L.cap_cnt);
@@ -200,6 +204,25 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_
             smem_u32(dst)),
         "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+// Same, with an L2 cache policy (from createpolicy) for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *tmap, uint64_t *bar, int x, int y,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -41,10 +41,11 @@ __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 
 // Tiles of one expert: its row segments (uncapped: one; capacity layout:
 // capacity slots then overflow) are cut into pieces and packed into tiles of
-// at most kTileRows rows, each piece starting on a 16-row boundary of the
-// tile and at most two pieces per tile.  Emits if `out` is non-null; returns
-// the tile count.
-__device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_start, int seg1_len, int4 *out) {
+// at most `cap` rows, each piece starting on a 16-row boundary of the tile and
+// at most two pieces per tile.  Emits if `out` is non-null; returns the tile
+// count.
+__device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_start, int seg1_len, int cap,
+                                 int4 *out) {
     int ntiles = 0, used = 0, np = 0;
     int p_start[2] = {0, 0}, p_len[2] = {0, 0};
     const int seg_start[2] = {seg0_start, seg1_start};
@@ -52,7 +53,7 @@ __device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_s
     for (int s = 0; s < 2; ++s) {
         int start = seg_start[s], len = seg_len[s];
         while (len > 0) {
-            if (used == kTileRows || np == 2) {
+            if (used == cap || np == 2) {
                 if (out) out[ntiles] = make_int4(e, p_start[0], p_len[0] | (p_len[1] << 16), p_start[1]);
                 ++ntiles;
                 used = 0;
@@ -60,7 +61,7 @@ __device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_s
                 p_len[1] = 0;
                 p_start[1] = 0;
             }
-            const int take = len < kTileRows - used ? len : kTileRows - used;
+            const int take = len < cap - used ? len : cap - used;
             p_start[np] = start;
             p_len[np] = take;
             ++np;
@@ -174,6 +175,22 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
             a.ws.spill_cnt[e] = n - cap;
         }
     }
+    // Row cap of the tiles: the largest padded row count of one expert (its
+    // capacity piece and its overflow piece each start on a 16-row boundary),
+    // capped at kTileRows.  Below the cap every expert is one tile, and the
+    // GEMM uses the spare shared memory for deeper pipelining.
+    __shared__ int s_cap;
+    if (tid == 0) s_cap = 16;
+    __syncthreads();
+    for (int e = tid; e < E; e += kScanThreads) {
+        const int n = hist[e];
+        const int cap = a.capped ? min(n, C) : n;
+        const int req = ((cap + 15) & ~15) + ((n - cap + 15) & ~15);
+        atomicMax(&s_cap, min(req, kTileRows));
+    }
+    __syncthreads();
+    const int row_cap = s_cap;
+    if (tid == 0) *a.ws.tile_rows = row_cap;
     // Expert order: descending count, ties by index (largest work first).
     __shared__ int s_rank[kMaxExperts];
     __shared__ int s_order[kMaxExperts];
@@ -192,9 +209,9 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
         if (n > 0) {
             if (a.capped) {
                 const int cap = min(n, C);
-                nt = pack_expert_tiles(e, e * C, cap, E * C + s_aux[e], n - cap, nullptr);
+                nt = pack_expert_tiles(e, e * C, cap, E * C + s_aux[e], n - cap, row_cap, nullptr);
             } else {
-                nt = pack_expert_tiles(e, s_scan[e], n, 0, 0, nullptr);
+                nt = pack_expert_tiles(e, s_scan[e], n, 0, 0, row_cap, nullptr);
             }
         }
         s_ntiles[e] = nt;
@@ -219,9 +236,9 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
         int4 *dst = a.ws.tile_map + s_scan[s_rank[e]];
         if (a.capped) {
             const int cap = min(n, C);
-            pack_expert_tiles(e, e * C, cap, E * C + a.ws.spill_off[e], n - cap, dst);
+            pack_expert_tiles(e, e * C, cap, E * C + a.ws.spill_off[e], n - cap, row_cap, dst);
         } else {
-            pack_expert_tiles(e, a.ws.offsets[e], n, 0, 0, dst);
+            pack_expert_tiles(e, a.ws.offsets[e], n, 0, 0, row_cap, dst);
         }
     }
 }

@@ -18,10 +18,16 @@
 // - Two accumulators per work unit share every B tile: gate and up for the
 //   same 128 features (mode 0), or two adjacent 128-feature blocks (mode 1).
 //   They live in tensor memory at columns [0, N) and [256, 256 + N).
-// - Persistent, warp-specialised: warp 0 issues TMA loads into a 3-stage
-//   ring of shared-memory stages (mbarrier expect-tx), warp 1 issues
-//   tcgen05.mma from one thread and commits each stage back to the producer,
-//   warps 2-5 drain tensor memory with tcgen05.ld and write bf16 results.
+// - Persistent, warp-specialised: warp 0 issues TMA loads into a ring of
+//   shared-memory stages (mbarrier expect-tx), warp 1 issues tcgen05.mma from
+//   one thread and commits each stage back to the producer, warps 2-5 drain
+//   tensor memory with tcgen05.ld and write bf16 results.
+// - Stage size follows the routing: a stage holds two 128-feature A tiles and
+//   tile_rows rows of B, where tile_rows (chosen on the device by the schedule
+//   builder from the actual counts) is the largest padded row count of any
+//   expert, capped at 256.  Fewer rows per tile leave room for more stages, so
+//   more weight bytes are in flight per SM in the weight-streaming regime
+//   (e.g. 4 stages at 144 rows, 6 at 32 rows, 3 at 256).
 // - The schedule is the device-built tile map: work unit u -> (expert group
 //   in descending-count order, feature block, row tile), feature-block-major
 //   inside an expert so that the row tiles of one expert that share a weight
@@ -42,14 +48,15 @@ namespace moe {
 namespace {
 
 constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 3;
+constexpr int kMaxStages = 8;
 constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 features (8 KiB)
 constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
-constexpr uint32_t kBBox = 16 * kBK * 2;       // TMA box: 16 rows x 64 K (2 KiB)
-constexpr uint32_t kBTile = kTileRows * kBK * 2;
-constexpr uint32_t kStage = 2 * kATile + kBTile;
+constexpr uint32_t kBRowBytes = kBK * 2;       // one B row of a stage: 128 bytes
+constexpr uint32_t kBBox = 16 * kBRowBytes;    // TMA box: 16 rows x 64 K (2 KiB)
 constexpr uint32_t kCtrlBytes = 2048;
-constexpr uint32_t kSmemBytes = kStages * kStage + 1024 + kCtrlBytes;
+constexpr uint32_t kSmemBytes = 226 * 1024;
+constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
+static_assert(2 * kATile + kTileRows * kBRowBytes <= kRingBytes, "a 256-row stage must fit");
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 256;
@@ -58,6 +65,7 @@ struct GemmArgs {
     const int4 *tile_map;
     const int *grp_tile_start;
     const int *num_tiles;
+    const int *tile_rows;  // row cap of the tiles, chosen by the schedule builder
     uint32_t *status;
     __nv_bfloat16 *out;
     int n_out;   // row length of `out`: F (mode 0) or H (mode 1)
@@ -75,7 +83,7 @@ struct Unit {
 };
 
 template <int MODE>
-__device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, Unit &U) {
+__device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, Unit &U) {
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -101,7 +109,7 @@ __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArg
     U.n0p = (U.p0l + 15) & ~15;
     U.N = U.n0p + ((U.p1l + 15) & ~15);
     U.nacc = (MODE == 0) ? 2 : ((U.fb * 256 + 128 < a.n_out) ? 2 : 1);
-    U.valid = (unsigned)U.e < (unsigned)a.E && U.N > 0 && U.N <= kTileRows && U.p0s >= 0 && U.p1s >= 0 &&
+    U.valid = (unsigned)U.e < (unsigned)a.E && U.N > 0 && U.N <= trows && U.p0s >= 0 && U.p1s >= 0 &&
               U.p0s + U.p0l <= a.P && U.p1s + U.p1l <= a.P && U.fb < a.num_fb;
 }
 
@@ -123,10 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // SW128 tiles need 1 KiB alignment
-    uint8_t *ctrl = smem + kStages * kStage;
+    uint8_t *ctrl = smem + kRingBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);
-    uint64_t *empty = full + kStages;
-    uint64_t *tfull = empty + kStages;
+    uint64_t *empty = full + kMaxStages;
+    uint64_t *tfull = empty + kMaxStages;
     uint64_t *tempty = tfull + 1;
     uint64_t *mma_done = tempty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -137,10 +145,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ntiles = *a.num_tiles;
     const int total = (ntiles < a.max_tiles ? ntiles : a.max_tiles) * a.num_fb;
     if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
+    // Stage geometry from the schedule's row cap (multiple of 16 in [16, 256]).
+    int trows = *a.tile_rows;
+    trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
+    const uint32_t stage_bytes = 2 * kATile + (uint32_t)trows * kBRowBytes;
+    const int fit = (int)(kRingBytes / stage_bytes);
+    const int nstages = fit > kMaxStages ? kMaxStages : fit;
 
     for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -170,11 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t ph = 0;
-            int issued_ph[kStages];
-            for (int s = 0; s < kStages; ++s) issued_ph[s] = -1;
+            int issued_ph[kMaxStages];
+            for (int s = 0; s < kMaxStages; ++s) issued_ph[s] = -1;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 Unit U;
-                decode_unit<MODE>(u, s_gts, a, U);
+                decode_unit<MODE>(u, s_gts, a, trows, U);
                 if (!U.valid) {
                     atomicOr(a.status, MOE_DEV_BAD_ROW);
                     continue;
@@ -190,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t *sa0 = smem + stage * kStage;
+                    uint8_t *sa0 = smem + stage * stage_bytes;
                     uint8_t *sa1 = sa0 + kATile;
                     uint8_t *sb = sa1 + kATile;
                     mbar_arrive_expect_tx(&full[stage], bytes);
@@ -205,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < nb1; ++i)
                         tma_load_2d(sb + U.n0p * (kBK * 2) + i * kBBox, &tmB, &full[stage], kx, U.p1s + 16 * i);
                     issued_ph[stage] = (int)ph;
-                    if (++stage == kStages) {
+                    if (++stage == nstages) {
                         stage = 0;
                         ph ^= 1u;
                     }
@@ -217,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Every issued copy must land before the CTA may leave.
             int never = 0;
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < nstages; ++s)
                 if (issued_ph[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)issued_ph[s], a.timeout_ns, &never);
         }
         __syncwarp();
@@ -230,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 Unit U;
-                decode_unit<MODE>(u, s_gts, a, U);
+                decode_unit<MODE>(u, s_gts, a, trows, U);
                 if (!U.valid) continue;
                 const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
                 if (!mbar_wait_bounded(tempty, tph ^ 1u, a.timeout_ns, s_abort)) {
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa0 = base + stage * kStage, sa1 = sa0 + kATile, sb = sa1 + kATile;
+                    const uint32_t sa0 = base + stage * stage_bytes, sa1 = sa0 + kATile, sb = sa1 + kATile;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // B: K-major, 16 K-elements (32 bytes) per MMA inside the 128-byte row.
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
-                    if (++stage == kStages) {
+                    if (++stage == nstages) {
                         stage = 0;
                         ph ^= 1u;
                     }
@@ -283,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t tph = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             Unit U;
-            decode_unit<MODE>(u, s_gts, a, U);
+            decode_unit<MODE>(u, s_gts, a, trows, U);
             if (!U.valid) continue;
             // The whole warp takes one decision, so the .sync.aligned loads
             // below never run with part of the warp.
@@ -377,6 +391,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.tile_map = p.tile_map;
     a.grp_tile_start = p.grp_tile_start;
     a.num_tiles = p.num_tiles;
+    a.tile_rows = p.tile_rows;
     a.status = p.status;
     a.out = (__nv_bfloat16 *)out;
     a.n_out = n_out;

@@ -120,6 +120,7 @@ moe_status moe_workspace_layout(const moe_shape *s, moe_ws_layout *out) {
     out->tile_map = L.tile_map;
     out->max_tiles = L.max_tiles;
     out->tile_rows = kTileRows;
+    out->row_cap = L.tile_rows;
     return MOE_OK;
 }
 

@@ -3,15 +3,20 @@
 // largest logits (equal logits to the lower expert index, NaN lowest) and the
 // softmax over the k selected logits.
 //
-// One CTA of 8 warps owns a block of TB = 8*TW tokens and all E experts.  The
-// logits are a small fp32 GEMM: x and W_r stream through shared memory in
-// chunks of HC hidden units (HC chosen so a chunk of W_r is about 16-40 KiB)
-// with a 2-4 stage cp.async pipeline, so several chunks are in flight per
-// CTA; each lane accumulates TW tokens x EJ experts in registers.  When E < 32 the spare lanes split the hidden dimension and
-// are folded together with shuffles at the end.  The top-k then runs one warp
-// per token: each lane holds ceil(E/32) candidates as 64-bit keys
-// (orderable logit << 32 | ~expert) and k rounds of a warp-wide max pick the
-// winners.
+// The logits are a small fp32 GEMM (T x H times H x E, E <= 256) that is
+// latency-bound at decode sizes and FMA-bound at prefill sizes:
+// - A CTA of 8 warps owns TB = 8*TW tokens (TW tokens per warp) and all E
+//   experts for a slice of the hidden dimension.  When there are few token
+//   blocks, the hidden dimension is split over a thread-block cluster of CL
+//   CTAs (CL <= 8) so that every SM gets work; the CL partial logits are summed
+//   by the cluster's rank-0 CTA through distributed shared memory, in rank
+//   order (deterministic).
+// - x and W_r stream through shared memory in chunks of HC hidden units with
+//   a 2-4 stage cp.async pipeline.  ES lanes of a warp split the experts (EJ
+//   each, a compile-time count) and HS = 32/ES lanes split the hidden units;
+//   the HS partial sums are folded with shuffles.
+// - Top-k: one warp per token, each lane holding ceil(E/32) candidates as
+//   64-bit keys (orderable logit << 32 | ~expert); k rounds of a warp max.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -20,20 +25,23 @@ namespace moe {
 
 namespace {
 
-
 struct RouteArgs {
     const __nv_bfloat16 *x;
     const float *w_router;
     const float *bias;
-    float *logits;       // output (or input with logits_in); may be null when not logits_in
+    float *logits;  // output (or input with logits_in); may be null when not logits_in
     int *topk_idx;
     float *topk_w;
     uint32_t *status;
     int T, H, E, k;
     int logits_in;
-    int hc;           // hidden units per pipeline chunk (power of two dividing H, >= 64)
+    int hc;           // hidden units per pipeline chunk (power of two, >= 64, divides slice)
     int stages;       // cp.async pipeline depth (2..4)
     int stage_bytes;  // bytes of one stage (16-byte multiple)
+    int cl;           // CTAs per cluster splitting the hidden dimension
+    int slice;        // hidden units per CTA = H / cl
+    int es;           // lanes across experts (power of two <= 32)
+    int part_off;     // byte offset of the partial-logit tile in dynamic shared memory
 };
 
 // Monotone map of a float onto uint32 (larger float -> larger key); -0 is
@@ -54,52 +62,69 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
     return v;
 }
 
-template <int TW>
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Reads a float at the same shared-memory offset in cluster CTA `rank`.
+__device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+template <int TW, int EJ>
 __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     constexpr int TB = 8 * TW;
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_nan;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * TB;
-    const int E = a.E, H = a.H, HC = a.hc, S = a.stages;
+    const int CL = a.cl;
+    const int rank = CL > 1 ? (int)cluster_rank() : 0;
+    const int t0 = (blockIdx.x / CL) * TB;
+    const int E = a.E;
     if (tid == 0) s_nan = 0;
-    // After the GEMM phase the pipeline buffers hold the logits tile.
+    // rank 0: the logits tile for the top-k, over the (finished) pipeline buffers
     float(*lg)[kMaxExperts + 1] = reinterpret_cast<float(*)[kMaxExperts + 1]>(smem);
 
     if (!a.logits_in) {
-        // Stage layout: x chunk [TB][HC] bf16, then the W_r chunk [HC][E] fp32.
+        float *part = reinterpret_cast<float *>(smem + a.part_off);  // [TB][E] partials of this slice
+        const int HC = a.hc, S = a.stages, stage_bytes = a.stage_bytes;
         const int xbytes = TB * HC * 2;
-        const int stage_bytes = a.stage_bytes;
-        const int nchunks = H / HC;
+        const int h_begin = rank * a.slice;
+        const int nchunks = a.slice / HC;
         auto issue = [&](int c, int st) {
             uint8_t *sx = smem + (size_t)st * stage_bytes;
             float *sw = reinterpret_cast<float *>(sx + xbytes);
+            const int h0 = h_begin + c * HC;
             const int vpr = HC / 8;  // 16-byte vectors per token row
             for (int i = tid; i < TB * vpr; i += 256) {
                 const int tok = i / vpr, v = i % vpr, t = t0 + tok;
                 void *dst = sx + ((size_t)tok * HC + v * 8) * 2;
                 if (t < a.T)
-                    cp_async16(dst, a.x + (size_t)t * H + (size_t)c * HC + v * 8);
+                    cp_async16(dst, a.x + (size_t)t * a.H + h0 + v * 8);
                 else
                     *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
             }
-            const float *src = a.w_router + (size_t)c * HC * E;  // rows c*HC .. +HC: contiguous
+            const float *src = a.w_router + (size_t)h0 * E;  // rows h0 .. h0+HC: contiguous
             for (int i = tid; i < HC * E / 4; i += 256) cp_async16(sw + 4 * i, src + 4 * i);
         };
-        // Lane split: ES lanes across experts, HS = 32/ES lanes across hidden units.
-        int ES = 1;
-        while (ES < E && ES < 32) ES <<= 1;
-        const int HS = 32 / ES;
+        const int ES = a.es, HS = 32 / ES;
         const int es = lane % ES, hs = lane / ES;
-        const int EJ = (E + ES - 1) / ES;  // <= 8
-        int ecol[8];
+        int ecol[EJ];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ecol[j] = min(es + ES * j, E - 1);  // reads past E are clamped and unused
-        float acc[TW][8];
+        for (int j = 0; j < EJ; ++j) ecol[j] = min(es + ES * j, E - 1);  // reads past E are clamped, unused
+        float acc[TW][EJ];
 #pragma unroll
         for (int i = 0; i < TW; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+            for (int j = 0; j < EJ; ++j) acc[i][j] = 0.0f;
 
         for (int s = 0; s < S - 1; ++s) {
             if (s < nchunks) issue(s, s);
@@ -111,25 +136,23 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             cp_async_wait_pending(S - 1);  // this thread's copies of chunk c have landed
             __syncthreads();               // ... and everyone else's
             const uint8_t *sx = smem + (size_t)(c % S) * stage_bytes;
-            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx);
+            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx) + (size_t)warp * TW * HC;
             const float *wsm = reinterpret_cast<const float *>(sx + xbytes);
             // Pairs of hidden units 2p, 2p+1; this lane takes p = hs, hs + HS, ...
+#pragma unroll 2
             for (int p = hs; p < HC / 2; p += HS) {
                 float2 xv[TW];
 #pragma unroll
                 for (int i = 0; i < TW; ++i)
-                    xv[i] = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(warp * TW + i) * HC + 2 * p));
+                    xv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)i * HC + 2 * p));
                 const float *w0 = wsm + (size_t)(2 * p) * E;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (j < EJ) {
-                        const float wa = w0[ecol[j]], wb = w0[E + ecol[j]];
+                for (int j = 0; j < EJ; ++j) {
+                    const float wa = w0[ecol[j]], wb = w0[E + ecol[j]];
 #pragma unroll
-                        for (int i = 0; i < TW; ++i) {
-                            acc[i][j] = fmaf(xv[i].x, wa, acc[i][j]);
-                            acc[i][j] = fmaf(xv[i].y, wb, acc[i][j]);
-                        }
+                    for (int i = 0; i < TW; ++i) {
+                        acc[i][j] = fmaf(xv[i].x, wa, acc[i][j]);
+                        acc[i][j] = fmaf(xv[i].y, wb, acc[i][j]);
                     }
                 }
             }
@@ -140,23 +163,33 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
 #pragma unroll
             for (int i = 0; i < TW; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
+                for (int j = 0; j < EJ; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
         if (hs == 0) {
 #pragma unroll
-            for (int i = 0; i < TW; ++i) {
-                const int tok = warp * TW + i, t = t0 + tok;
+            for (int i = 0; i < TW; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < EJ; ++j) {
                     const int e = es + ES * j;
-                    if (j < EJ && e < E) {
-                        float l = acc[i][j];
-                        if (a.bias) l = l + a.bias[e];
-                        lg[tok][e] = l;
-                        if (t < a.T && a.logits) a.logits[(size_t)t * E + e] = l;
-                    }
+                    if (e < E) part[(warp * TW + i) * E + e] = acc[i][j];
                 }
+        }
+        if (CL > 1)
+            cluster_sync_all();
+        else
+            __syncthreads();
+        if (rank == 0) {
+            // Sum the slices in rank order, add the bias, publish the logits.
+            for (int i = tid; i < TB * E; i += 256) {
+                const int tok = i / E, e = i % E, t = t0 + tok;
+                float l = part[i];
+                for (int r = 1; r < CL; ++r) l += ld_cluster_f32(part + i, (uint32_t)r);
+                if (a.bias) l = l + a.bias[e];
+                lg[tok][e] = l;
+                if (t < a.T && a.logits) a.logits[(size_t)t * E + e] = l;
             }
         }
+        if (CL > 1) cluster_sync_all();  // every slice stays readable until rank 0 is done
+        if (rank != 0) return;
     } else {
         for (int i = tid; i < TB * E; i += 256) {
             const int tok = i / E, e = i % E, t = t0 + tok;
@@ -218,20 +251,40 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     if (tid == 0 && s_nan) atomicOr(a.status, MOE_DEV_NAN_LOGIT);
 }
 
-}  // namespace
-
-template <int TW>
-cudaError_t launch_route_tw(const RouteArgs &a0, int smem_bytes, cudaStream_t stream) {
+template <int TW, int EJ>
+cudaError_t launch_one(const RouteArgs &a, int smem_bytes, int tiles, cudaStream_t stream) {
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_route<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(k_route<TW, EJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    const int TB = 8 * TW;
-    k_route<TW><<<(a0.T + TB - 1) / TB, 256, smem_bytes, stream>>>(a0);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * a.cl));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = (size_t)smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)a.cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.cl > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_route<TW, EJ>, a);
 }
+
+template <int TW>
+cudaError_t launch_tw(const RouteArgs &a, int ej, int smem, int tiles, cudaStream_t st) {
+    switch (ej) {
+        case 1: return launch_one<TW, 1>(a, smem, tiles, st);
+        case 2: return launch_one<TW, 2>(a, smem, tiles, st);
+        case 4: return launch_one<TW, 4>(a, smem, tiles, st);
+        default: return launch_one<TW, 8>(a, smem, tiles, st);
+    }
+}
+
+}  // namespace
 
 cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
                          int32_t *topk_idx, float *topk_w, uint32_t *status, int num_sms, cudaStream_t stream) {
@@ -251,20 +304,40 @@ cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_route
     // Four tokens per warp when that still gives every SM a block.
     const int TW = ((s.T + 31) / 32 >= num_sms) ? 4 : 1;
     const int TB = 8 * TW;
-    // Chunk: the largest power of two dividing H with the stage <= 40 KiB, >= 64.
+    const int tiles = (s.T + TB - 1) / TB;
+    // Split the hidden dimension over a cluster until there are ~2 blocks per SM.
+    int cl = 1;
+    if (!a.logits_in)
+        while (cl < 8 && tiles * cl < 2 * num_sms && s.H % (64 * 2 * cl) == 0) cl *= 2;
+    a.cl = cl;
+    a.slice = s.H / cl;
+    int es = 1;
+    while (es < s.E && es < 32) es <<= 1;
+    a.es = es;
+    int ej = (s.E + es - 1) / es;
+    ej = ej <= 1 ? 1 : ej <= 2 ? 2 : ej <= 4 ? 4 : 8;
+    // Chunk: the largest power of two dividing the slice with the stage <= 40 KiB, >= 64.
     int hc = 1024;
-    while (hc > 64 && (s.H % hc != 0 || hc * (4 * s.E + 2 * TB) > 40 * 1024)) hc >>= 1;
+    while (hc > 64 && (a.slice % hc != 0 || hc * (4 * s.E + 2 * TB) > 40 * 1024)) hc >>= 1;
     const int stage_bytes = (int)align_up((size_t)TB * hc * 2, 16) + (int)align_up((size_t)hc * s.E * 4, 16);
+    const int nchunks = a.slice / hc;
     int stages = (160 * 1024) / stage_bytes;
     stages = stages < 2 ? 2 : (stages > 4 ? 4 : stages);
+    if (stages > nchunks + 1) stages = nchunks + 1 < 2 ? 2 : nchunks + 1;
     a.hc = hc;
     a.stages = stages;
     a.stage_bytes = stage_bytes;
-    int smem = stages * stage_bytes;
     const int lg_bytes = TB * (kMaxExperts + 1) * 4;
-    if (a.logits_in || smem < lg_bytes) smem = smem > lg_bytes ? smem : lg_bytes;
-    if (a.logits_in) smem = lg_bytes;
-    return TW == 4 ? launch_route_tw<4>(a, smem, stream) : launch_route_tw<1>(a, smem, stream);
+    int smem;
+    if (a.logits_in) {
+        a.part_off = 0;
+        smem = lg_bytes;
+    } else {
+        const int pipe = stages * stage_bytes;
+        a.part_off = (int)align_up((size_t)(pipe > lg_bytes ? pipe : lg_bytes), 16);
+        smem = a.part_off + TB * s.E * 4;
+    }
+    return TW == 4 ? launch_tw<4>(a, ej, smem, tiles, stream) : launch_tw<1>(a, ej, smem, tiles, stream);
 }
 
 }  // namespace moe

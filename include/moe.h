@@ -129,7 +129,9 @@ typedef struct {
     size_t grp_tile_start; /* int32[E+1] first tile of the g-th expert of `order` */
     size_t tile_map;       /* int32[4*max_tiles] tiles: {e, row0, len0 | len1<<16, row1} */
     int32_t max_tiles;     /* capacity of tile_map */
-    int32_t tile_rows;     /* largest number of rows one tile holds */
+    int32_t tile_rows;     /* largest number of rows any tile can hold (256) */
+    size_t row_cap;        /* int32 row cap of the last schedule's tiles (<= tile_rows):
+                              the largest padded row count of one expert */
 } moe_ws_layout;
 
 /* Rows of the permuted buffers x_perm, h, y: T*k uncapped; with the capacity

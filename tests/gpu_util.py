@@ -96,6 +96,7 @@ def host(b, shape):
     r["grp_tile_start"] = i32(L.grp_tile_start, E + 1)
     r["tile_map"] = i32(L.tile_map, 4 * L.max_tiles).reshape(-1, 4)[:max(r["num_tiles"], 0)]
     r["max_tiles"] = L.max_tiles
+    r["row_cap"] = int(i32(L.row_cap, 1)[0])
     r["status"] = moe.moe_read_status(b["ws"], clear=True)
     return r
 
@@ -145,7 +146,7 @@ def check_tile_schedule(r, shape, counts, offsets, spill_off):
             l0, l1 = lens & 0xFFFF, (lens >> 16) & 0xFFFF
             assert te == e
             assert l0 >= 1
-            assert (l0 + 15) // 16 * 16 + (l1 + 15) // 16 * 16 <= 256
+            assert (l0 + 15) // 16 * 16 + (l1 + 15) // 16 * 16 <= r["row_cap"] <= 256
             for s, l in ((s0, l0), (s1, l1)):
                 if l:
                     assert np.all(own[s:s + l] == e), "tile rows outside expert %d" % e
@@ -153,3 +154,12 @@ def check_tile_schedule(r, shape, counts, offsets, spill_off):
         if counts[e] == 0:
             assert gts[g + 1] == gts[g]
     assert np.array_equal(covered, (own >= 0).astype(np.int64)), "every filled row in exactly one tile"
+    # the row cap is the largest padded per-expert row count, capped at 256
+    req = []
+    for e in range(E):
+        n = int(counts[e])
+        cap = min(n, C) if capped else n
+        req.append(min(256, (cap + 15) // 16 * 16 + (n - cap + 15) // 16 * 16))
+    assert r["row_cap"] == max(16, max(req))
+    if r["row_cap"] < 256:
+        assert all(gts[g + 1] - gts[g] == (1 if counts[e] else 0) for g, e in enumerate(order))
