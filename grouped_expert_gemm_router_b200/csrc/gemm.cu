@@ -17,11 +17,16 @@
 //   rounded only to 16 rows, not to a 128-row M tile.
 // - Two accumulators per work unit share every B tile: gate and up for the
 //   same 128 features (mode 0), or two adjacent 128-feature blocks (mode 1).
-//   They live in tensor memory at columns [0, N) and [256, 256 + N).
+//   Units of <= 128 rows take one 256-column half of tensor memory each, in
+//   turn, so the epilogue of one overlaps the MMAs of the next; larger units
+//   take both halves.  The epilogue finishes the values into registers and
+//   hands the accumulator back before its global stores whenever the
+//   results fit in 64 registers.
 // - Persistent, warp-specialised: warp 0 issues TMA loads into a ring of
 //   shared-memory stages (mbarrier expect-tx), warp 1 issues tcgen05.mma from
-//   one thread and commits each stage back to the producer, warps 2-5 drain
-//   tensor memory with tcgen05.ld and write bf16 results.
+//   one thread and commits each stage back to the producer, warps 2-9 drain
+//   tensor memory with tcgen05.ld (two warps per lane quarter, alternating
+//   16-column chunks) and write bf16 results.
 // - Stage size follows the routing: a stage holds two 128-feature A tiles and
 //   tile_rows rows of B, where tile_rows (chosen on the device by the schedule
 //   builder from the actual counts) is the largest padded row count of any
@@ -57,9 +62,9 @@ constexpr uint32_t kCtrlBytes = 2048;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
 static_assert(2 * kATile + kTileRows * kBRowBytes <= kRingBytes, "a 256-row stage must fit");
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                   // two per tensor-memory lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp, MMA warp, epilogue warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcc1Col = 256;
 
 struct GemmArgs {
     const int4 *tile_map;
@@ -119,6 +124,32 @@ __device__ __forceinline__ int unit_row(const Unit &U, int c) {
     return c1 < U.p1l ? U.p1s + c1 : -1;
 }
 
+// Tensor memory is two halves of 256 columns.  A unit with <= 128 rows keeps
+// both accumulators in one half (columns +0 and +128) and takes the halves in
+// turn, so the epilogue of one such unit overlaps the MMAs of the next; a
+// larger unit takes both halves (accumulator 0 in half 0, 1 in half 1).  The
+// MMA issuer and the epilogue walk the same sequence of units, so they derive
+// the same placement and barrier phases from this state.
+struct TmemPlan {
+    uint32_t uses[2] = {0u, 0u};  // completed uses of each half
+    uint32_t next = 0u;           // half for the next small unit
+    // Placement of a unit: first half and whether it spans both.
+    __device__ __forceinline__ void place(int N, uint32_t &h, bool &big) const {
+        big = N > 128;
+        h = big ? 0u : next;
+    }
+    __device__ __forceinline__ void advance(bool big, uint32_t h) {
+        if (big) {
+            ++uses[0];
+            ++uses[1];
+            next = 0u;
+        } else {
+            ++uses[h];
+            next = h ^ 1u;
+        }
+    }
+};
+
 __device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *status) {
     *abort = 1;
     atomicOr(status, MOE_DEV_GEMM_TIMEOUT);
@@ -134,9 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *ctrl = smem + kRingBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);
     uint64_t *empty = full + kMaxStages;
-    uint64_t *tfull = empty + kMaxStages;
-    uint64_t *tempty = tfull + 1;
-    uint64_t *mma_done = tempty + 1;
+    uint64_t *tfull = empty + kMaxStages;  // [2] accumulator buffer b is ready
+    uint64_t *tempty = tfull + 2;          // [2] accumulator buffer b is drained
+    uint64_t *mma_done = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);  // E + 1 <= 257 ints
@@ -158,8 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+        }
         mbar_init(mma_done, 1);
         *s_abort = 0;
         mbar_fence_init();
@@ -239,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------- MMA issuer ----
         if (lane == 0) {
             int stage = 0;
-            uint32_t ph = 0, tph = 0;
+            uint32_t ph = 0;
+            TmemPlan plan;
             const uint32_t base = smem_u32(smem);
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
@@ -247,10 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_unit<MODE>(u, s_gts, a, trows, U);
                 if (!U.valid) continue;
                 const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
-                if (!mbar_wait_bounded(tempty, tph ^ 1u, a.timeout_ns, s_abort)) {
-                    ok = false;
-                    break;
-                }
+                uint32_t h;
+                bool big;
+                plan.place(U.N, h, big);
+                const uint32_t d0 = tmem + h * 256u, d1 = big ? tmem + 256u : d0 + 128u;
+                // wait until the epilogue has drained the half(s) this unit takes
+                ok = mbar_wait_bounded(&tempty[h], (plan.uses[h] & 1u) ^ 1u, a.timeout_ns, s_abort);
+                if (ok && big) ok = mbar_wait_bounded(&tempty[1], (plan.uses[1] & 1u) ^ 1u, a.timeout_ns, s_abort);
+                if (!ok) break;
                 tc_fence_after();
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], ph, a.timeout_ns, s_abort)) {
@@ -266,10 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // A: MN-major, 16 K-rows (2 KiB) per MMA; the two 64-feature halves 8 KiB apart.
                         const uint64_t a0desc = sdesc_sw128(sa0 + kk * 2048, kABox, 1024);
                         const uint32_t accum = (kb | kk) ? 1u : 0u;
-                        tc_mma_bf16(tmem, a0desc, bdesc, idesc, accum);
+                        tc_mma_bf16(d0, a0desc, bdesc, idesc, accum);
                         if (U.nacc == 2) {
                             const uint64_t a1desc = sdesc_sw128(sa1 + kk * 2048, kABox, 1024);
-                            tc_mma_bf16(tmem + kAcc1Col, a1desc, bdesc, idesc, accum);
+                            tc_mma_bf16(d1, a1desc, bdesc, idesc, accum);
                         }
                     }
                     tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
@@ -279,8 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (!ok) break;
-                tc_commit(tfull);
-                tph ^= 1u;
+                tc_commit(&tfull[h]);
+                if (big) tc_commit(&tfull[1]);
+                plan.advance(big, h);
             }
             if (!ok && !*s_abort) raise_abort(s_abort, a.status);
             // All MMAs issued by this thread complete before tensor memory is freed.
@@ -291,46 +330,114 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // --------------------------------------------------- epilogue ----
-        const int q = warp & 3;           // tensor-memory lane quarter of this warp
-        const int L = q * 32 + lane;      // feature within a 128-feature accumulator
+        const int q = warp & 3;              // tensor-memory lane quarter of this warp
+        const int half = (warp - 2) >> 2;    // which 16-column chunks: half, half + 2, ...
+        const int L = q * 32 + lane;         // feature within a 128-feature accumulator
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-        uint32_t tph = 0;
+        TmemPlan plan;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             Unit U;
             decode_unit<MODE>(u, s_gts, a, trows, U);
             if (!U.valid) continue;
+            uint32_t h;
+            bool big;
+            plan.place(U.N, h, big);
             // The whole warp takes one decision, so the .sync.aligned loads
             // below never run with part of the warp.
-            const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, tph, a.timeout_ns, s_abort));
+            bool got = mbar_wait_bounded(&tfull[h], plan.uses[h] & 1u, a.timeout_ns, s_abort);
+            if (got && big) got = mbar_wait_bounded(&tfull[1], plan.uses[1] & 1u, a.timeout_ns, s_abort);
+            const bool ready = __all_sync(0xffffffffu, got);
             if (!ready) {
                 if (lane == 0 && !*s_abort) raise_abort(s_abort, a.status);
                 break;
             }
             tc_fence_after();
+            const uint32_t t0 = tq + h * 256u, t1 = big ? tq + 256u : t0 + 128u;
+            auto release = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&tempty[h]);
+                    if (big) mbar_arrive(&tempty[1]);
+                }
+            };
             const int f0 = MODE == 0 ? U.fb * 128 + L : U.fb * 256 + L;
-            for (int c0 = 0; c0 < U.N; c0 += 16) {
-                uint32_t r0[16], r1[16];
-                tmem_ld16(tq + (uint32_t)c0, r0);
-                if (U.nacc == 2) tmem_ld16(tq + kAcc1Col + (uint32_t)c0, r1);
-                tmem_ld_wait();
+            unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
+            if (MODE == 1 && big) {
+                // Two accumulators of up to 256 columns do not fit in
+                // registers: store while holding the accumulator.
+                for (int c0 = half * 16; c0 < U.N; c0 += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(t0 + (uint32_t)c0, r0);
+                    if (U.nacc == 2) tmem_ld16(t1 + (uint32_t)c0, r1);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int row = unit_row(U, c0 + j);
-                    if (row < 0) continue;
-                    __nv_bfloat16 *dst = a.out + (size_t)row * a.n_out + f0;
-                    if (MODE == 0) {
-                        const float g = __uint_as_float(r0[j]), v = __uint_as_float(r1[j]);
-                        dst[0] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * v);
-                    } else {
+                    for (int j = 0; j < 16; ++j) {
+                        const int row = unit_row(U, c0 + j);
+                        if (row < 0) continue;
+                        __nv_bfloat16 *dst = a.out + (size_t)row * a.n_out + f0;
                         dst[0] = __float2bfloat16_rn(__uint_as_float(r0[j]));
                         if (U.nacc == 2) dst[128] = __float2bfloat16_rn(__uint_as_float(r1[j]));
                     }
                 }
+                release();
+                plan.advance(big, h);
+                continue;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);
-            tph ^= 1u;
+            // Phase 1 (holds the accumulator): load this warp's 16-column
+            // chunks (half, half + 2, ...), finish the values and keep them as
+            // packed bf16 pairs in registers.
+            constexpr int kHoldChunks = MODE == 0 ? 8 : 4;  // mode 1 here: N <= 128
+            constexpr int kHoldWords = MODE == 0 ? 8 : 16;
+            uint32_t hold[kHoldChunks][kHoldWords];
+#pragma unroll
+            for (int i = 0; i < kHoldChunks; ++i) {
+                const int c0 = (half + 2 * i) * 16;
+                if (c0 < U.N) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(t0 + (uint32_t)c0, r0);
+                    if (U.nacc == 2) tmem_ld16(t1 + (uint32_t)c0, r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        if (MODE == 0) {
+                            const float g0 = __uint_as_float(r0[j]), v0 = __uint_as_float(r1[j]);
+                            const float g1 = __uint_as_float(r0[j + 1]), v1 = __uint_as_float(r1[j + 1]);
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * v0,
+                                                                           __fdividef(g1, 1.0f + __expf(-g1)) * v1);
+                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&p);
+                        } else {
+                            const __nv_bfloat162 p0 =
+                                __floats2bfloat162_rn(__uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
+                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&p0);
+                            if (U.nacc == 2) {
+                                const __nv_bfloat162 p1 =
+                                    __floats2bfloat162_rn(__uint_as_float(r1[j]), __uint_as_float(r1[j + 1]));
+                                hold[i][8 + j / 2] = *reinterpret_cast<const uint32_t *>(&p1);
+                            }
+                        }
+                    }
+                }
+            }
+            // Hand the accumulator back to the MMA warp before the stores.
+            release();
+            // Phase 2: the stores (one 2-byte value per row per thread; a warp
+            // covers 32 consecutive features, 64 contiguous bytes, per row).
+#pragma unroll
+            for (int i = 0; i < kHoldChunks; ++i) {
+                const int c0 = (half + 2 * i) * 16;
+                if (c0 < U.N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int row = unit_row(U, c0 + j);
+                        if (row < 0) continue;
+                        unsigned short *dst = outp + (size_t)row * a.n_out + f0;
+                        dst[0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
+                        if (MODE == 1 && U.nacc == 2) dst[128] = (unsigned short)(hold[i][8 + j / 2] >> (16 * (j & 1)));
+                    }
+                }
+            }
+            plan.advance(big, h);
         }
     }
 
