@@ -35,11 +35,20 @@ struct WsLayout {
     size_t scan_state;            // uint64[nchunks * E]
     size_t reset_end;
     size_t tile_map;              // int4[max_tiles]
+    size_t router_planes;         // bf16[3][H][router_plane_cols(E)] (tensor-core router only)
+    size_t router_logits;         // fp32[T][E] when the caller passes no logits buffer
     size_t total;
     int nchunks, max_tiles;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Router logits go to the tensor cores (three bf16 planes of W_r) for large
+// batches; below this many tokens the fp32 SIMT router is faster.
+constexpr int kTcRouterMinTokens = 2048;
+inline bool use_tc_router(int T) { return T >= kTcRouterMinTokens; }
+// Columns of one router-weight plane: E rounded up to the 64-column TMA box.
+inline int router_plane_cols(int E) { return (E + 63) / 64 * 64; }
 
 inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
     if (!capped) return (int64_t)T * k;
@@ -54,7 +63,7 @@ inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
 // 2E + P/kTileRows.
 inline int max_tiles_for(int64_t P, int E) { return (int)(2 * (int64_t)E + P / kTileRows + 1); }
 
-inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
+inline WsLayout ws_layout(int T, int H, int E, int k, int C, bool capped) {
     WsLayout L{};
     const int64_t R = (int64_t)T * k;
     const int64_t P = permuted_rows(T, E, k, C, capped);
@@ -81,6 +90,11 @@ inline WsLayout ws_layout(int T, int E, int k, int C, bool capped) {
     L.scan_state = arr(8 * (size_t)L.nchunks * E);
     L.reset_end = o;
     L.tile_map = arr(16 * (size_t)L.max_tiles);
+    L.router_planes = L.router_logits = 0;
+    if (use_tc_router(T)) {
+        L.router_planes = arr(3 * (size_t)H * router_plane_cols(E) * 2);
+        L.router_logits = arr(4 * (size_t)T * E);
+    }
     L.total = o;
     return L;
 }

@@ -6,6 +6,15 @@
 //           h[r, f] = bf16( silu(x_perm[r] . Wg[e][:, f]) * (x_perm[r] . Wu[e][:, f]) )
 //   mode 1, down projection (same page, desk editor letter):
 //           y[r, c] = bf16( h[r] . Wd[e][:, c] )
+//   mode 2, router logits of step 1 on the tensor cores (for large batches):
+//           logits[t, e] = fp32( x[t] . (P0 + P1 + P2)[:, e] ) + bias[e], where
+//           P0 + P1 + P2 is the exact three-way bf16 split of the fp32 router
+//           weights (to 2^-27 relative); every product of two bf16 values is
+//           exact in fp32.  The tensor cores' fp32 accumulator loses low bits
+//           on every accumulate, so the K loop is spread over kRouteGroups
+//           accumulators (k-block j goes to accumulator j mod kRouteGroups),
+//           each seeing a fraction of the steps, and the epilogue adds the
+//           partial sums in fp32 in a fixed order.
 //
 // Design (B200 first, not the page's Triton kernel):
 // - Swap-AB.  The MMA computes D[feature, row] = W^T[feature, k] * X^T[k, row]:
@@ -62,6 +71,7 @@ constexpr uint32_t kCtrlBytes = 2048;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
 static_assert(2 * kATile + kTileRows * kBRowBytes <= kRingBytes, "a 256-row stage must fit");
+constexpr int kRouteGroups = 8;                // mode 2: accumulators the K loop is spread over
 constexpr int kEpiWarps = 8;                   // two per tensor-memory lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp, MMA warp, epilogue warps
 constexpr uint32_t kTmemCols = 512;
@@ -80,6 +90,11 @@ struct GemmArgs {
     int P;          // rows of the permuted buffers
     int max_tiles;  // capacity of the tile map
     unsigned long long timeout_ns;
+    // mode 2 (router logits)
+    const float *bias;  // [E] or null
+    float *logits;      // [T, E]
+    int T;              // tokens
+    int route_rows;     // tokens per unit (multiple of 16, <= 256)
 };
 
 struct Unit {
@@ -89,6 +104,19 @@ struct Unit {
 
 template <int MODE>
 __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, Unit &U) {
+    if (MODE == 2) {  // unit u = tokens [u * route_rows, ...), all experts
+        U.e = 0;
+        U.fb = 0;
+        U.p0s = u * a.route_rows;
+        U.p0l = min(a.route_rows, a.T - U.p0s);
+        U.p1s = 0;
+        U.p1l = 0;
+        U.n0p = (U.p0l + 15) & ~15;
+        U.N = U.n0p;
+        U.nacc = a.E > 128 ? 2 : 1;
+        U.valid = U.p0l > 0;
+        return;
+    }
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -173,17 +201,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);  // E + 1 <= 257 ints
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ntiles = *a.num_tiles;
-    const int total = (ntiles < a.max_tiles ? ntiles : a.max_tiles) * a.num_fb;
+    int total, trows;
+    if (MODE == 2) {
+        total = (a.T + a.route_rows - 1) / a.route_rows;
+        trows = a.route_rows;
+    } else {
+        const int ntiles = *a.num_tiles;
+        total = (ntiles < a.max_tiles ? ntiles : a.max_tiles) * a.num_fb;
+        trows = *a.tile_rows;  // the schedule's row cap
+    }
     if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
-    // Stage geometry from the schedule's row cap (multiple of 16 in [16, 256]).
-    int trows = *a.tile_rows;
+    // Stage geometry: the A tiles (two accumulators; mode 2: three weight
+    // planes per accumulator) and trows rows of B (multiple of 16, <= 256).
     trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
-    const uint32_t stage_bytes = 2 * kATile + (uint32_t)trows * kBRowBytes;
+    const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
+    const uint32_t stage_bytes = a_tiles * kATile + (uint32_t)trows * kBRowBytes;
     const int fit = (int)(kRingBytes / stage_bytes);
     const int nstages = fit > kMaxStages ? kMaxStages : fit;
 
-    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
+    if (MODE != 2)
+        for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&full[s], 1);
@@ -229,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int fx0 = MODE == 0 ? U.fb * 128 : U.fb * 256;
                 const int fx1 = MODE == 0 ? U.fb * 128 : U.fb * 256 + 128;
                 const int nb0 = (U.p0l + 15) >> 4, nb1 = (U.p1l + 15) >> 4;
-                const uint32_t bytes = (uint32_t)U.nacc * kATile + (uint32_t)(nb0 + nb1) * kBBox;
+                const uint32_t a_used = MODE == 2 ? 3u * (uint32_t)U.nacc : (uint32_t)U.nacc;
+                const uint32_t bytes = a_used * kATile + (uint32_t)(nb0 + nb1) * kBBox;
                 const int krow = U.e * a.K;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -239,14 +277,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t *sa0 = smem + stage * stage_bytes;
                     uint8_t *sa1 = sa0 + kATile;
-                    uint8_t *sb = sa1 + kATile;
+                    uint8_t *sb = sa0 + a_tiles * kATile;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     const int ky = krow + kb * kBK, kx = kb * kBK;
-                    tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
-                    tma_load_2d(sa0 + kABox, &tmA0, &full[stage], fx0 + 64, ky);
-                    if (U.nacc == 2) {
-                        tma_load_2d(sa1, &tmA1, &full[stage], fx1, ky);
-                        tma_load_2d(sa1 + kABox, &tmA1, &full[stage], fx1 + 64, ky);
+                    if (MODE == 2) {
+                        // tile (plane p, accumulator c) at index p * nacc + c;
+                        // plane p holds rows [p*K, (p+1)*K) of the plane tensor
+                        for (int pl = 0; pl < 3; ++pl)
+                            for (int c = 0; c < U.nacc; ++c) {
+                                uint8_t *dst = sa0 + (uint32_t)(pl * U.nacc + c) * kATile;
+                                tma_load_2d(dst, &tmA0, &full[stage], c * 128, pl * a.K + kx);
+                                tma_load_2d(dst + kABox, &tmA0, &full[stage], c * 128 + 64, pl * a.K + kx);
+                            }
+                    } else {
+                        tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
+                        tma_load_2d(sa0 + kABox, &tmA0, &full[stage], fx0 + 64, ky);
+                        if (U.nacc == 2) {
+                            tma_load_2d(sa1, &tmA1, &full[stage], fx1, ky);
+                            tma_load_2d(sa1 + kABox, &tmA1, &full[stage], fx1 + 64, ky);
+                        }
                     }
                     for (int i = 0; i < nb0; ++i) tma_load_2d(sb + i * kBBox, &tmB, &full[stage], kx, U.p0s + 16 * i);
                     for (int i = 0; i < nb1; ++i)
@@ -283,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
                 uint32_t h;
                 bool big;
-                plan.place(U.N, h, big);
+                plan.place(MODE == 2 ? 256 : U.N, h, big);  // mode 2 uses all of tensor memory
                 const uint32_t d0 = tmem + h * 256u, d1 = big ? tmem + 256u : d0 + 128u;
                 // wait until the epilogue has drained the half(s) this unit takes
                 ok = mbar_wait_bounded(&tempty[h], (plan.uses[h] & 1u) ^ 1u, a.timeout_ns, s_abort);
@@ -296,7 +345,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa0 = base + stage * stage_bytes, sa1 = sa0 + kATile, sb = sa1 + kATile;
+                    const uint32_t sa0 = base + stage * stage_bytes, sa1 = sa0 + kATile, sb = sa0 + a_tiles * kATile;
+                    if (MODE == 2) {
+                        // accumulator (group g, expert block c) at column (g * nacc + c) * trows
+                        const int g = kb % kRouteGroups;
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t bdesc = sdesc_sw128(sb + kk * 32, 16, 1024);
+                            for (int pl = 0; pl < 3; ++pl)
+                                for (int c = 0; c < U.nacc; ++c) {
+                                    const uint32_t at = sa0 + (uint32_t)(pl * U.nacc + c) * kATile + kk * 2048;
+                                    const uint32_t dst = tmem + (uint32_t)((g * U.nacc + c) * trows);
+                                    const uint32_t accum = (kb >= kRouteGroups || kk || pl) ? 1u : 0u;
+                                    tc_mma_bf16(dst, sdesc_sw128(at, kABox, 1024), bdesc, idesc, accum);
+                                }
+                        }
+                    } else
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // B: K-major, 16 K-elements (32 bytes) per MMA inside the 128-byte row.
@@ -341,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!U.valid) continue;
             uint32_t h;
             bool big;
-            plan.place(U.N, h, big);
+            plan.place(MODE == 2 ? 256 : U.N, h, big);
             // The whole warp takes one decision, so the .sync.aligned loads
             // below never run with part of the warp.
             bool got = mbar_wait_bounded(&tfull[h], plan.uses[h] & 1u, a.timeout_ns, s_abort);
@@ -363,6 +427,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             const int f0 = MODE == 0 ? U.fb * 128 + L : U.fb * 256 + L;
             unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
+            if (MODE == 2) {
+                // fp32 logits + bias: lane L of expert block c is expert c*128 + L;
+                // the groups' partial sums are added in order g = 0, 1, ...
+                const int ng = nk < kRouteGroups ? nk : kRouteGroups;
+                for (int c0 = half * 16; c0 < U.N; c0 += 32) {
+                    for (int c = 0; c < U.nacc; ++c) {
+                        float acc[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+                        for (int g = 0; g < ng; ++g) {
+                            uint32_t r[16];
+                            tmem_ld16(tq + (uint32_t)((g * U.nacc + c) * trows + c0), r);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) acc[j] += __uint_as_float(r[j]);
+                        }
+                        const int e = c * 128 + L;
+                        const float be = (a.bias && e < a.E) ? a.bias[e] : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int row = unit_row(U, c0 + j);
+                            if (row >= 0 && e < a.E) a.logits[(size_t)row * a.E + e] = acc[j] + be;
+                        }
+                    }
+                }
+                release();
+                plan.advance(big, h);
+                continue;
+            }
             if (MODE == 1 && big) {
                 // Two accumulators of up to 256 columns do not fit in
                 // registers: store while holding the accumulator.
@@ -449,6 +542,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Exact three-way bf16 split of the router weights: p0 = bf16(w),
+// p1 = bf16(w - p0), p2 = bf16(w - p0 - p1) (each difference is exact in
+// fp32), written as planes[3][H][Ep]; columns e >= E are zero.
+__global__ void __launch_bounds__(256) k_router_planes(const float *__restrict__ w, __nv_bfloat16 *__restrict__ planes,
+                                                       int H, int E, int Ep) {
+    const size_t n = (size_t)H * Ep;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int h = (int)(i / Ep), e = (int)(i % Ep);
+        const float v = e < E ? w[(size_t)h * E + e] : 0.0f;
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(p1);
+        planes[i] = p0;
+        planes[n + i] = p1;
+        planes[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -478,6 +590,48 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
 }
 
 }  // namespace
+
+// Router logits on the tensor cores: planes of W_r into the workspace, then
+// mode 2 of the grouped GEMM (one unit per block of route_rows tokens).
+cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, const float *bias,
+                                    float *logits, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                    cudaStream_t stream) {
+    const int Ep = router_plane_cols(s.E);
+    __nv_bfloat16 *planes = (__nv_bfloat16 *)((char *)ws + L.router_planes);
+    const size_t n = (size_t)s.H * Ep;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 4 * num_sms) blocks = 4 * num_sms;
+    k_router_planes<<<blocks, 256, 0, stream>>>(w_router, planes, s.H, s.E, Ep);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    CUtensorMap tA, tB;
+    if (!make_tmap(&tA, planes, 3 * (uint64_t)s.H, (uint64_t)Ep, 64, 64) ||
+        !make_tmap(&tB, x, (uint64_t)s.T, (uint64_t)s.H, 64, 16))
+        return cudaErrorInvalidValue;
+    WsPtrs p = ws_ptrs(ws, L);
+    GemmArgs a = {};
+    a.status = p.status;
+    a.K = s.H;
+    a.E = s.E;
+    a.timeout_ns = timeout_ns;
+    a.bias = bias;
+    a.logits = logits;
+    a.T = s.T;
+    // kRouteGroups accumulators of nacc expert blocks must fit in 512 columns.
+    const int nacc = s.E > 128 ? 2 : 1;
+    const int max_rows = 512 / (kRouteGroups * nacc);
+    int rows = (s.T + num_sms - 1) / num_sms;
+    rows = (rows + 15) & ~15;
+    a.route_rows = rows < 16 ? 16 : (rows > max_rows ? max_rows : rows);
+    static bool attr_done = false;
+    if (!attr_done) {
+        err = cudaFuncSetAttribute(k_grouped_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (err != cudaSuccess) return err;
+        attr_done = true;
+    }
+    k_grouped_gemm<2><<<num_sms, kThreads, kSmemBytes, stream>>>(tA, tA, tB, a);
+    return cudaGetLastError();
+}
 
 // mode 0: act = x_perm [P,H], w0 = gate, w1 = up, out = h [P,F]
 // mode 1: act = h [P,F],      w0 = w1 = down,   out = y [P,H]

@@ -9,7 +9,8 @@
 
 namespace moe {
 cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
-                         int32_t *topk_idx, float *topk_w, uint32_t *status, int num_sms, cudaStream_t stream);
+                         int32_t *topk_idx, float *topk_w, const WsLayout &L, void *ws, uint64_t timeout_ns,
+                         int num_sms, cudaStream_t stream);
 cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
                            int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
                            void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
@@ -53,7 +54,7 @@ moe_status check_shape(const moe_shape *s) {
 }
 
 WsLayout layout_of(const moe_shape *s) {
-    return ws_layout(s->T, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
+    return ws_layout(s->T, s->H, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
 }
 
 // sm_100 check and SM count of the current device, cached per device.
@@ -149,8 +150,8 @@ moe_status moe_route(const moe_shape *s, const void *x, const float *w_router, c
     int sms = 0;
     if ((st = device_info(&sms)) != MOE_OK) return st;
     const WsLayout L = layout_of(s);
-    uint32_t *status = (uint32_t *)((char *)ws + L.status);
-    cudaError_t e = launch_route(*s, x, w_router, bias, logits, topk_idx, topk_w, status, sms, (cudaStream_t)stream);
+    cudaError_t e = launch_route(*s, x, w_router, bias, logits, topk_idx, topk_w, L, ws, g_timeout_ns.load(), sms,
+                                 (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
 }
 

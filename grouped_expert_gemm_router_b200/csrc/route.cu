@@ -286,8 +286,22 @@ cudaError_t launch_tw(const RouteArgs &a, int ej, int smem, int tiles, cudaStrea
 
 }  // namespace
 
-cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
-                         int32_t *topk_idx, float *topk_w, uint32_t *status, int num_sms, cudaStream_t stream) {
+cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, const float *bias,
+                                    float *logits, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                    cudaStream_t stream);
+
+cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_router, const float *bias, float *logits,
+                         int32_t *topk_idx, float *topk_w, const WsLayout &L, void *ws, uint64_t timeout_ns,
+                         int num_sms, cudaStream_t stream) {
+    uint32_t *status = (uint32_t *)((char *)ws + L.status);
+    moe_shape s = s0;
+    if (!(s.flags & MOE_FLAG_LOGITS_IN) && use_tc_router(s.T)) {
+        // Logits on the tensor cores, then the top-k below reads them.
+        if (!logits) logits = (float *)((char *)ws + L.router_logits);
+        cudaError_t err = launch_router_logits_tc(s, x, w_router, bias, logits, L, ws, timeout_ns, num_sms, stream);
+        if (err != cudaSuccess) return err;
+        s.flags |= MOE_FLAG_LOGITS_IN;
+    }
     RouteArgs a;
     a.x = (const __nv_bfloat16 *)x;
     a.w_router = w_router;

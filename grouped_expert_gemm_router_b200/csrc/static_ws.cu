@@ -72,11 +72,13 @@ extern "C" MOE_API moe_status moe_permute_static(const moe_shape *s, const void 
     if (!al(x, 16) || !al(x_perm, 16) || !al(topk_idx, 4) || !al(expert_counts, 4) || !al(expert_offsets, 4) ||
         !al(src_token, 4) || !al(dest_row, 4))
         return MOE_ERR_INVALID_ARG;
-    const moe::WsLayout L = moe::ws_layout(s->T, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
-    if (L.total > kStaticWsBytes) {
+    const moe::WsLayout L = moe::ws_layout(s->T, s->H, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
+    // The dispatch uses the workspace up to the router's buffers, which come last.
+    const size_t need = L.router_planes ? L.router_planes : L.total;
+    if (need > kStaticWsBytes) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "moe_permute_static: shape needs %zu bytes of scratch, the static area holds %zu",
-                      L.total, kStaticWsBytes);
+                      need, kStaticWsBytes);
         moe_internal_set_error(msg);
         return MOE_ERR_WORKSPACE;
     }
