@@ -31,17 +31,22 @@
 //   take both halves.  The epilogue finishes the values into registers and
 //   hands the accumulator back before its global stores whenever the
 //   results fit in 64 registers.
-// - Persistent, warp-specialised: warp 0 issues TMA loads into a ring of
-//   shared-memory stages (mbarrier expect-tx), warp 1 issues tcgen05.mma from
-//   one thread and commits each stage back to the producer, warps 2-9 drain
-//   tensor memory with tcgen05.ld (two warps per lane quarter, alternating
-//   16-column chunks) and write bf16 results.
-// - Stage size follows the routing: a stage holds two 128-feature A tiles and
-//   tile_rows rows of B, where tile_rows (chosen on the device by the schedule
-//   builder from the actual counts) is the largest padded row count of any
-//   expert, capped at 256.  Fewer rows per tile leave room for more stages, so
-//   more weight bytes are in flight per SM in the weight-streaming regime
-//   (e.g. 4 stages at 144 rows, 6 at 32 rows, 3 at 256).
+// - Persistent, warp-specialised: warp 0 streams weight tiles and warp 2
+//   token tiles with TMA into two rings of shared-memory stages (mbarrier
+//   expect-tx), warp 1 issues tcgen05.mma from one thread and commits each
+//   pair of stages back to the producers, warps 3-10 drain tensor memory with
+//   tcgen05.ld (two warps per lane quarter, alternating 16-column chunks) and
+//   write bf16 results.
+// - Stage sizes follow the routing.  A weight stage holds the two 128-feature
+//   A tiles of 64 K rows; a token stage holds tile_rows rows of B, where
+//   tile_rows (chosen on the device by the schedule builder from the actual
+//   counts) is the largest padded row count of any expert, capped at 256.
+//   The token ring has four stages while that leaves room for four weight
+//   stages, else three, and the weight ring takes the rest of shared
+//   memory: the fewer rows per tile, the more weight bytes are in flight per
+//   SM, which is what the weight-streaming regime of small per-expert
+//   batches is bound by (4 + 4 stages at 144 rows, 6 + 4 at 32 rows, 3 + 3
+//   at 256).
 // - The schedule is the device-built tile map: work unit u -> (expert group
 //   in descending-count order, feature block, row tile), feature-block-major
 //   inside an expert so that the row tiles of one expert that share a weight
@@ -62,7 +67,8 @@ namespace moe {
 namespace {
 
 constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row of bf16
-constexpr int kMaxStages = 8;
+constexpr int kMaxAStages = 8;
+constexpr int kMaxBStages = 4;                 // token stages: 4 while >= 4 weight stages still fit, else 3
 constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 features (8 KiB)
 constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
 constexpr uint32_t kBRowBytes = kBK * 2;       // one B row of a stage: 128 bytes
@@ -70,10 +76,12 @@ constexpr uint32_t kBBox = 16 * kBRowBytes;    // TMA box: 16 rows x 64 K (2 KiB
 constexpr uint32_t kCtrlBytes = 2048;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
-static_assert(2 * kATile + kTileRows * kBRowBytes <= kRingBytes, "a 256-row stage must fit");
+static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
+              "three weight stages and three token stages of 256 rows must fit");
 constexpr int kRouteGroups = 8;                // mode 2: accumulators the K loop is spread over
+constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
 constexpr int kEpiWarps = 8;                   // two per tensor-memory lane quarter
-constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp, MMA warp, epilogue warps
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
 
 struct GemmArgs {
@@ -191,10 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // SW128 tiles need 1 KiB alignment
     uint8_t *ctrl = smem + kRingBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(ctrl);
-    uint64_t *empty = full + kMaxStages;
-    uint64_t *tfull = empty + kMaxStages;  // [2] accumulator buffer b is ready
-    uint64_t *tempty = tfull + 2;          // [2] accumulator buffer b is drained
+    uint64_t *fullA = reinterpret_cast<uint64_t *>(ctrl);  // weight stage s has landed
+    uint64_t *emptyA = fullA + kMaxAStages;                  // weight stage s was read by its MMAs
+    uint64_t *fullB = emptyA + kMaxAStages;                  // token stage s has landed
+    uint64_t *emptyB = fullB + kMaxBStages;                  // token stage s was read by its MMAs
+    uint64_t *tfull = emptyB + kMaxBStages;                    // [2] accumulator half h is ready
+    uint64_t *tempty = tfull + 2;                            // [2] accumulator half h is drained
     uint64_t *mma_done = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -211,20 +221,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         trows = *a.tile_rows;  // the schedule's row cap
     }
     if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
-    // Stage geometry: the A tiles (two accumulators; mode 2: three weight
-    // planes per accumulator) and trows rows of B (multiple of 16, <= 256).
+    // Two rings: weight stages (the A tiles of both accumulators; mode 2:
+    // three weight planes per accumulator), streamed from HBM, and token
+    // stages of trows rows (multiple of 16, <= 256).  Four token stages
+    // while that leaves at least four weight stages, else three; the weight
+    // ring takes the rest, so that as many weight bytes as possible are in
+    // flight.
     trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
     const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
-    const uint32_t stage_bytes = a_tiles * kATile + (uint32_t)trows * kBRowBytes;
-    const int fit = (int)(kRingBytes / stage_bytes);
-    const int nstages = fit > kMaxStages ? kMaxStages : fit;
+    const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)trows * kBRowBytes;
+    int nb = kMaxBStages;
+    int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    if (fit < 4) {
+        nb = 3;
+        fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    }
+    const int na = fit > kMaxAStages ? kMaxAStages : fit;
+    uint8_t *ringB = smem + (uint32_t)na * a_bytes;  // a_bytes is a multiple of 16 KiB: 1 KiB aligned
 
     if (MODE != 2)
         for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kMaxAStages; ++s) {
+            mbar_init(&fullA[s], 1);
+            mbar_init(&emptyA[s], 1);
+        }
+        for (int s = 0; s < kMaxBStages; ++s) {
+            mbar_init(&fullB[s], 1);
+            mbar_init(&emptyB[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -249,25 +273,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int nk = a.K / kBK;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer ----
+    if (warp == 0 || warp == 2) {
+        // ----------------------------- TMA producers: warp 0 weights, warp 2 tokens ----
         if (lane == 0) {
+            const bool is_a = warp == 0;
+            const int nst = is_a ? na : nb;
+            uint64_t *full = is_a ? fullA : fullB;
+            uint64_t *empty = is_a ? emptyA : emptyB;
             int stage = 0;
             uint32_t ph = 0;
-            int issued_ph[kMaxStages];
-            for (int s = 0; s < kMaxStages; ++s) issued_ph[s] = -1;
+            int issued_ph[kMaxAStages];
+            for (int s = 0; s < kMaxAStages; ++s) issued_ph[s] = -1;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 Unit U;
                 decode_unit<MODE>(u, s_gts, a, trows, U);
                 if (!U.valid) {
-                    atomicOr(a.status, MOE_DEV_BAD_ROW);
+                    if (is_a) atomicOr(a.status, MOE_DEV_BAD_ROW);
                     continue;
                 }
                 const int fx0 = MODE == 0 ? U.fb * 128 : U.fb * 256;
                 const int fx1 = MODE == 0 ? U.fb * 128 : U.fb * 256 + 128;
                 const int nb0 = (U.p0l + 15) >> 4, nb1 = (U.p1l + 15) >> 4;
-                const uint32_t a_used = MODE == 2 ? 3u * (uint32_t)U.nacc : (uint32_t)U.nacc;
-                const uint32_t bytes = a_used * kATile + (uint32_t)(nb0 + nb1) * kBBox;
+                const uint32_t bytes = is_a ? (MODE == 2 ? 3u : 1u) * (uint32_t)U.nacc * kATile
+                                            : (uint32_t)(nb0 + nb1) * kBBox;
                 const int krow = U.e * a.K;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -275,14 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t *sa0 = smem + stage * stage_bytes;
-                    uint8_t *sa1 = sa0 + kATile;
-                    uint8_t *sb = sa0 + a_tiles * kATile;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     const int ky = krow + kb * kBK, kx = kb * kBK;
-                    if (MODE == 2) {
+                    if (!is_a) {
+                        uint8_t *sb = ringB + stage * b_bytes;
+                        for (int i = 0; i < nb0; ++i)
+                            tma_load_2d(sb + i * kBBox, &tmB, &full[stage], kx, U.p0s + 16 * i);
+                        for (int i = 0; i < nb1; ++i)
+                            tma_load_2d(sb + U.n0p * kBRowBytes + i * kBBox, &tmB, &full[stage], kx, U.p1s + 16 * i);
+                    } else if (MODE == 2) {
                         // tile (plane p, accumulator c) at index p * nacc + c;
                         // plane p holds rows [p*K, (p+1)*K) of the plane tensor
+                        uint8_t *sa0 = smem + stage * a_bytes;
                         for (int pl = 0; pl < 3; ++pl)
                             for (int c = 0; c < U.nacc; ++c) {
                                 uint8_t *dst = sa0 + (uint32_t)(pl * U.nacc + c) * kATile;
@@ -290,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_2d(dst + kABox, &tmA0, &full[stage], c * 128 + 64, pl * a.K + kx);
                             }
                     } else {
+                        uint8_t *sa0 = smem + stage * a_bytes, *sa1 = sa0 + kATile;
                         tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
                         tma_load_2d(sa0 + kABox, &tmA0, &full[stage], fx0 + 64, ky);
                         if (U.nacc == 2) {
@@ -297,11 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_2d(sa1 + kABox, &tmA1, &full[stage], fx1 + 64, ky);
                         }
                     }
-                    for (int i = 0; i < nb0; ++i) tma_load_2d(sb + i * kBBox, &tmB, &full[stage], kx, U.p0s + 16 * i);
-                    for (int i = 0; i < nb1; ++i)
-                        tma_load_2d(sb + U.n0p * (kBK * 2) + i * kBBox, &tmB, &full[stage], kx, U.p1s + 16 * i);
                     issued_ph[stage] = (int)ph;
-                    if (++stage == nstages) {
+                    if (++stage == nst) {
                         stage = 0;
                         ph ^= 1u;
                     }
@@ -313,17 +343,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Every issued copy must land before the CTA may leave.
             int never = 0;
-            for (int s = 0; s < nstages; ++s)
+            for (int s = 0; s < nst; ++s)
                 if (issued_ph[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)issued_ph[s], a.timeout_ns, &never);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
         if (lane == 0) {
-            int stage = 0;
-            uint32_t ph = 0;
+            int sa = 0, sb = 0;
+            uint32_t pha = 0, phb = 0;
             TmemPlan plan;
-            const uint32_t base = smem_u32(smem);
+            const uint32_t baseA = smem_u32(smem), baseB = smem_u32(ringB);
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 Unit U;
@@ -340,18 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], ph, a.timeout_ns, s_abort)) {
+                    if (!mbar_wait_bounded(&fullA[sa], pha, a.timeout_ns, s_abort) ||
+                        !mbar_wait_bounded(&fullB[sb], phb, a.timeout_ns, s_abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa0 = base + stage * stage_bytes, sa1 = sa0 + kATile, sb = sa0 + a_tiles * kATile;
+                    const uint32_t sa0 = baseA + sa * a_bytes, sa1 = sa0 + kATile, sbt = baseB + sb * b_bytes;
                     if (MODE == 2) {
                         // accumulator (group g, expert block c) at column (g * nacc + c) * trows
                         const int g = kb % kRouteGroups;
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
-                            const uint64_t bdesc = sdesc_sw128(sb + kk * 32, 16, 1024);
+                            const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
                             for (int pl = 0; pl < 3; ++pl)
                                 for (int c = 0; c < U.nacc; ++c) {
                                     const uint32_t at = sa0 + (uint32_t)(pl * U.nacc + c) * kATile + kk * 2048;
@@ -364,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // B: K-major, 16 K-elements (32 bytes) per MMA inside the 128-byte row.
-                        const uint64_t bdesc = sdesc_sw128(sb + kk * 32, 16, 1024);
+                        const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
                         // A: MN-major, 16 K-rows (2 KiB) per MMA; the two 64-feature halves 8 KiB apart.
                         const uint64_t a0desc = sdesc_sw128(sa0 + kk * 2048, kABox, 1024);
                         const uint32_t accum = (kb | kk) ? 1u : 0u;
@@ -374,10 +405,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_mma_bf16(d1, a1desc, bdesc, idesc, accum);
                         }
                     }
-                    tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
-                    if (++stage == nstages) {
-                        stage = 0;
-                        ph ^= 1u;
+                    // each stage is freed once these MMAs have read it
+                    tc_commit(&emptyA[sa]);
+                    tc_commit(&emptyB[sb]);
+                    if (++sa == na) {
+                        sa = 0;
+                        pha ^= 1u;
+                    }
+                    if (++sb == nb) {
+                        sb = 0;
+                        phb ^= 1u;
                     }
                 }
                 if (!ok) break;
@@ -395,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // --------------------------------------------------- epilogue ----
         const int q = warp & 3;              // tensor-memory lane quarter of this warp
-        const int half = (warp - 2) >> 2;    // which 16-column chunks: half, half + 2, ...
+        const int half = (warp - kEpiWarp0) >> 2;  // which 16-column chunks: half, half + 2, ...
         const int L = q * 32 + lane;         // feature within a 128-feature accumulator
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         TmemPlan plan;
