@@ -29,6 +29,7 @@ ABI_FUNCTIONS = (
     "moe_permuted_rows", "moe_workspace_bytes", "moe_workspace_layout", "moe_workspace_init", "moe_route",
     "moe_permute", "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward", "moe_read_status",
     "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version", "moe_permute_static",
+    "moe_route_dispatch", "moe_gather",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -85,6 +86,10 @@ def load_library(path: str = LIB_PATH):
     lib.moe_route.restype = st
     lib.moe_permute.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.moe_permute.restype = st
+    lib.moe_route_dispatch.argtypes = [sp] + [vp] * 12
+    lib.moe_route_dispatch.restype = st
+    lib.moe_gather.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.moe_gather.restype = st
     lib.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp]
     lib.moe_grouped_swiglu.restype = st
     lib.moe_grouped_down.argtypes = [sp, vp, vp, vp, vp, vp]
@@ -165,6 +170,19 @@ def moe_permute(shape, x, topk_idx, expert_counts, expert_offsets, src_token, de
     _check(load_library().moe_permute(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts),
                                       _ptr(expert_offsets), _ptr(src_token), _ptr(dest_row), _ptr(x_perm),
                                       _ptr(ws), _stream(stream)), "moe_permute")
+
+
+def moe_route_dispatch(shape, x, w_router, bias, logits, topk_idx, topk_w, expert_counts, expert_offsets, src_token,
+                       dest_row, ws, stream=None):
+    _check(load_library().moe_route_dispatch(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits),
+                                             _ptr(topk_idx), _ptr(topk_w), _ptr(expert_counts), _ptr(expert_offsets),
+                                             _ptr(src_token), _ptr(dest_row), _ptr(ws), _stream(stream)),
+           "moe_route_dispatch")
+
+
+def moe_gather(shape, x, src_token, x_perm, ws, stream=None):
+    _check(load_library().moe_gather(ctypes.byref(shape), _ptr(x), _ptr(src_token), _ptr(x_perm), _ptr(ws),
+                                     _stream(stream)), "moe_gather")
 
 
 def moe_permute_static(shape, x, topk_idx, expert_counts, expert_offsets, src_token, dest_row, x_perm, stream=None):

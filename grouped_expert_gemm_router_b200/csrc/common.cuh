@@ -31,7 +31,7 @@ struct WsLayout {
     size_t counts, offsets, cap_cnt, spill_cnt, spill_off, order, grp_tile_start;
     size_t chunk_excl;            // int32[nchunks * E] exclusive per-block prefix
     size_t reset_begin;           // start of the memset range
-    size_t ticket;                // uint32 dynamic block ticket
+    size_t ticket;                // uint32 dynamic block ticket, then uint32 router completion count
     size_t scan_state;            // uint64[nchunks * E]
     size_t reset_end;
     size_t tile_map;              // int4[max_tiles]
@@ -49,6 +49,15 @@ constexpr int kTcRouterMinTokens = 2048;
 inline bool use_tc_router(int T) { return T >= kTcRouterMinTokens; }
 // Columns of one router-weight plane: E rounded up to the 64-column TMA box.
 inline int router_plane_cols(int E) { return (E + 63) / 64 * 64; }
+
+// Routed pairs up to which moe_forward lets the router's last CTA build the
+// dispatch (histogram, scan, schedule, ranks) instead of separate kernels.
+constexpr int kFusedDispatchMaxPairs = 4096;
+
+// Outputs of the dispatch step when the router builds it (see above).
+struct FusedDispatch {
+    int32_t *counts, *offsets, *src_token, *dest_row;
+};
 
 inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
     if (!capped) return (int64_t)T * k;
@@ -106,6 +115,7 @@ struct WsPtrs {
     int *counts, *offsets, *cap_cnt, *spill_cnt, *spill_off, *order, *grp_tile_start;
     int *chunk_excl;
     uint32_t *ticket;
+    uint32_t *route_done;  // router CTAs that finished their top-k (fused dispatch)
     unsigned long long *scan_state;
     int4 *tile_map;
     int nchunks, max_tiles;
@@ -127,6 +137,7 @@ inline WsPtrs ws_ptrs(void *ws, const WsLayout &L) {
     p.grp_tile_start = (int *)(b + L.grp_tile_start);
     p.chunk_excl = (int *)(b + L.chunk_excl);
     p.ticket = (uint32_t *)(b + L.ticket);
+    p.route_done = p.ticket + 1;
     p.scan_state = (unsigned long long *)(b + L.scan_state);
     p.tile_map = (int4 *)(b + L.tile_map);
     p.nchunks = L.nchunks;

@@ -21,7 +21,7 @@
 //              zero rows for unfilled capacity slots.
 #include <cuda_bf16.h>
 
-#include "common.cuh"
+#include "dispatch_block.cuh"
 
 namespace moe {
 
@@ -37,50 +37,9 @@ struct ScanArgs {
     WsPtrs ws;
 };
 
-__device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
-
-// Tiles of one expert: its row segments (uncapped: one; capacity layout:
-// capacity slots then overflow) are cut into pieces and packed into tiles of
-// at most `cap` rows, each piece starting on a 16-row boundary of the tile and
-// at most two pieces per tile.  Emits if `out` is non-null; returns the tile
-// count.
-__device__ int pack_expert_tiles(int e, int seg0_start, int seg0_len, int seg1_start, int seg1_len, int cap,
-                                 int4 *out) {
-    int ntiles = 0, used = 0, np = 0;
-    int p_start[2] = {0, 0}, p_len[2] = {0, 0};
-    const int seg_start[2] = {seg0_start, seg1_start};
-    const int seg_len[2] = {seg0_len, seg1_len};
-    for (int s = 0; s < 2; ++s) {
-        int start = seg_start[s], len = seg_len[s];
-        while (len > 0) {
-            if (used == cap || np == 2) {
-                if (out) out[ntiles] = make_int4(e, p_start[0], p_len[0] | (p_len[1] << 16), p_start[1]);
-                ++ntiles;
-                used = 0;
-                np = 0;
-                p_len[1] = 0;
-                p_start[1] = 0;
-            }
-            const int take = len < cap - used ? len : cap - used;
-            p_start[np] = start;
-            p_len[np] = take;
-            ++np;
-            used += round16(take);
-            start += take;
-            len -= take;
-        }
-    }
-    if (np > 0) {
-        if (out) out[ntiles] = make_int4(e, p_start[0], p_len[0] | (p_len[1] << 16), p_start[1]);
-        ++ntiles;
-    }
-    return ntiles;
-}
-
 __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
-    __shared__ int hist[kMaxExperts];
-    __shared__ int s_scan[kMaxExperts + 1];
-    __shared__ int s_aux[kMaxExperts + 1];
+    __shared__ DispatchSmem sm;
+    int *hist = sm.hist;
     __shared__ int s_chunk, s_bad, s_timeout;
     const int tid = threadIdx.x, E = a.E;
     if (tid == 0) {
@@ -147,100 +106,7 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
     if (!last) return;
 
     // ---- the block with the last chunk: offsets, capacity layout, schedule ----
-    const int C = a.C;
-    if (tid == 0) {
-        int run = 0, spill = 0;
-        for (int e = 0; e < E; ++e) {
-            s_scan[e] = run;
-            run += hist[e];
-            s_aux[e] = spill;
-            const int cap = a.capped ? min(hist[e], C) : hist[e];
-            spill += hist[e] - cap;
-        }
-        s_scan[E] = run;
-        s_aux[E] = spill;
-        *a.ws.total_spill = spill;
-    }
-    __syncthreads();
-    for (int e = tid; e <= E; e += kScanThreads) {
-        a.offsets_out[e] = s_scan[e];
-        a.ws.offsets[e] = s_scan[e];
-        a.ws.spill_off[e] = s_aux[e];
-        if (e < E) {
-            const int n = hist[e];
-            const int cap = a.capped ? min(n, C) : n;
-            a.counts_out[e] = n;
-            a.ws.counts[e] = n;
-            a.ws.cap_cnt[e] = cap;
-            a.ws.spill_cnt[e] = n - cap;
-        }
-    }
-    // Row cap of the tiles: the largest padded row count of one expert (its
-    // capacity piece and its overflow piece each start on a 16-row boundary),
-    // capped at kTileRows.  Below the cap every expert is one tile, and the
-    // GEMM uses the spare shared memory for deeper pipelining.
-    __shared__ int s_cap;
-    if (tid == 0) s_cap = 16;
-    __syncthreads();
-    for (int e = tid; e < E; e += kScanThreads) {
-        const int n = hist[e];
-        const int cap = a.capped ? min(n, C) : n;
-        const int req = ((cap + 15) & ~15) + ((n - cap + 15) & ~15);
-        atomicMax(&s_cap, min(req, kTileRows));
-    }
-    __syncthreads();
-    const int row_cap = s_cap;
-    if (tid == 0) *a.ws.tile_rows = row_cap;
-    // Expert order: descending count, ties by index (largest work first).
-    __shared__ int s_rank[kMaxExperts];
-    __shared__ int s_order[kMaxExperts];
-    __shared__ int s_ntiles[kMaxExperts];
-    for (int e = tid; e < E; e += kScanThreads) {
-        const int n = hist[e];
-        int r = 0;
-        for (int f = 0; f < E; ++f) {
-            const int m = hist[f];
-            r += (m > n) || (m == n && f < e);
-        }
-        s_rank[e] = r;
-        s_order[r] = e;
-        a.ws.order[r] = e;
-        int nt = 0;
-        if (n > 0) {
-            if (a.capped) {
-                const int cap = min(n, C);
-                nt = pack_expert_tiles(e, e * C, cap, E * C + s_aux[e], n - cap, row_cap, nullptr);
-            } else {
-                nt = pack_expert_tiles(e, s_scan[e], n, 0, 0, row_cap, nullptr);
-            }
-        }
-        s_ntiles[e] = nt;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        // First tile of each expert in schedule order; s_scan held the
-        // offsets, which are in global memory by now.
-        int run = 0;
-        for (int g = 0; g < E; ++g) {
-            s_scan[g] = run;
-            run += s_ntiles[s_order[g]];
-        }
-        s_scan[E] = run;
-        *a.ws.num_tiles = run;
-    }
-    __syncthreads();
-    for (int g = tid; g <= E; g += kScanThreads) a.ws.grp_tile_start[g] = s_scan[g];
-    for (int e = tid; e < E; e += kScanThreads) {
-        const int n = hist[e];
-        if (n == 0) continue;
-        int4 *dst = a.ws.tile_map + s_scan[s_rank[e]];
-        if (a.capped) {
-            const int cap = min(n, C);
-            pack_expert_tiles(e, e * C, cap, E * C + a.ws.spill_off[e], n - cap, row_cap, dst);
-        } else {
-            pack_expert_tiles(e, a.ws.offsets[e], n, 0, 0, row_cap, dst);
-        }
-    }
+    build_schedule_block(sm, E, a.C, a.capped != 0, a.counts_out, a.offsets_out, a.ws);
 }
 
 struct RankArgs {
@@ -252,60 +118,21 @@ struct RankArgs {
 };
 
 __global__ void __launch_bounds__(kScanThreads) k_rank(RankArgs a) {
-    constexpr int W = kScanThreads / 32;
-    __shared__ int running[kMaxExperts];
-    __shared__ int wcnt[W][kMaxExperts];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, E = a.E;
+    __shared__ DispatchSmem sm;
     const int chunk = blockIdx.x;
-    for (int e = tid; e < E; e += kScanThreads) {
-        running[e] = a.ws.chunk_excl[(size_t)chunk * E + e];
-        for (int w = 0; w < W; ++w) wcnt[w][e] = 0;
+    for (int e = threadIdx.x; e <= a.E; e += kScanThreads) {
+        if (e < a.E) sm.running[e] = a.ws.chunk_excl[(size_t)chunk * a.E + e];
+        sm.offs[e] = a.ws.offsets[e];
+        sm.spoff[e] = a.ws.spill_off[e];
     }
-    __syncthreads();
     const int begin = chunk * kScanChunk, end = min(a.R, begin + kScanChunk);
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = begin; base < end; base += kScanThreads) {
-        const int i = base + tid;
-        int e = -1;
-        if (i < end) {
-            e = a.topk_idx[i];
-            if ((unsigned)e >= (unsigned)E) e = -1;
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int lrank = __popc(peers & lt_mask);
-        if (e >= 0 && lrank == 0) wcnt[warp][e] = __popc(peers);
-        __syncthreads();
-        if (e >= 0) {
-            int r = running[e] + lrank;
-            for (int w = 0; w < warp; ++w) r += wcnt[w][e];
-            int row;
-            if (!a.capped)
-                row = a.ws.offsets[e] + r;
-            else if (r < a.C)
-                row = e * a.C + r;
-            else
-                row = E * a.C + a.ws.spill_off[e] + (r - a.C);
-            if ((unsigned)row < (unsigned)a.P) {
-                a.dest_row[i] = row;
-                a.src_token[row] = i / a.k;
-            } else {
-                a.dest_row[i] = -1;
-                atomicOr(a.ws.status, MOE_DEV_BAD_ROW);
-            }
-        } else if (i < end) {
-            a.dest_row[i] = -1;
-        }
-        __syncthreads();
-        for (int f = tid; f < E; f += kScanThreads) {
-            int s = 0;
-            for (int w = 0; w < W; ++w) {
-                s += wcnt[w][f];
-                wcnt[w][f] = 0;
-            }
-            running[f] += s;
-        }
-        __syncthreads();
-    }
+    const int *topk_idx = a.topk_idx;
+    const int E = a.E;
+    auto expert_of = [topk_idx, E](int i) {
+        const int e = topk_idx[i];
+        return (unsigned)e < (unsigned)E ? e : -1;
+    };
+    rank_pairs_block(sm, expert_of, begin, end, a.E, a.k, a.C, a.capped != 0, a.P, a.dest_row, a.src_token, a.ws);
 }
 
 // One warp per permuted row; rows are [0, R) uncapped, or the E*C capacity
@@ -341,9 +168,30 @@ __global__ void __launch_bounds__(256) k_gather(const uint4 *__restrict__ x, con
 
 }  // namespace
 
-cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
-                           int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
-                           void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+// x_perm[row] = x[src_token[row]] for every filled permuted row.
+cudaError_t launch_gather(const moe_shape &s, const void *x, const int32_t *src_token, void *x_perm,
+                          const WsLayout &L, void *ws, int num_sms, cudaStream_t stream) {
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int R = s.T * s.k;
+    const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, capped);
+    WsPtrs p = ws_ptrs(ws, L);
+    const int H8 = s.H / 8;
+    const int fixed = capped ? -1 : R;
+    const int rows_hint = capped ? s.E * s.C + s.k * (s.T > s.C ? s.T - s.C : 0) : R;
+    int blocks = (rows_hint + 7) / 8;  // 8 warps per block, one row each
+    const int cap_blocks = num_sms * 8;
+    if (blocks > cap_blocks) blocks = cap_blocks;
+    if (blocks < 1) blocks = 1;
+    k_gather<<<blocks, 256, 0, stream>>>((const uint4 *)x, src_token, (uint4 *)x_perm, H8, s.T, P, fixed, s.E * s.C,
+                                         p.total_spill);
+    return cudaGetLastError();
+}
+
+// Histogram, scan, schedule and ranks (moe_permute without the row copy).
+cudaError_t launch_dispatch_index(const moe_shape &s, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                                  int32_t *src_token, int32_t *dest_row, const WsLayout &L, void *ws,
+                                  uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+    (void)num_sms;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int R = s.T * s.k;
     WsPtrs p = ws_ptrs(ws, L);
@@ -381,17 +229,16 @@ cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *top
     ra.src_token = src_token;
     ra.ws = p;
     k_rank<<<L.nchunks, kScanThreads, 0, stream>>>(ra);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const int H8 = s.H / 8;
-    const int fixed = capped ? -1 : R;
-    const int rows_hint = capped ? s.E * s.C + s.k * (s.T > s.C ? s.T - s.C : 0) : R;
-    int blocks = (rows_hint + 7) / 8;  // 8 warps per block, one row each
-    const int cap_blocks = num_sms * 8;
-    if (blocks > cap_blocks) blocks = cap_blocks;
-    if (blocks < 1) blocks = 1;
-    k_gather<<<blocks, 256, 0, stream>>>((const uint4 *)x, src_token, (uint4 *)x_perm, H8, s.T, ra.P, fixed,
-                                         s.E * s.C, p.total_spill);
     return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
+                           int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
+                           void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+    cudaError_t err =
+        launch_dispatch_index(s, topk_idx, counts, offsets, src_token, dest_row, L, ws, timeout_ns, num_sms, stream);
+    if (err != cudaSuccess) return err;
+    return launch_gather(s, x, src_token, x_perm, L, ws, num_sms, stream);
 }
 
 }  // namespace moe

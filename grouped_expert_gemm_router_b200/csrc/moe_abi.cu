@@ -10,7 +10,12 @@
 namespace moe {
 cudaError_t launch_route(const moe_shape &s, const void *x, const float *w_router, const float *bias, float *logits,
                          int32_t *topk_idx, float *topk_w, const WsLayout &L, void *ws, uint64_t timeout_ns,
-                         int num_sms, cudaStream_t stream);
+                         int num_sms, cudaStream_t stream, const FusedDispatch *fused);
+cudaError_t launch_gather(const moe_shape &s, const void *x, const int32_t *src_token, void *x_perm,
+                          const WsLayout &L, void *ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_dispatch_index(const moe_shape &s, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                                  int32_t *src_token, int32_t *dest_row, const WsLayout &L, void *ws,
+                                  uint64_t timeout_ns, int num_sms, cudaStream_t stream);
 cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,
                            int32_t *offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, const WsLayout &L,
                            void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
@@ -151,7 +156,7 @@ moe_status moe_route(const moe_shape *s, const void *x, const float *w_router, c
     if ((st = device_info(&sms)) != MOE_OK) return st;
     const WsLayout L = layout_of(s);
     cudaError_t e = launch_route(*s, x, w_router, bias, logits, topk_idx, topk_w, L, ws, g_timeout_ns.load(), sms,
-                                 (cudaStream_t)stream);
+                                 (cudaStream_t)stream, nullptr);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
 }
 
@@ -212,12 +217,64 @@ moe_status moe_combine(const moe_shape *s, const void *y, const int32_t *dest_ro
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine");
 }
 
+moe_status moe_route_dispatch(const moe_shape *s, const void *x, const float *w_router, const float *bias,
+                              float *logits, int32_t *topk_idx, float *topk_w, int32_t *expert_counts,
+                              int32_t *expert_offsets, int32_t *src_token, int32_t *dest_row, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if ((int64_t)s->T * s->k > kFusedDispatchMaxPairs || (s->flags & MOE_FLAG_TEST_STALL_SCAN)) {
+        st = moe_route(s, x, w_router, bias, logits, topk_idx, topk_w, ws, stream);
+        if (st != MOE_OK) return st;
+        if (!aligned(x, 16) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
+            !aligned(src_token, 4) || !aligned(dest_row, 4))
+            return MOE_ERR_INVALID_ARG;
+        int sms = 0;
+        if ((st = device_info(&sms)) != MOE_OK) return st;
+        const WsLayout L = layout_of(s);
+        cudaError_t e = launch_dispatch_index(*s, topk_idx, expert_counts, expert_offsets, src_token, dest_row, L, ws,
+                                              g_timeout_ns.load(), sms, (cudaStream_t)stream);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_dispatch");
+    }
+    const bool logits_in = (s->flags & MOE_FLAG_LOGITS_IN) != 0;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
+        !aligned(src_token, 4) || !aligned(dest_row, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (logits_in) {
+        if (!aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
+    } else {
+        if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_ERR_INVALID_ARG;
+        if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
+        if (logits && !aligned(logits, 4)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    const FusedDispatch fd{expert_counts, expert_offsets, src_token, dest_row};
+    cudaError_t e = launch_route(*s, x, w_router, bias, logits, topk_idx, topk_w, L, ws, g_timeout_ns.load(), sms,
+                                 (cudaStream_t)stream, &fd);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_dispatch");
+}
+
+moe_status moe_gather(const moe_shape *s, const void *x, const int32_t *src_token, void *x_perm, void *ws,
+                      void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_gather(*s, x, src_token, x_perm, L, ws, sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_gather");
+}
+
 moe_status moe_forward(const moe_shape *s, const moe_forward_args *a, void *ws, void *stream) {
     if (!a) return MOE_ERR_INVALID_ARG;
-    moe_status st = moe_route(s, a->x, a->w_router, a->bias, a->logits, a->topk_idx, a->topk_w, ws, stream);
+    moe_status st = moe_route_dispatch(s, a->x, a->w_router, a->bias, a->logits, a->topk_idx, a->topk_w,
+                                       a->expert_counts, a->expert_offsets, a->src_token, a->dest_row, ws, stream);
     if (st != MOE_OK) return st;
-    st = moe_permute(s, a->x, a->topk_idx, a->expert_counts, a->expert_offsets, a->src_token, a->dest_row, a->x_perm,
-                     ws, stream);
+    st = moe_gather(s, a->x, a->src_token, a->x_perm, ws, stream);
     if (st != MOE_OK) return st;
     st = moe_grouped_swiglu(s, a->x_perm, a->w_gate, a->w_up, a->h, ws, stream);
     if (st != MOE_OK) return st;

@@ -17,9 +17,14 @@
 //   the HS partial sums are folded with shuffles.
 // - Top-k: one warp per token, each lane holding ceil(E/32) candidates as
 //   64-bit keys (orderable logit << 32 | ~expert); k rounds of a warp max.
+// - Fused dispatch (small batches, called from moe_forward): every CTA that
+//   finished its top-k takes a ticket after a memory fence; the CTA that takes
+//   the last one (no CTA ever waits for another) builds the whole dispatch of
+//   steps 2-3 for all T*k pairs in its shared memory: histogram, scan,
+//   capacity layout, GEMM schedule and stable ranks.
 #include <cuda_bf16.h>
 
-#include "common.cuh"
+#include "dispatch_block.cuh"
 
 namespace moe {
 
@@ -42,7 +47,54 @@ struct RouteArgs {
     int slice;        // hidden units per CTA = H / cl
     int es;           // lanes across experts (power of two <= 32)
     int part_off;     // byte offset of the partial-logit tile in dynamic shared memory
+    // fused dispatch (fuse != 0)
+    int fuse;
+    int tiles;        // CTAs that run the top-k (one per token block)
+    int C, capped, P;
+    FusedDispatch out;
+    WsPtrs ws;
 };
+
+// The last router CTA to finish: the dispatch of all T*k routed pairs, in the
+// dynamic shared memory (DispatchSmem, then the pairs' experts).
+__device__ void fused_dispatch_tail(const RouteArgs &a, uint8_t *smem) {
+    DispatchSmem &sm = *reinterpret_cast<DispatchSmem *>(smem);
+    int *pairs = reinterpret_cast<int *>(smem + sizeof(DispatchSmem));
+    const int tid = threadIdx.x, E = a.E, R = a.T * a.k;
+    for (int e = tid; e < E; e += kScanThreads) {
+        sm.hist[e] = 0;
+        sm.running[e] = 0;
+    }
+    if (tid == 0) sm.flag = 0;
+    __syncthreads();
+    // All loads first (one L2 round trip), then the histogram.  The pairs were
+    // written by other CTAs: read them from L2.
+    constexpr int kPer = kFusedDispatchMaxPairs / kScanThreads;
+    int v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kScanThreads;
+        v[j] = i < R ? __ldcg(a.topk_idx + i) : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kScanThreads;
+        if (i >= R) break;
+        const int e = v[j];
+        if ((unsigned)e < (unsigned)E) {
+            pairs[i] = e;
+            atomicAdd(&sm.hist[e], 1);
+        } else {
+            pairs[i] = -1;
+            sm.flag = 1;
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && sm.flag) atomicOr(a.status, MOE_DEV_BAD_EXPERT);
+    build_schedule_block(sm, E, a.C, a.capped != 0, a.out.counts, a.out.offsets, a.ws);
+    auto expert_of = [pairs](int i) { return pairs[i]; };
+    rank_pairs_block(sm, expert_of, 0, R, E, a.k, a.C, a.capped != 0, a.P, a.out.dest_row, a.out.src_token, a.ws);
+}
 
 // Monotone map of a float onto uint32 (larger float -> larger key); -0 is
 // folded onto +0 and NaN maps to 0, below -inf (whose key is 0x007FFFFF).
@@ -198,7 +250,9 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
     __syncthreads();
 
-    // Top-k, one warp per token.
+    // Top-k, one warp per token.  Selected slot j lives in register m = j / 32
+    // of lane j % 32 (k <= E <= 256: at most 8 per lane), so the softmax needs
+    // no round trip through global memory.
     for (int i = 0; i < TW; ++i) {
         const int tok = warp * TW + i, t = t0 + tok;
         if (t >= a.T) break;
@@ -215,6 +269,10 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             }
         }
         if (__any_sync(0xffffffffu, nan) && lane == 0) s_nan = 1;
+        float sel[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) sel[m] = 0.0f;
+        float lmax = 0.0f;
         for (int j = 0; j < a.k; ++j) {
             unsigned long long best = 0ull;
 #pragma unroll
@@ -226,29 +284,48 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
                 for (int m = 0; m < 8; ++m)
                     if (m == (e >> 5)) key[m] = 0ull;
             }
-            if (lane == 0) {
-                a.topk_idx[(size_t)t * a.k + j] = e;
-                a.topk_w[(size_t)t * a.k + j] = lg[tok][e];  // selected logit, replaced below
+            const float l = lg[tok][e];  // same address in every lane: a broadcast
+            if (j == 0) lmax = l;
+            if ((j & 31) == lane) {
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    if (m == (j >> 5)) sel[m] = l;
+            }
+            if (lane == 0) a.topk_idx[(size_t)t * a.k + j] = e;
+        }
+        // Softmax over the k selected logits, reference = the largest (slot 0):
+        // per-lane partial sums over slots lane, lane + 32, ..., then a
+        // butterfly over the warp.
+        float ex[8];
+        float sum = 0.0f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            ex[m] = 0.0f;
+            if (lane + 32 * m < a.k) {
+                ex[m] = expf(sel[m] - lmax);
+                sum += ex[m];
             }
         }
-        __syncwarp();
-        // Softmax over the k selected logits, reference = the largest (slot 0).
-        const float lmax = a.topk_w[(size_t)t * a.k];
-        float s = 0.0f;
-        for (int j = lane; j < a.k; j += 32) s += expf(a.topk_w[(size_t)t * a.k + j] - lmax);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        // k <= E <= 256: at most 8 slots per lane.
-        float ex[8];
-        int n = 0;
-        for (int j = lane; j < a.k; j += 32) ex[n++] = expf(a.topk_w[(size_t)t * a.k + j] - lmax);
-        __syncwarp();
-        n = 0;
-        for (int j = lane; j < a.k; j += 32) a.topk_w[(size_t)t * a.k + j] = ex[n++] / s;
-        __syncwarp();
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            if (lane + 32 * m < a.k) a.topk_w[(size_t)t * a.k + lane + 32 * m] = ex[m] / sum;
     }
     __syncthreads();
     if (tid == 0 && s_nan) atomicOr(a.status, MOE_DEV_NAN_LOGIT);
+    if (a.fuse) {
+        // Publish this CTA's top-k, then take a ticket; the last CTA sees every
+        // other CTA's results after its own fence.
+        __threadfence();
+        __syncthreads();
+        __shared__ int s_last;
+        if (tid == 0) s_last = atomicAdd(a.ws.route_done, 1u) == (unsigned)(a.tiles - 1);
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        fused_dispatch_tail(a, smem);
+    }
 }
 
 template <int TW, int EJ>
@@ -292,9 +369,20 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
 
 cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_router, const float *bias, float *logits,
                          int32_t *topk_idx, float *topk_w, const WsLayout &L, void *ws, uint64_t timeout_ns,
-                         int num_sms, cudaStream_t stream) {
+                         int num_sms, cudaStream_t stream, const FusedDispatch *fused) {
     uint32_t *status = (uint32_t *)((char *)ws + L.status);
     moe_shape s = s0;
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
+    if (fused) {
+        if ((int64_t)s.T * s.k > kFusedDispatchMaxPairs) return cudaErrorInvalidValue;
+        // The same clearing the dispatch kernels start with.
+        cudaError_t err = cudaMemsetAsync((char *)ws + L.reset_begin, 0, L.reset_end - L.reset_begin, stream);
+        if (err != cudaSuccess) return err;
+        if (capped && (err = cudaMemsetAsync(fused->src_token, 0xFF, sizeof(int32_t) * (size_t)P, stream)) !=
+                          cudaSuccess)
+            return err;
+    }
     if (!(s.flags & MOE_FLAG_LOGITS_IN) && use_tc_router(s.T)) {
         // Logits on the tensor cores, then the top-k below reads them.
         if (!logits) logits = (float *)((char *)ws + L.router_logits);
@@ -315,14 +403,22 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     a.E = s.E;
     a.k = s.k;
     a.logits_in = (s.flags & MOE_FLAG_LOGITS_IN) ? 1 : 0;
+    a.fuse = fused ? 1 : 0;
+    a.C = s.C;
+    a.capped = capped ? 1 : 0;
+    a.P = (int)P;
+    a.out = fused ? *fused : FusedDispatch{nullptr, nullptr, nullptr, nullptr};
+    a.ws = ws_ptrs(ws, L);
     // Four tokens per warp when that still gives every SM a block.
     const int TW = ((s.T + 31) / 32 >= num_sms) ? 4 : 1;
     const int TB = 8 * TW;
     const int tiles = (s.T + TB - 1) / TB;
-    // Split the hidden dimension over a cluster until there are ~2 blocks per SM.
+    a.tiles = tiles;
+    // Split the hidden dimension over a cluster until there are about 3/4 as
+    // many blocks as SMs (measured best at 8 and 64 experts).
     int cl = 1;
     if (!a.logits_in)
-        while (cl < 8 && tiles * cl < 2 * num_sms && s.H % (64 * 2 * cl) == 0) cl *= 2;
+        while (cl < 8 && tiles * cl < (3 * num_sms) / 4 && s.H % (64 * 2 * cl) == 0) cl *= 2;
     a.cl = cl;
     a.slice = s.H / cl;
     int es = 1;
@@ -350,6 +446,10 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
         const int pipe = stages * stage_bytes;
         a.part_off = (int)align_up((size_t)(pipe > lg_bytes ? pipe : lg_bytes), 16);
         smem = a.part_off + TB * s.E * 4;
+    }
+    if (fused) {
+        const int need = (int)align_up(sizeof(DispatchSmem) + sizeof(int) * (size_t)s.T * s.k, 16);
+        if (smem < need) smem = need;
     }
     return TW == 4 ? launch_tw<4>(a, ej, smem, tiles, stream) : launch_tw<1>(a, ej, smem, tiles, stream);
 }

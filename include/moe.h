@@ -174,6 +174,24 @@ MOE_API moe_status moe_permute(const moe_shape *shape, const void *x, const int3
                        int32_t *expert_offsets, int32_t *src_token, int32_t *dest_row, void *x_perm, void *ws,
                        void *stream);
 
+/* Steps 1-3 without the row copy: moe_route, then the index part of
+ * moe_permute (expert_counts, expert_offsets, src_token, dest_row and the
+ * tile schedule in `ws`; x_perm is not written), with the same arguments,
+ * checks and results as those two calls.  For up to 4096 routed pairs
+ * (T*k <= 4096) the router's last CTA builds the dispatch in its shared
+ * memory (one kernel after a memset instead of three); above that the
+ * histogram and rank kernels of moe_permute run. */
+MOE_API moe_status moe_route_dispatch(const moe_shape *shape, const void *x, const float *w_router, const float *bias,
+                                      float *logits, int32_t *topk_idx, float *topk_w, int32_t *expert_counts,
+                                      int32_t *expert_offsets, int32_t *src_token, int32_t *dest_row, void *ws,
+                                      void *stream);
+
+/* The row copy of step 3: x_perm[row] = x[src_token[row]] for every permuted
+ * row (zeros where src_token is -1), as moe_permute writes it; reads the
+ * overflow size moe_permute / moe_route_dispatch left in `ws`. */
+MOE_API moe_status moe_gather(const moe_shape *shape, const void *x, const int32_t *src_token, void *x_perm, void *ws,
+                              void *stream);
+
 /* Step 4a, fused gate+up SwiGLU over every filled permuted row r of expert e
  * ("TritonMoE" verdict page, pith extraction key machinery):
  *   h[r,f] = bf16( silu(x_perm[r] . w_gate[e][:,f]) * (x_perm[r] . w_up[e][:,f]) ),
@@ -193,7 +211,9 @@ MOE_API moe_status moe_grouped_down(const moe_shape *shape, const void *h, const
 MOE_API moe_status moe_combine(const moe_shape *shape, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
                        void *stream);
 
-/* The five steps in order on one stream (no host sync; graph-capturable). */
+/* The five steps in order on one stream (no host sync; graph-capturable):
+ * moe_route_dispatch, moe_gather, moe_grouped_swiglu, moe_grouped_down,
+ * moe_combine. */
 MOE_API moe_status moe_forward(const moe_shape *shape, const moe_forward_args *args, void *ws, void *stream);
 
 /* Synchronises `stream`, copies the sticky device status word of `ws` to

@@ -86,8 +86,23 @@ def test_layer_parity(orc, name):
     assert_close_bf16(r["out"], o["out"], "out")
 
 
-def test_forward_entry_point_matches_steps(orc):
-    cfg = CASES["skew_E8_k3_H384"]
+# moe_forward builds the dispatch inside the router for up to 4096 routed
+# pairs and with the separate dispatch kernels above that; both must give the
+# step-by-step results bit for bit.
+FORWARD_CASES = {
+    "skew_E8_k3_H384": CASES["skew_E8_k3_H384"],
+    "capped_C7": synth.LayerConfig("t", 150, 128, 256, 12, 3, C=7, alpha=1.2, seed=10),
+    "pairs_at_fused_limit": synth.LayerConfig("t", 1024, 128, 128, 16, 4, alpha=0.7, seed=31),
+    "pairs_above_fused_limit": synth.LayerConfig("t", 1366, 128, 128, 16, 3, alpha=0.7, seed=32),
+}
+SAME_KEYS = ("logits", "topk_idx", "topk_w", "expert_counts", "expert_offsets", "dest_row", "num_tiles",
+             "total_spill", "cap_cnt", "spill_cnt", "spill_off", "order", "grp_tile_start", "tile_map", "row_cap",
+             "h", "y", "out", "status")
+
+
+@pytest.mark.parametrize("name", list(FORWARD_CASES))
+def test_forward_entry_point_matches_steps(orc, name):
+    cfg = FORWARD_CASES[name]
     L = synth.make_layer(cfg)
     shape = shape_of(cfg)
     dl = DeviceLayer(L)
@@ -96,8 +111,13 @@ def test_forward_entry_point_matches_steps(orc):
     moe.moe_forward(shape, b, b["ws"])
     torch.cuda.synchronize()
     f = host(b, shape)
-    for key in ("logits", "topk_idx", "topk_w", "dest_row", "h", "y", "out"):
+    for key in SAME_KEYS:
         assert np.array_equal(a[key], f[key]), key
+    assert a["status"] == 0
+    filled = a["src_token"] >= 0
+    assert np.array_equal(a["src_token"], f["src_token"]) if cfg.C > 0 else np.array_equal(a["src_token"][filled],
+                                                                                           f["src_token"][filled])
+    assert np.array_equal(a["x_perm"][filled], f["x_perm"][filled])
 
 
 def test_logits_in_ties(orc):
