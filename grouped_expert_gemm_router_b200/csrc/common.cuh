@@ -35,6 +35,7 @@ struct WsLayout {
     size_t scan_state;            // uint64[nchunks * E]
     size_t reset_end;
     size_t tile_map;              // int4[max_tiles]
+    size_t dispatch_end;          // end of what the dispatch step uses (the router's buffers follow)
     size_t router_planes;         // bf16[3][H][router_plane_cols(E)] (tensor-core router only)
     size_t router_logits;         // fp32[T][E] when the caller passes no logits buffer
     size_t total;
@@ -99,6 +100,7 @@ inline WsLayout ws_layout(int T, int H, int E, int k, int C, bool capped) {
     L.scan_state = arr(8 * (size_t)L.nchunks * E);
     L.reset_end = o;
     L.tile_map = arr(16 * (size_t)L.max_tiles);
+    L.dispatch_end = o;
     L.router_planes = L.router_logits = 0;
     if (use_tc_router(T)) {
         L.router_planes = arr(3 * (size_t)H * router_plane_cols(E) * 2);

@@ -34,9 +34,10 @@
 // - Persistent, warp-specialised: warp 0 streams weight tiles and warp 2
 //   token tiles with TMA into two rings of shared-memory stages (mbarrier
 //   expect-tx), warp 1 issues tcgen05.mma from one thread and commits each
-//   pair of stages back to the producers, warps 3-10 drain tensor memory with
-//   tcgen05.ld (two warps per lane quarter, alternating 16-column chunks) and
-//   write bf16 results.
+//   pair of stages back to the producers, warps 3-14 drain tensor memory with
+//   tcgen05.ld (three warps per lane quarter, taking 16-column chunks in
+//   turn) and write bf16 results.  The more epilogue warps, the sooner a
+//   finished accumulator is handed back to the MMA warp.
 // - Stage sizes follow the routing.  A weight stage holds the two 128-feature
 //   A tiles of 64 K rows; a token stage holds tile_rows rows of B, where
 //   tile_rows (chosen on the device by the schedule builder from the actual
@@ -80,7 +81,8 @@ static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
               "three weight stages and three token stages of 256 rows must fit");
 constexpr int kRouteGroups = 8;                // mode 2: accumulators the K loop is spread over
 constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
-constexpr int kEpiWarps = 8;                   // two per tensor-memory lane quarter
+constexpr int kEpiWarps = 12;                  // three per tensor-memory lane quarter
+constexpr int kEpiSub = kEpiWarps / 4;         // warps sharing one lane quarter
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
 
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // --------------------------------------------------- epilogue ----
         const int q = warp & 3;              // tensor-memory lane quarter of this warp
-        const int half = (warp - kEpiWarp0) >> 2;  // which 16-column chunks: half, half + 2, ...
+        const int sub = (warp - kEpiWarp0) >> 2;  // which 16-column chunks: sub, sub + kEpiSub, ...
         const int L = q * 32 + lane;         // feature within a 128-feature accumulator
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         TmemPlan plan;
@@ -468,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // fp32 logits + bias: lane L of expert block c is expert c*128 + L;
                 // the groups' partial sums are added in order g = 0, 1, ...
                 const int ng = nk < kRouteGroups ? nk : kRouteGroups;
-                for (int c0 = half * 16; c0 < U.N; c0 += 32) {
+                for (int c0 = sub * 16; c0 < U.N; c0 += 16 * kEpiSub) {
                     for (int c = 0; c < U.nacc; ++c) {
                         float acc[16];
 #pragma unroll
@@ -496,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (MODE == 1 && big) {
                 // Two accumulators of up to 256 columns do not fit in
                 // registers: store while holding the accumulator.
-                for (int c0 = half * 16; c0 < U.N; c0 += 32) {
+                for (int c0 = sub * 16; c0 < U.N; c0 += 16 * kEpiSub) {
                     uint32_t r0[16], r1[16];
                     tmem_ld16(t0 + (uint32_t)c0, r0);
                     if (U.nacc == 2) tmem_ld16(t1 + (uint32_t)c0, r1);
@@ -515,14 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             // Phase 1 (holds the accumulator): load this warp's 16-column
-            // chunks (half, half + 2, ...), finish the values and keep them as
+            // chunks (sub, sub + kEpiSub, ...), finish the values and keep them as
             // packed bf16 pairs in registers.
-            constexpr int kHoldChunks = MODE == 0 ? 8 : 4;  // mode 1 here: N <= 128
+            constexpr int kHoldChunks = MODE == 0 ? (16 + kEpiSub - 1) / kEpiSub   // N <= 256
+                                                  : (8 + kEpiSub - 1) / kEpiSub;   // mode 1 here: N <= 128
             constexpr int kHoldWords = MODE == 0 ? 8 : 16;
             uint32_t hold[kHoldChunks][kHoldWords];
 #pragma unroll
             for (int i = 0; i < kHoldChunks; ++i) {
-                const int c0 = (half + 2 * i) * 16;
+                const int c0 = (sub + kEpiSub * i) * 16;
                 if (c0 < U.N) {
                     uint32_t r0[16], r1[16];
                     tmem_ld16(t0 + (uint32_t)c0, r0);
@@ -555,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // covers 32 consecutive features, 64 contiguous bytes, per row).
 #pragma unroll
             for (int i = 0; i < kHoldChunks; ++i) {
-                const int c0 = (half + 2 * i) * 16;
+                const int c0 = (sub + kEpiSub * i) * 16;
                 if (c0 < U.N) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {

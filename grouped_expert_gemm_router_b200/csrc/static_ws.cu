@@ -73,8 +73,8 @@ extern "C" MOE_API moe_status moe_permute_static(const moe_shape *s, const void 
         !al(src_token, 4) || !al(dest_row, 4))
         return MOE_ERR_INVALID_ARG;
     const moe::WsLayout L = moe::ws_layout(s->T, s->H, s->E, s->k, s->C, (s->flags & MOE_FLAG_CAPACITY) != 0);
-    // The dispatch uses the workspace up to the router's buffers, which come last.
-    const size_t need = L.router_planes ? L.router_planes : L.total;
+    // The dispatch uses the workspace up to the GEMM's and the router's buffers, which come last.
+    const size_t need = L.dispatch_end;
     if (need > kStaticWsBytes) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "moe_permute_static: shape needs %zu bytes of scratch, the static area holds %zu",
