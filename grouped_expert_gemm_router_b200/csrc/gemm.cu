@@ -34,8 +34,8 @@
 // - Persistent, warp-specialised: warp 0 streams weight tiles and warp 2
 //   token tiles with TMA into two rings of shared-memory stages (mbarrier
 //   expect-tx), warp 1 issues tcgen05.mma from one thread and commits each
-//   pair of stages back to the producers, warps 3-14 drain tensor memory with
-//   tcgen05.ld (three warps per lane quarter, taking 16-column chunks in
+//   pair of stages back to the producers, warps 3-18 drain tensor memory with
+//   tcgen05.ld (four warps per lane quarter, taking 16-column chunks in
 //   turn) and write bf16 results.  The more epilogue warps, the sooner a
 //   finished accumulator is handed back to the MMA warp.
 // - Stage sizes follow the routing.  A weight stage holds the two 128-feature
@@ -81,7 +81,7 @@ static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
               "three weight stages and three token stages of 256 rows must fit");
 constexpr int kRouteGroups = 8;                // mode 2: accumulators the K loop is spread over
 constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
-constexpr int kEpiWarps = 12;                  // three per tensor-memory lane quarter
+constexpr int kEpiWarps = 16;                  // four per tensor-memory lane quarter
 constexpr int kEpiSub = kEpiWarps / 4;         // warps sharing one lane quarter
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
