@@ -29,7 +29,7 @@ ABI_FUNCTIONS = (
     "moe_permuted_rows", "moe_workspace_bytes", "moe_workspace_layout", "moe_workspace_init", "moe_route",
     "moe_permute", "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward", "moe_read_status",
     "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version", "moe_permute_static",
-    "moe_route_dispatch", "moe_gather",
+    "moe_route_dispatch", "moe_gather", "moe_grouped_swiglu_gather",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_route_dispatch.restype = st
     lib.moe_gather.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.moe_gather.restype = st
+    lib.moe_grouped_swiglu_gather.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
+    lib.moe_grouped_swiglu_gather.restype = st
     lib.moe_grouped_swiglu.argtypes = [sp, vp, vp, vp, vp, vp, vp]
     lib.moe_grouped_swiglu.restype = st
     lib.moe_grouped_down.argtypes = [sp, vp, vp, vp, vp, vp]
@@ -183,6 +185,12 @@ def moe_route_dispatch(shape, x, w_router, bias, logits, topk_idx, topk_w, exper
 def moe_gather(shape, x, src_token, x_perm, ws, stream=None):
     _check(load_library().moe_gather(ctypes.byref(shape), _ptr(x), _ptr(src_token), _ptr(x_perm), _ptr(ws),
                                      _stream(stream)), "moe_gather")
+
+
+def moe_grouped_swiglu_gather(shape, x, src_token, w_gate, w_up, h, ws, stream=None):
+    _check(load_library().moe_grouped_swiglu_gather(ctypes.byref(shape), _ptr(x), _ptr(src_token), _ptr(w_gate),
+                                                    _ptr(w_up), _ptr(h), _ptr(ws), _stream(stream)),
+           "moe_grouped_swiglu_gather")
 
 
 def moe_permute_static(shape, x, topk_idx, expert_counts, expert_offsets, src_token, dest_row, x_perm, stream=None):

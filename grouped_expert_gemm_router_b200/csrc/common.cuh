@@ -241,6 +241,18 @@ __device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *tmap, ui
         "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
+// Four rows (tensor-map row coordinates r0..r3) of one tensor-map box column
+// range starting at column x, into 4 consecutive box rows at dst.  The tensor
+// map's box must be one row high; with the 128-byte swizzle each row lands in
+// its own 128-byte line, swizzled by its shared-memory address.
+__device__ __forceinline__ void tma_gather4(void *dst, const void *tmap, uint64_t *bar, int x, int r0, int r1,
+                                            int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -74,7 +74,7 @@ constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 featur
 constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
 constexpr uint32_t kBRowBytes = kBK * 2;       // one B row of a stage: 128 bytes
 constexpr uint32_t kBBox = 16 * kBRowBytes;    // TMA box: 16 rows x 64 K (2 KiB)
-constexpr uint32_t kCtrlBytes = 2048;
+constexpr uint32_t kCtrlBytes = 3072;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
 static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
@@ -104,6 +104,8 @@ struct GemmArgs {
     const float *bias;  // [E] or null
     float *logits;      // [T, E]
     int T;              // tokens
+    // mode 0 with the row gather: the B rows come from x[src_token[row]]
+    const int *src_token;
     int route_rows;     // tokens per unit (multiple of 16, <= 256)
 };
 
@@ -193,10 +195,14 @@ __device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *statu
     atomicOr(status, MOE_DEV_GEMM_TIMEOUT);
 }
 
-template <int MODE>
+// GATHER (mode 0 only): tmB maps the tokens x [T, H] with one-row boxes and
+// the token-tile producer gathers each unit's rows x[src_token[row]] with
+// tile::gather4 loads, so the permuted copy x_perm is never materialised.
+template <int MODE, bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+    static_assert(!GATHER || MODE == 0, "the row gather feeds the SwiGLU GEMM");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // SW128 tiles need 1 KiB alignment
@@ -211,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);  // E + 1 <= 257 ints
+    int *s_rows = s_gts + 260;                             // GATHER: token of each row of the unit (<= 256)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int total, trows;
@@ -275,7 +282,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int nk = a.K / kBK;
 
-    if (warp == 0 || warp == 2) {
+    if (GATHER && warp == 2) {
+        // ------------------- token rows gathered from x by src_token (warp 2) ----
+        // tile::gather4 loads of four rows x[src_token[r]] each (one-row
+        // boxes, 128-byte swizzle by shared-memory address, so the rows land
+        // exactly where a tiled load of x_perm would put them).  The TMA unit
+        // moves these at a lower rate than whole tiles, so this pays off when
+        // units have few rows (the gather pass it replaces dominates then).
+        int stage = 0;
+        uint32_t ph = 0;
+        int issued_ph[kMaxBStages];
+        for (int s = 0; s < kMaxBStages; ++s) issued_ph[s] = -1;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            Unit U;
+            decode_unit<MODE>(u, s_gts, a, trows, U);
+            if (!U.valid) continue;
+            // The unit's tokens, one per tile row; padding rows repeat the
+            // first row (their results are never stored).  Loads already
+            // issued took their row coordinates from registers.
+            __syncwarp();
+            bool bad = false;
+            for (int c = lane; c < U.N; c += 32) {
+                int r = unit_row(U, c);
+                if (r < 0) r = U.p0s;
+                int t = a.src_token[r];
+                if ((unsigned)t >= (unsigned)a.T) {
+                    bad = true;
+                    t = 0;
+                }
+                s_rows[c] = t;
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, MOE_DEV_BAD_ROW);
+            __syncwarp();
+            const uint32_t bytes = (uint32_t)U.N * kBRowBytes;
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                int got = 1;
+                if (lane == 0) got = mbar_wait_bounded(&emptyB[stage], ph ^ 1u, a.timeout_ns, s_abort);
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&fullB[stage], bytes);
+                    uint8_t *sb = ringB + stage * b_bytes;
+                    const int kx = kb * kBK;
+                    for (int g = 0; g < U.N; g += 4)
+                        tma_gather4(sb + g * kBRowBytes, &tmB, &fullB[stage], kx, s_rows[g], s_rows[g + 1],
+                                    s_rows[g + 2], s_rows[g + 3]);
+                    issued_ph[stage] = (int)ph;
+                }
+                if (++stage == nb) {
+                    stage = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!ok) {
+                if (lane == 0 && !*s_abort) raise_abort(s_abort, a.status);
+                break;
+            }
+        }
+        // Every issued copy must land before the CTA may leave.
+        if (lane == 0) {
+            int never = 0;
+            for (int s = 0; s < nb; ++s)
+                if (issued_ph[s] >= 0) mbar_wait_bounded(&fullB[s], (uint32_t)issued_ph[s], a.timeout_ns, &never);
+        }
+        __syncwarp();
+    } else if (warp == 0 || warp == 2) {
         // ----------------------------- TMA producers: warp 0 weights, warp 2 tokens ----
         if (lane == 0) {
             const bool is_a = warp == 0;
@@ -674,10 +748,12 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
 }
 
 // mode 0: act = x_perm [P,H], w0 = gate, w1 = up, out = h [P,F]
+//         (with src_token: act = x [T,H], rows gathered as x[src_token[row]])
 // mode 1: act = h [P,F],      w0 = w1 = down,   out = y [P,H]
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const int32_t *src_token) {
+    const bool gather = mode == 0 && src_token != nullptr;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
     const int K = mode == 0 ? s.H : s.F;
@@ -685,10 +761,11 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     CUtensorMap tA0, tA1, tB;
     if (!make_tmap(&tA0, w0, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
         !make_tmap(&tA1, w1, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
-        !make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16))
+        !(gather ? make_tmap(&tB, act, (uint64_t)s.T, (uint64_t)K, 64, 1)
+                 : make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16)))
         return cudaErrorInvalidValue;
     WsPtrs p = ws_ptrs(ws, L);
-    GemmArgs a;
+    GemmArgs a = {};
     a.tile_map = p.tile_map;
     a.grp_tile_start = p.grp_tile_start;
     a.num_tiles = p.num_tiles;
@@ -702,9 +779,19 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.P = (int)P;
     a.max_tiles = L.max_tiles;
     a.timeout_ns = timeout_ns;
-    static bool attr_done[2] = {false, false};
+    a.T = s.T;
+    a.src_token = src_token;
+    static bool attr_done[3] = {false, false, false};
     cudaError_t err;
-    if (mode == 0) {
+    if (gather) {
+        if (!attr_done[2]) {
+            err = cudaFuncSetAttribute(k_grouped_gemm<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+            if (err != cudaSuccess) return err;
+            attr_done[2] = true;
+        }
+        k_grouped_gemm<0, true><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+    } else if (mode == 0) {
         if (!attr_done[0]) {
             err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (err != cudaSuccess) return err;

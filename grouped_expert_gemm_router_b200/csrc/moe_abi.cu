@@ -21,7 +21,7 @@ cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *top
                            void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const int32_t *src_token);
 cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
                            cudaStream_t stream);
 }  // namespace moe
@@ -188,8 +188,23 @@ moe_status moe_grouped_swiglu(const moe_shape *s, const void *x_perm, const void
     if ((st = device_info(&sms)) != MOE_OK) return st;
     const WsLayout L = layout_of(s);
     cudaError_t e = launch_grouped_gemm(0, *s, x_perm, w_gate, w_up, h, L, ws, g_timeout_ns.load(), sms,
-                                        (cudaStream_t)stream);
+                                        (cudaStream_t)stream, nullptr);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_swiglu");
+}
+
+moe_status moe_grouped_swiglu_gather(const moe_shape *s, const void *x, const int32_t *src_token, const void *w_gate,
+                                     const void *w_up, void *h, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(x, 16) || !aligned(src_token, 4) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(h, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_grouped_gemm(0, *s, x, w_gate, w_up, h, L, ws, g_timeout_ns.load(), sms,
+                                        (cudaStream_t)stream, src_token);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_swiglu_gather");
 }
 
 moe_status moe_grouped_down(const moe_shape *s, const void *h, const void *w_down, void *y, void *ws, void *stream) {
@@ -201,7 +216,7 @@ moe_status moe_grouped_down(const moe_shape *s, const void *h, const void *w_dow
     if ((st = device_info(&sms)) != MOE_OK) return st;
     const WsLayout L = layout_of(s);
     cudaError_t e = launch_grouped_gemm(1, *s, h, w_down, w_down, y, L, ws, g_timeout_ns.load(), sms,
-                                        (cudaStream_t)stream);
+                                        (cudaStream_t)stream, nullptr);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down");
 }
 
@@ -274,9 +289,13 @@ moe_status moe_forward(const moe_shape *s, const moe_forward_args *a, void *ws, 
     moe_status st = moe_route_dispatch(s, a->x, a->w_router, a->bias, a->logits, a->topk_idx, a->topk_w,
                                        a->expert_counts, a->expert_offsets, a->src_token, a->dest_row, ws, stream);
     if (st != MOE_OK) return st;
-    st = moe_gather(s, a->x, a->src_token, a->x_perm, ws, stream);
-    if (st != MOE_OK) return st;
-    st = moe_grouped_swiglu(s, a->x_perm, a->w_gate, a->w_up, a->h, ws, stream);
+    if (a->x_perm) {
+        st = moe_gather(s, a->x, a->src_token, a->x_perm, ws, stream);
+        if (st != MOE_OK) return st;
+        st = moe_grouped_swiglu(s, a->x_perm, a->w_gate, a->w_up, a->h, ws, stream);
+    } else {
+        st = moe_grouped_swiglu_gather(s, a->x, a->src_token, a->w_gate, a->w_up, a->h, ws, stream);
+    }
     if (st != MOE_OK) return st;
     st = moe_grouped_down(s, a->h, a->w_down, a->y, ws, stream);
     if (st != MOE_OK) return st;

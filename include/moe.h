@@ -110,7 +110,7 @@ typedef struct {
     int32_t *expert_offsets; /* [E+1] exclusive prefix sum of expert_counts */
     int32_t *src_token;    /* [P]     token of each permuted row, -1 = empty slot */
     int32_t *dest_row;     /* [T*k]   permuted row of each routed pair */
-    void *x_perm;          /* [P,H]   bf16 permuted tokens */
+    void *x_perm;          /* [P,H]   bf16 permuted tokens, or NULL: not produced (see moe_forward) */
     void *h;               /* [P,F]   bf16 SwiGLU activations */
     void *y;               /* [P,H]   bf16 expert outputs */
     void *out;             /* [T,H]   bf16 layer output */
@@ -200,6 +200,18 @@ MOE_API moe_status moe_gather(const moe_shape *shape, const void *x, const int32
 MOE_API moe_status moe_grouped_swiglu(const moe_shape *shape, const void *x_perm, const void *w_gate, const void *w_up,
                               void *h, void *ws, void *stream);
 
+/* Step 4a with the row copy of step 3 folded in: the same h as
+ * moe_grouped_swiglu on x_perm, reading each permuted row r straight from
+ * x[src_token[r]] (TMA gather of four token rows per load), so x_perm is
+ * neither written nor read.  It saves the row copy and the P x H buffer;
+ * the gathers move fewer bytes per cycle than whole tiles, so with many rows
+ * per expert (more than about 32 on average) moe_gather + moe_grouped_swiglu
+ * is faster.  src_token as moe_permute / moe_route_dispatch
+ * leave it; a row outside [0, T) is read as token 0 and reported as
+ * MOE_DEV_BAD_ROW. */
+MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape *shape, const void *x, const int32_t *src_token,
+                                             const void *w_gate, const void *w_up, void *h, void *ws, void *stream);
+
 /* Step 4b, down projection ("TritonMoE" verdict page, desk editor letter):
  *   y[r,c] = bf16( h[r] . w_down[e][:,c] ), fp32 accumulation. */
 MOE_API moe_status moe_grouped_down(const moe_shape *shape, const void *h, const void *w_down, void *y, void *ws,
@@ -213,7 +225,10 @@ MOE_API moe_status moe_combine(const moe_shape *shape, const void *y, const int3
 
 /* The five steps in order on one stream (no host sync; graph-capturable):
  * moe_route_dispatch, moe_gather, moe_grouped_swiglu, moe_grouped_down,
- * moe_combine. */
+ * moe_combine.  With args->x_perm == NULL the row copy is folded into the
+ * SwiGLU GEMM (moe_grouped_swiglu_gather) and x_perm is not produced: the
+ * faster choice for decode-sized batches (about 32 or fewer routed rows per
+ * expert), the slower one for large batches. */
 MOE_API moe_status moe_forward(const moe_shape *shape, const moe_forward_args *args, void *ws, void *stream);
 
 /* Synchronises `stream`, copies the sticky device status word of `ws` to

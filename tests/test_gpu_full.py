@@ -1,6 +1,6 @@
 """Parity at the full sizes of the five workload configs (config 5 at each skew
 alpha), through moe_forward as the benchmark runs it.  Everything integer
-(routing indices, counts, offsets, permutation, gathered rows, schedule) is
+(routing indices, counts, offsets, permutation, schedule) is
 checked in full; the GEMM outputs on sampled rows and the layer output on
 sampled tokens, which the oracle computes one by one."""
 import numpy as np
@@ -36,7 +36,8 @@ def test_full_config(orc, cid, alpha):
     shape = shape_of(cfg)
     dl = DeviceLayer(L)
     b = dl.bufs(shape)
-    moe.moe_forward(shape, b, b["ws"])
+    # as the benchmark runs it: no x_perm, the SwiGLU GEMM gathers its rows
+    moe.moe_forward(shape, b, b["ws"], args=moe.forward_args({**b, "x_perm": None}))
     torch.cuda.synchronize()
     r = host(b, shape)
     assert r["status"] == 0, hex(r["status"])
@@ -57,7 +58,6 @@ def test_full_config(orc, cid, alpha):
     assert np.array_equal(r["dest_row"], d["dest_row"])
     filled = d["src_token"] >= 0
     assert np.array_equal(r["src_token"][filled], d["src_token"][filled])
-    assert np.array_equal(r["x_perm"][filled], L.x[d["src_token"][filled]])
     check_tile_schedule(r, shape, d["counts"], d["offsets"], d["spill_off"])
 
     d["dest_row_expert"] = np.full(d["P"], -1)

@@ -7,8 +7,8 @@ import torch
 
 import grouped_expert_gemm_router_b200 as moe
 import synth
-from gpu_util import (LOGIT_TOL, WEIGHT_TOL, DeviceLayer, assert_close_bf16, check_tile_schedule, host, run_steps,
-                      shape_of)
+from gpu_util import (LOGIT_TOL, WEIGHT_TOL, DeviceLayer, assert_close_bf16, bf16_host, check_tile_schedule, host,
+                      run_steps, shape_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -100,15 +100,19 @@ SAME_KEYS = ("logits", "topk_idx", "topk_w", "expert_counts", "expert_offsets", 
              "h", "y", "out", "status")
 
 
+@pytest.mark.parametrize("with_x_perm", [True, False], ids=["x_perm", "gathered"])
 @pytest.mark.parametrize("name", list(FORWARD_CASES))
-def test_forward_entry_point_matches_steps(orc, name):
+def test_forward_entry_point_matches_steps(orc, name, with_x_perm):
+    """moe_forward against the five entry points called one by one; without
+    an x_perm buffer the SwiGLU GEMM gathers its rows from x itself."""
     cfg = FORWARD_CASES[name]
     L = synth.make_layer(cfg)
     shape = shape_of(cfg)
     dl = DeviceLayer(L)
     a = host(run_steps(dl, shape), shape)
     b = dl.bufs(shape)
-    moe.moe_forward(shape, b, b["ws"])
+    b["x_perm"].fill_(0)
+    moe.moe_forward(shape, b, b["ws"], args=moe.forward_args(b if with_x_perm else {**b, "x_perm": None}))
     torch.cuda.synchronize()
     f = host(b, shape)
     for key in SAME_KEYS:
@@ -117,7 +121,31 @@ def test_forward_entry_point_matches_steps(orc, name):
     filled = a["src_token"] >= 0
     assert np.array_equal(a["src_token"], f["src_token"]) if cfg.C > 0 else np.array_equal(a["src_token"][filled],
                                                                                            f["src_token"][filled])
-    assert np.array_equal(a["x_perm"][filled], f["x_perm"][filled])
+    if with_x_perm:
+        assert np.array_equal(a["x_perm"][filled], f["x_perm"][filled])
+    else:
+        assert not f["x_perm"].any(), "x_perm must stay untouched"
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_swiglu_gather_equals_permuted_copy(orc, name):
+    """The SwiGLU GEMM reading rows x[src_token[r]] with TMA gathers gives
+    the h of the GEMM on the permuted copy x_perm, bit for bit, on every
+    filled row (several tiles, ragged tails, capacity layout, E = 256)."""
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    b = run_steps(dl, shape)
+    h2 = torch.zeros_like(b["h"])
+    moe.moe_grouped_swiglu_gather(shape, b["x"], b["src_token"], b["w_gate"], b["w_up"], h2, b["ws"])
+    torch.cuda.synchronize()
+    r = host(b, shape)
+    assert r["status"] == 0
+    filled = r["src_token"] >= 0
+    g = bf16_host(h2)
+    assert np.array_equal(g[filled], r["h"][filled])
+    assert not g[~filled].any(), "rows no tile covers stay unwritten"
 
 
 def test_logits_in_ties(orc):
