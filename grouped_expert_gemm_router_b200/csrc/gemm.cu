@@ -110,12 +110,15 @@ struct GemmArgs {
 };
 
 struct Unit {
-    int e, fb, nacc, N, n0p, p0s, p0l, p1s, p1l;
+    int e, fb, fx, nacc, N, n0p, p0s, p0l, p1s, p1l;  // fx: first output feature of accumulator 0
     bool valid;  // false only for a corrupt schedule: every role then skips the unit
 };
 
 template <int MODE>
-__device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, Unit &U) {
+// num_fb / fbw: feature blocks per row tile and, in mode 1, their width (256
+// features in two accumulators, or 128 in one when that still fits one wave).
+__device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, int num_fb, int fbw,
+                                            Unit &U) {
     if (MODE == 2) {  // unit u = tokens [u * route_rows, ...), all experts
         U.e = 0;
         U.fb = 0;
@@ -132,7 +135,7 @@ __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArg
     int lo = 0, hi = a.E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (gts[mid] * a.num_fb <= u)
+        if (gts[mid] * num_fb <= u)
             lo = mid;
         else
             hi = mid - 1;
@@ -141,7 +144,7 @@ __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArg
     U.valid = false;
     U.N = 0;
     if (nt <= 0 || g0 < 0) return;
-    const int local = u - g0 * a.num_fb;
+    const int local = u - g0 * num_fb;
     U.fb = local / nt;
     const int tile = g0 + local % nt;
     if (tile >= a.max_tiles) return;
@@ -153,9 +156,10 @@ __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArg
     U.p1s = d.w;
     U.n0p = (U.p0l + 15) & ~15;
     U.N = U.n0p + ((U.p1l + 15) & ~15);
-    U.nacc = (MODE == 0) ? 2 : ((U.fb * 256 + 128 < a.n_out) ? 2 : 1);
+    U.fx = MODE == 0 ? U.fb * 128 : U.fb * fbw;
+    U.nacc = (MODE == 0) ? 2 : ((fbw == 256 && U.fx + 128 < a.n_out) ? 2 : 1);
     U.valid = (unsigned)U.e < (unsigned)a.E && U.N > 0 && U.N <= trows && U.p0s >= 0 && U.p1s >= 0 &&
-              U.p0s + U.p0l <= a.P && U.p1s + U.p1l <= a.P && U.fb < a.num_fb;
+              U.p0s + U.p0l <= a.P && U.p1s + U.p1l <= a.P && U.fb < num_fb;
 }
 
 __device__ __forceinline__ int unit_row(const Unit &U, int c) {
@@ -221,12 +225,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int total, trows;
+    int num_fb = a.num_fb, fbw = 256;
     if (MODE == 2) {
         total = (a.T + a.route_rows - 1) / a.route_rows;
         trows = a.route_rows;
     } else {
         const int ntiles = *a.num_tiles;
-        total = (ntiles < a.max_tiles ? ntiles : a.max_tiles) * a.num_fb;
+        const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
+        // Down projection with few row tiles: 128-feature units, twice as many,
+        // when they still fit one wave (otherwise 256-feature units, which read
+        // each token tile once for two accumulators).
+        if (MODE == 1 && nt * a.num_fb * 2 <= (int)gridDim.x) {
+            num_fb = a.n_out / 128;
+            fbw = 128;
+        }
+        total = nt * num_fb;
         trows = *a.tile_rows;  // the schedule's row cap
     }
     if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
@@ -295,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kMaxBStages; ++s) issued_ph[s] = -1;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             Unit U;
-            decode_unit<MODE>(u, s_gts, a, trows, U);
+            decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
             if (!U.valid) continue;
             // The unit's tokens, one per tile row; padding rows repeat the
             // first row (their results are never stored).  Loads already
@@ -362,13 +375,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < kMaxAStages; ++s) issued_ph[s] = -1;
             for (int u = blockIdx.x; u < total; u += gridDim.x) {
                 Unit U;
-                decode_unit<MODE>(u, s_gts, a, trows, U);
+                decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
                 if (!U.valid) {
                     if (is_a) atomicOr(a.status, MOE_DEV_BAD_ROW);
                     continue;
                 }
-                const int fx0 = MODE == 0 ? U.fb * 128 : U.fb * 256;
-                const int fx1 = MODE == 0 ? U.fb * 128 : U.fb * 256 + 128;
+                const int fx0 = U.fx;
+                const int fx1 = MODE == 0 ? U.fx : U.fx + 128;
                 const int nb0 = (U.p0l + 15) >> 4, nb1 = (U.p1l + 15) >> 4;
                 const uint32_t bytes = is_a ? (MODE == 2 ? 3u : 1u) * (uint32_t)U.nacc * kATile
                                             : (uint32_t)(nb0 + nb1) * kBBox;
@@ -433,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 Unit U;
-                decode_unit<MODE>(u, s_gts, a, trows, U);
+                decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
                 if (!U.valid) continue;
                 const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
                 uint32_t h;
@@ -514,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         TmemPlan plan;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
             Unit U;
-            decode_unit<MODE>(u, s_gts, a, trows, U);
+            decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
             if (!U.valid) continue;
             uint32_t h;
             bool big;
@@ -538,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (big) mbar_arrive(&tempty[1]);
                 }
             };
-            const int f0 = MODE == 0 ? U.fb * 128 + L : U.fb * 256 + L;
+            const int f0 = U.fx + L;
             unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
             if (MODE == 2) {
                 // fp32 logits + bias: lane L of expert block c is expert c*128 + L;
