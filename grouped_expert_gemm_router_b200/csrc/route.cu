@@ -5,16 +5,18 @@
 //
 // The logits are a small fp32 GEMM (T x H times H x E, E <= 256) that is
 // latency-bound at decode sizes and FMA-bound at prefill sizes:
-// - A CTA of 8 warps owns TB = 8*TW tokens (TW tokens per warp) and all E
-//   experts for a slice of the hidden dimension.  When there are few token
-//   blocks, the hidden dimension is split over a thread-block cluster of CL
-//   CTAs (CL <= 8) so that every SM gets work; the CL partial logits are summed
-//   by the cluster's rank-0 CTA through distributed shared memory, in rank
-//   order (deterministic).
+// - A CTA of 8 warps owns TB tokens (16, 8 or 4: fewer for more experts) and
+//   all E experts for a slice of the hidden dimension.  When there are few
+//   token blocks, the hidden dimension is split over a thread-block cluster of
+//   CL CTAs (CL <= 8) so that about 3/4 of the SMs get a CTA; the CL partial
+//   logits are summed by the cluster's rank-0 CTA through distributed shared
+//   memory, in rank order (deterministic).
 // - x and W_r stream through shared memory in chunks of HC hidden units with
-//   a 2-4 stage cp.async pipeline.  ES lanes of a warp split the experts (EJ
-//   each, a compile-time count) and HS = 32/ES lanes split the hidden units;
-//   the HS partial sums are folded with shuffles.
+//   a 2-4 stage cp.async pipeline.  The 8 warps split each chunk's hidden
+//   units; inside a warp ES lanes split the experts (EJ consecutive experts
+//   each) and HS = 32/ES lanes the hidden pairs.  Each thread holds a TB x EJ
+//   tile of sums, so every weight value it reads feeds TB multiply-adds; the
+//   warps' partial sums are added in warp order.
 // - Top-k: one warp per token, each lane holding ceil(E/32) candidates as
 //   64-bit keys (orderable logit << 32 | ~expert); k rounds of a warp max.
 // - Fused dispatch (small batches, called from moe_forward): every CTA that
@@ -92,8 +94,17 @@ __device__ void fused_dispatch_tail(const RouteArgs &a, uint8_t *smem) {
     __syncthreads();
     if (tid == 0 && sm.flag) atomicOr(a.status, MOE_DEV_BAD_EXPERT);
     build_schedule_block(sm, E, a.C, a.capped != 0, a.out.counts, a.out.offsets, a.ws);
+    if (a.capped) {
+        // Rows no pair fills: the capacity slots past each expert's count and
+        // the overflow rows past the total overflow.
+        for (int i = tid; i < E * a.C; i += kScanThreads)
+            if (i % a.C >= min(sm.hist[i / a.C], a.C)) a.out.src_token[i] = -1;
+        for (int i = E * a.C + sm.spoff[E] + tid; i < a.P; i += kScanThreads) a.out.src_token[i] = -1;
+    }
     auto expert_of = [pairs](int i) { return pairs[i]; };
     rank_pairs_block(sm, expert_of, 0, R, E, a.k, a.C, a.capped != 0, a.P, a.out.dest_row, a.out.src_token, a.ws);
+    // Every router CTA has taken its ticket: the count starts at zero again.
+    if (tid == 0) *a.ws.route_done = 0;
 }
 
 // Monotone map of a float onto uint32 (larger float -> larger key); -0 is
@@ -131,9 +142,8 @@ __device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t ran
     return v;
 }
 
-template <int TW, int EJ>
+template <int TB, int EJ>
 __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
-    constexpr int TB = 8 * TW;
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_nan;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -167,14 +177,20 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             const float *src = a.w_router + (size_t)h0 * E;  // rows h0 .. h0+HC: contiguous
             for (int i = tid; i < HC * E / 4; i += 256) cp_async16(sw + 4 * i, src + 4 * i);
         };
+        // All 8 warps share the CTA's TB tokens and split each chunk's hidden
+        // units (warp w takes pairs [w * PPW, (w + 1) * PPW)); inside a warp ES
+        // lanes split the experts (EJ consecutive experts each) and HS = 32/ES
+        // lanes the hidden pairs.  Each thread keeps a TB x EJ tile of sums, so
+        // every weight value read from shared memory feeds TB multiply-adds.
         const int ES = a.es, HS = 32 / ES;
         const int es = lane % ES, hs = lane / ES;
+        const int PPW = HC / 2 / 8;
         int ecol[EJ];
 #pragma unroll
-        for (int j = 0; j < EJ; ++j) ecol[j] = min(es + ES * j, E - 1);  // reads past E are clamped, unused
-        float acc[TW][EJ];
+        for (int j = 0; j < EJ; ++j) ecol[j] = min(es * EJ + j, E - 1);  // reads past E are clamped, unused
+        float acc[TB][EJ];
 #pragma unroll
-        for (int i = 0; i < TW; ++i)
+        for (int i = 0; i < TB; ++i)
 #pragma unroll
             for (int j = 0; j < EJ; ++j) acc[i][j] = 0.0f;
 
@@ -188,42 +204,55 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             cp_async_wait_pending(S - 1);  // this thread's copies of chunk c have landed
             __syncthreads();               // ... and everyone else's
             const uint8_t *sx = smem + (size_t)(c % S) * stage_bytes;
-            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx) + (size_t)warp * TW * HC;
+            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx);
             const float *wsm = reinterpret_cast<const float *>(sx + xbytes);
-            // Pairs of hidden units 2p, 2p+1; this lane takes p = hs, hs + HS, ...
-#pragma unroll 2
-            for (int p = hs; p < HC / 2; p += HS) {
-                float2 xv[TW];
-#pragma unroll
-                for (int i = 0; i < TW; ++i)
-                    xv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)i * HC + 2 * p));
+            // Pairs of hidden units 2p, 2p+1 of this warp's range; this lane
+            // takes p = p0 + hs, p0 + hs + HS, ...
+            const int p0 = warp * PPW;
+            for (int p = p0 + hs; p < p0 + PPW; p += HS) {
                 const float *w0 = wsm + (size_t)(2 * p) * E;
+                float wa[EJ], wb[EJ];
 #pragma unroll
                 for (int j = 0; j < EJ; ++j) {
-                    const float wa = w0[ecol[j]], wb = w0[E + ecol[j]];
+                    wa[j] = w0[ecol[j]];
+                    wb[j] = w0[E + ecol[j]];
+                }
 #pragma unroll
-                    for (int i = 0; i < TW; ++i) {
-                        acc[i][j] = fmaf(xv[i].x, wa, acc[i][j]);
-                        acc[i][j] = fmaf(xv[i].y, wb, acc[i][j]);
+                for (int i = 0; i < TB; ++i) {
+                    const float2 xv =
+                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)i * HC + 2 * p));
+#pragma unroll
+                    for (int j = 0; j < EJ; ++j) {
+                        acc[i][j] = fmaf(xv.x, wa[j], acc[i][j]);
+                        acc[i][j] = fmaf(xv.y, wb[j], acc[i][j]);
                     }
                 }
             }
             __syncthreads();  // stage c % S may be refilled from here on
         }
-        // Fold the hidden-unit split.
+        // Fold the hidden-pair split inside the warp, then the warps' partial
+        // sums in warp order (deterministic) through shared memory, which the
+        // pipeline no longer needs.
         for (int off = ES; off < 32; off <<= 1)
 #pragma unroll
-            for (int i = 0; i < TW; ++i)
+            for (int i = 0; i < TB; ++i)
 #pragma unroll
                 for (int j = 0; j < EJ; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
+        float *wpart = reinterpret_cast<float *>(smem);  // [8][TB][E]
         if (hs == 0) {
 #pragma unroll
-            for (int i = 0; i < TW; ++i)
+            for (int i = 0; i < TB; ++i)
 #pragma unroll
                 for (int j = 0; j < EJ; ++j) {
-                    const int e = es + ES * j;
-                    if (e < E) part[(warp * TW + i) * E + e] = acc[i][j];
+                    const int e = es * EJ + j;
+                    if (e < E) wpart[(warp * TB + i) * E + e] = acc[i][j];
                 }
+        }
+        __syncthreads();
+        for (int i = tid; i < TB * E; i += 256) {
+            float v = wpart[i];
+            for (int w = 1; w < 8; ++w) v += wpart[w * TB * E + i];
+            part[i] = v;
         }
         if (CL > 1)
             cluster_sync_all();
@@ -253,8 +282,8 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     // Top-k, one warp per token.  Selected slot j lives in register m = j / 32
     // of lane j % 32 (k <= E <= 256: at most 8 per lane), so the softmax needs
     // no round trip through global memory.
-    for (int i = 0; i < TW; ++i) {
-        const int tok = warp * TW + i, t = t0 + tok;
+    for (int tok = warp; tok < TB; tok += 8) {
+        const int t = t0 + tok;
         if (t >= a.T) break;
         unsigned long long key[8];
         bool nan = false;
@@ -328,11 +357,11 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
 }
 
-template <int TW, int EJ>
+template <int TB, int EJ>
 cudaError_t launch_one(const RouteArgs &a, int smem_bytes, int tiles, cudaStream_t stream) {
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_route<TW, EJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(k_route<TB, EJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
@@ -348,16 +377,18 @@ cudaError_t launch_one(const RouteArgs &a, int smem_bytes, int tiles, cudaStream
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.cl > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_route<TW, EJ>, a);
+    return cudaLaunchKernelEx(&cfg, k_route<TB, EJ>, a);
 }
 
-template <int TW>
-cudaError_t launch_tw(const RouteArgs &a, int ej, int smem, int tiles, cudaStream_t st) {
+// Tokens per CTA by experts per lane: a thread keeps at most 32 sums.
+constexpr int route_tile_tokens(int ej) { return ej <= 2 ? 16 : (ej == 4 ? 8 : 4); }
+
+cudaError_t launch_ej(const RouteArgs &a, int ej, int tb, int smem, int tiles, cudaStream_t st) {
     switch (ej) {
-        case 1: return launch_one<TW, 1>(a, smem, tiles, st);
-        case 2: return launch_one<TW, 2>(a, smem, tiles, st);
-        case 4: return launch_one<TW, 4>(a, smem, tiles, st);
-        default: return launch_one<TW, 8>(a, smem, tiles, st);
+        case 1: return tb == 8 ? launch_one<8, 1>(a, smem, tiles, st) : launch_one<16, 1>(a, smem, tiles, st);
+        case 2: return tb == 8 ? launch_one<8, 2>(a, smem, tiles, st) : launch_one<16, 2>(a, smem, tiles, st);
+        case 4: return launch_one<route_tile_tokens(4), 4>(a, smem, tiles, st);
+        default: return launch_one<route_tile_tokens(8), 8>(a, smem, tiles, st);
     }
 }
 
@@ -374,15 +405,10 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     moe_shape s = s0;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
-    if (fused) {
-        if ((int64_t)s.T * s.k > kFusedDispatchMaxPairs) return cudaErrorInvalidValue;
-        // The same clearing the dispatch kernels start with.
-        cudaError_t err = cudaMemsetAsync((char *)ws + L.reset_begin, 0, L.reset_end - L.reset_begin, stream);
-        if (err != cudaSuccess) return err;
-        if (capped && (err = cudaMemsetAsync(fused->src_token, 0xFF, sizeof(int32_t) * (size_t)P, stream)) !=
-                          cudaSuccess)
-            return err;
-    }
+    // The fused path needs no clearing launch: the CTA that builds the
+    // dispatch resets the completion count it used and writes the empty
+    // capacity slots' src_token itself.
+    if (fused && (int64_t)s.T * s.k > kFusedDispatchMaxPairs) return cudaErrorInvalidValue;
     if (!(s.flags & MOE_FLAG_LOGITS_IN) && use_tc_router(s.T)) {
         // Logits on the tensor cores, then the top-k below reads them.
         if (!logits) logits = (float *)((char *)ws + L.router_logits);
@@ -409,9 +435,15 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     a.P = (int)P;
     a.out = fused ? *fused : FusedDispatch{nullptr, nullptr, nullptr, nullptr};
     a.ws = ws_ptrs(ws, L);
-    // Four tokens per warp when that still gives every SM a block.
-    const int TW = ((s.T + 31) / 32 >= num_sms) ? 4 : 1;
-    const int TB = 8 * TW;
+    int es = 1;
+    while (es < s.E && es < 32) es <<= 1;
+    a.es = es;
+    int ej = (s.E + es - 1) / es;
+    ej = ej <= 1 ? 1 : ej <= 2 ? 2 : ej <= 4 ? 4 : 8;
+    int TB = route_tile_tokens(ej);
+    // Small batches: halve the tile while 8-CTA clusters of full tiles would
+    // leave more than a quarter of the SMs idle.
+    if (TB == 16 && !a.logits_in && ((s.T + 15) / 16) * 8 < (3 * num_sms) / 4) TB = 8;
     const int tiles = (s.T + TB - 1) / TB;
     a.tiles = tiles;
     // Split the hidden dimension over a cluster until there are about 3/4 as
@@ -421,11 +453,6 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
         while (cl < 8 && tiles * cl < (3 * num_sms) / 4 && s.H % (64 * 2 * cl) == 0) cl *= 2;
     a.cl = cl;
     a.slice = s.H / cl;
-    int es = 1;
-    while (es < s.E && es < 32) es <<= 1;
-    a.es = es;
-    int ej = (s.E + es - 1) / es;
-    ej = ej <= 1 ? 1 : ej <= 2 ? 2 : ej <= 4 ? 4 : 8;
     // Chunk: the largest power of two dividing the slice with the stage <= 40 KiB, >= 64.
     int hc = 1024;
     while (hc > 64 && (a.slice % hc != 0 || hc * (4 * s.E + 2 * TB) > 40 * 1024)) hc >>= 1;
@@ -443,15 +470,19 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
         a.part_off = 0;
         smem = lg_bytes;
     } else {
-        const int pipe = stages * stage_bytes;
-        a.part_off = (int)align_up((size_t)(pipe > lg_bytes ? pipe : lg_bytes), 16);
+        // the pipeline stages, later the per-warp partial sums [8][TB][E] and
+        // then rank 0's logits tile share the front of shared memory
+        int front = stages * stage_bytes;
+        if (front < lg_bytes) front = lg_bytes;
+        if (front < 8 * TB * s.E * 4) front = 8 * TB * s.E * 4;
+        a.part_off = (int)align_up((size_t)front, 16);
         smem = a.part_off + TB * s.E * 4;
     }
     if (fused) {
         const int need = (int)align_up(sizeof(DispatchSmem) + sizeof(int) * (size_t)s.T * s.k, 16);
         if (smem < need) smem = need;
     }
-    return TW == 4 ? launch_tw<4>(a, ej, smem, tiles, stream) : launch_tw<1>(a, ej, smem, tiles, stream);
+    return launch_ej(a, ej, TB, smem, tiles, stream);
 }
 
 }  // namespace moe
