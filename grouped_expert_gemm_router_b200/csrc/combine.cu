@@ -6,8 +6,9 @@
 // bit-identical to a plain sequential fp32 loop.
 //
 // HBM-bound gather: each thread owns 8 consecutive features (one 16-byte
-// vector) of one token, reads the k expert rows with 16-byte loads and writes
-// one 16-byte vector.  Grid: tokens x ceil(H/8 / 256) blocks of 256 threads.
+// vector) of one token, reads the k expert rows with 16-byte loads (for
+// k <= 8 all of them issued before the first is used) and writes one 16-byte
+// vector.  Grid: tokens x ceil(H/8 / 256) blocks of 256 threads.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -26,6 +27,9 @@ __device__ __forceinline__ void unpack8(const uint4 &q, float (&v)[8]) {
     }
 }
 
+// KMAX > 0: k <= KMAX, all k row loads issued before any is used; KMAX = 0:
+// any k, one row at a time.
+template <int KMAX>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const int *__restrict__ dest_row,
                                                  const float *__restrict__ w, uint4 *__restrict__ out, int k, int H8,
                                                  int P) {
@@ -35,14 +39,36 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        const int r = __ldg(dest_row + (size_t)t * k + j);
-        if ((unsigned)r >= (unsigned)P) continue;  // only after an earlier device error
-        const float wj = __ldg(w + (size_t)t * k + j);
-        float yv[8];
-        unpack8(__ldg(y + (size_t)r * H8 + v), yv);
+    if (KMAX > 0) {
+        int r[KMAX > 0 ? KMAX : 1];
+        float wj[KMAX > 0 ? KMAX : 1];
+        uint4 q[KMAX > 0 ? KMAX : 1];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, yv[i]));
+        for (int j = 0; j < KMAX; ++j) {
+            r[j] = j < k ? __ldg(dest_row + (size_t)t * k + j) : -1;
+            wj[j] = j < k ? __ldg(w + (size_t)t * k + j) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)  // an index outside [0, P) only after an earlier device error
+            q[j] = (unsigned)r[j] < (unsigned)P ? __ldg(y + (size_t)r[j] * H8 + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if ((unsigned)r[j] >= (unsigned)P) continue;
+            float yv[8];
+            unpack8(q[j], yv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj[j], yv[i]));
+        }
+    } else {
+        for (int j = 0; j < k; ++j) {
+            const int r = __ldg(dest_row + (size_t)t * k + j);
+            if ((unsigned)r >= (unsigned)P) continue;  // only after an earlier device error
+            const float wj = __ldg(w + (size_t)t * k + j);
+            float yv[8];
+            unpack8(__ldg(y + (size_t)r * H8 + v), yv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, yv[i]));
+        }
     }
     uint4 o;
     __nv_bfloat162 *ob = reinterpret_cast<__nv_bfloat162 *>(&o);
@@ -58,7 +84,12 @@ cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *des
     const int H8 = s.H / 8;
     const dim3 grid((unsigned)s.T, (unsigned)((H8 + 255) / 256));
     const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, (s.flags & MOE_FLAG_CAPACITY) != 0);
-    k_combine<<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+    if (s.k <= 2)
+        k_combine<2><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+    else if (s.k <= 8)
+        k_combine<8><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+    else
+        k_combine<0><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
     return cudaGetLastError();
 }
 

@@ -151,13 +151,13 @@ __global__ void __launch_bounds__(256) k_gather(const uint4 *__restrict__ x, con
         if ((unsigned)t < (unsigned)T) {
             const uint4 *src = x + (size_t)t * H8;
             int v = lane;
-            for (; v + 96 < H8; v += 128) {
-                const uint4 q0 = __ldg(src + v), q1 = __ldg(src + v + 32), q2 = __ldg(src + v + 64),
-                            q3 = __ldg(src + v + 96);
-                dst[v] = q0;
-                dst[v + 32] = q1;
-                dst[v + 64] = q2;
-                dst[v + 96] = q3;
+            // eight 16-byte loads per lane in flight before the stores
+            for (; v + 224 < H8; v += 256) {
+                uint4 q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[i] = __ldg(src + v + 32 * i);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[v + 32 * i] = q[i];
             }
             for (; v < H8; v += 32) dst[v] = __ldg(src + v);
         } else {
