@@ -22,6 +22,7 @@ MOE_DEV_NAN_LOGIT = 0x8
 MOE_DEV_BAD_ROW = 0x10
 MOE_FLAG_CAPACITY = 0x1
 MOE_FLAG_LOGITS_IN = 0x2
+MOE_FLAG_GEMM_PAIRS = 0x4
 MOE_FLAG_TEST_STALL_SCAN = 0x40000000
 
 # Every symbol include/moe.h declares (the CPU tests check the library exports each).

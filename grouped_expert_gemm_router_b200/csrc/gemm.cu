@@ -115,8 +115,9 @@ struct Unit {
 };
 
 template <int MODE>
-// num_fb / fbw: feature blocks per row tile and, in mode 1, their width (256
-// features in two accumulators, or 128 in one when that still fits one wave).
+// num_fb / fbw: feature blocks per row tile and their width (mode 0: 128
+// features per CTA, 256 per CTA pair; mode 1: 256 features in two
+// accumulators, or 128 in one when that still fits one wave).
 __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, int num_fb, int fbw,
                                             Unit &U) {
     if (MODE == 2) {  // unit u = tokens [u * route_rows, ...), all experts
@@ -156,7 +157,7 @@ __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArg
     U.p1s = d.w;
     U.n0p = (U.p0l + 15) & ~15;
     U.N = U.n0p + ((U.p1l + 15) & ~15);
-    U.fx = MODE == 0 ? U.fb * 128 : U.fb * fbw;
+    U.fx = U.fb * fbw;
     U.nacc = (MODE == 0) ? 2 : ((fbw == 256 && U.fx + 128 < a.n_out) ? 2 : 1);
     U.valid = (unsigned)U.e < (unsigned)a.E && U.N > 0 && U.N <= trows && U.p0s >= 0 && U.p1s >= 0 &&
               U.p0s + U.p0l <= a.P && U.p1s + U.p1l <= a.P && U.fb < num_fb;
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int total, trows;
-    int num_fb = a.num_fb, fbw = 256;
+    int num_fb = a.num_fb, fbw = MODE == 0 ? 128 : 256;
     if (MODE == 2) {
         total = (a.T + a.route_rows - 1) / a.route_rows;
         trows = a.route_rows;
@@ -669,6 +670,334 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Pairs of CTAs sharing one MMA (tcgen05 cta_group::2), modes 0 and 1.
+// A cluster of two CTAs takes units (expert group, 256-feature block, row
+// tile): CTA r of the pair holds the weights of features [256 fb + 128 r, +128)
+// (the MMA's M = 256 is split by CTA) and rows [r N/2, (r+1) N/2) of the token
+// tile (N split by CTA), so each CTA streams only half of every token tile.
+// Both CTAs' copies complete on the leader's (rank 0) barriers, which count
+// both halves' bytes; the leader alone issues the MMAs and multicasts their
+// commits to both CTAs' stage and accumulator barriers; each CTA drains its
+// own tensor memory (its 128 features for all N rows) and hands it back by
+// arriving on the leader's barrier.  Mode 0 keeps gate and up for the CTA's
+// 128 features (two accumulators); mode 1 one accumulator of up to 256
+// columns, so its units always alternate between the tensor-memory halves.
+// Selected by MOE_FLAG_GEMM_PAIRS.  Measured on B200 it is not faster than the
+// single-CTA kernel for the shapes of this library's benchmarks (the
+// weight-streaming shapes stream no faster per SM with the deeper weight ring
+// it allows, and the down projection of a 128-unit layer loses half of its
+// per-CTA rate), so it is off by default.
+constexpr int kPairMaxAStages = 12;
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
+    k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+    static_assert(MODE == 0 || MODE == 1, "pairs run the expert GEMMs");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    uint8_t *ctrl = smem + kRingBytes;
+    uint64_t *fullA = reinterpret_cast<uint64_t *>(ctrl);
+    uint64_t *emptyA = fullA + kPairMaxAStages;
+    uint64_t *fullB = emptyA + kPairMaxAStages;
+    uint64_t *emptyB = fullB + kMaxBStages;
+    uint64_t *tfull = emptyB + kMaxBStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *mma_done = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
+    const int ntiles = *a.num_tiles;
+    const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
+    const int num_fb = (a.n_out + 255) / 256;
+    const int total = nt * num_fb;
+    if (pair >= total) return;  // uniform over the pair: neither CTA has work
+    int trows = *a.tile_rows;
+    trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
+    const uint32_t a_tiles = MODE == 0 ? 2u : 1u;
+    const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)(trows / 2) * kBRowBytes;
+    int nb = kMaxBStages;
+    int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    if (fit < 4) {
+        nb = 3;
+        fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    }
+    const int na = fit > kPairMaxAStages ? kPairMaxAStages : fit;
+    uint8_t *ringB = smem + (uint32_t)na * a_bytes;
+
+    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairMaxAStages; ++s) {
+            mbar_init(&fullA[s], 1);
+            mbar_init(&emptyA[s], 1);
+        }
+        for (int s = 0; s < kMaxBStages; ++s) {
+            mbar_init(&fullB[s], 1);
+            mbar_init(&emptyB[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * kEpiWarps);  // both CTAs' epilogue warps (the leader's count)
+        }
+        mbar_init(mma_done, 1);
+        *s_abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmA1);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_arrive_wait();  // both CTAs' barriers are initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nk = a.K / kBK;
+
+    if (warp == 0 || warp == 2) {
+        // ------------- TMA producers (both CTAs): warp 0 weights, warp 2 token rows ----
+        if (lane == 0) {
+            const bool is_a = warp == 0;
+            const int nst = is_a ? na : nb;
+            uint64_t *full = is_a ? fullA : fullB;
+            uint64_t *empty = is_a ? emptyA : emptyB;
+            const uint32_t full_leader = mapa_shared(full, 0);  // the leader's barrier array
+            int stage = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int u = pair; u < total && ok; u += npairs) {
+                Unit U;
+                decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
+                if (!U.valid) {
+                    if (is_a && leader) atomicOr(a.status, MOE_DEV_BAD_ROW);
+                    continue;
+                }
+                const int fx = U.fx + 128 * (int)rank;  // this CTA's first feature
+                const int half_rows = U.N / 2;          // rows of the token tile this CTA holds
+                const uint32_t my_bytes = is_a ? a_tiles * kATile : (uint32_t)half_rows * kBRowBytes;
+                const int krow = U.e * a.K;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, a.timeout_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    // the leader expects both CTAs' bytes of this stage
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * my_bytes);
+                    const uint32_t bar = full_leader + 8u * (uint32_t)stage;
+                    const int ky = krow + kb * kBK, kx = kb * kBK;
+                    if (is_a) {
+                        uint8_t *sa0 = smem + stage * a_bytes;
+                        tma_load_2d_pair(sa0, &tmA0, bar, fx, ky);
+                        tma_load_2d_pair(sa0 + kABox, &tmA0, bar, fx + 64, ky);
+                        if (MODE == 0) {
+                            tma_load_2d_pair(sa0 + kATile, &tmA1, bar, fx, ky);
+                            tma_load_2d_pair(sa0 + kATile + kABox, &tmA1, bar, fx + 64, ky);
+                        }
+                    } else {
+                        // 8-row boxes of tile rows [rank * N/2, (rank + 1) * N/2); a
+                        // box never straddles the two row pieces (16-row aligned)
+                        uint8_t *sb = ringB + stage * b_bytes;
+                        const int c_begin = (int)rank * half_rows;
+                        for (int c = c_begin; c < c_begin + half_rows; c += 8) {
+                            const int row = c < U.n0p ? U.p0s + c : U.p1s + (c - U.n0p);
+                            tma_load_2d_pair(sb + (c - c_begin) * kBRowBytes, &tmB, bar, kx, row);
+                        }
+                    }
+                    if (++stage == nst) {
+                        stage = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok && !*s_abort) raise_abort(s_abort, a.status);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer (the leader only) ----
+        if (lane == 0 && leader) {
+            int sa = 0, sb = 0;
+            uint32_t pha = 0, phb = 0;
+            TmemPlan plan;
+            const uint32_t baseA = smem_u32(smem), baseB = smem_u32(ringB);
+            bool ok = true;
+            for (int u = pair; u < total && ok; u += npairs) {
+                Unit U;
+                decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
+                if (!U.valid) continue;
+                const uint32_t idesc = idesc_bf16_f32(256, U.N, 1, 0);
+                uint32_t h;
+                bool big;
+                plan.place(MODE == 0 ? U.N : 0, h, big);  // mode 1: one accumulator fits a half
+                const uint32_t d0 = tmem + h * 256u, d1 = big ? tmem + 256u : d0 + 128u;
+                ok = mbar_wait_bounded(&tempty[h], (plan.uses[h] & 1u) ^ 1u, a.timeout_ns, s_abort);
+                if (ok && big) ok = mbar_wait_bounded(&tempty[1], (plan.uses[1] & 1u) ^ 1u, a.timeout_ns, s_abort);
+                if (!ok) break;
+                tc_fence_after();
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(&fullA[sa], pha, a.timeout_ns, s_abort) ||
+                        !mbar_wait_bounded(&fullB[sb], phb, a.timeout_ns, s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa0 = baseA + sa * a_bytes, sa1 = sa0 + kATile, sbt = baseB + sb * b_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
+                        const uint32_t accum = (kb | kk) ? 1u : 0u;
+                        tc_mma_bf16_pair(d0, sdesc_sw128(sa0 + kk * 2048, kABox, 1024), bdesc, idesc, accum);
+                        if (MODE == 0)
+                            tc_mma_bf16_pair(d1, sdesc_sw128(sa1 + kk * 2048, kABox, 1024), bdesc, idesc, accum);
+                    }
+                    tc_commit_pair(&emptyA[sa], 3);  // both CTAs' stages are free once read
+                    tc_commit_pair(&emptyB[sb], 3);
+                    if (++sa == na) {
+                        sa = 0;
+                        pha ^= 1u;
+                    }
+                    if (++sb == nb) {
+                        sb = 0;
+                        phb ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(&tfull[h], 3);
+                if (big) tc_commit_pair(&tfull[1], 3);
+                plan.advance(big, h);
+            }
+            if (!ok && !*s_abort) raise_abort(s_abort, a.status);
+            int never = 0;
+            tc_commit_pair(mma_done, 1);
+            mbar_wait_bounded(mma_done, 0, a.timeout_ns, &never);
+        }
+        __syncwarp();
+    } else {
+        // -------------------------------------------- epilogue (both CTAs) ----
+        const int q = warp & 3;
+        const int sub = (warp - kEpiWarp0) >> 2;
+        const int L = q * 32 + lane;
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+        const uint32_t tempty_leader = mapa_shared(tempty, 0);
+        TmemPlan plan;
+        for (int u = pair; u < total; u += npairs) {
+            Unit U;
+            decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
+            if (!U.valid) continue;
+            uint32_t h;
+            bool big;
+            plan.place(MODE == 0 ? U.N : 0, h, big);
+            bool got = mbar_wait_bounded(&tfull[h], plan.uses[h] & 1u, a.timeout_ns, s_abort);
+            if (got && big) got = mbar_wait_bounded(&tfull[1], plan.uses[1] & 1u, a.timeout_ns, s_abort);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0 && !*s_abort) raise_abort(s_abort, a.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tq + h * 256u, t1 = big ? tq + 256u : t0 + 128u;
+            auto release = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_cluster(tempty_leader + 8u * h);
+                    if (big) mbar_arrive_cluster(tempty_leader + 8u);
+                }
+            };
+            const int f0 = U.fx + 128 * (int)rank + L;
+            const bool inside = f0 < a.n_out;  // the last block may have no second half
+            unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
+            if (MODE == 1) {
+                // one accumulator of up to 256 columns: hold up to 4 chunks per warp
+                constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
+                uint32_t hold[kChunks][8];
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) {
+                        uint32_t r0[16];
+                        tmem_ld16(t0 + (uint32_t)c0, r0);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            const __nv_bfloat162 pk =
+                                __floats2bfloat162_rn(__uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
+                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&pk);
+                        }
+                    }
+                }
+                release();
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N && inside) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int row = unit_row(U, c0 + j);
+                            if (row >= 0)
+                                outp[(size_t)row * a.n_out + f0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
+                        }
+                    }
+                }
+            } else {
+                constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
+                uint32_t hold[kChunks][8];
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) {
+                        uint32_t r0[16], r1[16];
+                        tmem_ld16(t0 + (uint32_t)c0, r0);
+                        tmem_ld16(t1 + (uint32_t)c0, r1);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            const float g0 = __uint_as_float(r0[j]), v0 = __uint_as_float(r1[j]);
+                            const float g1 = __uint_as_float(r0[j + 1]), v1 = __uint_as_float(r1[j + 1]);
+                            const __nv_bfloat162 pk = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * v0,
+                                                                            __fdividef(g1, 1.0f + __expf(-g1)) * v1);
+                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&pk);
+                        }
+                    }
+                }
+                release();
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N && inside) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int row = unit_row(U, c0 + j);
+                            if (row >= 0)
+                                outp[(size_t)row * a.n_out + f0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
+                        }
+                    }
+                }
+            }
+            plan.advance(big, h);
+        }
+    }
+
+    // Neither CTA leaves (or frees tensor memory) while the other may still
+    // read its shared memory, write its tensor memory or signal its barriers.
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive_wait();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
 // Exact three-way bf16 split of the router weights: p0 = bf16(w),
 // p1 = bf16(w - p0), p2 = bf16(w - p0 - p1) (each difference is exact in
 // fp32), written as planes[3][H][Ep]; columns e >= E are zero.
@@ -767,6 +1096,9 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
                                 cudaStream_t stream, const int32_t *src_token) {
     const bool gather = mode == 0 && src_token != nullptr;
+    // Pairs of CTAs sharing one MMA for the expert GEMMs, on request (not for
+    // the row gather).
+    const bool pairs = (s.flags & MOE_FLAG_GEMM_PAIRS) && !gather && num_sms >= 2;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
     const int K = mode == 0 ? s.H : s.F;
@@ -774,8 +1106,9 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     CUtensorMap tA0, tA1, tB;
     if (!make_tmap(&tA0, w0, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
         !make_tmap(&tA1, w1, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
-        !(gather ? make_tmap(&tB, act, (uint64_t)s.T, (uint64_t)K, 64, 1)
-                 : make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16)))
+        !(gather  ? make_tmap(&tB, act, (uint64_t)s.T, (uint64_t)K, 64, 1)
+          : pairs ? make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 8)
+                  : make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16)))
         return cudaErrorInvalidValue;
     WsPtrs p = ws_ptrs(ws, L);
     GemmArgs a = {};
@@ -794,9 +1127,28 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.timeout_ns = timeout_ns;
     a.T = s.T;
     a.src_token = src_token;
-    static bool attr_done[3] = {false, false, false};
+    static bool attr_done[5] = {false, false, false, false, false};
     cudaError_t err;
-    if (gather) {
+    if (pairs) {
+        const int grid = num_sms & ~1;
+        if (mode == 0) {
+            if (!attr_done[3]) {
+                err = cudaFuncSetAttribute(k_grouped_gemm_pair<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
+                if (err != cudaSuccess) return err;
+                attr_done[3] = true;
+            }
+            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+        } else {
+            if (!attr_done[4]) {
+                err = cudaFuncSetAttribute(k_grouped_gemm_pair<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemBytes);
+                if (err != cudaSuccess) return err;
+                attr_done[4] = true;
+            }
+            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+        }
+    } else if (gather) {
         if (!attr_done[2]) {
             err = cudaFuncSetAttribute(k_grouped_gemm<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);

@@ -80,6 +80,12 @@ typedef enum {
 #define MOE_FLAG_CAPACITY 0x1u  /* capacity layout: C slots per expert + overflow */
 #define MOE_FLAG_LOGITS_IN 0x2u /* moe_route/moe_forward read the caller's fp32
                                    logits instead of computing x * W_r + bias */
+#define MOE_FLAG_GEMM_PAIRS 0x4u /* run moe_grouped_swiglu / moe_grouped_down on
+                                   pairs of CTAs sharing one tcgen05 MMA
+                                   (cta_group::2, M = 256, the token tile split
+                                   between the two CTAs).  Same results; on B200
+                                   it is slower for the shapes measured so far,
+                                   so it is off by default. */
 #define MOE_FLAG_TEST_STALL_SCAN 0x40000000u /* test only: the first histogram
                                    block never publishes, so its successor's
                                    bounded wait expires and reports

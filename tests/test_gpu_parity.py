@@ -256,3 +256,25 @@ def test_scan_wait_expires_and_reports(orc):
     assert r["status"] == 0
     o = _oracle_full(orc, L, cfg, r["logits"])
     assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
+
+
+@pytest.mark.parametrize("name", ["two_tiles_E4_k2", "skew_E8_k3_H384", "capacity_E16_k4_C24", "E1_dense"])
+def test_gemm_pairs_match_single_cta(orc, name):
+    """MOE_FLAG_GEMM_PAIRS runs both grouped GEMMs on pairs of CTAs sharing
+    one MMA (cta_group::2, M = 256, the token tile split between the CTAs):
+    the same h and y as the single-CTA kernels on every filled row, within the
+    output tolerance against the oracle (ragged tails, a 128-feature last
+    block, the capacity layout, one expert)."""
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    s1 = shape_of(cfg)
+    s2 = shape_of(cfg, flags=moe.MOE_FLAG_GEMM_PAIRS)
+    a = host(run_steps(dl, s1), s1)
+    b = host(run_steps(dl, s2), s2)
+    assert a["status"] == 0 and b["status"] == 0
+    filled = a["src_token"] >= 0
+    for key in ("h", "y"):
+        assert np.array_equal(a[key][filled], b[key][filled]), key
+    o = _oracle_full(orc, L, cfg, b["logits"])
+    assert_close_bf16(b["out"], o["out"], "out with CTA pairs")
