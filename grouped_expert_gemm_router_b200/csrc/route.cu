@@ -17,8 +17,9 @@
 //   each) and HS = 32/ES lanes the hidden pairs.  Each thread holds a TB x EJ
 //   tile of sums, so every weight value it reads feeds TB multiply-adds; the
 //   warps' partial sums are added in warp order.
-// - Top-k: one warp per token, each lane holding ceil(E/32) candidates as
-//   64-bit keys (orderable logit << 32 | ~expert); k rounds of a warp max.
+// - Top-k: one warp per token, each lane holding ceil(E/32) candidates; k
+//   rounds of a warp max of the orderable logit and a warp min of the expert
+//   index among the lanes holding that maximum (redux.sync).
 // - Fused dispatch (small batches, called from moe_forward): every CTA that
 //   finished its top-k takes a ticket after a memory fence; the CTA that takes
 //   the last one (no CTA ever waits for another) builds the whole dispatch of
@@ -114,15 +115,6 @@ __device__ __forceinline__ uint32_t orderable(float f) {
     if (f == 0.0f) f = 0.0f;
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
-        v = o > v ? o : v;
-    }
-    return v;
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -279,22 +271,27 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
     __syncthreads();
 
-    // Top-k, one warp per token.  Selected slot j lives in register m = j / 32
-    // of lane j % 32 (k <= E <= 256: at most 8 per lane), so the softmax needs
-    // no round trip through global memory.
+    // Top-k, one warp per token.  Lane l holds experts l, l + 32, ... (E <= 256:
+    // at most 8); a round picks the largest orderable logit over the warp
+    // (redux max), then the lowest expert index among the lanes holding it
+    // (redux min) -- the larger logit, ties to the lower index, NaN below
+    // every number.  Selected slot j lives in register m = j / 32 of lane
+    // j % 32, so the softmax needs no round trip through global memory.
     for (int tok = warp; tok < TB; tok += 8) {
         const int t = t0 + tok;
         if (t >= a.T) break;
-        unsigned long long key[8];
+        uint32_t key[8];
+        uint32_t live = 0;  // bit m: candidate m (expert lane + 32 m) not yet taken
         bool nan = false;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int e = lane + 32 * m;
-            key[m] = 0ull;
+            key[m] = 0u;
             if (e < E) {
                 const float l = lg[tok][e];
                 nan |= (l != l);
-                key[m] = ((unsigned long long)orderable(l) << 32) | (0xFFFFFFFFu - (uint32_t)e);
+                key[m] = orderable(l);
+                live |= 1u << m;
             }
         }
         if (__any_sync(0xffffffffu, nan) && lane == 0) s_nan = 1;
@@ -303,16 +300,19 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
         for (int m = 0; m < 8; ++m) sel[m] = 0.0f;
         float lmax = 0.0f;
         for (int j = 0; j < a.k; ++j) {
-            unsigned long long best = 0ull;
+            // this lane's best live candidate (strict '>' keeps the lower index)
+            uint32_t bk = 0u;
+            int bm = -1;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) best = key[m] > best ? key[m] : best;
-            best = warp_max_u64(best);
-            const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-            if ((e & 31) == lane) {
-#pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    if (m == (e >> 5)) key[m] = 0ull;
-            }
+            for (int m = 0; m < 8; ++m)
+                if (((live >> m) & 1u) && (bm < 0 || key[m] > bk)) {
+                    bk = key[m];
+                    bm = m;
+                }
+            const uint32_t wk = __reduce_max_sync(0xffffffffu, bm >= 0 ? bk : 0u);
+            const uint32_t mine = (bm >= 0 && bk == wk) ? (uint32_t)(lane + 32 * bm) : 0xFFFFFFFFu;
+            const int e = (int)__reduce_min_sync(0xffffffffu, mine);
+            if ((e & 31) == lane) live &= ~(1u << (e >> 5));
             const float l = lg[tok][e];  // same address in every lane: a broadcast
             if (j == 0) lmax = l;
             if ((j & 31) == lane) {
@@ -442,7 +442,9 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     ej = ej <= 1 ? 1 : ej <= 2 ? 2 : ej <= 4 ? 4 : 8;
     int TB = route_tile_tokens(ej);
     // Small batches: halve the tile while 8-CTA clusters of full tiles would
-    // leave more than a quarter of the SMs idle.
+    // leave more than a quarter of the SMs idle.  (32-token tiles, which read
+    // each weight slice for more tokens, measured slower: smaller slices and
+    // longer top-k per CTA.)
     if (TB == 16 && !a.logits_in && ((s.T + 15) / 16) * 8 < (3 * num_sms) / 4) TB = 8;
     const int tiles = (s.T + TB - 1) / TB;
     a.tiles = tiles;
