@@ -243,6 +243,32 @@ def run_reference(args):
     return 0
 
 
+def replica_tokens(cfg, rank, L):
+    """The token batch of one replica: rank 0 the seeded batch of the layer,
+    rank r the batch drawn with seed offset r (same weights everywhere)."""
+    import synth
+    return L.x if rank == 0 else synth.x_tokens(cfg, seed_offset=rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings over every rank of the job
+    (the slowest replica sets the job's time); unchanged without a process
+    group of more than one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(tokens_per_replica_step, steps, world, total_ms):
+    """Tokens per second of the whole job: every replica's tokens over the
+    slowest replica's time."""
+    return tokens_per_replica_step * steps * world / (total_ms * 1e-3)
+
+
 def forward_launches(cfg):
     """Kernels one moe_forward launches: the router (plus the weight split and
     the tensor-core logits from 2048 tokens on), the histogram and rank
@@ -276,7 +302,7 @@ def run_ours(args):
     cfg = workload(args)
     t0 = time.time()
     L = synth.make_layer(cfg)
-    x_rank = synth.x_tokens(cfg, seed_offset=rank) if rank else L.x  # each replica its own tokens
+    x_rank = replica_tokens(cfg, rank, L)  # each replica its own tokens
     log("rank %d: generated %s in %.1f s" % (rank, cfg.name, time.time() - t0))
 
     def dev_bf16(a):
@@ -378,10 +404,7 @@ def run_ours(args):
     clocks = sampler.stop()
     total_ms = float(np.sum([a.elapsed_time(c) for a, c in gev]))
     del g
-    if world > 1:
-        t = torch.tensor([total_ms, eager_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, eager_ms = float(t[0].item()), float(t[1].item())
+    total_ms, eager_ms = max_over_ranks([total_ms, eager_ms], dev)
     status |= moe.moe_read_status(ws, stream)
 
     counts = b["expert_counts"].cpu().numpy()
@@ -406,15 +429,11 @@ def run_ours(args):
             eev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = float(np.sum([a.elapsed_time(c) for a, c in eev]))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     result = None
     if rank == 0:
-        tokens = cfg.T * K * world
-        value = tokens / (total_ms * 1e-3)
+        value = whole_job_rate(cfg.T, K, world, total_ms)
         # dominant kernel: the fused gate+up SwiGLU grouped GEMM
         t_sw = kmean[2]
         t_hbm = work["swiglu_bytes"] / (peaks["hbm_gbs"] * 1e9)
@@ -454,7 +473,7 @@ def run_ours(args):
                                >= work["layer_flops"] / (peaks["bf16_tflops"] * 1e12) else "tensor"},
             "kernels": kernels,
             "eager_entry_points_ms_per_step": eager_ms / K,
-            "e2e": {"value": cfg.T * K * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(cfg.T, K, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
             "gpu_launches": forward_launches(cfg) * K,
             "clocks": clocks,
