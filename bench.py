@@ -51,6 +51,8 @@ def parse_args():
     p.add_argument("--config", type=int, default=2)
     p.add_argument("--alpha", type=float, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--gemm-pairs", action="store_true",
+                   help="run the grouped GEMMs on CTA pairs (MOE_FLAG_GEMM_PAIRS; off by default: slower on B200)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     p.add_argument("--ref-budget-s", type=float, default=150.0)
     return p.parse_args()
@@ -308,7 +310,8 @@ def run_ours(args):
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=cfg.C > 0)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=cfg.C > 0,
+                           flags=moe.MOE_FLAG_GEMM_PAIRS if args.gemm_pairs else 0)
     b = moe.alloc_buffers(shape, dev)
     b.update(x=dev_bf16(x_rank), w_router=torch.from_numpy(L.w_router).to(dev),
              bias=None if L.bias is None else torch.from_numpy(L.bias).to(dev),
@@ -466,7 +469,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu"}),
+            "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu",
+                                        "gemm": "cta pairs" if args.gemm_pairs else "single cta"}),
             "roofline": roof,
             "layer_roofline": {"frac": layer_t / (total_ms * 1e-3 / K), "roofline_us": layer_t * 1e6,
                                "bound": "hbm" if work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
