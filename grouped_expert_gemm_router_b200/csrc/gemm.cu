@@ -689,6 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // it allows, and the down projection of a 128-unit layer loses half of its
 // per-CTA rate), so it is off by default.
 constexpr int kPairMaxAStages = 12;
+constexpr int kPairMaxBStages = 8;
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
@@ -702,8 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     uint64_t *fullA = reinterpret_cast<uint64_t *>(ctrl);
     uint64_t *emptyA = fullA + kPairMaxAStages;
     uint64_t *fullB = emptyA + kPairMaxAStages;
-    uint64_t *emptyB = fullB + kMaxBStages;
-    uint64_t *tfull = emptyB + kMaxBStages;
+    uint64_t *emptyB = fullB + kPairMaxBStages;
+    uint64_t *tfull = emptyB + kPairMaxBStages;
     uint64_t *tempty = tfull + 2;
     uint64_t *mma_done = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -723,12 +724,12 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
     const uint32_t a_tiles = MODE == 0 ? 2u : 1u;
     const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)(trows / 2) * kBRowBytes;
-    int nb = kMaxBStages;
+    // Both rings equally deep (a pipeline stage waits for its weight and its
+    // token tile alike, and both can come from HBM), then the rest of shared
+    // memory for more weight stages.
+    int nb = (int)(kRingBytes / (a_bytes + b_bytes));
+    nb = nb > kPairMaxBStages ? kPairMaxBStages : (nb < 2 ? 2 : nb);
     int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    if (fit < 4) {
-        nb = 3;
-        fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    }
     const int na = fit > kPairMaxAStages ? kPairMaxAStages : fit;
     uint8_t *ringB = smem + (uint32_t)na * a_bytes;
 
@@ -738,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
             mbar_init(&fullA[s], 1);
             mbar_init(&emptyA[s], 1);
         }
-        for (int s = 0; s < kMaxBStages; ++s) {
+        for (int s = 0; s < kPairMaxBStages; ++s) {
             mbar_init(&fullB[s], 1);
             mbar_init(&emptyB[s], 1);
         }
