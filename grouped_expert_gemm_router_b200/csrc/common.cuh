@@ -37,7 +37,7 @@ struct WsLayout {
     size_t tile_map;              // int4[max_tiles]
     size_t dispatch_end;          // end of what the dispatch step uses (the router's buffers follow)
     size_t router_planes;         // bf16[3][H][router_plane_cols(E)] (tensor-core router only)
-    size_t router_logits;         // fp32[T][E] when the caller passes no logits buffer
+    size_t router_part;           // fp32[q][T][E] partial logits of the K ranges (tensor-core router only)
     size_t total;
     int nchunks, max_tiles;
 };
@@ -50,6 +50,44 @@ constexpr int kTcRouterMinTokens = 2048;
 inline bool use_tc_router(int T) { return T >= kTcRouterMinTokens; }
 // Columns of one router-weight plane: E rounded up to the 64-column TMA box.
 inline int router_plane_cols(int E) { return (E + 63) / 64 * 64; }
+
+// Work split of the tensor-core router.  A unit is `rows` tokens times one
+// range of `kb` 64-wide K blocks; the hidden dimension is cut into q ranges
+// (each written as a partial-logit plane and added in range order by the
+// top-k kernel), and inside a unit the K blocks rotate over `groups`
+// accumulators.  Every logit is thus the fixed-order sum of q * groups >=
+// kRouteChains independent accumulation chains of at most ceil(H/64/8) K
+// blocks each, the accuracy the exact three-plane split needs from the
+// tensor cores' fp32 accumulator.  Tokens per unit: as many as one MMA takes
+// (256, or 128 with a second 128-expert accumulator), so that each weight
+// tile read from L2 feeds the most tokens (256; with a second 128-expert
+// accumulator 64, so that two stages of both operands still fit in shared
+// memory); the K split then fills the SMs.
+constexpr int kRouteChains = 8;
+constexpr int kRouteMaxQ = 16;
+constexpr int kRoutePlanMaxSms = 160;  // the workspace is sized for up to this many SMs
+struct RouterTcPlan {
+    int rows, groups, q, kb;
+};
+inline RouterTcPlan router_tc_plan(int T, int H, int E, int num_sms) {
+    const int nacc = E > 128 ? 2 : 1;
+    RouterTcPlan p;
+    p.rows = nacc == 1 ? 256 : 64;
+    p.groups = 512 / (nacc * p.rows);
+    if (p.groups > kRouteChains) p.groups = kRouteChains;
+    const int nk = H / 64;
+    const int ntb = (T + p.rows - 1) / p.rows;
+    if (num_sms > kRoutePlanMaxSms) num_sms = kRoutePlanMaxSms;
+    const int qmin = (kRouteChains + p.groups - 1) / p.groups;
+    int q = num_sms / ntb;
+    if (q < qmin) q = qmin;
+    if (q > kRouteMaxQ) q = kRouteMaxQ;
+    if (q > nk) q = nk;
+    if (q < 1) q = 1;
+    p.kb = (nk + q - 1) / q;
+    p.q = (nk + p.kb - 1) / p.kb;  // no empty range
+    return p;
+}
 
 // Routed pairs up to which moe_forward lets the router's last CTA build the
 // dispatch (histogram, scan, schedule, ranks) instead of separate kernels.
@@ -101,10 +139,11 @@ inline WsLayout ws_layout(int T, int H, int E, int k, int C, bool capped) {
     L.reset_end = o;
     L.tile_map = arr(16 * (size_t)L.max_tiles);
     L.dispatch_end = o;
-    L.router_planes = L.router_logits = 0;
+    L.router_planes = L.router_part = 0;
     if (use_tc_router(T)) {
         L.router_planes = arr(3 * (size_t)H * router_plane_cols(E) * 2);
-        L.router_logits = arr(4 * (size_t)T * E);
+        // q grows with the SM count: the bound of the largest device planned for
+        L.router_part = arr(4 * (size_t)router_tc_plan(T, H, E, kRoutePlanMaxSms).q * T * E);
     }
     L.total = o;
     return L;

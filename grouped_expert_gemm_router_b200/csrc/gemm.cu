@@ -7,14 +7,15 @@
 //   mode 1, down projection (same page, desk editor letter):
 //           y[r, c] = bf16( h[r] . Wd[e][:, c] )
 //   mode 2, router logits of step 1 on the tensor cores (for large batches):
-//           logits[t, e] = fp32( x[t] . (P0 + P1 + P2)[:, e] ) + bias[e], where
-//           P0 + P1 + P2 is the exact three-way bf16 split of the fp32 router
-//           weights (to 2^-27 relative); every product of two bf16 values is
-//           exact in fp32.  The tensor cores' fp32 accumulator loses low bits
-//           on every accumulate, so the K loop is spread over kRouteGroups
-//           accumulators (k-block j goes to accumulator j mod kRouteGroups),
-//           each seeing a fraction of the steps, and the epilogue adds the
-//           partial sums in fp32 in a fixed order.
+//           part[q, t, e] = fp32( x[t, Kq] . (P0 + P1 + P2)[Kq, e] ) over the
+//           q-th range Kq of the hidden dimension, where P0 + P1 + P2 is the
+//           exact three-way bf16 split of the fp32 router weights (to 2^-27
+//           relative); every product of two bf16 values is exact in fp32.  The
+//           top-k kernel adds the ranges in order and the bias.  The tensor
+//           cores' fp32 accumulator loses low bits on every accumulate, so
+//           inside a unit the K blocks rotate over route_groups accumulators
+//           (block j of the range to accumulator j mod route_groups) and the
+//           epilogue adds them in fp32 in a fixed order.
 //
 // Design (B200 first, not the page's Triton kernel):
 // - Swap-AB.  The MMA computes D[feature, row] = W^T[feature, k] * X^T[k, row]:
@@ -79,7 +80,6 @@ constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
 static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
               "three weight stages and three token stages of 256 rows must fit");
-constexpr int kRouteGroups = 8;                // mode 2: accumulators the K loop is spread over
 constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
 constexpr int kEpiWarps = 16;                  // four per tensor-memory lane quarter
 constexpr int kEpiSub = kEpiWarps / 4;         // warps sharing one lane quarter
@@ -101,12 +101,14 @@ struct GemmArgs {
     int max_tiles;  // capacity of the tile map
     unsigned long long timeout_ns;
     // mode 2 (router logits)
-    const float *bias;  // [E] or null
-    float *logits;      // [T, E]
+    float *logits;      // partial planes [route_q][T][E]
     int T;              // tokens
     // mode 0 with the row gather: the B rows come from x[src_token[row]]
     const int *src_token;
     int route_rows;     // tokens per unit (multiple of 16, <= 256)
+    int route_q;        // K ranges (units per token block)
+    int route_kb;       // K blocks per range
+    int route_groups;   // accumulators per unit: route_groups * nacc * route_rows <= 512 columns
 };
 
 struct Unit {
@@ -120,10 +122,12 @@ template <int MODE>
 // accumulators, or 128 in one when that still fits one wave).
 __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, int num_fb, int fbw,
                                             Unit &U) {
-    if (MODE == 2) {  // unit u = tokens [u * route_rows, ...), all experts
+    if (MODE == 2) {  // unit u = tokens [tb * route_rows, ...) x K range fb, all experts
+        const int tb = u / a.route_q;
         U.e = 0;
-        U.fb = 0;
-        U.p0s = u * a.route_rows;
+        U.fb = u - tb * a.route_q;
+        U.fx = 0;
+        U.p0s = tb * a.route_rows;
         U.p0l = min(a.route_rows, a.T - U.p0s);
         U.p1s = 0;
         U.p1l = 0;
@@ -228,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int total, trows;
     int num_fb = a.num_fb, fbw = MODE == 0 ? 128 : 256;
     if (MODE == 2) {
-        total = (a.T + a.route_rows - 1) / a.route_rows;
+        total = (a.T + a.route_rows - 1) / a.route_rows * a.route_q;
         trows = a.route_rows;
     } else {
         const int ntiles = *a.num_tiles;
@@ -249,13 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stages of trows rows (multiple of 16, <= 256).  Four token stages
     // while that leaves at least four weight stages, else three; the weight
     // ring takes the rest, so that as many weight bytes as possible are in
-    // flight.
+    // flight.  Mode 2 reads both operands from L2 and consumes one stage of
+    // each per K block: equally deep rings.
     trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
     const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
     const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)trows * kBRowBytes;
     int nb = kMaxBStages;
     int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    if (fit < 4) {
+    if (MODE == 2) {
+        nb = (int)(kRingBytes / (a_bytes + b_bytes));
+        nb = nb > kMaxBStages ? kMaxBStages : nb;
+        fit = nb;
+    } else if (fit < 4) {
         nb = 3;
         fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
     }
@@ -387,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bytes = is_a ? (MODE == 2 ? 3u : 1u) * (uint32_t)U.nacc * kATile
                                             : (uint32_t)(nb0 + nb1) * kBBox;
                 const int krow = U.e * a.K;
+                const int kb0 = MODE == 2 ? U.fb * a.route_kb : 0;
+                const int kb1 = MODE == 2 ? min(nk, kb0 + a.route_kb) : nk;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, a.timeout_ns, s_abort)) {
                         ok = false;
                         break;
@@ -459,7 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok && big) ok = mbar_wait_bounded(&tempty[1], (plan.uses[1] & 1u) ^ 1u, a.timeout_ns, s_abort);
                 if (!ok) break;
                 tc_fence_after();
-                for (int kb = 0; kb < nk; ++kb) {
+                const int kb0 = MODE == 2 ? U.fb * a.route_kb : 0;
+                const int kb1 = MODE == 2 ? min(nk, kb0 + a.route_kb) : nk;
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(&fullA[sa], pha, a.timeout_ns, s_abort) ||
                         !mbar_wait_bounded(&fullB[sb], phb, a.timeout_ns, s_abort)) {
                         ok = false;
@@ -469,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sa0 = baseA + sa * a_bytes, sa1 = sa0 + kATile, sbt = baseB + sb * b_bytes;
                     if (MODE == 2) {
                         // accumulator (group g, expert block c) at column (g * nacc + c) * trows
-                        const int g = kb % kRouteGroups;
+                        const int j = kb - kb0, g = j % a.route_groups;
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
                             const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
@@ -477,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int c = 0; c < U.nacc; ++c) {
                                     const uint32_t at = sa0 + (uint32_t)(pl * U.nacc + c) * kATile + kk * 2048;
                                     const uint32_t dst = tmem + (uint32_t)((g * U.nacc + c) * trows);
-                                    const uint32_t accum = (kb >= kRouteGroups || kk || pl) ? 1u : 0u;
+                                    const uint32_t accum = (j >= a.route_groups || kk || pl) ? 1u : 0u;
                                     tc_mma_bf16(dst, sdesc_sw128(at, kABox, 1024), bdesc, idesc, accum);
                                 }
                         }
@@ -555,9 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int f0 = U.fx + L;
             unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
             if (MODE == 2) {
-                // fp32 logits + bias: lane L of expert block c is expert c*128 + L;
-                // the groups' partial sums are added in order g = 0, 1, ...
-                const int ng = nk < kRouteGroups ? nk : kRouteGroups;
+                // fp32 partial logits of K range U.fb: lane L of expert block c
+                // is expert c*128 + L; the groups' sums are added in order
+                // g = 0, 1, ...
+                const int kb0 = U.fb * a.route_kb;
+                const int nkr = min(nk, kb0 + a.route_kb) - kb0;
+                const int ng = nkr < a.route_groups ? nkr : a.route_groups;
+                float *part = a.logits + (size_t)U.fb * a.T * a.E;
                 for (int c0 = sub * 16; c0 < U.N; c0 += 16 * kEpiSub) {
                     for (int c = 0; c < U.nacc; ++c) {
                         float acc[16];
@@ -571,11 +588,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int j = 0; j < 16; ++j) acc[j] += __uint_as_float(r[j]);
                         }
                         const int e = c * 128 + L;
-                        const float be = (a.bias && e < a.E) ? a.bias[e] : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int row = unit_row(U, c0 + j);
-                            if (row >= 0 && e < a.E) a.logits[(size_t)row * a.E + e] = acc[j] + be;
+                            if (row >= 0 && e < a.E) part[(size_t)row * a.E + e] = acc[j];
                         }
                     }
                 }
@@ -1049,9 +1065,11 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
 }  // namespace
 
 // Router logits on the tensor cores: planes of W_r into the workspace, then
-// mode 2 of the grouped GEMM (one unit per block of route_rows tokens).
-cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, const float *bias,
-                                    float *logits, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+// mode 2 of the grouped GEMM (one unit per block of route_rows tokens and
+// range of the hidden dimension), which writes the partial-logit planes
+// `part` [q][T][E]; returns q.
+cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, float *part, int *q,
+                                    const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
                                     cudaStream_t stream) {
     const int Ep = router_plane_cols(s.E);
     __nv_bfloat16 *planes = (__nv_bfloat16 *)((char *)ws + L.router_planes);
@@ -1071,21 +1089,20 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
     a.K = s.H;
     a.E = s.E;
     a.timeout_ns = timeout_ns;
-    a.bias = bias;
-    a.logits = logits;
+    a.logits = part;
     a.T = s.T;
-    // kRouteGroups accumulators of nacc expert blocks must fit in 512 columns.
-    const int nacc = s.E > 128 ? 2 : 1;
-    const int max_rows = 512 / (kRouteGroups * nacc);
-    int rows = (s.T + num_sms - 1) / num_sms;
-    rows = (rows + 15) & ~15;
-    a.route_rows = rows < 16 ? 16 : (rows > max_rows ? max_rows : rows);
+    const RouterTcPlan plan = router_tc_plan(s.T, s.H, s.E, num_sms);
+    a.route_rows = plan.rows;
+    a.route_q = plan.q;
+    a.route_kb = plan.kb;
+    a.route_groups = plan.groups;
     static bool attr_done = false;
     if (!attr_done) {
         err = cudaFuncSetAttribute(k_grouped_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (err != cudaSuccess) return err;
         attr_done = true;
     }
+    *q = plan.q;
     k_grouped_gemm<2><<<num_sms, kThreads, kSmemBytes, stream>>>(tA, tA, tB, a);
     return cudaGetLastError();
 }

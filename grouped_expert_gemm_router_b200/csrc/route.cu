@@ -37,7 +37,9 @@ struct RouteArgs {
     const __nv_bfloat16 *x;
     const float *w_router;
     const float *bias;
-    float *logits;  // output (or input with logits_in); may be null when not logits_in
+    float *logits;  // output (or input with logits_in and no lparts); may be null when output
+    const float *lparts;  // logits_in from the tensor cores: lq partial planes [lq][T][E] (bias not added)
+    int lq;
     int *topk_idx;
     float *topk_w;
     uint32_t *status;
@@ -263,6 +265,23 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
         }
         if (CL > 1) cluster_sync_all();  // every slice stays readable until rank 0 is done
         if (rank != 0) return;
+    } else if (a.lparts) {
+        // Partial planes of the hidden ranges, added in range order, then
+        // the bias; the logits are published for the caller.
+        const size_t plane = (size_t)a.T * E;
+        for (int i = tid; i < TB * E; i += 256) {
+            const int tok = i / E, e = i % E, t = t0 + tok;
+            float l = 0.0f;
+            if (t < a.T) {
+                const float *pp = a.lparts + (size_t)t * E + e;
+                l = pp[0];
+#pragma unroll 4
+                for (int q = 1; q < a.lq; ++q) l += pp[q * plane];
+                if (a.bias) l = l + a.bias[e];
+                if (a.logits) a.logits[(size_t)t * E + e] = l;
+            }
+            lg[tok][e] = l;
+        }
     } else {
         for (int i = tid; i < TB * E; i += 256) {
             const int tok = i / E, e = i % E, t = t0 + tok;
@@ -394,8 +413,8 @@ cudaError_t launch_ej(const RouteArgs &a, int ej, int tb, int smem, int tiles, c
 
 }  // namespace
 
-cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, const float *bias,
-                                    float *logits, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const float *w_router, float *part, int *q,
+                                    const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
                                     cudaStream_t stream);
 
 cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_router, const float *bias, float *logits,
@@ -409,11 +428,14 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     // dispatch resets the completion count it used and writes the empty
     // capacity slots' src_token itself.
     if (fused && (int64_t)s.T * s.k > kFusedDispatchMaxPairs) return cudaErrorInvalidValue;
+    const float *lparts = nullptr;
+    int lq = 0;
     if (!(s.flags & MOE_FLAG_LOGITS_IN) && use_tc_router(s.T)) {
-        // Logits on the tensor cores, then the top-k below reads them.
-        if (!logits) logits = (float *)((char *)ws + L.router_logits);
-        cudaError_t err = launch_router_logits_tc(s, x, w_router, bias, logits, L, ws, timeout_ns, num_sms, stream);
+        // Partial logits on the tensor cores, then the top-k below adds them.
+        float *part = (float *)((char *)ws + L.router_part);
+        cudaError_t err = launch_router_logits_tc(s, x, w_router, part, &lq, L, ws, timeout_ns, num_sms, stream);
         if (err != cudaSuccess) return err;
+        lparts = part;
         s.flags |= MOE_FLAG_LOGITS_IN;
     }
     RouteArgs a;
@@ -421,6 +443,8 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     a.w_router = w_router;
     a.bias = bias;
     a.logits = logits;
+    a.lparts = lparts;
+    a.lq = lq;
     a.topk_idx = topk_idx;
     a.topk_w = topk_w;
     a.status = status;
