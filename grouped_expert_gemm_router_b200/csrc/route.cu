@@ -20,6 +20,9 @@
 // - Top-k: one warp per token, each lane holding ceil(E/32) candidates; k
 //   rounds of a warp max of the orderable logit and a warp min of the expert
 //   index among the lanes holding that maximum (redux.sync).
+// - Logits computed elsewhere (given by the caller, or the tensor-core
+//   router's partial planes for large batches) go to k_topk: one warp per
+//   token loads its logits straight into registers, no CTA-wide staging.
 // - Fused dispatch (small batches, called from moe_forward): every CTA that
 //   finished its top-k takes a ticket after a memory fence; the CTA that takes
 //   the last one (no CTA ever waits for another) builds the whole dispatch of
@@ -111,12 +114,18 @@ __device__ void fused_dispatch_tail(const RouteArgs &a, uint8_t *smem) {
 }
 
 // Monotone map of a float onto uint32 (larger float -> larger key); -0 is
-// folded onto +0 and NaN maps to 0, below -inf (whose key is 0x007FFFFF).
+// folded onto +0 and NaN maps to 1, below -inf (whose key is 0x007FFFFF);
+// key 0 marks an empty candidate slot.
 __device__ __forceinline__ uint32_t orderable(float f) {
-    if (f != f) return 0u;
+    if (f != f) return 1u;
     if (f == 0.0f) f = 0.0f;
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// The float of a key (+0 for a folded -0, a quiet NaN for the NaN key).
+__device__ __forceinline__ float orderable_value(uint32_t k) {
+    if (k == 1u) return __uint_as_float(0x7FC00000u);
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -134,6 +143,145 @@ __device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t ran
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
     return v;
+}
+
+// logit = sum over q < lq of part[q * plane + i], in order q = 0, 1, ...,
+// then + bias[0] when bias is given (the tensor-core router's partial
+// planes of the hidden ranges).
+__device__ __forceinline__ float sum_partials(const float *__restrict__ part, size_t plane, int lq, size_t i,
+                                              const float *bias) {
+    float l = part[i];
+#pragma unroll 4
+    for (int q = 1; q < lq; ++q) l += part[(size_t)q * plane + i];
+    if (bias) l = l + *bias;
+    return l;
+}
+
+// Top-k and softmax of one token by one warp.  Lane l holds the logits of
+// experts l, l + 32, ..., l + 32 (MPL - 1) in v[] (MPL = 1, 2, 4 or 8 with
+// E <= 32 MPL; entries past E are ignored).  Each lane first sorts its
+// candidates (larger key first; a lane's candidates are in index order and
+// the insertion sort is stable, so equal keys keep the lower index first).
+// A round then takes the largest head key over the warp (redux max) and the
+// lowest expert index among the lanes whose head holds it (redux min) -- the
+// larger logit, ties to the lower index, NaN below every number -- and the
+// winning lane pops its head.  Selected slot j lives in register j / 32 of
+// lane j % 32, so the softmax needs no round trip through memory.  Writes
+// idx[0..k) and w[0..k); returns true (in every lane) if a logit was NaN.
+template <int MPL>
+__device__ __forceinline__ bool warp_topk_softmax(const float (&v)[MPL], int E, int k, int *idx, float *w) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[MPL];
+    int ix[MPL];
+    bool nan = false;
+#pragma unroll
+    for (int m = 0; m < MPL; ++m) {
+        const int e = lane + 32 * m;
+        key[m] = 0u;
+        ix[m] = 0x7FFFFFFF;
+        if (e < E) {
+            nan |= (v[m] != v[m]);
+            key[m] = orderable(v[m]);
+            ix[m] = e;
+        }
+    }
+#pragma unroll
+    for (int i = 1; i < MPL; ++i)
+#pragma unroll
+        for (int j = i; j > 0; --j)
+            if (key[j] > key[j - 1]) {
+                const uint32_t tk = key[j];
+                key[j] = key[j - 1];
+                key[j - 1] = tk;
+                const int ti = ix[j];
+                ix[j] = ix[j - 1];
+                ix[j - 1] = ti;
+            }
+    float sel[MPL];  // k <= E <= 32 MPL slots
+#pragma unroll
+    for (int m = 0; m < MPL; ++m) sel[m] = 0.0f;
+    float lmax = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, key[0]);
+        const int e = (int)__reduce_min_sync(0xffffffffu, key[0] == wk ? (uint32_t)ix[0] : 0xFFFFFFFFu);
+        if (ix[0] == e) {  // the owner pops its head
+#pragma unroll
+            for (int m = 0; m + 1 < MPL; ++m) {
+                key[m] = key[m + 1];
+                ix[m] = ix[m + 1];
+            }
+            key[MPL - 1] = 0u;
+            ix[MPL - 1] = 0x7FFFFFFF;
+        }
+        const float l = orderable_value(wk);
+        if (j == 0) lmax = l;
+        if ((j & 31) == lane) {
+#pragma unroll
+            for (int m = 0; m < MPL; ++m)
+                if (m == (j >> 5)) sel[m] = l;
+        }
+        if (lane == 0) idx[j] = e;
+    }
+    // Softmax over the k selected logits, reference = the largest (slot 0):
+    // per-lane partial sums over slots lane, lane + 32, ..., then a butterfly
+    // over the warp.
+    float ex[MPL];
+    float sum = 0.0f;
+#pragma unroll
+    for (int m = 0; m < MPL; ++m) {
+        ex[m] = 0.0f;
+        if (lane + 32 * m < k) {
+            ex[m] = expf(sel[m] - lmax);
+            sum += ex[m];
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll
+    for (int m = 0; m < MPL; ++m)
+        if (lane + 32 * m < k) w[lane + 32 * m] = ex[m] / sum;
+    return __any_sync(0xffffffffu, nan);
+}
+
+// Candidates per lane for E experts: 1, 2, 4 or 8.
+__host__ __device__ inline int topk_mpl(int E) { return E <= 32 ? 1 : (E <= 64 ? 2 : (E <= 128 ? 4 : 8)); }
+
+// Top-k of logits already computed (caller-given, or the tensor-core
+// router's partial planes), without the fused dispatch: one warp per token,
+// the logits straight into registers (all of a lane's loads issued before
+// the first is used), no shared-memory staging.
+template <int MPL>
+__global__ void __launch_bounds__(256) k_topk(RouteArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    if (t >= a.T) return;  // warp-uniform
+    const int E = a.E;
+    float v[MPL];
+    if (a.lparts) {
+        const size_t plane = (size_t)a.T * E;
+#pragma unroll
+        for (int m = 0; m < MPL; ++m) v[m] = lane + 32 * m < E ? a.lparts[(size_t)t * E + lane + 32 * m] : 0.0f;
+#pragma unroll 4
+        for (int q = 1; q < a.lq; ++q) {
+            const float *pq = a.lparts + (size_t)q * plane + (size_t)t * E;
+#pragma unroll
+            for (int m = 0; m < MPL; ++m)
+                if (lane + 32 * m < E) v[m] += pq[lane + 32 * m];
+        }
+#pragma unroll
+        for (int m = 0; m < MPL; ++m) {
+            const int e = lane + 32 * m;
+            if (e < E) {
+                if (a.bias) v[m] = v[m] + a.bias[e];
+                if (a.logits) a.logits[(size_t)t * E + e] = v[m];
+            }
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < MPL; ++m) v[m] = lane + 32 * m < E ? a.logits[(size_t)t * E + lane + 32 * m] : 0.0f;
+    }
+    if (warp_topk_softmax<MPL>(v, E, a.k, a.topk_idx + (size_t)t * a.k, a.topk_w + (size_t)t * a.k) && lane == 0)
+        atomicOr(a.status, MOE_DEV_NAN_LOGIT);
 }
 
 template <int TB, int EJ>
@@ -268,16 +416,11 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     } else if (a.lparts) {
         // Partial planes of the hidden ranges, added in range order, then
         // the bias; the logits are published for the caller.
-        const size_t plane = (size_t)a.T * E;
         for (int i = tid; i < TB * E; i += 256) {
             const int tok = i / E, e = i % E, t = t0 + tok;
             float l = 0.0f;
             if (t < a.T) {
-                const float *pp = a.lparts + (size_t)t * E + e;
-                l = pp[0];
-#pragma unroll 4
-                for (int q = 1; q < a.lq; ++q) l += pp[q * plane];
-                if (a.bias) l = l + a.bias[e];
+                l = sum_partials(a.lparts, (size_t)a.T * E, a.lq, (size_t)t * E + e, a.bias ? a.bias + e : nullptr);
                 if (a.logits) a.logits[(size_t)t * E + e] = l;
             }
             lg[tok][e] = l;
@@ -290,75 +433,16 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
     __syncthreads();
 
-    // Top-k, one warp per token.  Lane l holds experts l, l + 32, ... (E <= 256:
-    // at most 8); a round picks the largest orderable logit over the warp
-    // (redux max), then the lowest expert index among the lanes holding it
-    // (redux min) -- the larger logit, ties to the lower index, NaN below
-    // every number.  Selected slot j lives in register m = j / 32 of lane
-    // j % 32, so the softmax needs no round trip through global memory.
+    // Top-k, one warp per token.
     for (int tok = warp; tok < TB; tok += 8) {
         const int t = t0 + tok;
         if (t >= a.T) break;
-        uint32_t key[8];
-        uint32_t live = 0;  // bit m: candidate m (expert lane + 32 m) not yet taken
-        bool nan = false;
+        float v[EJ];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int e = lane + 32 * m;
-            key[m] = 0u;
-            if (e < E) {
-                const float l = lg[tok][e];
-                nan |= (l != l);
-                key[m] = orderable(l);
-                live |= 1u << m;
-            }
-        }
-        if (__any_sync(0xffffffffu, nan) && lane == 0) s_nan = 1;
-        float sel[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) sel[m] = 0.0f;
-        float lmax = 0.0f;
-        for (int j = 0; j < a.k; ++j) {
-            // this lane's best live candidate (strict '>' keeps the lower index)
-            uint32_t bk = 0u;
-            int bm = -1;
-#pragma unroll
-            for (int m = 0; m < 8; ++m)
-                if (((live >> m) & 1u) && (bm < 0 || key[m] > bk)) {
-                    bk = key[m];
-                    bm = m;
-                }
-            const uint32_t wk = __reduce_max_sync(0xffffffffu, bm >= 0 ? bk : 0u);
-            const uint32_t mine = (bm >= 0 && bk == wk) ? (uint32_t)(lane + 32 * bm) : 0xFFFFFFFFu;
-            const int e = (int)__reduce_min_sync(0xffffffffu, mine);
-            if ((e & 31) == lane) live &= ~(1u << (e >> 5));
-            const float l = lg[tok][e];  // same address in every lane: a broadcast
-            if (j == 0) lmax = l;
-            if ((j & 31) == lane) {
-#pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    if (m == (j >> 5)) sel[m] = l;
-            }
-            if (lane == 0) a.topk_idx[(size_t)t * a.k + j] = e;
-        }
-        // Softmax over the k selected logits, reference = the largest (slot 0):
-        // per-lane partial sums over slots lane, lane + 32, ..., then a
-        // butterfly over the warp.
-        float ex[8];
-        float sum = 0.0f;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            ex[m] = 0.0f;
-            if (lane + 32 * m < a.k) {
-                ex[m] = expf(sel[m] - lmax);
-                sum += ex[m];
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            if (lane + 32 * m < a.k) a.topk_w[(size_t)t * a.k + lane + 32 * m] = ex[m] / sum;
+        for (int m = 0; m < EJ; ++m) v[m] = lane + 32 * m < E ? lg[tok][lane + 32 * m] : 0.0f;
+        // EJ experts per lane in the sums above = ceil(E/32) rounded up to a power of two
+        if (warp_topk_softmax<EJ>(v, E, a.k, a.topk_idx + (size_t)t * a.k, a.topk_w + (size_t)t * a.k) && lane == 0)
+            s_nan = 1;
     }
     __syncthreads();
     if (tid == 0 && s_nan) atomicOr(a.status, MOE_DEV_NAN_LOGIT);
@@ -459,6 +543,18 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     a.P = (int)P;
     a.out = fused ? *fused : FusedDispatch{nullptr, nullptr, nullptr, nullptr};
     a.ws = ws_ptrs(ws, L);
+    if (a.logits_in && !fused) {
+        const int blocks = (int)(((int64_t)s.T * 32 + 255) / 256);
+        if (blocks > 0) {
+            switch (topk_mpl(s.E)) {
+                case 1: k_topk<1><<<blocks, 256, 0, stream>>>(a); break;
+                case 2: k_topk<2><<<blocks, 256, 0, stream>>>(a); break;
+                case 4: k_topk<4><<<blocks, 256, 0, stream>>>(a); break;
+                default: k_topk<8><<<blocks, 256, 0, stream>>>(a); break;
+            }
+        }
+        return cudaGetLastError();
+    }
     int es = 1;
     while (es < s.E && es < 32) es <<= 1;
     a.es = es;

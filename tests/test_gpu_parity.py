@@ -167,6 +167,37 @@ def test_logits_in_ties(orc):
     assert r["status"] & moe.MOE_DEV_NAN_LOGIT
 
 
+@pytest.mark.parametrize("T,E,k", [(257, 64, 7), (120, 100, 33), (257, 128, 8), (100, 200, 40), (300, 128, 8),
+                                   (40, 256, 256)])
+def test_logits_in_ties_wide(orc, T, E, k):
+    """Ties among each lane's several candidates (E > 32), zeros of both
+    signs, NaNs, and k past one warp's width: the step-by-step router and
+    moe_forward (which builds the dispatch inside the router for small
+    batches) both follow the lowest-index tie-break exactly."""
+    cfg = synth.LayerConfig("t", T, 128, 128, E, k, seed=9)
+    L = synth.make_layer(cfg)
+    rng = np.random.default_rng(E + k)
+    logits = rng.integers(-2, 3, size=(T, E)).astype(np.float32)
+    logits[(logits == 0) & (rng.random((T, E)) < 0.5)] = -0.0
+    logits[1, :] = np.nan
+    logits[2, ::3] = np.nan
+    shape = shape_of(cfg, logits_in=True)
+    dl = DeviceLayer(L)
+    idx, w, _ = orc.topk_softmax(logits, k)
+    ok = np.isfinite(w).all(axis=1)
+    r = host(run_steps(dl, shape, logits=logits), shape)
+    b = dl.bufs(shape)
+    b["logits"].copy_(torch.from_numpy(logits))
+    moe.moe_forward(shape, b, b["ws"], args=moe.forward_args(b))
+    torch.cuda.synchronize()
+    f = host(b, shape)
+    for got in (r, f):
+        assert np.array_equal(got["topk_idx"], idx)
+        assert np.max(np.abs(got["topk_w"][ok] - w[ok])) <= WEIGHT_TOL
+        assert got["status"] & moe.MOE_DEV_NAN_LOGIT
+    assert np.array_equal(r["out"], f["out"])
+
+
 def test_all_tokens_to_one_expert(orc):
     """A dominant bias sends every token to expert 0 (n_0 = T, 3 row tiles)."""
     cfg = synth.LayerConfig("t", 600, 128, 256, 8, 2, seed=9)
