@@ -12,7 +12,8 @@
 namespace moe {
 
 // ------------------------------------------------------------------ tiling --
-constexpr int kScanChunk = 2048;     // routed pairs per histogram / rank block
+constexpr int kScanChunk = 1024;     // routed pairs per histogram / rank block
+constexpr int kLookback = 16;        // predecessor chunks read at once by the scan's look-back
 constexpr int kScanThreads = 256;
 constexpr int kMaxExperts = 256;
 constexpr int kTileRows = 256;       // largest UMMA N: most permuted rows a GEMM tile holds
@@ -197,6 +198,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {

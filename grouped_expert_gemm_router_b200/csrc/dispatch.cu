@@ -7,9 +7,10 @@
 //
 // k_hist_scan  one pass over topk_idx.  Each block takes a ticket (its block
 //              index in launch-independent order), histograms its chunk of
-//              2048 pairs in shared memory and resolves, per expert, the count
+//              1024 pairs in shared memory and resolves, per expert, the count
 //              of that expert in all earlier chunks by decoupled look-back
-//              over per-(chunk, expert) flag words.  The block holding the
+//              over per-(chunk, expert) flag words, kLookback chunks per
+//              read.  The block holding the
 //              last chunk owns the totals and builds the per-expert offsets,
 //              the capacity/overflow offsets and the GEMM tile schedule, all
 //              on the device: nothing goes back to the host.
@@ -73,28 +74,47 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
             if (publish) st_release_u64(mine, ((unsigned long long)kFlagPrefix << 32) | (uint32_t)agg);
         } else {
             st_release_u64(mine, ((unsigned long long)kFlagAggregate << 32) | (uint32_t)agg);
+            // Look back over windows of kLookback predecessors, all of a
+            // window's words read at once: add the aggregates from the
+            // nearest chunk backwards until an inclusive prefix (chunk 0
+            // always publishes one).  A predecessor that has not published
+            // yet stops the walk there, and the window is read again after a
+            // short sleep (bounded by the timeout).  Every word holds its flag
+            // and value together, so relaxed loads suffice.
             int p = chunk - 1;
             uint64_t deadline = 0;
-            uint32_t spins = 0;
-            while (p >= 0) {
-                const unsigned long long v = ld_acquire_u64(a.ws.scan_state + (size_t)p * E + e);
-                const uint32_t flag = (uint32_t)(v >> 32);
-                if (flag == 0u) {
-                    if ((++spins & 63u) == 0) {
-                        const uint64_t now = globaltimer_ns();
-                        if (deadline == 0) {
-                            deadline = now + a.timeout_ns;
-                        } else if (now > deadline) {
-                            s_timeout = 1;
-                            break;
-                        }
+            while (true) {
+                unsigned long long v[kLookback];
+#pragma unroll
+                for (int i = 0; i < kLookback; ++i)
+                    v[i] = p - i >= 0 ? ld_relaxed_u64(a.ws.scan_state + (size_t)(p - i) * E + e)
+                                      : ((unsigned long long)kFlagPrefix << 32);  // before chunk 0: prefix 0
+                int used = 0;
+                bool done = false, blocked = false;
+#pragma unroll
+                for (int i = 0; i < kLookback; ++i) {
+                    const uint32_t flag = (uint32_t)(v[i] >> 32);
+                    if (done || blocked) continue;
+                    if (flag == 0u) {
+                        blocked = true;
+                        continue;
+                    }
+                    excl += (int)(uint32_t)v[i];
+                    ++used;
+                    done = flag == kFlagPrefix;
+                }
+                p -= used;
+                if (done) break;
+                if (blocked) {
+                    const uint64_t now = globaltimer_ns();
+                    if (deadline == 0) {
+                        deadline = now + a.timeout_ns;
+                    } else if (now > deadline) {
+                        s_timeout = 1;
+                        break;
                     }
                     __nanosleep(64);
-                    continue;
                 }
-                excl += (int)(uint32_t)v;
-                if (flag == kFlagPrefix) break;
-                --p;
             }
             st_release_u64(mine, ((unsigned long long)kFlagPrefix << 32) | (uint32_t)(excl + agg));
         }

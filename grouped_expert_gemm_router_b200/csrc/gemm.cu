@@ -75,6 +75,7 @@ constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 featur
 constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
 constexpr uint32_t kBRowBytes = kBK * 2;       // one B row of a stage: 128 bytes
 constexpr uint32_t kBBox = 16 * kBRowBytes;    // TMA box: 16 rows x 64 K (2 KiB)
+constexpr int kRowBoxes = 5;                   // token-tile boxes of 16, 32, 64, 128 and 256 rows
 constexpr uint32_t kCtrlBytes = 3072;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
@@ -109,7 +110,33 @@ struct GemmArgs {
     int route_q;        // K ranges (units per token block)
     int route_kb;       // K blocks per range
     int route_groups;   // accumulators per unit: route_groups * nacc * route_rows <= 512 columns
+    uint32_t row_boxes; // bit i: RowMaps::m[i] (boxes of 16 << i rows) is valid; bit 0 always
 };
+
+// Tensor maps of the token matrix (B operand) with boxes of 16 << i rows x 64
+// K; the row gather uses m[0] alone, with one-row boxes.
+struct RowMaps {
+    CUtensorMap m[kRowBoxes];
+};
+
+// Rows [row0, row0 + n) (n a multiple of 16, <= 256) of the token matrix at
+// K offset kx into consecutive 128-byte shared-memory rows from dst, largest
+// boxes first: a 256-row tile is one copy instead of sixteen, which keeps the
+// single producer thread's TMA issue off the critical path.
+__device__ __forceinline__ void tma_load_rows(uint8_t *dst, const RowMaps &rm, uint32_t boxes, uint64_t *bar, int kx,
+                                              int row0, int n) {
+#pragma unroll
+    for (int i = kRowBoxes - 1; i >= 0; --i) {
+        const int h = 16 << i;
+        if (!((boxes >> i) & 1u)) continue;
+        while (n >= h) {
+            tma_load_2d(dst, &rm.m[i], bar, kx, row0);
+            dst += h * kBRowBytes;
+            row0 += h;
+            n -= h;
+        }
+    }
+}
 
 struct Unit {
     int e, fb, fx, nacc, N, n0p, p0s, p0l, p1s, p1l;  // fx: first output feature of accumulator 0
@@ -210,7 +237,7 @@ __device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *statu
 template <int MODE, bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+                   const __grid_constant__ RowMaps tmB, GemmArgs a) {
     static_assert(!GATHER || MODE == 0, "the row gather feeds the SwiGLU GEMM");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -293,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA0);
         tma_prefetch_desc(&tmA1);
-        tma_prefetch_desc(&tmB);
+        for (int b = 0; b < kRowBoxes; ++b)
+            if ((a.row_boxes >> b) & 1u) tma_prefetch_desc(&tmB.m[b]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -351,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *sb = ringB + stage * b_bytes;
                     const int kx = kb * kBK;
                     for (int g = 0; g < U.N; g += 4)
-                        tma_gather4(sb + g * kBRowBytes, &tmB, &fullB[stage], kx, s_rows[g], s_rows[g + 1],
+                        tma_gather4(sb + g * kBRowBytes, &tmB.m[0], &fullB[stage], kx, s_rows[g], s_rows[g + 1],
                                     s_rows[g + 2], s_rows[g + 3]);
                     issued_ph[stage] = (int)ph;
                 }
@@ -408,10 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int ky = krow + kb * kBK, kx = kb * kBK;
                     if (!is_a) {
                         uint8_t *sb = ringB + stage * b_bytes;
-                        for (int i = 0; i < nb0; ++i)
-                            tma_load_2d(sb + i * kBBox, &tmB, &full[stage], kx, U.p0s + 16 * i);
-                        for (int i = 0; i < nb1; ++i)
-                            tma_load_2d(sb + U.n0p * kBRowBytes + i * kBBox, &tmB, &full[stage], kx, U.p1s + 16 * i);
+                        tma_load_rows(sb, tmB, a.row_boxes, &full[stage], kx, U.p0s, 16 * nb0);
+                        if (nb1) tma_load_rows(sb + U.n0p * kBRowBytes, tmB, a.row_boxes, &full[stage], kx, U.p1s, 16 * nb1);
                     } else if (MODE == 2) {
                         // tile (plane p, accumulator c) at index p * nacc + c;
                         // plane p holds rows [p*K, (p+1)*K) of the plane tensor
@@ -1062,6 +1088,15 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
     return r == CUDA_SUCCESS;
 }
 
+// The token matrix with boxes of 16, 32, ... 256 rows; returns the mask of the
+// maps that could be encoded (bit 0 is required).
+uint32_t make_row_maps(RowMaps *rm, const void *ptr, uint64_t rows, uint64_t cols) {
+    uint32_t boxes = 0;
+    for (int i = 0; i < kRowBoxes; ++i)
+        if (make_tmap(&rm->m[i], ptr, rows, cols, 64, 16u << i)) boxes |= 1u << i;
+    return (boxes & 1u) ? boxes : 0u;
+}
+
 }  // namespace
 
 // Router logits on the tensor cores: planes of W_r into the workspace, then
@@ -1079,10 +1114,11 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
     k_router_planes<<<blocks, 256, 0, stream>>>(w_router, planes, s.H, s.E, Ep);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    CUtensorMap tA, tB;
-    if (!make_tmap(&tA, planes, 3 * (uint64_t)s.H, (uint64_t)Ep, 64, 64) ||
-        !make_tmap(&tB, x, (uint64_t)s.T, (uint64_t)s.H, 64, 16))
-        return cudaErrorInvalidValue;
+    CUtensorMap tA;
+    RowMaps tB;
+    if (!make_tmap(&tA, planes, 3 * (uint64_t)s.H, (uint64_t)Ep, 64, 64)) return cudaErrorInvalidValue;
+    const uint32_t boxes = make_row_maps(&tB, x, (uint64_t)s.T, (uint64_t)s.H);
+    if (!boxes) return cudaErrorInvalidValue;
     WsPtrs p = ws_ptrs(ws, L);
     GemmArgs a = {};
     a.status = p.status;
@@ -1096,6 +1132,7 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
     a.route_q = plan.q;
     a.route_kb = plan.kb;
     a.route_groups = plan.groups;
+    a.row_boxes = boxes;
     static bool attr_done = false;
     if (!attr_done) {
         err = cudaFuncSetAttribute(k_grouped_gemm<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -1121,13 +1158,20 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
     const int K = mode == 0 ? s.H : s.F;
     const int n_out = mode == 0 ? s.F : s.H;
-    CUtensorMap tA0, tA1, tB;
+    CUtensorMap tA0, tA1, tB8;
+    RowMaps tB;
+    uint32_t boxes = 0;
     if (!make_tmap(&tA0, w0, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
-        !make_tmap(&tA1, w1, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
-        !(gather  ? make_tmap(&tB, act, (uint64_t)s.T, (uint64_t)K, 64, 1)
-          : pairs ? make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 8)
-                  : make_tmap(&tB, act, (uint64_t)P, (uint64_t)K, 64, 16)))
+        !make_tmap(&tA1, w1, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64))
         return cudaErrorInvalidValue;
+    if (gather) {
+        if (!make_tmap(&tB.m[0], act, (uint64_t)s.T, (uint64_t)K, 64, 1)) return cudaErrorInvalidValue;
+        boxes = 1u;
+    } else if (pairs) {
+        if (!make_tmap(&tB8, act, (uint64_t)P, (uint64_t)K, 64, 8)) return cudaErrorInvalidValue;
+    } else if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K))) {
+        return cudaErrorInvalidValue;
+    }
     WsPtrs p = ws_ptrs(ws, L);
     GemmArgs a = {};
     a.tile_map = p.tile_map;
@@ -1145,6 +1189,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.timeout_ns = timeout_ns;
     a.T = s.T;
     a.src_token = src_token;
+    a.row_boxes = boxes;
     static bool attr_done[5] = {false, false, false, false, false};
     cudaError_t err;
     if (pairs) {
@@ -1156,7 +1201,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
                 if (err != cudaSuccess) return err;
                 attr_done[3] = true;
             }
-            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB8, a);
         } else {
             if (!attr_done[4]) {
                 err = cudaFuncSetAttribute(k_grouped_gemm_pair<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1164,7 +1209,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
                 if (err != cudaSuccess) return err;
                 attr_done[4] = true;
             }
-            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB8, a);
         }
     } else if (gather) {
         if (!attr_done[2]) {

@@ -254,7 +254,7 @@ MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_stat
  *   - Shapes whose dispatch scratch exceeds MOE_STATIC_WS_BYTES are rejected
  *     with MOE_ERR_WORKSPACE (see moe_last_error_string).  The dispatch
  *     scratch is moe_workspace_bytes without the router buffers that large
- *     batches add (it grows with T*k/2048 and E).
+ *     batches add (it grows with T*k/1024 and E).
  *   - The first call on each device (with that device current) looks up the
  *     array's device address and zero-fills it on `stream`; make that first
  *     call before any stream capture begins.
