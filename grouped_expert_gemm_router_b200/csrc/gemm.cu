@@ -733,10 +733,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairMaxAStages = 12;
 constexpr int kPairMaxBStages = 8;
 
+// Rows [row0, row0 + n) (n a multiple of 8, <= 128) of the token matrix into
+// this CTA's shared memory from dst, completing on the leader's barrier;
+// boxes of 128, 64, 32, 16 and 8 rows (RowMaps with heights 8 << i), largest
+// first.
+__device__ __forceinline__ void tma_load_rows_pair(uint8_t *dst, const RowMaps &rm, uint32_t boxes, uint32_t bar,
+                                                   int kx, int row0, int n) {
+#pragma unroll
+    for (int i = kRowBoxes - 1; i >= 0; --i) {
+        const int h = 8 << i;
+        if (!((boxes >> i) & 1u)) continue;
+        while (n >= h) {
+            tma_load_2d_pair(dst, &rm.m[i], bar, kx, row0);
+            dst += h * kBRowBytes;
+            row0 += h;
+            n -= h;
+        }
+    }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+                        const __grid_constant__ RowMaps tmB, GemmArgs a) {
     static_assert(MODE == 0 || MODE == 1, "pairs run the expert GEMMs");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -796,7 +815,8 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA0);
         tma_prefetch_desc(&tmA1);
-        tma_prefetch_desc(&tmB);
+        for (int b = 0; b < kRowBoxes; ++b)
+            if ((a.row_boxes >> b) & 1u) tma_prefetch_desc(&tmB.m[b]);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -848,14 +868,16 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
                             tma_load_2d_pair(sa0 + kATile + kABox, &tmA1, bar, fx + 64, ky);
                         }
                     } else {
-                        // 8-row boxes of tile rows [rank * N/2, (rank + 1) * N/2); a
-                        // box never straddles the two row pieces (16-row aligned)
+                        // tile rows [rank * N/2, (rank + 1) * N/2): the part in
+                        // row piece 0 (tile rows [0, n0p)), then the part in
+                        // piece 1 (all lengths multiples of 8)
                         uint8_t *sb = ringB + stage * b_bytes;
-                        const int c_begin = (int)rank * half_rows;
-                        for (int c = c_begin; c < c_begin + half_rows; c += 8) {
-                            const int row = c < U.n0p ? U.p0s + c : U.p1s + (c - U.n0p);
-                            tma_load_2d_pair(sb + (c - c_begin) * kBRowBytes, &tmB, bar, kx, row);
-                        }
+                        const int cb = (int)rank * half_rows, ce = cb + half_rows;
+                        const int l0 = max(0, min(ce, U.n0p) - cb);
+                        const int c1 = max(cb, U.n0p);
+                        if (l0) tma_load_rows_pair(sb, tmB, a.row_boxes, bar, kx, U.p0s + cb, l0);
+                        if (ce > c1) tma_load_rows_pair(sb + l0 * kBRowBytes, tmB, a.row_boxes, bar, kx,
+                                                        U.p1s + (c1 - U.n0p), ce - c1);
                     }
                     if (++stage == nst) {
                         stage = 0;
@@ -1090,10 +1112,10 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
 
 // The token matrix with boxes of 16, 32, ... 256 rows; returns the mask of the
 // maps that could be encoded (bit 0 is required).
-uint32_t make_row_maps(RowMaps *rm, const void *ptr, uint64_t rows, uint64_t cols) {
+uint32_t make_row_maps(RowMaps *rm, const void *ptr, uint64_t rows, uint64_t cols, uint32_t min_rows = 16) {
     uint32_t boxes = 0;
     for (int i = 0; i < kRowBoxes; ++i)
-        if (make_tmap(&rm->m[i], ptr, rows, cols, 64, 16u << i)) boxes |= 1u << i;
+        if (make_tmap(&rm->m[i], ptr, rows, cols, 64, min_rows << i)) boxes |= 1u << i;
     return (boxes & 1u) ? boxes : 0u;
 }
 
@@ -1158,7 +1180,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
     const int K = mode == 0 ? s.H : s.F;
     const int n_out = mode == 0 ? s.F : s.H;
-    CUtensorMap tA0, tA1, tB8;
+    CUtensorMap tA0, tA1;
     RowMaps tB;
     uint32_t boxes = 0;
     if (!make_tmap(&tA0, w0, (uint64_t)s.E * K, (uint64_t)n_out, 64, 64) ||
@@ -1168,7 +1190,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
         if (!make_tmap(&tB.m[0], act, (uint64_t)s.T, (uint64_t)K, 64, 1)) return cudaErrorInvalidValue;
         boxes = 1u;
     } else if (pairs) {
-        if (!make_tmap(&tB8, act, (uint64_t)P, (uint64_t)K, 64, 8)) return cudaErrorInvalidValue;
+        if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K, 8))) return cudaErrorInvalidValue;
     } else if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K))) {
         return cudaErrorInvalidValue;
     }
@@ -1201,7 +1223,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
                 if (err != cudaSuccess) return err;
                 attr_done[3] = true;
             }
-            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB8, a);
+            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
         } else {
             if (!attr_done[4]) {
                 err = cudaFuncSetAttribute(k_grouped_gemm_pair<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1209,7 +1231,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
                 if (err != cudaSuccess) return err;
                 attr_done[4] = true;
             }
-            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB8, a);
+            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
         }
     } else if (gather) {
         if (!attr_done[2]) {
