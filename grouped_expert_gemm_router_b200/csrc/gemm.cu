@@ -78,7 +78,8 @@ constexpr uint32_t kBBox = 16 * kBRowBytes;    // TMA box: 16 rows x 64 K (2 KiB
 constexpr int kRowBoxes = 5;                   // token-tile boxes of 16, 32, 64, 128 and 256 rows
 constexpr uint32_t kCtrlBytes = 3072;
 constexpr uint32_t kSmemBytes = 226 * 1024;
-constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes) & ~1023u;
+constexpr uint32_t kEpiStageBytes = 512;      // per epilogue warp: one 8-row x 32-feature bf16 block
+constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes - 16 * kEpiStageBytes) & ~1023u;
 static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
               "three weight stages and three token stages of 256 rows must fit");
 constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
@@ -198,6 +199,78 @@ __device__ __forceinline__ int unit_row(const Unit &U, int c) {
     if (c < U.n0p) return c < U.p0l ? U.p0s + c : -1;
     const int c1 = c - U.n0p;
     return c1 < U.p1l ? U.p1s + c1 : -1;
+}
+
+// Stores a 32-feature x 16-row block of bf16 results held by one warp: lane l
+// holds feature fbase + l of unit rows c0 .. c0 + 15 as w[m] = (row 2m, row
+// 2m + 1).  Three butterfly exchanges (lanes ^1, ^2, ^4) leave each lane eight
+// consecutive features of unit rows c0 + (l & 7) and c0 + 8 + (l & 7), stored
+// as two 16-byte vectors: a warp writes the block with 2 store instructions
+// instead of 16, and the epilogue's time is set by its store instructions.
+__device__ __forceinline__ void store_block_32x16(const uint32_t (&w)[8], __nv_bfloat16 *out, int n_out, int fbase,
+                                                  const Unit &U, int c0) {
+    const int lane = threadIdx.x & 31;
+    const bool p = lane & 1, P = (lane >> 1) & 1, Q = (lane >> 2) & 1;
+    // (two rows, one feature) -> (one row, two features): x[m] = row 2m + p,
+    // features (l & ~1) and (l & ~1) + 1
+    uint32_t x[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, w[m], 1);
+        x[m] = p ? __byte_perm(o, w[m], 0x7632) : __byte_perm(w[m], o, 0x5410);
+    }
+    // keep m = 2t + P: y[t] = row 4t + 2P + p, features (l & ~3) .. + 3
+    uint32_t y[4][2];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const uint32_t keep = P ? x[2 * t + 1] : x[2 * t];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, P ? x[2 * t] : x[2 * t + 1], 2);
+        y[t][0] = P ? recv : keep;
+        y[t][1] = P ? keep : recv;
+    }
+    // keep t = 2s + Q: row 8s + (l & 7), features (l & ~7) .. + 7
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const uint32_t k0 = Q ? y[2 * s + 1][0] : y[2 * s][0], k1 = Q ? y[2 * s + 1][1] : y[2 * s][1];
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, Q ? y[2 * s][0] : y[2 * s + 1][0], 4);
+        const uint32_t r1 = __shfl_xor_sync(0xffffffffu, Q ? y[2 * s][1] : y[2 * s + 1][1], 4);
+        const int row = unit_row(U, c0 + 8 * s + (lane & 7));
+        if (row >= 0)
+            *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + (lane & ~7)) =
+                Q ? make_uint4(r0, r1, k0, k1) : make_uint4(k0, k1, r0, r1);
+    }
+}
+
+// Stores a 32-feature x 16-row block of bf16 results held by one warp in the
+// fragment layout of tmem_ld_frag16 (w[m] = the pair r[2m], r[2m + 1]: feature
+// 16 (m >> 2) + 8 (m & 1) + (t >> 2), rows 8 ((m >> 1) & 1) + 2 (t & 3) + {0, 1}
+// of unit rows c0 ..): per 8-row group one transposing stmatrix into the
+// warp's 512-byte staging block (rows of four 16-byte feature groups, the
+// group index XORed with bits 1-2 of the row so that neither side conflicts
+// on banks), then each lane reads back one 16-byte vector (8 features of one
+// row) and stores it.  Two 16-byte store instructions per warp for the
+// block instead of sixteen 2-byte ones.
+__device__ __forceinline__ void store_block_frag(const uint32_t (&w)[8], uint8_t *stg, __nv_bfloat16 *out, int n_out,
+                                                 int fbase, const Unit &U, int c0) {
+    const int lane = threadIdx.x & 31;
+    const int mi = lane >> 3, mj = lane & 7;  // stmatrix: row mj of matrix (feature group) mi
+    const int r = lane >> 2, c = lane & 3;    // read-back: row r, feature group c
+    const uint32_t st_addr = smem_u32(stg) + mj * 64 + 16 * (mi ^ ((mj >> 1) & 3));
+    const uint32_t ld_addr = smem_u32(stg) + r * 64 + 16 * (c ^ ((r >> 1) & 3));
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        stmatrix_x4_trans(st_addr, w[2 * k], w[2 * k + 1], w[4 + 2 * k], w[5 + 2 * k]);
+        __syncwarp();
+        const uint4 v = lds128(ld_addr);
+        __syncwarp();  // the block is rewritten by the next group
+        const int row = unit_row(U, c0 + 8 * k + r);
+        if (row >= 0) *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + 8 * c) = v;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 // Tensor memory is two halves of 256 columns.  A unit with <= 128 rows keeps
@@ -563,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;              // tensor-memory lane quarter of this warp
         const int sub = (warp - kEpiWarp0) >> 2;  // which 16-column chunks: sub, sub + kEpiSub, ...
         const int L = q * 32 + lane;         // feature within a 128-feature accumulator
+        uint8_t *stg = smem + kRingBytes + kCtrlBytes + (warp - kEpiWarp0) * kEpiStageBytes;
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         TmemPlan plan;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
@@ -591,8 +665,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (big) mbar_arrive(&tempty[1]);
                 }
             };
-            const int f0 = U.fx + L;
-            unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
             if (MODE == 2) {
                 // fp32 partial logits of K range U.fb: lane L of expert block c
                 // is expert c*128 + L; the groups' sums are added in order
@@ -630,16 +702,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // registers: store while holding the accumulator.
                 for (int c0 = sub * 16; c0 < U.N; c0 += 16 * kEpiSub) {
                     uint32_t r0[16], r1[16];
-                    tmem_ld16(t0 + (uint32_t)c0, r0);
-                    if (U.nacc == 2) tmem_ld16(t1 + (uint32_t)c0, r1);
+                    tmem_ld_frag16(t0 + (uint32_t)c0, r0);
+                    if (U.nacc == 2) tmem_ld_frag16(t1 + (uint32_t)c0, r1);
                     tmem_ld_wait();
+                    uint32_t w[8];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int row = unit_row(U, c0 + j);
-                        if (row < 0) continue;
-                        __nv_bfloat16 *dst = a.out + (size_t)row * a.n_out + f0;
-                        dst[0] = __float2bfloat16_rn(__uint_as_float(r0[j]));
-                        if (U.nacc == 2) dst[128] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+                    for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r0[2 * m], r0[2 * m + 1]);
+                    store_block_frag(w, stg, a.out, a.n_out, U.fx + q * 32, U, c0);
+                    if (U.nacc == 2) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r1[2 * m], r1[2 * m + 1]);
+                        store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
                     }
                 }
                 release();
@@ -658,8 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c0 = (sub + kEpiSub * i) * 16;
                 if (c0 < U.N) {
                     uint32_t r0[16], r1[16];
-                    tmem_ld16(t0 + (uint32_t)c0, r0);
-                    if (U.nacc == 2) tmem_ld16(t1 + (uint32_t)c0, r1);
+                    tmem_ld_frag16(t0 + (uint32_t)c0, r0);
+                    if (U.nacc == 2) tmem_ld_frag16(t1 + (uint32_t)c0, r1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
@@ -684,19 +757,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Hand the accumulator back to the MMA warp before the stores.
             release();
-            // Phase 2: the stores (one 2-byte value per row per thread; a warp
-            // covers 32 consecutive features, 64 contiguous bytes, per row).
+            // Phase 2: the stores, 16-byte vectors of eight features per row.
 #pragma unroll
             for (int i = 0; i < kHoldChunks; ++i) {
                 const int c0 = (sub + kEpiSub * i) * 16;
                 if (c0 < U.N) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int row = unit_row(U, c0 + j);
-                        if (row < 0) continue;
-                        unsigned short *dst = outp + (size_t)row * a.n_out + f0;
-                        dst[0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
-                        if (MODE == 1 && U.nacc == 2) dst[128] = (unsigned short)(hold[i][8 + j / 2] >> (16 * (j & 1)));
+                    for (int m = 0; m < 8; ++m) w[m] = hold[i][m];
+                    store_block_frag(w, stg, a.out, a.n_out, U.fx + q * 32, U, c0);
+                    if (MODE == 1 && U.nacc == 2) {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) w[m] = hold[i][8 + m];
+                        store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
                     }
                 }
             }
@@ -951,7 +1024,6 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
         // -------------------------------------------- epilogue (both CTAs) ----
         const int q = warp & 3;
         const int sub = (warp - kEpiWarp0) >> 2;
-        const int L = q * 32 + lane;
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         const uint32_t tempty_leader = mapa_shared(tempty, 0);
         TmemPlan plan;
@@ -978,9 +1050,8 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
                     if (big) mbar_arrive_cluster(tempty_leader + 8u);
                 }
             };
-            const int f0 = U.fx + 128 * (int)rank + L;
-            const bool inside = f0 < a.n_out;  // the last block may have no second half
-            unsigned short *outp = reinterpret_cast<unsigned short *>(a.out);
+            const int fb0 = U.fx + 128 * (int)rank + q * 32;  // this warp's first feature
+            const bool inside = fb0 < a.n_out;  // the last block may have no second half (warp-uniform)
             if (MODE == 1) {
                 // one accumulator of up to 256 columns: hold up to 4 chunks per warp
                 constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
@@ -1004,14 +1075,7 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
                     const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N && inside) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int row = unit_row(U, c0 + j);
-                            if (row >= 0)
-                                outp[(size_t)row * a.n_out + f0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
-                        }
-                    }
+                    if (c0 < U.N && inside) store_block_32x16(hold[i], a.out, a.n_out, fb0, U, c0);
                 }
             } else {
                 constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
@@ -1038,14 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
 #pragma unroll
                 for (int i = 0; i < kChunks; ++i) {
                     const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N && inside) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int row = unit_row(U, c0 + j);
-                            if (row >= 0)
-                                outp[(size_t)row * a.n_out + f0] = (unsigned short)(hold[i][j / 2] >> (16 * (j & 1)));
-                        }
-                    }
+                    if (c0 < U.N && inside) store_block_32x16(hold[i], a.out, a.n_out, fb0, U, c0);
                 }
             }
             plan.advance(big, h);
