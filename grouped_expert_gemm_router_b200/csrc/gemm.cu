@@ -31,7 +31,9 @@
 //   turn, so the epilogue of one overlaps the MMAs of the next; larger units
 //   take both halves.  The epilogue finishes the values into registers and
 //   hands the accumulator back before its global stores whenever the
-//   results fit in 64 registers.
+//   results fit in 64 registers; it stores 16-byte vectors of eight features
+//   of one row, transposed through a small per-warp staging block
+//   (stmatrix), since its time is set by its store instructions.
 // - Persistent, warp-specialised: warp 0 streams weight tiles and warp 2
 //   token tiles with TMA into two rings of shared-memory stages (mbarrier
 //   expect-tx), warp 1 issues tcgen05.mma from one thread and commits each
@@ -40,7 +42,8 @@
 //   turn) and write bf16 results.  The more epilogue warps, the sooner a
 //   finished accumulator is handed back to the MMA warp.
 // - Stage sizes follow the routing.  A weight stage holds the two 128-feature
-//   A tiles of 64 K rows; a token stage holds tile_rows rows of B, where
+//   A tiles of 64 K rows; a token stage holds tile_rows rows of B (loaded in
+//   TMA boxes of up to 256 rows, so that one producer thread keeps up), where
 //   tile_rows (chosen on the device by the schedule builder from the actual
 //   counts) is the largest padded row count of any expert, capped at 256.
 //   The token ring has four stages while that leaves room for four weight
@@ -54,7 +57,8 @@
 //   inside an expert so that the row tiles of one expert that share a weight
 //   tile run next to each other.  Nothing depends on the host knowing the
 //   routing, so the kernel is launched with one CTA per SM and can be
-//   captured in a CUDA graph.
+//   captured in a CUDA graph; the CTAs count the units on the device and
+//   only as many take work as balance the rounds.
 // - Every wait is bounded: on expiry the kernel records MOE_DEV_GEMM_TIMEOUT,
 //   tells the other roles to stop, lets in-flight copies and MMAs land, frees
 //   its tensor memory and returns.
@@ -347,7 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         total = nt * num_fb;
         trows = *a.tile_rows;  // the schedule's row cap
     }
-    if ((int)blockIdx.x >= total) return;  // uniform: this CTA has no work
+    // Balanced waves for the expert GEMMs: with R = ceil(total / grid) units
+    // for the busiest CTA, only ceil(total / R) CTAs take units (R or R - 1
+    // each), so the last round is not left to a few SMs while the rest idle
+    // (896 units on 148 SMs: 128 CTAs x 7 instead of 8 CTAs running a 7th).
+    const int rounds = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int stride = MODE == 2 || rounds == 0 ? (int)gridDim.x : (total + rounds - 1) / rounds;
+    if ((int)blockIdx.x >= total || (int)blockIdx.x >= stride) return;  // uniform: this CTA has no work
     // Two rings: weight stages (the A tiles of both accumulators; mode 2:
     // three weight planes per accumulator), streamed from HBM, and token
     // stages of trows rows (multiple of 16, <= 256).  Four token stages
@@ -417,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ph = 0;
         int issued_ph[kMaxBStages];
         for (int s = 0; s < kMaxBStages; ++s) issued_ph[s] = -1;
-        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        for (int u = blockIdx.x; u < total; u += stride) {
             Unit U;
             decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
             if (!U.valid) continue;
@@ -484,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             int issued_ph[kMaxAStages];
             for (int s = 0; s < kMaxAStages; ++s) issued_ph[s] = -1;
-            for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            for (int u = blockIdx.x; u < total; u += stride) {
                 Unit U;
                 decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
                 if (!U.valid) {
@@ -555,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             TmemPlan plan;
             const uint32_t baseA = smem_u32(smem), baseB = smem_u32(ringB);
             bool ok = true;
-            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < total && ok; u += stride) {
                 Unit U;
                 decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
                 if (!U.valid) continue;
@@ -639,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *stg = smem + kRingBytes + kCtrlBytes + (warp - kEpiWarp0) * kEpiStageBytes;
         const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         TmemPlan plan;
-        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        for (int u = blockIdx.x; u < total; u += stride) {
             Unit U;
             decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
             if (!U.valid) continue;
