@@ -17,9 +17,10 @@
 //   each) and HS = 32/ES lanes the hidden pairs.  Each thread holds a TB x EJ
 //   tile of sums, so every weight value it reads feeds TB multiply-adds; the
 //   warps' partial sums are added in warp order.
-// - Top-k: one warp per token, each lane holding ceil(E/32) candidates; k
-//   rounds of a warp max of the orderable logit and a warp min of the expert
-//   index among the lanes holding that maximum (redux.sync).
+// - Top-k: one warp per token, each lane holding ceil(E/32) candidates,
+//   sorted once per lane; k rounds of a warp max of the lanes' first orderable
+//   logit and a warp min of the expert index among the lanes holding that
+//   maximum (redux.sync), the winning lane dropping its first candidate.
 // - Logits computed elsewhere (given by the caller, or the tensor-core
 //   router's partial planes for large batches) go to k_topk: one warp per
 //   token loads its logits straight into registers, no CTA-wide staging.
