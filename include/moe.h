@@ -161,7 +161,11 @@ MOE_API moe_status moe_workspace_init(const moe_shape *shape, void *ws, void *st
  *                   logits to the lower index, NaN below every number;
  *   topk_w[t,j]   = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected.
  * With MOE_FLAG_LOGITS_IN, `logits` is read (w_router, bias unused).
- * Otherwise `logits` may be NULL (not written). */
+ * Otherwise `logits` may be NULL (not written).  From 2048 tokens the dot
+ * products run on the tensor cores against an exact three-way bf16 split of
+ * w_router, summed over at least eight fp32 partial accumulations in a fixed
+ * order (within 1e-5 relative of the fp32 definition; deterministic); the
+ * workspace then also holds the split weights and the partial logits. */
 MOE_API moe_status moe_route(const moe_shape *shape, const void *x, const float *w_router, const float *bias, float *logits,
                      int32_t *topk_idx, float *topk_w, void *ws, void *stream);
 
