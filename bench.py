@@ -51,6 +51,9 @@ def parse_args():
     p.add_argument("--config", type=int, default=2)
     p.add_argument("--alpha", type=float, default=None)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="time the headline workload only (default: every other workload too, on one GPU)")
+    p.add_argument("--per-config-steps", type=int, default=20)
     p.add_argument("--gemm-pairs", action="store_true",
                    help="run the grouped GEMMs on CTA pairs (MOE_FLAG_GEMM_PAIRS; off by default: slower on B200)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
@@ -203,7 +206,7 @@ def cpu_baseline(cfg, L, budget_s):
     t1 = run(1)
     S = int(max(1, min(cfg.T, budget_s / max(t1, 1e-6))))
     dt = run(S) if S > 1 else t1
-    return {"value": S / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    return {"value": S / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle", **host_info(),
             "sample": "first %d of the %d tokens of the same seeded batch through the whole oracle forward "
                       "(single-threaded C, fp64 accumulation); %.1f s" % (S, cfg.T, dt)}
 
@@ -239,7 +242,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_json(cfg, {"tokens_per_step": S}),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                             **host_info()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -284,8 +288,250 @@ def forward_launches(cfg):
     return router + dispatch + copy + 3
 
 
+def host_info():
+    """Host cores and CPU model (the CPU baseline's machine)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_nproc": os.cpu_count(), "host_cpu_model": model}
+
+
+class Bench:
+    """One process's device, stream, L2-cleaning buffers and clock sampler."""
+
+    def __init__(self, dev, world, local):
+        import torch
+        self.torch = torch
+        self.dev = dev
+        self.world = world
+        self.local = local
+        self.stream = torch.cuda.current_stream(dev)
+        self.flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush(self):
+        """Between timed steps: write 256 MiB (evicts everything), then read
+        another 256 MiB so the cache holds clean lines and the next step does
+        not pay for writing the first buffer back."""
+        self.flush_w.zero_()
+        self.flush_r.sum()
+
+    def barrier(self):
+        import torch.distributed as dist
+        if self.world > 1:
+            dist.barrier()
+        self.torch.cuda.synchronize(self.dev)
+
+    def upload(self, cfg, L, x_rank, flags=0):
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        torch, dev = self.torch, self.dev
+
+        def dev_bf16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=cfg.C > 0, flags=flags)
+        b = moe.alloc_buffers(shape, dev)
+        b.update(x=dev_bf16(x_rank), w_router=torch.from_numpy(L.w_router).to(dev),
+                 bias=None if L.bias is None else torch.from_numpy(L.bias).to(dev),
+                 w_gate=dev_bf16(L.w_gate), w_up=dev_bf16(L.w_up), w_down=dev_bf16(L.w_down))
+        return shape, b
+
+    def measure(self, cfg, shape, b, steps, warmup):
+        """Times one workload: (1) the entry points one by one with CUDA
+        events between them (per-kernel times), (2) moe_forward captured once
+        as a CUDA graph and replayed per step (the step time).  L2 is cleaned
+        before every step, outside the timed intervals."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        torch, dev, stream = self.torch, self.dev, self.stream
+        ws = b["ws"]
+        # moe_forward folds the row copy into the SwiGLU GEMM when given no
+        # x_perm buffer: the faster choice while the routed rows per expert are few
+        gather = cfg.T * cfg.k <= 32 * cfg.E
+        fwd_bufs = {**b, "x_perm": None} if gather else b
+
+        def step_events(ev):
+            ev[0].record(stream)
+            moe.moe_route_dispatch(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"],
+                                   b["expert_counts"], b["expert_offsets"], b["src_token"], b["dest_row"], ws, stream)
+            ev[1].record(stream)
+            if not gather:
+                moe.moe_gather(shape, b["x"], b["src_token"], b["x_perm"], ws, stream)
+            ev[2].record(stream)
+            if gather:
+                moe.moe_grouped_swiglu_gather(shape, b["x"], b["src_token"], b["w_gate"], b["w_up"], b["h"], ws,
+                                              stream)
+            else:
+                moe.moe_grouped_swiglu(shape, b["x_perm"], b["w_gate"], b["w_up"], b["h"], ws, stream)
+            ev[3].record(stream)
+            moe.moe_grouped_down(shape, b["h"], b["w_down"], b["y"], ws, stream)
+            ev[4].record(stream)
+            moe.moe_combine(shape, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
+            ev[5].record(stream)
+
+        wev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for _ in range(max(warmup, 3)):
+            self.flush()
+            step_events(wev)
+        torch.cuda.synchronize(dev)
+        status = moe.moe_read_status(ws, stream)
+        if status & ~moe.MOE_DEV_NAN_LOGIT:
+            raise RuntimeError("device status %#x after warm-up (%s)" % (status, cfg.name))
+
+        K = steps
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+        sampler = ClockSampler(gpu_id_for_smi(torch, self.local))
+        self.barrier()
+        sampler.start()
+        time.sleep(0.15)  # let the sampler take its first reading
+        wall0 = time.perf_counter()
+        for i in range(K):
+            self.flush()
+            step_events(evs[i])
+        self.barrier()
+        seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(K)])  # ms
+        eager_ms = float(seg.sum(axis=1).sum())
+        status |= moe.moe_read_status(ws, stream)
+
+        args_c = moe.forward_args(fwd_bufs)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+            moe.moe_forward(shape, b, ws, args=args_c)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(3):
+            self.flush()
+            g.replay()
+        self.barrier()
+        for i in range(K):
+            self.flush()
+            gev[i][0].record(stream)
+            g.replay()
+            gev[i][1].record(stream)
+        self.barrier()
+        wall = time.perf_counter() - wall0
+        clocks = sampler.stop()
+        total_ms = float(np.sum([a.elapsed_time(c) for a, c in gev]))
+        del g
+        total_ms, eager_ms = max_over_ranks([total_ms, eager_ms], dev)
+        status |= moe.moe_read_status(ws, stream)
+        return {"total_ms": total_ms, "eager_ms": eager_ms, "kmean_s": seg.mean(axis=0) * 1e-3, "gather": gather,
+                "fwd_bufs": fwd_bufs, "clocks": clocks, "status": status, "wall": wall,
+                "counts": b["expert_counts"].cpu().numpy()}
+
+    def e2e(self, cfg, shape, b, x_rank, fwd_bufs, steps):
+        """The same metric end to end: pinned-host tokens copied in, the layer,
+        the output copied back to pinned host memory, every step."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        torch, dev, stream = self.torch, self.dev, self.stream
+        x_host = torch.from_numpy(np.ascontiguousarray(x_rank).view(np.int16)).view(torch.bfloat16).pin_memory()
+        out_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+        args_e = moe.forward_args(fwd_bufs)
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(-3, steps):
+            self.flush()
+            if i >= 0:
+                eev[i][0].record(stream)
+            b["x"].copy_(x_host, non_blocking=True)
+            moe.moe_forward(shape, b, b["ws"], stream, args=args_e)
+            out_host.copy_(b["out"], non_blocking=True)
+            if i >= 0:
+                eev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = float(np.sum([a.elapsed_time(c) for a, c in eev]))
+        (e2e_ms,) = max_over_ranks([e2e_ms], dev)
+        return e2e_ms
+
+
+def summarize(cfg, m, steps, world, peaks, peak_src):
+    """Throughput, per-kernel times and roofline fractions of one measured
+    workload."""
+    counts = m["counts"]
+    work = algorithmic_work(cfg, counts)
+    kmean = m["kmean_s"]
+    names = ["route_dispatch", "row_copy", "grouped_swiglu", "grouped_down", "combine"]  # row_copy: 0 if gathered
+
+    def kernel_roof(bytes_, flops, t):
+        t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        if t_hbm >= t_tc:
+            a = bytes_ / t / 1e9
+            return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": a / peaks["hbm_gbs"]}
+        a = flops / t / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": a / peaks["bf16_tflops"]}
+
+    # dominant kernel: the fused gate+up SwiGLU grouped GEMM
+    roof = kernel_roof(work["swiglu_bytes"], work["swiglu_flops"], kmean[2])
+    roof.update({"traffic": dram_traffic(cfg),
+                 "kernel": "k_grouped_gemm<0> (moe_grouped_swiglu, or its row-gathering form)",
+                 "algorithmic_bytes": work["swiglu_bytes"], "algorithmic_flops": work["swiglu_flops"],
+                 "peak_source": peak_src})
+    down = kernel_roof(work["down_bytes"], work["down_flops"], kmean[3])
+    layer_hbm = work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    layer_tc = work["layer_flops"] / (peaks["bf16_tflops"] * 1e12)
+    layer_t = max(layer_hbm, layer_tc)
+    kernels = {nm + "_us": t * 1e6 for nm, t in zip(names, kmean)}
+    kernels["grouped_swiglu_GBps"] = work["swiglu_bytes"] / kmean[2] / 1e9
+    kernels["grouped_swiglu_TFLOPs"] = work["swiglu_flops"] / kmean[2] / 1e12
+    kernels["grouped_down_GBps"] = work["down_bytes"] / kmean[3] / 1e9
+    kernels["grouped_down_TFLOPs"] = work["down_flops"] / kmean[3] / 1e12
+    kernels["grouped_down_roofline"] = {k: down[k] for k in ("bound", "frac", "unit", "achieved")}
+    kernels["combine_GBps"] = work["combine_bytes"] / kmean[4] / 1e9
+    kernels["combine_hbm_frac"] = kernels["combine_GBps"] / peaks["hbm_gbs"]
+    if kmean[1] > 0 and not m["gather"]:
+        R = cfg.T * cfg.k
+        kernels["row_copy_GBps"] = (cfg.T * cfg.H * 2 + R * cfg.H * 2) / kmean[1] / 1e9
+        kernels["row_copy_hbm_frac"] = kernels["row_copy_GBps"] / peaks["hbm_gbs"]
+    kernels["swiglu_gathers_rows"] = bool(m["gather"])
+    kernels["route_dispatch_TFLOPs_fp32"] = work["route_flops"] / kmean[0] / 1e12
+    ms = m["total_ms"] / steps
+    return {
+        "value": whole_job_rate(cfg.T, steps, world, m["total_ms"]), "ms_per_step": ms,
+        "roofline": roof,
+        "layer_roofline": {"frac": layer_t / (ms * 1e-3), "roofline_us": layer_t * 1e6,
+                           "bound": "hbm" if layer_hbm >= layer_tc else "tensor"},
+        "kernels": kernels,
+        "eager_entry_points_ms_per_step": m["eager_ms"] / steps,
+        "clocks": m["clocks"],
+        "routing": routing_stats(counts, cfg.C),
+        "device_status": m["status"],
+        "wall_s_timed_region": m["wall"],
+    }
+
+
+def per_config_workloads(head):
+    """Every workload other than the headline one: configs 1-4 and config 5
+    at each skew alpha."""
+    import synth
+    out = []
+    for cid in sorted(synth.CONFIGS):
+        alphas = synth.CONFIG5_ALPHAS if cid == 5 else (None,)
+        for a in alphas:
+            cfg = synth.CONFIGS[cid] if a is None else synth.CONFIGS[cid].with_(alpha=a)
+            if (cfg.name, cfg.alpha) != (head.name, head.alpha):
+                out.append(cfg)
+    return out
+
+
+def workload_name(cfg):
+    return config_json(cfg)["workload"]
+
+
 def run_ours(args):
-    import numpy as np
+    import gc
+
     import torch
     import torch.distributed as dist
 
@@ -306,189 +552,64 @@ def run_ours(args):
     L = synth.make_layer(cfg)
     x_rank = replica_tokens(cfg, rank, L)  # each replica its own tokens
     log("rank %d: generated %s in %.1f s" % (rank, cfg.name, time.time() - t0))
-
-    def dev_bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=cfg.C > 0,
-                           flags=moe.MOE_FLAG_GEMM_PAIRS if args.gemm_pairs else 0)
-    b = moe.alloc_buffers(shape, dev)
-    b.update(x=dev_bf16(x_rank), w_router=torch.from_numpy(L.w_router).to(dev),
-             bias=None if L.bias is None else torch.from_numpy(L.bias).to(dev),
-             w_gate=dev_bf16(L.w_gate), w_up=dev_bf16(L.w_up), w_down=dev_bf16(L.w_down))
-    ws = b["ws"]
-    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    class _Flush:
-        """Between timed steps: write 256 MiB (evicts everything), then read
-        another 256 MiB so the cache holds clean lines and the next step does
-        not pay for writing the first buffer back."""
-
-        def zero_(self):
-            flush_w.zero_()
-            flush_r.sum()
-
-    flush = _Flush()
-
-    # moe_forward folds the row copy into the SwiGLU GEMM when given no x_perm
-    # buffer: the faster choice while the routed rows per expert are few
-    gather = cfg.T * cfg.k <= 32 * cfg.E
-    fwd_bufs = {**b, "x_perm": None} if gather else b
-
-    def step_events(ev):
-        ev[0].record(stream)
-        moe.moe_route_dispatch(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"],
-                               b["expert_counts"], b["expert_offsets"], b["src_token"], b["dest_row"], ws, stream)
-        ev[1].record(stream)
-        if not gather:
-            moe.moe_gather(shape, b["x"], b["src_token"], b["x_perm"], ws, stream)
-        ev[2].record(stream)
-        if gather:
-            moe.moe_grouped_swiglu_gather(shape, b["x"], b["src_token"], b["w_gate"], b["w_up"], b["h"], ws, stream)
-        else:
-            moe.moe_grouped_swiglu(shape, b["x_perm"], b["w_gate"], b["w_up"], b["h"], ws, stream)
-        ev[3].record(stream)
-        moe.moe_grouped_down(shape, b["h"], b["w_down"], b["y"], ws, stream)
-        ev[4].record(stream)
-        moe.moe_combine(shape, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
-        ev[5].record(stream)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-
-    # warm-up
-    wev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        step_events(wev)
-    torch.cuda.synchronize(dev)
-    status = moe.moe_read_status(ws, stream)
-    if status & ~moe.MOE_DEV_NAN_LOGIT:
-        raise RuntimeError("device status %#x after warm-up" % status)
-
-    # timed region 1: the entry points one by one (per-kernel breakdown)
+    bench = Bench(dev, world, local)
+    flags = moe.MOE_FLAG_GEMM_PAIRS if args.gemm_pairs else 0
+    shape, b = bench.upload(cfg, L, x_rank, flags)
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    sampler = ClockSampler(gpu_id_for_smi(torch, local))
-    barrier()
-    sampler.start()
-    time.sleep(0.15)  # let the sampler take its first reading
-    wall0 = time.perf_counter()
-    for i in range(K):
-        flush.zero_()
-        step_events(evs[i])
-    barrier()
-    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(K)])  # ms
-    eager_ms = float(seg.sum(axis=1).sum())
-    status = moe.moe_read_status(ws, stream)
-
-    # timed region 2 (the headline): the whole layer, moe_forward, captured
-    # once in a CUDA graph and replayed K times, L2 cleaned before each replay
-    args_c = moe.forward_args(fwd_bufs)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
-        moe.moe_forward(shape, b, ws, args=args_c)
-    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for i in range(3):
-        flush.zero_()
-        g.replay()
-    barrier()
-    for i in range(K):
-        flush.zero_()
-        gev[i][0].record(stream)
-        g.replay()
-        gev[i][1].record(stream)
-    barrier()
-    wall = time.perf_counter() - wall0
-    clocks = sampler.stop()
-    total_ms = float(np.sum([a.elapsed_time(c) for a, c in gev]))
-    del g
-    total_ms, eager_ms = max_over_ranks([total_ms, eager_ms], dev)
-    status |= moe.moe_read_status(ws, stream)
-
-    counts = b["expert_counts"].cpu().numpy()
-    work = algorithmic_work(cfg, counts)
+    m = bench.measure(cfg, shape, b, K, args.warmup)
+    e2e_ms = bench.e2e(cfg, shape, b, x_rank, m["fwd_bufs"], K)
     peaks, peak_src = load_peaks()
-    kmean = seg.mean(axis=0) * 1e-3  # s per launch
-    names = ["route_dispatch", "row_copy", "grouped_swiglu", "grouped_down", "combine"]  # row_copy: 0 if gathered
-
-    # end to end: pinned host tokens in, layer, host result out, each step
-    x_host = torch.from_numpy(np.ascontiguousarray(x_rank).view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
-    args_e = moe.forward_args(fwd_bufs)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for i in range(-3, K):
-        flush.zero_()
-        if i >= 0:
-            eev[i][0].record(stream)
-        b["x"].copy_(x_host, non_blocking=True)
-        moe.moe_forward(shape, b, ws, stream, args=args_e)
-        out_host.copy_(b["out"], non_blocking=True)
-        if i >= 0:
-            eev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = float(np.sum([a.elapsed_time(c) for a, c in eev]))
-    (e2e_ms,) = max_over_ranks([e2e_ms], dev)
 
     result = None
     if rank == 0:
-        value = whole_job_rate(cfg.T, K, world, total_ms)
-        # dominant kernel: the fused gate+up SwiGLU grouped GEMM
-        t_sw = kmean[2]
-        t_hbm = work["swiglu_bytes"] / (peaks["hbm_gbs"] * 1e9)
-        t_tc = work["swiglu_flops"] / (peaks["bf16_tflops"] * 1e12)
-        if t_hbm >= t_tc:
-            achieved = work["swiglu_bytes"] / t_sw / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"]}
-        else:
-            achieved = work["swiglu_flops"] / t_sw / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"]}
-        roof.update({"traffic": dram_traffic(cfg), "kernel": "k_grouped_gemm<0> (moe_grouped_swiglu, or its row-gathering form)",
-                     "algorithmic_bytes": work["swiglu_bytes"], "algorithmic_flops": work["swiglu_flops"],
-                     "peak_source": peak_src})
-        layer_t = max(work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9),
-                      work["layer_flops"] / (peaks["bf16_tflops"] * 1e12))
-        kernels = {}
-        for nm, t in zip(names, kmean):
-            kernels[nm + "_us"] = t * 1e6
-        kernels["grouped_swiglu_GBps"] = work["swiglu_bytes"] / kmean[2] / 1e9
-        kernels["grouped_swiglu_TFLOPs"] = work["swiglu_flops"] / kmean[2] / 1e12
-        kernels["grouped_down_GBps"] = work["down_bytes"] / kmean[3] / 1e9
-        kernels["grouped_down_TFLOPs"] = work["down_flops"] / kmean[3] / 1e12
-        kernels["grouped_down_hbm_frac"] = work["down_bytes"] / kmean[3] / 1e9 / peaks["hbm_gbs"]
-        kernels["combine_GBps"] = work["combine_bytes"] / kmean[4] / 1e9
-        kernels["swiglu_gathers_rows"] = bool(gather)
-        kernels["route_dispatch_TFLOPs_fp32"] = work["route_flops"] / kmean[0] / 1e12
+        s = summarize(cfg, m, K, world, peaks, peak_src)
         result = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": s["value"], "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": s["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu",
                                         "gemm": "cta pairs" if args.gemm_pairs else "single cta"}),
-            "roofline": roof,
-            "layer_roofline": {"frac": layer_t / (total_ms * 1e-3 / K), "roofline_us": layer_t * 1e6,
-                               "bound": "hbm" if work["layer_bytes"] / (peaks["hbm_gbs"] * 1e9)
-                               >= work["layer_flops"] / (peaks["bf16_tflops"] * 1e12) else "tensor"},
-            "kernels": kernels,
-            "eager_entry_points_ms_per_step": eager_ms / K,
+            "roofline": s["roofline"],
+            "layer_roofline": s["layer_roofline"],
+            "kernels": s["kernels"],
+            "eager_entry_points_ms_per_step": s["eager_entry_points_ms_per_step"],
             "e2e": {"value": whole_job_rate(cfg.T, K, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
             "gpu_launches": forward_launches(cfg) * K,
-            "clocks": clocks,
-            "routing": routing_stats(counts, cfg.C),
-            "device_status": status,
-            "wall_s_timed_region": wall,
+            "clocks": s["clocks"],
+            "routing": s["routing"],
+            "device_status": s["device_status"],
+            "wall_s_timed_region": s["wall_s_timed_region"],
         }
+    del b
+    gc.collect()
+    torch.cuda.empty_cache()
+
+    # every other workload, same protocol (one GPU only: replicas time the
+    # headline workload alone)
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = {}
+        for pc in per_config_workloads(cfg):
+            t0 = time.time()
+            Lp = synth.make_layer(pc)
+            shp, bp = bench.upload(pc, Lp, Lp.x, flags)
+            kp = min(K, args.per_config_steps)
+            mp = bench.measure(pc, shp, bp, kp, min(args.warmup, 5))
+            sp = summarize(pc, mp, kp, world, peaks, peak_src)
+            sp.update({"steps": kp, "config": config_json(pc), "gpu_launches": forward_launches(pc) * kp})
+            per_config[workload_name(pc)] = sp
+            log("per-config %s: %.0f tokens/s (%.1f s)" % (pc.name, sp["value"], time.time() - t0))
+            del bp, Lp
+            gc.collect()
+            torch.cuda.empty_cache()
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
+        if per_config is not None:
+            result["per_config"] = per_config
         if not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(cfg, L, args.cpu_budget_s)
         print(json.dumps(result), flush=True)
