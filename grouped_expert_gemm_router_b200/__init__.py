@@ -24,6 +24,7 @@ MOE_FLAG_CAPACITY = 0x1
 MOE_FLAG_LOGITS_IN = 0x2
 MOE_FLAG_GEMM_PAIRS = 0x4
 MOE_FLAG_TEST_STALL_SCAN = 0x40000000
+MOE_FLAG_TEST_STALL_GEMM = 0x20000000
 
 # Every symbol include/moe.h declares (the CPU tests check the library exports each).
 ABI_FUNCTIONS = (

@@ -116,6 +116,7 @@ struct GemmArgs {
     int route_kb;       // K blocks per range
     int route_groups;   // accumulators per unit: route_groups * nacc * route_rows <= 512 columns
     uint32_t row_boxes; // bit i: RowMaps::m[i] (boxes of 16 << i rows) is valid; bit 0 always
+    int stall_first_stage;  // test hook: CTA 0's token producer never loads its first stage
 };
 
 // Tensor maps of the token matrix (B operand) with boxes of 16 << i rows x 64
@@ -514,6 +515,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, a.timeout_ns, s_abort)) {
                         ok = false;
                         break;
+                    }
+                    if (!is_a && a.stall_first_stage && blockIdx.x == 0 && u == (int)blockIdx.x && kb == kb0) {
+                        // test hook: this stage is never loaded (no copy is in
+                        // flight for it), so the MMA issuer's wait expires
+                        if (++stage == nst) {
+                            stage = 0;
+                            ph ^= 1u;
+                        }
+                        continue;
                     }
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     const int ky = krow + kb * kBK, kx = kb * kBK;
@@ -1279,6 +1289,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.T = s.T;
     a.src_token = src_token;
     a.row_boxes = boxes;
+    a.stall_first_stage = (mode == 0 && !gather && (s.flags & MOE_FLAG_TEST_STALL_GEMM)) ? 1 : 0;
     static bool attr_done[5] = {false, false, false, false, false};
     cudaError_t err;
     if (pairs) {

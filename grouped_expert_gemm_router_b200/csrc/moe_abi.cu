@@ -33,7 +33,8 @@ namespace {
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 thread_local char g_last_error[160] = "no error";
 
-constexpr uint32_t kKnownFlags = MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FLAG_GEMM_PAIRS | MOE_FLAG_TEST_STALL_SCAN;
+constexpr uint32_t kKnownFlags =
+    MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FLAG_GEMM_PAIRS | MOE_FLAG_TEST_STALL_SCAN | MOE_FLAG_TEST_STALL_GEMM;
 
 bool aligned(const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
 

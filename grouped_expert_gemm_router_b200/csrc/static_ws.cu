@@ -14,9 +14,12 @@
 // cannot use the array's name as a device address (it names a host-side
 // stand-in), so the first call on each device, with that device current,
 // looks its address up with cudaGetSymbolAddress and zero-fills it; later
-// calls reuse the cached address.  Every call shares the array and leaves
-// its contents behind, so each call clears what must start at zero (the
-// look-back flags and block ticket) before its kernels run.
+// calls reuse the cached address.  The cache is keyed by the device's current
+// context, so a context that was torn down and recreated (cudaDeviceReset)
+// gets a fresh look-up and zero-fill instead of a stale address.  Every call
+// shares the array and leaves its contents behind, so each call clears what
+// must start at zero (the look-back flags and block ticket) before its
+// kernels run.
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -37,17 +40,40 @@ static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void *g_static_ptr[kMaxDevices] = {nullptr};
+void *g_static_ctx[kMaxDevices] = {nullptr};  // context the cached address belongs to
 
-// Device address of g_static_ws on the current device (set-up on first use).
+// The current context of the calling thread (a CUcontext), through the
+// driver entry point, so the library needs no link-time driver dependency.
+void *current_context() {
+    using Fn = int (*)(void **);
+    static Fn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<Fn>(p);
+        tried = true;
+    }
+    void *ctx = nullptr;
+    if (fn && fn(&ctx) != 0) ctx = nullptr;
+    return ctx;
+}
+
+// Device address of g_static_ws on the current device (set-up on the first
+// use in each context: look-up and zero-fill).
 cudaError_t static_ws_address(int dev, cudaStream_t stream, void **out) {
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_static_ptr[dev] == nullptr) {
+    void *ctx = current_context();
+    if (g_static_ptr[dev] == nullptr || g_static_ctx[dev] != ctx) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess) return e;
         e = cudaMemsetAsync(p, 0, kStaticWsBytes, stream);
         if (e != cudaSuccess) return e;
         g_static_ptr[dev] = p;
+        g_static_ctx[dev] = ctx;
     }
     *out = g_static_ptr[dev];
     return cudaSuccess;
@@ -68,6 +94,9 @@ extern "C" MOE_API moe_status moe_permute_static(const moe_shape *s, const void 
                                                  void *stream) {
     moe_status st = moe_internal_check_shape(s);
     if (st != MOE_OK) return st;
+    // The test hook that stalls the histogram's look-back would leave
+    // outputs this entry point has no way to flag: refused here.
+    if (s->flags & MOE_FLAG_TEST_STALL_SCAN) return MOE_ERR_INVALID_ARG;
     auto al = [](const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; };
     if (!al(x, 16) || !al(x_perm, 16) || !al(topk_idx, 4) || !al(expert_counts, 4) || !al(expert_offsets, 4) ||
         !al(src_token, 4) || !al(dest_row, 4))

@@ -90,6 +90,13 @@ typedef enum {
                                    block never publishes, so its successor's
                                    bounded wait expires and reports
                                    MOE_DEV_SCAN_TIMEOUT */
+#define MOE_FLAG_TEST_STALL_GEMM 0x20000000u /* test only: in moe_grouped_swiglu
+                                   (tiled form) the token-tile producer of
+                                   CTA 0 never loads its first stage, so the
+                                   MMA issuer's bounded wait expires; the
+                                   kernel reports MOE_DEV_GEMM_TIMEOUT, lets
+                                   its copies in flight land, frees its
+                                   tensor memory and returns */
 
 typedef struct {
     int32_t T;      /* tokens */
@@ -261,14 +268,18 @@ MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_stat
  *     batches add (it grows with T*k/1024 and E).
  *   - The first call on each device (with that device current) looks up the
  *     array's device address and zero-fills it on `stream`; make that first
- *     call before any stream capture begins.
+ *     call before any stream capture begins.  (A context that was torn
+ *     down and recreated gets the same set-up again on its first call.)
  *   - All calls share the array and it keeps the last call's contents; each
  *     call clears what must start at zero.  Calls that overlap on the GPU
  *     (other streams, other host threads) race on the array: order them.
  *   - The GEMM schedule it builds stays inside the array, so the grouped GEMM
- *     entry points still need the workspace form (moe_permute).  Device-side
- *     faults are not reported through a status word: a pair that cannot be
- *     placed gets dest_row = -1. */
+ *     entry points still need the workspace form (moe_permute).
+ *   - Device-side faults cannot be reported: there is no caller workspace to
+ *     hold the status word.  After one (an expert index outside [0, E), an
+ *     expired look-back wait) the outputs are undefined; a pair that cannot
+ *     be placed gets dest_row = -1.  MOE_FLAG_TEST_STALL_SCAN is refused
+ *     with MOE_ERR_INVALID_ARG. */
 #define MOE_STATIC_WS_BYTES (1u << 20)
 MOE_API moe_status moe_permute_static(const moe_shape *shape, const void *x, const int32_t *topk_idx,
                                       int32_t *expert_counts, int32_t *expert_offsets, int32_t *src_token,

@@ -128,3 +128,17 @@ def test_tile_bound_holds_for_adversarial_counts():
                 else:
                     tiles += _pack_expert([(0, n[e])])
             assert tiles <= 2 * E + P // 256 + 1
+
+
+def test_static_dispatch_refuses_the_scan_stall_hook(lib):
+    # the no-workspace dispatch has no status word to report the stalled
+    # look-back through, so it refuses the test hook before any CUDA call
+    s = moe.make_shape(64, 128, 256, 8, 2, flags=moe.MOE_FLAG_TEST_STALL_SCAN)
+    rc = lib.moe_permute_static(ctypes.byref(s), None, None, None, None, None, None, None, None)
+    assert rc == 1  # MOE_ERR_INVALID_ARG
+
+
+def test_test_hook_flags_are_known(lib):
+    for f in (moe.MOE_FLAG_TEST_STALL_SCAN, moe.MOE_FLAG_TEST_STALL_GEMM):
+        s = moe.make_shape(64, 128, 256, 8, 2, flags=f)
+        assert lib.moe_workspace_bytes(ctypes.byref(s)) > 0

@@ -289,6 +289,36 @@ def test_scan_wait_expires_and_reports(orc):
     assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
 
 
+def test_gemm_wait_expires_and_reports(orc):
+    """The SwiGLU GEMM's token producer in CTA 0 never loads its first stage:
+    the MMA issuer's bounded wait runs out, the kernel records the timeout,
+    lets the copies it issued land, frees its tensor memory and returns; the
+    context stays usable and a clean layer in it matches the oracle."""
+    cfg = CASES["two_tiles_E4_k2"]
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    shape = shape_of(cfg, flags=moe.MOE_FLAG_TEST_STALL_GEMM)
+    b = dl.bufs(shape)
+    moe.moe_set_wait_timeout_ns(50_000_000)
+    try:
+        moe.moe_route(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"], b["ws"])
+        moe.moe_permute(shape, b["x"], b["topk_idx"], b["expert_counts"], b["expert_offsets"], b["src_token"],
+                        b["dest_row"], b["x_perm"], b["ws"])
+        assert moe.moe_read_status(b["ws"], clear=True) == 0
+        moe.moe_grouped_swiglu(shape, b["x_perm"], b["w_gate"], b["w_up"], b["h"], b["ws"])
+        st = moe.moe_read_status(b["ws"], clear=True)
+    finally:
+        moe.moe_set_wait_timeout_ns(1_000_000_000)
+    assert st == moe.MOE_DEV_GEMM_TIMEOUT, hex(st)
+    ok = shape_of(cfg)
+    r = host(run_steps(dl, ok), ok)
+    assert r["status"] == 0
+    o = _oracle_full(orc, L, cfg, r["logits"])
+    filled = o["d"]["src_token"] >= 0
+    assert_close_bf16(r["h"][filled], o["h"][filled], "h after a GEMM timeout")
+    assert_close_bf16(r["out"], o["out"], "out after a GEMM timeout")
+
+
 @pytest.mark.parametrize("name", ["two_tiles_E4_k2", "skew_E8_k3_H384", "capacity_E16_k4_C24", "E1_dense"])
 def test_gemm_pairs_match_single_cta(orc, name):
     """MOE_FLAG_GEMM_PAIRS runs both grouped GEMMs on pairs of CTAs sharing
