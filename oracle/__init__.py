@@ -48,6 +48,15 @@ def _declare(lib):
     lib.oracle_forward.argtypes = [i32] * 8 + [vp] * 21
     lib.oracle_forward.restype = i32
     lib.oracle_token_outputs.argtypes = [i32, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_fp8_scale.argtypes = [ctypes.c_float]
+    lib.oracle_fp8_scale.restype = ctypes.c_float
+    lib.oracle_quantize_rows.argtypes = [i32, i32, vp, vp, vp]
+    lib.oracle_quantize_weights.argtypes = [i32, i32, i32, vp, vp, vp]
+    lib.oracle_dequantize.argtypes = [i64, i32, vp, vp, vp]
     return lib
 
 
@@ -190,3 +199,46 @@ class Oracle:
                                       _p(_c(w_gate, np.uint16)), _p(_c(w_up, np.uint16)),
                                       _p(_c(w_down, np.uint16)), _p(out))
         return out
+
+    # ---- fp8 (e4m3) variant: codes are uint8, scales float32 powers of two ----
+
+    def e4m3_decode(self, q: int) -> float:
+        return float(self.lib.oracle_e4m3_decode(int(q)))
+
+    def e4m3_encode(self, v: float) -> int:
+        return int(self.lib.oracle_e4m3_encode(float(v)))
+
+    def fp8_scale(self, amax: float) -> float:
+        return float(self.lib.oracle_fp8_scale(float(amax)))
+
+    def quantize_rows(self, v):
+        """bf16 [rows, n] -> (codes [rows, n] uint8, scales [rows] float32)."""
+        v = _c(v, np.uint16)
+        rows, n = v.shape
+        q = np.empty((rows, n), np.uint8)
+        s = np.empty(rows, np.float32)
+        self.lib.oracle_quantize_rows(rows, n, _p(v), _p(q), _p(s))
+        return q, s
+
+    def quantize_weights(self, w):
+        """bf16 [E, K, N] -> (codes [E, N, K] uint8, scales [E, N] float32)."""
+        w = _c(w, np.uint16)
+        E, K, N = w.shape
+        q = np.empty((E, N, K), np.uint8)
+        s = np.empty((E, N), np.float32)
+        self.lib.oracle_quantize_weights(E, K, N, _p(w), _p(q), _p(s))
+        return q, s
+
+    def dequantize(self, q, scale):
+        """codes with one scale per last-axis vector -> bf16 bits of the same shape."""
+        q = _c(q, np.uint8)
+        scale = _c(scale, np.float32)
+        out = np.empty(q.shape, np.uint16)
+        group = q.shape[-1] if q.ndim else 1
+        self.lib.oracle_dequantize(q.size, group, _p(q), _p(scale), _p(out))
+        return out
+
+    def dequantize_weights(self, q, scale):
+        """codes [E, N, K] + scales [E, N] -> bf16 weights [E, K, N] (the layout the
+        bf16 expert functions take)."""
+        return np.ascontiguousarray(self.dequantize(q, scale).transpose(0, 2, 1))

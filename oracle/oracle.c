@@ -321,3 +321,104 @@ void oracle_token_outputs(int ntok, const int32_t *tokens, int H, int F, int k, 
     free(yrows);
     free(hrow);
 }
+
+/* ------------------------------------------- fp8 expert weights (e4m3) ---- */
+
+/* The fp8 variant of the expert GEMMs ("TEMPO" verdict page, arXiv
+ * 2608.13057, referee report summary: the per-expert cost law is measured on
+ * an fp8 grouped GEMM, whose flat regime streams the expert's weights from
+ * HBM; 8-bit weights halve those bytes).  The pages fix neither the 8-bit
+ * format nor the scaling, so this variant takes the plainest reading:
+ *
+ *   - values are OCP 8-bit floats of the E4M3 kind: a sign bit, 4 exponent
+ *     bits with bias 7 and 3 mantissa bits; exponent field 0 holds the
+ *     subnormals m * 2^-9; there is no infinity, and S.1111.111 is NaN, so
+ *     the largest finite magnitude is 1.75 * 2^8 = 448;
+ *   - a vector is stored as codes q_i and one power-of-two scale s: the
+ *     value is decode(q_i) * s.  s = 2^(c - 8) with c the smallest integer
+ *     such that max_i |v_i| <= 2^c (s = 1 for an all-zero vector), so every
+ *     |v_i| / s <= 256 stays below 448 and v_i / s is exact;
+ *     q_i = encode(v_i / s), rounding to the nearest code, ties to the even
+ *     code;
+ *   - expert weights get one scale per expert and output column (the vector
+ *     is the column over the reduction dimension) and are stored with the
+ *     reduction dimension contiguous: Wq[e][n][k];
+ *   - activations (the tokens entering the SwiGLU projection, the SwiGLU
+ *     output entering the down projection) get one scale per row;
+ *   - since a code times a power of two has at most 4 significant bits, a
+ *     dequantized value is exactly a bf16 value: the fp8 layer is the same
+ *     five steps, run on dequantized weights and activations. */
+
+double oracle_e4m3_decode(uint8_t q) {
+    const int sign = q >> 7, ex = (q >> 3) & 15, man = q & 7;
+    if (ex == 15 && man == 7) return NAN;
+    const double mag = ex == 0 ? ldexp((double)man, -9) : ldexp(1.0 + man / 8.0, ex - 7);
+    return sign ? -mag : mag;
+}
+
+/* Nearest code to v (ties to the even code), |v| above 448 saturating to the
+ * largest finite code; NaN in, NaN code out. */
+uint8_t oracle_e4m3_encode(float v) {
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a == 0.0) return sign;
+    int ex;
+    frexp(a, &ex);  /* a = m * 2^ex, 0.5 <= m < 1, so 2^(ex-1) <= a < 2^ex */
+    int e = ex - 1; /* unbiased exponent of a's leading bit */
+    uint8_t code;
+    if (e < -6) {
+        /* subnormal range: multiples of 2^-9 (nearbyint rounds ties to even) */
+        const double r = nearbyint(ldexp(a, 9));
+        code = (uint8_t)r; /* r == 8 is the smallest normal, code 0x08 */
+    } else {
+        double r = nearbyint(ldexp(a, 3 - e)); /* in [8, 16] */
+        if (r == 16.0) {
+            r = 8.0;
+            e += 1;
+        }
+        if (e > 8 || (e == 8 && r > 14.0)) return (uint8_t)(sign | 0x7E); /* saturate to 448 */
+        code = (uint8_t)(((e + 7) << 3) | ((int)r - 8));
+    }
+    return (uint8_t)(sign | code);
+}
+
+/* The power-of-two scale of a vector whose largest magnitude is amax. */
+float oracle_fp8_scale(float amax) {
+    if (!(amax > 0.0f) || isinf(amax)) return 1.0f;
+    int ex;
+    const double m = frexp((double)amax, &ex); /* amax = m * 2^ex, 0.5 <= m < 1 */
+    const int c = (m == 0.5) ? ex - 1 : ex;    /* smallest c with amax <= 2^c */
+    return (float)ldexp(1.0, c - 8);
+}
+
+/* One bf16 vector of length n to codes and its scale. */
+float oracle_quantize_vector(int n, const uint16_t *v, int stride, uint8_t *q, int qstride) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        const float a = (float)fabs(bf16_to_double(v[(size_t)i * stride]));
+        if (a > amax) amax = a;
+    }
+    const float s = oracle_fp8_scale(amax);
+    for (int i = 0; i < n; ++i) q[(size_t)i * qstride] = oracle_e4m3_encode((float)(bf16_to_double(v[(size_t)i * stride]) / s));
+    return s;
+}
+
+/* Rows of a [rows, n] bf16 matrix: q [rows, n], one scale per row. */
+void oracle_quantize_rows(int rows, int n, const uint16_t *v, uint8_t *q, float *scale) {
+    for (int r = 0; r < rows; ++r) scale[r] = oracle_quantize_vector(n, v + (size_t)r * n, 1, q + (size_t)r * n, 1);
+}
+
+/* Expert weights w [E][K][N] (bf16) to q [E][N][K] with one scale per (e, n). */
+void oracle_quantize_weights(int E, int K, int N, const uint16_t *w, uint8_t *q, float *scale) {
+    for (int e = 0; e < E; ++e)
+        for (int n = 0; n < N; ++n)
+            scale[(size_t)e * N + n] = oracle_quantize_vector(K, w + (size_t)e * K * N + n, N,
+                                                              q + ((size_t)e * N + n) * K, 1);
+}
+
+/* Dequantize codes (with one scale per group of `group` consecutive codes)
+ * to bf16; exact, see above. */
+void oracle_dequantize(int64_t n, int group, const uint8_t *q, const float *scale, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16(oracle_e4m3_decode(q[i]) * (double)scale[i / group]);
+}

@@ -14,6 +14,11 @@ What pins what (nothing here re-types the oracle's own loops):
   experts    torch float64 matmul for the dense E=1, k=1 layer
   layer      identity experts with unit weights give bf16(k*x) exactly;
              capacity layout output bit-identical to the uncapped output
+  fp8        torch.float8_e4m3fn for every code's value and for rounding
+             (ties to even, subnormals, saturation); the power-of-two scale
+             against its closed-form bounds; row and weight quantizers
+             against a torch restatement (frexp + float8 cast); dequantized
+             values exactly decode(q) * s
 """
 from __future__ import annotations
 
@@ -257,7 +262,86 @@ def check_token_outputs(orc, seed=10):
     assert np.array_equal(o, r["out"][toks])
 
 
+def _torch_e4m3(v):
+    """float32 -> e4m3 codes by torch's cast (round to nearest even)."""
+    t = torch.as_tensor(np.asarray(v, np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def check_e4m3_decode_all_codes(orc):
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([orc.e4m3_decode(q) for q in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.nanmax(got) == 448.0 and got[1] == 2.0 ** -9
+
+
+def check_e4m3_encode_rounding(orc, seed=13):
+    vals = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    fin = np.unique(vals[np.isfinite(vals) & (vals >= 0)])
+    mids = (fin[1:] + fin[:-1]) / 2  # ties: round to the even code
+    rng = np.random.default_rng(seed)
+    rand = np.concatenate([rng.uniform(-448, 448, 3000), rng.uniform(-2 ** -5, 2 ** -5, 3000),
+                           rng.standard_normal(3000) * 40, np.linspace(448, 464, 17)])
+    v = np.concatenate([fin, -fin, mids, -mids, rand]).astype(np.float32)
+    got = np.array([orc.e4m3_encode(x) for x in v], np.uint8)
+    assert np.array_equal(got, _torch_e4m3(v))
+    # beyond 464 torch gives NaN; the oracle saturates (never reached with its scales)
+    assert orc.e4m3_encode(1000.0) == 0x7E and orc.e4m3_encode(-1000.0) == 0xFE
+
+
+def check_fp8_scale(orc, seed=14):
+    rng = np.random.default_rng(seed)
+    for a in np.concatenate([rng.lognormal(0, 8, 2000), 2.0 ** np.arange(-60, 60)]).astype(np.float32):
+        s = orc.fp8_scale(float(a))
+        m, e = math.frexp(s)
+        assert m == 0.5, "scale must be a power of two"
+        assert 128 * s < a <= 256 * s, (a, s)
+    for j in range(-40, 40):
+        assert orc.fp8_scale(2.0 ** j) == 2.0 ** (j - 8)
+    assert orc.fp8_scale(0.0) == 1.0
+
+
+def _torch_quant_rows(v_f32):
+    """Rows -> (codes, scales) restated with torch: scale 2^(ceil(log2 amax) - 8)."""
+    t = torch.as_tensor(v_f32, dtype=torch.float32)
+    amax = t.abs().amax(dim=-1)
+    m, e = torch.frexp(amax)
+    c = torch.where(m == 0.5, e - 1, e)
+    s = torch.where(amax > 0, torch.ldexp(torch.ones_like(amax), (c - 8).float()), torch.ones_like(amax))
+    q = (t / s[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q.numpy(), s.numpy()
+
+
+def check_quantize_rows_and_weights(orc, seed=15):
+    rng = np.random.default_rng(seed)
+    rows = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(
+        (rng.standard_normal((33, 160)) * rng.lognormal(0, 3, (33, 1))).astype(np.float32)))
+    rows[3] = 0.0
+    bits = synth.f32_to_bf16_bits(rows)
+    q, s = orc.quantize_rows(bits)
+    tq, ts = _torch_quant_rows(rows)
+    assert np.array_equal(s, ts) and np.array_equal(q, tq)
+    # weights [E, K, N] -> codes [E, N, K], one scale per (e, n) over K
+    w = synth.f32_to_bf16_bits((rng.standard_normal((3, 96, 40)) * 0.02).astype(np.float32))
+    wq, ws = orc.quantize_weights(w)
+    tq, ts = _torch_quant_rows(synth.bf16_bits_to_f32(w).transpose(0, 2, 1))
+    assert wq.shape == (3, 40, 96) and np.array_equal(wq, tq) and np.array_equal(ws, ts)
+    # dequantized values are exactly decode(q) * s, and within 2^-4 relative of the input
+    deq = synth.bf16_bits_to_f32(orc.dequantize(q, s)).astype(np.float64)
+    ref = torch.as_tensor(q).view(torch.float8_e4m3fn).double().numpy() * s[:, None].astype(np.float64)
+    assert np.array_equal(deq, ref)
+    err = np.abs(deq - rows)
+    assert np.all(err <= 2.0 ** -4 * np.abs(rows) + 2.0 ** -10 * s[:, None])
+    back = orc.dequantize_weights(wq, ws)
+    assert back.shape == w.shape
+    assert np.all(np.abs(synth.bf16_bits_to_f32(back) - synth.bf16_bits_to_f32(w)) <=
+                  2.0 ** -4 * np.abs(synth.bf16_bits_to_f32(w)) + 2.0 ** -10 * ws[:, None, :])
+
+
 ALL_CHECKS = [check_topk_bruteforce, check_topk_nan, check_softmax_weights, check_router_logits,
               check_dispatch_uncapped, check_dispatch_bruteforce, check_capacity_layout, check_identity_layer,
               check_identity_softmax_weights, check_combine_vs_torch, check_dense_swiglu_vs_torch,
-              check_capped_equals_uncapped, check_token_outputs]
+              check_capped_equals_uncapped, check_token_outputs, check_e4m3_decode_all_codes,
+              check_e4m3_encode_rounding, check_fp8_scale, check_quantize_rows_and_weights]

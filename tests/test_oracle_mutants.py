@@ -18,7 +18,9 @@ ORACLE_C = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 # normalised over all experts, an unstable order inside an expert, gate and
 # up swapped, a wrong SiLU sign, a transposed down-projection weight, an
 # unweighted combine, capacity slots filled in reverse, a reversed overflow
-# segment, logits accumulated in fp32.
+# segment, logits accumulated in fp32; for the fp8 variant a wrong exponent
+# bias, ties rounded away from zero, subnormals flushed to zero, a scale one
+# binade too high and weight codes left in the untransposed layout.
 MUTANTS = [
     ("tie_break_highest_index", "    return i < j;\n}", "    return i > j;\n}"),
     ("bias_dropped", "if (bias) l = l + bias[e];", "(void)bias;"),
@@ -40,6 +42,11 @@ MUTANTS = [
     ("capacity_slots_reversed", "row = (int64_t)e * C + r;", "row = (int64_t)e * C + (C - 1 - r);"),
     ("overflow_reversed", "row = (int64_t)E * C + spill_off[e] + (r - C);",
      "row = (int64_t)E * C + spill_off[e + 1] - 1 - (r - C);"),
+    ("e4m3_exponent_bias_8", "ldexp(1.0 + man / 8.0, ex - 7)", "ldexp(1.0 + man / 8.0, ex - 8)"),
+    ("e4m3_ties_away_from_zero", "double r = nearbyint(ldexp(a, 3 - e));", "double r = round(ldexp(a, 3 - e));"),
+    ("e4m3_subnormals_flushed", "code = (uint8_t)r; /* r == 8", "code = (uint8_t)(r >= 8.0 ? r : 0.0); /* r == 8"),
+    ("fp8_scale_one_binade_high", "return (float)ldexp(1.0, c - 8);", "return (float)ldexp(1.0, c - 7);"),
+    ("fp8_weights_not_transposed", "q + ((size_t)e * N + n) * K, 1);", "q + (size_t)e * K * N + n, N);"),
     ("logit_accumulated_in_float",
      "            double s = 0.0;\n            for (int h = 0; h < H; ++h) s += bf16_to_double",
      "            float s = 0.0f;\n            for (int h = 0; h < H; ++h) s += (float)bf16_to_double"),
