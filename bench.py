@@ -54,8 +54,7 @@ def parse_args():
     p.add_argument("--no-per-config", action="store_true",
                    help="time the headline workload only (default: every other workload too, on one GPU)")
     p.add_argument("--per-config-steps", type=int, default=20)
-    p.add_argument("--gemm-pairs", action="store_true",
-                   help="run the grouped GEMMs on CTA pairs (MOE_FLAG_GEMM_PAIRS; off by default: slower on B200)")
+    p.add_argument("--no-fp8", action="store_true", help="skip the fp8 (e4m3) variant of the layer")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     p.add_argument("--ref-budget-s", type=float, default=150.0)
     return p.parse_args()
@@ -305,6 +304,29 @@ def host_info():
 class Bench:
     """One process's device, stream, L2-cleaning buffers and clock sampler."""
 
+    def graph_ms(self, launch, steps):
+        """Total device time of `steps` replays of one captured call (L2
+        cleaned before each replay, outside the timed interval)."""
+        import numpy as np
+        torch, dev, stream = self.torch, self.dev, self.stream
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+            launch()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for _ in range(3):
+            self.flush()
+            g.replay()
+        self.barrier()
+        for i in range(steps):
+            self.flush()
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+        self.barrier()
+        total = float(np.sum([a.elapsed_time(c) for a, c in ev]))
+        del g
+        return total
+
     def __init__(self, dev, world, local):
         import torch
         self.torch = torch
@@ -421,11 +443,90 @@ class Bench:
         clocks = sampler.stop()
         total_ms = float(np.sum([a.elapsed_time(c) for a, c in gev]))
         del g
-        total_ms, eager_ms = max_over_ranks([total_ms, eager_ms], dev)
+        # the same layer with the combine inside the down GEMM's epilogue
+        sf = moe.make_shape(shape.T, shape.H, shape.F, shape.E, shape.k, shape.C, flags=shape.flags |
+                            moe.MOE_FLAG_FUSED_COMBINE)
+        fused_ms = self.graph_ms(lambda: moe.moe_forward(sf, b, ws, args=args_c), K)
+        total_ms, eager_ms, fused_ms = max_over_ranks([total_ms, eager_ms, fused_ms], dev)
         status |= moe.moe_read_status(ws, stream)
         return {"total_ms": total_ms, "eager_ms": eager_ms, "kmean_s": seg.mean(axis=0) * 1e-3, "gather": gather,
-                "fwd_bufs": fwd_bufs, "clocks": clocks, "status": status, "wall": wall,
+                "fwd_bufs": fwd_bufs, "clocks": clocks, "status": status, "wall": wall, "fused_ms": fused_ms,
                 "counts": b["expert_counts"].cpu().numpy()}
+
+    def measure_fp8(self, cfg, shape, b, steps, warmup):
+        """The fp8 (e4m3) layer, same protocol: weights quantized once before
+        timing; per step the router/dispatch, the token-row quantization (the
+        row copy, or token rows for the row-gathering GEMM), the fp8 SwiGLU
+        GEMM, the h quantization, the fp8 down GEMM and the combine."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        torch, dev, stream = self.torch, self.dev, self.stream
+        ws = b["ws"]
+        per_token = cfg.T * cfg.k <= 32 * cfg.E
+        b.update(moe.alloc_fp8_buffers(shape, per_token=per_token, device=dev))
+        moe.quantize_layer_weights_fp8(shape, b, stream)
+        src_tok = b["src_token"] if per_token else None
+
+        def step_events(ev):
+            ev[0].record(stream)
+            moe.moe_route_dispatch(shape, b["x"], b["w_router"], b["bias"], b["logits"], b["topk_idx"], b["topk_w"],
+                                   b["expert_counts"], b["expert_offsets"], b["src_token"], b["dest_row"], ws, stream)
+            ev[1].record(stream)
+            moe.moe_quantize_rows_fp8(shape, moe.MOE_ROWS_TOKENS if per_token else moe.MOE_ROWS_X_PERM, b["x"],
+                                      b["src_token"], b["x_q"], b["x_scale"], ws, stream)
+            ev[2].record(stream)
+            moe.moe_grouped_swiglu_fp8(shape, b["x_q"], b["x_scale"], src_tok, b["wg_q"], b["wg_scale"], b["wu_q"],
+                                       b["wu_scale"], b["h"], ws, stream)
+            ev[3].record(stream)
+            moe.moe_quantize_rows_fp8(shape, moe.MOE_ROWS_H, b["h"], b["src_token"], b["h_q"], b["h_scale"], ws,
+                                      stream)
+            ev[4].record(stream)
+            moe.moe_grouped_down_fp8(shape, b["h_q"], b["h_scale"], b["wd_q"], b["wd_scale"], b["y"], ws, stream)
+            ev[5].record(stream)
+            moe.moe_combine(shape, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
+            ev[6].record(stream)
+
+        wev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        for _ in range(max(warmup, 3)):
+            self.flush()
+            step_events(wev)
+        torch.cuda.synchronize(dev)
+        status = moe.moe_read_status(ws, stream)
+        if status & ~moe.MOE_DEV_NAN_LOGIT:
+            raise RuntimeError("device status %#x after fp8 warm-up (%s)" % (status, cfg.name))
+        K = steps
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+        self.barrier()
+        for i in range(K):
+            self.flush()
+            step_events(evs[i])
+        self.barrier()
+        seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)] for i in range(K)])
+        args_c = moe.forward_fp8_args(b, per_token)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+            moe.moe_forward_fp8(shape, b, ws, args=args_c)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(3):
+            self.flush()
+            g.replay()
+        self.barrier()
+        for i in range(K):
+            self.flush()
+            gev[i][0].record(stream)
+            g.replay()
+            gev[i][1].record(stream)
+        self.barrier()
+        total_ms = float(np.sum([a.elapsed_time(c) for a, c in gev]))
+        del g
+        sf = moe.make_shape(shape.T, shape.H, shape.F, shape.E, shape.k, shape.C, flags=shape.flags |
+                            moe.MOE_FLAG_FUSED_COMBINE)
+        fused_ms = self.graph_ms(lambda: moe.moe_forward_fp8(sf, b, ws, args=args_c), K)
+        total_ms, fused_ms = max_over_ranks([total_ms, fused_ms], dev)
+        status |= moe.moe_read_status(ws, stream)
+        return {"total_ms": total_ms, "kmean_s": seg.mean(axis=0) * 1e-3, "per_token": per_token, "status": status,
+                "fused_ms": fused_ms, "counts": b["expert_counts"].cpu().numpy()}
 
     def e2e(self, cfg, shape, b, x_rank, fwd_bufs, steps):
         """The same metric end to end: pinned-host tokens copied in, the layer,
@@ -504,10 +605,57 @@ def summarize(cfg, m, steps, world, peaks, peak_src):
                            "bound": "hbm" if layer_hbm >= layer_tc else "tensor"},
         "kernels": kernels,
         "eager_entry_points_ms_per_step": m["eager_ms"] / steps,
+        "fused_combine": {"value": whole_job_rate(cfg.T, steps, world, m["fused_ms"]),
+                          "ms_per_step": m["fused_ms"] / steps,
+                          "what": "moe_forward with MOE_FLAG_FUSED_COMBINE (combine in the down GEMM's epilogue)"},
         "clocks": m["clocks"],
         "routing": routing_stats(counts, cfg.C),
         "device_status": m["status"],
         "wall_s_timed_region": m["wall"],
+    }
+
+
+def summarize_fp8(cfg, m, steps, world, peaks, peak_src):
+    """Throughput and rooflines of the fp8 layer.  Tensor peak for e4m3
+    operands: the measured bf16 peak times the nominal fp8/bf16 ratio (2)."""
+    counts = m["counts"]
+    T, H, F, k = cfg.T, cfg.H, cfg.F, cfg.k
+    R = T * k
+    touched = sum(1 for c in counts if c > 0)
+    kmean = m["kmean_s"]
+    names = ["route_dispatch", "quant_x", "grouped_swiglu_fp8", "quant_h", "grouped_down_fp8", "combine"]
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+
+    def roof(bytes_, flops, t):
+        t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (fp8_peak * 1e12)
+        if t_hbm >= t_tc:
+            a = bytes_ / t / 1e9
+            return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": a / peaks["hbm_gbs"]}
+        a = flops / t / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": fp8_peak, "unit": "TFLOP/s", "frac": a / fp8_peak,
+                "peak_note": "measured bf16 peak x 2 (nominal e4m3/bf16 ratio)"}
+
+    sw_bytes = touched * 2 * H * F + R * H + R * F * 2
+    sw_flops = 4 * R * H * F
+    dn_bytes = touched * F * H + R * F + R * H * 2
+    dn_flops = 2 * R * F * H
+    ms = m["total_ms"] / steps
+    layer_bytes = touched * 3 * H * F + 2 * T * H * 2 + H * cfg.E * 4
+    layer_flops = sw_flops + dn_flops + 2 * T * H * cfg.E
+    layer_t = max(layer_bytes / (peaks["hbm_gbs"] * 1e9), layer_flops / (fp8_peak * 1e12))
+    sw = roof(sw_bytes, sw_flops, kmean[2])
+    sw.update({"algorithmic_bytes": sw_bytes, "algorithmic_flops": sw_flops, "peak_source": peak_src,
+               "kernel": "k_grouped_gemm<0, *, FP8> (moe_grouped_swiglu_fp8)"})
+    return {
+        "value": whole_job_rate(T, steps, world, m["total_ms"]), "ms_per_step": ms, "dtype": "e4m3 weights and "
+        "activations (per-column / per-row power-of-two scales), fp32 accumulate, bf16 h, y, out",
+        "kernels": {nm + "_us": t * 1e6 for nm, t in zip(names, kmean)},
+        "roofline": sw,
+        "grouped_down_roofline": roof(dn_bytes, dn_flops, kmean[4]),
+        "layer_roofline": {"frac": layer_t / (ms * 1e-3), "roofline_us": layer_t * 1e6},
+        "token_rows_gathered": bool(m["per_token"]), "device_status": m["status"],
+        "fused_combine": {"value": whole_job_rate(T, steps, world, m["fused_ms"]), "ms_per_step": m["fused_ms"] / steps},
     }
 
 
@@ -553,12 +701,13 @@ def run_ours(args):
     x_rank = replica_tokens(cfg, rank, L)  # each replica its own tokens
     log("rank %d: generated %s in %.1f s" % (rank, cfg.name, time.time() - t0))
     bench = Bench(dev, world, local)
-    flags = moe.MOE_FLAG_GEMM_PAIRS if args.gemm_pairs else 0
+    flags = 0
     shape, b = bench.upload(cfg, L, x_rank, flags)
     K = args.steps
     m = bench.measure(cfg, shape, b, K, args.warmup)
     e2e_ms = bench.e2e(cfg, shape, b, x_rank, m["fwd_bufs"], K)
     peaks, peak_src = load_peaks()
+    m8 = None if args.no_fp8 else bench.measure_fp8(cfg, shape, b, K, args.warmup)
 
     result = None
     if rank == 0:
@@ -567,12 +716,12 @@ def run_ours(args):
             "metric": METRIC, "value": s["value"], "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": s["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu",
-                                        "gemm": "cta pairs" if args.gemm_pairs else "single cta"}),
+            "config": config_json(cfg, {"parallelism": "replicas" if world > 1 else "single-gpu"}),
             "roofline": s["roofline"],
             "layer_roofline": s["layer_roofline"],
             "kernels": s["kernels"],
             "eager_entry_points_ms_per_step": s["eager_entry_points_ms_per_step"],
+            "fused_combine": s["fused_combine"],
             "e2e": {"value": whole_job_rate(cfg.T, K, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
             "gpu_launches": forward_launches(cfg) * K,
@@ -581,6 +730,8 @@ def run_ours(args):
             "device_status": s["device_status"],
             "wall_s_timed_region": s["wall_s_timed_region"],
         }
+        if m8 is not None:
+            result["fp8"] = summarize_fp8(cfg, m8, K, world, peaks, peak_src)
     del b
     gc.collect()
     torch.cuda.empty_cache()
@@ -598,6 +749,9 @@ def run_ours(args):
             mp = bench.measure(pc, shp, bp, kp, min(args.warmup, 5))
             sp = summarize(pc, mp, kp, world, peaks, peak_src)
             sp.update({"steps": kp, "config": config_json(pc), "gpu_launches": forward_launches(pc) * kp})
+            if not args.no_fp8 and pc.T * pc.k > 256:  # the tiny layer has nothing to stream
+                sp["fp8"] = summarize_fp8(pc, bench.measure_fp8(pc, shp, bp, kp, min(args.warmup, 5)), kp, world,
+                                          peaks, peak_src)
             per_config[workload_name(pc)] = sp
             log("per-config %s: %.0f tokens/s (%.1f s)" % (pc.name, sp["value"], time.time() - t0))
             del bp, Lp

@@ -22,16 +22,23 @@ MOE_DEV_NAN_LOGIT = 0x8
 MOE_DEV_BAD_ROW = 0x10
 MOE_FLAG_CAPACITY = 0x1
 MOE_FLAG_LOGITS_IN = 0x2
-MOE_FLAG_GEMM_PAIRS = 0x4
+MOE_FLAG_FUSED_COMBINE = 0x8
 MOE_FLAG_TEST_STALL_SCAN = 0x40000000
 MOE_FLAG_TEST_STALL_GEMM = 0x20000000
+MOE_WEIGHTS_GATE_UP = 0
+MOE_WEIGHTS_DOWN = 1
+MOE_ROWS_X_PERM = 0
+MOE_ROWS_TOKENS = 1
+MOE_ROWS_H = 2
 
 # Every symbol include/moe.h declares (the CPU tests check the library exports each).
 ABI_FUNCTIONS = (
     "moe_permuted_rows", "moe_workspace_bytes", "moe_workspace_layout", "moe_workspace_init", "moe_route",
     "moe_permute", "moe_grouped_swiglu", "moe_grouped_down", "moe_combine", "moe_forward", "moe_read_status",
     "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version", "moe_permute_static",
-    "moe_route_dispatch", "moe_gather", "moe_grouped_swiglu_gather",
+    "moe_route_dispatch", "moe_gather", "moe_grouped_swiglu_gather", "moe_quantize_weights_fp8",
+    "moe_quantize_rows_fp8", "moe_grouped_swiglu_fp8", "moe_grouped_down_fp8", "moe_forward_fp8",
+    "moe_grouped_down_combine", "moe_grouped_down_fp8_combine",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -49,6 +56,13 @@ class MoeForwardArgs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "x", "w_router", "bias", "w_gate", "w_up", "w_down", "logits", "topk_idx", "topk_w", "expert_counts",
         "expert_offsets", "src_token", "dest_row", "x_perm", "h", "y", "out")]
+
+
+class MoeForwardFp8Args(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "x", "w_router", "bias", "wg_q", "wg_scale", "wu_q", "wu_scale", "wd_q", "wd_scale", "logits", "topk_idx",
+        "topk_w", "expert_counts", "expert_offsets", "src_token", "dest_row", "x_q", "x_scale")] + [
+        ("x_q_per_token", ctypes.c_int32)] + [(n, ctypes.c_void_p) for n in ("h", "h_q", "h_scale", "y", "out")]
 
 
 class MoeWsLayout(ctypes.Structure):
@@ -114,6 +128,20 @@ def load_library(path: str = LIB_PATH):
     lib.moe_version.restype = ctypes.c_int32
     lib.moe_permute_static.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.moe_permute_static.restype = st
+    lib.moe_quantize_weights_fp8.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp]
+    lib.moe_quantize_weights_fp8.restype = st
+    lib.moe_quantize_rows_fp8.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, vp, vp]
+    lib.moe_quantize_rows_fp8.restype = st
+    lib.moe_grouped_swiglu_fp8.argtypes = [sp] + [vp] * 10
+    lib.moe_grouped_swiglu_fp8.restype = st
+    lib.moe_grouped_down_fp8.argtypes = [sp] + [vp] * 7
+    lib.moe_grouped_down_fp8.restype = st
+    lib.moe_forward_fp8.argtypes = [sp, ctypes.POINTER(MoeForwardFp8Args), vp, vp]
+    lib.moe_forward_fp8.restype = st
+    lib.moe_grouped_down_combine.argtypes = [sp] + [vp] * 9
+    lib.moe_grouped_down_combine.restype = st
+    lib.moe_grouped_down_fp8_combine.argtypes = [sp] + [vp] * 11
+    lib.moe_grouped_down_fp8_combine.restype = st
     _lib = lib
     return lib
 
@@ -215,6 +243,20 @@ def moe_grouped_down(shape, h, w_down, y, ws, stream=None):
                                            _stream(stream)), "moe_grouped_down")
 
 
+def moe_grouped_down_combine(shape, h, w_down, src_token, dest_row, topk_w, y, out, ws, stream=None):
+    _check(load_library().moe_grouped_down_combine(ctypes.byref(shape), _ptr(h), _ptr(w_down), _ptr(src_token),
+                                                   _ptr(dest_row), _ptr(topk_w), _ptr(y), _ptr(out), _ptr(ws),
+                                                   _stream(stream)), "moe_grouped_down_combine")
+
+
+def moe_grouped_down_fp8_combine(shape, h_q, h_scale, wd_q, wd_scale, src_token, dest_row, topk_w, y, out, ws,
+                                 stream=None):
+    _check(load_library().moe_grouped_down_fp8_combine(ctypes.byref(shape), _ptr(h_q), _ptr(h_scale), _ptr(wd_q),
+                                                       _ptr(wd_scale), _ptr(src_token), _ptr(dest_row), _ptr(topk_w),
+                                                       _ptr(y), _ptr(out), _ptr(ws), _stream(stream)),
+           "moe_grouped_down_fp8_combine")
+
+
 def moe_combine(shape, y, dest_row, topk_w, out, stream=None):
     _check(load_library().moe_combine(ctypes.byref(shape), _ptr(y), _ptr(dest_row), _ptr(topk_w), _ptr(out),
                                       _stream(stream)), "moe_combine")
@@ -275,3 +317,72 @@ def alloc_buffers(shape: MoeShape, device="cuda"):
     moe_workspace_init(shape, ws)
     b["ws"] = ws
     return b
+
+
+# ---------------------------------------------------------------- fp8 (e4m3) --
+
+def moe_quantize_weights_fp8(shape, which, w, w_q, w_scale, stream=None):
+    _check(load_library().moe_quantize_weights_fp8(ctypes.byref(shape), int(which), _ptr(w), _ptr(w_q), _ptr(w_scale),
+                                                   _stream(stream)), "moe_quantize_weights_fp8")
+
+
+def moe_quantize_rows_fp8(shape, which, src, src_token, q, scale, ws, stream=None):
+    _check(load_library().moe_quantize_rows_fp8(ctypes.byref(shape), int(which), _ptr(src), _ptr(src_token), _ptr(q),
+                                                _ptr(scale), _ptr(ws), _stream(stream)), "moe_quantize_rows_fp8")
+
+
+def moe_grouped_swiglu_fp8(shape, x_q, x_scale, src_token, wg_q, wg_scale, wu_q, wu_scale, h, ws, stream=None):
+    _check(load_library().moe_grouped_swiglu_fp8(ctypes.byref(shape), _ptr(x_q), _ptr(x_scale), _ptr(src_token),
+                                                 _ptr(wg_q), _ptr(wg_scale), _ptr(wu_q), _ptr(wu_scale), _ptr(h),
+                                                 _ptr(ws), _stream(stream)), "moe_grouped_swiglu_fp8")
+
+
+def moe_grouped_down_fp8(shape, h_q, h_scale, wd_q, wd_scale, y, ws, stream=None):
+    _check(load_library().moe_grouped_down_fp8(ctypes.byref(shape), _ptr(h_q), _ptr(h_scale), _ptr(wd_q),
+                                               _ptr(wd_scale), _ptr(y), _ptr(ws), _stream(stream)),
+           "moe_grouped_down_fp8")
+
+
+def forward_fp8_args(bufs: dict, per_token=False) -> MoeForwardFp8Args:
+    a = MoeForwardFp8Args()
+    for name, _ in MoeForwardFp8Args._fields_:
+        if name != "x_q_per_token":
+            setattr(a, name, _ptr(bufs.get(name)))
+    a.x_q_per_token = 1 if per_token else 0
+    return a
+
+
+def moe_forward_fp8(shape, bufs: dict, ws, stream=None, args: MoeForwardFp8Args | None = None, per_token=False):
+    a = args if args is not None else forward_fp8_args(bufs, per_token)
+    _check(load_library().moe_forward_fp8(ctypes.byref(shape), ctypes.byref(a), _ptr(ws), _stream(stream)),
+           "moe_forward_fp8")
+
+
+def alloc_fp8_buffers(shape: MoeShape, per_token=False, device="cuda"):
+    """Device buffers of the fp8 layer that moe_forward's buffers do not hold:
+    weight codes and scales, token-row codes and scales, h codes and scales."""
+    import torch
+    T, H, F, E = shape.T, shape.H, shape.F, shape.E
+    P = moe_permuted_rows(shape)
+    dev = torch.device(device)
+    xr = T if per_token else P
+    return dict(
+        wg_q=torch.empty((E, F, H), dtype=torch.uint8, device=dev),
+        wg_scale=torch.empty((E, F), dtype=torch.float32, device=dev),
+        wu_q=torch.empty((E, F, H), dtype=torch.uint8, device=dev),
+        wu_scale=torch.empty((E, F), dtype=torch.float32, device=dev),
+        wd_q=torch.empty((E, H, F), dtype=torch.uint8, device=dev),
+        wd_scale=torch.empty((E, H), dtype=torch.float32, device=dev),
+        x_q=torch.empty((xr, H), dtype=torch.uint8, device=dev),
+        x_scale=torch.empty((xr,), dtype=torch.float32, device=dev),
+        h_q=torch.empty((P, F), dtype=torch.uint8, device=dev),
+        h_scale=torch.empty((P,), dtype=torch.float32, device=dev),
+    )
+
+
+def quantize_layer_weights_fp8(shape, bufs, stream=None):
+    """Codes and scales of w_gate, w_up, w_down (bufs as alloc_buffers +
+    alloc_fp8_buffers fill it)."""
+    moe_quantize_weights_fp8(shape, MOE_WEIGHTS_GATE_UP, bufs["w_gate"], bufs["wg_q"], bufs["wg_scale"], stream)
+    moe_quantize_weights_fp8(shape, MOE_WEIGHTS_GATE_UP, bufs["w_up"], bufs["wu_q"], bufs["wu_scale"], stream)
+    moe_quantize_weights_fp8(shape, MOE_WEIGHTS_DOWN, bufs["w_down"], bufs["wd_q"], bufs["wd_scale"], stream)

@@ -33,6 +33,8 @@ template <int KMAX>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const int *__restrict__ dest_row,
                                                  const float *__restrict__ w, uint4 *__restrict__ out, int k, int H8,
                                                  int P) {
+    pdl_trigger();
+    pdl_wait();
     const int t = blockIdx.x;
     const int v = blockIdx.y * blockDim.x + threadIdx.x;
     if (v >= H8) return;
@@ -85,11 +87,14 @@ cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *des
     const dim3 grid((unsigned)s.T, (unsigned)((H8 + 255) / 256));
     const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, (s.flags & MOE_FLAG_CAPACITY) != 0);
     if (s.k <= 2)
-        k_combine<2><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+        return launch_pdl(k_combine<2>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
+                          s.k, H8, P);
     else if (s.k <= 8)
-        k_combine<8><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+        return launch_pdl(k_combine<8>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
+                          s.k, H8, P);
     else
-        k_combine<0><<<grid, 256, 0, stream>>>((const uint4 *)y, dest_row, topk_w, (uint4 *)out, s.k, H8, P);
+        return launch_pdl(k_combine<0>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
+                          s.k, H8, P);
     return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@ struct WsLayout {
     size_t dispatch_end;          // end of what the dispatch step uses (the router's buffers follow)
     size_t router_planes;         // bf16[3][H][router_plane_cols(E)] (tensor-core router only)
     size_t router_part;           // fp32[q][T][E] partial logits of the K ranges (tensor-core router only)
+    size_t combine_cnt;           // int32[T][H/128] arrival counts of the combine fused into the down GEMM
     size_t total;
     int nchunks, max_tiles;
 };
@@ -99,6 +100,13 @@ struct FusedDispatch {
     int32_t *counts, *offsets, *src_token, *dest_row;
 };
 
+// Inputs and output of the combine when it runs in the down GEMM's epilogue.
+struct CombineOut {
+    const int32_t *src_token, *dest_row;
+    const float *topk_w;
+    void *out;
+};
+
 inline int64_t permuted_rows(int T, int E, int k, int C, bool capped) {
     if (!capped) return (int64_t)T * k;
     return (int64_t)E * C + (int64_t)k * (T > C ? T - C : 0);
@@ -146,6 +154,8 @@ inline WsLayout ws_layout(int T, int H, int E, int k, int C, bool capped) {
         // q grows with the SM count: the bound of the largest device planned for
         L.router_part = arr(4 * (size_t)router_tc_plan(T, H, E, kRoutePlanMaxSms).q * T * E);
     }
+    // zero after moe_workspace_init; every fused down+combine launch leaves it zero again
+    L.combine_cnt = arr(4 * (size_t)T * (H / 128));
     L.total = o;
     return L;
 }
@@ -186,6 +196,36 @@ inline WsPtrs ws_ptrs(void *ws, const WsLayout &L) {
     p.max_tiles = L.max_tiles;
     return p;
 }
+
+// ------------------------------------------- programmatic dependent launch --
+// The kernels after the first one of the layer are launched with the
+// programmatic-serialization attribute: such a kernel may be scheduled while
+// the kernel before it on the stream is still running, once every CTA of that
+// kernel has called pdl_trigger (or exited).  It calls pdl_wait -- which
+// returns when the kernel before it has completed and its memory is visible --
+// before its first global-memory access, so only its launch and its prologue
+// (barrier set-up, tensor-memory allocation, descriptor prefetch) overlap the
+// previous kernel.  Launched without the attribute, both calls do nothing.
+#if defined(__CUDACC__)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+#endif
 
 // ------------------------------------------------------------ device helpers --
 #if defined(__CUDACC__)
@@ -332,67 +372,6 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-// ----- pairs of CTAs (a cluster of two) sharing one MMA: cta_group::2 -----
-// The pair's even CTA ("leader") issues the MMAs; M = 256 splits into 128 rows
-// per CTA (A and D), N splits into halves (B), both read at the same
-// shared-memory offsets in the two CTAs.
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_arrive_wait() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Shared::cluster address of the same shared-memory location in CTA `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(const void *p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-// One arrive on an mbarrier of another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
-}
-// TMA tile load into this CTA's shared memory whose completed bytes are
-// counted on an mbarrier of the pair (normally the leader's).
-__device__ __forceinline__ void tma_load_2d_pair(void *dst, const void *tmap, uint32_t bar_cluster_addr, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(tmap), "r"(bar_cluster_addr), "r"(x), "r"(y)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// Arrives once on `bar` (same offset) in every CTA of `cta_mask` when the
-// pair MMAs issued so far by this thread complete.
-__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"(cta_mask)
-        : "memory");
-}
-__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate.
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -400,6 +379,18 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc], both operands 8-bit floats of the
+// kind the instruction descriptor names (kind::f8f6f4), fp32 accumulate;
+// K = 32 per instruction.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -467,6 +458,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with both operands E4M3
+// (type code 0 in bits 7-9 and 10-12), both K-major (bits 15, 16 clear), fp32
+// accumulator (bits 4-5 = 1), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace moe

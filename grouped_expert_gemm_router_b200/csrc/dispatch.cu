@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(kScanThreads) k_hist_scan(ScanArgs a) {
     int *hist = sm.hist;
     __shared__ int s_chunk, s_bad, s_timeout;
     const int tid = threadIdx.x, E = a.E;
+    pdl_trigger();
     if (tid == 0) {
         s_chunk = (int)atomicAdd(a.ws.ticket, 1u);
         s_bad = 0;
@@ -139,6 +140,8 @@ struct RankArgs {
 
 __global__ void __launch_bounds__(kScanThreads) k_rank(RankArgs a) {
     __shared__ DispatchSmem sm;
+    pdl_trigger();
+    pdl_wait();
     const int chunk = blockIdx.x;
     for (int e = threadIdx.x; e <= a.E; e += kScanThreads) {
         if (e < a.E) sm.running[e] = a.ws.chunk_excl[(size_t)chunk * a.E + e];
@@ -156,10 +159,15 @@ __global__ void __launch_bounds__(kScanThreads) k_rank(RankArgs a) {
 }
 
 // One warp per permuted row; rows are [0, R) uncapped, or the E*C capacity
-// slots plus the used part of the overflow region.
+// slots plus the used part of the overflow region.  The rows are written with
+// streaming (evict-first) stores: x_perm is k times larger than x, and a
+// token's k copies are made at different times, so ordinary stores would
+// evict x from L2 between them and every copy would re-read it from DRAM.
 __global__ void __launch_bounds__(256) k_gather(const uint4 *__restrict__ x, const int *__restrict__ src_token,
                                                 uint4 *__restrict__ x_perm, int H8, int T, int P, int fixed_rows,
                                                 int cap_rows, const int *total_spill) {
+    pdl_trigger();
+    pdl_wait();
     int rows = fixed_rows >= 0 ? fixed_rows : cap_rows + *total_spill;
     if (rows > P) rows = P;
     const int lane = threadIdx.x & 31;
@@ -177,9 +185,9 @@ __global__ void __launch_bounds__(256) k_gather(const uint4 *__restrict__ x, con
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = __ldg(src + v + 32 * i);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dst[v + 32 * i] = q[i];
+                for (int i = 0; i < 8; ++i) __stcs(dst + v + 32 * i, q[i]);
             }
-            for (; v < H8; v += 32) dst[v] = __ldg(src + v);
+            for (; v < H8; v += 32) __stcs(dst + v, __ldg(src + v));
         } else {
             for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
         }
@@ -202,9 +210,8 @@ cudaError_t launch_gather(const moe_shape &s, const void *x, const int32_t *src_
     const int cap_blocks = num_sms * 8;
     if (blocks > cap_blocks) blocks = cap_blocks;
     if (blocks < 1) blocks = 1;
-    k_gather<<<blocks, 256, 0, stream>>>((const uint4 *)x, src_token, (uint4 *)x_perm, H8, s.T, P, fixed, s.E * s.C,
-                                         p.total_spill);
-    return cudaGetLastError();
+    return launch_pdl(k_gather, dim3(blocks), dim3(256), 0, stream, (const uint4 *)x, src_token, (uint4 *)x_perm, H8,
+                      s.T, P, fixed, s.E * s.C, (const int *)p.total_spill);
 }
 
 // Histogram, scan, schedule and ranks (moe_permute without the row copy).
@@ -248,8 +255,7 @@ cudaError_t launch_dispatch_index(const moe_shape &s, const int32_t *topk_idx, i
     ra.dest_row = dest_row;
     ra.src_token = src_token;
     ra.ws = p;
-    k_rank<<<L.nchunks, kScanThreads, 0, stream>>>(ra);
-    return cudaGetLastError();
+    return launch_pdl(k_rank, dim3(L.nchunks), dim3(kScanThreads), 0, stream, ra);
 }
 
 cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *topk_idx, int32_t *counts,

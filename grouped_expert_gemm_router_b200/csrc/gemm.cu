@@ -117,6 +117,21 @@ struct GemmArgs {
     int route_groups;   // accumulators per unit: route_groups * nacc * route_rows <= 512 columns
     uint32_t row_boxes; // bit i: RowMaps::m[i] (boxes of 16 << i rows) is valid; bit 0 always
     int stall_first_stage;  // test hook: CTA 0's token producer never loads its first stage
+    // FP8 (e4m3 operands): value = code * scale, one power-of-two scale per
+    // expert and output feature (w_scale0/1: [E][n_out], for the weights of
+    // accumulators 0 and 1) and one per row of the token matrix (row_scale,
+    // indexed by permuted row, or by token when the rows are gathered)
+    const float *w_scale0, *w_scale1, *row_scale;
+    // COMBINE (mode 1): step 5 fused into the down projection's epilogue.
+    // comb_cnt [T][n_out / 128] counts, per token and 128-feature block, the
+    // (row, lane-quarter warp) pieces of y stored so far; the warp whose piece
+    // completes a token's block (4 k pieces) combines that block from y into
+    // comb_out and sets the count back to zero.
+    const int *dest_row;
+    const float *topk_w;
+    __nv_bfloat16 *comb_out;
+    int *comb_cnt;
+    int k;
 };
 
 // Tensor maps of the token matrix (B operand) with boxes of 16 << i rows x 64
@@ -151,8 +166,8 @@ struct Unit {
 
 template <int MODE>
 // num_fb / fbw: feature blocks per row tile and their width (mode 0: 128
-// features per CTA, 256 per CTA pair; mode 1: 256 features in two
-// accumulators, or 128 in one when that still fits one wave).
+// features, gate and up; mode 1: 256 features in two accumulators, or 128 in
+// one when that still fits one wave).
 __device__ __forceinline__ void decode_unit(int u, const int *gts, const GemmArgs &a, int trows, int num_fb, int fbw,
                                             Unit &U) {
     if (MODE == 2) {  // unit u = tokens [tb * route_rows, ...) x K range fb, all experts
@@ -206,46 +221,6 @@ __device__ __forceinline__ int unit_row(const Unit &U, int c) {
     return c1 < U.p1l ? U.p1s + c1 : -1;
 }
 
-// Stores a 32-feature x 16-row block of bf16 results held by one warp: lane l
-// holds feature fbase + l of unit rows c0 .. c0 + 15 as w[m] = (row 2m, row
-// 2m + 1).  Three butterfly exchanges (lanes ^1, ^2, ^4) leave each lane eight
-// consecutive features of unit rows c0 + (l & 7) and c0 + 8 + (l & 7), stored
-// as two 16-byte vectors: a warp writes the block with 2 store instructions
-// instead of 16, and the epilogue's time is set by its store instructions.
-__device__ __forceinline__ void store_block_32x16(const uint32_t (&w)[8], __nv_bfloat16 *out, int n_out, int fbase,
-                                                  const Unit &U, int c0) {
-    const int lane = threadIdx.x & 31;
-    const bool p = lane & 1, P = (lane >> 1) & 1, Q = (lane >> 2) & 1;
-    // (two rows, one feature) -> (one row, two features): x[m] = row 2m + p,
-    // features (l & ~1) and (l & ~1) + 1
-    uint32_t x[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const uint32_t o = __shfl_xor_sync(0xffffffffu, w[m], 1);
-        x[m] = p ? __byte_perm(o, w[m], 0x7632) : __byte_perm(w[m], o, 0x5410);
-    }
-    // keep m = 2t + P: y[t] = row 4t + 2P + p, features (l & ~3) .. + 3
-    uint32_t y[4][2];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const uint32_t keep = P ? x[2 * t + 1] : x[2 * t];
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, P ? x[2 * t] : x[2 * t + 1], 2);
-        y[t][0] = P ? recv : keep;
-        y[t][1] = P ? keep : recv;
-    }
-    // keep t = 2s + Q: row 8s + (l & 7), features (l & ~7) .. + 7
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-        const uint32_t k0 = Q ? y[2 * s + 1][0] : y[2 * s][0], k1 = Q ? y[2 * s + 1][1] : y[2 * s][1];
-        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, Q ? y[2 * s][0] : y[2 * s + 1][0], 4);
-        const uint32_t r1 = __shfl_xor_sync(0xffffffffu, Q ? y[2 * s][1] : y[2 * s + 1][1], 4);
-        const int row = unit_row(U, c0 + 8 * s + (lane & 7));
-        if (row >= 0)
-            *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + (lane & ~7)) =
-                Q ? make_uint4(r0, r1, k0, k1) : make_uint4(k0, k1, r0, r1);
-    }
-}
-
 // Stores a 32-feature x 16-row block of bf16 results held by one warp in the
 // fragment layout of tmem_ld_frag16 (w[m] = the pair r[2m], r[2m + 1]: feature
 // 16 (m >> 2) + 8 (m & 1) + (t >> 2), rows 8 ((m >> 1) & 1) + 2 (t & 3) + {0, 1}
@@ -271,6 +246,17 @@ __device__ __forceinline__ void store_block_frag(const uint32_t (&w)[8], uint8_t
         const int row = unit_row(U, c0 + 8 * k + r);
         if (row >= 0) *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + 8 * c) = v;
     }
+}
+
+// silu(z) = z * sigmoid(z) = z/2 + (z/2) tanh(z/2): one MUFU operation
+// (tanh.approx, relative error below 2^-10, far inside the bf16 rounding of
+// h) instead of an exponential and a reciprocal.  The epilogue of the SwiGLU
+// GEMM holds the accumulator while it evaluates 32,768 of these per unit.
+__device__ __forceinline__ float silu_f(float z) {
+    const float hz = 0.5f * z;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hz));
+    return fmaf(hz, t, hz);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
@@ -304,6 +290,153 @@ struct TmemPlan {
     }
 };
 
+// FP8 epilogue: in the fragment layout of tmem_ld_frag16, register j of a
+// 16-column chunk holds feature (lane >> 2) + 8 * fidx(j) of the warp's lane
+// quarter and unit row c0 + 2 * (lane & 3) + 8 * ((j >> 2) & 1) + (j & 1):
+// four features and four rows per thread.
+__device__ __forceinline__ int frag_fidx(int j) { return 2 * (j >> 3) + ((j >> 1) & 1); }
+__device__ __forceinline__ int frag_ridx(int j) { return 2 * ((j >> 2) & 1) + (j & 1); }
+__device__ __forceinline__ int frag_row_offset(int ri, int lane) { return 2 * (lane & 3) + 8 * (ri >> 1) + (ri & 1); }
+
+// Scales of the four rows a thread holds in the chunk at unit column c0
+// (0 for padding rows, whose results are never stored).
+template <bool GATHER>
+__device__ __forceinline__ void load_row_scales(const GemmArgs &a, const Unit &U, int c0, int lane, float (&rs)[4]) {
+#pragma unroll
+    for (int ri = 0; ri < 4; ++ri) {
+        const int row = unit_row(U, c0 + frag_row_offset(ri, lane));
+        float v = 0.0f;
+        if (row >= 0) {
+            if (GATHER) {
+                const int t = __ldg(a.src_token + row);
+                v = (unsigned)t < (unsigned)a.T ? __ldg(a.row_scale + t) : 0.0f;
+            } else {
+                v = __ldg(a.row_scale + row);
+            }
+        }
+        rs[ri] = v;
+    }
+}
+
+// Multiplies the 16 accumulator values of a chunk by their feature's and
+// row's scales (powers of two: exact).
+__device__ __forceinline__ void scale_frag(uint32_t (&r)[16], const float (&fs)[4], const float (&rs)[4]) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * fs[frag_fidx(j)] * rs[frag_ridx(j)]);
+}
+
+// Step 5 for one token t and one 128-feature block b, by 16 lanes (lane l of
+// the half-warp owns features 128 b + 8 l .. + 7): out[t] = bf16( sum_j
+// w[t,j] * y[dest_row[t,j]] ) in fp32, in slot order, each product and each
+// sum rounded on its own -- the arithmetic of the separate combine kernel, so
+// the results are identical.  The rows were stored by other warps and other
+// SMs: read through L2, all of them in flight at once (k <= 8 per pass).
+__device__ __forceinline__ void combine_block_half(const GemmArgs &a, int t, int b, int hl) {
+    const int H = a.n_out;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    const int *dr = a.dest_row + (size_t)t * a.k;
+    const float *wr = a.topk_w + (size_t)t * a.k;
+    for (int j0 = 0; j0 < a.k; j0 += 8) {
+        const int nj = min(8, a.k - j0);
+        uint4 v[8];
+        float w[8];
+        int r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            r[j] = j < nj ? __ldg(dr + j0 + j) : -1;
+            w[j] = j < nj ? __ldg(wr + j0 + j) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = (unsigned)r[j] < (unsigned)a.P
+                       ? __ldcg(reinterpret_cast<const uint4 *>(a.out + (size_t)r[j] * H + 128 * b + 8 * hl))
+                       : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if ((unsigned)r[j] >= (unsigned)a.P) continue;
+            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(p[i]);
+                acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w[j], f.x));
+                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(w[j], f.y));
+            }
+        }
+    }
+    uint4 o;
+    uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 pk = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        ow[i] = *reinterpret_cast<const uint32_t *>(&pk);
+    }
+    *reinterpret_cast<uint4 *>(a.comb_out + (size_t)t * H + 128 * b + 8 * hl) = o;
+}
+
+// After a warp has stored its pieces of a down-projection unit (its lane
+// quarter's 32 features of every 128-feature block, for its chunks of 16
+// rows): one arrival per (row, block), all issued before any result is used
+// (one round trip to L2); the warp whose arrival completes a token's block
+// combines it, two tokens at a time (one per half-warp).  Every lane fences
+// its own stores first, so a combining warp that sees the full count also sees
+// every piece of y.
+__device__ __forceinline__ void arrive_and_combine(const GemmArgs &a, const Unit &U, int sub, int lane) {
+    constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
+    __threadfence();
+    __syncwarp();
+    const int nblk = a.n_out / 128;
+    const int b0 = U.fx / 128;
+    int tok[kChunks];
+    int old[kChunks][2];
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int c0 = (sub + kEpiSub * i) * 16;
+        tok[i] = -1;
+        old[i][0] = old[i][1] = -1;
+        if (c0 < U.N && lane < 16) {
+            const int row = unit_row(U, c0 + lane);
+            if (row >= 0) {
+                const int t = __ldg(a.src_token + row);
+                if ((unsigned)t < (unsigned)a.T) {
+                    tok[i] = t;
+                    old[i][0] = atomicAdd(a.comb_cnt + (size_t)t * nblk + b0, 1);
+                    if (U.nacc == 2) old[i][1] = atomicAdd(a.comb_cnt + (size_t)t * nblk + b0 + 1, 1);
+                }
+            }
+        }
+    }
+    const int full = 4 * a.k - 1;
+    bool fenced = false;
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        for (int acc = 0; acc < U.nacc; ++acc) {
+            unsigned mask = __ballot_sync(0xffffffffu, old[i][acc] == full);
+            if (mask && !fenced) {
+                __threadfence();
+                fenced = true;
+            }
+            while (mask) {
+                const int sa = __ffs(mask) - 1;
+                mask &= mask - 1;
+                int sb = -1;
+                if (mask) {
+                    sb = __ffs(mask) - 1;
+                    mask &= mask - 1;
+                }
+                const int ta = __shfl_sync(0xffffffffu, tok[i], sa);
+                const int tb = __shfl_sync(0xffffffffu, tok[i], sb < 0 ? sa : sb);
+                const int t = lane < 16 ? ta : tb;
+                if (lane < 16 || sb >= 0) {
+                    combine_block_half(a, t, b0 + acc, lane & 15);
+                    if ((lane & 15) == 0) a.comb_cnt[(size_t)t * nblk + b0 + acc] = 0;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *status) {
     *abort = 1;
     atomicOr(status, MOE_DEV_GEMM_TIMEOUT);
@@ -312,11 +445,20 @@ __device__ __forceinline__ void raise_abort(volatile int *abort, uint32_t *statu
 // GATHER (mode 0 only): tmB maps the tokens x [T, H] with one-row boxes and
 // the token-tile producer gathers each unit's rows x[src_token[row]] with
 // tile::gather4 loads, so the permuted copy x_perm is never materialised.
-template <int MODE, bool GATHER = false>
+// FP8 (modes 0 and 1): weights and tokens are e4m3 codes, both K-major (the
+// weights stored [E][n_out][K]), 128 K per stage (still 128-byte rows), MMAs
+// of kind::f8f6f4; the epilogue multiplies each accumulator by its row's and
+// its feature's power-of-two scales (exact) before the bf16 results.
+// COMBINE (mode 1 only): the weighted combine of step 5 in the epilogue (see
+// arrive_and_combine).
+template <int MODE, bool GATHER = false, bool FP8 = false, bool COMBINE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ RowMaps tmB, GemmArgs a) {
     static_assert(!GATHER || MODE == 0, "the row gather feeds the SwiGLU GEMM");
+    static_assert(!COMBINE || MODE == 1, "the combine follows the down projection");
+    static_assert(!FP8 || MODE != 2, "the router runs on bf16 planes");
+    constexpr int kStageK = FP8 ? 128 : kBK;  // K elements per stage: 128 bytes of each row
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // SW128 tiles need 1 KiB alignment
@@ -334,56 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *s_rows = s_gts + 260;                             // GATHER: token of each row of the unit (<= 256)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int total, trows;
-    int num_fb = a.num_fb, fbw = MODE == 0 ? 128 : 256;
-    if (MODE == 2) {
-        total = (a.T + a.route_rows - 1) / a.route_rows * a.route_q;
-        trows = a.route_rows;
-    } else {
-        const int ntiles = *a.num_tiles;
-        const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
-        // Down projection with few row tiles: 128-feature units, twice as many,
-        // when they still fit one wave (otherwise 256-feature units, which read
-        // each token tile once for two accumulators).
-        if (MODE == 1 && nt * a.num_fb * 2 <= (int)gridDim.x) {
-            num_fb = a.n_out / 128;
-            fbw = 128;
-        }
-        total = nt * num_fb;
-        trows = *a.tile_rows;  // the schedule's row cap
-    }
-    // Balanced waves for the expert GEMMs: with R = ceil(total / grid) units
-    // for the busiest CTA, only ceil(total / R) CTAs take units (R or R - 1
-    // each), so the last round is not left to a few SMs while the rest idle
-    // (896 units on 148 SMs: 128 CTAs x 7 instead of 8 CTAs running a 7th).
-    const int rounds = (total + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int stride = MODE == 2 || rounds == 0 ? (int)gridDim.x : (total + rounds - 1) / rounds;
-    if ((int)blockIdx.x >= total || (int)blockIdx.x >= stride) return;  // uniform: this CTA has no work
-    // Two rings: weight stages (the A tiles of both accumulators; mode 2:
-    // three weight planes per accumulator), streamed from HBM, and token
-    // stages of trows rows (multiple of 16, <= 256).  Four token stages
-    // while that leaves at least four weight stages, else three; the weight
-    // ring takes the rest, so that as many weight bytes as possible are in
-    // flight.  Mode 2 reads both operands from L2 and consumes one stage of
-    // each per K block: equally deep rings.
-    trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
-    const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
-    const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)trows * kBRowBytes;
-    int nb = kMaxBStages;
-    int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    if (MODE == 2) {
-        nb = (int)(kRingBytes / (a_bytes + b_bytes));
-        nb = nb > kMaxBStages ? kMaxBStages : nb;
-        fit = nb;
-    } else if (fit < 4) {
-        nb = 3;
-        fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    }
-    const int na = fit > kMaxAStages ? kMaxAStages : fit;
-    uint8_t *ringB = smem + (uint32_t)na * a_bytes;  // a_bytes is a multiple of 16 KiB: 1 KiB aligned
-
-    if (MODE != 2)
-        for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
+    pdl_trigger();
+    // Set-up that reads nothing an earlier kernel writes: barriers, tensor-map
+    // prefetch, tensor memory (overlaps the previous kernel's tail when this
+    // kernel is launched as its programmatic dependent).
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxAStages; ++s) {
             mbar_init(&fullA[s], 1);
@@ -415,7 +511,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int nk = a.K / kBK;
+    pdl_wait();  // the schedule and the token rows come from earlier kernels
+    int total, trows;
+    int num_fb = a.num_fb, fbw = MODE == 0 ? 128 : 256;
+    if (MODE == 2) {
+        total = (a.T + a.route_rows - 1) / a.route_rows * a.route_q;
+        trows = a.route_rows;
+    } else {
+        const int ntiles = *a.num_tiles;
+        const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
+        // Down projection with few row tiles: 128-feature units, twice as many,
+        // when they still fit one wave (otherwise 256-feature units, which read
+        // each token tile once for two accumulators).
+        if (MODE == 1 && nt * a.num_fb * 2 <= (int)gridDim.x) {
+            num_fb = a.n_out / 128;
+            fbw = 128;
+        }
+        total = nt * num_fb;
+        trows = *a.tile_rows;  // the schedule's row cap
+    }
+    // Balanced waves for the expert GEMMs: with R = ceil(total / grid) units
+    // for the busiest CTA, only ceil(total / R) CTAs take units (R or R - 1
+    // each), so the last round is not left to a few SMs while the rest idle
+    // (896 units on 148 SMs: 128 CTAs x 7 instead of 8 CTAs running a 7th).
+    const int rounds = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int stride = MODE == 2 || rounds == 0 ? (int)gridDim.x : (total + rounds - 1) / rounds;
+    if ((int)blockIdx.x >= total || (int)blockIdx.x >= stride) {  // uniform: this CTA has no work
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem, kTmemCols);
+        }
+        return;
+    }
+    // Two rings: weight stages (the A tiles of both accumulators; mode 2:
+    // three weight planes per accumulator), streamed from HBM, and token
+    // stages of trows rows (multiple of 16, <= 256).  Four token stages
+    // while that leaves at least four weight stages, else three; the weight
+    // ring takes the rest, so that as many weight bytes as possible are in
+    // flight.  Mode 2 reads both operands from L2 and consumes one stage of
+    // each per K block: equally deep rings.
+    trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
+    const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
+    const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)trows * kBRowBytes;
+    int nb = kMaxBStages;
+    int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    if (MODE == 2) {
+        nb = (int)(kRingBytes / (a_bytes + b_bytes));
+        nb = nb > kMaxBStages ? kMaxBStages : nb;
+        fit = nb;
+    } else if (fit < 4) {
+        nb = 3;
+        fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
+    }
+    const int na = fit > kMaxAStages ? kMaxAStages : fit;
+    uint8_t *ringB = smem + (uint32_t)na * a_bytes;  // a_bytes is a multiple of 16 KiB: 1 KiB aligned
+
+    if (MODE != 2)
+        for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
+    __syncthreads();
+    const int nk = a.K / kStageK;
 
     if (GATHER && warp == 2) {
         // ------------------- token rows gathered from x by src_token (warp 2) ----
@@ -461,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&fullB[stage], bytes);
                     uint8_t *sb = ringB + stage * b_bytes;
-                    const int kx = kb * kBK;
+                    const int kx = kb * kStageK;
                     for (int g = 0; g < U.N; g += 4)
                         tma_gather4(sb + g * kBRowBytes, &tmB.m[0], &fullB[stage], kx, s_rows[g], s_rows[g + 1],
                                     s_rows[g + 2], s_rows[g + 3]);
@@ -526,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         continue;
                     }
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    const int ky = krow + kb * kBK, kx = kb * kBK;
+                    const int ky = krow + kb * kBK, kx = kb * kStageK;
                     if (!is_a) {
                         uint8_t *sb = ringB + stage * b_bytes;
                         tma_load_rows(sb, tmB, a.row_boxes, &full[stage], kx, U.p0s, 16 * nb0);
@@ -541,6 +697,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_2d(dst, &tmA0, &full[stage], c * 128, pl * a.K + kx);
                                 tma_load_2d(dst + kABox, &tmA0, &full[stage], c * 128 + 64, pl * a.K + kx);
                             }
+                    } else if (FP8) {
+                        // one 128-feature x 128-K box of codes per accumulator,
+                        // K-major ([E * n_out][K] bytes)
+                        uint8_t *sa0 = smem + stage * a_bytes;
+                        tma_load_2d(sa0, &tmA0, &full[stage], kx, U.e * a.n_out + fx0);
+                        if (U.nacc == 2) tma_load_2d(sa0 + kATile, &tmA1, &full[stage], kx, U.e * a.n_out + fx1);
                     } else {
                         uint8_t *sa0 = smem + stage * a_bytes, *sa1 = sa0 + kATile;
                         tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
@@ -579,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Unit U;
                 decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
                 if (!U.valid) continue;
-                const uint32_t idesc = idesc_bf16_f32(128, U.N, 1, 0);
+                const uint32_t idesc = FP8 ? idesc_e4m3_f32(128, U.N) : idesc_bf16_f32(128, U.N, 1, 0);
                 uint32_t h;
                 bool big;
                 plan.place(MODE == 2 ? 256 : U.N, h, big);  // mode 2 uses all of tensor memory
@@ -612,6 +774,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     const uint32_t accum = (j >= a.route_groups || kk || pl) ? 1u : 0u;
                                     tc_mma_bf16(dst, sdesc_sw128(at, kABox, 1024), bdesc, idesc, accum);
                                 }
+                        }
+                    } else if (FP8) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            // A and B K-major: 32 K (32 bytes) per MMA inside the 128-byte rows
+                            const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
+                            const uint32_t accum = (kb | kk) ? 1u : 0u;
+                            tc_mma_f8(d0, sdesc_sw128(sa0 + kk * 32, 16, 1024), bdesc, idesc, accum);
+                            if (U.nacc == 2) tc_mma_f8(d1, sdesc_sw128(sa1 + kk * 32, 16, 1024), bdesc, idesc, accum);
                         }
                     } else
 #pragma unroll
@@ -663,6 +834,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             Unit U;
             decode_unit<MODE>(u, s_gts, a, trows, num_fb, fbw, U);
             if (!U.valid) continue;
+            // FP8: the scales of this thread's four features in each accumulator
+            float fs0[4] = {1.0f, 1.0f, 1.0f, 1.0f}, fs1[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+            if (FP8) {
+                const size_t fb0 = (size_t)U.e * a.n_out + U.fx + q * 32 + (lane >> 2);
+                const size_t fb1 = MODE == 0 ? fb0 : fb0 + 128;
+#pragma unroll
+                for (int fi = 0; fi < 4; ++fi) {
+                    fs0[fi] = __ldg(a.w_scale0 + fb0 + 8 * fi);
+                    if (MODE == 0 || U.nacc == 2) fs1[fi] = __ldg(a.w_scale1 + fb1 + 8 * fi);
+                }
+            }
             uint32_t h;
             bool big;
             plan.place(MODE == 2 ? 256 : U.N, h, big);
@@ -718,24 +900,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             if (MODE == 1 && big) {
-                // Two accumulators of up to 256 columns do not fit in
-                // registers: store while holding the accumulator.
-                for (int c0 = sub * 16; c0 < U.N; c0 += 16 * kEpiSub) {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld_frag16(t0 + (uint32_t)c0, r0);
-                    if (U.nacc == 2) tmem_ld_frag16(t1 + (uint32_t)c0, r1);
-                    tmem_ld_wait();
-                    uint32_t w[8];
+                // Two accumulators of up to 256 columns each: accumulator 0 of
+                // every chunk and accumulator 1 of the first kHold1 chunks go to
+                // registers as packed bf16; the rest of accumulator 1 is stored
+                // while the accumulator is held.  Then the accumulator goes back
+                // to the MMA warp and the registers are stored, overlapping the
+                // next unit's MMAs (when every CTA stores its whole unit while
+                // holding it, the stores of all SMs collide and the tensor cores
+                // wait for them).
+                constexpr int kBigChunks = (16 + kEpiSub - 1) / kEpiSub;
+                constexpr int kHold1 = 1;
+                uint32_t h0[kBigChunks][8], h1[kHold1 > 0 ? kHold1 : 1][8];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r0[2 * m], r0[2 * m + 1]);
-                    store_block_frag(w, stg, a.out, a.n_out, U.fx + q * 32, U, c0);
-                    if (U.nacc == 2) {
+                for (int i = 0; i < kBigChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) {
+                        uint32_t r[16];
+                        float rs[4];
+                        if (FP8) load_row_scales<GATHER>(a, U, c0, lane, rs);
+                        tmem_ld_frag16(t0 + (uint32_t)c0, r);
+                        tmem_ld_wait();
+                        if (FP8) scale_frag(r, fs0, rs);
 #pragma unroll
-                        for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r1[2 * m], r1[2 * m + 1]);
-                        store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                        for (int m = 0; m < 8; ++m) h0[i][m] = pack_bf16x2(r[2 * m], r[2 * m + 1]);
+                    }
+                }
+                if (U.nacc == 2) {
+#pragma unroll
+                    for (int i = 0; i < kBigChunks; ++i) {
+                        const int c0 = (sub + kEpiSub * i) * 16;
+                        if (c0 < U.N) {
+                            uint32_t r[16];
+                            float rs[4];
+                            if (FP8) load_row_scales<GATHER>(a, U, c0, lane, rs);
+                            tmem_ld_frag16(t1 + (uint32_t)c0, r);
+                            tmem_ld_wait();
+                            if (FP8) scale_frag(r, fs1, rs);
+                            if (i < kHold1) {
+#pragma unroll
+                                for (int m = 0; m < 8; ++m) h1[i][m] = pack_bf16x2(r[2 * m], r[2 * m + 1]);
+                            } else {
+                                uint32_t w[8];
+#pragma unroll
+                                for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r[2 * m], r[2 * m + 1]);
+                                store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                            }
+                        }
                     }
                 }
                 release();
+#pragma unroll
+                for (int i = 0; i < kBigChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) {
+                        store_block_frag(h0[i], stg, a.out, a.n_out, U.fx + q * 32, U, c0);
+                        if (i < kHold1 && U.nacc == 2) store_block_frag(h1[i], stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                    }
+                }
+                if (COMBINE) arrive_and_combine(a, U, sub, lane);
                 plan.advance(big, h);
                 continue;
             }
@@ -751,16 +973,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c0 = (sub + kEpiSub * i) * 16;
                 if (c0 < U.N) {
                     uint32_t r0[16], r1[16];
+                    float rs[4];
+                    if (FP8) load_row_scales<GATHER>(a, U, c0, lane, rs);
                     tmem_ld_frag16(t0 + (uint32_t)c0, r0);
                     if (U.nacc == 2) tmem_ld_frag16(t1 + (uint32_t)c0, r1);
                     tmem_ld_wait();
+                    if (FP8) {
+                        scale_frag(r0, fs0, rs);
+                        if (U.nacc == 2) scale_frag(r1, fs1, rs);
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
                         if (MODE == 0) {
                             const float g0 = __uint_as_float(r0[j]), v0 = __uint_as_float(r1[j]);
                             const float g1 = __uint_as_float(r0[j + 1]), v1 = __uint_as_float(r1[j + 1]);
-                            const __nv_bfloat162 p = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * v0,
-                                                                           __fdividef(g1, 1.0f + __expf(-g1)) * v1);
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(silu_f(g0) * v0, silu_f(g1) * v1);
                             hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&p);
                         } else {
                             const __nv_bfloat162 p0 =
@@ -793,6 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if (COMBINE) arrive_and_combine(a, U, sub, lane);
             plan.advance(big, h);
         }
     }
@@ -805,346 +1033,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------------------
-// Pairs of CTAs sharing one MMA (tcgen05 cta_group::2), modes 0 and 1.
-// A cluster of two CTAs takes units (expert group, 256-feature block, row
-// tile): CTA r of the pair holds the weights of features [256 fb + 128 r, +128)
-// (the MMA's M = 256 is split by CTA) and rows [r N/2, (r+1) N/2) of the token
-// tile (N split by CTA), so each CTA streams only half of every token tile.
-// Both CTAs' copies complete on the leader's (rank 0) barriers, which count
-// both halves' bytes; the leader alone issues the MMAs and multicasts their
-// commits to both CTAs' stage and accumulator barriers; each CTA drains its
-// own tensor memory (its 128 features for all N rows) and hands it back by
-// arriving on the leader's barrier.  Mode 0 keeps gate and up for the CTA's
-// 128 features (two accumulators); mode 1 one accumulator of up to 256
-// columns, so its units always alternate between the tensor-memory halves.
-// Selected by MOE_FLAG_GEMM_PAIRS.  Measured on B200 it is not faster than the
-// single-CTA kernel for the shapes of this library's benchmarks (the
-// weight-streaming shapes stream no faster per SM with the deeper weight ring
-// it allows, and the down projection of a 128-unit layer loses half of its
-// per-CTA rate), so it is off by default.
-constexpr int kPairMaxAStages = 12;
-constexpr int kPairMaxBStages = 8;
-
-// Rows [row0, row0 + n) (n a multiple of 8, <= 128) of the token matrix into
-// this CTA's shared memory from dst, completing on the leader's barrier;
-// boxes of 128, 64, 32, 16 and 8 rows (RowMaps with heights 8 << i), largest
-// first.
-__device__ __forceinline__ void tma_load_rows_pair(uint8_t *dst, const RowMaps &rm, uint32_t boxes, uint32_t bar,
-                                                   int kx, int row0, int n) {
-#pragma unroll
-    for (int i = kRowBoxes - 1; i >= 0; --i) {
-        const int h = 8 << i;
-        if (!((boxes >> i) & 1u)) continue;
-        while (n >= h) {
-            tma_load_2d_pair(dst, &rm.m[i], bar, kx, row0);
-            dst += h * kBRowBytes;
-            row0 += h;
-            n -= h;
-        }
-    }
-}
-
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) __cluster_dims__(2, 1, 1)
-    k_grouped_gemm_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ RowMaps tmB, GemmArgs a) {
-    static_assert(MODE == 0 || MODE == 1, "pairs run the expert GEMMs");
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    uint8_t *ctrl = smem + kRingBytes;
-    uint64_t *fullA = reinterpret_cast<uint64_t *>(ctrl);
-    uint64_t *emptyA = fullA + kPairMaxAStages;
-    uint64_t *fullB = emptyA + kPairMaxAStages;
-    uint64_t *emptyB = fullB + kPairMaxBStages;
-    uint64_t *tfull = emptyB + kPairMaxBStages;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *mma_done = tempty + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
-    volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *s_gts = reinterpret_cast<int *>(tmem_slot + 2);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const bool leader = rank == 0;
-    const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
-    const int ntiles = *a.num_tiles;
-    const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
-    const int num_fb = (a.n_out + 255) / 256;
-    const int total = nt * num_fb;
-    if (pair >= total) return;  // uniform over the pair: neither CTA has work
-    int trows = *a.tile_rows;
-    trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
-    const uint32_t a_tiles = MODE == 0 ? 2u : 1u;
-    const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)(trows / 2) * kBRowBytes;
-    // Both rings equally deep (a pipeline stage waits for its weight and its
-    // token tile alike, and both can come from HBM), then the rest of shared
-    // memory for more weight stages.
-    int nb = (int)(kRingBytes / (a_bytes + b_bytes));
-    nb = nb > kPairMaxBStages ? kPairMaxBStages : (nb < 2 ? 2 : nb);
-    int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
-    const int na = fit > kPairMaxAStages ? kPairMaxAStages : fit;
-    uint8_t *ringB = smem + (uint32_t)na * a_bytes;
-
-    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_gts[i] = a.grp_tile_start[i];
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kPairMaxAStages; ++s) {
-            mbar_init(&fullA[s], 1);
-            mbar_init(&emptyA[s], 1);
-        }
-        for (int s = 0; s < kPairMaxBStages; ++s) {
-            mbar_init(&fullB[s], 1);
-            mbar_init(&emptyB[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 2 * kEpiWarps);  // both CTAs' epilogue warps (the leader's count)
-        }
-        mbar_init(mma_done, 1);
-        *s_abort = 0;
-        mbar_fence_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA0);
-        tma_prefetch_desc(&tmA1);
-        for (int b = 0; b < kRowBoxes; ++b)
-            if ((a.row_boxes >> b) & 1u) tma_prefetch_desc(&tmB.m[b]);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(tmem_slot, kTmemCols);
-        tmem_relinquish_pair();
-    }
-    tc_fence_before();
-    cluster_arrive_wait();  // both CTAs' barriers are initialised before any remote use
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const int nk = a.K / kBK;
-
-    if (warp == 0 || warp == 2) {
-        // ------------- TMA producers (both CTAs): warp 0 weights, warp 2 token rows ----
-        if (lane == 0) {
-            const bool is_a = warp == 0;
-            const int nst = is_a ? na : nb;
-            uint64_t *full = is_a ? fullA : fullB;
-            uint64_t *empty = is_a ? emptyA : emptyB;
-            const uint32_t full_leader = mapa_shared(full, 0);  // the leader's barrier array
-            int stage = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int u = pair; u < total && ok; u += npairs) {
-                Unit U;
-                decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
-                if (!U.valid) {
-                    if (is_a && leader) atomicOr(a.status, MOE_DEV_BAD_ROW);
-                    continue;
-                }
-                const int fx = U.fx + 128 * (int)rank;  // this CTA's first feature
-                const int half_rows = U.N / 2;          // rows of the token tile this CTA holds
-                const uint32_t my_bytes = is_a ? a_tiles * kATile : (uint32_t)half_rows * kBRowBytes;
-                const int krow = U.e * a.K;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, a.timeout_ns, s_abort)) {
-                        ok = false;
-                        break;
-                    }
-                    // the leader expects both CTAs' bytes of this stage
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * my_bytes);
-                    const uint32_t bar = full_leader + 8u * (uint32_t)stage;
-                    const int ky = krow + kb * kBK, kx = kb * kBK;
-                    if (is_a) {
-                        uint8_t *sa0 = smem + stage * a_bytes;
-                        tma_load_2d_pair(sa0, &tmA0, bar, fx, ky);
-                        tma_load_2d_pair(sa0 + kABox, &tmA0, bar, fx + 64, ky);
-                        if (MODE == 0) {
-                            tma_load_2d_pair(sa0 + kATile, &tmA1, bar, fx, ky);
-                            tma_load_2d_pair(sa0 + kATile + kABox, &tmA1, bar, fx + 64, ky);
-                        }
-                    } else {
-                        // tile rows [rank * N/2, (rank + 1) * N/2): the part in
-                        // row piece 0 (tile rows [0, n0p)), then the part in
-                        // piece 1 (all lengths multiples of 8)
-                        uint8_t *sb = ringB + stage * b_bytes;
-                        const int cb = (int)rank * half_rows, ce = cb + half_rows;
-                        const int l0 = max(0, min(ce, U.n0p) - cb);
-                        const int c1 = max(cb, U.n0p);
-                        if (l0) tma_load_rows_pair(sb, tmB, a.row_boxes, bar, kx, U.p0s + cb, l0);
-                        if (ce > c1) tma_load_rows_pair(sb + l0 * kBRowBytes, tmB, a.row_boxes, bar, kx,
-                                                        U.p1s + (c1 - U.n0p), ce - c1);
-                    }
-                    if (++stage == nst) {
-                        stage = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
-            if (!ok && !*s_abort) raise_abort(s_abort, a.status);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------- MMA issuer (the leader only) ----
-        if (lane == 0 && leader) {
-            int sa = 0, sb = 0;
-            uint32_t pha = 0, phb = 0;
-            TmemPlan plan;
-            const uint32_t baseA = smem_u32(smem), baseB = smem_u32(ringB);
-            bool ok = true;
-            for (int u = pair; u < total && ok; u += npairs) {
-                Unit U;
-                decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
-                if (!U.valid) continue;
-                const uint32_t idesc = idesc_bf16_f32(256, U.N, 1, 0);
-                uint32_t h;
-                bool big;
-                plan.place(MODE == 0 ? U.N : 0, h, big);  // mode 1: one accumulator fits a half
-                const uint32_t d0 = tmem + h * 256u, d1 = big ? tmem + 256u : d0 + 128u;
-                ok = mbar_wait_bounded(&tempty[h], (plan.uses[h] & 1u) ^ 1u, a.timeout_ns, s_abort);
-                if (ok && big) ok = mbar_wait_bounded(&tempty[1], (plan.uses[1] & 1u) ^ 1u, a.timeout_ns, s_abort);
-                if (!ok) break;
-                tc_fence_after();
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait_bounded(&fullA[sa], pha, a.timeout_ns, s_abort) ||
-                        !mbar_wait_bounded(&fullB[sb], phb, a.timeout_ns, s_abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sa0 = baseA + sa * a_bytes, sa1 = sa0 + kATile, sbt = baseB + sb * b_bytes;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t bdesc = sdesc_sw128(sbt + kk * 32, 16, 1024);
-                        const uint32_t accum = (kb | kk) ? 1u : 0u;
-                        tc_mma_bf16_pair(d0, sdesc_sw128(sa0 + kk * 2048, kABox, 1024), bdesc, idesc, accum);
-                        if (MODE == 0)
-                            tc_mma_bf16_pair(d1, sdesc_sw128(sa1 + kk * 2048, kABox, 1024), bdesc, idesc, accum);
-                    }
-                    tc_commit_pair(&emptyA[sa], 3);  // both CTAs' stages are free once read
-                    tc_commit_pair(&emptyB[sb], 3);
-                    if (++sa == na) {
-                        sa = 0;
-                        pha ^= 1u;
-                    }
-                    if (++sb == nb) {
-                        sb = 0;
-                        phb ^= 1u;
-                    }
-                }
-                if (!ok) break;
-                tc_commit_pair(&tfull[h], 3);
-                if (big) tc_commit_pair(&tfull[1], 3);
-                plan.advance(big, h);
-            }
-            if (!ok && !*s_abort) raise_abort(s_abort, a.status);
-            int never = 0;
-            tc_commit_pair(mma_done, 1);
-            mbar_wait_bounded(mma_done, 0, a.timeout_ns, &never);
-        }
-        __syncwarp();
-    } else {
-        // -------------------------------------------- epilogue (both CTAs) ----
-        const int q = warp & 3;
-        const int sub = (warp - kEpiWarp0) >> 2;
-        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t tempty_leader = mapa_shared(tempty, 0);
-        TmemPlan plan;
-        for (int u = pair; u < total; u += npairs) {
-            Unit U;
-            decode_unit<MODE>(u, s_gts, a, trows, num_fb, 256, U);
-            if (!U.valid) continue;
-            uint32_t h;
-            bool big;
-            plan.place(MODE == 0 ? U.N : 0, h, big);
-            bool got = mbar_wait_bounded(&tfull[h], plan.uses[h] & 1u, a.timeout_ns, s_abort);
-            if (got && big) got = mbar_wait_bounded(&tfull[1], plan.uses[1] & 1u, a.timeout_ns, s_abort);
-            if (!__all_sync(0xffffffffu, got)) {
-                if (lane == 0 && !*s_abort) raise_abort(s_abort, a.status);
-                break;
-            }
-            tc_fence_after();
-            const uint32_t t0 = tq + h * 256u, t1 = big ? tq + 256u : t0 + 128u;
-            auto release = [&]() {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_cluster(tempty_leader + 8u * h);
-                    if (big) mbar_arrive_cluster(tempty_leader + 8u);
-                }
-            };
-            const int fb0 = U.fx + 128 * (int)rank + q * 32;  // this warp's first feature
-            const bool inside = fb0 < a.n_out;  // the last block may have no second half (warp-uniform)
-            if (MODE == 1) {
-                // one accumulator of up to 256 columns: hold up to 4 chunks per warp
-                constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
-                uint32_t hold[kChunks][8];
-#pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N) {
-                        uint32_t r0[16];
-                        tmem_ld16(t0 + (uint32_t)c0, r0);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 16; j += 2) {
-                            const __nv_bfloat162 pk =
-                                __floats2bfloat162_rn(__uint_as_float(r0[j]), __uint_as_float(r0[j + 1]));
-                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&pk);
-                        }
-                    }
-                }
-                release();
-#pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N && inside) store_block_32x16(hold[i], a.out, a.n_out, fb0, U, c0);
-                }
-            } else {
-                constexpr int kChunks = (16 + kEpiSub - 1) / kEpiSub;
-                uint32_t hold[kChunks][8];
-#pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N) {
-                        uint32_t r0[16], r1[16];
-                        tmem_ld16(t0 + (uint32_t)c0, r0);
-                        tmem_ld16(t1 + (uint32_t)c0, r1);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 16; j += 2) {
-                            const float g0 = __uint_as_float(r0[j]), v0 = __uint_as_float(r1[j]);
-                            const float g1 = __uint_as_float(r0[j + 1]), v1 = __uint_as_float(r1[j + 1]);
-                            const __nv_bfloat162 pk = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * v0,
-                                                                            __fdividef(g1, 1.0f + __expf(-g1)) * v1);
-                            hold[i][j / 2] = *reinterpret_cast<const uint32_t *>(&pk);
-                        }
-                    }
-                }
-                release();
-#pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N && inside) store_block_32x16(hold[i], a.out, a.n_out, fb0, U, c0);
-                }
-            }
-            plan.advance(big, h);
-        }
-    }
-
-    // Neither CTA leaves (or frees tensor memory) while the other may still
-    // read its shared memory, write its tensor memory or signal its barriers.
-    tc_fence_before();
-    __syncthreads();
-    cluster_arrive_wait();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem, kTmemCols);
-    }
-}
-
 // Exact three-way bf16 split of the router weights: p0 = bf16(w),
 // p1 = bf16(w - p0), p2 = bf16(w - p0 - p1) (each difference is exact in
 // fp32), written as planes[3][H][Ep]; columns e >= E are zero.
 __global__ void __launch_bounds__(256) k_router_planes(const float *__restrict__ w, __nv_bfloat16 *__restrict__ planes,
                                                        int H, int E, int Ep) {
+    pdl_trigger();
     const size_t n = (size_t)H * Ep;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         const int h = (int)(i / Ep), e = (int)(i % Ep);
@@ -1171,17 +1065,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix with the 128-byte
-// swizzle; box = box_cols x box_rows (box_cols * 2 bytes must be 128).
+// 2-D tensor map over a row-major [rows, cols] matrix of bf16 (or, with
+// bytes = true, of 8-bit codes) with the 128-byte swizzle; box = box_cols x
+// box_rows (box_cols elements must span 128 bytes).
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_cols,
-               uint32_t box_rows) {
+               uint32_t box_rows, bool bytes = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
+    cuuint64_t strides[1] = {cols * (bytes ? 1 : 2)};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+    const CUresult r = fn(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void *>(ptr), dims, strides, box, es,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -1189,10 +1085,11 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
 
 // The token matrix with boxes of 16, 32, ... 256 rows; returns the mask of the
 // maps that could be encoded (bit 0 is required).
-uint32_t make_row_maps(RowMaps *rm, const void *ptr, uint64_t rows, uint64_t cols, uint32_t min_rows = 16) {
+uint32_t make_row_maps(RowMaps *rm, const void *ptr, uint64_t rows, uint64_t cols, uint32_t min_rows = 16,
+                       bool bytes = false) {
     uint32_t boxes = 0;
     for (int i = 0; i < kRowBoxes; ++i)
-        if (make_tmap(&rm->m[i], ptr, rows, cols, 64, min_rows << i)) boxes |= 1u << i;
+        if (make_tmap(&rm->m[i], ptr, rows, cols, bytes ? 128 : 64, min_rows << i, bytes)) boxes |= 1u << i;
     return (boxes & 1u) ? boxes : 0u;
 }
 
@@ -1239,20 +1136,17 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
         attr_done = true;
     }
     *q = plan.q;
-    k_grouped_gemm<2><<<num_sms, kThreads, kSmemBytes, stream>>>(tA, tA, tB, a);
-    return cudaGetLastError();
+    return launch_pdl(k_grouped_gemm<2>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA, tA, tB, a);
 }
 
 // mode 0: act = x_perm [P,H], w0 = gate, w1 = up, out = h [P,F]
 //         (with src_token: act = x [T,H], rows gathered as x[src_token[row]])
 // mode 1: act = h [P,F],      w0 = w1 = down,   out = y [P,H]
+// comb (mode 1, nullable): the combine of step 5 in the epilogue, into comb->out.
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream, const int32_t *src_token) {
+                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb) {
     const bool gather = mode == 0 && src_token != nullptr;
-    // Pairs of CTAs sharing one MMA for the expert GEMMs, on request (not for
-    // the row gather).
-    const bool pairs = (s.flags & MOE_FLAG_GEMM_PAIRS) && !gather && num_sms >= 2;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
     const int K = mode == 0 ? s.H : s.F;
@@ -1266,8 +1160,6 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     if (gather) {
         if (!make_tmap(&tB.m[0], act, (uint64_t)s.T, (uint64_t)K, 64, 1)) return cudaErrorInvalidValue;
         boxes = 1u;
-    } else if (pairs) {
-        if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K, 8))) return cudaErrorInvalidValue;
     } else if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K))) {
         return cudaErrorInvalidValue;
     }
@@ -1290,27 +1182,23 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.src_token = src_token;
     a.row_boxes = boxes;
     a.stall_first_stage = (mode == 0 && !gather && (s.flags & MOE_FLAG_TEST_STALL_GEMM)) ? 1 : 0;
-    static bool attr_done[5] = {false, false, false, false, false};
+    static bool attr_done[6] = {false, false, false, false, false, false};
     cudaError_t err;
-    if (pairs) {
-        const int grid = num_sms & ~1;
-        if (mode == 0) {
-            if (!attr_done[3]) {
-                err = cudaFuncSetAttribute(k_grouped_gemm_pair<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kSmemBytes);
-                if (err != cudaSuccess) return err;
-                attr_done[3] = true;
-            }
-            k_grouped_gemm_pair<0><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
-        } else {
-            if (!attr_done[4]) {
-                err = cudaFuncSetAttribute(k_grouped_gemm_pair<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kSmemBytes);
-                if (err != cudaSuccess) return err;
-                attr_done[4] = true;
-            }
-            k_grouped_gemm_pair<1><<<grid, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+    if (mode == 1 && comb) {
+        a.src_token = comb->src_token;
+        a.dest_row = comb->dest_row;
+        a.topk_w = comb->topk_w;
+        a.comb_out = (__nv_bfloat16 *)comb->out;
+        a.comb_cnt = (int *)((char *)ws + L.combine_cnt);
+        a.k = s.k;
+        if (!attr_done[5]) {
+            err = cudaFuncSetAttribute(k_grouped_gemm<1, false, false, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (err != cudaSuccess) return err;
+            attr_done[5] = true;
         }
+        err = launch_pdl(k_grouped_gemm<1, false, false, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
     } else if (gather) {
         if (!attr_done[2]) {
             err = cudaFuncSetAttribute(k_grouped_gemm<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1318,21 +1206,104 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
             if (err != cudaSuccess) return err;
             attr_done[2] = true;
         }
-        k_grouped_gemm<0, true><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+        err = launch_pdl(k_grouped_gemm<0, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
     } else if (mode == 0) {
         if (!attr_done[0]) {
             err = cudaFuncSetAttribute(k_grouped_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (err != cudaSuccess) return err;
             attr_done[0] = true;
         }
-        k_grouped_gemm<0><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+        err = launch_pdl(k_grouped_gemm<0>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
     } else {
         if (!attr_done[1]) {
             err = cudaFuncSetAttribute(k_grouped_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (err != cudaSuccess) return err;
             attr_done[1] = true;
         }
-        k_grouped_gemm<1><<<num_sms, kThreads, kSmemBytes, stream>>>(tA0, tA1, tB, a);
+        err = launch_pdl(k_grouped_gemm<1>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
+    }
+    return cudaGetLastError();
+}
+
+// FP8 expert GEMMs.  mode 0: act = the e4m3 token rows (x_perm codes [P,H],
+// or with src_token the per-token codes [T,H] gathered by row), w0/w1 = gate/
+// up codes [E][F][H] with scales [E][F]; mode 1: act = h codes [P,F], w0 = w1
+// = down codes [E][H][F] with scales [E][H].  row_scale: one per row of act.
+cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *act, const float *row_scale,
+                                    const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
+                                    void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb) {
+    const bool gather = mode == 0 && src_token != nullptr;
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
+    const int K = mode == 0 ? s.H : s.F;
+    const int n_out = mode == 0 ? s.F : s.H;
+    CUtensorMap tA0, tA1;
+    RowMaps tB;
+    uint32_t boxes = 0;
+    if (!make_tmap(&tA0, w0, (uint64_t)s.E * n_out, (uint64_t)K, 128, 128, true) ||
+        !make_tmap(&tA1, w1, (uint64_t)s.E * n_out, (uint64_t)K, 128, 128, true))
+        return cudaErrorInvalidValue;
+    if (gather) {
+        if (!make_tmap(&tB.m[0], act, (uint64_t)s.T, (uint64_t)K, 128, 1, true)) return cudaErrorInvalidValue;
+        boxes = 1u;
+    } else if (!(boxes = make_row_maps(&tB, act, (uint64_t)P, (uint64_t)K, 16, true))) {
+        return cudaErrorInvalidValue;
+    }
+    WsPtrs p = ws_ptrs(ws, L);
+    GemmArgs a = {};
+    a.tile_map = p.tile_map;
+    a.grp_tile_start = p.grp_tile_start;
+    a.num_tiles = p.num_tiles;
+    a.tile_rows = p.tile_rows;
+    a.status = p.status;
+    a.out = (__nv_bfloat16 *)out;
+    a.n_out = n_out;
+    a.K = K;
+    a.num_fb = mode == 0 ? s.F / 128 : (s.H + 255) / 256;
+    a.E = s.E;
+    a.P = (int)P;
+    a.max_tiles = L.max_tiles;
+    a.timeout_ns = timeout_ns;
+    a.T = s.T;
+    a.src_token = src_token;
+    a.row_boxes = boxes;
+    a.w_scale0 = w0_scale;
+    a.w_scale1 = w1_scale;
+    a.row_scale = row_scale;
+    static bool attr_done[4] = {false, false, false, false};
+    cudaError_t err;
+    auto setup = [&](const void *fn, int i) -> cudaError_t {
+        if (attr_done[i]) return cudaSuccess;
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e == cudaSuccess) attr_done[i] = true;
+        return e;
+    };
+    if (mode == 1 && comb) {
+        a.src_token = comb->src_token;
+        a.dest_row = comb->dest_row;
+        a.topk_w = comb->topk_w;
+        a.comb_out = (__nv_bfloat16 *)comb->out;
+        a.comb_cnt = (int *)((char *)ws + L.combine_cnt);
+        a.k = s.k;
+        if ((err = setup((const void *)k_grouped_gemm<1, false, true, true>, 3)) != cudaSuccess) return err;
+        err = launch_pdl(k_grouped_gemm<1, false, true, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
+    } else if (gather) {
+        if ((err = setup((const void *)k_grouped_gemm<0, true, true>, 0)) != cudaSuccess) return err;
+        err = launch_pdl(k_grouped_gemm<0, true, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
+    } else if (mode == 0) {
+        if ((err = setup((const void *)k_grouped_gemm<0, false, true>, 1)) != cudaSuccess) return err;
+        err = launch_pdl(k_grouped_gemm<0, false, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
+    } else {
+        if ((err = setup((const void *)k_grouped_gemm<1, false, true>, 2)) != cudaSuccess) return err;
+        err = launch_pdl(k_grouped_gemm<1, false, true>, dim3(num_sms), dim3(kThreads), kSmemBytes, stream, tA0, tA1, tB, a);
+        if (err != cudaSuccess) return err;
     }
     return cudaGetLastError();
 }

@@ -2,6 +2,7 @@
 // workspace carving and kernel launches.  No entry point allocates, frees or
 // synchronises except moe_read_status.
 #include <atomic>
+#include <climits>
 #include <cstdint>
 #include <cstdio>
 
@@ -21,9 +22,19 @@ cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *top
                            void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream, const int32_t *src_token);
+                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr);
 cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
                            cudaStream_t stream);
+cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *act, const float *row_scale,
+                                    const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
+                                    void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
+                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr);
+cudaError_t launch_quant_weights(int E, int K, int N, const void *w, void *q, float *scale, cudaStream_t stream);
+cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int src_rows, const int32_t *idx,
+                              bool gather, void *q, float *scale, const WsLayout &L, void *ws, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_quant_tokens(const moe_shape &s, const void *x, void *q, float *scale, int num_sms,
+                                cudaStream_t stream);
 }  // namespace moe
 
 using namespace moe;
@@ -33,8 +44,8 @@ namespace {
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 thread_local char g_last_error[160] = "no error";
 
-constexpr uint32_t kKnownFlags =
-    MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FLAG_GEMM_PAIRS | MOE_FLAG_TEST_STALL_SCAN | MOE_FLAG_TEST_STALL_GEMM;
+constexpr uint32_t kKnownFlags = MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FLAG_FUSED_COMBINE |
+                                  MOE_FLAG_TEST_STALL_SCAN | MOE_FLAG_TEST_STALL_GEMM;
 
 bool aligned(const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
 
@@ -221,6 +232,24 @@ moe_status moe_grouped_down(const moe_shape *s, const void *h, const void *w_dow
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down");
 }
 
+moe_status moe_grouped_down_combine(const moe_shape *s, const void *h, const void *w_down, const int32_t *src_token,
+                                    const int32_t *dest_row, const float *topk_w, void *y, void *out, void *ws,
+                                    void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(h, 16) || !aligned(w_down, 16) || !aligned(y, 16) || !aligned(out, 16) || !aligned(src_token, 4) ||
+        !aligned(dest_row, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    const CombineOut comb{src_token, dest_row, topk_w, out};
+    cudaError_t e = launch_grouped_gemm(1, *s, h, w_down, w_down, y, L, ws, g_timeout_ns.load(), sms,
+                                        (cudaStream_t)stream, nullptr, &comb);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down_combine");
+}
+
 moe_status moe_combine(const moe_shape *s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
                        void *stream) {
     moe_status st = check_shape(s);
@@ -298,7 +327,125 @@ moe_status moe_forward(const moe_shape *s, const moe_forward_args *a, void *ws, 
         st = moe_grouped_swiglu_gather(s, a->x, a->src_token, a->w_gate, a->w_up, a->h, ws, stream);
     }
     if (st != MOE_OK) return st;
+    if (s->flags & MOE_FLAG_FUSED_COMBINE)
+        return moe_grouped_down_combine(s, a->h, a->w_down, a->src_token, a->dest_row, a->topk_w, a->y, a->out, ws,
+                                        stream);
     st = moe_grouped_down(s, a->h, a->w_down, a->y, ws, stream);
+    if (st != MOE_OK) return st;
+    return moe_combine(s, a->y, a->dest_row, a->topk_w, a->out, stream);
+}
+
+moe_status moe_quantize_weights_fp8(const moe_shape *s, int which, const void *w, void *w_q, float *w_scale,
+                                    void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if ((which != MOE_WEIGHTS_GATE_UP && which != MOE_WEIGHTS_DOWN) || !aligned(w, 16) || !aligned(w_q, 16) ||
+        !aligned(w_scale, 4))
+        return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const int K = which == MOE_WEIGHTS_GATE_UP ? s->H : s->F;
+    const int N = which == MOE_WEIGHTS_GATE_UP ? s->F : s->H;
+    cudaError_t e = launch_quant_weights(s->E, K, N, w, w_q, w_scale, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_quantize_weights_fp8");
+}
+
+moe_status moe_quantize_rows_fp8(const moe_shape *s, int which, const void *src, const int32_t *src_token, void *q,
+                                 float *scale, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (which != MOE_ROWS_X_PERM && which != MOE_ROWS_TOKENS && which != MOE_ROWS_H) return MOE_ERR_INVALID_ARG;
+    if (!aligned(src, 16) || !aligned(q, 16) || !aligned(scale, 4)) return MOE_ERR_INVALID_ARG;
+    if (which != MOE_ROWS_TOKENS && !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
+    if (which != MOE_ROWS_TOKENS && (st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e;
+    if (which == MOE_ROWS_TOKENS) {
+        e = launch_quant_tokens(*s, src, q, scale, sms, (cudaStream_t)stream);
+    } else {
+        const WsLayout L = layout_of(s);
+        const bool xp = which == MOE_ROWS_X_PERM;
+        e = launch_quant_rows(*s, xp ? s->H : s->F, src, xp ? s->T : INT32_MAX, src_token, xp, q, scale, L, ws, sms,
+                              (cudaStream_t)stream);
+    }
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_quantize_rows_fp8");
+}
+
+moe_status moe_grouped_swiglu_fp8(const moe_shape *s, const void *x_q, const float *x_scale, const int32_t *src_token,
+                                  const void *wg_q, const float *wg_scale, const void *wu_q, const float *wu_scale,
+                                  void *h, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(x_q, 16) || !aligned(x_scale, 4) || !aligned(wg_q, 16) || !aligned(wg_scale, 4) ||
+        !aligned(wu_q, 16) || !aligned(wu_scale, 4) || !aligned(h, 16))
+        return MOE_ERR_INVALID_ARG;
+    if (src_token && !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_grouped_gemm_fp8(0, *s, x_q, x_scale, wg_q, wg_scale, wu_q, wu_scale, h, L, ws,
+                                            g_timeout_ns.load(), sms, (cudaStream_t)stream, src_token);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_swiglu_fp8");
+}
+
+moe_status moe_grouped_down_fp8(const moe_shape *s, const void *h_q, const float *h_scale, const void *wd_q,
+                                const float *wd_scale, void *y, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(h_q, 16) || !aligned(h_scale, 4) || !aligned(wd_q, 16) || !aligned(wd_scale, 4) || !aligned(y, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_grouped_gemm_fp8(1, *s, h_q, h_scale, wd_q, wd_scale, wd_q, wd_scale, y, L, ws,
+                                            g_timeout_ns.load(), sms, (cudaStream_t)stream, nullptr);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down_fp8");
+}
+
+moe_status moe_grouped_down_fp8_combine(const moe_shape *s, const void *h_q, const float *h_scale, const void *wd_q,
+                                        const float *wd_scale, const int32_t *src_token, const int32_t *dest_row,
+                                        const float *topk_w, void *y, void *out, void *ws, void *stream) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!aligned(h_q, 16) || !aligned(h_scale, 4) || !aligned(wd_q, 16) || !aligned(wd_scale, 4) || !aligned(y, 16) ||
+        !aligned(out, 16) || !aligned(src_token, 4) || !aligned(dest_row, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    const CombineOut comb{src_token, dest_row, topk_w, out};
+    cudaError_t e = launch_grouped_gemm_fp8(1, *s, h_q, h_scale, wd_q, wd_scale, wd_q, wd_scale, y, L, ws,
+                                            g_timeout_ns.load(), sms, (cudaStream_t)stream, nullptr, &comb);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_grouped_down_fp8_combine");
+}
+
+moe_status moe_forward_fp8(const moe_shape *s, const moe_forward_fp8_args *a, void *ws, void *stream) {
+    if (!a) return MOE_ERR_INVALID_ARG;
+    moe_status st = moe_route_dispatch(s, a->x, a->w_router, a->bias, a->logits, a->topk_idx, a->topk_w,
+                                       a->expert_counts, a->expert_offsets, a->src_token, a->dest_row, ws, stream);
+    if (st != MOE_OK) return st;
+    if (a->x_q_per_token) {
+        st = moe_quantize_rows_fp8(s, MOE_ROWS_TOKENS, a->x, nullptr, a->x_q, a->x_scale, ws, stream);
+        if (st != MOE_OK) return st;
+        st = moe_grouped_swiglu_fp8(s, a->x_q, a->x_scale, a->src_token, a->wg_q, a->wg_scale, a->wu_q, a->wu_scale,
+                                    a->h, ws, stream);
+    } else {
+        st = moe_quantize_rows_fp8(s, MOE_ROWS_X_PERM, a->x, a->src_token, a->x_q, a->x_scale, ws, stream);
+        if (st != MOE_OK) return st;
+        st = moe_grouped_swiglu_fp8(s, a->x_q, a->x_scale, nullptr, a->wg_q, a->wg_scale, a->wu_q, a->wu_scale, a->h,
+                                    ws, stream);
+    }
+    if (st != MOE_OK) return st;
+    st = moe_quantize_rows_fp8(s, MOE_ROWS_H, a->h, a->src_token, a->h_q, a->h_scale, ws, stream);
+    if (st != MOE_OK) return st;
+    if (s->flags & MOE_FLAG_FUSED_COMBINE)
+        return moe_grouped_down_fp8_combine(s, a->h_q, a->h_scale, a->wd_q, a->wd_scale, a->src_token, a->dest_row,
+                                            a->topk_w, a->y, a->out, ws, stream);
+    st = moe_grouped_down_fp8(s, a->h_q, a->h_scale, a->wd_q, a->wd_scale, a->y, ws, stream);
     if (st != MOE_OK) return st;
     return moe_combine(s, a->y, a->dest_row, a->topk_w, a->out, stream);
 }

@@ -1,0 +1,286 @@
+// fp8 (e4m3) operands of the expert GEMMs ("TEMPO" verdict page, arXiv
+// 2608.13057, referee report summary: the per-expert cost law is measured on
+// an fp8 grouped GEMM, whose flat regime streams the expert's weights from
+// HBM, so 8-bit weights halve the bytes that bound it).
+//
+// Format: OCP E4M3 codes and one power-of-two scale per vector,
+// s = 2^(c - 8) with c the smallest integer such that max|v| <= 2^c (s = 1 for
+// an all-zero vector); code = nearest e4m3 value of v / s, ties to even.  So
+// |v| / s <= 256 (below e4m3's 448), v / s is exact, and code * s is exactly a
+// bf16 value.  Expert weights get one scale per expert and output column and
+// are stored with the reduction dimension contiguous (the K-major operand of
+// the MMA); activations get one scale per row.
+//
+// k_quant_weights  w [E][K][N] bf16 -> codes [E][N][K], scales [E][N]
+//                  (one-time preparation of a layer's weights).
+// k_quant_rows     rows of a bf16 matrix -> codes + one scale per row: a row
+//                  is held in registers by 32-256 threads (all its loads in
+//                  flight at once), its largest magnitude comes from warp and
+//                  block reductions, the codes go out with streaming 8-byte
+//                  stores.  Optionally reads row r from src[idx[r]] (the row
+//                  copy of the dispatch, x_perm) or skips rows whose idx is
+//                  negative (h: unfilled slots).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+// The power-of-two scale of a vector of largest magnitude amax, s = 2^(c - 8),
+// and the factor that divides by it: v / s = (v * p0) * p1 exactly, p0 * p1 =
+// 2^(8 - c) split in two so that neither factor overflows (c can be as low as
+// -133 for bf16 subnormals).  A product by a power of two is exact, or rounds
+// once to nearest like the division would, so the codes equal those of v / s.
+struct Fp8Scale {
+    float s, p0, p1;
+};
+__device__ __forceinline__ Fp8Scale fp8_scale(float amax) {
+    if (!(amax > 0.0f) || isinf(amax)) return {1.0f, 1.0f, 1.0f};
+    int ex;
+    const float m = frexpf(amax, &ex);  // amax = m * 2^ex, 0.5 <= m < 1
+    const int c = (m == 0.5f) ? ex - 1 : ex;
+    const int e = 8 - c;                // in [-119, 141]
+    const int e0 = e > 64 ? 64 : e;
+    return {ldexpf(1.0f, c - 8), ldexpf(1.0f, e0), ldexpf(1.0f, e - e0)};
+}
+
+// Two values / s to two e4m3 codes (low byte = first).
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b, const Fp8Scale &sc) {
+    const float2 v = make_float2(__fmul_rn(__fmul_rn(a, sc.p0), sc.p1), __fmul_rn(__fmul_rn(b, sc.p0), sc.p1));
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Eight bf16 values (one 16-byte vector) / s to eight codes.
+__device__ __forceinline__ uint2 quant8(const uint4 &v, const Fp8Scale &sc) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        c[i] = e4m3x2(f.x, f.y, sc);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ float amax8(const uint4 &v, float m) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    return m;
+}
+
+// Block of 256 threads: expert e = blockIdx.y, columns [32 blockIdx.x, +32).
+__global__ void __launch_bounds__(256) k_quant_weights(const __nv_bfloat16 *__restrict__ w, uint8_t *__restrict__ q,
+                                                       float *__restrict__ scale, int K, int N) {
+    __shared__ float s_red[8][32];
+    __shared__ Fp8Scale s_scale[32];
+    __shared__ __nv_bfloat16 tile[128][33];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int e = blockIdx.y, n0 = blockIdx.x * 32;
+    const __nv_bfloat16 *we = w + (size_t)e * K * N;
+    float m = 0.0f;
+    for (int k = ty; k < K; k += 8) m = fmaxf(m, fabsf(__bfloat162float(we[(size_t)k * N + n0 + tx])));
+    s_red[ty][tx] = m;
+    __syncthreads();
+    if (ty == 0) {
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i][tx]);
+        const Fp8Scale sc = fp8_scale(m);
+        s_scale[tx] = sc;
+        scale[(size_t)e * N + n0 + tx] = sc.s;
+    }
+    __syncthreads();
+    // codes [e][n0 + i][k0 + 16 c ...]: thread (i = t / 8, c = t % 8) writes 16 bytes
+    const int i = threadIdx.x >> 3, c = threadIdx.x & 7;
+    const Fp8Scale s = s_scale[i];
+    uint8_t *qe = q + ((size_t)e * N + n0 + i) * K;
+    for (int k0 = 0; k0 < K; k0 += 128) {
+        for (int r = ty; r < 128; r += 8) tile[r][tx] = we[(size_t)(k0 + r) * N + n0 + tx];
+        __syncthreads();
+        uint32_t word[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int kk = 16 * c + 4 * v;
+            const uint32_t lo = e4m3x2(__bfloat162float(tile[kk][i]), __bfloat162float(tile[kk + 1][i]), s);
+            const uint32_t hi = e4m3x2(__bfloat162float(tile[kk + 2][i]), __bfloat162float(tile[kk + 3][i]), s);
+            word[v] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint4 *>(qe + k0 + 16 * c) = make_uint4(word[0], word[1], word[2], word[3]);
+        __syncthreads();
+    }
+}
+
+// Rows of TPR threads (TPR = 32 << g, 256 / TPR rows per block): row r < rows
+// (rows = fixed_rows, or cap_rows + *total_spill when fixed_rows < 0).
+// gather: row r is src[idx[r]] (idx outside [0, src_rows): a zero row with
+// scale 1); otherwise row r is src[r], skipped when idx != nullptr and
+// idx[r] < 0.  Each thread loads its VPT 16-byte vectors of the row into
+// registers (all loads in flight at once), the row's largest magnitude comes
+// from a warp reduction and, for TPR > 32, a reduction over the row's warps in
+// shared memory; the codes are written from the registers with streaming
+// stores (the codes are read once, by the GEMM).
+template <int TPR, int VPT>
+__global__ void __launch_bounds__(256) k_quant_rows(const uint4 *__restrict__ src, const int *__restrict__ idx,
+                                                    int gather, uint2 *__restrict__ q, float *__restrict__ scale,
+                                                    int K8, int src_rows, int P, int fixed_rows, int cap_rows,
+                                                    const int *total_spill) {
+    constexpr int kRowsPerBlock = 256 / TPR, kWarpsPerRow = TPR / 32;
+    __shared__ float s_max[8];
+    pdl_trigger();
+    pdl_wait();
+    int rows = fixed_rows >= 0 ? fixed_rows : cap_rows + *total_spill;
+    if (rows > P) rows = P;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = threadIdx.x / TPR, tr = threadIdx.x % TPR;
+    // every thread of the block runs the same number of iterations (the
+    // shared-memory reduction below needs the whole block)
+    for (int base = blockIdx.x * kRowsPerBlock; base < rows; base += gridDim.x * kRowsPerBlock) {
+        const int row = base + g;
+        bool active = row < rows;
+        int sr = row;
+        if (active && idx) {
+            const int t = idx[row];
+            if (!gather && t < 0) active = false;
+            if (gather) sr = t;
+        }
+        const bool valid = active && (unsigned)sr < (unsigned)src_rows;
+        uint4 v[VPT];
+        float m = 0.0f;
+        if (valid) {
+            const uint4 *s_row = src + (size_t)sr * K8;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int c = tr + i * TPR;
+                v[i] = c < K8 ? __ldg(s_row + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) m = amax8(v[i], m);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (kWarpsPerRow > 1) {
+            if (lane == 0) s_max[warp] = m;
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < kWarpsPerRow; ++w) m = fmaxf(m, s_max[g * kWarpsPerRow + w]);
+            __syncthreads();
+        }
+        if (!active) continue;
+        uint2 *dst = q + (size_t)row * K8;
+        if (!valid) {
+            for (int c = tr; c < K8; c += TPR) dst[c] = make_uint2(0, 0);
+            if (tr == 0) scale[row] = 1.0f;
+            continue;
+        }
+        const Fp8Scale sc = fp8_scale(m);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int c = tr + i * TPR;
+            if (c < K8) __stcs(dst + c, quant8(v[i], sc));
+        }
+        if (tr == 0) scale[row] = sc.s;
+    }
+}
+
+// Two passes over the row (rows longer than 256 threads x 16 vectors).
+__global__ void __launch_bounds__(256) k_quant_rows_long(const uint4 *__restrict__ src, const int *__restrict__ idx,
+                                                         int gather, uint2 *__restrict__ q, float *__restrict__ scale,
+                                                         int K8, int src_rows, int P, int fixed_rows, int cap_rows,
+                                                         const int *total_spill) {
+    __shared__ float s_max[8];
+    pdl_trigger();
+    pdl_wait();
+    int rows = fixed_rows >= 0 ? fixed_rows : cap_rows + *total_spill;
+    if (rows > P) rows = P;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+        int sr = row;
+        if (idx) {
+            const int t = idx[row];
+            if (!gather && t < 0) continue;  // block-uniform
+            if (gather) sr = t;
+        }
+        uint2 *dst = q + (size_t)row * K8;
+        if ((unsigned)sr >= (unsigned)src_rows) {
+            for (int c = threadIdx.x; c < K8; c += 256) dst[c] = make_uint2(0, 0);
+            if (threadIdx.x == 0) scale[row] = 1.0f;
+            continue;
+        }
+        const uint4 *s_row = src + (size_t)sr * K8;
+        float m = 0.0f;
+        for (int c = threadIdx.x; c < K8; c += 256) m = amax8(__ldg(s_row + c), m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_max[warp] = m;
+        __syncthreads();
+        for (int w = 0; w < 8; ++w) m = fmaxf(m, s_max[w]);
+        __syncthreads();
+        const Fp8Scale sc = fp8_scale(m);
+        for (int c = threadIdx.x; c < K8; c += 256) __stcs(dst + c, quant8(__ldg(s_row + c), sc));
+        if (threadIdx.x == 0) scale[row] = sc.s;
+    }
+}
+
+// Row quantization launch: threads per row chosen so that a row's vectors fit
+// 8 (up to 16) registers per thread.
+cudaError_t launch_rows(const uint4 *src, const int *idx, int gather, uint2 *q, float *scale, int K8, int src_rows,
+                        int P, int fixed_rows, int cap_rows, const int *total_spill, int row_hint, int num_sms,
+                        cudaStream_t stream) {
+    int tpr = 32;
+    while (tpr < 256 && K8 > tpr * 8) tpr <<= 1;
+    const int rpb = 256 / tpr;
+    int blocks = (row_hint + rpb - 1) / rpb;
+    const int cap = num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+#define MOE_QROWS(T, V)                                                                                        \
+    return launch_pdl(k_quant_rows<T, V>, dim3(blocks), dim3(256), 0, stream, src, idx, gather, q, scale, K8, src_rows, \
+                      P, fixed_rows, cap_rows, total_spill)
+    if (K8 <= 32 * 8) MOE_QROWS(32, 8);
+    if (K8 <= 64 * 8) MOE_QROWS(64, 8);
+    if (K8 <= 128 * 8) MOE_QROWS(128, 8);
+    if (K8 <= 256 * 8) MOE_QROWS(256, 8);
+    if (K8 <= 256 * 16) MOE_QROWS(256, 16);
+#undef MOE_QROWS
+    return launch_pdl(k_quant_rows_long, dim3(blocks), dim3(256), 0, stream, src, idx, gather, q, scale, K8, src_rows,
+                      P, fixed_rows, cap_rows, total_spill);
+}
+
+}  // namespace
+
+// Expert weights w [E][K][N] bf16 -> codes [E][N][K] and scales [E][N].
+cudaError_t launch_quant_weights(int E, int K, int N, const void *w, void *q, float *scale, cudaStream_t stream) {
+    const dim3 grid((unsigned)(N / 32), (unsigned)E);
+    k_quant_weights<<<grid, 256, 0, stream>>>((const __nv_bfloat16 *)w, (uint8_t *)q, scale, K, N);
+    return cudaGetLastError();
+}
+
+// Codes + row scales of the rows of the permuted buffers (P rows of length
+// K, the used rows only).  gather: row r = src[idx[r]] with src holding
+// src_rows rows (the row copy of x); otherwise row r = src[r], rows with
+// idx[r] < 0 skipped (h).
+cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int src_rows, const int32_t *idx,
+                              bool gather, void *q, float *scale, const WsLayout &L, void *ws, int num_sms,
+                              cudaStream_t stream) {
+    const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
+    const int R = s.T * s.k;
+    const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, capped);
+    WsPtrs p = ws_ptrs(ws, L);
+    return launch_rows((const uint4 *)src, idx, gather ? 1 : 0, (uint2 *)q, scale, K / 8, src_rows, P,
+                       capped ? -1 : R, s.E * s.C, p.total_spill, P, num_sms, stream);
+}
+
+// Codes + scales of every token row of x [T, K] (the form the row-gathering
+// SwiGLU GEMM reads).
+cudaError_t launch_quant_tokens(const moe_shape &s, const void *x, void *q, float *scale, int num_sms,
+                                cudaStream_t stream) {
+    return launch_rows((const uint4 *)x, nullptr, 0, (uint2 *)q, scale, s.H / 8, s.T, s.T, s.T, 0, nullptr, s.T,
+                       num_sms, stream);
+}
+
+}  // namespace moe

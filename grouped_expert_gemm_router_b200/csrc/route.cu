@@ -253,6 +253,8 @@ __host__ __device__ inline int topk_mpl(int E) { return E <= 32 ? 1 : (E <= 64 ?
 // the first is used), no shared-memory staging.
 template <int MPL>
 __global__ void __launch_bounds__(256) k_topk(RouteArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     if (t >= a.T) return;  // warp-uniform
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_nan;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();  // the next kernel may set up while the router runs
     const int CL = a.cl;
     const int rank = CL > 1 ? (int)cluster_rank() : 0;
     const int t0 = (blockIdx.x / CL) * TB;
@@ -548,10 +551,10 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
         const int blocks = (int)(((int64_t)s.T * 32 + 255) / 256);
         if (blocks > 0) {
             switch (topk_mpl(s.E)) {
-                case 1: k_topk<1><<<blocks, 256, 0, stream>>>(a); break;
-                case 2: k_topk<2><<<blocks, 256, 0, stream>>>(a); break;
-                case 4: k_topk<4><<<blocks, 256, 0, stream>>>(a); break;
-                default: k_topk<8><<<blocks, 256, 0, stream>>>(a); break;
+                case 1: return launch_pdl(k_topk<1>, dim3(blocks), dim3(256), 0, stream, a);
+                case 2: return launch_pdl(k_topk<2>, dim3(blocks), dim3(256), 0, stream, a);
+                case 4: return launch_pdl(k_topk<4>, dim3(blocks), dim3(256), 0, stream, a);
+                default: return launch_pdl(k_topk<8>, dim3(blocks), dim3(256), 0, stream, a);
             }
         }
         return cudaGetLastError();

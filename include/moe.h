@@ -80,12 +80,10 @@ typedef enum {
 #define MOE_FLAG_CAPACITY 0x1u  /* capacity layout: C slots per expert + overflow */
 #define MOE_FLAG_LOGITS_IN 0x2u /* moe_route/moe_forward read the caller's fp32
                                    logits instead of computing x * W_r + bias */
-#define MOE_FLAG_GEMM_PAIRS 0x4u /* run moe_grouped_swiglu / moe_grouped_down on
-                                   pairs of CTAs sharing one tcgen05 MMA
-                                   (cta_group::2, M = 256, the token tile split
-                                   between the two CTAs).  Same results; on B200
-                                   it is slower for the shapes measured so far,
-                                   so it is off by default. */
+#define MOE_FLAG_FUSED_COMBINE 0x8u /* moe_forward / moe_forward_fp8 run the
+                                   combine of step 5 inside the down GEMM
+                                   (moe_grouped_down_combine): same out, bit
+                                   for bit, and y is still written */
 #define MOE_FLAG_TEST_STALL_SCAN 0x40000000u /* test only: the first histogram
                                    block never publishes, so its successor's
                                    bounded wait expires and reports
@@ -234,6 +232,23 @@ MOE_API moe_status moe_grouped_swiglu_gather(const moe_shape *shape, const void 
 MOE_API moe_status moe_grouped_down(const moe_shape *shape, const void *h, const void *w_down, void *y, void *ws,
                             void *stream);
 
+/* Steps 4b and 5 in one kernel: the down projection of moe_grouped_down
+ * (y is written as there), and, in its epilogue, the weighted combine of
+ * moe_combine.  The "TritonMoE" verdict page (desk editor letter) notes that
+ * its fused kernel stops before the down projection; here the combine follows
+ * the down projection's stores without another launch: after a warp has
+ * stored its piece of a unit's rows it counts one arrival per (token,
+ * 128-feature block) in the workspace, and the warp whose arrival completes a
+ * token's block (all k of its rows stored) combines that block, in slot
+ * order, with exactly moe_combine's arithmetic: `out` is bit-identical to
+ * moe_combine's on the same y.  The counts start at zero after
+ * moe_workspace_init and every complete call leaves them at zero; after a
+ * device-side fault (status word non-zero) re-initialise the workspace.
+ * src_token and dest_row as moe_permute / moe_route_dispatch leave them. */
+MOE_API moe_status moe_grouped_down_combine(const moe_shape *shape, const void *h, const void *w_down,
+                                            const int32_t *src_token, const int32_t *dest_row, const float *topk_w,
+                                            void *y, void *out, void *ws, void *stream);
+
 /* Step 5, weighted unpermutation ("TritonMoE" verdict page, referee report
  * summary):  out[t] = bf16( sum_j topk_w[t,j] * y[dest_row[t*k+j]] ), the
  * sum in fp32 in slot order j, products and sums rounded separately. */
@@ -242,7 +257,8 @@ MOE_API moe_status moe_combine(const moe_shape *shape, const void *y, const int3
 
 /* The five steps in order on one stream (no host sync; graph-capturable):
  * moe_route_dispatch, moe_gather, moe_grouped_swiglu, moe_grouped_down,
- * moe_combine.  With args->x_perm == NULL the row copy is folded into the
+ * moe_combine (with MOE_FLAG_FUSED_COMBINE: moe_grouped_down_combine in place
+ * of the last two).  With args->x_perm == NULL the row copy is folded into the
  * SwiGLU GEMM (moe_grouped_swiglu_gather) and x_perm is not produced: the
  * faster choice for decode-sized batches (about 32 or fewer routed rows per
  * expert), the slower one for large batches. */
@@ -284,6 +300,106 @@ MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_stat
 MOE_API moe_status moe_permute_static(const moe_shape *shape, const void *x, const int32_t *topk_idx,
                                       int32_t *expert_counts, int32_t *expert_offsets, int32_t *src_token,
                                       int32_t *dest_row, void *x_perm, void *stream);
+
+/* ------------------------------------------------------------------------
+ * fp8 (e4m3) expert GEMMs ("TEMPO" verdict page, pith.science, arXiv
+ * 2608.13057, referee report summary: its per-expert cost law is measured on
+ * an fp8 grouped GEMM, whose flat regime streams the expert's weights from
+ * HBM; 8-bit weights halve those bytes).
+ *
+ * Format (the pages fix none; this is the plainest reading): OCP E4M3 codes
+ * (uint8: sign, 4 exponent bits with bias 7, 3 mantissa bits, max 448) with
+ * one power-of-two fp32 scale per vector, s = 2^(c - 8) for the smallest
+ * integer c with max|v| <= 2^c (s = 1 for an all-zero vector); code = the
+ * nearest e4m3 value of v / s, ties to even.  value = code * s, which is
+ * exactly a bf16 value, so the fp8 layer is the bf16 layer applied to the
+ * dequantized weights and activations.  Expert weights: one scale per expert
+ * and output column, codes stored with the reduction dimension contiguous.
+ * Activations: one scale per row.  The GEMMs multiply products of codes on
+ * the tensor cores (tcgen05 kind::f8f6f4, fp32 accumulation) and apply the
+ * row and column scales in the epilogue; h and y stay bf16, the combine is
+ * the bf16 one.
+ * ------------------------------------------------------------------------ */
+#define MOE_WEIGHTS_GATE_UP 0 /* w [E,H,F] bf16 -> codes [E,F,H], scales [E,F] */
+#define MOE_WEIGHTS_DOWN 1    /* w [E,F,H] bf16 -> codes [E,H,F], scales [E,H] */
+#define MOE_ROWS_X_PERM 0     /* codes [P,H] of x[src_token[r]] (the row copy of step 3; zero codes
+                                 with scale 1 where src_token is -1), scales [P] */
+#define MOE_ROWS_TOKENS 1     /* codes [T,H] of every token row of x, scales [T] */
+#define MOE_ROWS_H 2          /* codes [P,F] of h[r] for every filled row r (src_token[r] >= 0; the
+                                 other rows are left unwritten), scales [P] */
+
+/* One-time preparation of expert weights: `which` = MOE_WEIGHTS_GATE_UP (w is
+ * w_gate or w_up, [E,H,F]) or MOE_WEIGHTS_DOWN (w is w_down, [E,F,H]).
+ * w_q: 16-byte aligned device buffer of E*H*F bytes; w_scale: E*F (gate/up)
+ * or E*H (down) floats. */
+MOE_API moe_status moe_quantize_weights_fp8(const moe_shape *shape, int which, const void *w, void *w_q,
+                                            float *w_scale, void *stream);
+
+/* Row quantization (see MOE_ROWS_*): `src` is x ([T,H] bf16) for X_PERM and
+ * TOKENS, h ([P,F] bf16) for H; src_token as moe_permute / moe_route_dispatch
+ * leave it (unused for TOKENS).  X_PERM and H read the overflow size from
+ * `ws`. */
+MOE_API moe_status moe_quantize_rows_fp8(const moe_shape *shape, int which, const void *src, const int32_t *src_token,
+                                         void *q, float *scale, void *ws, void *stream);
+
+/* Step 4a on fp8 operands: the same h as moe_grouped_swiglu on the
+ * dequantized operands (up to fp32 summation order):
+ *   h[r,f] = bf16( silu(g) * u ),  g = sx[r] * swg[e,f] * sum_k xq[r,k] * wgq[e,f,k]
+ * (u likewise with the up weights).  With src_token == NULL, x_q / x_scale
+ * hold the permuted rows ([P,H] codes, [P] scales: MOE_ROWS_X_PERM);
+ * otherwise they hold the token rows ([T,H], [T]: MOE_ROWS_TOKENS) and row r
+ * is gathered from token src_token[r] (like moe_grouped_swiglu_gather). */
+MOE_API moe_status moe_grouped_swiglu_fp8(const moe_shape *shape, const void *x_q, const float *x_scale,
+                                          const int32_t *src_token, const void *wg_q, const float *wg_scale,
+                                          const void *wu_q, const float *wu_scale, void *h, void *ws, void *stream);
+
+/* Step 4b on fp8 operands: y[r,c] = bf16( sh[r] * swd[e,c] * sum_f hq[r,f] * wdq[e,c,f] ),
+ * h_q / h_scale as MOE_ROWS_H writes them. */
+MOE_API moe_status moe_grouped_down_fp8(const moe_shape *shape, const void *h_q, const float *h_scale,
+                                        const void *wd_q, const float *wd_scale, void *y, void *ws, void *stream);
+
+/* moe_grouped_down_fp8 with the combine of step 5 in its epilogue, as
+ * moe_grouped_down_combine does for the bf16 projection. */
+MOE_API moe_status moe_grouped_down_fp8_combine(const moe_shape *shape, const void *h_q, const float *h_scale,
+                                                const void *wd_q, const float *wd_scale, const int32_t *src_token,
+                                                const int32_t *dest_row, const float *topk_w, void *y, void *out,
+                                                void *ws, void *stream);
+
+/* Every pointer argument of the fp8 layer, for moe_forward_fp8. */
+typedef struct {
+    const void *x;           /* [T,H]   bf16 tokens */
+    const float *w_router;   /* [H,E]   fp32 */
+    const float *bias;       /* [E]     fp32, or NULL */
+    const void *wg_q;        /* [E,F,H] e4m3 gate codes */
+    const float *wg_scale;   /* [E,F] */
+    const void *wu_q;        /* [E,F,H] e4m3 up codes */
+    const float *wu_scale;   /* [E,F] */
+    const void *wd_q;        /* [E,H,F] e4m3 down codes */
+    const float *wd_scale;   /* [E,H] */
+    float *logits;           /* [T,E]   as in moe_forward_args */
+    int32_t *topk_idx;       /* [T,k] */
+    float *topk_w;           /* [T,k] */
+    int32_t *expert_counts;  /* [E] */
+    int32_t *expert_offsets; /* [E+1] */
+    int32_t *src_token;      /* [P] */
+    int32_t *dest_row;       /* [T*k] */
+    void *x_q;               /* [P,H] codes (x_q_per_token == 0) or [T,H] (== 1) */
+    float *x_scale;          /* [P] or [T] */
+    int32_t x_q_per_token;   /* 1: token rows gathered by the SwiGLU GEMM (no row copy) */
+    void *h;                 /* [P,F]   bf16 */
+    void *h_q;               /* [P,F]   e4m3 codes */
+    float *h_scale;          /* [P] */
+    void *y;                 /* [P,H]   bf16 */
+    void *out;               /* [T,H]   bf16 layer output */
+} moe_forward_fp8_args;
+
+/* The fp8 layer on one stream (no host sync; graph-capturable):
+ * moe_route_dispatch, moe_quantize_rows_fp8 (X_PERM, or TOKENS with
+ * x_q_per_token), moe_grouped_swiglu_fp8, moe_quantize_rows_fp8 (H),
+ * moe_grouped_down_fp8, moe_combine (with MOE_FLAG_FUSED_COMBINE:
+ * moe_grouped_down_fp8_combine in place of the last two).  Weights must have been prepared with
+ * moe_quantize_weights_fp8. */
+MOE_API moe_status moe_forward_fp8(const moe_shape *shape, const moe_forward_fp8_args *args, void *ws, void *stream);
 
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);

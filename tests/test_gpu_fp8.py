@@ -1,0 +1,266 @@
+"""The fp8 (e4m3) expert GEMMs through the C ABI against the CPU oracle.
+
+Quantization decisions are integers taken from floating point, so both sides
+take them from the same values: weight and token codes from the layer's
+inputs, h codes from the GPU's own h; they must match bit for bit.  The GEMM
+outputs are compared with the oracle's bf16 expert functions run on the
+dequantized operands (every code times its power-of-two scale is exactly a
+bf16 value), within the output tolerance; the layer output with the oracle's
+own fp8 layer.  The distance of the fp8 layer from the bf16 layer is a
+property of the format, reported (and bounded loosely), not a parity check."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_expert_gemm_router_b200 as moe
+import synth
+from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, shape_of
+
+pytestmark = pytest.mark.gpu
+
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+CASES = {
+    "two_tiles_E4_k2": synth.LayerConfig("t", 700, 256, 384, 4, 2, seed=1),
+    "skew_E8_k3_H384": synth.LayerConfig("t", 300, 384, 256, 8, 3, alpha=1.5, seed=2),
+    "capacity_E16_k4_C24": synth.LayerConfig("t", 200, 256, 256, 16, 4, C=24, alpha=1.0, seed=3),
+    "tiny_config": synth.CONFIGS[1],
+    "single_token": synth.LayerConfig("t", 1, 128, 128, 1, 1, seed=4),
+    "E1_dense": synth.LayerConfig("t", 300, 128, 256, 1, 1, seed=6),
+    "many_experts_E256_k8": synth.LayerConfig("t", 96, 128, 128, 256, 8, alpha=0.5, seed=7),
+}
+
+
+def _u8(t):
+    return t.detach().cpu().contiguous().numpy()
+
+
+def _run_fp8(dl, shape, per_token):
+    b = dl.bufs(shape)
+    b.update(moe.alloc_fp8_buffers(shape, per_token=per_token))
+    moe.quantize_layer_weights_fp8(shape, b)
+    moe.moe_forward_fp8(shape, b, b["ws"], per_token=per_token)
+    torch.cuda.synchronize()
+    return b
+
+
+class Fp8Ref:
+    """The oracle's fp8 layer pieces for one seeded layer."""
+
+    def __init__(self, orc, L):
+        self.orc = orc
+        self.L = L
+        self.wg_q, self.wg_s = orc.quantize_weights(L.w_gate)
+        self.wu_q, self.wu_s = orc.quantize_weights(L.w_up)
+        self.wd_q, self.wd_s = orc.quantize_weights(L.w_down)
+        self.wg = orc.dequantize_weights(self.wg_q, self.wg_s)
+        self.wu = orc.dequantize_weights(self.wu_q, self.wu_s)
+        self.wd = orc.dequantize_weights(self.wd_q, self.wd_s)
+        self.x_q, self.x_s = orc.quantize_rows(L.x)
+        self.xd = orc.dequantize(self.x_q, self.x_s)
+
+
+@pytest.mark.parametrize("per_token", [False, True], ids=["x_perm", "token_rows"])
+@pytest.mark.parametrize("name", list(CASES))
+def test_fp8_layer_parity(orc, name, per_token):
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    b = _run_fp8(dl, shape, per_token)
+    assert moe.moe_read_status(b["ws"], clear=True) == 0
+    ref = Fp8Ref(orc, L)
+
+    # weight codes and scales: bit-exact
+    for q, s, rq, rs in (("wg_q", "wg_scale", ref.wg_q, ref.wg_s), ("wu_q", "wu_scale", ref.wu_q, ref.wu_s),
+                         ("wd_q", "wd_scale", ref.wd_q, ref.wd_s)):
+        assert np.array_equal(_u8(b[q]), rq), q
+        assert np.array_equal(b[s].cpu().numpy(), rs), s
+
+    # routing as the bf16 path (the same kernels): oracle top-k on the GPU logits
+    logits = b["logits"].cpu().numpy()
+    idx, w, _ = orc.topk_softmax(logits, cfg.k)
+    assert np.array_equal(b["topk_idx"].cpu().numpy(), idx)
+    d = orc.dispatch(idx, cfg.E, C=cfg.C, capped=cfg.C > 0)
+    assert np.array_equal(b["dest_row"].cpu().numpy(), d["dest_row"])
+    src = d["src_token"]
+    filled = src >= 0
+    rows = np.flatnonzero(filled)
+
+    # token codes: bit-exact (permuted rows, or the token rows)
+    xq = _u8(b["x_q"])
+    xs = b["x_scale"].cpu().numpy()
+    if per_token:
+        assert np.array_equal(xq, ref.x_q) and np.array_equal(xs, ref.x_s)
+    else:
+        assert np.array_equal(xq[rows], ref.x_q[src[rows]]) and np.array_equal(xs[rows], ref.x_s[src[rows]])
+        if cfg.C > 0:  # empty capacity slots: zero codes, scale 1
+            empty = np.flatnonzero(src[:cfg.E * cfg.C] < 0)
+            assert np.all(xq[empty] == 0) and np.all(xs[empty] == 1.0)
+
+    # h against the oracle's SwiGLU on the dequantized operands
+    flat = idx.reshape(-1)
+    row_e = np.full(d["P"], -1)
+    row_e[d["dest_row"]] = flat
+    h = bf16_host(b["h"])
+    h_ref = np.stack([orc.swiglu_row(ref.xd[src[r]], ref.wg[row_e[r]], ref.wu[row_e[r]]) for r in rows])
+    assert_close_bf16(h[rows], h_ref, "fp8 h")
+
+    # h codes from the GPU's own h: bit-exact
+    hq_ref, hs_ref = orc.quantize_rows(h[rows])
+    assert np.array_equal(_u8(b["h_q"])[rows], hq_ref)
+    assert np.array_equal(b["h_scale"].cpu().numpy()[rows], hs_ref)
+
+    # y against the oracle's down projection of the GPU's h codes
+    hd = orc.dequantize(hq_ref, hs_ref)
+    y = bf16_host(b["y"])
+    y_ref = np.stack([orc.down_row(hd[i], ref.wd[row_e[r]]) for i, r in enumerate(rows)])
+    assert_close_bf16(y[rows], y_ref, "fp8 y")
+
+    # the combine is the bf16 one: bit-exact given the GPU's y
+    out = bf16_host(b["out"])
+    assert np.array_equal(out, orc.combine(y, b["dest_row"].cpu().numpy(), b["topk_w"].cpu().numpy()))
+
+    # the layer against the oracle's own fp8 layer (its own h and h codes)
+    h_o = np.zeros((d["P"], cfg.F), np.uint16)
+    for r in rows:
+        h_o[r] = orc.swiglu_row(ref.xd[src[r]], ref.wg[row_e[r]], ref.wu[row_e[r]])
+    hq_o, hs_o = orc.quantize_rows(h_o)
+    hd_o = orc.dequantize(hq_o, hs_o)
+    y_o = np.zeros((d["P"], cfg.H), np.uint16)
+    for r in rows:
+        y_o[r] = orc.down_row(hd_o[r], ref.wd[row_e[r]])
+    out_o = orc.combine(y_o, d["dest_row"], w)
+    assert_close_bf16(out, out_o, "fp8 out")
+
+
+@pytest.mark.parametrize("name", ["two_tiles_E4_k2", "capacity_E16_k4_C24", "many_experts_E256_k8"])
+def test_fp8_fused_combine(name):
+    """moe_forward_fp8 with the combine in the fp8 down GEMM's epilogue: the
+    same h, y and out, bit for bit, as the separate combine."""
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    a = _run_fp8(dl, shape_of(cfg), False)
+    sf = shape_of(cfg, flags=moe.MOE_FLAG_FUSED_COMBINE)
+    b = _run_fp8(dl, sf, False)
+    assert moe.moe_read_status(b["ws"], clear=True) == 0
+    filled = a["src_token"].cpu().numpy() >= 0
+    for key in ("h", "y"):
+        assert np.array_equal(bf16_host(a[key])[filled], bf16_host(b[key])[filled]), key
+    assert np.array_equal(bf16_host(a["out"]), bf16_host(b["out"]))
+
+
+def test_fp8_distance_from_bf16_layer(orc):
+    """The fp8 layer approximates the bf16 layer; the gap is the format's, not
+    a parity question.  e4m3 keeps 4 significant bits (a relative rounding
+    error up to 2^-4 per weight and per activation), so single outputs can
+    move by several percent of max|ref|; measured 7.3e-2 on this layer.  The
+    bound only catches a gross error (a wrong scale gives O(1) or worse)."""
+    cfg = synth.LayerConfig("t", 256, 512, 768, 8, 2, seed=40)
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    b = _run_fp8(DeviceLayer(L), shape, False)
+    idx, w, _ = orc.topk_softmax(b["logits"].cpu().numpy(), cfg.k)
+    ref = orc.token_outputs(np.arange(cfg.T, dtype=np.int32), L.x, idx, w, L.w_gate, L.w_up, L.w_down)
+    g = synth.bf16_bits_to_f32(bf16_host(b["out"])).astype(np.float64)
+    r = synth.bf16_bits_to_f32(ref).astype(np.float64)
+    rel = np.max(np.abs(g - r)) / np.max(np.abs(r))
+    print("fp8 layer vs bf16 layer: max|diff| / max|ref| = %.3e" % rel)
+    assert rel <= 0.15
+
+
+FULL = [(2, None), (3, None), (4, None), (5, 0.0)]
+
+
+@pytest.mark.parametrize("cid,alpha", FULL, ids=["cfg%d%s" % (c, "" if a is None else "-a%g" % a) for c, a in FULL])
+def test_fp8_full_config(orc, cid, alpha):
+    """Full sizes: the first expert's weight codes and all token codes
+    bit-exact; h and y on one row of every tile; out on 32 tokens."""
+    cfg = synth.CONFIGS[cid] if alpha is None else synth.CONFIGS[cid].with_(alpha=alpha)
+    L = synth.make_layer(cfg)
+    shape = shape_of(cfg)
+    per_token = cfg.T * cfg.k <= 32 * cfg.E  # as the benchmark chooses
+    b = _run_fp8(DeviceLayer(L), shape, per_token)
+    assert moe.moe_read_status(b["ws"], clear=True) == 0
+    rng = np.random.default_rng(cid)
+    refw = {}
+    for name, wt in (("wg", L.w_gate), ("wu", L.w_up), ("wd", L.w_down)):
+        for e in (0,):
+            q, s = orc.quantize_weights(wt[e:e + 1])
+            assert np.array_equal(_u8(b[name + "_q"][e]), q[0]), (name, e)
+            assert np.array_equal(b[name + "_scale"][e].cpu().numpy(), s[0]), (name, e)
+    wq = {n: _u8(b[n + "_q"]) for n in ("wg", "wu", "wd")}
+    ws = {n: b[n + "_scale"].cpu().numpy() for n in ("wg", "wu", "wd")}
+
+    def deq_w(name, e):
+        key = (name, e)
+        if key not in refw:
+            refw[key] = orc.dequantize_weights(wq[name][e:e + 1], ws[name][e:e + 1])[0]
+        return refw[key]
+
+    x_q, x_s = orc.quantize_rows(L.x)
+    idx, w, _ = orc.topk_softmax(b["logits"].cpu().numpy(), cfg.k)
+    assert np.array_equal(b["topk_idx"].cpu().numpy(), idx)
+    d = orc.dispatch(idx, cfg.E, C=cfg.C, capped=cfg.C > 0)
+    src = d["src_token"]
+    gq, gs = _u8(b["x_q"]), b["x_scale"].cpu().numpy()
+    filled = np.flatnonzero(src >= 0)
+    if per_token:
+        assert np.array_equal(gq, x_q) and np.array_equal(gs, x_s)
+    else:
+        assert np.array_equal(gq[filled], x_q[src[filled]]) and np.array_equal(gs[filled], x_s[src[filled]])
+    xd = orc.dequantize(x_q, x_s)
+    row_e = np.full(d["P"], -1)
+    row_e[d["dest_row"]] = idx.reshape(-1)
+
+    L_ = moe.moe_workspace_layout(shape)
+    wsb = b["ws"].cpu().numpy()
+    nt = int(wsb[L_.num_tiles:L_.num_tiles + 4].view(np.int32)[0])
+    tmap = wsb[L_.tile_map:L_.tile_map + 16 * nt].view(np.int32).reshape(-1, 4)
+    rows = []
+    for e, s0, lens, s1 in tmap:
+        l0, l1 = lens & 0xFFFF, (lens >> 16) & 0xFFFF
+        c = int(rng.integers(l0 + l1))
+        rows.append(int(s0 + c) if c < l0 else int(s1 + c - l0))
+    rows = sorted(set(rows))
+    h = bf16_host(b["h"])
+    hq, hs = _u8(b["h_q"]), b["h_scale"].cpu().numpy()
+    hq_ref, hs_ref = orc.quantize_rows(h[rows])
+    assert np.array_equal(hq[rows], hq_ref) and np.array_equal(hs[rows], hs_ref)
+    hd = orc.dequantize(hq_ref, hs_ref)
+    with ThreadPoolExecutor(THREADS) as pool:
+        for r in rows:  # dequantize the needed experts once, outside the threads
+            deq_w("wg", row_e[r]), deq_w("wu", row_e[r]), deq_w("wd", row_e[r])
+        h_ref = np.stack(list(pool.map(lambda r: orc.swiglu_row(xd[src[r]], deq_w("wg", row_e[r]),
+                                                                  deq_w("wu", row_e[r])), rows)))
+        y_ref = np.stack(list(pool.map(lambda i: orc.down_row(hd[i], deq_w("wd", row_e[rows[i]])),
+                                       range(len(rows)))))
+    assert_close_bf16(h[rows], h_ref, "fp8 h (one row per tile, %d rows)" % len(rows))
+    assert_close_bf16(bf16_host(b["y"])[rows], y_ref, "fp8 y (one row per tile)")
+    out = bf16_host(b["out"])
+    assert np.array_equal(out, orc.combine(bf16_host(b["y"]), b["dest_row"].cpu().numpy(),
+                                           b["topk_w"].cpu().numpy()))
+
+    # the layer output of 32 tokens against the oracle's own fp8 layer
+    tk = np.sort(rng.choice(cfg.T, size=min(cfg.T, 32), replace=False))
+
+    def token_out(t):
+        ys = []
+        for j in range(cfg.k):
+            e = idx[t, j]
+            hr = orc.swiglu_row(xd[t], deq_w("wg", e), deq_w("wu", e))
+            q, s = orc.quantize_rows(hr[None, :])
+            ys.append(orc.down_row(orc.dequantize(q, s)[0], deq_w("wd", e)))
+        yk = np.stack(ys)
+        return orc.combine(yk, np.arange(cfg.k, dtype=np.int32), w[t:t + 1])[0]
+
+    for t in tk:
+        for e in idx[t]:
+            deq_w("wg", e), deq_w("wu", e), deq_w("wd", e)
+    with ThreadPoolExecutor(THREADS) as pool:
+        out_ref = np.stack(list(pool.map(token_out, tk)))
+    assert_close_bf16(out[tk], out_ref, "fp8 out (%d tokens)" % len(tk))

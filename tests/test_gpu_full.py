@@ -2,7 +2,8 @@
 alpha), through moe_forward in both of its forms: with an x_perm buffer (the
 row copy, then the tiled SwiGLU GEMM: what the benchmark runs when a batch
 has more than 32 routed rows per expert) and without one (the SwiGLU GEMM
-gathers its rows from x).
+gathers its rows from x); and with the combine fused into the down GEMM,
+whose output must equal the separate combine's bit for bit.
 
 Everything integer (routing indices, counts, offsets, permutation, schedule)
 is checked in full.  The GEMM outputs are checked on rows the oracle computes
@@ -90,18 +91,23 @@ def test_full_config(orc, cid, alpha):
     shape = shape_of(cfg)
     dl = DeviceLayer(L)
     runs = {}
-    for form in ("tiled", "gather"):
+    fused = shape_of(cfg, flags=moe.MOE_FLAG_FUSED_COMBINE)
+    for form in ("tiled", "gather", "fused_combine"):
         b = dl.bufs(shape)
         if form == "tiled":
             moe.moe_forward(shape, b, b["ws"])  # row copy into x_perm, tiled SwiGLU GEMM
-        else:
+        elif form == "gather":
             moe.moe_forward(shape, b, b["ws"], args=moe.forward_args({**b, "x_perm": None}))
+        else:  # the combine inside the down GEMM's epilogue
+            moe.moe_forward(fused, b, b["ws"])
         torch.cuda.synchronize()
         r = host(b, shape)
         assert r["status"] == 0, "%s: device status %#x" % (form, r["status"])
         runs[form] = (b, r)
     b, r = runs["tiled"]
     rg = runs["gather"][1]
+    # the fused combine: out bit-identical to the separate combine's
+    assert np.array_equal(runs.pop("fused_combine")[1]["out"], r["out"])
     rng = np.random.default_rng(cid * 10 + int(alpha or 0))
 
     # routing and dispatch: in full, and identical in both forms

@@ -289,6 +289,41 @@ def test_scan_wait_expires_and_reports(orc):
     assert np.array_equal(r["dest_row"], o["d"]["dest_row"])
 
 
+@pytest.mark.parametrize("name", ["two_tiles_E4_k2", "skew_E8_k3_H384", "capacity_E16_k4_C24", "tiny_config",
+                                  "single_token", "k_equals_E", "E1_dense", "many_experts_E256_k8"])
+def test_down_with_fused_combine(orc, name):
+    """The combine of step 5 inside the down GEMM's epilogue: the same y, and
+    out bit-identical to the separate combine kernel's, on two calls in a row
+    (the arrival counts must return to zero after each call)."""
+    cfg = CASES[name]
+    L = synth.make_layer(cfg)
+    dl = DeviceLayer(L)
+    shape = shape_of(cfg)
+    b = run_steps(dl, shape)  # route, permute, swiglu, down, combine
+    y_ref = bf16_host(b["y"])
+    out_ref = bf16_host(b["out"])
+    for _ in range(2):
+        b["y"].fill_(0)
+        b["out"].fill_(0)
+        moe.moe_grouped_down_combine(shape, b["h"], b["w_down"], b["src_token"], b["dest_row"], b["topk_w"], b["y"],
+                                     b["out"], b["ws"])
+        torch.cuda.synchronize()
+        assert moe.moe_read_status(b["ws"], clear=True) == 0
+        filled = b["src_token"].cpu().numpy() >= 0
+        assert np.array_equal(bf16_host(b["y"])[filled], y_ref[filled])
+        assert np.array_equal(bf16_host(b["out"]), out_ref)
+    # and the whole layer with the flag, against the oracle
+    sf = shape_of(cfg, flags=moe.MOE_FLAG_FUSED_COMBINE)
+    bf = dl.bufs(sf)
+    moe.moe_forward(sf, bf, bf["ws"])
+    torch.cuda.synchronize()
+    r = host(bf, sf)
+    assert r["status"] == 0
+    o = _oracle_full(orc, L, cfg, r["logits"])
+    assert np.array_equal(r["out"], orc.combine(r["y"], r["dest_row"], r["topk_w"]))
+    assert_close_bf16(r["out"], o["out"], "out (fused combine)")
+
+
 def test_gemm_wait_expires_and_reports(orc):
     """The SwiGLU GEMM's token producer in CTA 0 never loads its first stage:
     the MMA issuer's bounded wait runs out, the kernel records the timeout,
@@ -319,23 +354,3 @@ def test_gemm_wait_expires_and_reports(orc):
     assert_close_bf16(r["out"], o["out"], "out after a GEMM timeout")
 
 
-@pytest.mark.parametrize("name", ["two_tiles_E4_k2", "skew_E8_k3_H384", "capacity_E16_k4_C24", "E1_dense"])
-def test_gemm_pairs_match_single_cta(orc, name):
-    """MOE_FLAG_GEMM_PAIRS runs both grouped GEMMs on pairs of CTAs sharing
-    one MMA (cta_group::2, M = 256, the token tile split between the CTAs):
-    the same h and y as the single-CTA kernels on every filled row, within the
-    output tolerance against the oracle (ragged tails, a 128-feature last
-    block, the capacity layout, one expert)."""
-    cfg = CASES[name]
-    L = synth.make_layer(cfg)
-    dl = DeviceLayer(L)
-    s1 = shape_of(cfg)
-    s2 = shape_of(cfg, flags=moe.MOE_FLAG_GEMM_PAIRS)
-    a = host(run_steps(dl, s1), s1)
-    b = host(run_steps(dl, s2), s2)
-    assert a["status"] == 0 and b["status"] == 0
-    filled = a["src_token"] >= 0
-    for key in ("h", "y"):
-        assert np.array_equal(a[key][filled], b[key][filled]), key
-    o = _oracle_full(orc, L, cfg, b["logits"])
-    assert_close_bf16(b["out"], o["out"], "out with CTA pairs")
