@@ -73,7 +73,7 @@ namespace moe {
 namespace {
 
 constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row of bf16
-constexpr int kMaxAStages = 8;
+constexpr int kMaxAStages = 16;
 constexpr int kMaxBStages = 4;                 // token stages: 4 while >= 4 weight stages still fit, else 3
 constexpr uint32_t kABox = 64 * 64 * 2;        // TMA box: 64 K rows x 64 features (8 KiB)
 constexpr uint32_t kATile = 2 * kABox;         // one accumulator's A: 128 features x 64 K
@@ -262,6 +262,15 @@ __device__ __forceinline__ float silu_f(float z) {
 __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
     return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Rows of the placement rule below: a unit needs N columns per accumulator;
+// the rule takes half the columns the unit occupies.  Mode 2 fills all of
+// tensor memory.
+template <int MODE>
+__device__ __forceinline__ int tmem_width(const Unit &U) {
+    if (MODE == 2) return 256;
+    return MODE == 1 && U.nacc == 1 ? (U.N + 1) / 2 : U.N;
 }
 
 // Tensor memory is two halves of 256 columns.  A unit with <= 128 rows keeps
@@ -520,10 +529,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         const int ntiles = *a.num_tiles;
         const int nt = ntiles < a.max_tiles ? ntiles : a.max_tiles;
-        // Down projection with few row tiles: 128-feature units, twice as many,
-        // when they still fit one wave (otherwise 256-feature units, which read
-        // each token tile once for two accumulators).
-        if (MODE == 1 && nt * a.num_fb * 2 <= (int)gridDim.x) {
+        // Down projection: 128-feature units (one accumulator of up to 256
+        // columns: half of tensor memory, so a unit's epilogue overlaps the
+        // next unit's MMAs) when they give each CTA fewer operand bytes to
+        // load -- rounds x (weight columns + token rows) per K row -- else
+        // 256-feature units, which read each token tile once for two
+        // accumulators.  With e4m3 operands and full tiles (192 or more rows
+        // per tile on average) also 128-feature units: the 8-bit mainloop of a
+        // full tile is short enough for its epilogue to set the pace otherwise.
+        const int grid = (int)gridDim.x;
+        const int tr = *a.tile_rows;
+        const int r256 = (nt * a.num_fb + grid - 1) / grid, r128 = (nt * (a.n_out / 128) + grid - 1) / grid;
+        const bool full_tiles = (int64_t)a.P >= (int64_t)192 * nt;
+        if (MODE == 1 && ((FP8 && full_tiles) || r128 * (128 + tr) < r256 * (256 + tr))) {
             num_fb = a.n_out / 128;
             fbw = 128;
         }
@@ -553,7 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // flight.  Mode 2 reads both operands from L2 and consumes one stage of
     // each per K block: equally deep rings.
     trows = trows < 16 ? 16 : (trows > kTileRows ? kTileRows : (trows + 15) & ~15);
-    const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : 2u;
+    // weight tiles per stage: both accumulators' (gate and up, or two
+    // 128-feature blocks), one for 128-feature down units (twice the stages)
+    const uint32_t a_tiles = MODE == 2 ? 3u * (a.E > 128 ? 2u : 1u) : (MODE == 1 && fbw == 128 ? 1u : 2u);
     const uint32_t a_bytes = a_tiles * kATile, b_bytes = (uint32_t)trows * kBRowBytes;
     int nb = kMaxBStages;
     int fit = (int)((kRingBytes - (uint32_t)nb * b_bytes) / a_bytes);
@@ -744,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = FP8 ? idesc_e4m3_f32(128, U.N) : idesc_bf16_f32(128, U.N, 1, 0);
                 uint32_t h;
                 bool big;
-                plan.place(MODE == 2 ? 256 : U.N, h, big);  // mode 2 uses all of tensor memory
+                plan.place(tmem_width<MODE>(U), h, big);  // mode 2 uses all of tensor memory
                 const uint32_t d0 = tmem + h * 256u, d1 = big ? tmem + 256u : d0 + 128u;
                 // wait until the epilogue has drained the half(s) this unit takes
                 ok = mbar_wait_bounded(&tempty[h], (plan.uses[h] & 1u) ^ 1u, a.timeout_ns, s_abort);
@@ -847,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint32_t h;
             bool big;
-            plan.place(MODE == 2 ? 256 : U.N, h, big);
+            plan.place(tmem_width<MODE>(U), h, big);
             // The whole warp takes one decision, so the .sync.aligned loads
             // below never run with part of the warp.
             bool got = mbar_wait_bounded(&tfull[h], plan.uses[h] & 1u, a.timeout_ns, s_abort);
@@ -956,6 +976,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         store_block_frag(h0[i], stg, a.out, a.n_out, U.fx + q * 32, U, c0);
                         if (i < kHold1 && U.nacc == 2) store_block_frag(h1[i], stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
                     }
+                }
+                if (COMBINE) arrive_and_combine(a, U, sub, lane);
+                plan.advance(big, h);
+                continue;
+            }
+            if (MODE == 1 && U.nacc == 1) {
+                // One accumulator of up to 256 columns in one half: up to four
+                // 16-column chunks per warp, packed into registers, then handed
+                // back before the stores.
+                constexpr int kOneChunks = (16 + kEpiSub - 1) / kEpiSub;
+                uint32_t h0[kOneChunks][8];
+#pragma unroll
+                for (int i = 0; i < kOneChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) {
+                        uint32_t r[16];
+                        float rs[4];
+                        if (FP8) load_row_scales<GATHER>(a, U, c0, lane, rs);
+                        tmem_ld_frag16(t0 + (uint32_t)c0, r);
+                        tmem_ld_wait();
+                        if (FP8) scale_frag(r, fs0, rs);
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) h0[i][m] = pack_bf16x2(r[2 * m], r[2 * m + 1]);
+                    }
+                }
+                release();
+#pragma unroll
+                for (int i = 0; i < kOneChunks; ++i) {
+                    const int c0 = (sub + kEpiSub * i) * 16;
+                    if (c0 < U.N) store_block_frag(h0[i], stg, a.out, a.n_out, U.fx + q * 32, U, c0);
                 }
                 if (COMBINE) arrive_and_combine(a, U, sub, lane);
                 plan.advance(big, h);

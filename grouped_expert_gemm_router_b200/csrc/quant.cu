@@ -47,32 +47,41 @@ __device__ __forceinline__ Fp8Scale fp8_scale(float amax) {
     return {ldexpf(1.0f, c - 8), ldexpf(1.0f, e0), ldexpf(1.0f, e - e0)};
 }
 
-// Two values / s to two e4m3 codes (low byte = first).
+// Two values / s to two e4m3 codes (low byte = first).  ONE: 1/s = p0 is a
+// normal power of two (p1 == 1), one product per value (the common case).
+template <bool ONE>
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b, const Fp8Scale &sc) {
-    const float2 v = make_float2(__fmul_rn(__fmul_rn(a, sc.p0), sc.p1), __fmul_rn(__fmul_rn(b, sc.p0), sc.p1));
+    const float2 v = ONE ? make_float2(__fmul_rn(a, sc.p0), __fmul_rn(b, sc.p0))
+                         : make_float2(__fmul_rn(__fmul_rn(a, sc.p0), sc.p1), __fmul_rn(__fmul_rn(b, sc.p0), sc.p1));
     return (uint32_t)__nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, __NV_E4M3);
 }
 
 // Eight bf16 values (one 16-byte vector) / s to eight codes.
-__device__ __forceinline__ uint2 quant8(const uint4 &v, const Fp8Scale &sc) {
+template <bool ONE>
+__device__ __forceinline__ uint2 quant8_t(const uint4 &v, const Fp8Scale &sc) {
     const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(b[i]);
-        c[i] = e4m3x2(f.x, f.y, sc);
+        c[i] = e4m3x2<ONE>(f.x, f.y, sc);
     }
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
+__device__ __forceinline__ uint2 quant8(const uint4 &v, const Fp8Scale &sc) {
+    return sc.p1 == 1.0f ? quant8_t<true>(v, sc) : quant8_t<false>(v, sc);
+}
 
-__device__ __forceinline__ float amax8(const uint4 &v, float m) {
+// Largest magnitude of eight bf16 values folded into m (packed bf16 max of
+// the magnitudes: exact, NaN ignored as fmaxf ignores it).
+__device__ __forceinline__ __nv_bfloat162 amax8(const uint4 &v, __nv_bfloat162 m) {
     const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(b[i]);
-        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-    }
+    for (int i = 0; i < 4; ++i) m = __hmax2(m, __habs2(b[i]));
     return m;
+}
+__device__ __forceinline__ float amax_of(__nv_bfloat162 m) {
+    return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
 }
 
 // Block of 256 threads: expert e = blockIdx.y, columns [32 blockIdx.x, +32).
@@ -106,8 +115,8 @@ __global__ void __launch_bounds__(256) k_quant_weights(const __nv_bfloat16 *__re
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const int kk = 16 * c + 4 * v;
-            const uint32_t lo = e4m3x2(__bfloat162float(tile[kk][i]), __bfloat162float(tile[kk + 1][i]), s);
-            const uint32_t hi = e4m3x2(__bfloat162float(tile[kk + 2][i]), __bfloat162float(tile[kk + 3][i]), s);
+            const uint32_t lo = e4m3x2<false>(__bfloat162float(tile[kk][i]), __bfloat162float(tile[kk + 1][i]), s);
+            const uint32_t hi = e4m3x2<false>(__bfloat162float(tile[kk + 2][i]), __bfloat162float(tile[kk + 3][i]), s);
             word[v] = lo | (hi << 16);
         }
         *reinterpret_cast<uint4 *>(qe + k0 + 16 * c) = make_uint4(word[0], word[1], word[2], word[3]);
@@ -158,8 +167,10 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint4 *__restrict__ sr
                 const int c = tr + i * TPR;
                 v[i] = c < K8 ? __ldg(s_row + c) : make_uint4(0, 0, 0, 0);
             }
+            __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
 #pragma unroll
-            for (int i = 0; i < VPT; ++i) m = amax8(v[i], m);
+            for (int i = 0; i < VPT; ++i) m2 = amax8(v[i], m2);
+            m = amax_of(m2);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -212,8 +223,9 @@ __global__ void __launch_bounds__(256) k_quant_rows_long(const uint4 *__restrict
             continue;
         }
         const uint4 *s_row = src + (size_t)sr * K8;
-        float m = 0.0f;
-        for (int c = threadIdx.x; c < K8; c += 256) m = amax8(__ldg(s_row + c), m);
+        __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+        for (int c = threadIdx.x; c < K8; c += 256) m2 = amax8(__ldg(s_row + c), m2);
+        float m = amax_of(m2);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) s_max[warp] = m;

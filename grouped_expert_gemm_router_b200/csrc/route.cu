@@ -334,11 +334,15 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
         int ecol[EJ];
 #pragma unroll
         for (int j = 0; j < EJ; ++j) ecol[j] = min(es * EJ + j, E - 1);  // reads past E are clamped, unused
-        float acc[TB][EJ];
+        // sums of tokens 2i and 2i + 1 side by side: one packed fp32 FMA
+        // (fma.rn.f32x2) updates both, each element rounded exactly as a
+        // scalar fmaf would round it
+        static_assert(TB % 2 == 0, "tokens are processed in pairs");
+        float2 acc2[TB / 2][EJ];
 #pragma unroll
-        for (int i = 0; i < TB; ++i)
+        for (int i = 0; i < TB / 2; ++i)
 #pragma unroll
-            for (int j = 0; j < EJ; ++j) acc[i][j] = 0.0f;
+            for (int j = 0; j < EJ; ++j) acc2[i][j] = make_float2(0.0f, 0.0f);
 
         for (int s = 0; s < S - 1; ++s) {
             if (s < nchunks) issue(s, s);
@@ -364,18 +368,29 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
                     wb[j] = w0[E + ecol[j]];
                 }
 #pragma unroll
-                for (int i = 0; i < TB; ++i) {
-                    const float2 xv =
-                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)i * HC + 2 * p));
+                for (int i = 0; i < TB / 2; ++i) {
+                    const float2 xa = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i) * HC + 2 * p));
+                    const float2 xb = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i + 1) * HC + 2 * p));
+                    const float2 x0 = make_float2(xa.x, xb.x), x1 = make_float2(xa.y, xb.y);
 #pragma unroll
                     for (int j = 0; j < EJ; ++j) {
-                        acc[i][j] = fmaf(xv.x, wa[j], acc[i][j]);
-                        acc[i][j] = fmaf(xv.y, wb[j], acc[i][j]);
+                        acc2[i][j] = __ffma2_rn(x0, make_float2(wa[j], wa[j]), acc2[i][j]);
+                        acc2[i][j] = __ffma2_rn(x1, make_float2(wb[j], wb[j]), acc2[i][j]);
                     }
                 }
             }
             __syncthreads();  // stage c % S may be refilled from here on
         }
+        float acc[TB][EJ];
+#pragma unroll
+        for (int i = 0; i < TB / 2; ++i)
+#pragma unroll
+            for (int j = 0; j < EJ; ++j) {
+                acc[2 * i][j] = acc2[i][j].x;
+                acc[2 * i + 1][j] = acc2[i][j].y;
+            }
         // Fold the hidden-pair split inside the warp, then the warps' partial
         // sums in warp order (deterministic) through shared memory, which the
         // pipeline no longer needs.
