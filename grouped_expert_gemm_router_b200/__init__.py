@@ -38,7 +38,8 @@ ABI_FUNCTIONS = (
     "moe_set_wait_timeout_ns", "moe_status_string", "moe_last_error_string", "moe_version", "moe_permute_static",
     "moe_route_dispatch", "moe_gather", "moe_grouped_swiglu_gather", "moe_quantize_weights_fp8",
     "moe_quantize_rows_fp8", "moe_grouped_swiglu_fp8", "moe_grouped_down_fp8", "moe_forward_fp8",
-    "moe_grouped_down_combine", "moe_grouped_down_fp8_combine",
+    "moe_grouped_down_combine", "moe_grouped_down_fp8_combine", "moe_ep_overflow_rows", "moe_ep_workspace_bytes",
+    "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -142,6 +143,21 @@ def load_library(path: str = LIB_PATH):
     lib.moe_grouped_down_combine.restype = st
     lib.moe_grouped_down_fp8_combine.argtypes = [sp] + [vp] * 11
     lib.moe_grouped_down_fp8_combine.restype = st
+    i32 = ctypes.c_int32
+    lib.moe_ep_overflow_rows.argtypes = [sp, i32]
+    lib.moe_ep_overflow_rows.restype = ctypes.c_int64
+    lib.moe_ep_workspace_bytes.argtypes = [sp, i32]
+    lib.moe_ep_workspace_bytes.restype = ctypes.c_size_t
+    lib.moe_ep_local_shape.argtypes = [sp, i32, sp]
+    lib.moe_ep_local_shape.restype = st
+    lib.moe_ep_pack.argtypes = [sp, i32] + [vp] * 6
+    lib.moe_ep_pack.restype = st
+    lib.moe_ep_local_dispatch.argtypes = [sp, i32] + [vp] * 7
+    lib.moe_ep_local_dispatch.restype = st
+    lib.moe_ep_local_return.argtypes = [sp, i32] + [vp] * 5
+    lib.moe_ep_local_return.restype = st
+    lib.moe_ep_unpack.argtypes = [sp, i32] + [vp] * 4
+    lib.moe_ep_unpack.restype = st
     _lib = lib
     return lib
 
@@ -386,3 +402,40 @@ def quantize_layer_weights_fp8(shape, bufs, stream=None):
     moe_quantize_weights_fp8(shape, MOE_WEIGHTS_GATE_UP, bufs["w_gate"], bufs["wg_q"], bufs["wg_scale"], stream)
     moe_quantize_weights_fp8(shape, MOE_WEIGHTS_GATE_UP, bufs["w_up"], bufs["wu_q"], bufs["wu_scale"], stream)
     moe_quantize_weights_fp8(shape, MOE_WEIGHTS_DOWN, bufs["w_down"], bufs["wd_q"], bufs["wd_scale"], stream)
+
+
+# ---------------------------------------------------- expert-parallel dispatch --
+
+def moe_ep_overflow_rows(shape, G) -> int:
+    return int(load_library().moe_ep_overflow_rows(ctypes.byref(shape), int(G)))
+
+
+def moe_ep_workspace_bytes(shape, G) -> int:
+    return int(load_library().moe_ep_workspace_bytes(ctypes.byref(shape), int(G)))
+
+
+def moe_ep_local_shape(shape, G) -> MoeShape:
+    out = MoeShape()
+    _check(load_library().moe_ep_local_shape(ctypes.byref(shape), int(G), ctypes.byref(out)), "moe_ep_local_shape")
+    return out
+
+
+def moe_ep_pack(shape, G, x_perm, ws, send_ovf, send_meta, ep_ws, stream=None):
+    _check(load_library().moe_ep_pack(ctypes.byref(shape), int(G), _ptr(x_perm), _ptr(ws), _ptr(send_ovf),
+                                      _ptr(send_meta), _ptr(ep_ws), _stream(stream)), "moe_ep_pack")
+
+
+def moe_ep_local_dispatch(shape, G, recv_meta, recv_cap, recv_ovf, x_loc, ws_loc, ep_ws, stream=None):
+    _check(load_library().moe_ep_local_dispatch(ctypes.byref(shape), int(G), _ptr(recv_meta), _ptr(recv_cap),
+                                                _ptr(recv_ovf), _ptr(x_loc), _ptr(ws_loc), _ptr(ep_ws),
+                                                _stream(stream)), "moe_ep_local_dispatch")
+
+
+def moe_ep_local_return(shape, G, y_loc, back_cap, back_ovf, ep_ws, stream=None):
+    _check(load_library().moe_ep_local_return(ctypes.byref(shape), int(G), _ptr(y_loc), _ptr(back_cap),
+                                              _ptr(back_ovf), _ptr(ep_ws), _stream(stream)), "moe_ep_local_return")
+
+
+def moe_ep_unpack(shape, G, recv_back_ovf, y, ep_ws, stream=None):
+    _check(load_library().moe_ep_unpack(ctypes.byref(shape), int(G), _ptr(recv_back_ovf), _ptr(y), _ptr(ep_ws),
+                                        _stream(stream)), "moe_ep_unpack")

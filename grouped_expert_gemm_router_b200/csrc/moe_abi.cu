@@ -35,6 +35,17 @@ cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int sr
                               cudaStream_t stream);
 cudaError_t launch_quant_tokens(const moe_shape &s, const void *x, void *q, float *scale, int num_sms,
                                 cudaStream_t stream);
+int64_t ep_overflow_rows(const moe_shape &s, int G);
+size_t ep_workspace_bytes(const moe_shape &s, int G);
+cudaError_t launch_ep_pack(const moe_shape &s, int G, const void *x_perm, const WsLayout &L, void *ws, void *send_ovf,
+                           int32_t *send_meta, void *ep_ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_local_dispatch(const moe_shape &s, int G, const int32_t *recv_meta, const void *recv_cap,
+                                     const void *recv_ovf, void *x_loc, const WsLayout &Lloc, void *ws_loc,
+                                     void *ep_ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_local_return(const moe_shape &s, int G, const void *y_loc, void *back_cap, void *back_ovf,
+                                   void *ep_ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_unpack(const moe_shape &s, int G, const void *recv_back_ovf, void *y, void *ep_ws, int num_sms,
+                             cudaStream_t stream);
 }  // namespace moe
 
 using namespace moe;
@@ -48,6 +59,8 @@ constexpr uint32_t kKnownFlags = MOE_FLAG_CAPACITY | MOE_FLAG_LOGITS_IN | MOE_FL
                                   MOE_FLAG_TEST_STALL_SCAN | MOE_FLAG_TEST_STALL_GEMM;
 
 bool aligned(const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
+// A buffer of zero rows may be null.
+bool aligned_or_empty(const void *p, uintptr_t a, bool empty) { return (empty && p == nullptr) || aligned(p, a); }
 
 moe_status cuda_fail(cudaError_t e, const char *where) {
     std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
@@ -448,6 +461,108 @@ moe_status moe_forward_fp8(const moe_shape *s, const moe_forward_fp8_args *a, vo
     st = moe_grouped_down_fp8(s, a->h_q, a->h_scale, a->wd_q, a->wd_scale, a->y, ws, stream);
     if (st != MOE_OK) return st;
     return moe_combine(s, a->y, a->dest_row, a->topk_w, a->out, stream);
+}
+
+// ------------------------------------------------------------ expert parallel --
+namespace {
+moe_status check_ep(const moe_shape *s, int32_t G) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if (!(s->flags & MOE_FLAG_CAPACITY) || G < 1 || s->E % G != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int64_t S = ep_overflow_rows(*s, G);
+    const int64_t Tloc = (int64_t)G * ((int64_t)(s->E / G) * s->C + S);
+    if (Tloc < 1 || Tloc >= (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+moe_shape ep_local(const moe_shape *s, int32_t G) {
+    const int64_t S = ep_overflow_rows(*s, G);
+    moe_shape l;
+    l.T = (int32_t)((int64_t)G * ((int64_t)(s->E / G) * s->C + S));
+    l.H = s->H;
+    l.F = s->F;
+    l.E = s->E / G;
+    l.k = 1;
+    l.C = 0;
+    l.flags = 0;
+    return l;
+}
+}  // namespace
+
+int64_t moe_ep_overflow_rows(const moe_shape *s, int32_t G) {
+    if (check_ep(s, G) != MOE_OK) return -1;
+    return ep_overflow_rows(*s, G);
+}
+
+size_t moe_ep_workspace_bytes(const moe_shape *s, int32_t G) {
+    if (check_ep(s, G) != MOE_OK) return 0;
+    return ep_workspace_bytes(*s, G);
+}
+
+moe_status moe_ep_local_shape(const moe_shape *s, int32_t G, moe_shape *local) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    if (!local) return MOE_ERR_INVALID_ARG;
+    *local = ep_local(s, G);
+    return check_shape(local);
+}
+
+moe_status moe_ep_pack(const moe_shape *s, int32_t G, const void *x_perm, const void *ws, void *send_ovf,
+                       int32_t *send_meta, void *ep_ws, void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    const bool no_ovf = ep_overflow_rows(*s, G) == 0;
+    if (!aligned(x_perm, 16) || !aligned_or_empty(send_ovf, 16, no_ovf) || !aligned(send_meta, 4) ||
+        !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(const_cast<void *>(ws))) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_ep_pack(*s, G, x_perm, L, const_cast<void *>(ws), send_ovf, send_meta, ep_ws, sms,
+                                   (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_pack");
+}
+
+moe_status moe_ep_local_dispatch(const moe_shape *s, int32_t G, const int32_t *recv_meta, const void *recv_cap,
+                                 const void *recv_ovf, void *x_loc, void *ws_loc, void *ep_ws, void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(recv_meta, 4) || !aligned_or_empty(recv_cap, 16, s->C == 0) ||
+        !aligned_or_empty(recv_ovf, 16, ep_overflow_rows(*s, G) == 0) || !aligned(x_loc, 16) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws_loc)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const moe_shape l = ep_local(s, G);
+    const WsLayout Lloc = layout_of(&l);
+    cudaError_t e = launch_ep_local_dispatch(*s, G, recv_meta, recv_cap, recv_ovf, x_loc, Lloc, ws_loc, ep_ws, sms,
+                                             (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_local_dispatch");
+}
+
+moe_status moe_ep_local_return(const moe_shape *s, int32_t G, const void *y_loc, void *back_cap, void *back_ovf,
+                               void *ep_ws, void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(y_loc, 16) || !aligned_or_empty(back_cap, 16, s->C == 0) ||
+        !aligned_or_empty(back_ovf, 16, ep_overflow_rows(*s, G) == 0) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e = launch_ep_local_return(*s, G, y_loc, back_cap, back_ovf, ep_ws, sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_local_return");
+}
+
+moe_status moe_ep_unpack(const moe_shape *s, int32_t G, const void *recv_back_ovf, void *y, void *ep_ws,
+                         void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned_or_empty(recv_back_ovf, 16, ep_overflow_rows(*s, G) == 0) || !aligned(y, 16) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e = launch_ep_unpack(*s, G, recv_back_ovf, y, ep_ws, sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_unpack");
 }
 
 moe_status moe_read_status(void *ws, void *stream, uint32_t *device_status, int clear) {

@@ -401,6 +401,83 @@ typedef struct {
  * moe_quantize_weights_fp8. */
 MOE_API moe_status moe_forward_fp8(const moe_shape *shape, const moe_forward_fp8_args *args, void *ws, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Expert-parallel Cap-and-Spill dispatch ("Cap-and-Spill" critique page,
+ * juhe.plus, section "Cap-and-Spill": a capacity pass with C slots per
+ * expert, then a pass for the compacted overflow, whose buffer is sized for
+ * the largest possible overflow so that it exists before the routing is
+ * known; no token is dropped and no host synchronisation sits between the
+ * passes).
+ *
+ * G ranks, E experts (E divisible by G); rank d owns experts
+ * [d*E/G, (d+1)*E/G) and its local expert weights are the [E/G, ...] slices of
+ * the layer's weights.  `shape` is the global shape of one rank's batch (its
+ * T tokens over all E experts) and must carry MOE_FLAG_CAPACITY.  One layer on
+ * rank r, buffers as moe_forward's plus the EP ones (rows of H bf16 values):
+ *   1. moe_route_dispatch + moe_gather: x_perm in the capacity layout.
+ *   2. moe_ep_pack: send_meta [G][2][E/G] int32 (each destination's capacity
+ *      and overflow counts) and send_ovf [G][S] rows (each destination's
+ *      compacted overflow rows at the start of its slot), S =
+ *      moe_ep_overflow_rows.
+ *   3. all-to-all (equal splits) of x_perm[0, E*C) into recv_cap
+ *      [G][E/G*C] rows (pass 1), of send_meta into recv_meta, and of
+ *      send_ovf into recv_ovf [G][S] rows (pass 2).
+ *   4. moe_ep_local_dispatch: the received rows in expert-contiguous order in
+ *      x_loc and the local GEMM schedule in ws_loc, a workspace of the local
+ *      shape (moe_ep_local_shape: T = G*(E/G*C + S), E/G experts, k = 1).
+ *   5. moe_grouped_swiglu / moe_grouped_down (or their fp8 forms) on the
+ *      local shape: x_loc -> h_loc -> y_loc with the local weights.
+ *   6. moe_ep_local_return: y_loc rows into back_cap [G][E/G*C] and back_ovf
+ *      [G][S] at the positions their inputs arrived at.
+ *   7. all-to-all of back_cap into y[0, E*C) and of back_ovf into
+ *      recv_back_ovf [G][S] rows.
+ *   8. moe_ep_unpack: the overflow rows' results into y's overflow region.
+ *   9. moe_combine: out from y, dest_row, topk_w -- the result equals
+ *      moe_forward's on the rank's tokens with all E experts.
+ * ep_ws: moe_ep_workspace_bytes bytes, 16-byte aligned; written by
+ * moe_ep_pack and moe_ep_local_dispatch and read by the later steps of the
+ * same layer.  Row buffers are caller-owned device memory, 16-byte aligned;
+ * the capacity buffers (recv_cap, back_cap) may be null when C = 0 and the
+ * overflow buffers (send_ovf, recv_ovf, back_ovf, recv_back_ovf) when S = 0.
+ * Errors: MOE_ERR_UNSUPPORTED_SHAPE (no MOE_FLAG_CAPACITY, G < 1, E not
+ * divisible by G, local T >= 2^30), MOE_ERR_INVALID_ARG (null or misaligned
+ * pointer), MOE_ERR_CUDA (launch failure).  Counts in recv_meta that exceed
+ * what the buffers hold (never produced by moe_ep_pack) are clamped and set
+ * MOE_DEV_BAD_ROW in ws_loc's status.
+ * ------------------------------------------------------------------------ */
+
+/* S: rows of one (source, destination) overflow slot, min(k, E/G) *
+ * max(0, T - C) (one source's tokens send at most min(k, E/G) pairs each to
+ * one destination, and an expert overflows by at most T - C).  -1 for an
+ * unsupported shape or G. */
+MOE_API int64_t moe_ep_overflow_rows(const moe_shape *shape, int32_t G);
+
+/* Bytes of the EP workspace, or 0 for an unsupported shape or G. */
+MOE_API size_t moe_ep_workspace_bytes(const moe_shape *shape, int32_t G);
+
+/* The local shape of step 5: T = G*(E/G*C + S), H, F, E/G experts, k = 1,
+ * C = 0, flags 0. */
+MOE_API moe_status moe_ep_local_shape(const moe_shape *shape, int32_t G, moe_shape *local);
+
+/* Step 2 (reads the capacity and overflow counts moe_route_dispatch /
+ * moe_permute left in ws). */
+MOE_API moe_status moe_ep_pack(const moe_shape *shape, int32_t G, const void *x_perm, const void *ws,
+                               void *send_ovf, int32_t *send_meta, void *ep_ws, void *stream);
+
+/* Step 4.  ws_loc: a workspace of the local shape, initialised once
+ * (moe_workspace_init with the local shape). */
+MOE_API moe_status moe_ep_local_dispatch(const moe_shape *shape, int32_t G, const int32_t *recv_meta,
+                                         const void *recv_cap, const void *recv_ovf, void *x_loc, void *ws_loc,
+                                         void *ep_ws, void *stream);
+
+/* Step 6. */
+MOE_API moe_status moe_ep_local_return(const moe_shape *shape, int32_t G, const void *y_loc, void *back_cap,
+                                       void *back_ovf, void *ep_ws, void *stream);
+
+/* Step 8. */
+MOE_API moe_status moe_ep_unpack(const moe_shape *shape, int32_t G, const void *recv_back_ovf, void *y, void *ep_ws,
+                                 void *stream);
+
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
 

@@ -163,3 +163,23 @@ def check_tile_schedule(r, shape, counts, offsets, spill_off):
     assert r["row_cap"] == max(16, max(req))
     if r["row_cap"] < 256:
         assert all(gts[g + 1] - gts[g] == (1 if counts[e] else 0) for g, e in enumerate(order))
+
+
+def oracle_layer(orc, L, cfg, logits_gpu):
+    """Oracle routing from the GPU logits (same fp32 logits on both sides),
+    then the oracle's own dispatch, experts and combine."""
+    idx, w, _ = orc.topk_softmax(logits_gpu, cfg.k)
+    capped = cfg.C > 0
+    d = orc.dispatch(idx, cfg.E, C=cfg.C, capped=capped)
+    P = d["P"]
+    x_perm = np.zeros((P, cfg.H), np.uint16)
+    h = np.zeros((P, cfg.F), np.uint16)
+    y = np.zeros((P, cfg.H), np.uint16)
+    flat = idx.reshape(-1)
+    for i, r in enumerate(d["dest_row"]):
+        t, e = i // cfg.k, flat[i]
+        x_perm[r] = L.x[t]
+        h[r] = orc.swiglu_row(L.x[t], L.w_gate[e], L.w_up[e])
+        y[r] = orc.down_row(h[r], L.w_down[e])
+    out = orc.combine(y, d["dest_row"], w)
+    return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)

@@ -9,6 +9,7 @@ import grouped_expert_gemm_router_b200 as moe
 import synth
 from gpu_util import (LOGIT_TOL, WEIGHT_TOL, DeviceLayer, assert_close_bf16, bf16_host, check_tile_schedule, host,
                       run_steps, shape_of)
+from gpu_util import oracle_layer as _oracle_full
 
 pytestmark = pytest.mark.gpu
 
@@ -24,26 +25,6 @@ CASES = {
     "E1_dense": synth.LayerConfig("t", 300, 128, 256, 1, 1, seed=6),
     "many_experts_E256_k8": synth.LayerConfig("t", 96, 128, 128, 256, 8, alpha=0.5, seed=7),
 }
-
-
-def _oracle_full(orc, L, cfg, logits_gpu):
-    """Oracle routing from the GPU logits (same fp32 logits on both sides),
-    then the oracle's own dispatch, experts and combine."""
-    idx, w, _ = orc.topk_softmax(logits_gpu, cfg.k)
-    capped = cfg.C > 0
-    d = orc.dispatch(idx, cfg.E, C=cfg.C, capped=capped)
-    P = d["P"]
-    x_perm = np.zeros((P, cfg.H), np.uint16)
-    h = np.zeros((P, cfg.F), np.uint16)
-    y = np.zeros((P, cfg.H), np.uint16)
-    flat = idx.reshape(-1)
-    for i, r in enumerate(d["dest_row"]):
-        t, e = i // cfg.k, flat[i]
-        x_perm[r] = L.x[t]
-        h[r] = orc.swiglu_row(L.x[t], L.w_gate[e], L.w_up[e])
-        y[r] = orc.down_row(h[r], L.w_down[e])
-    out = orc.combine(y, d["dest_row"], w)
-    return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)
 
 
 @pytest.mark.parametrize("name", list(CASES))
