@@ -16,6 +16,11 @@ Multi-GPU: the path has no exchange step, so N GPUs run N independent
 replicas (one process per GPU, its own token batch); the only collectives are
 the barrier and the max-over-ranks of the elapsed time.
 
+Also reported: the end-to-end rate with host copies (pipelined across steps,
+and serial), the fp8 layer, every other workload (per_config), the combine
+fused into the down GEMM, and the expert-parallel layer with 8 ranks emulated
+on one GPU (ep: per-rank kernel times and the bytes of each all-to-all pass).
+
 Prints one JSON line (rank 0).
 """
 from __future__ import annotations
@@ -55,6 +60,8 @@ def parse_args():
                    help="time the headline workload only (default: every other workload too, on one GPU)")
     p.add_argument("--per-config-steps", type=int, default=20)
     p.add_argument("--no-fp8", action="store_true", help="skip the fp8 (e4m3) variant of the layer")
+    p.add_argument("--no-ep", action="store_true",
+                   help="skip the expert-parallel layer (8 ranks emulated on one GPU, decode-shaped workload)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     p.add_argument("--ref-budget-s", type=float, default=150.0)
     return p.parse_args()
@@ -81,7 +88,8 @@ def workload(args):
 def config_json(cfg, extra=None):
     d = {"workload": cfg.name + ("" if cfg.alpha in (0.0,) else "-alpha%g" % cfg.alpha), "T": cfg.T, "H": cfg.H,
          "F": cfg.F, "E": cfg.E, "k": cfg.k, "C": cfg.C, "alpha": cfg.alpha, "seed": cfg.seed,
-         "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)",
+         "l2": "flushed between timed steps (256 MiB write, then 256 MiB read); not in the pipelined e2e, "
+               "whose per-step inputs (the expert weights) are larger than L2 on every workload but the tiny one",
          "timing": "moe_forward captured once as a CUDA graph, replayed per step, CUDA events around each replay"}
     if extra:
         d.update(extra)
@@ -553,6 +561,132 @@ class Bench:
         (e2e_ms,) = max_over_ranks([e2e_ms], dev)
         return e2e_ms
 
+    def measure_ep(self, cfg, L, G, steps, warmup):
+        """The expert-parallel Cap-and-Spill layer with G ranks held by this
+        process on its one GPU: each rank's phases run on its own buffers
+        with CUDA events around each, the all-to-alls are carried out as
+        device copies (untimed: on G GPUs they cross NVLink).  L2 cleaned
+        before every step.  Returns per-phase device times summed over the
+        ranks, and each rank's overflow rows."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        from grouped_expert_gemm_router_b200.ep import CapAndSpillEP, exchange_in_process
+        torch, dev, stream = self.torch, self.dev, self.stream
+
+        def dev_bf16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=True)
+        wg, wu, wd = dev_bf16(L.w_gate), dev_bf16(L.w_up), dev_bf16(L.w_down)
+        wr = torch.from_numpy(L.w_router).to(dev)
+        bias = None if L.bias is None else torch.from_numpy(L.bias).to(dev)
+        xs = [dev_bf16(replica_tokens(cfg, r, L)) for r in range(G)]
+        ranks = [CapAndSpillEP(shape, G, dev) for _ in range(G)]
+        Eg = cfg.E // G
+        sl = [slice(r * Eg, (r + 1) * Eg) for r in range(G)]
+        phases = ("route_and_pack", "receive", "experts", "send_back", "finish")
+        calls = {
+            "route_and_pack": lambda r: ranks[r].route_and_pack(xs[r], wr, bias, stream),
+            "receive": lambda r: ranks[r].receive(stream),
+            "experts": lambda r: ranks[r].experts(wg[sl[r]], wu[sl[r]], wd[sl[r]], stream),
+            "send_back": lambda r: ranks[r].send_back(stream),
+            "finish": lambda r: ranks[r].finish(stream),
+        }
+
+        def step(timed):
+            ev = {}
+            for ph in phases:
+                if ph == "receive":
+                    exchange_in_process(ranks, "exchange_in")
+                if ph == "finish":
+                    exchange_in_process(ranks, "exchange_out")
+                for r in range(G):
+                    if timed:
+                        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                        calls[ph](r)
+                        c.record(stream)
+                        ev[(ph, r)] = (a, c)
+                    else:
+                        calls[ph](r)
+            return ev
+
+        for _ in range(warmup):
+            self.flush()
+            step(False)
+        self.barrier()
+        evs = []
+        for _ in range(steps):
+            self.flush()
+            evs.append(step(True))
+        self.barrier()
+        per_phase = {ph: float(np.mean([sum(e[(ph, r)][0].elapsed_time(e[(ph, r)][1]) for r in range(G))
+                                         for e in evs])) * 1e3 for ph in phases}
+        lay = moe.moe_workspace_layout(shape)
+        spill = [int(ep.ws[lay.total_spill:lay.total_spill + 4].cpu().numpy().view(np.int32)[0]) for ep in ranks]
+        status = [moe.moe_read_status(ep.ws) | moe.moe_read_status(ep.ws_loc) for ep in ranks]
+        S = ranks[0].S
+        # the single-GPU layer on rank 0's tokens, same protocol, for comparison
+        shp1, b1 = self.upload(cfg, L, replica_tokens(cfg, 0, L))
+        m1 = self.measure(cfg, shp1, b1, steps, warmup)
+        del b1, ranks
+        return {"G": G, "S": S, "per_phase_us_all_ranks": per_phase, "overflow_rows": spill,
+                "device_status": status, "single_gpu_layer_us": m1["total_ms"] / steps * 1e3}
+
+    def e2e_pipelined(self, cfg, shape, b, x_rank, fwd_bufs, steps, warmup):
+        """End to end as a serving loop runs it: step i's tokens are copied in
+        on one copy stream while step i-1's layer runs, and step i-1's output
+        is copied out on another while step i's runs (x and out
+        double-buffered on the device).  Timed from the first copy in to the
+        last copy out; every step still moves its own tokens and output
+        across the host link.  No L2 cleaning between steps (it would sit
+        inside the timed interval): the expert weights each step streams are
+        larger than L2."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        torch, dev, comp = self.torch, self.dev, self.stream
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        x_host = torch.from_numpy(np.ascontiguousarray(x_rank).view(np.int16)).view(torch.bfloat16).pin_memory()
+        outs_h = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        xs = [b["x"], torch.empty_like(b["x"])]
+        outs = [fwd_bufs["out"], torch.empty_like(fwd_bufs["out"])]
+        bufs = [{**fwd_bufs, "x": xs[j], "out": outs[j]} for j in range(2)]
+        args = [moe.forward_args(bb) for bb in bufs]
+
+        def run(n):
+            ev_up = [torch.cuda.Event() for _ in range(n)]
+            ev_comp = [torch.cuda.Event() for _ in range(n)]
+            ev_down = [torch.cuda.Event() for _ in range(n)]
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record(up)
+            for i in range(n):
+                j = i % 2
+                if i >= 2:
+                    up.wait_event(ev_comp[i - 2])       # the layer of step i-2 has read xs[j]
+                with torch.cuda.stream(up):
+                    xs[j].copy_(x_host, non_blocking=True)
+                ev_up[i].record(up)
+                comp.wait_event(ev_up[i])
+                if i >= 2:
+                    comp.wait_event(ev_down[i - 2])     # outs[j] of step i-2 is on the host
+                moe.moe_forward(shape, bufs[j], b["ws"], comp, args=args[j])
+                ev_comp[i].record(comp)
+                down.wait_event(ev_comp[i])
+                with torch.cuda.stream(down):
+                    outs_h[j].copy_(outs[j], non_blocking=True)
+                ev_down[i].record(down)
+            end.record(down)
+            return start, end
+
+        run(warmup)
+        self.barrier()
+        start, end = run(steps)
+        self.barrier()
+        (ms,) = max_over_ranks([start.elapsed_time(end)], dev)
+        return ms
+
 
 def summarize(cfg, m, steps, world, peaks, peak_src):
     """Throughput, per-kernel times and roofline fractions of one measured
@@ -612,6 +746,40 @@ def summarize(cfg, m, steps, world, peaks, peak_src):
         "routing": routing_stats(counts, cfg.C),
         "device_status": m["status"],
         "wall_s_timed_region": m["wall"],
+    }
+
+
+# Peer copy bandwidth per direction between two B200s over NVLink 5, measured
+# on this machine type (an exchange model only: no run here had two GPUs).
+NVLINK_PEER_GBS = 770.0
+
+
+def summarize_ep(cfg, e, peaks):
+    """The expert-parallel layer per rank: kernel time of each phase, and the
+    bytes each rank sends per all-to-all pass (received bytes are the same)."""
+    G, S, row = e["G"], e["S"], cfg.H * 2
+    Eg = cfg.E // G
+    per_rank = {ph: t / G for ph, t in e["per_phase_us_all_ranks"].items()}
+    p1, p2, meta = cfg.E * cfg.C * row, G * S * row, G * 2 * Eg * 4
+    real = float(sum(e["overflow_rows"])) / G * row
+    w_bytes = 3 * Eg * cfg.H * cfg.F * 2
+    t_exp = per_rank["experts"] * 1e-6
+    return {
+        "workload": workload_name(cfg), "G": G,
+        "ranks": "G ranks emulated on one GPU (each rank's phases on its own buffers); the all-to-alls done as "
+                 "device copies and not timed",
+        "per_rank_us": per_rank, "per_rank_kernels_us": sum(per_rank.values()),
+        "single_gpu_layer_us": e["single_gpu_layer_us"],
+        "experts_roofline": {"bound": "hbm", "bytes": w_bytes, "achieved": w_bytes / t_exp / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": w_bytes / t_exp / 1e9 / peaks["hbm_gbs"],
+                             "note": "the rank's expert weights over the local SwiGLU + down time"},
+        "exchange_per_rank": {"pass1_bytes": p1, "pass2_bytes": p2, "meta_bytes": meta,
+                              "real_overflow_bytes": real, "pass2_padding_frac": 1.0 - real / p2 if p2 else 0.0,
+                              "nvlink_model_us": 2 * (p1 + p2 + meta) / (NVLINK_PEER_GBS * 1e9) * 1e6,
+                              "nvlink_model": "dispatch and return passes, each rank's sent bytes at %g GB/s per "
+                                              "direction (a model, not a measurement)" % NVLINK_PEER_GBS},
+        "device_status": e["device_status"],
     }
 
 
@@ -706,6 +874,7 @@ def run_ours(args):
     K = args.steps
     m = bench.measure(cfg, shape, b, K, args.warmup)
     e2e_ms = bench.e2e(cfg, shape, b, x_rank, m["fwd_bufs"], K)
+    e2e_pipe_ms = bench.e2e_pipelined(cfg, shape, b, x_rank, m["fwd_bufs"], K, args.warmup)
     peaks, peak_src = load_peaks()
     m8 = None if args.no_fp8 else bench.measure_fp8(cfg, shape, b, K, args.warmup)
 
@@ -722,8 +891,18 @@ def run_ours(args):
             "kernels": s["kernels"],
             "eager_entry_points_ms_per_step": s["eager_entry_points_ms_per_step"],
             "fused_combine": s["fused_combine"],
-            "e2e": {"value": whole_job_rate(cfg.T, K, world, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2},
+            "e2e": {"value": whole_job_rate(cfg.T, K, world, e2e_pipe_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+                    "ms_per_step": e2e_pipe_ms / K,
+                    "mode": "pipelined: step i's tokens copied in from pinned host memory and step i-1's output "
+                            "copied out to pinned host memory on two copy streams while the layer runs; timed "
+                            "from the first copy in to the last copy out; L2 not cleaned between steps (expert "
+                            "weights: %.3f GB)" % (3.0 * cfg.E * cfg.H * cfg.F * 2 / 1e9)},
+            "e2e_serial": {"value": whole_job_rate(cfg.T, K, world, e2e_ms), "unit": "tokens/s",
+                           "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 2,
+                           "ms_per_step": e2e_ms / K,
+                           "mode": "copy in, moe_forward, copy out on one stream, each step timed alone; "
+                                   "L2 cleaned before each step outside the timed interval"},
             "gpu_launches": forward_launches(cfg) * K,
             "clocks": s["clocks"],
             "routing": s["routing"],
@@ -758,12 +937,29 @@ def run_ours(args):
             gc.collect()
             torch.cuda.empty_cache()
 
+    # the expert-parallel layer on the decode-shaped workload (C = 16), 8 ranks
+    # emulated on this GPU
+    ep = None
+    if world == 1 and not args.no_ep:
+        import synth
+        t0 = time.time()
+        ce = synth.CONFIGS[4]
+        Le = synth.make_layer(ce)
+        ep = summarize_ep(ce, bench.measure_ep(ce, Le, 8, min(K, args.per_config_steps), min(args.warmup, 5)), peaks)
+        log("expert-parallel %s G=8: %.1f us of kernels per rank (%.1f s)" % (ce.name, ep["per_rank_kernels_us"],
+                                                                              time.time() - t0))
+        del Le
+        gc.collect()
+        torch.cuda.empty_cache()
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         if per_config is not None:
             result["per_config"] = per_config
+        if ep is not None:
+            result["ep"] = ep
         if not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(cfg, L, args.cpu_budget_s)
         print(json.dumps(result), flush=True)

@@ -20,7 +20,7 @@ and the combine.  This module allocates the buffers and calls the entry points
 and the collectives in order.
 
 The layer's steps are exposed as phases (route_and_pack, exchange_in,
-local_experts, exchange_out, finish) so that the exchange can be any function
+local_experts = receive + experts + send_back, exchange_out, finish) so that the exchange can be any function
 with the semantics of torch.distributed.all_to_all_single(out, inp): forward()
 uses the process group's; one process can drive several ranks' phases with an
 exchange that copies between their buffers.
@@ -97,16 +97,29 @@ class CapAndSpillEP:
         all_to_all(self.recv_meta, self.send_meta)
         all_to_all(self.recv_ovf, self.send_ovf)
 
-    def local_experts(self, w_gate, w_up, w_down, stream=None):
-        """The received rows of this rank's experts through the grouped GEMMs
-        (weights: this rank's [E/G, ...] slices), and back to the return
-        buffers."""
-        s, L = self.shape, self.local
-        moe.moe_ep_local_dispatch(s, self.G, self.recv_meta, self.recv_cap, self.recv_ovf, self.x_loc, self.ws_loc,
-                                  self.ep_ws, stream)
+    def receive(self, stream=None):
+        """The received rows in the local expert-contiguous layout, and the
+        local GEMM schedule."""
+        moe.moe_ep_local_dispatch(self.shape, self.G, self.recv_meta, self.recv_cap, self.recv_ovf, self.x_loc,
+                                  self.ws_loc, self.ep_ws, stream)
+
+    def experts(self, w_gate, w_up, w_down, stream=None):
+        """The grouped GEMMs of this rank's experts (weights: its [E/G, ...]
+        slices) on the received rows."""
+        L = self.local
         moe.moe_grouped_swiglu(L, self.x_loc, w_gate, w_up, self.h_loc, self.ws_loc, stream)
         moe.moe_grouped_down(L, self.h_loc, w_down, self.y_loc, self.ws_loc, stream)
-        moe.moe_ep_local_return(s, self.G, self.y_loc, self.back_cap, self.back_ovf, self.ep_ws, stream)
+
+    def send_back(self, stream=None):
+        """Each result row to the position its input arrived at in the
+        return buffers."""
+        moe.moe_ep_local_return(self.shape, self.G, self.y_loc, self.back_cap, self.back_ovf, self.ep_ws, stream)
+
+    def local_experts(self, w_gate, w_up, w_down, stream=None):
+        """receive, experts, send_back."""
+        self.receive(stream)
+        self.experts(w_gate, w_up, w_down, stream)
+        self.send_back(stream)
 
     def exchange_out(self, all_to_all):
         """The two passes back: results of the capacity rows straight into y,
