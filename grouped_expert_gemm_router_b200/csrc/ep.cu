@@ -16,15 +16,17 @@
 // pairs each to one destination, and an expert's overflow is at most T - C),
 // an equal-split all-to-all as well.
 //
-// k_ep_plan_send   per destination: its experts' capacity and overflow
-//                  counts (sent ahead of the rows) and the range of its
-//                  overflow rows (the pack and unpack copies).
+// k_ep_spill_rows  the overflow rows between x_perm's compacted overflow
+//                  region and the per-destination slots (pack: also the
+//                  counts sent ahead of the rows; unpack: the same copies
+//                  reversed), a warp per row over every block.
 // k_ep_plan_recv   on the receiving rank, from the counts of every source:
 //                  an expert-contiguous local layout (per expert, each
-//                  source's capacity rows then its overflow rows), the copy
-//                  segments into it and back, and the local grouped-GEMM
-//                  schedule (the block schedule builder of the dispatch).
-// k_copy_segments  row copies by segment list, forward or reversed.
+//                  source's capacity rows then its overflow rows), its GEMM
+//                  schedule (the block schedule builder of the dispatch) and
+//                  the source of every local row.
+// k_ep_local_rows  the received rows into the local layout, or the local
+//                  results back to the return buffers, a warp per row.
 #include <cuda_bf16.h>
 
 #include "dispatch_block.cuh"
@@ -33,107 +35,156 @@ namespace moe {
 
 namespace {
 
-constexpr int kSegThreads = 256;
+constexpr int kRowThreads = 256;
+constexpr int kRowWarps = kRowThreads / 32;
 
-// Per destination d: meta[d][0][e] = capacity count, meta[d][1][e] =
-// overflow count of its expert d E_g + e; seg[d] = {first overflow row in
-// x_perm, first row of d's slot in the send buffer, rows, 0}.
-__global__ void __launch_bounds__(kSegThreads) k_ep_plan_send(WsPtrs ws, int E, int G, int C, int S,
-                                                              int32_t *meta, int4 *seg) {
-    pdl_trigger();
-    pdl_wait();
-    const int Eg = E / G;
-    for (int i = threadIdx.x; i < E; i += kSegThreads) {
-        const int d = i / Eg, e = i % Eg;
-        meta[(size_t)d * 2 * Eg + e] = ws.cap_cnt[i];
-        meta[(size_t)d * 2 * Eg + Eg + e] = ws.spill_cnt[i];
-    }
-    for (int d = threadIdx.x; d < G; d += kSegThreads) {
-        const int a = ws.spill_off[d * Eg], b = ws.spill_off[(d + 1) * Eg];
-        int len = b - a;
-        if (len > S) {  // cannot happen for a valid routing; never copy past the slot
-            atomicOr(ws.status, MOE_DEV_BAD_ROW);
-            len = S;
-        }
-        seg[d] = make_int4(E * C + a, d * S, len, 0);
-    }
+// One row of H8 16-byte vectors, by one warp.
+__device__ __forceinline__ void copy_row(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8, int lane) {
+    for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
 }
 
-// Rows source s sent for local expert e, clamped to what the buffers hold
-// (capacity rows to C, each source's overflow rows to its slot of S rows);
-// counts from moe_ep_pack never need the clamp.  ovf: the source's overflow
-// rows before expert e's in its slot.
-__device__ inline void ep_recv_counts(const int32_t *meta, int s, int e, int Eg, int C, int S, int &nc, int &no,
-                                      int &ovf, bool &bad) {
-    const int32_t *m = meta + (size_t)s * 2 * Eg;
-    ovf = 0;
-    for (int e2 = 0; e2 < e; ++e2) ovf += min(max(m[Eg + e2], 0), S - ovf);
-    const int rc = m[e], ro = m[Eg + e];
-    nc = min(max(rc, 0), C);
-    no = min(max(ro, 0), S - ovf);
-    bad = nc != rc || no != ro;
+// Overflow row q of x_perm (row E C + q) belongs to destination d, the last
+// with starts[d * stride] <= q, and sits at row d S + (q - starts[d * stride])
+// of the slots.  pack (reverse = 0): a = x_perm, b = send slots, b <- a, and
+// block 0 writes meta (per destination: its experts' capacity counts, then
+// their overflow counts) and the destination starts into ep_starts for
+// unpack; unpack (reverse = 1): a = y, b = received slots, a <- b, with the
+// starts read back from ep_starts.
+__global__ void __launch_bounds__(kRowThreads) k_ep_spill_rows(WsPtrs ws, const int32_t *ep_starts_in, int E, int G,
+                                                               int C, int S, int P, int H8, uint4 *a, uint4 *b,
+                                                               int reverse, int32_t *meta, int32_t *ep_starts_out) {
+    __shared__ int starts[kMaxExperts + 1];
+    pdl_trigger();
+    pdl_wait();
+    const int Eg = E / G, tid = threadIdx.x;
+    for (int d = tid; d <= G; d += kRowThreads) starts[d] = reverse ? ep_starts_in[d] : ws.spill_off[d * Eg];
+    if (!reverse && blockIdx.x == 0) {
+        for (int i = tid; i < E; i += kRowThreads) {
+            const int d = i / Eg, e = i % Eg;
+            meta[(size_t)d * 2 * Eg + e] = ws.cap_cnt[i];
+            meta[(size_t)d * 2 * Eg + Eg + e] = ws.spill_cnt[i];
+        }
+        for (int d = tid; d <= G; d += kRowThreads) ep_starts_out[d] = ws.spill_off[d * Eg];
+    }
+    __syncthreads();
+    const int total = min(starts[G], P - E * C);
+    const int lane = tid & 31;
+    for (int q = blockIdx.x * kRowWarps + (tid >> 5); q < total; q += gridDim.x * kRowWarps) {
+        int lo = 0, hi = G - 1;  // last d with starts[d] <= q
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (starts[mid] <= q) lo = mid;
+            else hi = mid - 1;
+        }
+        const int j = q - starts[lo];
+        if (j >= S) {  // cannot happen for a valid routing; never touch past the slot
+            if (lane == 0 && !reverse) atomicOr(ws.status, MOE_DEV_BAD_ROW);  // unpack: flagged by the pack
+            continue;
+        }
+        uint4 *ra = a + (size_t)(E * C + q) * H8, *rb = b + (size_t)(lo * S + j) * H8;
+        if (reverse)
+            copy_row(rb, ra, H8, lane);
+        else
+            copy_row(ra, rb, H8, lane);
+    }
 }
 
 // Receiving rank, one block.  meta[s][0][e], meta[s][1][e]: capacity and
-// overflow rows source s sent for local expert e.  Local row order: expert,
-// then source, then the capacity rows before the overflow rows.
-// cap_seg[s E_g + e] = {row in the received capacity buffer, local row, len};
-// ovf_seg[s E_g + e] = {row in the received overflow buffer, local row, len}.
-// The local rows total at most G (E_g C + S), the local shape's T.
+// overflow rows source s sent for local expert e, clamped to what the buffers
+// hold (capacity rows to C, each source's overflow rows to its slot of S
+// rows; counts from a pack never need it).  Local row order: expert, then
+// source, then the capacity rows before the overflow rows; the local rows
+// total at most G (E_g C + S), the local shape's T.  row_src[r] = the row of
+// the received capacity buffer that local row r comes from, or -1 - its row
+// in the received overflow buffer.
 __global__ void __launch_bounds__(kScanThreads) k_ep_plan_recv(const int32_t *meta, int G, int Eg, int C, int S,
-                                                               int4 *cap_seg, int4 *ovf_seg, int32_t *loc_counts,
-                                                               int32_t *loc_offsets, WsPtrs lws) {
+                                                               int32_t *loc_counts, int32_t *loc_offsets,
+                                                               int32_t *row_src, WsPtrs lws) {
     __shared__ DispatchSmem sm;
+    __shared__ int nc[kMaxExperts], no[kMaxExperts], ovf_pre[kMaxExperts], seg[kMaxExperts];
+    __shared__ int any_bad;
     pdl_trigger();
     pdl_wait();
-    const int tid = threadIdx.x;
-    bool any_bad = false;
+    const int tid = threadIdx.x;  // (source s, local expert e) pairs are indexed s E_g + e
+    if (tid == 0) any_bad = 0;
+    __syncthreads();
+    for (int s = tid; s < G; s += kScanThreads) {
+        int pre = 0;
+        bool bad = false;
+        for (int e = 0; e < Eg; ++e) {
+            const int rc = meta[(size_t)s * 2 * Eg + e], ro = meta[(size_t)s * 2 * Eg + Eg + e];
+            const int c = min(max(rc, 0), C), o = min(max(ro, 0), S - pre);
+            bad |= c != rc || o != ro;
+            nc[s * Eg + e] = c;
+            no[s * Eg + e] = o;
+            ovf_pre[s * Eg + e] = pre;
+            pre += o;
+        }
+        if (bad) any_bad = 1;
+    }
+    __syncthreads();
+    if (tid == 0 && any_bad) atomicOr(lws.status, MOE_DEV_BAD_ROW);
     for (int e = tid; e < Eg; e += kScanThreads) {
         int n = 0;
-        for (int s = 0; s < G; ++s) {
-            int nc, no, ovf;
-            bool bad;
-            ep_recv_counts(meta, s, e, Eg, C, S, nc, no, ovf, bad);
-            n += nc + no;
-            any_bad |= bad;
-        }
+        for (int s = 0; s < G; ++s) n += nc[s * Eg + e] + no[s * Eg + e];
         sm.hist[e] = n;
     }
-    if (any_bad) atomicOr(lws.status, MOE_DEV_BAD_ROW);
     __syncthreads();
     // offsets, local schedule (uncapped layout of the local experts)
     build_schedule_block(sm, Eg, 0, false, loc_counts, loc_offsets, lws);
-    for (int i = tid; i < G * Eg; i += kScanThreads) {
-        const int s = i / Eg, e = i % Eg;
+    for (int e = tid; e < Eg; e += kScanThreads) {
         int row = sm.offs[e];
-        int nc, no, ovf;
-        bool bad;
-        for (int s2 = 0; s2 < s; ++s2) {
-            ep_recv_counts(meta, s2, e, Eg, C, S, nc, no, ovf, bad);
-            row += nc + no;
+        for (int s = 0; s < G; ++s) {
+            seg[s * Eg + e] = row;
+            row += nc[s * Eg + e] + no[s * Eg + e];
         }
-        ep_recv_counts(meta, s, e, Eg, C, S, nc, no, ovf, bad);
-        cap_seg[i] = make_int4(s * Eg * C + e * C, row, nc, 0);
-        ovf_seg[i] = make_int4(s * S + ovf, row + nc, no, 0);
+    }
+    __syncthreads();
+    const int total = sm.offs[Eg];
+    for (int r = tid; r < total; r += kScanThreads) {
+        int lo = 0, hi = Eg - 1;  // expert: last e with offs[e] <= r
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sm.offs[mid] <= r) lo = mid;
+            else hi = mid - 1;
+        }
+        const int e = lo;
+        lo = 0;
+        hi = G - 1;  // source: last s with seg[s][e] <= r (empty segments share a start)
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg[mid * Eg + e] <= r) lo = mid;
+            else hi = mid - 1;
+        }
+        const int i = lo * Eg + e, j = r - seg[i];
+        row_src[r] = j < nc[i] ? lo * Eg * C + e * C + j : -1 - (lo * S + ovf_pre[i] + (j - nc[i]));
     }
 }
 
-// Row copies: segment i moves rows [src, src + len) of `a` to [dst, dst + len)
-// of `b` (reverse: from b's dst rows to a's src rows).  A block per segment
-// (grid-stride), a warp per row, 16-byte vectors.
-__global__ void __launch_bounds__(kSegThreads) k_copy_segments(const uint4 *a, uint4 *b, const uint4 *rb, uint4 *ra,
-                                                               int H8, const int4 *seg, int nseg, int reverse) {
+// Local row r <-> its received row (row_src[r]: capacity buffer row, or
+// -1 - overflow buffer row); forward: loc <- cap / ovf, reverse: cap / ovf
+// <- loc.  total = loc_offsets[E_g], at most Tloc.
+__global__ void __launch_bounds__(kRowThreads) k_ep_local_rows(const int32_t *row_src, const int32_t *loc_total,
+                                                               int Tloc, int H8, uint4 *cap, uint4 *ovf, uint4 *loc,
+                                                               int reverse) {
     pdl_trigger();
     pdl_wait();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = blockIdx.x; i < nseg; i += gridDim.x) {
-        const int4 sg = seg[i];
-        for (int r = warp; r < sg.z; r += kSegThreads / 32) {
-            const uint4 *src = reverse ? rb + (size_t)(sg.y + r) * H8 : a + (size_t)(sg.x + r) * H8;
-            uint4 *dst = reverse ? ra + (size_t)(sg.x + r) * H8 : b + (size_t)(sg.y + r) * H8;
-            for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
-        }
+    const int lane = threadIdx.x & 31;
+    const int total = min(*loc_total, Tloc);
+    for (int r = blockIdx.x * kRowWarps + (threadIdx.x >> 5); r < total; r += gridDim.x * kRowWarps) {
+        const int src = row_src[r];
+        uint4 *rx = src >= 0 ? cap + (size_t)src * H8 : ovf + (size_t)(-1 - src) * H8;
+        uint4 *rl = loc + (size_t)r * H8;
+        if (reverse)
+            copy_row(rl, rx, H8, lane);
+        else
+            copy_row(rx, rl, H8, lane);
     }
+}
+
+int row_grid(int64_t rows, int num_sms) {
+    const int64_t g = (rows + kRowWarps - 1) / kRowWarps;
+    return (int)(g < 1 ? 1 : (g > 2 * num_sms ? 2 * num_sms : g));
 }
 
 }  // namespace
@@ -144,26 +195,30 @@ int64_t ep_overflow_rows(const moe_shape &s, int G) {
     return (int64_t)(s.k < Eg ? s.k : Eg) * (s.T > s.C ? s.T - s.C : 0);
 }
 
-// EP workspace: pack segments [G], capacity and overflow receive segments
-// [E] each, local counts [E/G], local offsets [E/G + 1] (all 16-byte units).
-size_t ep_workspace_bytes(const moe_shape &s, int G) {
-    const int Eg = s.E / G;
-    return 16 * ((size_t)G + 2 * (size_t)s.E) + 4 * align_up((size_t)(2 * Eg + 1), 4);
+static int64_t ep_local_rows(const moe_shape &s, int G) {
+    return (int64_t)G * ((int64_t)(s.E / G) * s.C + ep_overflow_rows(s, G));
 }
 
+// EP workspace (int32 arrays, each padded to 16 bytes): destination starts
+// [G + 1], local counts [E/G], local offsets [E/G + 1], row sources [local T].
 struct EpWs {
-    int4 *pack_seg, *cap_seg, *ovf_seg;
-    int32_t *loc_counts, *loc_offsets;
+    int32_t *starts, *loc_counts, *loc_offsets, *row_src;
 };
 static EpWs ep_ptrs(void *ep_ws, const moe_shape &s, int G) {
-    char *b = (char *)ep_ws;
+    int32_t *b = (int32_t *)ep_ws;
+    const int Eg = s.E / G;
     EpWs p;
-    p.pack_seg = (int4 *)b;
-    p.cap_seg = p.pack_seg + G;
-    p.ovf_seg = p.cap_seg + s.E;
-    p.loc_counts = (int32_t *)(p.ovf_seg + s.E);
-    p.loc_offsets = p.loc_counts + s.E / G;
+    p.starts = b;
+    p.loc_counts = p.starts + align_up((size_t)G + 1, 4);
+    p.loc_offsets = p.loc_counts + align_up((size_t)Eg, 4);
+    p.row_src = p.loc_offsets + align_up((size_t)Eg + 1, 4);
     return p;
+}
+
+size_t ep_workspace_bytes(const moe_shape &s, int G) {
+    const int Eg = s.E / G;
+    return 4 * (align_up((size_t)G + 1, 4) + align_up((size_t)Eg, 4) + align_up((size_t)Eg + 1, 4) +
+                align_up((size_t)ep_local_rows(s, G), 4));
 }
 
 // Source side: counts per destination into send_meta, each destination's
@@ -172,13 +227,10 @@ cudaError_t launch_ep_pack(const moe_shape &s, int G, const void *x_perm, const 
                            int32_t *send_meta, void *ep_ws, int num_sms, cudaStream_t stream) {
     const EpWs p = ep_ptrs(ep_ws, s, G);
     const int S = (int)ep_overflow_rows(s, G);
-    cudaError_t e = launch_pdl(k_ep_plan_send, dim3(1), dim3(kSegThreads), 0, stream, ws_ptrs(ws, L), s.E, G, s.C, S,
-                               send_meta, p.pack_seg);
-    if (e != cudaSuccess) return e;
-    int grid = G < num_sms ? G : num_sms;
-    return launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)x_perm,
-                      (uint4 *)send_ovf, (const uint4 *)nullptr, (uint4 *)nullptr, s.H / 8, (const int4 *)p.pack_seg, G,
-                      0);
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, true);
+    return launch_pdl(k_ep_spill_rows, dim3(row_grid(P - (int64_t)s.E * s.C, num_sms)), dim3(kRowThreads), 0, stream,
+                      ws_ptrs(ws, L), (const int32_t *)nullptr, s.E, G, s.C, S, (int)P, s.H / 8, (uint4 *)x_perm,
+                      (uint4 *)send_ovf, 0, send_meta, p.starts);
 }
 
 // Receiving side: the local layout, its GEMM schedule in the local workspace,
@@ -188,16 +240,13 @@ cudaError_t launch_ep_local_dispatch(const moe_shape &s, int G, const int32_t *r
                                      void *ep_ws, int num_sms, cudaStream_t stream) {
     const EpWs p = ep_ptrs(ep_ws, s, G);
     const int S = (int)ep_overflow_rows(s, G), Eg = s.E / G;
+    const int64_t Tloc = ep_local_rows(s, G);
     cudaError_t e = launch_pdl(k_ep_plan_recv, dim3(1), dim3(kScanThreads), 0, stream, recv_meta, G, Eg, s.C, S,
-                               p.cap_seg, p.ovf_seg, p.loc_counts, p.loc_offsets, ws_ptrs(ws_loc, Lloc));
+                               p.loc_counts, p.loc_offsets, p.row_src, ws_ptrs(ws_loc, Lloc));
     if (e != cudaSuccess) return e;
-    const int grid = s.E < 4 * num_sms ? s.E : 4 * num_sms;
-    e = launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)recv_cap, (uint4 *)x_loc,
-                   (const uint4 *)nullptr, (uint4 *)nullptr, s.H / 8, (const int4 *)p.cap_seg, s.E, 0);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)recv_ovf,
-                      (uint4 *)x_loc, (const uint4 *)nullptr, (uint4 *)nullptr, s.H / 8, (const int4 *)p.ovf_seg, s.E,
-                      0);
+    return launch_pdl(k_ep_local_rows, dim3(row_grid(Tloc, num_sms)), dim3(kRowThreads), 0, stream,
+                      (const int32_t *)p.row_src, (const int32_t *)(p.loc_offsets + Eg), (int)Tloc, s.H / 8,
+                      (uint4 *)recv_cap, (uint4 *)recv_ovf, (uint4 *)x_loc, 0);
 }
 
 // Receiving side, after the local experts: y_loc rows back to where their
@@ -206,25 +255,23 @@ cudaError_t launch_ep_local_dispatch(const moe_shape &s, int G, const int32_t *r
 cudaError_t launch_ep_local_return(const moe_shape &s, int G, const void *y_loc, void *back_cap, void *back_ovf,
                                    void *ep_ws, int num_sms, cudaStream_t stream) {
     const EpWs p = ep_ptrs(ep_ws, s, G);
-    const int grid = s.E < 4 * num_sms ? s.E : 4 * num_sms;
-    cudaError_t e = launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)nullptr,
-                               (uint4 *)nullptr, (const uint4 *)y_loc, (uint4 *)back_cap, s.H / 8,
-                               (const int4 *)p.cap_seg, s.E, 1);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)nullptr,
-                      (uint4 *)nullptr, (const uint4 *)y_loc, (uint4 *)back_ovf, s.H / 8, (const int4 *)p.ovf_seg, s.E,
-                      1);
+    const int64_t Tloc = ep_local_rows(s, G);
+    return launch_pdl(k_ep_local_rows, dim3(row_grid(Tloc, num_sms)), dim3(kRowThreads), 0, stream,
+                      (const int32_t *)p.row_src, (const int32_t *)(p.loc_offsets + s.E / G), (int)Tloc, s.H / 8,
+                      (uint4 *)back_cap, (uint4 *)back_ovf, (uint4 *)y_loc, 1);
 }
 
 // Source side, after the return passes: the overflow rows' results from
-// their slots back into y's overflow rows (the pack copies reversed).
+// their slots back into y's overflow region (the pack copies reversed).
 cudaError_t launch_ep_unpack(const moe_shape &s, int G, const void *recv_back_ovf, void *y, void *ep_ws, int num_sms,
                              cudaStream_t stream) {
     const EpWs p = ep_ptrs(ep_ws, s, G);
-    const int grid = G < num_sms ? G : num_sms;
-    return launch_pdl(k_copy_segments, dim3(grid), dim3(kSegThreads), 0, stream, (const uint4 *)nullptr,
-                      (uint4 *)nullptr, (const uint4 *)recv_back_ovf, (uint4 *)y, s.H / 8, (const int4 *)p.pack_seg, G,
-                      1);
+    const int S = (int)ep_overflow_rows(s, G);
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, true);
+    const WsPtrs none = {};  // no status word: the pack already flagged a bad row
+    return launch_pdl(k_ep_spill_rows, dim3(row_grid(P - (int64_t)s.E * s.C, num_sms)), dim3(kRowThreads), 0, stream,
+                      none, (const int32_t *)p.starts, s.E, G, s.C, S, (int)P, s.H / 8, (uint4 *)y,
+                      (uint4 *)recv_back_ovf, 1, (int32_t *)nullptr, (int32_t *)nullptr);
 }
 
 }  // namespace moe
