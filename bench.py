@@ -585,11 +585,14 @@ class Bench:
         ranks = [CapAndSpillEP(shape, G, dev) for _ in range(G)]
         Eg = cfg.E // G
         sl = [slice(r * Eg, (r + 1) * Eg) for r in range(G)]
-        phases = ("route_and_pack", "receive", "experts", "send_back", "finish")
+        phases = ("route_and_pack", "receive", "experts_swiglu", "experts_down", "send_back", "finish")
         calls = {
             "route_and_pack": lambda r: ranks[r].route_and_pack(xs[r], wr, bias, stream),
             "receive": lambda r: ranks[r].receive(stream),
-            "experts": lambda r: ranks[r].experts(wg[sl[r]], wu[sl[r]], wd[sl[r]], stream),
+            "experts_swiglu": lambda r: moe.moe_grouped_swiglu(ranks[r].local, ranks[r].x_loc, wg[sl[r]], wu[sl[r]],
+                                                               ranks[r].h_loc, ranks[r].ws_loc, stream),
+            "experts_down": lambda r: moe.moe_grouped_down(ranks[r].local, ranks[r].h_loc, wd[sl[r]], ranks[r].y_loc,
+                                                           ranks[r].ws_loc, stream),
             "send_back": lambda r: ranks[r].send_back(stream),
             "finish": lambda r: ranks[r].finish(stream),
         }
@@ -763,17 +766,23 @@ def summarize_ep(cfg, e, peaks):
     p1, p2, meta = cfg.E * cfg.C * row, G * S * row, G * 2 * Eg * 4
     real = float(sum(e["overflow_rows"])) / G * row
     w_bytes = 3 * Eg * cfg.H * cfg.F * 2
+    per_rank["experts"] = per_rank["experts_swiglu"] + per_rank["experts_down"]
     t_exp = per_rank["experts"] * 1e-6
     return {
         "workload": workload_name(cfg), "G": G,
         "ranks": "G ranks emulated on one GPU (each rank's phases on its own buffers); the all-to-alls done as "
                  "device copies and not timed",
-        "per_rank_us": per_rank, "per_rank_kernels_us": sum(per_rank.values()),
+        "per_rank_us": per_rank,
+        "per_rank_kernels_us": sum(v for k, v in per_rank.items() if k != "experts"),
         "single_gpu_layer_us": e["single_gpu_layer_us"],
         "experts_roofline": {"bound": "hbm", "bytes": w_bytes, "achieved": w_bytes / t_exp / 1e9,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": w_bytes / t_exp / 1e9 / peaks["hbm_gbs"],
-                             "note": "the rank's expert weights over the local SwiGLU + down time"},
+                             "note": "the rank's expert weights over the local SwiGLU + down time",
+                             "swiglu_frac": (2 * Eg * cfg.H * cfg.F * 2) / (per_rank["experts_swiglu"] * 1e-6) / 1e9
+                             / peaks["hbm_gbs"],
+                             "down_frac": (Eg * cfg.H * cfg.F * 2) / (per_rank["experts_down"] * 1e-6) / 1e9
+                             / peaks["hbm_gbs"]},
         "exchange_per_rank": {"pass1_bytes": p1, "pass2_bytes": p2, "meta_bytes": meta,
                               "real_overflow_bytes": real, "pass2_padding_frac": 1.0 - real / p2 if p2 else 0.0,
                               "nvlink_model_us": 2 * (p1 + p2 + meta) / (NVLINK_PEER_GBS * 1e9) * 1e6,

@@ -102,17 +102,19 @@ __global__ void __launch_bounds__(kScanThreads) k_ep_plan_recv(const int32_t *me
                                                                int32_t *row_src, WsPtrs lws) {
     __shared__ DispatchSmem sm;
     __shared__ int nc[kMaxExperts], no[kMaxExperts], ovf_pre[kMaxExperts], seg[kMaxExperts];
+    __shared__ int m[2 * kMaxExperts];
     __shared__ int any_bad;
     pdl_trigger();
     pdl_wait();
     const int tid = threadIdx.x;  // (source s, local expert e) pairs are indexed s E_g + e
     if (tid == 0) any_bad = 0;
+    for (int i = tid; i < 2 * G * Eg; i += kScanThreads) m[i] = meta[i];  // all loads in one round trip
     __syncthreads();
     for (int s = tid; s < G; s += kScanThreads) {
         int pre = 0;
         bool bad = false;
         for (int e = 0; e < Eg; ++e) {
-            const int rc = meta[(size_t)s * 2 * Eg + e], ro = meta[(size_t)s * 2 * Eg + Eg + e];
+            const int rc = m[s * 2 * Eg + e], ro = m[s * 2 * Eg + Eg + e];
             const int c = min(max(rc, 0), C), o = min(max(ro, 0), S - pre);
             bad |= c != rc || o != ro;
             nc[s * Eg + e] = c;
