@@ -37,6 +37,9 @@ namespace moe {
 
 namespace {
 
+// Dynamic shared memory of a router CTA, at most.
+constexpr int kRouteSmemMax = 200 * 1024;
+
 struct RouteArgs {
     const __nv_bfloat16 *x;
     const float *w_router;
@@ -287,6 +290,32 @@ __global__ void __launch_bounds__(256) k_topk(RouteArgs a) {
         atomicOr(a.status, MOE_DEV_NAN_LOGIT);
 }
 
+// A lane's EJ consecutive experts of one weight row: one 8- or 16-byte load
+// when they all exist (the row start and es * EJ are multiples of EJ floats),
+// else clamped scalar loads (ecol[j] = min(es * EJ + j, E - 1); the values
+// past E are never used).
+template <int EJ>
+__device__ __forceinline__ void load_weights(const float *row, int E, int es, const int *ecol, float *w) {
+    if constexpr (EJ == 2 || EJ == 4) {
+        if (es * EJ + EJ <= E && (E % EJ) == 0) {
+            if constexpr (EJ == 2) {
+                const float2 v = *reinterpret_cast<const float2 *>(row + es * EJ);
+                w[0] = v.x;
+                w[1] = v.y;
+            } else {
+                const float4 v = *reinterpret_cast<const float4 *>(row + es * EJ);
+                w[0] = v.x;
+                w[1] = v.y;
+                w[2] = v.z;
+                w[3] = v.w;
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) w[j] = row[ecol[j]];
+}
+
 template <int TB, int EJ>
 __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -348,6 +377,11 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             if (s < nchunks) issue(s, s);
             cp_async_commit();
         }
+        // x of the chunk in fp32, token pairs interleaved: x2[i][p] =
+        // (x[2i][2p], x[2i+1][2p], x[2i][2p+1], x[2i+1][2p+1]), the two packed
+        // operands of hidden units 2p and 2p+1 in one 16-byte load
+        float4 *x2 = reinterpret_cast<float4 *>(smem + (size_t)S * stage_bytes);
+        const int HP = HC / 2;
         for (int c = 0; c < nchunks; ++c) {
             if (c + S - 1 < nchunks) issue(c + S - 1, (c + S - 1) % S);
             cp_async_commit();
@@ -356,24 +390,27 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             const uint8_t *sx = smem + (size_t)(c % S) * stage_bytes;
             const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(sx);
             const float *wsm = reinterpret_cast<const float *>(sx + xbytes);
+            for (int idx = tid; idx < (TB / 2) * HP; idx += 256) {
+                const int i = idx / HP, p = idx - i * HP;
+                const float2 xa =
+                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i) * HC + 2 * p));
+                const float2 xb = __bfloat1622float2(
+                    *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i + 1) * HC + 2 * p));
+                x2[idx] = make_float4(xa.x, xb.x, xa.y, xb.y);
+            }
+            __syncthreads();
             // Pairs of hidden units 2p, 2p+1 of this warp's range; this lane
             // takes p = p0 + hs, p0 + hs + HS, ...
             const int p0 = warp * PPW;
             for (int p = p0 + hs; p < p0 + PPW; p += HS) {
                 const float *w0 = wsm + (size_t)(2 * p) * E;
                 float wa[EJ], wb[EJ];
-#pragma unroll
-                for (int j = 0; j < EJ; ++j) {
-                    wa[j] = w0[ecol[j]];
-                    wb[j] = w0[E + ecol[j]];
-                }
+                load_weights<EJ>(w0, E, es, ecol, wa);
+                load_weights<EJ>(w0 + E, E, es, ecol, wb);
 #pragma unroll
                 for (int i = 0; i < TB / 2; ++i) {
-                    const float2 xa = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i) * HC + 2 * p));
-                    const float2 xb = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)(2 * i + 1) * HC + 2 * p));
-                    const float2 x0 = make_float2(xa.x, xb.x), x1 = make_float2(xa.y, xb.y);
+                    const float4 xv = x2[i * HP + p];
+                    const float2 x0 = make_float2(xv.x, xv.y), x1 = make_float2(xv.z, xv.w);
 #pragma unroll
                     for (int j = 0; j < EJ; ++j) {
                         acc2[i][j] = __ffma2_rn(x0, make_float2(wa[j], wa[j]), acc2[i][j]);
@@ -381,7 +418,7 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
                     }
                 }
             }
-            __syncthreads();  // stage c % S may be refilled from here on
+            __syncthreads();  // stage c % S and the fp32 tile may be refilled from here on
         }
         float acc[TB][EJ];
 #pragma unroll
@@ -483,7 +520,7 @@ template <int TB, int EJ>
 cudaError_t launch_one(const RouteArgs &a, int smem_bytes, int tiles, cudaStream_t stream) {
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_route<TB, EJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(k_route<TB, EJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouteSmemMax);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
@@ -611,12 +648,18 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
         a.part_off = 0;
         smem = lg_bytes;
     } else {
-        // the pipeline stages, later the per-warp partial sums [8][TB][E] and
-        // then rank 0's logits tile share the front of shared memory
-        int front = stages * stage_bytes;
-        if (front < lg_bytes) front = lg_bytes;
-        if (front < 8 * TB * s.E * 4) front = 8 * TB * s.E * 4;
-        a.part_off = (int)align_up((size_t)front, 16);
+        // the pipeline stages and the chunk's fp32 x tile, later the per-warp
+        // partial sums [8][TB][E] and then rank 0's logits tile share the
+        // front of shared memory; fewer stages if it would not fit
+        const int x2_bytes = TB * hc * 4;
+        auto front_of = [&](int st) {
+            int f = st * stage_bytes + x2_bytes;
+            if (f < lg_bytes) f = lg_bytes;
+            if (f < 8 * TB * s.E * 4) f = 8 * TB * s.E * 4;
+            return (int)align_up((size_t)f, 16);
+        };
+        while (a.stages > 2 && front_of(a.stages) + TB * s.E * 4 > kRouteSmemMax) --a.stages;
+        a.part_off = front_of(a.stages);
         smem = a.part_off + TB * s.E * 4;
     }
     if (fused) {
