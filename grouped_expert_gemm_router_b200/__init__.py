@@ -40,6 +40,8 @@ ABI_FUNCTIONS = (
     "moe_quantize_rows_fp8", "moe_grouped_swiglu_fp8", "moe_grouped_down_fp8", "moe_forward_fp8",
     "moe_grouped_down_combine", "moe_grouped_down_fp8_combine", "moe_ep_overflow_rows", "moe_ep_workspace_bytes",
     "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
+    "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
+    "moe_ep_direct_dispatch", "moe_ep_direct_return",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -158,6 +160,18 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_local_return.restype = st
     lib.moe_ep_unpack.argtypes = [sp, i32] + [vp] * 4
     lib.moe_ep_unpack.restype = st
+    lib.moe_ep_direct_local_rows.argtypes = [sp, i32]
+    lib.moe_ep_direct_local_rows.restype = ctypes.c_int64
+    lib.moe_ep_direct_workspace_bytes.argtypes = [sp, i32]
+    lib.moe_ep_direct_workspace_bytes.restype = ctypes.c_size_t
+    lib.moe_ep_direct_local_shape.argtypes = [sp, i32, sp]
+    lib.moe_ep_direct_local_shape.restype = st
+    lib.moe_ep_direct_plan.argtypes = [sp, i32, i32] + [vp] * 4
+    lib.moe_ep_direct_plan.restype = st
+    lib.moe_ep_direct_dispatch.argtypes = [sp, i32] + [vp] * 8
+    lib.moe_ep_direct_dispatch.restype = st
+    lib.moe_ep_direct_return.argtypes = [sp, i32] + [vp] * 4
+    lib.moe_ep_direct_return.restype = st
     _lib = lib
     return lib
 
@@ -439,3 +453,37 @@ def moe_ep_local_return(shape, G, y_loc, back_cap, back_ovf, ep_ws, stream=None)
 def moe_ep_unpack(shape, G, recv_back_ovf, y, ep_ws, stream=None):
     _check(load_library().moe_ep_unpack(ctypes.byref(shape), int(G), _ptr(recv_back_ovf), _ptr(y), _ptr(ep_ws),
                                         _stream(stream)), "moe_ep_unpack")
+
+
+def moe_ep_direct_local_rows(shape, G) -> int:
+    return int(load_library().moe_ep_direct_local_rows(ctypes.byref(shape), int(G)))
+
+
+def moe_ep_direct_workspace_bytes(shape, G) -> int:
+    return int(load_library().moe_ep_direct_workspace_bytes(ctypes.byref(shape), int(G)))
+
+
+def moe_ep_direct_local_shape(shape, G) -> MoeShape:
+    out = MoeShape()
+    _check(load_library().moe_ep_direct_local_shape(ctypes.byref(shape), int(G), ctypes.byref(out)),
+           "moe_ep_direct_local_shape")
+    return out
+
+
+def moe_ep_direct_plan(shape, G, rank, cnt_all, ws_loc, ep_ws, stream=None):
+    _check(load_library().moe_ep_direct_plan(ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(ws_loc),
+                                             _ptr(ep_ws), _stream(stream)), "moe_ep_direct_plan")
+
+
+def moe_ep_direct_dispatch(shape, G, x, topk_idx, dest_row, expert_offsets, peer_x_loc, ws, ep_ws, stream=None):
+    """peer_x_loc: a device tensor of G int64 addresses (rank d's x_loc)."""
+    _check(load_library().moe_ep_direct_dispatch(ctypes.byref(shape), int(G), _ptr(x), _ptr(topk_idx),
+                                                 _ptr(dest_row), _ptr(expert_offsets), _ptr(peer_x_loc), _ptr(ws),
+                                                 _ptr(ep_ws), _stream(stream)), "moe_ep_direct_dispatch")
+
+
+def moe_ep_direct_return(shape, G, y_loc, peer_y, ep_ws, stream=None):
+    """peer_y: a device tensor of G int64 addresses (rank s's y)."""
+    _check(load_library().moe_ep_direct_return(ctypes.byref(shape), int(G), _ptr(y_loc), _ptr(peer_y), _ptr(ep_ws),
+                                                _stream(stream)), "moe_ep_direct_return")
+

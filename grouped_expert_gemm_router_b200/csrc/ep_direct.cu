@@ -1,0 +1,276 @@
+// Expert-parallel dispatch and return by device-initiated peer stores: the
+// all-to-all of the layer written as two kernels that store rows straight
+// into the other ranks' buffers over NVLink (peer pointers from symmetric
+// memory or CUDA IPC), instead of collective passes over fixed-size slots.
+//
+// G ranks, E experts, rank d owns experts [d E_g, (d + 1) E_g), E_g = E / G.
+// Each rank routes its T tokens with the uncapped dispatch (expert-contiguous
+// rows, pair i of expert e at row offsets[e] + its rank among e's pairs), and
+// the ranks all-gather their per-expert counts cnt[G][E].  From the same
+// counts every rank derives the same layouts:
+//   destination d's local rows: per local expert, each source's pairs in
+//     source order, each source's in its own dispatch order (so an expert's
+//     rows are its tokens in (source, token) order, as on one GPU);
+//   source s's row for pair i of expert e in d's local rows:
+//     base_d[e] + sum over s' < s of cnt[s'][e] + (dest_row[i] - offsets_s[e]);
+//   the way back: local row -> (source, its uncapped row offsets_s[e] + j).
+// Only the routed rows cross the links (no padding), the receiver needs no
+// copy into its layout, and the return stores land in each source's y rows,
+// where moe_combine reads them.  The counts are clamped the same way on every
+// rank (each source's rows to one destination to at most T min(k, E_g), each
+// (source, expert) to at most T), so corrupt counts never move a store outside
+// a buffer; such counts set MOE_DEV_BAD_ROW.
+//
+// k_ep_direct_plan    one block: clamped counts, this rank's send bases, its
+//                     local layout, GEMM schedule and return segments.
+// k_ep_direct_put     source: a warp per routed pair, x[t] -> the
+//                     destination's x_loc row.
+// k_ep_direct_return  destination: a warp per local row, y_loc -> the
+//                     source's y row.
+// Each put kernel ends with a system-scope fence, so a stream-ordered
+// collective after it (a barrier) orders its peer stores before any later
+// work on every rank.
+#include <cuda_bf16.h>
+
+#include "dispatch_block.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kDirThreads = 256;
+constexpr int kDirWarps = kDirThreads / 32;
+
+__device__ __forceinline__ void copy_row16(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8, int lane) {
+    for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
+}
+
+// Smallest per-rank figures: at most kDirMaxCounts (source, expert) counts.
+constexpr int kDirMaxCounts = 4096;
+
+struct DirPlanArgs {
+    const int32_t *cnt_all;  // [G][E] as gathered
+    int G, E, T, k, rank;
+    int32_t *send_base, *send_cnt;               // [E]
+    int32_t *seg_start, *seg_cnt, *seg_ysrc;     // [G][E_g]
+    int32_t *loc_counts, *loc_offsets;           // [E_g], [E_g + 1]
+    WsPtrs lws;
+};
+
+__global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) {
+    __shared__ DispatchSmem sm;
+    __shared__ int c[kDirMaxCounts];
+    __shared__ int base[kMaxExperts];  // destination layout offsets of each expert (over all sources)
+    __shared__ int any_bad;
+    pdl_trigger();
+    pdl_wait();
+    const int tid = threadIdx.x, G = a.G, E = a.E, Eg = E / G, r = a.rank;
+    const int per_dest = a.T * (a.k < Eg ? a.k : Eg);
+    if (tid == 0) any_bad = 0;
+    for (int i = tid; i < G * E; i += kScanThreads) c[i] = a.cnt_all[i];
+    __syncthreads();
+    // Clamp: (source s, destination d): its experts' counts to [0, T] and
+    // their running sum to the per-destination bound, in expert order.
+    for (int sd = tid; sd < G * G; sd += kScanThreads) {
+        const int s = sd / G, d = sd % G;
+        int run = 0;
+        bool bad = false;
+        for (int el = 0; el < Eg; ++el) {
+            const int i = s * E + d * Eg + el, v = c[i];
+            const int w = min(min(max(v, 0), a.T), per_dest - run);
+            bad |= w != v;
+            c[i] = w;
+            run += w;
+        }
+        if (bad) any_bad = 1;
+    }
+    __syncthreads();
+    if (tid == 0 && any_bad) atomicOr(a.lws.status, MOE_DEV_BAD_ROW);
+    // Every destination's offsets of its experts (over all sources).
+    for (int e = tid; e < E; e += kScanThreads) {
+        const int d = e / Eg, el = e % Eg;
+        int off = 0;
+        for (int e2 = d * Eg; e2 < d * Eg + el; ++e2)
+            for (int s = 0; s < G; ++s) off += c[s * E + e2];
+        base[e] = off;
+    }
+    __syncthreads();
+    // Source role: where this rank's pairs of expert e start in the
+    // destination's local rows.
+    for (int e = tid; e < E; e += kScanThreads) {
+        int b = base[e];
+        for (int s = 0; s < r; ++s) b += c[s * E + e];
+        a.send_base[e] = b;
+        a.send_cnt[e] = c[r * E + e];
+    }
+    // Destination role: the local layout and its GEMM schedule.
+    for (int el = tid; el < Eg; el += kScanThreads) {
+        int n = 0;
+        for (int s = 0; s < G; ++s) n += c[s * E + r * Eg + el];
+        sm.hist[el] = n;
+    }
+    __syncthreads();
+    build_schedule_block(sm, Eg, 0, false, a.loc_counts, a.loc_offsets, a.lws);
+    // Return segments: (source s, local expert el) -> first local row, rows,
+    // first row in the source's y (its uncapped offset of the expert).
+    for (int i = tid; i < G * Eg; i += kScanThreads) {
+        const int s = i / Eg, el = i % Eg, e = r * Eg + el;
+        int start = sm.offs[el];
+        for (int s2 = 0; s2 < s; ++s2) start += c[s2 * E + e];
+        int ysrc = 0;
+        for (int e2 = 0; e2 < e; ++e2) ysrc += c[s * E + e2];
+        a.seg_start[i] = start;
+        a.seg_cnt[i] = c[s * E + e];
+        a.seg_ysrc[i] = ysrc;
+    }
+}
+
+// Source side: pair i = t k + j of expert e goes to row send_base[e] +
+// (dest_row[i] - offsets[e]) of rank e / E_g's x_loc.
+__global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(const uint4 *x, const int32_t *topk_idx,
+                                                                const int32_t *dest_row, const int32_t *offsets,
+                                                                const int32_t *send_base, const int32_t *send_cnt,
+                                                                const unsigned long long *peer_x_loc, int R, int k,
+                                                                int E, int Eg, int Tloc, int H8, uint32_t *status) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    for (int i = blockIdx.x * kDirWarps + (threadIdx.x >> 5); i < R; i += gridDim.x * kDirWarps) {
+        const int e = topk_idx[i];
+        if ((unsigned)e >= (unsigned)E) continue;  // reported by the router
+        const int ri = dest_row[i] - offsets[e];
+        const int pos = send_base[e] + ri;
+        if (ri < 0 || ri >= send_cnt[e] || (unsigned)pos >= (unsigned)Tloc) {
+            bad = true;
+            continue;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(peer_x_loc[e / Eg]) + (size_t)pos * H8;
+        copy_row16(x + (size_t)(i / k) * H8, dst, H8, lane);
+    }
+    if (bad && lane == 0) atomicOr(status, MOE_DEV_BAD_ROW);
+    __threadfence_system();
+}
+
+// Destination side: local row r of segment (s, el) goes to row seg_ysrc +
+// (r - seg_start) of rank s's y.
+__global__ void __launch_bounds__(kDirThreads) k_ep_direct_return(const uint4 *y_loc, const int32_t *seg_start,
+                                                                   const int32_t *seg_cnt, const int32_t *seg_ysrc,
+                                                                   const int32_t *loc_offsets,
+                                                                   const unsigned long long *peer_y, int G, int Eg,
+                                                                   int Tloc, int P, int H8) {
+    __shared__ int offs[kMaxExperts + 1];
+    pdl_trigger();
+    pdl_wait();
+    for (int i = threadIdx.x; i <= Eg; i += kDirThreads) offs[i] = loc_offsets[i];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int total = min(offs[Eg], Tloc);
+    for (int r = blockIdx.x * kDirWarps + (threadIdx.x >> 5); r < total; r += gridDim.x * kDirWarps) {
+        int lo = 0, hi = Eg - 1;  // local expert: last el with offs[el] <= r
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offs[mid] <= r) lo = mid;
+            else hi = mid - 1;
+        }
+        const int el = lo;
+        lo = 0;
+        hi = G - 1;  // source: last s with seg_start[s][el] <= r (empty segments share a start)
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg_start[mid * Eg + el] <= r) lo = mid;
+            else hi = mid - 1;
+        }
+        const int i = lo * Eg + el, j = r - seg_start[i];
+        const int yrow = seg_ysrc[i] + j;
+        if (j >= seg_cnt[i] || (unsigned)yrow >= (unsigned)P) continue;  // cannot happen: the plan's layout
+        uint4 *dst = reinterpret_cast<uint4 *>(peer_y[lo]) + (size_t)yrow * H8;
+        copy_row16(y_loc + (size_t)r * H8, dst, H8, lane);
+    }
+    __threadfence_system();
+}
+
+int dir_grid(int64_t rows, int num_sms) {
+    const int64_t g = (rows + kDirWarps - 1) / kDirWarps;
+    return (int)(g < 1 ? 1 : (g > 2 * num_sms ? 2 * num_sms : g));
+}
+
+}  // namespace
+
+// Local rows of one rank at most: every source sends it at most T min(k, E/G)
+// pairs.
+int64_t ep_direct_local_rows(const moe_shape &s, int G) {
+    const int Eg = s.E / G;
+    return (int64_t)G * s.T * (s.k < Eg ? s.k : Eg);
+}
+
+bool ep_direct_counts_fit(const moe_shape &s, int G) { return (int64_t)G * s.E <= kDirMaxCounts; }
+
+// Direct EP workspace (int32 arrays, each padded to 16 bytes): send bases and
+// counts [E] each, return segments (start, rows, source row) [G E_g] each,
+// local counts [E_g], local offsets [E_g + 1].
+struct DirWs {
+    int32_t *send_base, *send_cnt, *seg_start, *seg_cnt, *seg_ysrc, *loc_counts, *loc_offsets;
+};
+static DirWs dir_ptrs(void *ep_ws, const moe_shape &s, int G) {
+    int32_t *b = (int32_t *)ep_ws;
+    const size_t E4 = align_up((size_t)s.E, 4), Eg = (size_t)(s.E / G);
+    DirWs p;
+    p.send_base = b;
+    p.send_cnt = p.send_base + E4;
+    p.seg_start = p.send_cnt + E4;
+    p.seg_cnt = p.seg_start + E4;
+    p.seg_ysrc = p.seg_cnt + E4;
+    p.loc_counts = p.seg_ysrc + E4;
+    p.loc_offsets = p.loc_counts + align_up(Eg, 4);
+    return p;
+}
+
+size_t ep_direct_workspace_bytes(const moe_shape &s, int G) {
+    const size_t E4 = align_up((size_t)s.E, 4), Eg = (size_t)(s.E / G);
+    return 4 * (5 * E4 + align_up(Eg, 4) + align_up(Eg + 1, 4));
+}
+
+cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const WsLayout &Lloc,
+                                  void *ws_loc, void *ep_ws, cudaStream_t stream) {
+    const DirWs p = dir_ptrs(ep_ws, s, G);
+    DirPlanArgs a;
+    a.cnt_all = cnt_all;
+    a.G = G;
+    a.E = s.E;
+    a.T = s.T;
+    a.k = s.k;
+    a.rank = rank;
+    a.send_base = p.send_base;
+    a.send_cnt = p.send_cnt;
+    a.seg_start = p.seg_start;
+    a.seg_cnt = p.seg_cnt;
+    a.seg_ysrc = p.seg_ysrc;
+    a.loc_counts = p.loc_counts;
+    a.loc_offsets = p.loc_offsets;
+    a.lws = ws_ptrs(ws_loc, Lloc);
+    return launch_pdl(k_ep_direct_plan, dim3(1), dim3(kScanThreads), 0, stream, a);
+}
+
+cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
+                                 const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
+                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream) {
+    const DirWs p = dir_ptrs(ep_ws, s, G);
+    const int64_t R = (int64_t)s.T * s.k;
+    return launch_pdl(k_ep_direct_put, dim3(dir_grid(R, num_sms)), dim3(kDirThreads), 0, stream, (const uint4 *)x,
+                      topk_idx, dest_row, offsets, (const int32_t *)p.send_base, (const int32_t *)p.send_cnt,
+                      (const unsigned long long *)peer_x_loc, (int)R, s.k, s.E, s.E / G,
+                      (int)ep_direct_local_rows(s, G), s.H / 8, status);
+}
+
+cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,
+                                    int num_sms, cudaStream_t stream) {
+    const DirWs p = dir_ptrs(ep_ws, s, G);
+    const int64_t Tloc = ep_direct_local_rows(s, G);
+    return launch_pdl(k_ep_direct_return, dim3(dir_grid(Tloc, num_sms)), dim3(kDirThreads), 0, stream,
+                      (const uint4 *)y_loc, (const int32_t *)p.seg_start, (const int32_t *)p.seg_cnt,
+                      (const int32_t *)p.seg_ysrc, (const int32_t *)p.loc_offsets,
+                      (const unsigned long long *)peer_y, G, s.E / G, (int)Tloc, s.T * s.k, s.H / 8);
+}
+
+}  // namespace moe

@@ -46,6 +46,16 @@ cudaError_t launch_ep_local_return(const moe_shape &s, int G, const void *y_loc,
                                    void *ep_ws, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_unpack(const moe_shape &s, int G, const void *recv_back_ovf, void *y, void *ep_ws, int num_sms,
                              cudaStream_t stream);
+int64_t ep_direct_local_rows(const moe_shape &s, int G);
+bool ep_direct_counts_fit(const moe_shape &s, int G);
+size_t ep_direct_workspace_bytes(const moe_shape &s, int G);
+cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const WsLayout &Lloc,
+                                  void *ws_loc, void *ep_ws, cudaStream_t stream);
+cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
+                                 const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
+                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,
+                                    int num_sms, cudaStream_t stream);
 }  // namespace moe
 
 using namespace moe;
@@ -596,3 +606,87 @@ const char *moe_last_error_string(void) { return g_last_error; }
 int32_t moe_version(void) { return 100; }
 
 }  // extern "C"
+
+// ------------------------------------------- expert parallel, peer stores --
+namespace {
+moe_status check_ep_direct(const moe_shape *s, int32_t G) {
+    moe_status st = check_shape(s);
+    if (st != MOE_OK) return st;
+    if ((s->flags & MOE_FLAG_CAPACITY) || G < 1 || s->E % G != 0 || !ep_direct_counts_fit(*s, G))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int64_t Tloc = ep_direct_local_rows(*s, G);
+    if (Tloc < 1 || Tloc >= (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+moe_shape ep_direct_local(const moe_shape *s, int32_t G) {
+    moe_shape l;
+    l.T = (int32_t)ep_direct_local_rows(*s, G);
+    l.H = s->H;
+    l.F = s->F;
+    l.E = s->E / G;
+    l.k = 1;
+    l.C = 0;
+    l.flags = 0;
+    return l;
+}
+}  // namespace
+
+int64_t moe_ep_direct_local_rows(const moe_shape *s, int32_t G) {
+    if (check_ep_direct(s, G) != MOE_OK) return -1;
+    return ep_direct_local_rows(*s, G);
+}
+
+size_t moe_ep_direct_workspace_bytes(const moe_shape *s, int32_t G) {
+    if (check_ep_direct(s, G) != MOE_OK) return 0;
+    return ep_direct_workspace_bytes(*s, G);
+}
+
+moe_status moe_ep_direct_local_shape(const moe_shape *s, int32_t G, moe_shape *local) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!local) return MOE_ERR_INVALID_ARG;
+    *local = ep_direct_local(s, G);
+    return check_shape(local);
+}
+
+moe_status moe_ep_direct_plan(const moe_shape *s, int32_t G, int32_t rank, const int32_t *cnt_all, void *ws_loc,
+                              void *ep_ws, void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (rank < 0 || rank >= G) return MOE_ERR_INVALID_ARG;
+    if (!aligned(cnt_all, 4) || !aligned(ep_ws, 16)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws_loc)) != MOE_OK) return st;
+    const moe_shape l = ep_direct_local(s, G);
+    const WsLayout Lloc = layout_of(&l);
+    cudaError_t e = launch_ep_direct_plan(*s, G, rank, cnt_all, Lloc, ws_loc, ep_ws, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_plan");
+}
+
+moe_status moe_ep_direct_dispatch(const moe_shape *s, int32_t G, const void *x, const int32_t *topk_idx,
+                                  const int32_t *dest_row, const int32_t *expert_offsets, const void *peer_x_loc,
+                                  void *ws, void *ep_ws, void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(dest_row, 4) || !aligned(expert_offsets, 4) ||
+        !aligned(peer_x_loc, 8) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    uint32_t *status = (uint32_t *)((char *)ws + L.status);
+    cudaError_t e = launch_ep_direct_put(*s, G, x, topk_idx, dest_row, expert_offsets, peer_x_loc, ep_ws, status, sms,
+                                         (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_dispatch");
+}
+
+moe_status moe_ep_direct_return(const moe_shape *s, int32_t G, const void *y_loc, const void *peer_y, void *ep_ws,
+                                void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(y_loc, 16) || !aligned(peer_y, 8) || !aligned(ep_ws, 16)) return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e = launch_ep_direct_return(*s, G, y_loc, peer_y, ep_ws, sms, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_return");
+}

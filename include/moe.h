@@ -478,6 +478,71 @@ MOE_API moe_status moe_ep_local_return(const moe_shape *shape, int32_t G, const 
 MOE_API moe_status moe_ep_unpack(const moe_shape *shape, int32_t G, const void *recv_back_ovf, void *y, void *ep_ws,
                                  void *stream);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism by device-initiated peer stores ("direct" form).
+ *
+ * The same layer and the same result per rank as above, with the all-to-all
+ * written as two kernels that store rows straight into the other ranks'
+ * buffers (peer pointers, e.g. from symmetric memory or CUDA IPC over
+ * NVLink): only the routed rows cross the links (no worst-case slots), the
+ * receiver needs no copy into its layout, and the results land in each
+ * source's y rows.  The Cap-and-Spill page's two passes move a buffer sized
+ * for the worst case (the critique's point that they send as much as one
+ * padded pass); here the receive buffers are still sized for the worst case,
+ * but only the real rows move.
+ *
+ * `shape`: one rank's batch (T tokens, all E experts), uncapped layout (no
+ * MOE_FLAG_CAPACITY); E divisible by G; G * E <= 4096.  One layer on rank r:
+ *   1. moe_route_dispatch (uncapped): topk_idx, expert_counts, expert_offsets,
+ *      dest_row on rank r.
+ *   2. all-gather of expert_counts into cnt_all [G][E] int32 (every rank the
+ *      same array).
+ *   3. moe_ep_direct_plan(rank r): this rank's send positions, its local
+ *      layout and GEMM schedule (ws_loc: a workspace of the local shape,
+ *      moe_ep_direct_local_shape, initialised once) and its return segments.
+ *   4. moe_ep_direct_dispatch: each routed pair's x row into the x_loc of its
+ *      expert's rank; then a barrier over the ranks (a stream-ordered
+ *      collective), after which every rank's x_loc holds its rows.
+ *   5. moe_grouped_swiglu / moe_grouped_down on the local shape with the
+ *      local weights: x_loc -> h_loc -> y_loc.
+ *   6. moe_ep_direct_return: each local result row into its source's y row;
+ *      then a barrier.
+ *   7. moe_combine on rank r (y, dest_row, topk_w): equals moe_forward's out
+ *      on the rank's tokens with all E experts.
+ * peer_x_loc, peer_y: DEVICE arrays of G pointers (uint64), entry d = rank
+ * d's x_loc / y as this rank's kernels address it (its own entry included).
+ * x_loc holds moe_ep_direct_local_rows rows; y is moe_forward's y (T*k rows).
+ * The put kernels end with a system-scope fence.  ep_ws:
+ * moe_ep_direct_workspace_bytes bytes, written by the plan, read by the two
+ * puts of the same layer.  Errors as for the Cap-and-Spill calls; counts in
+ * cnt_all beyond what the buffers hold (each (source, expert) above T, each
+ * source's rows for one rank above T*min(k, E/G)) are clamped identically on
+ * every rank and set MOE_DEV_BAD_ROW in ws_loc's status.
+ * ------------------------------------------------------------------------ */
+
+/* Local rows of one rank, G*T*min(k, E/G); -1 for an unsupported shape or G. */
+MOE_API int64_t moe_ep_direct_local_rows(const moe_shape *shape, int32_t G);
+
+/* Bytes of the direct-form EP workspace, or 0 for an unsupported shape or G. */
+MOE_API size_t moe_ep_direct_workspace_bytes(const moe_shape *shape, int32_t G);
+
+/* The local shape of step 5: T = moe_ep_direct_local_rows, H, F, E/G experts,
+ * k = 1, C = 0, flags 0. */
+MOE_API moe_status moe_ep_direct_local_shape(const moe_shape *shape, int32_t G, moe_shape *local);
+
+/* Step 3.  cnt_all: device [G][E] int32; rank in [0, G). */
+MOE_API moe_status moe_ep_direct_plan(const moe_shape *shape, int32_t G, int32_t rank, const int32_t *cnt_all,
+                                      void *ws_loc, void *ep_ws, void *stream);
+
+/* Step 4 (ws: the rank's routing workspace, for its status word). */
+MOE_API moe_status moe_ep_direct_dispatch(const moe_shape *shape, int32_t G, const void *x, const int32_t *topk_idx,
+                                          const int32_t *dest_row, const int32_t *expert_offsets,
+                                          const void *peer_x_loc, void *ws, void *ep_ws, void *stream);
+
+/* Step 6. */
+MOE_API moe_status moe_ep_direct_return(const moe_shape *shape, int32_t G, const void *y_loc, const void *peer_y,
+                                        void *ep_ws, void *stream);
+
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
 

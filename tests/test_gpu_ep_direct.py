@@ -1,0 +1,165 @@
+"""Expert-parallel layer with device-initiated peer stores, G ranks held by one
+process on one GPU: each rank's peer tables point at the other ranks' own
+x_loc and y (connect_in_process) and the counts all-gather is done by copies.
+The put kernels store into other ranks' buffers and never wait on another
+rank, so running the ranks one after another on one GPU is safe.
+
+Each rank's output must equal, bit for bit, the single-GPU moe_forward of its
+own tokens, and match the oracle within the output tolerance; the rows each
+rank receives are checked bit-exactly against the routing (per local expert,
+every source's tokens in (source, token) order)."""
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_expert_gemm_router_b200 as moe
+import synth
+from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer
+from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "decode_E64_k6": (synth.LayerConfig("epd", 128, 256, 256, 64, 6, alpha=1.2, seed=51), (1, 2, 4, 8)),
+    "E16_k4_F384": (synth.LayerConfig("epd", 200, 256, 384, 16, 4, alpha=1.0, seed=52), (2, 4)),
+    "E8_k2_skew": (synth.LayerConfig("epd", 96, 128, 256, 8, 2, alpha=3.0, seed=53), (2, 8)),
+    "k_equals_E": (synth.LayerConfig("epd", 40, 128, 128, 4, 4, seed=54), (2, 4)),
+    "several_tiles_E4_k2": (synth.LayerConfig("epd", 700, 256, 256, 4, 2, alpha=0.3, seed=55), (2,)),
+}
+
+
+def _cases():
+    return [(name, G) for name, (_, gs) in CASES.items() for G in gs]
+
+
+def _shape(cfg):
+    return moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
+
+
+def run_direct(dl, shape, G):
+    """The layer on G emulated ranks; rank r holds tokens [r T, (r+1) T)."""
+    T, Eg = shape.T, shape.E // G
+    ranks = [DirectEP(shape, G, r) for r in range(G)]
+    connect_in_process(ranks)
+    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
+    for r, ep in enumerate(ranks):
+        ep.route(xs[r], dl.w_router, dl.bias)
+    gather_counts_in_process(ranks)
+    for ep in ranks:
+        ep.plan()
+    for r, ep in enumerate(ranks):
+        ep.dispatch(xs[r])
+    for r, ep in enumerate(ranks):
+        sl = slice(r * Eg, (r + 1) * Eg)
+        ep.experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+    for ep in ranks:
+        ep.send_back()
+    for ep in ranks:
+        ep.finish()
+    torch.cuda.synchronize()
+    return ranks, xs
+
+
+def _single_gpu(dl, shape, x):
+    b = dl.bufs(shape)
+    b["x"] = x
+    moe.moe_forward(shape, b, b["ws"], args=moe.forward_args(b))
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(b["ws"]) == 0
+    return b
+
+
+def _check_received_rows(ranks, xs, G, E, H):
+    Eg = E // G
+    idx = [ep.b["topk_idx"].cpu().numpy() for ep in ranks]
+    xh = [bf16_host(x) for x in xs]
+    for d, ep in enumerate(ranks):
+        x_loc = bf16_host(ep.x_loc)
+        row = 0
+        for el in range(Eg):
+            e = d * Eg + el
+            want = np.concatenate([xh[s][np.nonzero((idx[s] == e).any(axis=1))[0]] for s in range(G)]).reshape(-1, H)
+            assert np.array_equal(x_loc[row:row + len(want)], want), (d, el)
+            row += len(want)
+
+
+@pytest.mark.parametrize("name,G", _cases(), ids=["%s-G%d" % c for c in _cases()])
+def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G):
+    cfg, _ = CASES[name]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    ranks, xs = run_direct(dl, shape, G)
+    for ep in ranks:
+        assert moe.moe_read_status(ep.ws) == 0
+        assert moe.moe_read_status(ep.ws_loc) == 0
+    _check_received_rows(ranks, xs, G, cfg.E, cfg.H)
+    for r, ep in enumerate(ranks):
+        ref = _single_gpu(dl, shape, xs[r])
+        assert torch.equal(ep.b["topk_idx"], ref["topk_idx"])
+        assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(ref["out"])), "rank %d" % r
+        view = types.SimpleNamespace(x=L.x[r * cfg.T:(r + 1) * cfg.T], w_gate=L.w_gate, w_up=L.w_up,
+                                     w_down=L.w_down)
+        o = oracle_layer(orc, view, cfg, ep.b["logits"].cpu().numpy())
+        assert_close_bf16(bf16_host(ep.b["out"]), o["out"], "out rank %d" % r)
+
+
+# Full size: the Mixtral-8x7B-shaped layer (T = 512 per rank, H = 4096,
+# F = 14336, E = 8, k = 2) on 2 and 8 ranks, bit for bit against each rank's
+# single-GPU layer (which the full-size parity tests pin to the oracle).
+@pytest.mark.parametrize("G", [2, 8])
+def test_direct_ep_full_size_mixtral_matches_single_gpu(G):
+    cfg = synth.CONFIGS[2]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    ranks, xs = run_direct(dl, shape, G)
+    for r, ep in enumerate(ranks):
+        assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
+        ref = _single_gpu(dl, shape, xs[r])
+        assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(ref["out"])), "rank %d" % r
+
+
+def test_direct_ep_clamps_counts_beyond_the_buffers():
+    """Gathered counts past what the buffers hold (a source claiming more
+    rows than it can send) are clamped the same way on every rank: nothing
+    is stored outside a buffer, MOE_DEV_BAD_ROW is raised, and a clean layer
+    in the same context still matches the single-GPU one."""
+    cfg = CASES["E16_k4_F384"][0]
+    G = 2
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    ranks = [DirectEP(shape, G, r) for r in range(G)]
+    connect_in_process(ranks)
+    for r, ep in enumerate(ranks):
+        ep.route(dl.x[r * cfg.T:(r + 1) * cfg.T], dl.w_router, dl.bias)
+    gather_counts_in_process(ranks)
+    for ep in ranks:
+        ep.cnt_all[0, 3] = 1 << 24  # more than T pairs for one expert
+        ep.cnt_all[1, :] = cfg.T    # more rows than one source can send a rank
+        ep.plan()
+    torch.cuda.synchronize()
+    for r, ep in enumerate(ranks):
+        ep.dispatch(dl.x[r * cfg.T:(r + 1) * cfg.T])
+    torch.cuda.synchronize()
+    assert all(moe.moe_read_status(ep.ws_loc) & moe.MOE_DEV_BAD_ROW for ep in ranks)
+    for ep in ranks:
+        moe.moe_read_status(ep.ws)  # clear
+    ranks2, xs = run_direct(dl, shape, G)
+    for r, ep in enumerate(ranks2):
+        assert moe.moe_read_status(ep.ws_loc) == 0
+        ref = _single_gpu(dl, shape, xs[r])
+        assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(ref["out"]))
+
+
+def test_direct_ep_rejects_unsupported_shapes():
+    cfg = CASES["E16_k4_F384"][0]
+    with pytest.raises(moe.MoeError):
+        DirectEP(moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=8, capacity=True), 2, 0)
+    with pytest.raises(moe.MoeError):
+        DirectEP(_shape(cfg), 3, 0)  # E % G != 0
+    with pytest.raises(moe.MoeError):
+        DirectEP(_shape(cfg), 2, 2)  # rank out of range
