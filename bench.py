@@ -637,6 +637,77 @@ class Bench:
         return {"G": G, "S": S, "per_phase_us_all_ranks": per_phase, "overflow_rows": spill,
                 "device_status": status, "single_gpu_layer_us": m1["total_ms"] / steps * 1e3}
 
+    def measure_ep_direct(self, cfg, L, G, steps, warmup):
+        """The peer-store expert-parallel layer with G ranks held by this
+        process: peer tables point at the other ranks' own buffers, so the
+        stores stay on this GPU (on G GPUs they cross NVLink); the counts
+        all-gather is done by copies (untimed).  Per-phase device times summed
+        over the ranks, L2 cleaned before every step."""
+        import numpy as np
+
+        import grouped_expert_gemm_router_b200 as moe
+        from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
+        torch, dev, stream = self.torch, self.dev, self.stream
+
+        def dev_bf16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
+        wg, wu, wd = dev_bf16(L.w_gate), dev_bf16(L.w_up), dev_bf16(L.w_down)
+        wr = torch.from_numpy(L.w_router).to(dev)
+        bias = None if L.bias is None else torch.from_numpy(L.bias).to(dev)
+        xs = [dev_bf16(replica_tokens(cfg, r, L)) for r in range(G)]
+        ranks = [DirectEP(shape, G, r, dev) for r in range(G)]
+        connect_in_process(ranks)
+        Eg = cfg.E // G
+        sl = [slice(r * Eg, (r + 1) * Eg) for r in range(G)]
+        phases = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "finish")
+        calls = {
+            "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
+            "plan": lambda r: ranks[r].plan(stream),
+            "dispatch": lambda r: ranks[r].dispatch(xs[r], stream),
+            "experts_swiglu": lambda r: moe.moe_grouped_swiglu(ranks[r].local, ranks[r].x_loc, wg[sl[r]], wu[sl[r]],
+                                                               ranks[r].h_loc, ranks[r].ws_loc, stream),
+            "experts_down": lambda r: moe.moe_grouped_down(ranks[r].local, ranks[r].h_loc, wd[sl[r]], ranks[r].y_loc,
+                                                           ranks[r].ws_loc, stream),
+            "send_back": lambda r: ranks[r].send_back(stream),
+            "finish": lambda r: ranks[r].finish(stream),
+        }
+
+        def step(timed):
+            ev = {}
+            for ph in phases:
+                if ph == "plan":
+                    gather_counts_in_process(ranks)
+                for r in range(G):
+                    if timed:
+                        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                        calls[ph](r)
+                        c.record(stream)
+                        ev[(ph, r)] = (a, c)
+                    else:
+                        calls[ph](r)
+            return ev
+
+        for _ in range(warmup):
+            self.flush()
+            step(False)
+        self.barrier()
+        evs = []
+        for _ in range(steps):
+            self.flush()
+            evs.append(step(True))
+        self.barrier()
+        per_phase = {ph: float(np.mean([sum(e[(ph, r)][0].elapsed_time(e[(ph, r)][1]) for r in range(G))
+                                         for e in evs])) * 1e3 for ph in phases}
+        status = [moe.moe_read_status(ep.ws) | moe.moe_read_status(ep.ws_loc) for ep in ranks]
+        shp1, b1 = self.upload(cfg, L, replica_tokens(cfg, 0, L))
+        m1 = self.measure(cfg, shp1, b1, steps, warmup)
+        del b1, ranks
+        return {"G": G, "per_phase_us_all_ranks": per_phase, "device_status": status,
+                "single_gpu_layer_us": m1["total_ms"] / steps * 1e3}
+
     def e2e_pipelined(self, cfg, shape, b, x_rank, fwd_bufs, steps, warmup):
         """End to end as a serving loop runs it: step i's tokens are copied in
         on one copy stream while step i-1's layer runs, and step i-1's output
@@ -788,6 +859,45 @@ def summarize_ep(cfg, e, peaks):
                               "nvlink_model_us": 2 * (p1 + p2 + meta) / (NVLINK_PEER_GBS * 1e9) * 1e6,
                               "nvlink_model": "dispatch and return passes, each rank's sent bytes at %g GB/s per "
                                               "direction (a model, not a measurement)" % NVLINK_PEER_GBS},
+        "device_status": e["device_status"],
+    }
+
+
+def experts_roofline(cfg, G, t, peaks):
+    """The local grouped GEMMs of one rank (SwiGLU + down, t seconds) against
+    the larger of the rank's expert-weight bytes over HBM bandwidth and its
+    average rows' (T k) FLOPs over the bf16 tensor peak."""
+    Eg = cfg.E // G
+    w_bytes = 3 * Eg * cfg.H * cfg.F * 2
+    flops = 2.0 * cfg.T * cfg.k * cfg.H * cfg.F * 3
+    if w_bytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12):
+        a = w_bytes / t / 1e9
+        return {"bound": "hbm", "bytes": w_bytes, "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": a / peaks["hbm_gbs"]}
+    a = flops / t / 1e12
+    return {"bound": "tensor", "flops": flops, "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": a / peaks["bf16_tflops"]}
+
+
+def summarize_ep_direct(cfg, e, peaks):
+    """The peer-store expert-parallel layer per rank: kernel time of each
+    phase and the bytes each rank stores into other ranks per direction."""
+    G, row = e["G"], cfg.H * 2
+    Eg = cfg.E // G
+    per_rank = {ph: t / G for ph, t in e["per_phase_us_all_ranks"].items()}
+    sent = cfg.T * cfg.k * row  # every routed row once out, its result once back
+    t_exp = (per_rank["experts_swiglu"] + per_rank["experts_down"]) * 1e-6
+    return {
+        "workload": workload_name(cfg) + "-uncapped", "G": G,
+        "ranks": "G ranks emulated on one GPU: each rank's peer stores go to the other ranks' buffers on the same "
+                 "device; the counts all-gather done by copies and not timed",
+        "per_rank_us": per_rank, "per_rank_kernels_us": sum(per_rank.values()),
+        "single_gpu_layer_us": e["single_gpu_layer_us"],
+        "experts_roofline": experts_roofline(cfg, G, t_exp, peaks),
+        "exchange_per_rank": {"dispatch_bytes": sent, "return_bytes": sent, "counts_bytes": G * cfg.E * 4,
+                              "nvlink_model_us": 2 * sent / (NVLINK_PEER_GBS * 1e9) * 1e6,
+                              "nvlink_model": "routed rows out and results back at %g GB/s per direction (a "
+                                              "model, not a measurement)" % NVLINK_PEER_GBS},
         "device_status": e["device_status"],
     }
 
@@ -957,7 +1067,19 @@ def run_ours(args):
         ep = summarize_ep(ce, bench.measure_ep(ce, Le, 8, min(K, args.per_config_steps), min(args.warmup, 5)), peaks)
         log("expert-parallel %s G=8: %.1f us of kernels per rank (%.1f s)" % (ce.name, ep["per_rank_kernels_us"],
                                                                               time.time() - t0))
+        # the same layer by peer stores (uncapped), and the Mixtral-shaped one
+        ep["direct"] = summarize_ep_direct(ce, bench.measure_ep_direct(
+            ce, Le, 8, min(K, args.per_config_steps), min(args.warmup, 5)), peaks)
         del Le
+        gc.collect()
+        torch.cuda.empty_cache()
+        cm = synth.CONFIGS[2]
+        Lm = synth.make_layer(cm)
+        ep["direct_mixtral"] = summarize_ep_direct(cm, bench.measure_ep_direct(
+            cm, Lm, 8, min(K, args.per_config_steps), min(args.warmup, 5)), peaks)
+        log("peer-store EP G=8: %.1f / %.1f us of kernels per rank (%.1f s)" % (
+            ep["direct"]["per_rank_kernels_us"], ep["direct_mixtral"]["per_rank_kernels_us"], time.time() - t0))
+        del Lm
         gc.collect()
         torch.cuda.empty_cache()
 

@@ -45,8 +45,10 @@ __device__ __forceinline__ void copy_row16(const uint4 *__restrict__ src, uint4 
     for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
 }
 
-// Smallest per-rank figures: at most kDirMaxCounts (source, expert) counts.
+// At most kDirMaxCounts (source, expert) counts; the return kernel keeps up
+// to kDirSmemSegs segment starts in shared memory.
 constexpr int kDirMaxCounts = 4096;
+constexpr int kDirSmemSegs = 1024;
 
 struct DirPlanArgs {
     const int32_t *cnt_all;  // [G][E] as gathered
@@ -160,10 +162,15 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_return(const uint4 *y
                                                                    const unsigned long long *peer_y, int G, int Eg,
                                                                    int Tloc, int P, int H8) {
     __shared__ int offs[kMaxExperts + 1];
+    __shared__ int sstart[kDirSmemSegs];
     pdl_trigger();
     pdl_wait();
     for (int i = threadIdx.x; i <= Eg; i += kDirThreads) offs[i] = loc_offsets[i];
+    const bool staged = G * Eg <= kDirSmemSegs;  // segment starts searched in shared memory
+    if (staged)
+        for (int i = threadIdx.x; i < G * Eg; i += kDirThreads) sstart[i] = seg_start[i];
     __syncthreads();
+    const int *starts = staged ? sstart : seg_start;
     const int lane = threadIdx.x & 31;
     const int total = min(offs[Eg], Tloc);
     for (int r = blockIdx.x * kDirWarps + (threadIdx.x >> 5); r < total; r += gridDim.x * kDirWarps) {
@@ -178,10 +185,10 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_return(const uint4 *y
         hi = G - 1;  // source: last s with seg_start[s][el] <= r (empty segments share a start)
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (seg_start[mid * Eg + el] <= r) lo = mid;
+            if (starts[mid * Eg + el] <= r) lo = mid;
             else hi = mid - 1;
         }
-        const int i = lo * Eg + el, j = r - seg_start[i];
+        const int i = lo * Eg + el, j = r - starts[i];
         const int yrow = seg_ysrc[i] + j;
         if (j >= seg_cnt[i] || (unsigned)yrow >= (unsigned)P) continue;  // cannot happen: the plan's layout
         uint4 *dst = reinterpret_cast<uint4 *>(peer_y[lo]) + (size_t)yrow * H8;
