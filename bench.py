@@ -661,7 +661,10 @@ class Bench:
         connect_in_process(ranks)
         Eg = cfg.E // G
         sl = [slice(r * Eg, (r + 1) * Eg) for r in range(G)]
-        phases = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "finish")
+        # experts_down + send_back and their fused form (the down GEMM storing
+        # into the owners' y) both run each step; the totals count one or the other
+        phases = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "down_return_fused",
+                  "finish")
         calls = {
             "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
             "plan": lambda r: ranks[r].plan(stream),
@@ -671,6 +674,8 @@ class Bench:
             "experts_down": lambda r: moe.moe_grouped_down(ranks[r].local, ranks[r].h_loc, wd[sl[r]], ranks[r].y_loc,
                                                            ranks[r].ws_loc, stream),
             "send_back": lambda r: ranks[r].send_back(stream),
+            "down_return_fused": lambda r: moe.moe_ep_direct_down_return(shape, G, ranks[r].h_loc, wd[sl[r]],
+                                                                         ranks[r].ws_loc, ranks[r].ep_ws, stream),
             "finish": lambda r: ranks[r].finish(stream),
         }
 
@@ -891,7 +896,10 @@ def summarize_ep_direct(cfg, e, peaks):
         "workload": workload_name(cfg) + "-uncapped", "G": G,
         "ranks": "G ranks emulated on one GPU: each rank's peer stores go to the other ranks' buffers on the same "
                  "device; the counts all-gather done by copies and not timed",
-        "per_rank_us": per_rank, "per_rank_kernels_us": sum(per_rank.values()),
+        "per_rank_us": per_rank,
+        "per_rank_kernels_us": sum(v for k, v in per_rank.items() if k != "down_return_fused"),
+        "per_rank_kernels_fused_return_us": sum(v for k, v in per_rank.items()
+                                                if k not in ("experts_down", "send_back")),
         "single_gpu_layer_us": e["single_gpu_layer_us"],
         "experts_roofline": experts_roofline(cfg, G, t_exp, peaks),
         "exchange_per_rank": {"dispatch_bytes": sent, "return_bytes": sent, "counts_bytes": G * cfg.E * 4,

@@ -41,7 +41,7 @@ ABI_FUNCTIONS = (
     "moe_grouped_down_combine", "moe_grouped_down_fp8_combine", "moe_ep_overflow_rows", "moe_ep_workspace_bytes",
     "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
-    "moe_ep_direct_dispatch", "moe_ep_direct_return",
+    "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -166,12 +166,14 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_direct_workspace_bytes.restype = ctypes.c_size_t
     lib.moe_ep_direct_local_shape.argtypes = [sp, i32, sp]
     lib.moe_ep_direct_local_shape.restype = st
-    lib.moe_ep_direct_plan.argtypes = [sp, i32, i32] + [vp] * 4
+    lib.moe_ep_direct_plan.argtypes = [sp, i32, i32] + [vp] * 5
     lib.moe_ep_direct_plan.restype = st
     lib.moe_ep_direct_dispatch.argtypes = [sp, i32] + [vp] * 8
     lib.moe_ep_direct_dispatch.restype = st
     lib.moe_ep_direct_return.argtypes = [sp, i32] + [vp] * 4
     lib.moe_ep_direct_return.restype = st
+    lib.moe_ep_direct_down_return.argtypes = [sp, i32] + [vp] * 5
+    lib.moe_ep_direct_down_return.restype = st
     _lib = lib
     return lib
 
@@ -470,9 +472,10 @@ def moe_ep_direct_local_shape(shape, G) -> MoeShape:
     return out
 
 
-def moe_ep_direct_plan(shape, G, rank, cnt_all, ws_loc, ep_ws, stream=None):
-    _check(load_library().moe_ep_direct_plan(ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(ws_loc),
-                                             _ptr(ep_ws), _stream(stream)), "moe_ep_direct_plan")
+def moe_ep_direct_plan(shape, G, rank, cnt_all, peer_y, ws_loc, ep_ws, stream=None):
+    """peer_y: a device tensor of G int64 addresses, or None."""
+    _check(load_library().moe_ep_direct_plan(ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(peer_y),
+                                             _ptr(ws_loc), _ptr(ep_ws), _stream(stream)), "moe_ep_direct_plan")
 
 
 def moe_ep_direct_dispatch(shape, G, x, topk_idx, dest_row, expert_offsets, peer_x_loc, ws, ep_ws, stream=None):
@@ -487,3 +490,8 @@ def moe_ep_direct_return(shape, G, y_loc, peer_y, ep_ws, stream=None):
     _check(load_library().moe_ep_direct_return(ctypes.byref(shape), int(G), _ptr(y_loc), _ptr(peer_y), _ptr(ep_ws),
                                                 _stream(stream)), "moe_ep_direct_return")
 
+
+def moe_ep_direct_down_return(shape, G, h_loc, w_down, ws_loc, ep_ws, stream=None):
+    _check(load_library().moe_ep_direct_down_return(ctypes.byref(shape), int(G), _ptr(h_loc), _ptr(w_down),
+                                                    _ptr(ws_loc), _ptr(ep_ws), _stream(stream)),
+           "moe_ep_direct_down_return")

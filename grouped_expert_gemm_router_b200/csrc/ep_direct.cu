@@ -56,6 +56,9 @@ struct DirPlanArgs {
     int32_t *send_base, *send_cnt;               // [E]
     int32_t *seg_start, *seg_cnt, *seg_ysrc;     // [G][E_g]
     int32_t *loc_counts, *loc_offsets;           // [E_g], [E_g + 1]
+    const unsigned long long *peer_y;            // [G] or null
+    unsigned long long *row_addr;                // [local T]: byte address of each local row's result
+    int H, P;
     WsPtrs lws;
 };
 
@@ -115,6 +118,8 @@ __global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) 
     build_schedule_block(sm, Eg, 0, false, a.loc_counts, a.loc_offsets, a.lws);
     // Return segments: (source s, local expert el) -> first local row, rows,
     // first row in the source's y (its uncapped offset of the expert).
+    // G E_g = E segments, kept in shared memory (base[] is free again).
+    int *sstart = base;
     for (int i = tid; i < G * Eg; i += kScanThreads) {
         const int s = i / Eg, el = i % Eg, e = r * Eg + el;
         int start = sm.offs[el];
@@ -124,6 +129,34 @@ __global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) 
         a.seg_start[i] = start;
         a.seg_cnt[i] = c[s * E + e];
         a.seg_ysrc[i] = ysrc;
+        sstart[i] = start;
+        sm.running[i] = ysrc;  // scratch: the segment's first row in the source's y
+    }
+    __syncthreads();
+    // Each local row's destination: the byte address of its row in its
+    // token's rank's y (0 without peer addresses), for the down projection
+    // that stores its results there itself.
+    const int total = sm.offs[Eg];
+    for (int row = tid; row < total; row += kScanThreads) {
+        int lo = 0, hi = Eg - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sm.offs[mid] <= row) lo = mid;
+            else hi = mid - 1;
+        }
+        const int el = lo;
+        lo = 0;
+        hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sstart[mid * Eg + el] <= row) lo = mid;
+            else hi = mid - 1;
+        }
+        const int i = lo * Eg + el;
+        const int yrow = sm.running[i] + (row - sstart[i]);
+        a.row_addr[row] = (a.peer_y && (unsigned)yrow < (unsigned)a.P)
+                              ? a.peer_y[lo] + (unsigned long long)yrow * (unsigned long long)a.H * 2ull
+                              : 0ull;
     }
 }
 
@@ -217,12 +250,14 @@ bool ep_direct_counts_fit(const moe_shape &s, int G) { return (int64_t)G * s.E <
 // counts [E] each, return segments (start, rows, source row) [G E_g] each,
 // local counts [E_g], local offsets [E_g + 1].
 struct DirWs {
+    unsigned long long *row_addr;
     int32_t *send_base, *send_cnt, *seg_start, *seg_cnt, *seg_ysrc, *loc_counts, *loc_offsets;
 };
 static DirWs dir_ptrs(void *ep_ws, const moe_shape &s, int G) {
-    int32_t *b = (int32_t *)ep_ws;
     const size_t E4 = align_up((size_t)s.E, 4), Eg = (size_t)(s.E / G);
     DirWs p;
+    p.row_addr = (unsigned long long *)ep_ws;
+    int32_t *b = (int32_t *)(p.row_addr + align_up((size_t)ep_direct_local_rows(s, G), 2));
     p.send_base = b;
     p.send_cnt = p.send_base + E4;
     p.seg_start = p.send_cnt + E4;
@@ -235,11 +270,15 @@ static DirWs dir_ptrs(void *ep_ws, const moe_shape &s, int G) {
 
 size_t ep_direct_workspace_bytes(const moe_shape &s, int G) {
     const size_t E4 = align_up((size_t)s.E, 4), Eg = (size_t)(s.E / G);
-    return 4 * (5 * E4 + align_up(Eg, 4) + align_up(Eg + 1, 4));
+    return 8 * align_up((size_t)ep_direct_local_rows(s, G), 2) + 4 * (5 * E4 + align_up(Eg, 4) + align_up(Eg + 1, 4));
 }
 
-cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const WsLayout &Lloc,
-                                  void *ws_loc, void *ep_ws, cudaStream_t stream) {
+const unsigned long long *ep_direct_row_addr(void *ep_ws, const moe_shape &s, int G) {
+    return dir_ptrs(ep_ws, s, G).row_addr;
+}
+
+cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
+                                  const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream) {
     const DirWs p = dir_ptrs(ep_ws, s, G);
     DirPlanArgs a;
     a.cnt_all = cnt_all;
@@ -255,6 +294,10 @@ cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int
     a.seg_ysrc = p.seg_ysrc;
     a.loc_counts = p.loc_counts;
     a.loc_offsets = p.loc_offsets;
+    a.peer_y = (const unsigned long long *)peer_y;
+    a.row_addr = p.row_addr;
+    a.H = s.H;
+    a.P = s.T * s.k;
     a.lws = ws_ptrs(ws_loc, Lloc);
     return launch_pdl(k_ep_direct_plan, dim3(1), dim3(kScanThreads), 0, stream, a);
 }

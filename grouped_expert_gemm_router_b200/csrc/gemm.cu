@@ -100,6 +100,10 @@ struct GemmArgs {
     uint32_t *status;
     __nv_bfloat16 *out;
     int n_out;   // row length of `out`: F (mode 0) or H (mode 1)
+    // mode 1 without the fused combine: when set, row r of the result goes to
+    // row_addr[r] (a byte address, anywhere the GPU can store: another GPU's
+    // memory included) instead of out + r * n_out; entries of 0 are skipped
+    const unsigned long long *row_addr;
     int K;       // reduction length: H (mode 0) or F (mode 1)
     int num_fb;  // feature blocks per row tile
     int E;
@@ -231,7 +235,8 @@ __device__ __forceinline__ int unit_row(const Unit &U, int c) {
 // row) and stores it.  Two 16-byte store instructions per warp for the
 // block instead of sixteen 2-byte ones.
 __device__ __forceinline__ void store_block_frag(const uint32_t (&w)[8], uint8_t *stg, __nv_bfloat16 *out, int n_out,
-                                                 int fbase, const Unit &U, int c0) {
+                                                 const unsigned long long *row_addr, int fbase, const Unit &U,
+                                                 int c0) {
     const int lane = threadIdx.x & 31;
     const int mi = lane >> 3, mj = lane & 7;  // stmatrix: row mj of matrix (feature group) mi
     const int r = lane >> 2, c = lane & 3;    // read-back: row r, feature group c
@@ -244,7 +249,13 @@ __device__ __forceinline__ void store_block_frag(const uint32_t (&w)[8], uint8_t
         const uint4 v = lds128(ld_addr);
         __syncwarp();  // the block is rewritten by the next group
         const int row = unit_row(U, c0 + 8 * k + r);
-        if (row >= 0) *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + 8 * c) = v;
+        if (row < 0) continue;
+        if (row_addr) {  // the row's own destination (another GPU's memory, say); 0 = none
+            const unsigned long long d = row_addr[row];
+            if (d) *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(d) + fbase + 8 * c) = v;
+        } else {
+            *reinterpret_cast<uint4 *>(out + (size_t)row * n_out + fbase + 8 * c) = v;
+        }
     }
 }
 
@@ -963,7 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 uint32_t w[8];
 #pragma unroll
                                 for (int m = 0; m < 8; ++m) w[m] = pack_bf16x2(r[2 * m], r[2 * m + 1]);
-                                store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                                store_block_frag(w, stg, a.out, a.n_out, a.row_addr, U.fx + 128 + q * 32, U, c0);
                             }
                         }
                     }
@@ -973,8 +984,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < kBigChunks; ++i) {
                     const int c0 = (sub + kEpiSub * i) * 16;
                     if (c0 < U.N) {
-                        store_block_frag(h0[i], stg, a.out, a.n_out, U.fx + q * 32, U, c0);
-                        if (i < kHold1 && U.nacc == 2) store_block_frag(h1[i], stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                        store_block_frag(h0[i], stg, a.out, a.n_out, a.row_addr, U.fx + q * 32, U, c0);
+                        if (i < kHold1 && U.nacc == 2) store_block_frag(h1[i], stg, a.out, a.n_out, a.row_addr, U.fx + 128 + q * 32, U, c0);
                     }
                 }
                 if (COMBINE) arrive_and_combine(a, U, sub, lane);
@@ -1005,7 +1016,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < kOneChunks; ++i) {
                     const int c0 = (sub + kEpiSub * i) * 16;
-                    if (c0 < U.N) store_block_frag(h0[i], stg, a.out, a.n_out, U.fx + q * 32, U, c0);
+                    if (c0 < U.N) store_block_frag(h0[i], stg, a.out, a.n_out, a.row_addr, U.fx + q * 32, U, c0);
                 }
                 if (COMBINE) arrive_and_combine(a, U, sub, lane);
                 plan.advance(big, h);
@@ -1062,11 +1073,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t w[8];
 #pragma unroll
                     for (int m = 0; m < 8; ++m) w[m] = hold[i][m];
-                    store_block_frag(w, stg, a.out, a.n_out, U.fx + q * 32, U, c0);
+                    store_block_frag(w, stg, a.out, a.n_out, a.row_addr, U.fx + q * 32, U, c0);
                     if (MODE == 1 && U.nacc == 2) {
 #pragma unroll
                         for (int m = 0; m < 8; ++m) w[m] = hold[i][8 + m];
-                        store_block_frag(w, stg, a.out, a.n_out, U.fx + 128 + q * 32, U, c0);
+                        store_block_frag(w, stg, a.out, a.n_out, a.row_addr, U.fx + 128 + q * 32, U, c0);
                     }
                 }
             }
@@ -1195,7 +1206,8 @@ cudaError_t launch_router_logits_tc(const moe_shape &s, const void *x, const flo
 // comb (mode 1, nullable): the combine of step 5 in the epilogue, into comb->out.
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb) {
+                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb,
+                                const unsigned long long *row_addr) {
     const bool gather = mode == 0 && src_token != nullptr;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
@@ -1232,6 +1244,7 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
     a.src_token = src_token;
     a.row_boxes = boxes;
     a.stall_first_stage = (mode == 0 && !gather && (s.flags & MOE_FLAG_TEST_STALL_GEMM)) ? 1 : 0;
+    a.row_addr = (mode == 1 && !comb) ? row_addr : nullptr;
     static bool attr_done[6] = {false, false, false, false, false, false};
     cudaError_t err;
     if (mode == 1 && comb) {
@@ -1285,7 +1298,8 @@ cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, c
 cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *act, const float *row_scale,
                                     const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
                                     void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb) {
+                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb,
+                                const unsigned long long *row_addr) {
     const bool gather = mode == 0 && src_token != nullptr;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);

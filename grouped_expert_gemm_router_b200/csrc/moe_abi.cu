@@ -22,13 +22,15 @@ cudaError_t launch_permute(const moe_shape &s, const void *x, const int32_t *top
                            void *ws, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm(int mode, const moe_shape &s, const void *act, const void *w0, const void *w1,
                                 void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr);
+                                cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr,
+                                const unsigned long long *row_addr = nullptr);
 cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *dest_row, const float *topk_w, void *out,
                            cudaStream_t stream);
 cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *act, const float *row_scale,
                                     const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
                                     void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
-                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr);
+                                    cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr,
+                                const unsigned long long *row_addr = nullptr);
 cudaError_t launch_quant_weights(int E, int K, int N, const void *w, void *q, float *scale, cudaStream_t stream);
 cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int src_rows, const int32_t *idx,
                               bool gather, void *q, float *scale, const WsLayout &L, void *ws, int num_sms,
@@ -49,8 +51,9 @@ cudaError_t launch_ep_unpack(const moe_shape &s, int G, const void *recv_back_ov
 int64_t ep_direct_local_rows(const moe_shape &s, int G);
 bool ep_direct_counts_fit(const moe_shape &s, int G);
 size_t ep_direct_workspace_bytes(const moe_shape &s, int G);
-cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const WsLayout &Lloc,
-                                  void *ws_loc, void *ep_ws, cudaStream_t stream);
+cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
+                                  const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream);
+const unsigned long long *ep_direct_row_addr(void *ep_ws, const moe_shape &s, int G);
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
                                  const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
                                  void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream);
@@ -649,16 +652,16 @@ moe_status moe_ep_direct_local_shape(const moe_shape *s, int32_t G, moe_shape *l
     return check_shape(local);
 }
 
-moe_status moe_ep_direct_plan(const moe_shape *s, int32_t G, int32_t rank, const int32_t *cnt_all, void *ws_loc,
-                              void *ep_ws, void *stream) {
+moe_status moe_ep_direct_plan(const moe_shape *s, int32_t G, int32_t rank, const int32_t *cnt_all,
+                              const void *peer_y, void *ws_loc, void *ep_ws, void *stream) {
     moe_status st = check_ep_direct(s, G);
     if (st != MOE_OK) return st;
     if (rank < 0 || rank >= G) return MOE_ERR_INVALID_ARG;
-    if (!aligned(cnt_all, 4) || !aligned(ep_ws, 16)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(cnt_all, 4) || !aligned(ep_ws, 16) || (peer_y && !aligned(peer_y, 8))) return MOE_ERR_INVALID_ARG;
     if ((st = check_ws(ws_loc)) != MOE_OK) return st;
     const moe_shape l = ep_direct_local(s, G);
     const WsLayout Lloc = layout_of(&l);
-    cudaError_t e = launch_ep_direct_plan(*s, G, rank, cnt_all, Lloc, ws_loc, ep_ws, (cudaStream_t)stream);
+    cudaError_t e = launch_ep_direct_plan(*s, G, rank, cnt_all, peer_y, Lloc, ws_loc, ep_ws, (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_plan");
 }
 
@@ -690,3 +693,19 @@ moe_status moe_ep_direct_return(const moe_shape *s, int32_t G, const void *y_loc
     cudaError_t e = launch_ep_direct_return(*s, G, y_loc, peer_y, ep_ws, sms, (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_return");
 }
+
+moe_status moe_ep_direct_down_return(const moe_shape *s, int32_t G, const void *h_loc, const void *w_down,
+                                     void *ws_loc, void *ep_ws, void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(h_loc, 16) || !aligned(w_down, 16) || !aligned(ep_ws, 16)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws_loc)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const moe_shape l = ep_direct_local(s, G);
+    const WsLayout Lloc = layout_of(&l);
+    cudaError_t e = launch_grouped_gemm(1, l, h_loc, w_down, w_down, nullptr, Lloc, ws_loc, g_timeout_ns.load(), sms,
+                                        (cudaStream_t)stream, nullptr, nullptr, ep_direct_row_addr(ep_ws, *s, G));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_down_return");
+}
+

@@ -87,7 +87,8 @@ class DirectEP:
 
     def plan(self, stream=None):
         """Send positions, the local layout and schedule, the return segments."""
-        moe.moe_ep_direct_plan(self.shape, self.G, self.rank, self.cnt_all, self.ws_loc, self.ep_ws, stream)
+        moe.moe_ep_direct_plan(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, self.ws_loc, self.ep_ws,
+                               stream)
 
     def dispatch(self, x, stream=None):
         """Each routed token row into its expert's rank's x_loc (peer stores)."""
@@ -100,6 +101,14 @@ class DirectEP:
         L = self.local
         moe.moe_grouped_swiglu(L, self.x_loc, w_gate, w_up, self.h_loc, self.ws_loc, stream)
         moe.moe_grouped_down(L, self.h_loc, w_down, self.y_loc, self.ws_loc, stream)
+
+    def experts_and_return(self, w_gate, w_up, w_down, stream=None):
+        """The grouped SwiGLU GEMM, then the down projection whose epilogue
+        stores each result row straight into its token's rank's y (one
+        kernel for the down GEMM and the return)."""
+        L = self.local
+        moe.moe_grouped_swiglu(L, self.x_loc, w_gate, w_up, self.h_loc, self.ws_loc, stream)
+        moe.moe_ep_direct_down_return(self.shape, self.G, self.h_loc, w_down, self.ws_loc, self.ep_ws, stream)
 
     def send_back(self, stream=None):
         """Each result row into its token's rank's y (peer stores)."""
@@ -135,8 +144,10 @@ class DirectEP:
         ep._group = group
         return ep
 
-    def forward(self, x, w_router, bias, w_gate, w_up, w_down):
-        """One layer on this rank (every rank of the group calls it)."""
+    def forward(self, x, w_router, bias, w_gate, w_up, w_down, fused_return=True):
+        """One layer on this rank (every rank of the group calls it);
+        fused_return: the down GEMM stores the results into the owners' y
+        itself (else a separate return kernel)."""
         import torch.distributed as dist
         group = self._group
 
@@ -148,8 +159,11 @@ class DirectEP:
         self.plan()
         self.dispatch(x)
         barrier()
-        self.experts(w_gate, w_up, w_down)
-        self.send_back()
+        if fused_return:
+            self.experts_and_return(w_gate, w_up, w_down)
+        else:
+            self.experts(w_gate, w_up, w_down)
+            self.send_back()
         barrier()
         return self.finish()
 

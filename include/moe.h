@@ -530,9 +530,11 @@ MOE_API size_t moe_ep_direct_workspace_bytes(const moe_shape *shape, int32_t G);
  * k = 1, C = 0, flags 0. */
 MOE_API moe_status moe_ep_direct_local_shape(const moe_shape *shape, int32_t G, moe_shape *local);
 
-/* Step 3.  cnt_all: device [G][E] int32; rank in [0, G). */
+/* Step 3.  cnt_all: device [G][E] int32; rank in [0, G); peer_y: the device
+ * array of step 6 (may be null when moe_ep_direct_down_return is not used):
+ * the plan also records each local row's destination address for it. */
 MOE_API moe_status moe_ep_direct_plan(const moe_shape *shape, int32_t G, int32_t rank, const int32_t *cnt_all,
-                                      void *ws_loc, void *ep_ws, void *stream);
+                                      const void *peer_y, void *ws_loc, void *ep_ws, void *stream);
 
 /* Step 4 (ws: the rank's routing workspace, for its status word). */
 MOE_API moe_status moe_ep_direct_dispatch(const moe_shape *shape, int32_t G, const void *x, const int32_t *topk_idx,
@@ -542,6 +544,15 @@ MOE_API moe_status moe_ep_direct_dispatch(const moe_shape *shape, int32_t G, con
 /* Step 6. */
 MOE_API moe_status moe_ep_direct_return(const moe_shape *shape, int32_t G, const void *y_loc, const void *peer_y,
                                         void *ep_ws, void *stream);
+
+/* Steps 5b and 6 in one kernel: the local down projection (h_loc [local T][F]
+ * bf16, w_down: the rank's [E/G][F][H] slice) whose epilogue stores each
+ * result row straight into its token's rank's y, at the address the plan
+ * recorded from peer_y (rows without one are not stored).  Replaces
+ * moe_grouped_down + moe_ep_direct_return; the plan must have been given
+ * peer_y.  A barrier over the ranks follows, as after step 6. */
+MOE_API moe_status moe_ep_direct_down_return(const moe_shape *shape, int32_t G, const void *h_loc,
+                                             const void *w_down, void *ws_loc, void *ep_ws, void *stream);
 
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);

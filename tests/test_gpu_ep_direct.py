@@ -38,8 +38,9 @@ def _shape(cfg):
     return moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
 
 
-def run_direct(dl, shape, G):
-    """The layer on G emulated ranks; rank r holds tokens [r T, (r+1) T)."""
+def run_direct(dl, shape, G, fused_return=False):
+    """The layer on G emulated ranks; rank r holds tokens [r T, (r+1) T).
+    fused_return: the down GEMM stores its results into the owners' y."""
     T, Eg = shape.T, shape.E // G
     ranks = [DirectEP(shape, G, r) for r in range(G)]
     connect_in_process(ranks)
@@ -53,9 +54,13 @@ def run_direct(dl, shape, G):
         ep.dispatch(xs[r])
     for r, ep in enumerate(ranks):
         sl = slice(r * Eg, (r + 1) * Eg)
-        ep.experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
-    for ep in ranks:
-        ep.send_back()
+        if fused_return:
+            ep.experts_and_return(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+        else:
+            ep.experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+    if not fused_return:
+        for ep in ranks:
+            ep.send_back()
     for ep in ranks:
         ep.finish()
     torch.cuda.synchronize()
@@ -85,13 +90,19 @@ def _check_received_rows(ranks, xs, G, E, H):
             row += len(want)
 
 
+FUSED = [("decode_E64_k6", 8), ("E16_k4_F384", 4), ("E8_k2_skew", 2), ("several_tiles_E4_k2", 2)]
+
+
+@pytest.mark.parametrize("fused_return", [False, True], ids=["return_kernel", "fused_return"])
 @pytest.mark.parametrize("name,G", _cases(), ids=["%s-G%d" % c for c in _cases()])
-def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G):
+def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G, fused_return):
+    if fused_return and (name, G) not in FUSED:
+        pytest.skip("fused return checked on a subset")
     cfg, _ = CASES[name]
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct(dl, shape, G)
+    ranks, xs = run_direct(dl, shape, G, fused_return)
     for ep in ranks:
         assert moe.moe_read_status(ep.ws) == 0
         assert moe.moe_read_status(ep.ws_loc) == 0
@@ -109,13 +120,13 @@ def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G):
 # Full size: the Mixtral-8x7B-shaped layer (T = 512 per rank, H = 4096,
 # F = 14336, E = 8, k = 2) on 2 and 8 ranks, bit for bit against each rank's
 # single-GPU layer (which the full-size parity tests pin to the oracle).
-@pytest.mark.parametrize("G", [2, 8])
-def test_direct_ep_full_size_mixtral_matches_single_gpu(G):
+@pytest.mark.parametrize("G,fused_return", [(2, False), (8, False), (8, True)])
+def test_direct_ep_full_size_mixtral_matches_single_gpu(G, fused_return):
     cfg = synth.CONFIGS[2]
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct(dl, shape, G)
+    ranks, xs = run_direct(dl, shape, G, fused_return)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])
