@@ -1,10 +1,9 @@
 // moe_permute_static: the dispatch step (histogram, scan, stable permutation,
 // gather) for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc at all: code that runs while a stream
-// is being captured in global capture mode (where allocation calls are
-// refused), or a plug-in whose host application owns every device
-// allocation and hands it only the tensors it works on.  Such a caller can
+// Some callers cannot call cudaMalloc at all: a plug-in whose host
+// application owns every device allocation and hands it only the tensors it
+// works on, for instance.  Such a caller can
 // still provide its inputs and outputs, but not the scratch workspace that
 // moe_permute needs.  This entry point takes its scratch from a fixed-size
 // array compiled into the library instead.

@@ -22,9 +22,11 @@
  *   passed as `void *` holding IEEE bfloat16 values.  All matrices are dense
  *   and row-major with the leading dimension equal to the row length.
  * - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  Each
- *   call only enqueues work on it and returns; every call is
- *   stream-ordered, performs no host synchronisation and may be captured in
- *   a CUDA graph.  Grid sizes depend only on the shape and the SM count,
+ *   call only enqueues work on it and returns; every call other than
+ *   moe_read_status and moe_permute_static is stream-ordered, performs no
+ *   host synchronisation and may be captured in a CUDA graph (this header
+ *   states nothing about graphs for moe_permute_static, whose section below
+ *   gives its own rules).  Grid sizes depend only on the shape and the SM count,
  *   never on the routing, so a captured graph stays valid for any input
  *   values of the same shape.
  * - Errors: a bad argument or an unsupported shape returns a non-zero
@@ -270,10 +272,9 @@ MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_stat
 
 /* Dispatch for callers that cannot allocate device memory.  (This entry
  * point has no counterpart on the source pages; it is an interface
- * convenience.)  Some callers cannot call cudaMalloc: code running while a
- * stream is captured in global capture mode, where allocation calls are
- * refused, or a plug-in whose host application owns every device
- * allocation.  moe_permute_static computes exactly what moe_permute computes
+ * convenience.)  Some callers cannot call cudaMalloc: a plug-in whose host
+ * application owns every device allocation, for instance, and hands it only
+ * the tensors it works on.  moe_permute_static computes exactly what moe_permute computes
  * (same arguments, minus `ws`) but takes its scratch from an array of
  * MOE_STATIC_WS_BYTES bytes compiled into the library, which every GPU that
  * loads the library holds until the process exits.
@@ -283,9 +284,9 @@ MOE_API moe_status moe_read_status(void *ws, void *stream, uint32_t *device_stat
  *     scratch is moe_workspace_bytes without the router buffers that large
  *     batches add (it grows with T*k/1024 and E).
  *   - The first call on each device (with that device current) looks up the
- *     array's device address and zero-fills it on `stream`; make that first
- *     call before any stream capture begins.  (A context that was torn
- *     down and recreated gets the same set-up again on its first call.)
+ *     array's device address and zero-fills it on `stream`.  (A context that
+ *     was torn down and recreated gets the same set-up again on its first
+ *     call.)
  *   - All calls share the array and it keeps the last call's contents; each
  *     call clears what must start at zero.  Calls that overlap on the GPU
  *     (other streams, other host threads) race on the array: order them.

@@ -1,6 +1,6 @@
 """moe_permute_static, the dispatch entry point for callers that cannot
-allocate device memory (for example code running inside a stream capture in
-global mode, or a plug-in whose host application owns all device memory).
+allocate device memory (for example a plug-in whose host application owns all
+device memory).
 
 It must give exactly what moe_permute gives with a caller-allocated
 workspace, call after call: the second call below routes different tokens
