@@ -307,6 +307,31 @@ def moe_forward(shape, bufs: dict, ws, stream=None, args: MoeForwardArgs | None 
     _check(load_library().moe_forward(ctypes.byref(shape), ctypes.byref(a), _ptr(ws), _stream(stream)), "moe_forward")
 
 
+class ForwardGraph:
+    """moe_forward on fixed buffers, captured once as a CUDA graph (its launch
+    grid depends only on the shape, so one capture serves any inputs written
+    into the same buffers); replay() enqueues the whole layer on a stream."""
+
+    def __init__(self, shape, bufs: dict, ws, stream=None):
+        import torch
+        self.args = forward_args(bufs)
+        self.keep = (bufs, ws)  # the graph holds their addresses
+        moe_forward(shape, bufs, ws, stream, args=self.args)  # first launches outside the capture
+        self.graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream() if stream is None else stream)
+        with torch.cuda.graph(self.graph, stream=cap):
+            moe_forward(shape, bufs, ws, cap, args=self.args)
+
+    def replay(self, stream=None):
+        import torch
+        if stream is None:
+            self.graph.replay()
+        else:
+            with torch.cuda.stream(stream):
+                self.graph.replay()
+
+
 def moe_read_status(ws, stream=None, clear=True) -> int:
     v = ctypes.c_uint32(0)
     _check(load_library().moe_read_status(_ptr(ws), _stream(stream), ctypes.byref(v), int(bool(clear))),

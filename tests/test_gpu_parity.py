@@ -335,3 +335,27 @@ def test_gemm_wait_expires_and_reports(orc):
     assert_close_bf16(r["out"], o["out"], "out after a GEMM timeout")
 
 
+
+
+def test_forward_graph_replays_with_new_inputs(orc):
+    """moe.ForwardGraph: moe_forward captured once; replays on new tokens
+    written into the same buffers give the eager moe_forward's results bit
+    for bit (the launch grid depends only on the shape)."""
+    cfg = FORWARD_CASES["capped_C7"]
+    L = synth.make_layer(cfg.with_(T=cfg.T * 3))
+    shape = shape_of(cfg)
+    dl = DeviceLayer(L)
+    b = dl.bufs(shape)
+    b["x"] = dl.x[:cfg.T].clone()
+    g = moe.ForwardGraph(shape, b, b["ws"])
+    ref = dl.bufs(shape)
+    for part in (1, 2):
+        xs = dl.x[part * cfg.T:(part + 1) * cfg.T]
+        b["x"].copy_(xs)
+        g.replay()
+        ref["x"] = xs
+        moe.moe_forward(shape, ref, ref["ws"], args=moe.forward_args(ref))
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_host(b["out"]), bf16_host(ref["out"])), part
+        assert torch.equal(b["topk_idx"], ref["topk_idx"])
+    assert moe.moe_read_status(b["ws"]) == 0
