@@ -424,6 +424,7 @@ def alloc_fp8_buffers(shape: MoeShape, per_token=False, device="cuda"):
     dev = torch.device(device)
     xr = T if per_token else P
     return dict(
+        # weight codes tile-blocked (see fp8_weight_codes_plain): [E][N/128][K/128][128][128]
         wg_q=torch.empty((E, F, H), dtype=torch.uint8, device=dev),
         wg_scale=torch.empty((E, F), dtype=torch.float32, device=dev),
         wu_q=torch.empty((E, F, H), dtype=torch.uint8, device=dev),
@@ -520,3 +521,15 @@ def moe_ep_direct_down_return(shape, G, h_loc, w_down, ws_loc, ep_ws, stream=Non
     _check(load_library().moe_ep_direct_down_return(ctypes.byref(shape), int(G), _ptr(h_loc), _ptr(w_down),
                                                     _ptr(ws_loc), _ptr(ep_ws), _stream(stream)),
            "moe_ep_direct_down_return")
+
+
+def fp8_weight_codes_plain(q, N, K):
+    """Host-side view of expert weight codes as moe_quantize_weights_fp8 leaves
+    them (tile-blocked: tiles of 128 output columns x 128 K, each 16 KB
+    contiguous, K-major inside) as a plain [E, N, K] numpy array (code of
+    expert e, output column n, reduction index k).  q: a numpy array or CPU
+    tensor holding the codes of one or more whole experts."""
+    import numpy as np
+    a = np.asarray(q).reshape(-1, N // 128, K // 128, 128, 128)
+    return np.ascontiguousarray(a.transpose(0, 1, 3, 2, 4)).reshape(-1, N, K)
+

@@ -729,11 +729,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_2d(dst + kABox, &tmA0, &full[stage], c * 128 + 64, pl * a.K + kx);
                             }
                     } else if (FP8) {
-                        // one 128-feature x 128-K box of codes per accumulator,
-                        // K-major ([E * n_out][K] bytes)
+                        // one 128-feature x 128-K tile of codes per accumulator,
+                        // 16 KB contiguous (tile-blocked, K-major inside: rows
+                        // of 128 bytes, tile (e, n / 128, k / 128) at row
+                        // ((e * n_out / 128 + n / 128) * K / 128 + k / 128) * 128)
                         uint8_t *sa0 = smem + stage * a_bytes;
-                        tma_load_2d(sa0, &tmA0, &full[stage], kx, U.e * a.n_out + fx0);
-                        if (U.nacc == 2) tma_load_2d(sa0 + kATile, &tmA1, &full[stage], kx, U.e * a.n_out + fx1);
+                        const int nbk = a.n_out / 128, kbk = a.K / 128;
+                        const int trow0 = ((U.e * nbk + fx0 / 128) * kbk + kx / 128) * 128;
+                        tma_load_2d(sa0, &tmA0, &full[stage], 0, trow0);
+                        if (U.nacc == 2)
+                            tma_load_2d(sa0 + kATile, &tmA1, &full[stage], 0,
+                                        ((U.e * nbk + fx1 / 128) * kbk + kx / 128) * 128);
                     } else {
                         uint8_t *sa0 = smem + stage * a_bytes, *sa1 = sa0 + kATile;
                         tma_load_2d(sa0, &tmA0, &full[stage], fx0, ky);
@@ -1308,8 +1314,11 @@ cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *ac
     CUtensorMap tA0, tA1;
     RowMaps tB;
     uint32_t boxes = 0;
-    if (!make_tmap(&tA0, w0, (uint64_t)s.E * n_out, (uint64_t)K, 128, 128, true) ||
-        !make_tmap(&tA1, w1, (uint64_t)s.E * n_out, (uint64_t)K, 128, 128, true))
+    // the tile-blocked codes as rows of 128 bytes (E * n_out * K / 128 rows,
+    // addressed with int32 coordinates)
+    if ((int64_t)s.E * n_out * (K / 128) >= (1ll << 31)) return cudaErrorInvalidValue;
+    if (!make_tmap(&tA0, w0, (uint64_t)s.E * n_out * (K / 128), 128, 128, 128, true) ||
+        !make_tmap(&tA1, w1, (uint64_t)s.E * n_out * (K / 128), 128, 128, 128, true))
         return cudaErrorInvalidValue;
     if (gather) {
         if (!make_tmap(&tB.m[0], act, (uint64_t)s.T, (uint64_t)K, 128, 1, true)) return cudaErrorInvalidValue;

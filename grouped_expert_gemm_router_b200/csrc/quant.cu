@@ -11,8 +11,13 @@
 // are stored with the reduction dimension contiguous (the K-major operand of
 // the MMA); activations get one scale per row.
 //
-// k_quant_weights  w [E][K][N] bf16 -> codes [E][N][K], scales [E][N]
-//                  (one-time preparation of a layer's weights).
+// k_quant_weights  w [E][K][N] bf16 -> codes, scales [E][N] (one-time
+//                  preparation of a layer's weights).  The codes are K-major
+//                  inside tiles of 128 output columns x 128 K, each tile 16 KB
+//                  contiguous: code (e, n, k) at byte
+//                  ((e (N/128) + n/128) (K/128) + k/128) 16384 + (n%128) 128 + k%128,
+//                  so each weight load of the GEMM streams one contiguous
+//                  16 KB tile from HBM.
 // k_quant_rows     rows of a bf16 matrix -> codes + one scale per row: a row
 //                  is held in registers by 32-256 threads (all its loads in
 //                  flight at once), its largest magnitude comes from warp and
@@ -104,10 +109,12 @@ __global__ void __launch_bounds__(256) k_quant_weights(const __nv_bfloat16 *__re
         scale[(size_t)e * N + n0 + tx] = sc.s;
     }
     __syncthreads();
-    // codes [e][n0 + i][k0 + 16 c ...]: thread (i = t / 8, c = t % 8) writes 16 bytes
+    // codes (e, n0 + i, k0 + 16 c ...): thread (i = t / 8, c = t % 8) writes 16
+    // bytes into row (n0 + i) % 128 of tile (e, (n0 + i) / 128, k0 / 128)
     const int i = threadIdx.x >> 3, c = threadIdx.x & 7;
     const Fp8Scale s = s_scale[i];
-    uint8_t *qe = q + ((size_t)e * N + n0 + i) * K;
+    const int n = n0 + i, KB = K / 128;
+    uint8_t *qe = q + ((size_t)e * (N / 128) + n / 128) * (size_t)KB * 16384 + (size_t)(n % 128) * 128;
     for (int k0 = 0; k0 < K; k0 += 128) {
         for (int r = ty; r < 128; r += 8) tile[r][tx] = we[(size_t)(k0 + r) * N + n0 + tx];
         __syncthreads();
@@ -119,7 +126,7 @@ __global__ void __launch_bounds__(256) k_quant_weights(const __nv_bfloat16 *__re
             const uint32_t hi = e4m3x2<false>(__bfloat162float(tile[kk + 2][i]), __bfloat162float(tile[kk + 3][i]), s);
             word[v] = lo | (hi << 16);
         }
-        *reinterpret_cast<uint4 *>(qe + k0 + 16 * c) = make_uint4(word[0], word[1], word[2], word[3]);
+        *reinterpret_cast<uint4 *>(qe + (size_t)(k0 / 128) * 16384 + 16 * c) = make_uint4(word[0], word[1], word[2], word[3]);
         __syncthreads();
     }
 }

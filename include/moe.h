@@ -320,9 +320,14 @@ MOE_API moe_status moe_permute_static(const moe_shape *shape, const void *x, con
  * the tensor cores (tcgen05 kind::f8f6f4, fp32 accumulation) and apply the
  * row and column scales in the epilogue; h and y stay bf16, the combine is
  * the bf16 one.
+ * Weight codes are tile-blocked: for N output columns and reduction length K
+ * (gate/up: N = F, K = H; down: N = H, K = F), the code of expert e, column n,
+ * index k is byte ((e*(N/128) + n/128)*(K/128) + k/128)*16384 + (n%128)*128 +
+ * k%128 -- tiles of 128 columns x 128 K, each 16 KB contiguous and K-major
+ * inside, so each load of the GEMMs streams one contiguous 16 KB tile.
  * ------------------------------------------------------------------------ */
-#define MOE_WEIGHTS_GATE_UP 0 /* w [E,H,F] bf16 -> codes [E,F,H], scales [E,F] */
-#define MOE_WEIGHTS_DOWN 1    /* w [E,F,H] bf16 -> codes [E,H,F], scales [E,H] */
+#define MOE_WEIGHTS_GATE_UP 0 /* w [E,H,F] bf16 -> E*F*H codes (N = F, K = H), scales [E,F] */
+#define MOE_WEIGHTS_DOWN 1    /* w [E,F,H] bf16 -> E*H*F codes (N = H, K = F), scales [E,H] */
 #define MOE_ROWS_X_PERM 0     /* codes [P,H] of x[src_token[r]] (the row copy of step 3; zero codes
                                  with scale 1 where src_token is -1), scales [P] */
 #define MOE_ROWS_TOKENS 1     /* codes [T,H] of every token row of x, scales [T] */

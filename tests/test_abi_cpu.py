@@ -142,3 +142,17 @@ def test_test_hook_flags_are_known(lib):
     for f in (moe.MOE_FLAG_TEST_STALL_SCAN, moe.MOE_FLAG_TEST_STALL_GEMM):
         s = moe.make_shape(64, 128, 256, 8, 2, flags=f)
         assert lib.moe_workspace_bytes(ctypes.byref(s)) > 0
+
+
+def test_fp8_weight_codes_plain_follows_the_tile_layout():
+    """The host view of the tile-blocked fp8 weight codes: the code of expert
+    e, column n, index k sits at the byte the header gives."""
+    import numpy as np
+    E, N, K = 2, 256, 384
+    plain = np.random.default_rng(0).integers(0, 256, (E, N, K)).astype(np.uint8)
+    e, n, k = np.meshgrid(np.arange(E), np.arange(N), np.arange(K), indexing="ij")
+    off = ((e * (N // 128) + n // 128) * (K // 128) + k // 128) * 16384 + (n % 128) * 128 + k % 128
+    blocked = np.zeros(E * N * K, np.uint8)
+    blocked[off.reshape(-1)] = plain.reshape(-1)
+    assert np.array_equal(moe.fp8_weight_codes_plain(blocked, N, K), plain)
+

@@ -77,7 +77,8 @@ def test_fp8_layer_parity(orc, name, per_token):
     # weight codes and scales: bit-exact
     for q, s, rq, rs in (("wg_q", "wg_scale", ref.wg_q, ref.wg_s), ("wu_q", "wu_scale", ref.wu_q, ref.wu_s),
                          ("wd_q", "wd_scale", ref.wd_q, ref.wd_s)):
-        assert np.array_equal(_u8(b[q]), rq), q
+        N, K = (cfg.H, cfg.F) if q == "wd_q" else (cfg.F, cfg.H)
+        assert np.array_equal(moe.fp8_weight_codes_plain(_u8(b[q]), N, K), rq), q
         assert np.array_equal(b[s].cpu().numpy(), rs), s
 
     # routing as the bf16 path (the same kernels): oracle top-k on the GPU logits
@@ -191,9 +192,11 @@ def test_fp8_full_config(orc, cid, alpha):
     for name, wt in (("wg", L.w_gate), ("wu", L.w_up), ("wd", L.w_down)):
         for e in (0,):
             q, s = orc.quantize_weights(wt[e:e + 1])
-            assert np.array_equal(_u8(b[name + "_q"][e]), q[0]), (name, e)
+            N, K = (cfg.H, cfg.F) if name == "wd" else (cfg.F, cfg.H)
+            assert np.array_equal(moe.fp8_weight_codes_plain(_u8(b[name + "_q"][e]), N, K)[0], q[0]), (name, e)
             assert np.array_equal(b[name + "_scale"][e].cpu().numpy(), s[0]), (name, e)
-    wq = {n: _u8(b[n + "_q"]) for n in ("wg", "wu", "wd")}
+    wq = {n: moe.fp8_weight_codes_plain(_u8(b[n + "_q"]), *((cfg.H, cfg.F) if n == "wd" else (cfg.F, cfg.H)))
+          for n in ("wg", "wu", "wd")}
     ws = {n: b[n + "_scale"].cpu().numpy() for n in ("wg", "wu", "wd")}
 
     def deq_w(name, e):
