@@ -183,3 +183,53 @@ def oracle_layer(orc, L, cfg, logits_gpu):
         y[r] = orc.down_row(h[r], L.w_down[e])
     out = orc.combine(y, d["dest_row"], w)
     return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)
+
+
+def run_cap_and_spill_ep(dl, shape, G):
+    """The two-pass expert-parallel layer on G ranks held by this process;
+    rank r holds tokens [r T, (r+1) T) of the layer dl."""
+    from grouped_expert_gemm_router_b200.ep import CapAndSpillEP, exchange_in_process
+    T, Eg = shape.T, shape.E // G
+    ranks = [CapAndSpillEP(shape, G) for _ in range(G)]
+    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
+    for r, ep in enumerate(ranks):
+        ep.route_and_pack(xs[r], dl.w_router, dl.bias)
+    exchange_in_process(ranks, "exchange_in")
+    for r, ep in enumerate(ranks):
+        sl = slice(r * Eg, (r + 1) * Eg)
+        ep.local_experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+    exchange_in_process(ranks, "exchange_out")
+    for ep in ranks:
+        ep.finish()
+    torch.cuda.synchronize()
+    return ranks, xs
+
+
+def run_direct_ep(dl, shape, G, fused_return=False):
+    """The peer-store expert-parallel layer on G ranks held by this process
+    (fused_return: the down GEMM stores its results into the owners' y)."""
+    from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
+    T, Eg = shape.T, shape.E // G
+    ranks = [DirectEP(shape, G, r) for r in range(G)]
+    connect_in_process(ranks)
+    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
+    for r, ep in enumerate(ranks):
+        ep.route(xs[r], dl.w_router, dl.bias)
+    gather_counts_in_process(ranks)
+    for ep in ranks:
+        ep.plan()
+    for r, ep in enumerate(ranks):
+        ep.dispatch(xs[r])
+    for r, ep in enumerate(ranks):
+        sl = slice(r * Eg, (r + 1) * Eg)
+        if fused_return:
+            ep.experts_and_return(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+        else:
+            ep.experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
+    if not fused_return:
+        for ep in ranks:
+            ep.send_back()
+    for ep in ranks:
+        ep.finish()
+    torch.cuda.synchronize()
+    return ranks, xs

@@ -19,8 +19,8 @@ import torch
 
 import grouped_expert_gemm_router_b200 as moe
 import synth
-from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer
-from grouped_expert_gemm_router_b200.ep import CapAndSpillEP, exchange_in_process
+from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer, run_cap_and_spill_ep
+from grouped_expert_gemm_router_b200.ep import CapAndSpillEP
 
 pytestmark = pytest.mark.gpu
 
@@ -43,24 +43,6 @@ def _cases():
 
 def _shape(cfg):
     return moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=True)
-
-
-def _run_ep(dl, shape, G):
-    """The layer on G emulated ranks; rank r holds tokens [r T, (r+1) T)."""
-    T, Eg = shape.T, shape.E // G
-    ranks = [CapAndSpillEP(shape, G) for _ in range(G)]
-    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
-    for r, ep in enumerate(ranks):
-        ep.route_and_pack(xs[r], dl.w_router, dl.bias)
-    exchange_in_process(ranks, "exchange_in")
-    for r, ep in enumerate(ranks):
-        sl = slice(r * Eg, (r + 1) * Eg)
-        ep.local_experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
-    exchange_in_process(ranks, "exchange_out")
-    for ep in ranks:
-        ep.finish()
-    torch.cuda.synchronize()
-    return ranks, xs
 
 
 def _single_gpu(dl, shape, x):
@@ -98,7 +80,7 @@ def test_ep_layer_matches_single_gpu_and_oracle(orc, name, G):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = _run_ep(dl, shape, G)
+    ranks, xs = run_cap_and_spill_ep(dl, shape, G)
     for ep in ranks:
         assert moe.moe_read_status(ep.ws) == 0
         assert moe.moe_read_status(ep.ws_loc) == 0
@@ -124,7 +106,7 @@ def test_ep_full_size_decode_matches_single_gpu(G):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = _run_ep(dl, shape, G)
+    ranks, xs = run_cap_and_spill_ep(dl, shape, G)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])

@@ -16,7 +16,7 @@ import torch
 
 import grouped_expert_gemm_router_b200 as moe
 import synth
-from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer
+from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer, run_direct_ep
 from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
 
 pytestmark = pytest.mark.gpu
@@ -36,35 +36,6 @@ def _cases():
 
 def _shape(cfg):
     return moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
-
-
-def run_direct(dl, shape, G, fused_return=False):
-    """The layer on G emulated ranks; rank r holds tokens [r T, (r+1) T).
-    fused_return: the down GEMM stores its results into the owners' y."""
-    T, Eg = shape.T, shape.E // G
-    ranks = [DirectEP(shape, G, r) for r in range(G)]
-    connect_in_process(ranks)
-    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
-    for r, ep in enumerate(ranks):
-        ep.route(xs[r], dl.w_router, dl.bias)
-    gather_counts_in_process(ranks)
-    for ep in ranks:
-        ep.plan()
-    for r, ep in enumerate(ranks):
-        ep.dispatch(xs[r])
-    for r, ep in enumerate(ranks):
-        sl = slice(r * Eg, (r + 1) * Eg)
-        if fused_return:
-            ep.experts_and_return(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
-        else:
-            ep.experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
-    if not fused_return:
-        for ep in ranks:
-            ep.send_back()
-    for ep in ranks:
-        ep.finish()
-    torch.cuda.synchronize()
-    return ranks, xs
 
 
 def _single_gpu(dl, shape, x):
@@ -102,7 +73,7 @@ def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G, fused_return):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct(dl, shape, G, fused_return)
+    ranks, xs = run_direct_ep(dl, shape, G, fused_return)
     for ep in ranks:
         assert moe.moe_read_status(ep.ws) == 0
         assert moe.moe_read_status(ep.ws_loc) == 0
@@ -126,7 +97,7 @@ def test_direct_ep_full_size_mixtral_matches_single_gpu(G, fused_return):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct(dl, shape, G, fused_return)
+    ranks, xs = run_direct_ep(dl, shape, G, fused_return)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])
@@ -159,7 +130,7 @@ def test_direct_ep_clamps_counts_beyond_the_buffers():
     assert all(moe.moe_read_status(ep.ws_loc) & moe.MOE_DEV_BAD_ROW for ep in ranks)
     for ep in ranks:
         moe.moe_read_status(ep.ws)  # clear
-    ranks2, xs = run_direct(dl, shape, G)
+    ranks2, xs = run_direct_ep(dl, shape, G)
     for r, ep in enumerate(ranks2):
         assert moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])
