@@ -545,14 +545,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // next unit's MMAs) when they give each CTA fewer operand bytes to
         // load -- rounds x (weight columns + token rows) per K row -- else
         // 256-feature units, which read each token tile once for two
-        // accumulators.  With e4m3 operands and full tiles (192 or more rows
-        // per tile on average) also 128-feature units: the 8-bit mainloop of a
-        // full tile is short enough for its epilogue to set the pace otherwise.
+        // accumulators (also with e4m3 operands: 128-feature units for full
+        // tiles measured 13% slower on the 8192-token prefill).
         const int grid = (int)gridDim.x;
         const int tr = *a.tile_rows;
         const int r256 = (nt * a.num_fb + grid - 1) / grid, r128 = (nt * (a.n_out / 128) + grid - 1) / grid;
-        const bool full_tiles = (int64_t)a.P >= (int64_t)192 * nt;
-        if (MODE == 1 && ((FP8 && full_tiles) || r128 * (128 + tr) < r256 * (256 + tr))) {
+        if (MODE == 1 && r128 * (128 + tr) < r256 * (256 + tr)) {
             num_fb = a.n_out / 128;
             fbw = 128;
         }
