@@ -140,11 +140,15 @@ __global__ void __launch_bounds__(256) k_quant_weights(const __nv_bfloat16 *__re
 // from a warp reduction and, for TPR > 32, a reduction over the row's warps in
 // shared memory; the codes are written from the registers with streaming
 // stores (the codes are read once, by the GEMM).
-template <int TPR, int VPT>
+template <int TPR, int VPT, int RPG>
 __global__ void __launch_bounds__(256) k_quant_rows(const uint4 *__restrict__ src, const int *__restrict__ idx,
                                                     int gather, uint2 *__restrict__ q, float *__restrict__ scale,
                                                     int K8, int src_rows, int P, int fixed_rows, int cap_rows,
                                                     const int *total_spill) {
+    // RPG rows per thread group and iteration (all their loads in flight
+    // before the first reduction; rows of a few vectors per thread are
+    // otherwise bound by one load latency per row)
+    static_assert(RPG == 1 || TPR == 32, "several rows per group only for one-warp rows");
     constexpr int kRowsPerBlock = 256 / TPR, kWarpsPerRow = TPR / 32;
     __shared__ float s_max[8];
     pdl_trigger();
@@ -155,53 +159,67 @@ __global__ void __launch_bounds__(256) k_quant_rows(const uint4 *__restrict__ sr
     const int g = threadIdx.x / TPR, tr = threadIdx.x % TPR;
     // every thread of the block runs the same number of iterations (the
     // shared-memory reduction below needs the whole block)
-    for (int base = blockIdx.x * kRowsPerBlock; base < rows; base += gridDim.x * kRowsPerBlock) {
-        const int row = base + g;
-        bool active = row < rows;
-        int sr = row;
-        if (active && idx) {
-            const int t = idx[row];
-            if (!gather && t < 0) active = false;
-            if (gather) sr = t;
+    for (int base = blockIdx.x * kRowsPerBlock * RPG; base < rows; base += gridDim.x * kRowsPerBlock * RPG) {
+        int row[RPG];
+        bool active[RPG], valid[RPG];
+        uint4 v[RPG][VPT];
+        float m[RPG];
+#pragma unroll
+        for (int j = 0; j < RPG; ++j) {
+            row[j] = base + j * kRowsPerBlock + g;
+            active[j] = row[j] < rows;
+            int sr = row[j];
+            if (active[j] && idx) {
+                const int t = idx[row[j]];
+                if (!gather && t < 0) active[j] = false;
+                if (gather) sr = t;
+            }
+            valid[j] = active[j] && (unsigned)sr < (unsigned)src_rows;
+            if (valid[j]) {
+                const uint4 *s_row = src + (size_t)sr * K8;
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) {
+                    const int c = tr + i * TPR;
+                    v[j][i] = c < K8 ? __ldg(s_row + c) : make_uint4(0, 0, 0, 0);
+                }
+            }
         }
-        const bool valid = active && (unsigned)sr < (unsigned)src_rows;
-        uint4 v[VPT];
-        float m = 0.0f;
-        if (valid) {
-            const uint4 *s_row = src + (size_t)sr * K8;
+#pragma unroll
+        for (int j = 0; j < RPG; ++j) {
+            m[j] = 0.0f;
+            if (valid[j]) {
+                __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) m2 = amax8(v[j][i], m2);
+                m[j] = amax_of(m2);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+        }
+        if (kWarpsPerRow > 1) {
+            if (lane == 0) s_max[warp] = m[0];
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < kWarpsPerRow; ++w) m[0] = fmaxf(m[0], s_max[g * kWarpsPerRow + w]);
+            __syncthreads();
+        }
+#pragma unroll
+        for (int j = 0; j < RPG; ++j) {
+            if (!active[j]) continue;
+            uint2 *dst = q + (size_t)row[j] * K8;
+            if (!valid[j]) {
+                for (int c = tr; c < K8; c += TPR) dst[c] = make_uint2(0, 0);
+                if (tr == 0) scale[row[j]] = 1.0f;
+                continue;
+            }
+            const Fp8Scale sc = fp8_scale(m[j]);
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int c = tr + i * TPR;
-                v[i] = c < K8 ? __ldg(s_row + c) : make_uint4(0, 0, 0, 0);
+                if (c < K8) __stcs(dst + c, quant8(v[j][i], sc));
             }
-            __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) m2 = amax8(v[i], m2);
-            m = amax_of(m2);
+            if (tr == 0) scale[row[j]] = sc.s;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (kWarpsPerRow > 1) {
-            if (lane == 0) s_max[warp] = m;
-            __syncthreads();
-#pragma unroll
-            for (int w = 0; w < kWarpsPerRow; ++w) m = fmaxf(m, s_max[g * kWarpsPerRow + w]);
-            __syncthreads();
-        }
-        if (!active) continue;
-        uint2 *dst = q + (size_t)row * K8;
-        if (!valid) {
-            for (int c = tr; c < K8; c += TPR) dst[c] = make_uint2(0, 0);
-            if (tr == 0) scale[row] = 1.0f;
-            continue;
-        }
-        const Fp8Scale sc = fp8_scale(m);
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int c = tr + i * TPR;
-            if (c < K8) __stcs(dst + c, quant8(v[i], sc));
-        }
-        if (tr == 0) scale[row] = sc.s;
     }
 }
 
@@ -257,14 +275,15 @@ cudaError_t launch_rows(const uint4 *src, const int *idx, int gather, uint2 *q, 
     const int cap = num_sms * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-#define MOE_QROWS(T, V)                                                                                        \
-    return launch_pdl(k_quant_rows<T, V>, dim3(blocks), dim3(256), 0, stream, src, idx, gather, q, scale, K8, src_rows, \
-                      P, fixed_rows, cap_rows, total_spill)
-    if (K8 <= 32 * 8) MOE_QROWS(32, 8);
-    if (K8 <= 64 * 8) MOE_QROWS(64, 8);
-    if (K8 <= 128 * 8) MOE_QROWS(128, 8);
-    if (K8 <= 256 * 8) MOE_QROWS(256, 8);
-    if (K8 <= 256 * 16) MOE_QROWS(256, 16);
+#define MOE_QROWS(T, V, R)                                                                                  \
+    return launch_pdl(k_quant_rows<T, V, R>, dim3(blocks), dim3(256), 0, stream, src, idx, gather, q, scale, K8,    \
+                      src_rows, P, fixed_rows, cap_rows, total_spill)
+    if (K8 <= 32 * 4) MOE_QROWS(32, 4, 2);  // short rows: two rows per warp in flight
+    if (K8 <= 32 * 8) MOE_QROWS(32, 8, 1);
+    if (K8 <= 64 * 8) MOE_QROWS(64, 8, 1);
+    if (K8 <= 128 * 8) MOE_QROWS(128, 8, 1);
+    if (K8 <= 256 * 8) MOE_QROWS(256, 8, 1);
+    if (K8 <= 256 * 16) MOE_QROWS(256, 16, 1);
 #undef MOE_QROWS
     return launch_pdl(k_quant_rows_long, dim3(blocks), dim3(256), 0, stream, src, idx, gather, q, scale, K8, src_rows,
                       P, fixed_rows, cap_rows, total_spill);
