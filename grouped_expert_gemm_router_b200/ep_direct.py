@@ -136,6 +136,8 @@ class DirectEP:
         x_loc = symm_mem.empty((Tloc, shape.H), dtype=torch.bfloat16, device=dev)
         y = symm_mem.empty((P, shape.H), dtype=torch.bfloat16, device=dev)
         gname = (group if group is not None else dist.group.WORLD).group_name
+        if hasattr(symm_mem, "enable_symm_mem_for_group"):  # required before rendezvous by some versions
+            symm_mem.enable_symm_mem_for_group(gname)
         hx, hy = symm_mem.rendezvous(x_loc, gname), symm_mem.rendezvous(y, gname)
         ep = cls(shape, G, rank, dev, x_loc=x_loc, y=y)
         ep.set_peers(hx.buffer_ptrs, hy.buffer_ptrs)
