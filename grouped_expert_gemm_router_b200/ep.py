@@ -138,9 +138,13 @@ class CapAndSpillEP:
     def forward(self, x, w_router, bias, w_gate, w_up, w_down, group=None):
         """One layer on this rank (every rank of `group` calls it; G must be
         the group's size).  Returns this rank's out [T, H]."""
+        import torch
         import torch.distributed as dist
 
         def a2a(out, inp):
+            # bf16 rows as their bytes (same splits; any backend moves bytes)
+            if out.dtype == torch.bfloat16:
+                out, inp = out.view(torch.uint8), inp.view(torch.uint8)
             dist.all_to_all_single(out, inp, group=group)
 
         self.route_and_pack(x, w_router, bias)
