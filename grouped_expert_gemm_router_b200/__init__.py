@@ -41,7 +41,8 @@ ABI_FUNCTIONS = (
     "moe_grouped_down_combine", "moe_grouped_down_fp8_combine", "moe_ep_overflow_rows", "moe_ep_workspace_bytes",
     "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
-    "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return",
+    "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
+    "moe_ep_direct_down_return_fp8",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -174,6 +175,10 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_direct_return.restype = st
     lib.moe_ep_direct_down_return.argtypes = [sp, i32] + [vp] * 5
     lib.moe_ep_direct_down_return.restype = st
+    lib.moe_ep_direct_dispatch_fp8.argtypes = [sp, i32] + [vp] * 10
+    lib.moe_ep_direct_dispatch_fp8.restype = st
+    lib.moe_ep_direct_down_return_fp8.argtypes = [sp, i32] + [vp] * 7
+    lib.moe_ep_direct_down_return_fp8.restype = st
     _lib = lib
     return lib
 
@@ -532,4 +537,18 @@ def fp8_weight_codes_plain(q, N, K):
     import numpy as np
     a = np.asarray(q).reshape(-1, N // 128, K // 128, 128, 128)
     return np.ascontiguousarray(a.transpose(0, 1, 3, 2, 4)).reshape(-1, N, K)
+
+
+def moe_ep_direct_dispatch_fp8(shape, G, x_q, x_scale, topk_idx, dest_row, expert_offsets, peer_x_loc_q,
+                               peer_scale_loc, ws, ep_ws, stream=None):
+    _check(load_library().moe_ep_direct_dispatch_fp8(ctypes.byref(shape), int(G), _ptr(x_q), _ptr(x_scale),
+                                                     _ptr(topk_idx), _ptr(dest_row), _ptr(expert_offsets),
+                                                     _ptr(peer_x_loc_q), _ptr(peer_scale_loc), _ptr(ws), _ptr(ep_ws),
+                                                     _stream(stream)), "moe_ep_direct_dispatch_fp8")
+
+
+def moe_ep_direct_down_return_fp8(shape, G, h_q, h_scale, wd_q, wd_scale, ws_loc, ep_ws, stream=None):
+    _check(load_library().moe_ep_direct_down_return_fp8(ctypes.byref(shape), int(G), _ptr(h_q), _ptr(h_scale),
+                                                        _ptr(wd_q), _ptr(wd_scale), _ptr(ws_loc), _ptr(ep_ws),
+                                                        _stream(stream)), "moe_ep_direct_down_return_fp8")
 

@@ -161,12 +161,16 @@ __global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) 
 }
 
 // Source side: pair i = t k + j of expert e goes to row send_base[e] +
-// (dest_row[i] - offsets[e]) of rank e / E_g's x_loc.
+// (dest_row[i] - offsets[e]) of rank e / E_g's x_loc.  Rows of H8 16-byte
+// vectors (bf16 rows, or e4m3 code rows); with x_scale, the row's scale goes
+// to the same row of the rank's scale array (peer_scale).
 __global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(const uint4 *x, const int32_t *topk_idx,
                                                                 const int32_t *dest_row, const int32_t *offsets,
                                                                 const int32_t *send_base, const int32_t *send_cnt,
                                                                 const unsigned long long *peer_x_loc, int R, int k,
-                                                                int E, int Eg, int Tloc, int H8, uint32_t *status) {
+                                                                int E, int Eg, int Tloc, int H8, uint32_t *status,
+                                                                const float *x_scale,
+                                                                const unsigned long long *peer_scale) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -182,6 +186,7 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(const uint4 *x, c
         }
         uint4 *dst = reinterpret_cast<uint4 *>(peer_x_loc[e / Eg]) + (size_t)pos * H8;
         copy_row16(x + (size_t)(i / k) * H8, dst, H8, lane);
+        if (x_scale && lane == 0) reinterpret_cast<float *>(peer_scale[e / Eg])[pos] = x_scale[i / k];
     }
     if (bad && lane == 0) atomicOr(status, MOE_DEV_BAD_ROW);
     __threadfence_system();
@@ -302,15 +307,18 @@ cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int
     return launch_pdl(k_ep_direct_plan, dim3(1), dim3(kScanThreads), 0, stream, a);
 }
 
+// x: bf16 rows (x_scale null), or e4m3 code rows with their scales.
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
                                  const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
-                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream) {
+                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream,
+                                 const float *x_scale, const void *peer_scale) {
     const DirWs p = dir_ptrs(ep_ws, s, G);
     const int64_t R = (int64_t)s.T * s.k;
     return launch_pdl(k_ep_direct_put, dim3(dir_grid(R, num_sms)), dim3(kDirThreads), 0, stream, (const uint4 *)x,
                       topk_idx, dest_row, offsets, (const int32_t *)p.send_base, (const int32_t *)p.send_cnt,
                       (const unsigned long long *)peer_x_loc, (int)R, s.k, s.E, s.E / G,
-                      (int)ep_direct_local_rows(s, G), s.H / 8, status);
+                      (int)ep_direct_local_rows(s, G), x_scale ? s.H / 16 : s.H / 8, status, x_scale,
+                      (const unsigned long long *)peer_scale);
 }
 
 cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,

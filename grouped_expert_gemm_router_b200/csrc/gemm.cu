@@ -1303,7 +1303,7 @@ cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *ac
                                     const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
                                     void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
                                     cudaStream_t stream, const int32_t *src_token, const CombineOut *comb,
-                                const unsigned long long *row_addr) {
+                                    const unsigned long long *row_addr) {
     const bool gather = mode == 0 && src_token != nullptr;
     const bool capped = (s.flags & MOE_FLAG_CAPACITY) != 0;
     const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, capped);
@@ -1345,6 +1345,7 @@ cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *ac
     a.w_scale0 = w0_scale;
     a.w_scale1 = w1_scale;
     a.row_scale = row_scale;
+    a.row_addr = (mode == 1 && !comb) ? row_addr : nullptr;
     static bool attr_done[4] = {false, false, false, false};
     cudaError_t err;
     auto setup = [&](const void *fn, int i) -> cudaError_t {

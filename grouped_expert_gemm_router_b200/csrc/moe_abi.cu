@@ -30,7 +30,7 @@ cudaError_t launch_grouped_gemm_fp8(int mode, const moe_shape &s, const void *ac
                                     const void *w0, const float *w0_scale, const void *w1, const float *w1_scale,
                                     void *out, const WsLayout &L, void *ws, uint64_t timeout_ns, int num_sms,
                                     cudaStream_t stream, const int32_t *src_token, const CombineOut *comb = nullptr,
-                                const unsigned long long *row_addr = nullptr);
+                                    const unsigned long long *row_addr = nullptr);
 cudaError_t launch_quant_weights(int E, int K, int N, const void *w, void *q, float *scale, cudaStream_t stream);
 cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int src_rows, const int32_t *idx,
                               bool gather, void *q, float *scale, const WsLayout &L, void *ws, int num_sms,
@@ -56,7 +56,8 @@ cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int
 const unsigned long long *ep_direct_row_addr(void *ep_ws, const moe_shape &s, int G);
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
                                  const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
-                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream);
+                                 void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream,
+                                 const float *x_scale = nullptr, const void *peer_scale = nullptr);
 cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,
                                     int num_sms, cudaStream_t stream);
 }  // namespace moe
@@ -382,7 +383,8 @@ moe_status moe_quantize_rows_fp8(const moe_shape *s, int which, const void *src,
     if (st != MOE_OK) return st;
     if (which != MOE_ROWS_X_PERM && which != MOE_ROWS_TOKENS && which != MOE_ROWS_H) return MOE_ERR_INVALID_ARG;
     if (!aligned(src, 16) || !aligned(q, 16) || !aligned(scale, 4)) return MOE_ERR_INVALID_ARG;
-    if (which != MOE_ROWS_TOKENS && !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
+    if (which == MOE_ROWS_X_PERM && !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
+    if (which == MOE_ROWS_H && src_token && !aligned(src_token, 4)) return MOE_ERR_INVALID_ARG;
     if (which != MOE_ROWS_TOKENS && (st = check_ws(ws)) != MOE_OK) return st;
     int sms = 0;
     if ((st = device_info(&sms)) != MOE_OK) return st;
@@ -707,5 +709,43 @@ moe_status moe_ep_direct_down_return(const moe_shape *s, int32_t G, const void *
     cudaError_t e = launch_grouped_gemm(1, l, h_loc, w_down, w_down, nullptr, Lloc, ws_loc, g_timeout_ns.load(), sms,
                                         (cudaStream_t)stream, nullptr, nullptr, ep_direct_row_addr(ep_ws, *s, G));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_down_return");
+}
+
+moe_status moe_ep_direct_dispatch_fp8(const moe_shape *s, int32_t G, const void *x_q, const float *x_scale,
+                                      const int32_t *topk_idx, const int32_t *dest_row, const int32_t *expert_offsets,
+                                      const void *peer_x_loc_q, const void *peer_scale_loc, void *ws, void *ep_ws,
+                                      void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(x_q, 16) || !aligned(x_scale, 4) || !aligned(topk_idx, 4) || !aligned(dest_row, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(peer_x_loc_q, 8) || !aligned(peer_scale_loc, 8) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    uint32_t *status = (uint32_t *)((char *)ws + L.status);
+    cudaError_t e = launch_ep_direct_put(*s, G, x_q, topk_idx, dest_row, expert_offsets, peer_x_loc_q, ep_ws, status,
+                                         sms, (cudaStream_t)stream, x_scale, peer_scale_loc);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_dispatch_fp8");
+}
+
+moe_status moe_ep_direct_down_return_fp8(const moe_shape *s, int32_t G, const void *h_q, const float *h_scale,
+                                         const void *wd_q, const float *wd_scale, void *ws_loc, void *ep_ws,
+                                         void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(h_q, 16) || !aligned(h_scale, 4) || !aligned(wd_q, 16) || !aligned(wd_scale, 4) ||
+        !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws_loc)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const moe_shape l = ep_direct_local(s, G);
+    const WsLayout Lloc = layout_of(&l);
+    cudaError_t e = launch_grouped_gemm_fp8(1, l, h_q, h_scale, wd_q, wd_scale, wd_q, wd_scale, nullptr, Lloc, ws_loc,
+                                            g_timeout_ns.load(), sms, (cudaStream_t)stream, nullptr, nullptr,
+                                            ep_direct_row_addr(ep_ws, *s, G));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_down_return_fp8");
 }
 

@@ -31,7 +31,8 @@ class DirectEP:
              can store into them); allocated here otherwise.
     """
 
-    def __init__(self, shape, G: int, rank: int, device="cuda", x_loc=None, y=None):
+    def __init__(self, shape, G: int, rank: int, device="cuda", x_loc=None, y=None, fp8=False, x_loc_q=None,
+                 scale_loc=None):
         import torch
         if shape.flags & moe.MOE_FLAG_CAPACITY:
             raise moe.MoeError("the peer-store layer uses the uncapped layout")
@@ -56,6 +57,17 @@ class DirectEP:
             raise moe.MoeError("x_loc must be [%d, %d] and y [%d, %d]" % (self.Tloc, H, P, H))
         self.h_loc = e((self.Tloc, shape.F), dtype=bf16, device=dev)
         self.y_loc = e((self.Tloc, H), dtype=bf16, device=dev)
+        self.fp8 = bool(fp8)
+        if self.fp8:  # e4m3 rows on the links: token codes + scales, received codes + scales, h codes
+            u8 = torch.uint8
+            self.x_q = e((T, H), dtype=u8, device=dev)
+            self.x_scale = e((T,), dtype=f32, device=dev)
+            self.x_loc_q = x_loc_q if x_loc_q is not None else e((self.Tloc, H), dtype=u8, device=dev)
+            self.scale_loc = scale_loc if scale_loc is not None else e((self.Tloc,), dtype=f32, device=dev)
+            self.h_q = e((self.Tloc, shape.F), dtype=u8, device=dev)
+            self.h_scale = e((self.Tloc,), dtype=f32, device=dev)
+            self.peer_x_loc_q = torch.zeros((G,), dtype=torch.int64, device=dev)
+            self.peer_scale_loc = torch.zeros((G,), dtype=torch.int64, device=dev)
         self.cnt_all = e((G, E), dtype=i32, device=dev)
         self.peer_x_loc = torch.zeros((G,), dtype=torch.int64, device=dev)
         self.peer_y = torch.zeros((G,), dtype=torch.int64, device=dev)
@@ -67,11 +79,19 @@ class DirectEP:
             moe.moe_workspace_init(shape, self.ws)
             moe.moe_workspace_init(self.local, self.ws_loc)
 
-    def set_peers(self, x_loc_addrs, y_addrs):
-        """Rank d's x_loc and y addresses as this rank's kernels reach them."""
+    def set_peers(self, x_loc_addrs, y_addrs, x_loc_q_addrs=None, scale_loc_addrs=None):
+        """Rank d's x_loc and y (and, fp8, x_loc_q and scale_loc) addresses as
+        this rank's kernels reach them."""
         import torch
-        self.peer_x_loc.copy_(torch.tensor([int(a) for a in x_loc_addrs], dtype=torch.int64))
-        self.peer_y.copy_(torch.tensor([int(a) for a in y_addrs], dtype=torch.int64))
+
+        def put(table, addrs):
+            table.copy_(torch.tensor([int(a) for a in addrs], dtype=torch.int64))
+
+        put(self.peer_x_loc, x_loc_addrs)
+        put(self.peer_y, y_addrs)
+        if self.fp8:
+            put(self.peer_x_loc_q, x_loc_q_addrs)
+            put(self.peer_scale_loc, scale_loc_addrs)
 
     # ---- phases -------------------------------------------------------------
     def route(self, x, w_router, bias, stream=None):
@@ -95,6 +115,31 @@ class DirectEP:
         b = self.b
         moe.moe_ep_direct_dispatch(self.shape, self.G, x, b["topk_idx"], b["dest_row"], b["expert_offsets"],
                                    self.peer_x_loc, self.ws, self.ep_ws, stream)
+
+    # ---- fp8: e4m3 rows on the links, fp8 GEMMs on the local experts -------------
+    def quantize_tokens(self, x, stream=None):
+        """This rank's token rows as e4m3 codes with one scale per row."""
+        moe.moe_quantize_rows_fp8(self.shape, moe.MOE_ROWS_TOKENS, x, None, self.x_q, self.x_scale, self.ws, stream)
+
+    def dispatch_fp8(self, stream=None):
+        """Each routed token's code row and scale into its expert's rank's
+        x_loc_q and scale_loc (peer stores)."""
+        b = self.b
+        moe.moe_ep_direct_dispatch_fp8(self.shape, self.G, self.x_q, self.x_scale, b["topk_idx"], b["dest_row"],
+                                       b["expert_offsets"], self.peer_x_loc_q, self.peer_scale_loc, self.ws,
+                                       self.ep_ws, stream)
+
+    def experts_fp8_and_return(self, wg_q, wg_scale, wu_q, wu_scale, wd_q, wd_scale, stream=None):
+        """The fp8 SwiGLU GEMM on the received code rows, h quantized per row,
+        then the fp8 down projection storing each result row straight into
+        its token's rank's y (weights: the rank's slices of the codes and
+        scales moe_quantize_weights_fp8 leaves)."""
+        L = self.local
+        moe.moe_grouped_swiglu_fp8(L, self.x_loc_q, self.scale_loc, None, wg_q, wg_scale, wu_q, wu_scale, self.h_loc,
+                                   self.ws_loc, stream)
+        moe.moe_quantize_rows_fp8(L, moe.MOE_ROWS_H, self.h_loc, None, self.h_q, self.h_scale, self.ws_loc, stream)
+        moe.moe_ep_direct_down_return_fp8(self.shape, self.G, self.h_q, self.h_scale, wd_q, wd_scale, self.ws_loc,
+                                          self.ep_ws, stream)
 
     def experts(self, w_gate, w_up, w_down, stream=None):
         """The grouped GEMMs of this rank's experts on the rows it received."""
@@ -122,9 +167,10 @@ class DirectEP:
 
     # ---- the layer on a process group ------------------------------------------
     @classmethod
-    def on_process_group(cls, shape, group=None, device=None):
-        """One rank per process of `group` (NCCL), x_loc and y in symmetric
-        memory so that every rank can store into every other rank's."""
+    def on_process_group(cls, shape, group=None, device=None, fp8=False):
+        """One rank per process of `group` (NCCL), x_loc and y (fp8: also
+        x_loc_q and scale_loc) in symmetric memory so that every rank can store
+        into every other rank's."""
         import torch
         import torch.distributed as dist
         import torch.distributed._symmetric_memory as symm_mem
@@ -139,9 +185,15 @@ class DirectEP:
         if hasattr(symm_mem, "enable_symm_mem_for_group"):  # required before rendezvous by some versions
             symm_mem.enable_symm_mem_for_group(gname)
         hx, hy = symm_mem.rendezvous(x_loc, gname), symm_mem.rendezvous(y, gname)
-        ep = cls(shape, G, rank, dev, x_loc=x_loc, y=y)
-        ep.set_peers(hx.buffer_ptrs, hy.buffer_ptrs)
-        ep._handles = (hx, hy)  # keep the mappings alive
+        handles, xq, sc = [hx, hy], None, None
+        if fp8:
+            xq = symm_mem.empty((Tloc, shape.H), dtype=torch.uint8, device=dev)
+            sc = symm_mem.empty((Tloc,), dtype=torch.float32, device=dev)
+            handles += [symm_mem.rendezvous(xq, gname), symm_mem.rendezvous(sc, gname)]
+        ep = cls(shape, G, rank, dev, x_loc=x_loc, y=y, fp8=fp8, x_loc_q=xq, scale_loc=sc)
+        ep.set_peers(hx.buffer_ptrs, hy.buffer_ptrs, handles[2].buffer_ptrs if fp8 else None,
+                     handles[3].buffer_ptrs if fp8 else None)
+        ep._handles = handles  # keep the mappings alive
         ep._flag = torch.zeros((1,), dtype=torch.int32, device=dev)
         ep._group = group
         return ep
@@ -170,13 +222,34 @@ class DirectEP:
         return self.finish()
 
 
+    def forward_fp8(self, x, w_router, bias, wg_q, wg_scale, wu_q, wu_scale, wd_q, wd_scale):
+        """One layer of the fp8 form on this rank (e4m3 rows on the links;
+        every rank of the group calls it)."""
+        import torch.distributed as dist
+        group = self._group
+
+        def barrier():
+            dist.all_reduce(self._flag, group=group)
+
+        self.route(x, w_router, bias)
+        self.quantize_tokens(x)
+        self.gather_counts(lambda out, inp: dist.all_gather_into_tensor(out, inp, group=group))
+        self.plan()
+        self.dispatch_fp8()
+        barrier()
+        self.experts_fp8_and_return(wg_q, wg_scale, wu_q, wu_scale, wd_q, wd_scale)
+        barrier()
+        return self.finish()
+
 def connect_in_process(ranks) -> None:
     """Several ranks held by one process on one device: each rank's peer
-    tables point at the other ranks' own x_loc and y."""
+    tables point at the other ranks' own x_loc and y (and x_loc_q, scale_loc)."""
     xs = [r.x_loc.data_ptr() for r in ranks]
     ys = [r.b["y"].data_ptr() for r in ranks]
+    xq = [r.x_loc_q.data_ptr() for r in ranks] if ranks[0].fp8 else None
+    sc = [r.scale_loc.data_ptr() for r in ranks] if ranks[0].fp8 else None
     for r in ranks:
-        r.set_peers(xs, ys)
+        r.set_peers(xs, ys, xq, sc)
 
 
 def gather_counts_in_process(ranks) -> None:

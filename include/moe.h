@@ -332,7 +332,7 @@ MOE_API moe_status moe_permute_static(const moe_shape *shape, const void *x, con
                                  with scale 1 where src_token is -1), scales [P] */
 #define MOE_ROWS_TOKENS 1     /* codes [T,H] of every token row of x, scales [T] */
 #define MOE_ROWS_H 2          /* codes [P,F] of h[r] for every filled row r (src_token[r] >= 0; the
-                                 other rows are left unwritten), scales [P] */
+                                 other rows are left unwritten; src_token null: every row), scales [P] */
 
 /* One-time preparation of expert weights: `which` = MOE_WEIGHTS_GATE_UP (w is
  * w_gate or w_up, [E,H,F]) or MOE_WEIGHTS_DOWN (w is w_down, [E,F,H]).
@@ -559,6 +559,28 @@ MOE_API moe_status moe_ep_direct_return(const moe_shape *shape, int32_t G, const
  * peer_y.  A barrier over the ranks follows, as after step 6. */
 MOE_API moe_status moe_ep_direct_down_return(const moe_shape *shape, int32_t G, const void *h_loc,
                                              const void *w_down, void *ws_loc, void *ep_ws, void *stream);
+
+/* The fp8 layer in the peer-store form: e4m3 rows on the links (half the
+ * bytes of bf16 rows).  Each rank quantizes its token rows once
+ * (moe_quantize_rows_fp8, MOE_ROWS_TOKENS: x_q [T,H] codes, x_scale [T]);
+ * step 4 becomes moe_ep_direct_dispatch_fp8, which stores each routed pair's
+ * code row into its expert's rank's x_loc_q [local T, H] and the row's scale
+ * into that rank's scale_loc [local T] (peer_x_loc_q, peer_scale_loc: device
+ * arrays of G addresses); step 5 is moe_grouped_swiglu_fp8 on the local shape
+ * (x_loc_q, scale_loc, no src_token; the rank's weight codes and scales, as
+ * moe_quantize_weights_fp8 leaves them, sliced to its experts), then
+ * moe_quantize_rows_fp8 (MOE_ROWS_H, no src_token) and
+ * moe_ep_direct_down_return_fp8, the fp8 down projection storing each result
+ * row straight into its token's rank's y.  Each rank's out equals
+ * moe_forward_fp8's on its tokens. */
+MOE_API moe_status moe_ep_direct_dispatch_fp8(const moe_shape *shape, int32_t G, const void *x_q,
+                                              const float *x_scale, const int32_t *topk_idx, const int32_t *dest_row,
+                                              const int32_t *expert_offsets, const void *peer_x_loc_q,
+                                              const void *peer_scale_loc, void *ws, void *ep_ws, void *stream);
+
+MOE_API moe_status moe_ep_direct_down_return_fp8(const moe_shape *shape, int32_t G, const void *h_q,
+                                                 const float *h_scale, const void *wd_q, const float *wd_scale,
+                                                 void *ws_loc, void *ep_ws, void *stream);
 
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);

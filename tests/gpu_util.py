@@ -233,3 +233,32 @@ def run_direct_ep(dl, shape, G, fused_return=False):
         ep.finish()
     torch.cuda.synchronize()
     return ranks, xs
+
+
+def run_direct_ep_fp8(dl, shape, G, wq):
+    """The fp8 peer-store layer on G ranks held by this process: each rank
+    quantizes its tokens, stores code rows and scales into the owners'
+    buffers, runs the fp8 GEMMs on its experts (wq: the layer's weight codes
+    and scales from moe_quantize_weights_fp8, sliced per rank here) and the
+    down GEMM stores the results into the tokens' owners' y."""
+    from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
+    T, Eg = shape.T, shape.E // G
+    ranks = [DirectEP(shape, G, r, fp8=True) for r in range(G)]
+    connect_in_process(ranks)
+    xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
+    for r, ep in enumerate(ranks):
+        ep.route(xs[r], dl.w_router, dl.bias)
+        ep.quantize_tokens(xs[r])
+    gather_counts_in_process(ranks)
+    for ep in ranks:
+        ep.plan()
+    for ep in ranks:
+        ep.dispatch_fp8()
+    for r, ep in enumerate(ranks):
+        sl = slice(r * Eg, (r + 1) * Eg)
+        ep.experts_fp8_and_return(wq["wg_q"][sl], wq["wg_scale"][sl], wq["wu_q"][sl], wq["wu_scale"][sl],
+                                  wq["wd_q"][sl], wq["wd_scale"][sl])
+    for ep in ranks:
+        ep.finish()
+    torch.cuda.synchronize()
+    return ranks, xs

@@ -16,7 +16,7 @@ import torch
 
 import grouped_expert_gemm_router_b200 as moe
 import synth
-from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer, run_direct_ep
+from gpu_util import DeviceLayer, assert_close_bf16, bf16_host, oracle_layer, run_direct_ep, run_direct_ep_fp8
 from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
 
 pytestmark = pytest.mark.gpu
@@ -145,3 +145,54 @@ def test_direct_ep_rejects_unsupported_shapes():
         DirectEP(_shape(cfg), 3, 0)  # E % G != 0
     with pytest.raises(moe.MoeError):
         DirectEP(_shape(cfg), 2, 2)  # rank out of range
+
+
+@pytest.mark.parametrize("name,G", [("decode_E64_k6", 8), ("E16_k4_F384", 4), ("E8_k2_skew", 2),
+                                    ("several_tiles_E4_k2", 2)], ids=lambda v: str(v))
+def test_direct_ep_fp8_matches_single_gpu_fp8(name, G):
+    """e4m3 rows on the links: each rank's out equals moe_forward_fp8 on its
+    tokens bit for bit (per-row token codes and scales are the same whichever
+    rank quantizes them; the same fp8 GEMM arithmetic on the same rows)."""
+    cfg, _ = CASES[name]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    wq = dl.bufs(shape)
+    wq.update(moe.alloc_fp8_buffers(shape))
+    moe.quantize_layer_weights_fp8(shape, wq)
+    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq)
+    for r, ep in enumerate(ranks):
+        assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
+        b = dl.bufs(shape)
+        b["x"] = xs[r]
+        b.update({k: wq[k] for k in ("wg_q", "wg_scale", "wu_q", "wu_scale", "wd_q", "wd_scale")})
+        f = moe.alloc_fp8_buffers(shape)
+        b.update({k: f[k] for k in ("x_q", "x_scale", "h_q", "h_scale")})
+        moe.moe_forward_fp8(shape, b, b["ws"])
+        torch.cuda.synchronize()
+        assert moe.moe_read_status(b["ws"]) == 0
+        assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(b["out"])), "rank %d" % r
+
+
+def test_direct_ep_fp8_full_size_decode():
+    """The DeepSeek-V2-Lite-shaped layer (uncapped) on 8 ranks in fp8, bit
+    for bit against each rank's moe_forward_fp8."""
+    cfg = synth.CONFIGS[4].with_(C=0)
+    G = 8
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    wq = dl.bufs(shape)
+    wq.update(moe.alloc_fp8_buffers(shape))
+    moe.quantize_layer_weights_fp8(shape, wq)
+    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq)
+    for r, ep in enumerate(ranks):
+        b = dl.bufs(shape)
+        b["x"] = xs[r]
+        b.update({k: wq[k] for k in ("wg_q", "wg_scale", "wu_q", "wu_scale", "wd_q", "wd_scale")})
+        f = moe.alloc_fp8_buffers(shape)
+        b.update({k: f[k] for k in ("x_q", "x_scale", "h_q", "h_scale")})
+        moe.moe_forward_fp8(shape, b, b["ws"])
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(b["out"])), "rank %d" % r
+
