@@ -637,7 +637,7 @@ class Bench:
         return {"G": G, "S": S, "per_phase_us_all_ranks": per_phase, "overflow_rows": spill,
                 "device_status": status, "single_gpu_layer_us": m1["total_ms"] / steps * 1e3}
 
-    def measure_ep_direct(self, cfg, L, G, steps, warmup):
+    def measure_ep_direct(self, cfg, L, G, steps, warmup, fp8=False):
         """The peer-store expert-parallel layer with G ranks held by this
         process: peer tables point at the other ranks' own buffers, so the
         stores stay on this GPU (on G GPUs they cross NVLink); the counts
@@ -657,10 +657,14 @@ class Bench:
         wr = torch.from_numpy(L.w_router).to(dev)
         bias = None if L.bias is None else torch.from_numpy(L.bias).to(dev)
         xs = [dev_bf16(replica_tokens(cfg, r, L)) for r in range(G)]
-        ranks = [DirectEP(shape, G, r, dev) for r in range(G)]
+        ranks = [DirectEP(shape, G, r, dev, fp8=fp8) for r in range(G)]
         connect_in_process(ranks)
         Eg = cfg.E // G
         sl = [slice(r * Eg, (r + 1) * Eg) for r in range(G)]
+        if fp8:  # the layer's weight codes and scales, sliced per rank below
+            wq = {"w_gate": wg, "w_up": wu, "w_down": wd}
+            wq.update(moe.alloc_fp8_buffers(shape, device=dev))
+            moe.quantize_layer_weights_fp8(shape, wq, stream)
         # experts_down + send_back and their fused form (the down GEMM storing
         # into the owners' y) both run each step; the totals count one or the other
         phases = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "down_return_fused",
@@ -678,6 +682,27 @@ class Bench:
                                                                          ranks[r].ws_loc, ranks[r].ep_ws, stream),
             "finish": lambda r: ranks[r].finish(stream),
         }
+
+        if fp8:
+            L_ = ranks[0].local
+            phases = ("route", "quantize_tokens", "plan", "dispatch", "experts_swiglu", "quantize_h",
+                      "down_return_fused", "finish")
+            calls = {
+                "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
+                "quantize_tokens": lambda r: ranks[r].quantize_tokens(xs[r], stream),
+                "plan": lambda r: ranks[r].plan(stream),
+                "dispatch": lambda r: ranks[r].dispatch_fp8(stream),
+                "experts_swiglu": lambda r: moe.moe_grouped_swiglu_fp8(
+                    L_, ranks[r].x_loc_q, ranks[r].scale_loc, None, wq["wg_q"][sl[r]], wq["wg_scale"][sl[r]],
+                    wq["wu_q"][sl[r]], wq["wu_scale"][sl[r]], ranks[r].h_loc, ranks[r].ws_loc, stream),
+                "quantize_h": lambda r: moe.moe_quantize_rows_fp8(L_, moe.MOE_ROWS_H, ranks[r].h_loc, None,
+                                                                  ranks[r].h_q, ranks[r].h_scale, ranks[r].ws_loc,
+                                                                  stream),
+                "down_return_fused": lambda r: moe.moe_ep_direct_down_return_fp8(
+                    shape, G, ranks[r].h_q, ranks[r].h_scale, wq["wd_q"][sl[r]], wq["wd_scale"][sl[r]],
+                    ranks[r].ws_loc, ranks[r].ep_ws, stream),
+                "finish": lambda r: ranks[r].finish(stream),
+            }
 
         def step(timed):
             ev = {}
@@ -708,9 +733,9 @@ class Bench:
                                          for e in evs])) * 1e3 for ph in phases}
         status = [moe.moe_read_status(ep.ws) | moe.moe_read_status(ep.ws_loc) for ep in ranks]
         shp1, b1 = self.upload(cfg, L, replica_tokens(cfg, 0, L))
-        m1 = self.measure(cfg, shp1, b1, steps, warmup)
+        m1 = self.measure_fp8(cfg, shp1, b1, steps, warmup) if fp8 else self.measure(cfg, shp1, b1, steps, warmup)
         del b1, ranks
-        return {"G": G, "per_phase_us_all_ranks": per_phase, "device_status": status,
+        return {"G": G, "fp8": fp8, "per_phase_us_all_ranks": per_phase, "device_status": status,
                 "single_gpu_layer_us": m1["total_ms"] / steps * 1e3}
 
     def e2e_pipelined(self, cfg, shape, b, x_rank, fwd_bufs, steps, warmup):
@@ -871,20 +896,21 @@ def summarize_ep(cfg, e, peaks):
     }
 
 
-def experts_roofline(cfg, G, t, peaks):
+def experts_roofline(cfg, G, t, peaks, fp8=False):
     """The local grouped GEMMs of one rank (SwiGLU + down, t seconds) against
     the larger of the rank's expert-weight bytes over HBM bandwidth and its
-    average rows' (T k) FLOPs over the bf16 tensor peak."""
+    average rows' (T k) FLOPs over the tensor peak (fp8: one-byte weights,
+    twice the bf16 peak)."""
     Eg = cfg.E // G
-    w_bytes = 3 * Eg * cfg.H * cfg.F * 2
+    w_bytes = 3 * Eg * cfg.H * cfg.F * (1 if fp8 else 2)
     flops = 2.0 * cfg.T * cfg.k * cfg.H * cfg.F * 3
-    if w_bytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12):
+    tc = peaks["bf16_tflops"] * (2 if fp8 else 1)
+    if w_bytes / (peaks["hbm_gbs"] * 1e9) >= flops / (tc * 1e12):
         a = w_bytes / t / 1e9
         return {"bound": "hbm", "bytes": w_bytes, "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": a / peaks["hbm_gbs"]}
     a = flops / t / 1e12
-    return {"bound": "tensor", "flops": flops, "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": a / peaks["bf16_tflops"]}
+    return {"bound": "tensor", "flops": flops, "achieved": a, "peak": tc, "unit": "TFLOP/s", "frac": a / tc}
 
 
 def summarize_ep_direct(cfg, e, peaks):
@@ -894,19 +920,22 @@ def summarize_ep_direct(cfg, e, peaks):
     Eg = cfg.E // G
     per_rank = {ph: t / G for ph, t in e["per_phase_us_all_ranks"].items()}
     sent = cfg.T * cfg.k * row  # every routed row once out, its result once back
-    t_exp = (per_rank["experts_swiglu"] + per_rank["experts_down"]) * 1e-6
+    out_bytes = cfg.T * cfg.k * (cfg.H + 4) if e.get("fp8") else sent  # fp8: code rows and a scale each
+    fp8 = bool(e.get("fp8"))
+    down = per_rank["down_return_fused"] if fp8 else per_rank["experts_down"]
+    t_exp = (per_rank["experts_swiglu"] + down) * 1e-6
     return {
-        "workload": workload_name(cfg) + "-uncapped", "G": G,
+        "workload": workload_name(cfg) + "-uncapped" + ("-fp8" if fp8 else ""), "G": G,
         "ranks": "G ranks emulated on one GPU: each rank's peer stores go to the other ranks' buffers on the same "
                  "device; the counts all-gather done by copies and not timed",
         "per_rank_us": per_rank,
-        "per_rank_kernels_us": sum(v for k, v in per_rank.items() if k != "down_return_fused"),
+        "per_rank_kernels_us": sum(v for k, v in per_rank.items() if fp8 or k != "down_return_fused"),
         "per_rank_kernels_fused_return_us": sum(v for k, v in per_rank.items()
                                                 if k not in ("experts_down", "send_back")),
         "single_gpu_layer_us": e["single_gpu_layer_us"],
-        "experts_roofline": experts_roofline(cfg, G, t_exp, peaks),
-        "exchange_per_rank": {"dispatch_bytes": sent, "return_bytes": sent, "counts_bytes": G * cfg.E * 4,
-                              "nvlink_model_us": 2 * sent / (NVLINK_PEER_GBS * 1e9) * 1e6,
+        "experts_roofline": experts_roofline(cfg, G, t_exp, peaks, fp8),
+        "exchange_per_rank": {"dispatch_bytes": out_bytes, "return_bytes": sent, "counts_bytes": G * cfg.E * 4,
+                              "nvlink_model_us": (out_bytes + sent) / (NVLINK_PEER_GBS * 1e9) * 1e6,
                               "nvlink_model": "routed rows out and results back at %g GB/s per direction (a "
                                               "model, not a measurement)" % NVLINK_PEER_GBS},
         "device_status": e["device_status"],
@@ -1089,6 +1118,8 @@ def run_ours(args):
         Lm = synth.make_layer(cm)
         ep["direct_mixtral"] = summarize_ep_direct(cm, bench.measure_ep_direct(
             cm, Lm, 8, min(K, args.per_config_steps), min(args.warmup, 5)), peaks)
+        ep["direct_fp8"] = summarize_ep_direct(ce, bench.measure_ep_direct(
+            ce, synth.make_layer(ce), 8, min(K, args.per_config_steps), min(args.warmup, 5), fp8=True), peaks)
         log("peer-store EP G=8: %.1f / %.1f us of kernels per rank (%.1f s)" % (
             ep["direct"]["per_rank_kernels_us"], ep["direct_mixtral"]["per_rank_kernels_us"], time.time() - t0))
         del Lm

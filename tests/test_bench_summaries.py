@@ -64,3 +64,18 @@ def test_peer_store_summary_and_bound():
     # the decode layer's eight experts per rank stream their weights: HBM-bound
     r = bench.experts_roofline(synth.CONFIGS[4], G, 60e-6, PEAKS)
     assert r["bound"] == "hbm" and r["bytes"] == 3 * 8 * 2048 * 1408 * 2
+
+
+def test_peer_store_fp8_summary():
+    G = 8
+    phases = {"route": 80.0, "quantize_tokens": 24.0, "plan": 40.0, "dispatch": 40.0, "experts_swiglu": 160.0,
+              "quantize_h": 32.0, "down_return_fused": 120.0, "finish": 64.0}
+    e = {"G": G, "fp8": True, "per_phase_us_all_ranks": phases, "device_status": [0] * G,
+         "single_gpu_layer_us": 150.0}
+    cfg = synth.CONFIGS[4]
+    s = bench.summarize_ep_direct(cfg, e, PEAKS)
+    assert s["per_rank_kernels_us"] == pytest.approx(sum(phases.values()) / G)
+    assert s["exchange_per_rank"]["dispatch_bytes"] == 128 * 6 * (2048 + 4)   # code rows and a scale each
+    assert s["exchange_per_rank"]["return_bytes"] == 128 * 6 * 2048 * 2       # bf16 results
+    r = s["experts_roofline"]
+    assert r["bound"] == "hbm" and r["bytes"] == 3 * 8 * 2048 * 1408           # one-byte weights
