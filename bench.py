@@ -695,9 +695,8 @@ class Bench:
                 "experts_swiglu": lambda r: moe.moe_grouped_swiglu_fp8(
                     L_, ranks[r].x_loc_q, ranks[r].scale_loc, None, wq["wg_q"][sl[r]], wq["wg_scale"][sl[r]],
                     wq["wu_q"][sl[r]], wq["wu_scale"][sl[r]], ranks[r].h_loc, ranks[r].ws_loc, stream),
-                "quantize_h": lambda r: moe.moe_quantize_rows_fp8(L_, moe.MOE_ROWS_H, ranks[r].h_loc, None,
-                                                                  ranks[r].h_q, ranks[r].h_scale, ranks[r].ws_loc,
-                                                                  stream),
+                "quantize_h": lambda r: moe.moe_ep_direct_quantize_h(shape, G, ranks[r].h_loc, ranks[r].h_q,
+                                                                     ranks[r].h_scale, ranks[r].ep_ws, stream),
                 "down_return_fused": lambda r: moe.moe_ep_direct_down_return_fp8(
                     shape, G, ranks[r].h_q, ranks[r].h_scale, wq["wd_q"][sl[r]], wq["wd_scale"][sl[r]],
                     ranks[r].ws_loc, ranks[r].ep_ws, stream),

@@ -42,7 +42,7 @@ ABI_FUNCTIONS = (
     "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
     "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
-    "moe_ep_direct_down_return_fp8",
+    "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -179,6 +179,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_direct_dispatch_fp8.restype = st
     lib.moe_ep_direct_down_return_fp8.argtypes = [sp, i32] + [vp] * 7
     lib.moe_ep_direct_down_return_fp8.restype = st
+    lib.moe_ep_direct_quantize_h.argtypes = [sp, i32] + [vp] * 5
+    lib.moe_ep_direct_quantize_h.restype = st
     _lib = lib
     return lib
 
@@ -551,4 +553,10 @@ def moe_ep_direct_down_return_fp8(shape, G, h_q, h_scale, wd_q, wd_scale, ws_loc
     _check(load_library().moe_ep_direct_down_return_fp8(ctypes.byref(shape), int(G), _ptr(h_q), _ptr(h_scale),
                                                         _ptr(wd_q), _ptr(wd_scale), _ptr(ws_loc), _ptr(ep_ws),
                                                         _stream(stream)), "moe_ep_direct_down_return_fp8")
+
+
+def moe_ep_direct_quantize_h(shape, G, h_loc, h_q, h_scale, ep_ws, stream=None):
+    _check(load_library().moe_ep_direct_quantize_h(ctypes.byref(shape), int(G), _ptr(h_loc), _ptr(h_q),
+                                                   _ptr(h_scale), _ptr(ep_ws), _stream(stream)),
+           "moe_ep_direct_quantize_h")
 

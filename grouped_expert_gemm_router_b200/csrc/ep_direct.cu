@@ -282,6 +282,11 @@ const unsigned long long *ep_direct_row_addr(void *ep_ws, const moe_shape &s, in
     return dir_ptrs(ep_ws, s, G).row_addr;
 }
 
+// The number of local rows the plan laid out (device int).
+const int32_t *ep_direct_local_total(void *ep_ws, const moe_shape &s, int G) {
+    return dir_ptrs(ep_ws, s, G).loc_offsets + s.E / G;
+}
+
 cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
                                   const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream) {
     const DirWs p = dir_ptrs(ep_ws, s, G);

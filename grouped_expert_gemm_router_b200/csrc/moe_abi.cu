@@ -54,6 +54,9 @@ size_t ep_direct_workspace_bytes(const moe_shape &s, int G);
 cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
                                   const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream);
 const unsigned long long *ep_direct_row_addr(void *ep_ws, const moe_shape &s, int G);
+const int32_t *ep_direct_local_total(void *ep_ws, const moe_shape &s, int G);
+cudaError_t launch_quant_rows_counted(const void *src, int K, int rows_cap, const int *rows_dev, void *q,
+                                      float *scale, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
                                  const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
                                  void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream,
@@ -747,5 +750,19 @@ moe_status moe_ep_direct_down_return_fp8(const moe_shape *s, int32_t G, const vo
                                             g_timeout_ns.load(), sms, (cudaStream_t)stream, nullptr, nullptr,
                                             ep_direct_row_addr(ep_ws, *s, G));
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_down_return_fp8");
+}
+
+moe_status moe_ep_direct_quantize_h(const moe_shape *s, int32_t G, const void *h_loc, void *h_q, float *h_scale,
+                                    void *ep_ws, void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned(h_loc, 16) || !aligned(h_q, 16) || !aligned(h_scale, 4) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    cudaError_t e = launch_quant_rows_counted(h_loc, s->F, (int)ep_direct_local_rows(*s, G),
+                                              ep_direct_local_total(ep_ws, *s, G), h_q, h_scale, sms,
+                                              (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_quantize_h");
 }
 

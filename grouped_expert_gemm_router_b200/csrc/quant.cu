@@ -313,6 +313,14 @@ cudaError_t launch_quant_rows(const moe_shape &s, int K, const void *src, int sr
                        capped ? -1 : R, s.E * s.C, p.total_spill, P, num_sms, stream);
 }
 
+// Codes + scales of rows [0, *rows_dev) of src [rows_cap, K] (rows_dev: a
+// device count, at most rows_cap; the rest are left unwritten).
+cudaError_t launch_quant_rows_counted(const void *src, int K, int rows_cap, const int *rows_dev, void *q,
+                                      float *scale, int num_sms, cudaStream_t stream) {
+    return launch_rows((const uint4 *)src, nullptr, 0, (uint2 *)q, scale, K / 8, rows_cap, rows_cap, -1, 0, rows_dev,
+                       rows_cap, num_sms, stream);
+}
+
 // Codes + scales of every token row of x [T, K] (the form the row-gathering
 // SwiGLU GEMM reads).
 cudaError_t launch_quant_tokens(const moe_shape &s, const void *x, void *q, float *scale, int num_sms,

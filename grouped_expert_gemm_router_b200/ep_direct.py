@@ -137,7 +137,7 @@ class DirectEP:
         L = self.local
         moe.moe_grouped_swiglu_fp8(L, self.x_loc_q, self.scale_loc, None, wg_q, wg_scale, wu_q, wu_scale, self.h_loc,
                                    self.ws_loc, stream)
-        moe.moe_quantize_rows_fp8(L, moe.MOE_ROWS_H, self.h_loc, None, self.h_q, self.h_scale, self.ws_loc, stream)
+        moe.moe_ep_direct_quantize_h(self.shape, self.G, self.h_loc, self.h_q, self.h_scale, self.ep_ws, stream)
         moe.moe_ep_direct_down_return_fp8(self.shape, self.G, self.h_q, self.h_scale, wd_q, wd_scale, self.ws_loc,
                                           self.ep_ws, stream)
 

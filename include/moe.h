@@ -569,8 +569,8 @@ MOE_API moe_status moe_ep_direct_down_return(const moe_shape *shape, int32_t G, 
  * arrays of G addresses); step 5 is moe_grouped_swiglu_fp8 on the local shape
  * (x_loc_q, scale_loc, no src_token; the rank's weight codes and scales, as
  * moe_quantize_weights_fp8 leaves them, sliced to its experts), then
- * moe_quantize_rows_fp8 (MOE_ROWS_H, no src_token) and
- * moe_ep_direct_down_return_fp8, the fp8 down projection storing each result
+ * moe_ep_direct_quantize_h (or moe_quantize_rows_fp8, MOE_ROWS_H, no
+ * src_token: every row) and moe_ep_direct_down_return_fp8, the fp8 down projection storing each result
  * row straight into its token's rank's y.  Each rank's out equals
  * moe_forward_fp8's on its tokens. */
 MOE_API moe_status moe_ep_direct_dispatch_fp8(const moe_shape *shape, int32_t G, const void *x_q,
@@ -581,6 +581,13 @@ MOE_API moe_status moe_ep_direct_dispatch_fp8(const moe_shape *shape, int32_t G,
 MOE_API moe_status moe_ep_direct_down_return_fp8(const moe_shape *shape, int32_t G, const void *h_q,
                                                  const float *h_scale, const void *wd_q, const float *wd_scale,
                                                  void *ws_loc, void *ep_ws, void *stream);
+
+/* The fp8 form's h quantization limited to the local rows the plan laid out
+ * (the received rows, read from ep_ws on the device): h_loc [local T, F] bf16
+ * -> h_q [local T, F] codes, h_scale [local T]; rows past them are left
+ * unwritten.  Same codes as moe_quantize_rows_fp8 (MOE_ROWS_H) on those rows. */
+MOE_API moe_status moe_ep_direct_quantize_h(const moe_shape *shape, int32_t G, const void *h_loc, void *h_q,
+                                            float *h_scale, void *ep_ws, void *stream);
 
 /* Upper bound, in nanoseconds, of every bounded device wait (default 1e9). */
 MOE_API void moe_set_wait_timeout_ns(uint64_t ns);
