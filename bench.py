@@ -667,12 +667,11 @@ class Bench:
             moe.quantize_layer_weights_fp8(shape, wq, stream)
         # experts_down + send_back and their fused form (the down GEMM storing
         # into the owners' y) both run each step; the totals count one or the other
-        phases = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "down_return_fused",
+        phases = ("route", "plan_dispatch", "experts_swiglu", "experts_down", "send_back", "down_return_fused",
                   "finish")
         calls = {
             "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
-            "plan": lambda r: ranks[r].plan(stream),
-            "dispatch": lambda r: ranks[r].dispatch(xs[r], stream),
+            "plan_dispatch": lambda r: ranks[r].plan_and_dispatch(xs[r], stream),
             "experts_swiglu": lambda r: moe.moe_grouped_swiglu(ranks[r].local, ranks[r].x_loc, wg[sl[r]], wu[sl[r]],
                                                                ranks[r].h_loc, ranks[r].ws_loc, stream),
             "experts_down": lambda r: moe.moe_grouped_down(ranks[r].local, ranks[r].h_loc, wd[sl[r]], ranks[r].y_loc,
@@ -685,13 +684,12 @@ class Bench:
 
         if fp8:
             L_ = ranks[0].local
-            phases = ("route", "quantize_tokens", "plan", "dispatch", "experts_swiglu", "quantize_h",
+            phases = ("route", "quantize_tokens", "plan_dispatch", "experts_swiglu", "quantize_h",
                       "down_return_fused", "finish")
             calls = {
                 "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
                 "quantize_tokens": lambda r: ranks[r].quantize_tokens(xs[r], stream),
-                "plan": lambda r: ranks[r].plan(stream),
-                "dispatch": lambda r: ranks[r].dispatch_fp8(stream),
+                "plan_dispatch": lambda r: ranks[r].plan_and_dispatch(None, stream),
                 "experts_swiglu": lambda r: moe.moe_grouped_swiglu_fp8(
                     L_, ranks[r].x_loc_q, ranks[r].scale_loc, None, wq["wg_q"][sl[r]], wq["wg_scale"][sl[r]],
                     wq["wu_q"][sl[r]], wq["wu_scale"][sl[r]], ranks[r].h_loc, ranks[r].ws_loc, stream),
@@ -706,7 +704,7 @@ class Bench:
         def step(timed):
             ev = {}
             for ph in phases:
-                if ph == "plan":
+                if ph in ("plan", "plan_dispatch"):
                     gather_counts_in_process(ranks)
                 for r in range(G):
                     if timed:

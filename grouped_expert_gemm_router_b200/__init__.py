@@ -42,7 +42,7 @@ ABI_FUNCTIONS = (
     "moe_ep_local_shape", "moe_ep_pack", "moe_ep_local_dispatch", "moe_ep_local_return", "moe_ep_unpack",
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
     "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
-    "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h",
+    "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h", "moe_ep_direct_plan_dispatch",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -181,6 +181,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_direct_down_return_fp8.restype = st
     lib.moe_ep_direct_quantize_h.argtypes = [sp, i32] + [vp] * 5
     lib.moe_ep_direct_quantize_h.restype = st
+    lib.moe_ep_direct_plan_dispatch.argtypes = [sp, i32, i32] + [vp] * 13
+    lib.moe_ep_direct_plan_dispatch.restype = st
     _lib = lib
     return lib
 
@@ -559,4 +561,13 @@ def moe_ep_direct_quantize_h(shape, G, h_loc, h_q, h_scale, ep_ws, stream=None):
     _check(load_library().moe_ep_direct_quantize_h(ctypes.byref(shape), int(G), _ptr(h_loc), _ptr(h_q),
                                                    _ptr(h_scale), _ptr(ep_ws), _stream(stream)),
            "moe_ep_direct_quantize_h")
+
+
+def moe_ep_direct_plan_dispatch(shape, G, rank, cnt_all, peer_y, x, x_scale, topk_idx, dest_row, expert_offsets,
+                                peer_x_loc, peer_scale_loc, ws, ws_loc, ep_ws, stream=None):
+    """x_scale None: bf16 rows; else e4m3 code rows with their scales."""
+    _check(load_library().moe_ep_direct_plan_dispatch(
+        ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(peer_y), _ptr(x), _ptr(x_scale), _ptr(topk_idx),
+        _ptr(dest_row), _ptr(expert_offsets), _ptr(peer_x_loc), _ptr(peer_scale_loc), _ptr(ws), _ptr(ws_loc),
+        _ptr(ep_ws), _stream(stream)), "moe_ep_direct_plan_dispatch")
 

@@ -25,6 +25,8 @@
 //                     local layout, GEMM schedule and return segments.
 // k_ep_direct_put     source: a warp per routed pair, x[t] -> the
 //                     destination's x_loc row.
+// k_ep_direct_plan_put  both in one launch: every block derives the send
+//                     positions itself, block 0 also lays out the local rows.
 // k_ep_direct_return  destination: a warp per local row, y_loc -> the
 //                     source's y row.
 // Each put kernel ends with a system-scope fence, so a stream-ordered
@@ -62,72 +64,78 @@ struct DirPlanArgs {
     WsPtrs lws;
 };
 
-__global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) {
-    __shared__ DispatchSmem sm;
-    __shared__ int c[kDirMaxCounts];
-    __shared__ int base[kMaxExperts];  // destination layout offsets of each expert (over all sources)
-    __shared__ int any_bad;
-    pdl_trigger();
-    pdl_wait();
+// Shared-memory state of a planning block.
+struct DirPlanSmem {
+    DispatchSmem sm;
+    int c[kDirMaxCounts];      // gathered counts, clamped
+    int base[kMaxExperts];     // per expert: this rank's first row in its owner's x_loc; later segment starts
+    int cnt[kMaxExperts];      // per expert: this rank's rows for it
+    int sstart[kMaxExperts];   // return segments' first local rows
+    int any_bad;
+};
+
+// The gathered counts, clamped identically on every rank ((source s,
+// destination d): its experts' counts to [0, T] and their running sum to the
+// per-destination bound T min(k, E_g), in expert order), and this rank's
+// send positions: base[e] = rows of expert e's owner before expert e's rows
+// from this rank, cnt[e] = this rank's rows for e.  All threads of the block.
+__device__ void plan_send(const DirPlanArgs &a, DirPlanSmem &p) {
     const int tid = threadIdx.x, G = a.G, E = a.E, Eg = E / G, r = a.rank;
     const int per_dest = a.T * (a.k < Eg ? a.k : Eg);
-    if (tid == 0) any_bad = 0;
-    for (int i = tid; i < G * E; i += kScanThreads) c[i] = a.cnt_all[i];
+    if (tid == 0) p.any_bad = 0;
+    for (int i = tid; i < G * E; i += kScanThreads) p.c[i] = a.cnt_all[i];
     __syncthreads();
-    // Clamp: (source s, destination d): its experts' counts to [0, T] and
-    // their running sum to the per-destination bound, in expert order.
     for (int sd = tid; sd < G * G; sd += kScanThreads) {
         const int s = sd / G, d = sd % G;
         int run = 0;
         bool bad = false;
         for (int el = 0; el < Eg; ++el) {
-            const int i = s * E + d * Eg + el, v = c[i];
+            const int i = s * E + d * Eg + el, v = p.c[i];
             const int w = min(min(max(v, 0), a.T), per_dest - run);
             bad |= w != v;
-            c[i] = w;
+            p.c[i] = w;
             run += w;
         }
-        if (bad) any_bad = 1;
+        if (bad) p.any_bad = 1;
     }
     __syncthreads();
-    if (tid == 0 && any_bad) atomicOr(a.lws.status, MOE_DEV_BAD_ROW);
-    // Every destination's offsets of its experts (over all sources).
     for (int e = tid; e < E; e += kScanThreads) {
         const int d = e / Eg, el = e % Eg;
         int off = 0;
         for (int e2 = d * Eg; e2 < d * Eg + el; ++e2)
-            for (int s = 0; s < G; ++s) off += c[s * E + e2];
-        base[e] = off;
+            for (int s = 0; s < G; ++s) off += p.c[s * E + e2];
+        for (int s = 0; s < r; ++s) off += p.c[s * E + e];
+        p.base[e] = off;
+        p.cnt[e] = p.c[r * E + e];
     }
     __syncthreads();
-    // Source role: where this rank's pairs of expert e start in the
-    // destination's local rows.
-    for (int e = tid; e < E; e += kScanThreads) {
-        int b = base[e];
-        for (int s = 0; s < r; ++s) b += c[s * E + e];
-        a.send_base[e] = b;
-        a.send_cnt[e] = c[r * E + e];
-    }
-    // Destination role: the local layout and its GEMM schedule.
+}
+
+// This rank as a destination: the local layout and its GEMM schedule, the
+// return segments and each local row's destination address.  All threads of
+// the block, after plan_send (base[] and cnt[] are left as they were).
+__device__ void plan_local(const DirPlanArgs &a, DirPlanSmem &p) {
+    DispatchSmem &sm = p.sm;
+    const int tid = threadIdx.x, G = a.G, E = a.E, Eg = E / G, r = a.rank;
+    if (tid == 0 && p.any_bad) atomicOr(a.lws.status, MOE_DEV_BAD_ROW);
     for (int el = tid; el < Eg; el += kScanThreads) {
         int n = 0;
-        for (int s = 0; s < G; ++s) n += c[s * E + r * Eg + el];
+        for (int s = 0; s < G; ++s) n += p.c[s * E + r * Eg + el];
         sm.hist[el] = n;
     }
     __syncthreads();
     build_schedule_block(sm, Eg, 0, false, a.loc_counts, a.loc_offsets, a.lws);
     // Return segments: (source s, local expert el) -> first local row, rows,
     // first row in the source's y (its uncapped offset of the expert).
-    // G E_g = E segments, kept in shared memory (base[] is free again).
-    int *sstart = base;
+    int *sstart = p.sstart;
     for (int i = tid; i < G * Eg; i += kScanThreads) {
         const int s = i / Eg, el = i % Eg, e = r * Eg + el;
         int start = sm.offs[el];
-        for (int s2 = 0; s2 < s; ++s2) start += c[s2 * E + e];
+        for (int s2 = 0; s2 < s; ++s2) start += p.c[s2 * E + e];
         int ysrc = 0;
-        for (int e2 = 0; e2 < e; ++e2) ysrc += c[s * E + e2];
+        for (int e2 = 0; e2 < e; ++e2) ysrc += p.c[s * E + e2];
         a.seg_start[i] = start;
-        a.seg_cnt[i] = c[s * E + e];
+        a.seg_cnt[i] = p.c[s * E + e];
         a.seg_ysrc[i] = ysrc;
         sstart[i] = start;
         sm.running[i] = ysrc;  // scratch: the segment's first row in the source's y
@@ -160,36 +168,71 @@ __global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) 
     }
 }
 
-// Source side: pair i = t k + j of expert e goes to row send_base[e] +
+__global__ void __launch_bounds__(kScanThreads) k_ep_direct_plan(DirPlanArgs a) {
+    __shared__ DirPlanSmem p;
+    pdl_trigger();
+    pdl_wait();
+    plan_send(a, p);
+    for (int e = threadIdx.x; e < a.E; e += kScanThreads) {
+        a.send_base[e] = p.base[e];
+        a.send_cnt[e] = p.cnt[e];
+    }
+    plan_local(a, p);
+}
+
+// Source side: pair i = t k + j of expert e goes to row base[e] +
 // (dest_row[i] - offsets[e]) of rank e / E_g's x_loc.  Rows of H8 16-byte
 // vectors (bf16 rows, or e4m3 code rows); with x_scale, the row's scale goes
 // to the same row of the rank's scale array (peer_scale).
-__global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(const uint4 *x, const int32_t *topk_idx,
-                                                                const int32_t *dest_row, const int32_t *offsets,
-                                                                const int32_t *send_base, const int32_t *send_cnt,
-                                                                const unsigned long long *peer_x_loc, int R, int k,
-                                                                int E, int Eg, int Tloc, int H8, uint32_t *status,
-                                                                const float *x_scale,
-                                                                const unsigned long long *peer_scale) {
-    pdl_trigger();
-    pdl_wait();
+struct DirPutArgs {
+    const uint4 *x;
+    const int32_t *topk_idx, *dest_row, *offsets;
+    const unsigned long long *peer_x_loc;
+    int R, k, E, Eg, Tloc, H8;
+    uint32_t *status;
+    const float *x_scale;
+    const unsigned long long *peer_scale;
+};
+
+__device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt) {
     const int lane = threadIdx.x & 31;
     bool bad = false;
-    for (int i = blockIdx.x * kDirWarps + (threadIdx.x >> 5); i < R; i += gridDim.x * kDirWarps) {
-        const int e = topk_idx[i];
-        if ((unsigned)e >= (unsigned)E) continue;  // reported by the router
-        const int ri = dest_row[i] - offsets[e];
-        const int pos = send_base[e] + ri;
-        if (ri < 0 || ri >= send_cnt[e] || (unsigned)pos >= (unsigned)Tloc) {
+    for (int i = blockIdx.x * kDirWarps + (threadIdx.x >> 5); i < q.R; i += gridDim.x * kDirWarps) {
+        const int e = q.topk_idx[i];
+        if ((unsigned)e >= (unsigned)q.E) continue;  // reported by the router
+        const int ri = q.dest_row[i] - q.offsets[e];
+        const int pos = base[e] + ri;
+        if (ri < 0 || ri >= cnt[e] || (unsigned)pos >= (unsigned)q.Tloc) {
             bad = true;
             continue;
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(peer_x_loc[e / Eg]) + (size_t)pos * H8;
-        copy_row16(x + (size_t)(i / k) * H8, dst, H8, lane);
-        if (x_scale && lane == 0) reinterpret_cast<float *>(peer_scale[e / Eg])[pos] = x_scale[i / k];
+        uint4 *dst = reinterpret_cast<uint4 *>(q.peer_x_loc[e / q.Eg]) + (size_t)pos * q.H8;
+        copy_row16(q.x + (size_t)(i / q.k) * q.H8, dst, q.H8, lane);
+        if (q.x_scale && lane == 0) reinterpret_cast<float *>(q.peer_scale[e / q.Eg])[pos] = q.x_scale[i / q.k];
     }
-    if (bad && lane == 0) atomicOr(status, MOE_DEV_BAD_ROW);
+    if (bad && lane == 0) atomicOr(q.status, MOE_DEV_BAD_ROW);
     __threadfence_system();
+}
+
+// The dispatch after a separate plan (send positions from the workspace).
+__global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(DirPutArgs q, const int32_t *send_base,
+                                                                const int32_t *send_cnt) {
+    pdl_trigger();
+    pdl_wait();
+    put_rows(q, send_base, send_cnt);
+}
+
+// Plan and dispatch in one launch: every block derives this rank's send
+// positions from the gathered counts itself, so the stores start at once;
+// block 0 also lays out this rank's local rows (schedule, return segments,
+// row addresses) for the kernels after the barrier.
+__global__ void __launch_bounds__(kDirThreads) k_ep_direct_plan_put(DirPlanArgs a, DirPutArgs q) {
+    __shared__ DirPlanSmem p;
+    pdl_trigger();
+    pdl_wait();
+    plan_send(a, p);
+    put_rows(q, p.base, p.cnt);
+    if (blockIdx.x == 0) plan_local(a, p);
 }
 
 // Destination side: local row r of segment (s, el) goes to row seg_ysrc +
@@ -287,8 +330,8 @@ const int32_t *ep_direct_local_total(void *ep_ws, const moe_shape &s, int G) {
     return dir_ptrs(ep_ws, s, G).loc_offsets + s.E / G;
 }
 
-cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
-                                  const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream) {
+static DirPlanArgs plan_args(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
+                             const WsLayout &Lloc, void *ws_loc, void *ep_ws) {
     const DirWs p = dir_ptrs(ep_ws, s, G);
     DirPlanArgs a;
     a.cnt_all = cnt_all;
@@ -309,21 +352,55 @@ cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int
     a.H = s.H;
     a.P = s.T * s.k;
     a.lws = ws_ptrs(ws_loc, Lloc);
-    return launch_pdl(k_ep_direct_plan, dim3(1), dim3(kScanThreads), 0, stream, a);
+    return a;
 }
 
 // x: bf16 rows (x_scale null), or e4m3 code rows with their scales.
+static DirPutArgs put_args(const moe_shape &s, int G, const void *x, const int32_t *topk_idx, const int32_t *dest_row,
+                           const int32_t *offsets, const void *peer_x_loc, uint32_t *status, const float *x_scale,
+                           const void *peer_scale) {
+    DirPutArgs q;
+    q.x = (const uint4 *)x;
+    q.topk_idx = topk_idx;
+    q.dest_row = dest_row;
+    q.offsets = offsets;
+    q.peer_x_loc = (const unsigned long long *)peer_x_loc;
+    q.R = s.T * s.k;
+    q.k = s.k;
+    q.E = s.E;
+    q.Eg = s.E / G;
+    q.Tloc = (int)ep_direct_local_rows(s, G);
+    q.H8 = x_scale ? s.H / 16 : s.H / 8;
+    q.status = status;
+    q.x_scale = x_scale;
+    q.peer_scale = (const unsigned long long *)peer_scale;
+    return q;
+}
+
+cudaError_t launch_ep_direct_plan(const moe_shape &s, int G, int rank, const int32_t *cnt_all, const void *peer_y,
+                                  const WsLayout &Lloc, void *ws_loc, void *ep_ws, cudaStream_t stream) {
+    return launch_pdl(k_ep_direct_plan, dim3(1), dim3(kScanThreads), 0, stream,
+                      plan_args(s, G, rank, cnt_all, peer_y, Lloc, ws_loc, ep_ws));
+}
+
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
                                  const int32_t *dest_row, const int32_t *offsets, const void *peer_x_loc,
                                  void *ep_ws, uint32_t *status, int num_sms, cudaStream_t stream,
                                  const float *x_scale, const void *peer_scale) {
     const DirWs p = dir_ptrs(ep_ws, s, G);
-    const int64_t R = (int64_t)s.T * s.k;
-    return launch_pdl(k_ep_direct_put, dim3(dir_grid(R, num_sms)), dim3(kDirThreads), 0, stream, (const uint4 *)x,
-                      topk_idx, dest_row, offsets, (const int32_t *)p.send_base, (const int32_t *)p.send_cnt,
-                      (const unsigned long long *)peer_x_loc, (int)R, s.k, s.E, s.E / G,
-                      (int)ep_direct_local_rows(s, G), x_scale ? s.H / 16 : s.H / 8, status, x_scale,
-                      (const unsigned long long *)peer_scale);
+    return launch_pdl(k_ep_direct_put, dim3(dir_grid((int64_t)s.T * s.k, num_sms)), dim3(kDirThreads), 0, stream,
+                      put_args(s, G, x, topk_idx, dest_row, offsets, peer_x_loc, status, x_scale, peer_scale),
+                      (const int32_t *)p.send_base, (const int32_t *)p.send_cnt);
+}
+
+cudaError_t launch_ep_direct_plan_put(const moe_shape &s, int G, int rank, const int32_t *cnt_all,
+                                      const void *peer_y, const WsLayout &Lloc, void *ws_loc, const void *x,
+                                      const int32_t *topk_idx, const int32_t *dest_row, const int32_t *offsets,
+                                      const void *peer_x_loc, void *ep_ws, uint32_t *status, int num_sms,
+                                      cudaStream_t stream, const float *x_scale, const void *peer_scale) {
+    return launch_pdl(k_ep_direct_plan_put, dim3(dir_grid((int64_t)s.T * s.k, num_sms)), dim3(kDirThreads), 0,
+                      stream, plan_args(s, G, rank, cnt_all, peer_y, Lloc, ws_loc, ep_ws),
+                      put_args(s, G, x, topk_idx, dest_row, offsets, peer_x_loc, status, x_scale, peer_scale));
 }
 
 cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,

@@ -141,6 +141,19 @@ class DirectEP:
         moe.moe_ep_direct_down_return_fp8(self.shape, self.G, self.h_q, self.h_scale, wd_q, wd_scale, self.ws_loc,
                                           self.ep_ws, stream)
 
+    def plan_and_dispatch(self, x, stream=None):
+        """plan() and dispatch() (fp8: dispatch_fp8(), x unused) in one launch."""
+        b = self.b
+        if self.fp8:
+            moe.moe_ep_direct_plan_dispatch(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, self.x_q,
+                                            self.x_scale, b["topk_idx"], b["dest_row"], b["expert_offsets"],
+                                            self.peer_x_loc_q, self.peer_scale_loc, self.ws, self.ws_loc, self.ep_ws,
+                                            stream)
+        else:
+            moe.moe_ep_direct_plan_dispatch(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, x, None,
+                                            b["topk_idx"], b["dest_row"], b["expert_offsets"], self.peer_x_loc,
+                                            None, self.ws, self.ws_loc, self.ep_ws, stream)
+
     def experts(self, w_gate, w_up, w_down, stream=None):
         """The grouped GEMMs of this rank's experts on the rows it received."""
         L = self.local
@@ -210,8 +223,7 @@ class DirectEP:
 
         self.route(x, w_router, bias)
         self.gather_counts(lambda out, inp: dist.all_gather_into_tensor(out, inp, group=group))
-        self.plan()
-        self.dispatch(x)
+        self.plan_and_dispatch(x)
         barrier()
         if fused_return:
             self.experts_and_return(w_gate, w_up, w_down)
@@ -234,8 +246,7 @@ class DirectEP:
         self.route(x, w_router, bias)
         self.quantize_tokens(x)
         self.gather_counts(lambda out, inp: dist.all_gather_into_tensor(out, inp, group=group))
-        self.plan()
-        self.dispatch_fp8()
+        self.plan_and_dispatch(x)
         barrier()
         self.experts_fp8_and_return(wg_q, wg_scale, wu_q, wu_scale, wd_q, wd_scale)
         barrier()

@@ -542,6 +542,20 @@ MOE_API moe_status moe_ep_direct_local_shape(const moe_shape *shape, int32_t G, 
 MOE_API moe_status moe_ep_direct_plan(const moe_shape *shape, int32_t G, int32_t rank, const int32_t *cnt_all,
                                       const void *peer_y, void *ws_loc, void *ep_ws, void *stream);
 
+/* Steps 3 and 4 in one launch (the form the layer uses): every block of the
+ * dispatch derives this rank's send positions from cnt_all itself, so the
+ * stores start at once, and one block also lays out the local rows as
+ * moe_ep_direct_plan does.  x_scale null: x is bf16 [T,H] and peer_x_loc the
+ * owners' x_loc; else x holds e4m3 codes [T,H] with scales x_scale [T], and
+ * peer_x_loc / peer_scale_loc the owners' x_loc_q / scale_loc (the fp8 form).
+ * ws: the rank's routing workspace; ws_loc: its local workspace. */
+MOE_API moe_status moe_ep_direct_plan_dispatch(const moe_shape *shape, int32_t G, int32_t rank,
+                                               const int32_t *cnt_all, const void *peer_y, const void *x,
+                                               const float *x_scale, const int32_t *topk_idx, const int32_t *dest_row,
+                                               const int32_t *expert_offsets, const void *peer_x_loc,
+                                               const void *peer_scale_loc, void *ws, void *ws_loc, void *ep_ws,
+                                               void *stream);
+
 /* Step 4 (ws: the rank's routing workspace, for its status word). */
 MOE_API moe_status moe_ep_direct_dispatch(const moe_shape *shape, int32_t G, const void *x, const int32_t *topk_idx,
                                           const int32_t *dest_row, const int32_t *expert_offsets,

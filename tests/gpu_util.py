@@ -205,9 +205,10 @@ def run_cap_and_spill_ep(dl, shape, G):
     return ranks, xs
 
 
-def run_direct_ep(dl, shape, G, fused_return=False):
+def run_direct_ep(dl, shape, G, fused_return=False, fused_plan=False):
     """The peer-store expert-parallel layer on G ranks held by this process
-    (fused_return: the down GEMM stores its results into the owners' y)."""
+    (fused_return: the down GEMM stores its results into the owners' y;
+    fused_plan: plan and dispatch in one launch)."""
     from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
     T, Eg = shape.T, shape.E // G
     ranks = [DirectEP(shape, G, r) for r in range(G)]
@@ -216,10 +217,14 @@ def run_direct_ep(dl, shape, G, fused_return=False):
     for r, ep in enumerate(ranks):
         ep.route(xs[r], dl.w_router, dl.bias)
     gather_counts_in_process(ranks)
-    for ep in ranks:
-        ep.plan()
-    for r, ep in enumerate(ranks):
-        ep.dispatch(xs[r])
+    if fused_plan:
+        for r, ep in enumerate(ranks):
+            ep.plan_and_dispatch(xs[r])
+    else:
+        for ep in ranks:
+            ep.plan()
+        for r, ep in enumerate(ranks):
+            ep.dispatch(xs[r])
     for r, ep in enumerate(ranks):
         sl = slice(r * Eg, (r + 1) * Eg)
         if fused_return:
@@ -235,7 +240,7 @@ def run_direct_ep(dl, shape, G, fused_return=False):
     return ranks, xs
 
 
-def run_direct_ep_fp8(dl, shape, G, wq):
+def run_direct_ep_fp8(dl, shape, G, wq, fused_plan=True):
     """The fp8 peer-store layer on G ranks held by this process: each rank
     quantizes its tokens, stores code rows and scales into the owners'
     buffers, runs the fp8 GEMMs on its experts (wq: the layer's weight codes
@@ -250,10 +255,14 @@ def run_direct_ep_fp8(dl, shape, G, wq):
         ep.route(xs[r], dl.w_router, dl.bias)
         ep.quantize_tokens(xs[r])
     gather_counts_in_process(ranks)
-    for ep in ranks:
-        ep.plan()
-    for ep in ranks:
-        ep.dispatch_fp8()
+    if fused_plan:
+        for r, ep in enumerate(ranks):
+            ep.plan_and_dispatch(xs[r])
+    else:
+        for ep in ranks:
+            ep.plan()
+        for ep in ranks:
+            ep.dispatch_fp8()
     for r, ep in enumerate(ranks):
         sl = slice(r * Eg, (r + 1) * Eg)
         ep.experts_fp8_and_return(wq["wg_q"][sl], wq["wg_scale"][sl], wq["wu_q"][sl], wq["wu_scale"][sl],

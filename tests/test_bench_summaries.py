@@ -48,7 +48,7 @@ def test_two_pass_summary():
 
 def test_peer_store_summary_and_bound():
     G = 8
-    phases = {"route": 80.0, "plan": 40.0, "dispatch": 48.0, "experts_swiglu": 1600.0, "experts_down": 1200.0,
+    phases = {"route": 80.0, "plan_dispatch": 88.0, "experts_swiglu": 1600.0, "experts_down": 1200.0,
               "send_back": 120.0, "down_return_fused": 1240.0, "finish": 64.0}
     e = {"G": G, "per_phase_us_all_ranks": phases, "device_status": [0] * G, "single_gpu_layer_us": 500.0}
     cfg = synth.CONFIGS[2]  # one expert per rank: the local GEMMs are tensor-bound
@@ -68,7 +68,7 @@ def test_peer_store_summary_and_bound():
 
 def test_peer_store_fp8_summary():
     G = 8
-    phases = {"route": 80.0, "quantize_tokens": 24.0, "plan": 40.0, "dispatch": 40.0, "experts_swiglu": 160.0,
+    phases = {"route": 80.0, "quantize_tokens": 24.0, "plan_dispatch": 80.0, "experts_swiglu": 160.0,
               "quantize_h": 32.0, "down_return_fused": 120.0, "finish": 64.0}
     e = {"G": G, "fp8": True, "per_phase_us_all_ranks": phases, "device_status": [0] * G,
          "single_gpu_layer_us": 150.0}

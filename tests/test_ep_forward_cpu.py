@@ -6,7 +6,7 @@ Two-pass form: two gloo ranks run the real forward(); the stand-in "experts"
 send every received row straight back, so after the two return passes each
 rank's y capacity rows and overflow slots must hold exactly the rows it sent
 (the exchange is its own inverse).  Peer-store form: a recorded run checks the
-order of phases and collectives (counts all-gather, plan, dispatch, barrier,
+order of phases and collectives (counts all-gather, plan and dispatch, barrier,
 experts with the fused return, barrier, combine)."""
 import os
 import socket
@@ -80,13 +80,14 @@ def test_peer_store_forward_order(monkeypatch):
     import torch.distributed as dist
     ep = DirectEP(moe.make_shape(40, 128, 128, 16, 3), G, 1, device="cpu")
     calls = []
-    for name in ("route", "plan", "dispatch", "experts", "experts_and_return", "send_back", "finish"):
+    for name in ("route", "plan_and_dispatch", "experts", "experts_and_return", "send_back", "finish"):
         monkeypatch.setattr(ep, name, (lambda n: (lambda *a, **k: calls.append(n)))(name))
     monkeypatch.setattr(dist, "all_gather_into_tensor", lambda out, inp, group=None: calls.append("all_gather"))
     monkeypatch.setattr(dist, "all_reduce", lambda t, group=None: calls.append("barrier"))
     ep._flag, ep._group = torch.zeros(1, dtype=torch.int32), None
     ep.forward(None, None, None, None, None, None)
-    assert calls == ["route", "all_gather", "plan", "dispatch", "barrier", "experts_and_return", "barrier", "finish"]
+    assert calls == ["route", "all_gather", "plan_and_dispatch", "barrier", "experts_and_return", "barrier", "finish"]
     calls.clear()
     ep.forward(None, None, None, None, None, None, fused_return=False)
-    assert calls == ["route", "all_gather", "plan", "dispatch", "barrier", "experts", "send_back", "barrier", "finish"]
+    assert calls == ["route", "all_gather", "plan_and_dispatch", "barrier", "experts", "send_back", "barrier",
+                     "finish"]

@@ -73,7 +73,7 @@ def test_direct_ep_matches_single_gpu_and_oracle(orc, name, G, fused_return):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct_ep(dl, shape, G, fused_return)
+    ranks, xs = run_direct_ep(dl, shape, G, fused_return, fused_plan=fused_return)
     for ep in ranks:
         assert moe.moe_read_status(ep.ws) == 0
         assert moe.moe_read_status(ep.ws_loc) == 0
@@ -97,7 +97,7 @@ def test_direct_ep_full_size_mixtral_matches_single_gpu(G, fused_return):
     L = synth.make_layer(cfg.with_(T=cfg.T * G))
     dl = DeviceLayer(L)
     shape = _shape(cfg)
-    ranks, xs = run_direct_ep(dl, shape, G, fused_return)
+    ranks, xs = run_direct_ep(dl, shape, G, fused_return, fused_plan=fused_return)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])
@@ -147,9 +147,10 @@ def test_direct_ep_rejects_unsupported_shapes():
         DirectEP(_shape(cfg), 2, 2)  # rank out of range
 
 
+@pytest.mark.parametrize("fused_plan", [True, False], ids=["plan_dispatch", "plan_then_dispatch"])
 @pytest.mark.parametrize("name,G", [("decode_E64_k6", 8), ("E16_k4_F384", 4), ("E8_k2_skew", 2),
                                     ("several_tiles_E4_k2", 2)], ids=lambda v: str(v))
-def test_direct_ep_fp8_matches_single_gpu_fp8(name, G):
+def test_direct_ep_fp8_matches_single_gpu_fp8(name, G, fused_plan):
     """e4m3 rows on the links: each rank's out equals moe_forward_fp8 on its
     tokens bit for bit (per-row token codes and scales are the same whichever
     rank quantizes them; the same fp8 GEMM arithmetic on the same rows)."""
@@ -160,7 +161,7 @@ def test_direct_ep_fp8_matches_single_gpu_fp8(name, G):
     wq = dl.bufs(shape)
     wq.update(moe.alloc_fp8_buffers(shape))
     moe.quantize_layer_weights_fp8(shape, wq)
-    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq)
+    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq, fused_plan)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         b = dl.bufs(shape)

@@ -84,7 +84,7 @@ def test_random_expert_parallel_matches_single_gpu(cfg, G):
         ranks, xs = run_cap_and_spill_ep(dl, shape, G)
     else:
         shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
-        ranks, xs = run_direct_ep(dl, shape, G, fused_return=bool(cfg.seed % 2))
+        ranks, xs = run_direct_ep(dl, shape, G, fused_return=bool(cfg.seed % 2), fused_plan=bool(cfg.T % 2))
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         b = dl.bufs(shape)
