@@ -104,7 +104,8 @@ def test_direct_ep_full_size_mixtral_matches_single_gpu(G, fused_return):
         assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(ref["out"])), "rank %d" % r
 
 
-def test_direct_ep_clamps_counts_beyond_the_buffers():
+@pytest.mark.parametrize("fused_plan", [False, True], ids=["plan_then_dispatch", "plan_dispatch"])
+def test_direct_ep_clamps_counts_beyond_the_buffers(fused_plan):
     """Gathered counts past what the buffers hold (a source claiming more
     rows than it can send) are clamped the same way on every rank: nothing
     is stored outside a buffer, MOE_DEV_BAD_ROW is raised, and a clean layer
@@ -122,15 +123,20 @@ def test_direct_ep_clamps_counts_beyond_the_buffers():
     for ep in ranks:
         ep.cnt_all[0, 3] = 1 << 24  # more than T pairs for one expert
         ep.cnt_all[1, :] = cfg.T    # more rows than one source can send a rank
-        ep.plan()
-    torch.cuda.synchronize()
     for r, ep in enumerate(ranks):
-        ep.dispatch(dl.x[r * cfg.T:(r + 1) * cfg.T])
+        if fused_plan:
+            ep.plan_and_dispatch(dl.x[r * cfg.T:(r + 1) * cfg.T])
+        else:
+            ep.plan()
+    torch.cuda.synchronize()
+    if not fused_plan:
+        for r, ep in enumerate(ranks):
+            ep.dispatch(dl.x[r * cfg.T:(r + 1) * cfg.T])
     torch.cuda.synchronize()
     assert all(moe.moe_read_status(ep.ws_loc) & moe.MOE_DEV_BAD_ROW for ep in ranks)
     for ep in ranks:
         moe.moe_read_status(ep.ws)  # clear
-    ranks2, xs = run_direct_ep(dl, shape, G)
+    ranks2, xs = run_direct_ep(dl, shape, G, fused_plan=fused_plan)
     for r, ep in enumerate(ranks2):
         assert moe.moe_read_status(ep.ws_loc) == 0
         ref = _single_gpu(dl, shape, xs[r])
