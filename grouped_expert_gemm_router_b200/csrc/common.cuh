@@ -230,6 +230,21 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
 // ------------------------------------------------------------ device helpers --
 #if defined(__CUDACC__)
 
+// One row of H8 16-byte vectors copied by one warp, eight loads per lane in
+// flight before their stores (one memory round trip per 4 KB of row).
+__device__ __forceinline__ void copy_row_warp(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8,
+                                              int lane) {
+    int v = lane;
+    for (; v + 224 < H8; v += 256) {
+        uint4 q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __ldg(src + v + 32 * i);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[v + 32 * i] = q[i];
+    }
+    for (; v < H8; v += 32) dst[v] = __ldg(src + v);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

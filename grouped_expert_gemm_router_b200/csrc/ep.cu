@@ -38,11 +38,6 @@ namespace {
 constexpr int kRowThreads = 256;
 constexpr int kRowWarps = kRowThreads / 32;
 
-// One row of H8 16-byte vectors, by one warp.
-__device__ __forceinline__ void copy_row(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8, int lane) {
-    for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
-}
-
 // Overflow row q of x_perm (row E C + q) belongs to destination d, the last
 // with starts[d * stride] <= q, and sits at row d S + (q - starts[d * stride])
 // of the slots.  pack (reverse = 0): a = x_perm, b = send slots, b <- a, and
@@ -83,9 +78,9 @@ __global__ void __launch_bounds__(kRowThreads) k_ep_spill_rows(WsPtrs ws, const 
         }
         uint4 *ra = a + (size_t)(E * C + q) * H8, *rb = b + (size_t)(lo * S + j) * H8;
         if (reverse)
-            copy_row(rb, ra, H8, lane);
+            copy_row_warp(rb, ra, H8, lane);
         else
-            copy_row(ra, rb, H8, lane);
+            copy_row_warp(ra, rb, H8, lane);
     }
 }
 
@@ -178,9 +173,9 @@ __global__ void __launch_bounds__(kRowThreads) k_ep_local_rows(const int32_t *ro
         uint4 *rx = src >= 0 ? cap + (size_t)src * H8 : ovf + (size_t)(-1 - src) * H8;
         uint4 *rl = loc + (size_t)r * H8;
         if (reverse)
-            copy_row(rl, rx, H8, lane);
+            copy_row_warp(rl, rx, H8, lane);
         else
-            copy_row(rx, rl, H8, lane);
+            copy_row_warp(rx, rl, H8, lane);
     }
 }
 

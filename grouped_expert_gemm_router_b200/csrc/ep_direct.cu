@@ -43,10 +43,6 @@ namespace {
 constexpr int kDirThreads = 256;
 constexpr int kDirWarps = kDirThreads / 32;
 
-__device__ __forceinline__ void copy_row16(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8, int lane) {
-    for (int v = lane; v < H8; v += 32) dst[v] = __ldg(src + v);
-}
-
 // At most kDirMaxCounts (source, expert) counts; the return kernel keeps up
 // to kDirSmemSegs segment starts in shared memory.
 constexpr int kDirMaxCounts = 4096;
@@ -207,7 +203,7 @@ __device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt) {
             continue;
         }
         uint4 *dst = reinterpret_cast<uint4 *>(q.peer_x_loc[e / q.Eg]) + (size_t)pos * q.H8;
-        copy_row16(q.x + (size_t)(i / q.k) * q.H8, dst, q.H8, lane);
+        copy_row_warp(q.x + (size_t)(i / q.k) * q.H8, dst, q.H8, lane);
         if (q.x_scale && lane == 0) reinterpret_cast<float *>(q.peer_scale[e / q.Eg])[pos] = q.x_scale[i / q.k];
     }
     if (bad && lane == 0) atomicOr(q.status, MOE_DEV_BAD_ROW);
@@ -273,7 +269,7 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_return(const uint4 *y
         const int yrow = seg_ysrc[i] + j;
         if (j >= seg_cnt[i] || (unsigned)yrow >= (unsigned)P) continue;  // cannot happen: the plan's layout
         uint4 *dst = reinterpret_cast<uint4 *>(peer_y[lo]) + (size_t)yrow * H8;
-        copy_row16(y_loc + (size_t)r * H8, dst, H8, lane);
+        copy_row_warp(y_loc + (size_t)r * H8, dst, H8, lane);
     }
     __threadfence_system();
 }
