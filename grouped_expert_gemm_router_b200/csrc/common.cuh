@@ -230,6 +230,14 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
 // ------------------------------------------------------------ device helpers --
 #if defined(__CUDACC__)
 
+// End of a block's stores into other GPUs' memory: a block barrier (every
+// thread's stores happen before it), then one system-scope fence by thread 0,
+// which is cumulative over them.  All threads of the block call it.
+__device__ __forceinline__ void fence_block_stores_system() {
+    __syncthreads();
+    if (threadIdx.x == 0) __threadfence_system();
+}
+
 // One row of H8 16-byte vectors copied by one warp, eight loads per lane in
 // flight before their stores (one memory round trip per 4 KB of row).
 __device__ __forceinline__ void copy_row_warp(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int H8,

@@ -26,12 +26,14 @@
 // k_ep_direct_put     source: a warp per routed pair, x[t] -> the
 //                     destination's x_loc row.
 // k_ep_direct_plan_put  both in one launch: every block derives the send
-//                     positions itself, block 0 also lays out the local rows.
+//                     positions itself; one extra block lays out the local
+//                     rows while the others store.
 // k_ep_direct_return  destination: a warp per local row, y_loc -> the
 //                     source's y row.
-// Each put kernel ends with a system-scope fence, so a stream-ordered
-// collective after it (a barrier) orders its peer stores before any later
-// work on every rank.
+// Every block of a kernel that stores into peer memory ends with a block
+// barrier and one system-scope fence (cumulative over the block's stores), so
+// a stream-ordered collective after it (a barrier) orders its peer stores
+// before any later work on every rank.
 #include <cuda_bf16.h>
 
 #include "dispatch_block.cuh"
@@ -190,13 +192,33 @@ struct DirPutArgs {
     const unsigned long long *peer_scale;
 };
 
-__device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt) {
+// A routed pair's expert (-1 past the end or for an id the router reported)
+// and its rank among the expert's pairs on this rank.
+struct PairRef {
+    int e, ri;
+};
+__device__ __forceinline__ PairRef load_pair(const DirPutArgs &q, int i) {
+    PairRef r = {-1, 0};
+    if (i < q.R) {
+        const int e = q.topk_idx[i];
+        if ((unsigned)e < (unsigned)q.E) {
+            r.e = e;
+            r.ri = q.dest_row[i] - q.offsets[e];
+        }
+    }
+    return r;
+}
+
+// Blocks [0, nblocks) of the grid share the pairs, a warp per pair; `first`
+// is the warp's first pair, loaded by the caller.
+__device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt, int nblocks, PairRef first) {
     const int lane = threadIdx.x & 31;
     bool bad = false;
-    for (int i = blockIdx.x * kDirWarps + (threadIdx.x >> 5); i < q.R; i += gridDim.x * kDirWarps) {
-        const int e = q.topk_idx[i];
-        if ((unsigned)e >= (unsigned)q.E) continue;  // reported by the router
-        const int ri = q.dest_row[i] - q.offsets[e];
+    PairRef pr = first;
+    for (int i = blockIdx.x * kDirWarps + (threadIdx.x >> 5); i < q.R; i += nblocks * kDirWarps) {
+        if (i != blockIdx.x * kDirWarps + (threadIdx.x >> 5)) pr = load_pair(q, i);
+        const int e = pr.e, ri = pr.ri;
+        if (e < 0) continue;  // reported by the router
         const int pos = base[e] + ri;
         if (ri < 0 || ri >= cnt[e] || (unsigned)pos >= (unsigned)q.Tloc) {
             bad = true;
@@ -207,7 +229,7 @@ __device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt) {
         if (q.x_scale && lane == 0) reinterpret_cast<float *>(q.peer_scale[e / q.Eg])[pos] = q.x_scale[i / q.k];
     }
     if (bad && lane == 0) atomicOr(q.status, MOE_DEV_BAD_ROW);
-    __threadfence_system();
+    fence_block_stores_system();
 }
 
 // The dispatch after a separate plan (send positions from the workspace).
@@ -215,20 +237,25 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_put(DirPutArgs q, con
                                                                 const int32_t *send_cnt) {
     pdl_trigger();
     pdl_wait();
-    put_rows(q, send_base, send_cnt);
+    put_rows(q, send_base, send_cnt, (int)gridDim.x, load_pair(q, blockIdx.x * kDirWarps + (threadIdx.x >> 5)));
 }
 
 // Plan and dispatch in one launch: every block derives this rank's send
-// positions from the gathered counts itself, so the stores start at once;
-// block 0 also lays out this rank's local rows (schedule, return segments,
-// row addresses) for the kernels after the barrier.
+// positions from the gathered counts itself (its warps' first pairs loaded
+// meanwhile), so the stores start at once; the last block instead lays out
+// this rank's local rows (schedule, return segments, row addresses) for the
+// kernels after the barrier, alongside the stores.
 __global__ void __launch_bounds__(kDirThreads) k_ep_direct_plan_put(DirPlanArgs a, DirPutArgs q) {
     __shared__ DirPlanSmem p;
     pdl_trigger();
     pdl_wait();
+    const bool planner = blockIdx.x == gridDim.x - 1;
+    const PairRef first = planner ? PairRef{-1, 0} : load_pair(q, blockIdx.x * kDirWarps + (threadIdx.x >> 5));
     plan_send(a, p);
-    put_rows(q, p.base, p.cnt);
-    if (blockIdx.x == 0) plan_local(a, p);
+    if (planner)
+        plan_local(a, p);
+    else
+        put_rows(q, p.base, p.cnt, (int)gridDim.x - 1, first);
 }
 
 // Destination side: local row r of segment (s, el) goes to row seg_ysrc +
@@ -271,7 +298,7 @@ __global__ void __launch_bounds__(kDirThreads) k_ep_direct_return(const uint4 *y
         uint4 *dst = reinterpret_cast<uint4 *>(peer_y[lo]) + (size_t)yrow * H8;
         copy_row_warp(y_loc + (size_t)r * H8, dst, H8, lane);
     }
-    __threadfence_system();
+    fence_block_stores_system();
 }
 
 int dir_grid(int64_t rows, int num_sms) {
@@ -394,7 +421,7 @@ cudaError_t launch_ep_direct_plan_put(const moe_shape &s, int G, int rank, const
                                       const int32_t *topk_idx, const int32_t *dest_row, const int32_t *offsets,
                                       const void *peer_x_loc, void *ep_ws, uint32_t *status, int num_sms,
                                       cudaStream_t stream, const float *x_scale, const void *peer_scale) {
-    return launch_pdl(k_ep_direct_plan_put, dim3(dir_grid((int64_t)s.T * s.k, num_sms)), dim3(kDirThreads), 0,
+    return launch_pdl(k_ep_direct_plan_put, dim3(dir_grid((int64_t)s.T * s.k, num_sms) + 1), dim3(kDirThreads), 0,
                       stream, plan_args(s, G, rank, cnt_all, peer_y, Lloc, ws_loc, ep_ws),
                       put_args(s, G, x, topk_idx, dest_row, offsets, peer_x_loc, status, x_scale, peer_scale));
 }

@@ -1092,6 +1092,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    // Results stored into other GPUs' memory (row addresses): one
+    // system-scope fence, cumulative over the block's stores, before the
+    // collective that follows the kernel.
+    if (MODE == 1 && a.row_addr && threadIdx.x == 0) __threadfence_system();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);

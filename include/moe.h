@@ -518,7 +518,9 @@ MOE_API moe_status moe_ep_unpack(const moe_shape *shape, int32_t G, const void *
  * peer_x_loc, peer_y: DEVICE arrays of G pointers (uint64), entry d = rank
  * d's x_loc / y as this rank's kernels address it (its own entry included).
  * x_loc holds moe_ep_direct_local_rows rows; y is moe_forward's y (T*k rows).
- * The put kernels end with a system-scope fence.  ep_ws:
+ * Every kernel that stores into peer memory (the puts, the return, the down
+ * projection with its return) ends each block with a block barrier and one
+ * system-scope fence.  ep_ws:
  * moe_ep_direct_workspace_bytes bytes, written by the plan, read by the two
  * puts of the same layer.  Errors as for the Cap-and-Spill calls; counts in
  * cnt_all beyond what the buffers hold (each (source, expert) above T, each
