@@ -684,12 +684,11 @@ class Bench:
 
         if fp8:
             L_ = ranks[0].local
-            phases = ("route", "quantize_tokens", "plan_dispatch", "experts_swiglu", "quantize_h",
-                      "down_return_fused", "finish")
+            phases = ("route", "plan_dispatch_quantize", "experts_swiglu", "quantize_h", "down_return_fused",
+                      "finish")
             calls = {
                 "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
-                "quantize_tokens": lambda r: ranks[r].quantize_tokens(xs[r], stream),
-                "plan_dispatch": lambda r: ranks[r].plan_and_dispatch(None, stream),
+                "plan_dispatch_quantize": lambda r: ranks[r].plan_and_dispatch(xs[r], stream),
                 "experts_swiglu": lambda r: moe.moe_grouped_swiglu_fp8(
                     L_, ranks[r].x_loc_q, ranks[r].scale_loc, None, wq["wg_q"][sl[r]], wq["wg_scale"][sl[r]],
                     wq["wu_q"][sl[r]], wq["wu_scale"][sl[r]], ranks[r].h_loc, ranks[r].ws_loc, stream),
@@ -704,7 +703,7 @@ class Bench:
         def step(timed):
             ev = {}
             for ph in phases:
-                if ph in ("plan", "plan_dispatch"):
+                if ph.startswith("plan"):
                     gather_counts_in_process(ranks)
                 for r in range(G):
                     if timed:

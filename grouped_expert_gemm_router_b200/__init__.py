@@ -43,6 +43,7 @@ ABI_FUNCTIONS = (
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
     "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
     "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h", "moe_ep_direct_plan_dispatch",
+    "moe_ep_direct_plan_dispatch_quantize",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -183,6 +184,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_direct_quantize_h.restype = st
     lib.moe_ep_direct_plan_dispatch.argtypes = [sp, i32, i32] + [vp] * 13
     lib.moe_ep_direct_plan_dispatch.restype = st
+    lib.moe_ep_direct_plan_dispatch_quantize.argtypes = [sp, i32, i32] + [vp] * 12
+    lib.moe_ep_direct_plan_dispatch_quantize.restype = st
     _lib = lib
     return lib
 
@@ -570,4 +573,13 @@ def moe_ep_direct_plan_dispatch(shape, G, rank, cnt_all, peer_y, x, x_scale, top
         ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(peer_y), _ptr(x), _ptr(x_scale), _ptr(topk_idx),
         _ptr(dest_row), _ptr(expert_offsets), _ptr(peer_x_loc), _ptr(peer_scale_loc), _ptr(ws), _ptr(ws_loc),
         _ptr(ep_ws), _stream(stream)), "moe_ep_direct_plan_dispatch")
+
+
+def moe_ep_direct_plan_dispatch_quantize(shape, G, rank, cnt_all, peer_y, x, topk_idx, dest_row, expert_offsets,
+                                         peer_x_loc_q, peer_scale_loc, ws, ws_loc, ep_ws, stream=None):
+    """x: bf16 token rows, quantized to e4m3 rows on the way to the owners."""
+    _check(load_library().moe_ep_direct_plan_dispatch_quantize(
+        ctypes.byref(shape), int(G), int(rank), _ptr(cnt_all), _ptr(peer_y), _ptr(x), _ptr(topk_idx), _ptr(dest_row),
+        _ptr(expert_offsets), _ptr(peer_x_loc_q), _ptr(peer_scale_loc), _ptr(ws), _ptr(ws_loc), _ptr(ep_ws),
+        _stream(stream)), "moe_ep_direct_plan_dispatch_quantize")
 

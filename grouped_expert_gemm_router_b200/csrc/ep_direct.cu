@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 
 #include "dispatch_block.cuh"
+#include "fp8_rows.cuh"
 
 namespace moe {
 
@@ -190,7 +191,40 @@ struct DirPutArgs {
     uint32_t *status;
     const float *x_scale;
     const unsigned long long *peer_scale;
+    int quantize;  // x: bf16 rows, quantized on the way (codes and scale into peer_x_loc / peer_scale)
 };
+
+// One bf16 row of H8 16-byte vectors stored as e4m3 codes (H8 8-byte groups)
+// with its scale, by one warp, exactly as the row quantizer does it: the
+// row's largest magnitude (eight loads per lane in flight), then the codes
+// from a second read of the row, which comes from L1 or L2.
+__device__ __forceinline__ void put_row_quantized(const uint4 *__restrict__ src, uint2 *__restrict__ dst, int H8,
+                                                  int lane, float *scale_dst) {
+    __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+    int v = lane;
+    for (; v + 224 < H8; v += 256) {
+        uint4 t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = __ldg(src + v + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m2 = amax8(t[j], m2);
+    }
+    for (; v < H8; v += 32) m2 = amax8(__ldg(src + v), m2);
+    float m = amax_of(m2);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const Fp8Scale sc = fp8_scale(m);
+    v = lane;
+    for (; v + 224 < H8; v += 256) {
+        uint4 t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = __ldg(src + v + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[v + 32 * j] = quant8(t[j], sc);
+    }
+    for (; v < H8; v += 32) dst[v] = quant8(__ldg(src + v), sc);
+    if (lane == 0) *scale_dst = sc.s;
+}
 
 // A routed pair's expert (-1 past the end or for an id the router reported)
 // and its rank among the expert's pairs on this rank.
@@ -222,6 +256,12 @@ __device__ void put_rows(const DirPutArgs &q, const int *base, const int *cnt, i
         const int pos = base[e] + ri;
         if (ri < 0 || ri >= cnt[e] || (unsigned)pos >= (unsigned)q.Tloc) {
             bad = true;
+            continue;
+        }
+        if (q.quantize) {
+            put_row_quantized(q.x + (size_t)(i / q.k) * q.H8,
+                              reinterpret_cast<uint2 *>(q.peer_x_loc[e / q.Eg]) + (size_t)pos * q.H8, q.H8, lane,
+                              reinterpret_cast<float *>(q.peer_scale[e / q.Eg]) + pos);
             continue;
         }
         uint4 *dst = reinterpret_cast<uint4 *>(q.peer_x_loc[e / q.Eg]) + (size_t)pos * q.H8;
@@ -381,7 +421,7 @@ static DirPlanArgs plan_args(const moe_shape &s, int G, int rank, const int32_t 
 // x: bf16 rows (x_scale null), or e4m3 code rows with their scales.
 static DirPutArgs put_args(const moe_shape &s, int G, const void *x, const int32_t *topk_idx, const int32_t *dest_row,
                            const int32_t *offsets, const void *peer_x_loc, uint32_t *status, const float *x_scale,
-                           const void *peer_scale) {
+                           const void *peer_scale, bool quantize = false) {
     DirPutArgs q;
     q.x = (const uint4 *)x;
     q.topk_idx = topk_idx;
@@ -397,6 +437,7 @@ static DirPutArgs put_args(const moe_shape &s, int G, const void *x, const int32
     q.status = status;
     q.x_scale = x_scale;
     q.peer_scale = (const unsigned long long *)peer_scale;
+    q.quantize = quantize ? 1 : 0;  // H8 = H / 8: bf16 vectors in, 8-byte code groups out
     return q;
 }
 
@@ -420,10 +461,12 @@ cudaError_t launch_ep_direct_plan_put(const moe_shape &s, int G, int rank, const
                                       const void *peer_y, const WsLayout &Lloc, void *ws_loc, const void *x,
                                       const int32_t *topk_idx, const int32_t *dest_row, const int32_t *offsets,
                                       const void *peer_x_loc, void *ep_ws, uint32_t *status, int num_sms,
-                                      cudaStream_t stream, const float *x_scale, const void *peer_scale) {
+                                      cudaStream_t stream, const float *x_scale, const void *peer_scale,
+                                      bool quantize) {
     return launch_pdl(k_ep_direct_plan_put, dim3(dir_grid((int64_t)s.T * s.k, num_sms) + 1), dim3(kDirThreads), 0,
                       stream, plan_args(s, G, rank, cnt_all, peer_y, Lloc, ws_loc, ep_ws),
-                      put_args(s, G, x, topk_idx, dest_row, offsets, peer_x_loc, status, x_scale, peer_scale));
+                      put_args(s, G, x, topk_idx, dest_row, offsets, peer_x_loc, status, quantize ? nullptr : x_scale,
+                               peer_scale, quantize));
 }
 
 cudaError_t launch_ep_direct_return(const moe_shape &s, int G, const void *y_loc, const void *peer_y, void *ep_ws,

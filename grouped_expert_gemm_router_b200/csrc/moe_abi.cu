@@ -59,7 +59,8 @@ cudaError_t launch_ep_direct_plan_put(const moe_shape &s, int G, int rank, const
                                       const void *peer_y, const WsLayout &Lloc, void *ws_loc, const void *x,
                                       const int32_t *topk_idx, const int32_t *dest_row, const int32_t *offsets,
                                       const void *peer_x_loc, void *ep_ws, uint32_t *status, int num_sms,
-                                      cudaStream_t stream, const float *x_scale, const void *peer_scale);
+                                      cudaStream_t stream, const float *x_scale, const void *peer_scale,
+                                      bool quantize);
 cudaError_t launch_quant_rows_counted(const void *src, int K, int rows_cap, const int *rows_dev, void *q,
                                       float *scale, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_direct_put(const moe_shape &s, int G, const void *x, const int32_t *topk_idx,
@@ -792,7 +793,32 @@ moe_status moe_ep_direct_plan_dispatch(const moe_shape *s, int32_t G, int32_t ra
     uint32_t *status = (uint32_t *)((char *)ws + L.status);
     cudaError_t e = launch_ep_direct_plan_put(*s, G, rank, cnt_all, peer_y, Lloc, ws_loc, x, topk_idx, dest_row,
                                               expert_offsets, peer_x_loc, ep_ws, status, sms, (cudaStream_t)stream,
-                                              x_scale, x_scale ? peer_scale_loc : nullptr);
+                                              x_scale, x_scale ? peer_scale_loc : nullptr, false);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_plan_dispatch");
+}
+
+moe_status moe_ep_direct_plan_dispatch_quantize(const moe_shape *s, int32_t G, int32_t rank, const int32_t *cnt_all,
+                                                const void *peer_y, const void *x, const int32_t *topk_idx,
+                                                const int32_t *dest_row, const int32_t *expert_offsets,
+                                                const void *peer_x_loc_q, const void *peer_scale_loc, void *ws,
+                                                void *ws_loc, void *ep_ws, void *stream) {
+    moe_status st = check_ep_direct(s, G);
+    if (st != MOE_OK) return st;
+    if (rank < 0 || rank >= G) return MOE_ERR_INVALID_ARG;
+    if (!aligned(cnt_all, 4) || (peer_y && !aligned(peer_y, 8)) || !aligned(x, 16) || !aligned(topk_idx, 4) ||
+        !aligned(dest_row, 4) || !aligned(expert_offsets, 4) || !aligned(peer_x_loc_q, 8) ||
+        !aligned(peer_scale_loc, 8) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK || (st = check_ws(ws_loc)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    const moe_shape l = ep_direct_local(s, G);
+    const WsLayout Lloc = layout_of(&l);
+    uint32_t *status = (uint32_t *)((char *)ws + L.status);
+    cudaError_t e = launch_ep_direct_plan_put(*s, G, rank, cnt_all, peer_y, Lloc, ws_loc, x, topk_idx, dest_row,
+                                              expert_offsets, peer_x_loc_q, ep_ws, status, sms, (cudaStream_t)stream,
+                                              nullptr, peer_scale_loc, true);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_direct_plan_dispatch_quantize");
 }
 

@@ -142,13 +142,20 @@ class DirectEP:
                                           self.ep_ws, stream)
 
     def plan_and_dispatch(self, x, stream=None):
-        """plan() and dispatch() (fp8: dispatch_fp8(), x unused) in one launch."""
+        """plan() and dispatch() in one launch.  fp8: x None sends the code
+        rows quantize_tokens() left (dispatch_fp8()); x given (bf16 token
+        rows) is quantized on the way, by the warps that send its rows."""
         b = self.b
-        if self.fp8:
+        if self.fp8 and x is None:
             moe.moe_ep_direct_plan_dispatch(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, self.x_q,
                                             self.x_scale, b["topk_idx"], b["dest_row"], b["expert_offsets"],
                                             self.peer_x_loc_q, self.peer_scale_loc, self.ws, self.ws_loc, self.ep_ws,
                                             stream)
+        elif self.fp8:
+            moe.moe_ep_direct_plan_dispatch_quantize(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, x,
+                                                     b["topk_idx"], b["dest_row"], b["expert_offsets"],
+                                                     self.peer_x_loc_q, self.peer_scale_loc, self.ws, self.ws_loc,
+                                                     self.ep_ws, stream)
         else:
             moe.moe_ep_direct_plan_dispatch(self.shape, self.G, self.rank, self.cnt_all, self.peer_y, x, None,
                                             b["topk_idx"], b["dest_row"], b["expert_offsets"], self.peer_x_loc,
@@ -244,9 +251,8 @@ class DirectEP:
             dist.all_reduce(self._flag, group=group)
 
         self.route(x, w_router, bias)
-        self.quantize_tokens(x)
         self.gather_counts(lambda out, inp: dist.all_gather_into_tensor(out, inp, group=group))
-        self.plan_and_dispatch(x)
+        self.plan_and_dispatch(x)  # quantizes the rows it sends
         barrier()
         self.experts_fp8_and_return(wg_q, wg_scale, wu_q, wu_scale, wd_q, wd_scale)
         barrier()

@@ -558,6 +558,22 @@ MOE_API moe_status moe_ep_direct_plan_dispatch(const moe_shape *shape, int32_t G
                                                const void *peer_scale_loc, void *ws, void *ws_loc, void *ep_ws,
                                                void *stream);
 
+/* Steps 3 and 4 of the fp8 form in one launch, the token rows quantized on
+ * the way: x is the rank's bf16 token rows [T,H]; each routed pair's row is
+ * quantized by the warp that sends it, with the arithmetic of
+ * moe_quantize_rows_fp8 (the same codes and scale bit for bit), and its e4m3
+ * code row and scale are stored into the owner's x_loc_q and scale_loc
+ * (peer_x_loc_q, peer_scale_loc: device arrays of G addresses).  Replaces
+ * moe_quantize_rows_fp8 (MOE_ROWS_TOKENS) + moe_ep_direct_plan_dispatch with
+ * codes; a token sent to k experts is quantized k times.  Other arguments and
+ * errors as moe_ep_direct_plan_dispatch. */
+MOE_API moe_status moe_ep_direct_plan_dispatch_quantize(const moe_shape *shape, int32_t G, int32_t rank,
+                                                        const int32_t *cnt_all, const void *peer_y, const void *x,
+                                                        const int32_t *topk_idx, const int32_t *dest_row,
+                                                        const int32_t *expert_offsets, const void *peer_x_loc_q,
+                                                        const void *peer_scale_loc, void *ws, void *ws_loc,
+                                                        void *ep_ws, void *stream);
+
 /* Step 4 (ws: the rank's routing workspace, for its status word). */
 MOE_API moe_status moe_ep_direct_dispatch(const moe_shape *shape, int32_t G, const void *x, const int32_t *topk_idx,
                                           const int32_t *dest_row, const int32_t *expert_offsets,

@@ -240,12 +240,15 @@ def run_direct_ep(dl, shape, G, fused_return=False, fused_plan=False):
     return ranks, xs
 
 
-def run_direct_ep_fp8(dl, shape, G, wq, fused_plan=True):
-    """The fp8 peer-store layer on G ranks held by this process: each rank
-    quantizes its tokens, stores code rows and scales into the owners'
-    buffers, runs the fp8 GEMMs on its experts (wq: the layer's weight codes
+def run_direct_ep_fp8(dl, shape, G, wq, mode="quantize"):
+    """The fp8 peer-store layer on G ranks held by this process: each rank's
+    token rows become e4m3 code rows and scales in the owners' buffers, the
+    owners run the fp8 GEMMs on their experts (wq: the layer's weight codes
     and scales from moe_quantize_weights_fp8, sliced per rank here) and the
-    down GEMM stores the results into the tokens' owners' y."""
+    down GEMM stores the results into the tokens' owners' y.  mode
+    "quantize": plan and dispatch in one launch that quantizes the rows it
+    sends; "codes": the tokens quantized first, then plan and dispatch in one
+    launch; "separate": quantize, plan, dispatch as three launches."""
     from grouped_expert_gemm_router_b200.ep_direct import DirectEP, connect_in_process, gather_counts_in_process
     T, Eg = shape.T, shape.E // G
     ranks = [DirectEP(shape, G, r, fp8=True) for r in range(G)]
@@ -253,11 +256,12 @@ def run_direct_ep_fp8(dl, shape, G, wq, fused_plan=True):
     xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
     for r, ep in enumerate(ranks):
         ep.route(xs[r], dl.w_router, dl.bias)
-        ep.quantize_tokens(xs[r])
+        if mode != "quantize":
+            ep.quantize_tokens(xs[r])
     gather_counts_in_process(ranks)
-    if fused_plan:
+    if mode != "separate":
         for r, ep in enumerate(ranks):
-            ep.plan_and_dispatch(xs[r])
+            ep.plan_and_dispatch(xs[r] if mode == "quantize" else None)
     else:
         for ep in ranks:
             ep.plan()

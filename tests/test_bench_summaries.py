@@ -68,7 +68,7 @@ def test_peer_store_summary_and_bound():
 
 def test_peer_store_fp8_summary():
     G = 8
-    phases = {"route": 80.0, "quantize_tokens": 24.0, "plan_dispatch": 80.0, "experts_swiglu": 160.0,
+    phases = {"route": 80.0, "plan_dispatch_quantize": 104.0, "experts_swiglu": 160.0,
               "quantize_h": 32.0, "down_return_fused": 120.0, "finish": 64.0}
     e = {"G": G, "fp8": True, "per_phase_us_all_ranks": phases, "device_status": [0] * G,
          "single_gpu_layer_us": 150.0}

@@ -153,10 +153,10 @@ def test_direct_ep_rejects_unsupported_shapes():
         DirectEP(_shape(cfg), 2, 2)  # rank out of range
 
 
-@pytest.mark.parametrize("fused_plan", [True, False], ids=["plan_dispatch", "plan_then_dispatch"])
+@pytest.mark.parametrize("mode", ["quantize", "codes", "separate"])
 @pytest.mark.parametrize("name,G", [("decode_E64_k6", 8), ("E16_k4_F384", 4), ("E8_k2_skew", 2),
                                     ("several_tiles_E4_k2", 2)], ids=lambda v: str(v))
-def test_direct_ep_fp8_matches_single_gpu_fp8(name, G, fused_plan):
+def test_direct_ep_fp8_matches_single_gpu_fp8(name, G, mode):
     """e4m3 rows on the links: each rank's out equals moe_forward_fp8 on its
     tokens bit for bit (per-row token codes and scales are the same whichever
     rank quantizes them; the same fp8 GEMM arithmetic on the same rows)."""
@@ -167,7 +167,7 @@ def test_direct_ep_fp8_matches_single_gpu_fp8(name, G, fused_plan):
     wq = dl.bufs(shape)
     wq.update(moe.alloc_fp8_buffers(shape))
     moe.quantize_layer_weights_fp8(shape, wq)
-    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq, fused_plan)
+    ranks, xs = run_direct_ep_fp8(dl, shape, G, wq, mode)
     for r, ep in enumerate(ranks):
         assert moe.moe_read_status(ep.ws) == 0 and moe.moe_read_status(ep.ws_loc) == 0
         b = dl.bufs(shape)
@@ -179,6 +179,28 @@ def test_direct_ep_fp8_matches_single_gpu_fp8(name, G, fused_plan):
         torch.cuda.synchronize()
         assert moe.moe_read_status(b["ws"]) == 0
         assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(b["out"])), "rank %d" % r
+
+
+@pytest.mark.parametrize("name,G", [("decode_E64_k6", 8), ("E8_k2_skew", 2)], ids=lambda v: str(v))
+def test_direct_ep_quantizing_dispatch_stores_the_row_quantizer_codes(name, G):
+    """The dispatch that quantizes the rows it sends leaves in every owner's
+    x_loc_q and scale_loc exactly the codes and scales of the rows
+    moe_quantize_rows_fp8 makes before a plain dispatch of codes."""
+    cfg, _ = CASES[name]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    wq = dl.bufs(shape)
+    wq.update(moe.alloc_fp8_buffers(shape))
+    moe.quantize_layer_weights_fp8(shape, wq)
+    got, _ = run_direct_ep_fp8(dl, shape, G, wq, "quantize")
+    ref, _ = run_direct_ep_fp8(dl, shape, G, wq, "codes")
+    Eg = cfg.E // G
+    for r in range(G):
+        n = int(ref[r].cnt_all[:, r * Eg:(r + 1) * Eg].sum())
+        assert n == int(got[r].cnt_all[:, r * Eg:(r + 1) * Eg].sum()) and n > 0
+        assert torch.equal(got[r].x_loc_q[:n], ref[r].x_loc_q[:n]), "rank %d codes" % r
+        assert torch.equal(got[r].scale_loc[:n], ref[r].scale_loc[:n]), "rank %d scales" % r
 
 
 def test_direct_ep_fp8_full_size_decode():
