@@ -665,12 +665,16 @@ class Bench:
             wq = {"w_gate": wg, "w_up": wu, "w_down": wd}
             wq.update(moe.alloc_fp8_buffers(shape, device=dev))
             moe.quantize_layer_weights_fp8(shape, wq, stream)
-        # experts_down + send_back and their fused form (the down GEMM storing
-        # into the owners' y) both run each step; the totals count one or the other
-        phases = ("route", "plan_dispatch", "experts_swiglu", "experts_down", "send_back", "down_return_fused",
-                  "finish")
+        # The separate launches (plan, dispatch, experts_down, send_back) and
+        # their fused forms (plan_dispatch; down_return_fused: the down GEMM
+        # storing into the owners' y) all run each step; the totals count one
+        # set or the other.
+        phases = ("route", "plan", "dispatch", "plan_dispatch", "experts_swiglu", "experts_down", "send_back",
+                  "down_return_fused", "finish")
         calls = {
             "route": lambda r: ranks[r].route(xs[r], wr, bias, stream),
+            "plan": lambda r: ranks[r].plan(stream),
+            "dispatch": lambda r: ranks[r].dispatch(xs[r], stream),
             "plan_dispatch": lambda r: ranks[r].plan_and_dispatch(xs[r], stream),
             "experts_swiglu": lambda r: moe.moe_grouped_swiglu(ranks[r].local, ranks[r].x_loc, wg[sl[r]], wu[sl[r]],
                                                                ranks[r].h_loc, ranks[r].ws_loc, stream),
@@ -925,9 +929,12 @@ def summarize_ep_direct(cfg, e, peaks):
         "ranks": "G ranks emulated on one GPU: each rank's peer stores go to the other ranks' buffers on the same "
                  "device; the counts all-gather done by copies and not timed",
         "per_rank_us": per_rank,
-        "per_rank_kernels_us": sum(v for k, v in per_rank.items() if fp8 or k != "down_return_fused"),
+        # bf16: separate launches (plan, dispatch, down GEMM, return stores)
+        # against the fused ones (plan_dispatch, down_return_fused)
+        "per_rank_kernels_us": sum(v for k, v in per_rank.items()
+                                   if fp8 or k not in ("plan_dispatch", "down_return_fused")),
         "per_rank_kernels_fused_return_us": sum(v for k, v in per_rank.items()
-                                                if k not in ("experts_down", "send_back")),
+                                                if fp8 or k not in ("plan", "dispatch", "experts_down", "send_back")),
         "single_gpu_layer_us": e["single_gpu_layer_us"],
         "experts_roofline": experts_roofline(cfg, G, t_exp, peaks, fp8),
         "exchange_per_rank": {"dispatch_bytes": out_bytes, "return_bytes": sent, "counts_bytes": G * cfg.E * 4,

@@ -48,15 +48,17 @@ def test_two_pass_summary():
 
 def test_peer_store_summary_and_bound():
     G = 8
-    phases = {"route": 80.0, "plan_dispatch": 88.0, "experts_swiglu": 1600.0, "experts_down": 1200.0,
+    phases = {"route": 80.0, "plan": 40.0, "dispatch": 48.0, "plan_dispatch": 72.0, "experts_swiglu": 1600.0,
+              "experts_down": 1200.0,
               "send_back": 120.0, "down_return_fused": 1240.0, "finish": 64.0}
     e = {"G": G, "per_phase_us_all_ranks": phases, "device_status": [0] * G, "single_gpu_layer_us": 500.0}
     cfg = synth.CONFIGS[2]  # one expert per rank: the local GEMMs are tensor-bound
     s = bench.summarize_ep_direct(cfg, e, PEAKS)
     per = {k: v / G for k, v in phases.items()}
-    assert s["per_rank_kernels_us"] == pytest.approx(sum(v for k, v in per.items() if k != "down_return_fused"))
-    assert s["per_rank_kernels_fused_return_us"] == pytest.approx(
-        sum(v for k, v in per.items() if k not in ("experts_down", "send_back")))
+    sep = ("route", "plan", "dispatch", "experts_swiglu", "experts_down", "send_back", "finish")
+    fused = ("route", "plan_dispatch", "experts_swiglu", "down_return_fused", "finish")
+    assert s["per_rank_kernels_us"] == pytest.approx(sum(per[k] for k in sep))
+    assert s["per_rank_kernels_fused_return_us"] == pytest.approx(sum(per[k] for k in fused))
     assert s["exchange_per_rank"]["dispatch_bytes"] == 512 * 2 * 4096 * 2
     assert s["experts_roofline"]["bound"] == "tensor"
     t = (per["experts_swiglu"] + per["experts_down"]) * 1e-6
