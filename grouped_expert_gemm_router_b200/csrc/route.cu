@@ -8,9 +8,10 @@
 // - A CTA of 8 warps owns TB tokens (16, 8 or 4: fewer for more experts) and
 //   all E experts for a slice of the hidden dimension.  When there are few
 //   token blocks, the hidden dimension is split over a thread-block cluster of
-//   CL CTAs (CL <= 8) so that about 3/4 of the SMs get a CTA; the CL partial
-//   logits are summed by the cluster's rank-0 CTA through distributed shared
-//   memory, in rank order (deterministic).
+//   CL CTAs (CL <= 8) so that about 3/4 of the SMs get a CTA; rank r of the
+//   cluster sums the CL partial logits of tokens r, r + CL, ... through
+//   distributed shared memory, in rank order (deterministic), and runs their
+//   top-k.
 // - x and W_r stream through shared memory in chunks of HC hidden units with
 //   a 2-4 stage cp.async pipeline.  The 8 warps split each chunk's hidden
 //   units; inside a warp ES lanes split the experts (EJ consecutive experts
@@ -61,7 +62,6 @@ struct RouteArgs {
     int part_off;     // byte offset of the partial-logit tile in dynamic shared memory
     // fused dispatch (fuse != 0)
     int fuse;
-    int tiles;        // CTAs that run the top-k (one per token block)
     int C, capped, P;
     FusedDispatch out;
     WsPtrs ws;
@@ -456,19 +456,19 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
             cluster_sync_all();
         else
             __syncthreads();
-        if (rank == 0) {
-            // Sum the slices in rank order, add the bias, publish the logits.
-            for (int i = tid; i < TB * E; i += 256) {
-                const int tok = i / E, e = i % E, t = t0 + tok;
-                float l = part[i];
-                for (int r = 1; r < CL; ++r) l += ld_cluster_f32(part + i, (uint32_t)r);
-                if (a.bias) l = l + a.bias[e];
-                lg[tok][e] = l;
-                if (t < a.T && a.logits) a.logits[(size_t)t * E + e] = l;
-            }
+        // Rank r of the cluster takes tokens r, r + CL, ...: it sums their
+        // slices in rank order (every token in the same order), adds the
+        // bias, publishes their logits and runs their top-k below.
+        const int mine = (TB - rank + CL - 1) / CL;  // tokens of this rank
+        for (int i = tid; i < mine * E; i += 256) {
+            const int tok = rank + CL * (i / E), e = i % E, t = t0 + tok;
+            const int pi = tok * E + e;
+            float l = CL > 1 ? ld_cluster_f32(part + pi, 0u) : part[pi];
+            for (int r = 1; r < CL; ++r) l += ld_cluster_f32(part + pi, (uint32_t)r);
+            if (a.bias) l = l + a.bias[e];
+            lg[tok][e] = l;
+            if (t < a.T && a.logits) a.logits[(size_t)t * E + e] = l;
         }
-        if (CL > 1) cluster_sync_all();  // every slice stays readable until rank 0 is done
-        if (rank != 0) return;
     } else if (a.lparts) {
         // Partial planes of the hidden ranges, added in range order, then
         // the bias; the logits are published for the caller.
@@ -489,8 +489,8 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
     __syncthreads();
 
-    // Top-k, one warp per token.
-    for (int tok = warp; tok < TB; tok += 8) {
+    // Top-k, one warp per token (with a cluster: this rank's tokens).
+    for (int tok = rank + CL * warp; tok < TB; tok += 8 * CL) {
         const int t = t0 + tok;
         if (t >= a.T) break;
         float v[EJ];
@@ -502,13 +502,14 @@ __global__ void __launch_bounds__(256) k_route(RouteArgs a) {
     }
     __syncthreads();
     if (tid == 0 && s_nan) atomicOr(a.status, MOE_DEV_NAN_LOGIT);
+    if (CL > 1) cluster_sync_all();  // every slice stays readable until the cluster has summed it
     if (a.fuse) {
         // Publish this CTA's top-k, then take a ticket; the last CTA sees every
         // other CTA's results after its own fence.
         __threadfence();
         __syncthreads();
         __shared__ int s_last;
-        if (tid == 0) s_last = atomicAdd(a.ws.route_done, 1u) == (unsigned)(a.tiles - 1);
+        if (tid == 0) s_last = atomicAdd(a.ws.route_done, 1u) == gridDim.x - 1;
         __syncthreads();
         if (!s_last) return;
         __threadfence();
@@ -623,7 +624,6 @@ cudaError_t launch_route(const moe_shape &s0, const void *x, const float *w_rout
     // longer top-k per CTA.)
     if (TB == 16 && !a.logits_in && ((s.T + 15) / 16) * 8 < (3 * num_sms) / 4) TB = 8;
     const int tiles = (s.T + TB - 1) / TB;
-    a.tiles = tiles;
     // Split the hidden dimension over a cluster until there are about 3/4 as
     // many blocks as SMs (measured best at 8 and 64 experts).
     int cl = 1;
