@@ -20,13 +20,15 @@
 //                  region and the per-destination slots (pack: also the
 //                  counts sent ahead of the rows; unpack: the same copies
 //                  reversed), a warp per row over every block.
-// k_ep_plan_recv   on the receiving rank, from the counts of every source:
+// k_ep_receive     on the receiving rank, from the counts of every source:
 //                  an expert-contiguous local layout (per expert, each
-//                  source's capacity rows then its overflow rows), its GEMM
-//                  schedule (the block schedule builder of the dispatch) and
-//                  the source of every local row.
-// k_ep_local_rows  the received rows into the local layout, or the local
-//                  results back to the return buffers, a warp per row.
+//                  source's capacity rows then its overflow rows), the
+//                  received rows copied into it (a warp per row, every block
+//                  deriving the layout itself) and, by one extra block, its
+//                  GEMM schedule (the block schedule builder of the dispatch)
+//                  and the source of every local row.
+// k_ep_local_rows  the local results back to the return buffers, a warp per
+//                  row.
 #include <cuda_bf16.h>
 
 #include "dispatch_block.cuh"
@@ -92,69 +94,119 @@ __global__ void __launch_bounds__(kRowThreads) k_ep_spill_rows(WsPtrs ws, const 
 // total at most G (E_g C + S), the local shape's T.  row_src[r] = the row of
 // the received capacity buffer that local row r comes from, or -1 - its row
 // in the received overflow buffer.
-__global__ void __launch_bounds__(kScanThreads) k_ep_plan_recv(const int32_t *meta, int G, int Eg, int C, int S,
-                                                               int32_t *loc_counts, int32_t *loc_offsets,
-                                                               int32_t *row_src, WsPtrs lws) {
-    __shared__ DispatchSmem sm;
-    __shared__ int nc[kMaxExperts], no[kMaxExperts], ovf_pre[kMaxExperts], seg[kMaxExperts];
-    __shared__ int m[2 * kMaxExperts];
-    __shared__ int any_bad;
-    pdl_trigger();
-    pdl_wait();
-    const int tid = threadIdx.x;  // (source s, local expert e) pairs are indexed s E_g + e
-    if (tid == 0) any_bad = 0;
-    for (int i = tid; i < 2 * G * Eg; i += kScanThreads) m[i] = meta[i];  // all loads in one round trip
+// Shared-memory state of a receiving block: the received counts of every
+// (source s, local expert e), indexed s E_g + e, clamped.
+struct RecvSmem {
+    DispatchSmem sm;
+    int nc[kMaxExperts], no[kMaxExperts], ovf_pre[kMaxExperts], seg[kMaxExperts];
+    int m[2 * kMaxExperts];
+    int any_bad;
+};
+
+// The received counts (all loads in one round trip), clamped to what the
+// buffers hold (capacity rows to C, each source's overflow rows to S in
+// expert order); all threads of the block.
+__device__ void recv_counts(const int32_t *meta, int G, int Eg, int C, int S, RecvSmem &p) {
+    const int tid = threadIdx.x;
+    if (tid == 0) p.any_bad = 0;
+    for (int i = tid; i < 2 * G * Eg; i += kScanThreads) p.m[i] = meta[i];
     __syncthreads();
     for (int s = tid; s < G; s += kScanThreads) {
         int pre = 0;
         bool bad = false;
         for (int e = 0; e < Eg; ++e) {
-            const int rc = m[s * 2 * Eg + e], ro = m[s * 2 * Eg + Eg + e];
+            const int rc = p.m[s * 2 * Eg + e], ro = p.m[s * 2 * Eg + Eg + e];
             const int c = min(max(rc, 0), C), o = min(max(ro, 0), S - pre);
             bad |= c != rc || o != ro;
-            nc[s * Eg + e] = c;
-            no[s * Eg + e] = o;
-            ovf_pre[s * Eg + e] = pre;
+            p.nc[s * Eg + e] = c;
+            p.no[s * Eg + e] = o;
+            p.ovf_pre[s * Eg + e] = pre;
             pre += o;
         }
-        if (bad) any_bad = 1;
+        if (bad) p.any_bad = 1;
     }
     __syncthreads();
-    if (tid == 0 && any_bad) atomicOr(lws.status, MOE_DEV_BAD_ROW);
-    for (int e = tid; e < Eg; e += kScanThreads) {
-        int n = 0;
-        for (int s = 0; s < G; ++s) n += nc[s * Eg + e] + no[s * Eg + e];
-        sm.hist[e] = n;
-    }
-    __syncthreads();
-    // offsets, local schedule (uncapped layout of the local experts)
-    build_schedule_block(sm, Eg, 0, false, loc_counts, loc_offsets, lws);
-    for (int e = tid; e < Eg; e += kScanThreads) {
-        int row = sm.offs[e];
+}
+
+// First local row of each (source, expert) segment: expert e's rows are its
+// sources' rows in source order from offs[e].  All threads of the block.
+__device__ void recv_segments(RecvSmem &p, const int *offs, int G, int Eg) {
+    for (int e = threadIdx.x; e < Eg; e += kScanThreads) {
+        int row = offs[e];
         for (int s = 0; s < G; ++s) {
-            seg[s * Eg + e] = row;
-            row += nc[s * Eg + e] + no[s * Eg + e];
+            p.seg[s * Eg + e] = row;
+            row += p.nc[s * Eg + e] + p.no[s * Eg + e];
         }
     }
     __syncthreads();
-    const int total = sm.offs[Eg];
-    for (int r = tid; r < total; r += kScanThreads) {
-        int lo = 0, hi = Eg - 1;  // expert: last e with offs[e] <= r
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (sm.offs[mid] <= r) lo = mid;
-            else hi = mid - 1;
-        }
-        const int e = lo;
-        lo = 0;
-        hi = G - 1;  // source: last s with seg[s][e] <= r (empty segments share a start)
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (seg[mid * Eg + e] <= r) lo = mid;
-            else hi = mid - 1;
-        }
-        const int i = lo * Eg + e, j = r - seg[i];
-        row_src[r] = j < nc[i] ? lo * Eg * C + e * C + j : -1 - (lo * S + ovf_pre[i] + (j - nc[i]));
+}
+
+// Received row of local row r: capacity buffer row (>= 0) or -1 - overflow
+// buffer row.
+__device__ __forceinline__ int recv_row_source(const RecvSmem &p, const int *offs, int r, int G, int Eg, int C,
+                                               int S) {
+    int lo = 0, hi = Eg - 1;  // expert: last e with offs[e] <= r
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offs[mid] <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    const int e = lo;
+    lo = 0;
+    hi = G - 1;  // source: last s with seg[s][e] <= r (empty segments share a start)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.seg[mid * Eg + e] <= r) lo = mid;
+        else hi = mid - 1;
+    }
+    const int i = lo * Eg + e, j = r - p.seg[i];
+    return j < p.nc[i] ? lo * Eg * C + e * C + j : -1 - (lo * S + p.ovf_pre[i] + (j - p.nc[i]));
+}
+
+// The receiving side in one launch.  Every block derives the local layout
+// from the received counts itself and copies its share of the received rows
+// into x_loc (a warp per local row); the last block instead builds what the
+// later kernels read: the local counts, offsets and GEMM schedule (uncapped
+// layout of the local experts) and the source of every local row (row_src,
+// for the return).
+__global__ void __launch_bounds__(kScanThreads) k_ep_receive(const int32_t *meta, int G, int Eg, int C, int S,
+                                                             int32_t *loc_counts, int32_t *loc_offsets,
+                                                             int32_t *row_src, WsPtrs lws, int Tloc, int H8,
+                                                             const uint4 *cap, const uint4 *ovf, uint4 *loc) {
+    __shared__ RecvSmem p;
+    DispatchSmem &sm = p.sm;
+    pdl_trigger();
+    pdl_wait();
+    const int tid = threadIdx.x;
+    recv_counts(meta, G, Eg, C, S, p);
+    const int n = tid < Eg ? [&] {
+        int v = 0;
+        for (int s = 0; s < G; ++s) v += p.nc[s * Eg + tid] + p.no[s * Eg + tid];
+        return v;
+    }() : 0;
+    if (blockIdx.x == gridDim.x - 1) {
+        if (tid == 0 && p.any_bad) atomicOr(lws.status, MOE_DEV_BAD_ROW);
+        if (tid < Eg) sm.hist[tid] = n;
+        __syncthreads();
+        build_schedule_block(sm, Eg, 0, false, loc_counts, loc_offsets, lws);
+        recv_segments(p, sm.offs, G, Eg);
+        const int total = sm.offs[Eg];
+        for (int r = tid; r < total; r += kScanThreads) row_src[r] = recv_row_source(p, sm.offs, r, G, Eg, C, S);
+        return;
+    }
+    // exclusive offsets of the local experts (the schedule builder's own)
+    int incl = n, unused = 0;
+    block_inclusive_scan2(sm, incl, unused);
+    if (tid < Eg) sm.offs[tid] = incl - n;
+    if (tid == Eg - 1) sm.offs[Eg] = incl;
+    __syncthreads();
+    recv_segments(p, sm.offs, G, Eg);
+    const int lane = tid & 31;
+    const int total = min(sm.offs[Eg], Tloc);
+    for (int r = blockIdx.x * kRowWarps + (tid >> 5); r < total; r += ((int)gridDim.x - 1) * kRowWarps) {
+        const int src = recv_row_source(p, sm.offs, r, G, Eg, C, S);
+        const uint4 *rx = src >= 0 ? cap + (size_t)src * H8 : ovf + (size_t)(-1 - src) * H8;
+        copy_row_warp(rx, loc + (size_t)r * H8, H8, lane);
     }
 }
 
@@ -238,12 +290,9 @@ cudaError_t launch_ep_local_dispatch(const moe_shape &s, int G, const int32_t *r
     const EpWs p = ep_ptrs(ep_ws, s, G);
     const int S = (int)ep_overflow_rows(s, G), Eg = s.E / G;
     const int64_t Tloc = ep_local_rows(s, G);
-    cudaError_t e = launch_pdl(k_ep_plan_recv, dim3(1), dim3(kScanThreads), 0, stream, recv_meta, G, Eg, s.C, S,
-                               p.loc_counts, p.loc_offsets, p.row_src, ws_ptrs(ws_loc, Lloc));
-    if (e != cudaSuccess) return e;
-    return launch_pdl(k_ep_local_rows, dim3(row_grid(Tloc, num_sms)), dim3(kRowThreads), 0, stream,
-                      (const int32_t *)p.row_src, (const int32_t *)(p.loc_offsets + Eg), (int)Tloc, s.H / 8,
-                      (uint4 *)recv_cap, (uint4 *)recv_ovf, (uint4 *)x_loc, 0);
+    return launch_pdl(k_ep_receive, dim3(row_grid(Tloc, num_sms) + 1), dim3(kScanThreads), 0, stream, recv_meta, G,
+                      Eg, s.C, S, p.loc_counts, p.loc_offsets, p.row_src, ws_ptrs(ws_loc, Lloc), (int)Tloc, s.H / 8,
+                      (const uint4 *)recv_cap, (const uint4 *)recv_ovf, (uint4 *)x_loc);
 }
 
 // Receiving side, after the local experts: y_loc rows back to where their
