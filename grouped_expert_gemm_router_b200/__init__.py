@@ -43,7 +43,7 @@ ABI_FUNCTIONS = (
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
     "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
     "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h", "moe_ep_direct_plan_dispatch",
-    "moe_ep_direct_plan_dispatch_quantize",
+    "moe_ep_direct_plan_dispatch_quantize", "moe_ep_unpack_combine",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -162,6 +162,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_local_return.restype = st
     lib.moe_ep_unpack.argtypes = [sp, i32] + [vp] * 4
     lib.moe_ep_unpack.restype = st
+    lib.moe_ep_unpack_combine.argtypes = [sp, i32] + [vp] * 7
+    lib.moe_ep_unpack_combine.restype = st
     lib.moe_ep_direct_local_rows.argtypes = [sp, i32]
     lib.moe_ep_direct_local_rows.restype = ctypes.c_int64
     lib.moe_ep_direct_workspace_bytes.argtypes = [sp, i32]
@@ -493,6 +495,14 @@ def moe_ep_local_return(shape, G, y_loc, back_cap, back_ovf, ep_ws, stream=None)
 def moe_ep_unpack(shape, G, recv_back_ovf, y, ep_ws, stream=None):
     _check(load_library().moe_ep_unpack(ctypes.byref(shape), int(G), _ptr(recv_back_ovf), _ptr(y), _ptr(ep_ws),
                                         _stream(stream)), "moe_ep_unpack")
+
+
+def moe_ep_unpack_combine(shape, G, recv_back_ovf, y, dest_row, topk_w, out, ep_ws, stream=None):
+    """moe_ep_unpack + moe_combine in one launch (overflow results read from
+    the return slots)."""
+    _check(load_library().moe_ep_unpack_combine(ctypes.byref(shape), int(G), _ptr(recv_back_ovf), _ptr(y),
+                                                 _ptr(dest_row), _ptr(topk_w), _ptr(out), _ptr(ep_ws),
+                                                 _stream(stream)), "moe_ep_unpack_combine")
 
 
 def moe_ep_direct_local_rows(shape, G) -> int:

@@ -27,14 +27,44 @@ __device__ __forceinline__ void unpack8(const uint4 &q, float (&v)[8]) {
     }
 }
 
+// Overflow rows read from where an expert-parallel exchange left them: row
+// E C + q of y is row d S + (q - starts[d]) of `ovf`, d the last destination
+// with starts[d] <= q (the rows the unpack would copy into y); any other row
+// is read from y.
+struct OvfRows {
+    const uint4 *ovf;
+    const int32_t *starts;  // [G + 1]
+    int cap_rows, S, G;
+};
+
 // KMAX > 0: k <= KMAX, all k row loads issued before any is used; KMAX = 0:
-// any k, one row at a time.
-template <int KMAX>
+// any k, one row at a time.  REDIR: overflow rows through OvfRows.
+template <int KMAX, bool REDIR = false>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const int *__restrict__ dest_row,
                                                  const float *__restrict__ w, uint4 *__restrict__ out, int k, int H8,
-                                                 int P) {
+                                                 int P, OvfRows orw) {
+    __shared__ int st[REDIR ? kMaxExperts + 1 : 1];
     pdl_trigger();
     pdl_wait();
+    if (REDIR) {
+        for (int d = threadIdx.x; d <= orw.G; d += blockDim.x) st[d] = orw.starts[d];
+        __syncthreads();
+    }
+    const int total = REDIR ? min(st[REDIR ? orw.G : 0], P - orw.cap_rows) : 0;
+    auto row_ptr = [&](int r) -> const uint4 * {
+        if (REDIR && r >= orw.cap_rows && r - orw.cap_rows < total) {
+            const int q = r - orw.cap_rows;
+            int lo = 0, hi = orw.G - 1;  // last d with st[d] <= q
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (st[mid] <= q) lo = mid;
+                else hi = mid - 1;
+            }
+            const int j = q - st[lo];
+            if (j < orw.S) return orw.ovf + (size_t)(lo * orw.S + j) * H8;
+        }
+        return y + (size_t)r * H8;
+    };
     const int t = blockIdx.x;
     const int v = blockIdx.y * blockDim.x + threadIdx.x;
     if (v >= H8) return;
@@ -52,7 +82,7 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
         }
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)  // an index outside [0, P) only after an earlier device error
-            q[j] = (unsigned)r[j] < (unsigned)P ? __ldg(y + (size_t)r[j] * H8 + v) : make_uint4(0, 0, 0, 0);
+            q[j] = (unsigned)r[j] < (unsigned)P ? __ldg(row_ptr(r[j]) + v) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
             if ((unsigned)r[j] >= (unsigned)P) continue;
@@ -67,7 +97,7 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
             if ((unsigned)r >= (unsigned)P) continue;  // only after an earlier device error
             const float wj = __ldg(w + (size_t)t * k + j);
             float yv[8];
-            unpack8(__ldg(y + (size_t)r * H8 + v), yv);
+            unpack8(__ldg(row_ptr(r) + v), yv);
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, yv[i]));
         }
@@ -88,14 +118,35 @@ cudaError_t launch_combine(const moe_shape &s, const void *y, const int32_t *des
     const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, (s.flags & MOE_FLAG_CAPACITY) != 0);
     if (s.k <= 2)
         return launch_pdl(k_combine<2>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
-                          s.k, H8, P);
+                          s.k, H8, P, OvfRows{});
     else if (s.k <= 8)
         return launch_pdl(k_combine<8>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
-                          s.k, H8, P);
+                          s.k, H8, P, OvfRows{});
     else
         return launch_pdl(k_combine<0>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w, (uint4 *)out,
-                          s.k, H8, P);
+                          s.k, H8, P, OvfRows{});
     return cudaGetLastError();
+}
+
+// The combine reading each overflow row from the received return slots
+// (ovf [G][S] rows, destination starts [G + 1] from the expert-parallel
+// workspace) instead of from y: the unpack and the combine in one launch,
+// bit-identical to the two.
+cudaError_t launch_combine_ovf(const moe_shape &s, int G, int S, const void *y, const void *ovf,
+                               const int32_t *starts, const int32_t *dest_row, const float *topk_w, void *out,
+                               cudaStream_t stream) {
+    const int H8 = s.H / 8;
+    const dim3 grid((unsigned)s.T, (unsigned)((H8 + 255) / 256));
+    const int P = (int)permuted_rows(s.T, s.E, s.k, s.C, (s.flags & MOE_FLAG_CAPACITY) != 0);
+    const OvfRows o = {(const uint4 *)ovf, starts, s.E * s.C, S, G};
+    if (s.k <= 2)
+        return launch_pdl(k_combine<2, true>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w,
+                          (uint4 *)out, s.k, H8, P, o);
+    else if (s.k <= 8)
+        return launch_pdl(k_combine<8, true>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w,
+                          (uint4 *)out, s.k, H8, P, o);
+    return launch_pdl(k_combine<0, true>, grid, dim3(256), 0, stream, (const uint4 *)y, dest_row, topk_w,
+                      (uint4 *)out, s.k, H8, P, o);
 }
 
 }  // namespace moe

@@ -320,4 +320,17 @@ cudaError_t launch_ep_unpack(const moe_shape &s, int G, const void *recv_back_ov
                       (uint4 *)recv_back_ovf, 1, (int32_t *)nullptr, (int32_t *)nullptr);
 }
 
+// The unpack folded into the combine: overflow results read from the
+// received return slots where the unpack would have copied them from.
+cudaError_t launch_combine_ovf(const moe_shape &s, int G, int S, const void *y, const void *ovf,
+                               const int32_t *starts, const int32_t *dest_row, const float *topk_w, void *out,
+                               cudaStream_t stream);
+cudaError_t launch_ep_unpack_combine(const moe_shape &s, int G, const void *recv_back_ovf, const void *y,
+                                     const int32_t *dest_row, const float *topk_w, void *out, void *ep_ws,
+                                     cudaStream_t stream) {
+    const EpWs p = ep_ptrs(ep_ws, s, G);
+    return launch_combine_ovf(s, G, (int)ep_overflow_rows(s, G), y, recv_back_ovf, p.starts, dest_row, topk_w, out,
+                              stream);
+}
+
 }  // namespace moe

@@ -41,6 +41,9 @@ int64_t ep_overflow_rows(const moe_shape &s, int G);
 size_t ep_workspace_bytes(const moe_shape &s, int G);
 cudaError_t launch_ep_pack(const moe_shape &s, int G, const void *x_perm, const WsLayout &L, void *ws, void *send_ovf,
                            int32_t *send_meta, void *ep_ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_unpack_combine(const moe_shape &s, int G, const void *recv_back_ovf, const void *y,
+                                     const int32_t *dest_row, const float *topk_w, void *out, void *ep_ws,
+                                     cudaStream_t stream);
 cudaError_t launch_ep_local_dispatch(const moe_shape &s, int G, const int32_t *recv_meta, const void *recv_cap,
                                      const void *recv_ovf, void *x_loc, const WsLayout &Lloc, void *ws_loc,
                                      void *ep_ws, int num_sms, cudaStream_t stream);
@@ -575,6 +578,18 @@ moe_status moe_ep_local_return(const moe_shape *s, int32_t G, const void *y_loc,
     if ((st = device_info(&sms)) != MOE_OK) return st;
     cudaError_t e = launch_ep_local_return(*s, G, y_loc, back_cap, back_ovf, ep_ws, sms, (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_local_return");
+}
+
+moe_status moe_ep_unpack_combine(const moe_shape *s, int32_t G, const void *recv_back_ovf, const void *y,
+                                 const int32_t *dest_row, const float *topk_w, void *out, void *ep_ws, void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    if (!aligned_or_empty(recv_back_ovf, 16, ep_overflow_rows(*s, G) == 0) || !aligned(y, 16) ||
+        !aligned(dest_row, 4) || !aligned(topk_w, 4) || !aligned(out, 16) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    cudaError_t e = launch_ep_unpack_combine(*s, G, recv_back_ovf, y, dest_row, topk_w, out, ep_ws,
+                                             (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_unpack_combine");
 }
 
 moe_status moe_ep_unpack(const moe_shape *s, int32_t G, const void *recv_back_ovf, void *y, void *ep_ws,

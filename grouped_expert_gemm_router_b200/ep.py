@@ -127,11 +127,16 @@ class CapAndSpillEP:
         all_to_all(self.b["y"][:self.cap_rows], self.back_cap)
         all_to_all(self.recv_back_ovf, self.back_ovf)
 
-    def finish(self, stream=None):
-        """Overflow results into y, then the weighted combine into out."""
+    def finish(self, stream=None, fused=True):
+        """The weighted combine into out, the overflow results read from the
+        return slots (fused=False: copied into y first, then combined)."""
         s, b = self.shape, self.b
-        moe.moe_ep_unpack(s, self.G, self.recv_back_ovf, b["y"], self.ep_ws, stream)
-        moe.moe_combine(s, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
+        if fused:
+            moe.moe_ep_unpack_combine(s, self.G, self.recv_back_ovf, b["y"], b["dest_row"], b["topk_w"], b["out"],
+                                      self.ep_ws, stream)
+        else:
+            moe.moe_ep_unpack(s, self.G, self.recv_back_ovf, b["y"], self.ep_ws, stream)
+            moe.moe_combine(s, b["y"], b["dest_row"], b["topk_w"], b["out"], stream)
         return b["out"]
 
     # ---- the layer on a process group ------------------------------------------

@@ -484,6 +484,15 @@ MOE_API moe_status moe_ep_local_return(const moe_shape *shape, int32_t G, const 
 MOE_API moe_status moe_ep_unpack(const moe_shape *shape, int32_t G, const void *recv_back_ovf, void *y, void *ep_ws,
                                  void *stream);
 
+/* Steps 8 and 9 in one launch: moe_combine (y, dest_row, topk_w -> out) that
+ * reads each overflow row's result from recv_back_ovf, where moe_ep_unpack
+ * would have copied it from, instead of from y (y's overflow region is left
+ * as it was).  out equals that of moe_ep_unpack + moe_combine bit for bit.
+ * dest_row, topk_w: device [T*k]; out: device bf16 [T,H], 16-byte aligned. */
+MOE_API moe_status moe_ep_unpack_combine(const moe_shape *shape, int32_t G, const void *recv_back_ovf,
+                                         const void *y, const int32_t *dest_row, const float *topk_w, void *out,
+                                         void *ep_ws, void *stream);
+
 /* ------------------------------------------------------------------------
  * Expert parallelism by device-initiated peer stores ("direct" form).
  *

@@ -185,9 +185,10 @@ def oracle_layer(orc, L, cfg, logits_gpu):
     return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)
 
 
-def run_cap_and_spill_ep(dl, shape, G):
+def run_cap_and_spill_ep(dl, shape, G, fused_finish=True):
     """The two-pass expert-parallel layer on G ranks held by this process;
-    rank r holds tokens [r T, (r+1) T) of the layer dl."""
+    rank r holds tokens [r T, (r+1) T) of the layer dl (fused_finish: the
+    unpack folded into the combine)."""
     from grouped_expert_gemm_router_b200.ep import CapAndSpillEP, exchange_in_process
     T, Eg = shape.T, shape.E // G
     ranks = [CapAndSpillEP(shape, G) for _ in range(G)]
@@ -200,7 +201,7 @@ def run_cap_and_spill_ep(dl, shape, G):
         ep.local_experts(dl.w_gate[sl], dl.w_up[sl], dl.w_down[sl])
     exchange_in_process(ranks, "exchange_out")
     for ep in ranks:
-        ep.finish()
+        ep.finish(fused=fused_finish)
     torch.cuda.synchronize()
     return ranks, xs
 

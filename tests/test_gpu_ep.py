@@ -113,6 +113,25 @@ def test_ep_full_size_decode_matches_single_gpu(G):
         assert np.array_equal(bf16_host(ep.b["out"]), bf16_host(ref["out"])), "rank %d" % r
 
 
+@pytest.mark.parametrize("name,G", [("decode_E64_k6_C16", 8), ("E16_k4_C24_F384", 4), ("C0_all_overflow", 2)],
+                         ids=lambda v: str(v))
+def test_ep_unpack_combine_equals_unpack_then_combine(name, G):
+    """The combine that reads the overflow results from the return slots
+    gives the out of the unpack followed by the combine, bit for bit."""
+    cfg, _ = CASES[name]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    ranks, _ = run_cap_and_spill_ep(dl, shape, G, fused_finish=True)
+    fused = [ep.b["out"].clone() for ep in ranks]
+    assert any(int(ep.send_meta.view(G, 2, -1)[:, 1].sum()) > 0 for ep in ranks), "no overflow rows"
+    for r, ep in enumerate(ranks):
+        ep.b["out"].zero_()
+        ep.finish(fused=False)
+        torch.cuda.synchronize()
+        assert torch.equal(ep.b["out"], fused[r]), "rank %d" % r
+
+
 def test_ep_rejects_uncapped_layout():
     cfg = CASES["E16_k4_C24_F384"][0]
     with pytest.raises(moe.MoeError):
