@@ -43,7 +43,7 @@ ABI_FUNCTIONS = (
     "moe_ep_direct_local_rows", "moe_ep_direct_workspace_bytes", "moe_ep_direct_local_shape", "moe_ep_direct_plan",
     "moe_ep_direct_dispatch", "moe_ep_direct_return", "moe_ep_direct_down_return", "moe_ep_direct_dispatch_fp8",
     "moe_ep_direct_down_return_fp8", "moe_ep_direct_quantize_h", "moe_ep_direct_plan_dispatch",
-    "moe_ep_direct_plan_dispatch_quantize", "moe_ep_unpack_combine",
+    "moe_ep_direct_plan_dispatch_quantize", "moe_ep_unpack_combine", "moe_ep_gather_pack",
 )
 MOE_STATIC_WS_BYTES = 1 << 20
 
@@ -164,6 +164,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_ep_unpack.restype = st
     lib.moe_ep_unpack_combine.argtypes = [sp, i32] + [vp] * 7
     lib.moe_ep_unpack_combine.restype = st
+    lib.moe_ep_gather_pack.argtypes = [sp, i32] + [vp] * 8
+    lib.moe_ep_gather_pack.restype = st
     lib.moe_ep_direct_local_rows.argtypes = [sp, i32]
     lib.moe_ep_direct_local_rows.restype = ctypes.c_int64
     lib.moe_ep_direct_workspace_bytes.argtypes = [sp, i32]
@@ -495,6 +497,14 @@ def moe_ep_local_return(shape, G, y_loc, back_cap, back_ovf, ep_ws, stream=None)
 def moe_ep_unpack(shape, G, recv_back_ovf, y, ep_ws, stream=None):
     _check(load_library().moe_ep_unpack(ctypes.byref(shape), int(G), _ptr(recv_back_ovf), _ptr(y), _ptr(ep_ws),
                                         _stream(stream)), "moe_ep_unpack")
+
+
+def moe_ep_gather_pack(shape, G, x, src_token, x_perm, ws, send_ovf, send_meta, ep_ws, stream=None):
+    """moe_gather + moe_ep_pack in one launch (overflow rows straight into
+    the send slots)."""
+    _check(load_library().moe_ep_gather_pack(ctypes.byref(shape), int(G), _ptr(x), _ptr(src_token), _ptr(x_perm),
+                                              _ptr(ws), _ptr(send_ovf), _ptr(send_meta), _ptr(ep_ws),
+                                              _stream(stream)), "moe_ep_gather_pack")
 
 
 def moe_ep_unpack_combine(shape, G, recv_back_ovf, y, dest_row, topk_w, out, ep_ws, stream=None):

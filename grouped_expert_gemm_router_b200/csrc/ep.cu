@@ -86,6 +86,70 @@ __global__ void __launch_bounds__(kRowThreads) k_ep_spill_rows(WsPtrs ws, const 
     }
 }
 
+// The row copy of the dispatch and the pack in one launch: capacity slot
+// rows of x_perm from x (zero rows for unfilled slots), overflow rows
+// straight into their destination's slot of `send` (x_perm's overflow region
+// is not written); block 0 also writes the counts sent ahead (meta) and the
+// destination starts, as the pack does.  A warp per row, eight 16-byte loads
+// per lane in flight, streaming stores (each row is read once, by the
+// exchange).
+__global__ void __launch_bounds__(kRowThreads) k_ep_gather_pack(WsPtrs ws, const uint4 *__restrict__ x,
+                                                                const int32_t *__restrict__ src_token, int T, int E,
+                                                                int G, int C, int S, int P, int H8, uint4 *x_perm,
+                                                                uint4 *send, int32_t *meta, int32_t *ep_starts_out) {
+    __shared__ int starts[kMaxExperts + 1];
+    pdl_trigger();
+    pdl_wait();
+    const int Eg = E / G, tid = threadIdx.x;
+    for (int d = tid; d <= G; d += kRowThreads) starts[d] = ws.spill_off[d * Eg];
+    if (blockIdx.x == 0) {
+        for (int i = tid; i < E; i += kRowThreads) {
+            const int d = i / Eg, e = i % Eg;
+            meta[(size_t)d * 2 * Eg + e] = ws.cap_cnt[i];
+            meta[(size_t)d * 2 * Eg + Eg + e] = ws.spill_cnt[i];
+        }
+        for (int d = tid; d <= G; d += kRowThreads) ep_starts_out[d] = ws.spill_off[d * Eg];
+    }
+    __syncthreads();
+    const int cap = E * C, rows = min(cap + starts[G], P);
+    const int lane = tid & 31;
+    for (int row = blockIdx.x * kRowWarps + (tid >> 5); row < rows; row += gridDim.x * kRowWarps) {
+        uint4 *dst;
+        if (row < cap) {
+            dst = x_perm + (size_t)row * H8;
+        } else {
+            const int q = row - cap;
+            int lo = 0, hi = G - 1;  // last d with starts[d] <= q
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (starts[mid] <= q) lo = mid;
+                else hi = mid - 1;
+            }
+            const int j = q - starts[lo];
+            if (j >= S) {  // cannot happen for a valid routing; never touch past the slot
+                if (lane == 0) atomicOr(ws.status, MOE_DEV_BAD_ROW);
+                continue;
+            }
+            dst = send + (size_t)(lo * S + j) * H8;
+        }
+        const int t = src_token[row];
+        if ((unsigned)t < (unsigned)T) {
+            const uint4 *src = x + (size_t)t * H8;
+            int v = lane;
+            for (; v + 224 < H8; v += 256) {
+                uint4 q8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q8[i] = __ldg(src + v + 32 * i);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) __stcs(dst + v + 32 * i, q8[i]);
+            }
+            for (; v < H8; v += 32) __stcs(dst + v, __ldg(src + v));
+        } else {
+            for (int v = lane; v < H8; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
 // Receiving rank, one block.  meta[s][0][e], meta[s][1][e]: capacity and
 // overflow rows source s sent for local expert e, clamped to what the buffers
 // hold (capacity rows to C, each source's overflow rows to its slot of S
@@ -280,6 +344,19 @@ cudaError_t launch_ep_pack(const moe_shape &s, int G, const void *x_perm, const 
     return launch_pdl(k_ep_spill_rows, dim3(row_grid(P - (int64_t)s.E * s.C, num_sms)), dim3(kRowThreads), 0, stream,
                       ws_ptrs(ws, L), (const int32_t *)nullptr, s.E, G, s.C, S, (int)P, s.H / 8, (uint4 *)x_perm,
                       (uint4 *)send_ovf, 0, send_meta, p.starts);
+}
+
+// Source side, the row copy and the pack in one launch.
+cudaError_t launch_ep_gather_pack(const moe_shape &s, int G, const void *x, const int32_t *src_token, void *x_perm,
+                                  const WsLayout &L, void *ws, void *send_ovf, int32_t *send_meta, void *ep_ws,
+                                  int num_sms, cudaStream_t stream) {
+    const EpWs p = ep_ptrs(ep_ws, s, G);
+    const int S = (int)ep_overflow_rows(s, G);
+    const int64_t P = permuted_rows(s.T, s.E, s.k, s.C, true);
+    const int64_t rows_hint = (int64_t)s.E * s.C + (int64_t)s.k * (s.T > s.C ? s.T - s.C : 0);
+    return launch_pdl(k_ep_gather_pack, dim3(row_grid(rows_hint < P ? rows_hint : P, num_sms)), dim3(kRowThreads), 0,
+                      stream, ws_ptrs(ws, L), (const uint4 *)x, src_token, s.T, s.E, G, s.C, S, (int)P, s.H / 8,
+                      (uint4 *)x_perm, (uint4 *)send_ovf, send_meta, p.starts);
 }
 
 // Receiving side: the local layout, its GEMM schedule in the local workspace,

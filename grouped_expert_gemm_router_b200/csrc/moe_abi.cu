@@ -41,6 +41,9 @@ int64_t ep_overflow_rows(const moe_shape &s, int G);
 size_t ep_workspace_bytes(const moe_shape &s, int G);
 cudaError_t launch_ep_pack(const moe_shape &s, int G, const void *x_perm, const WsLayout &L, void *ws, void *send_ovf,
                            int32_t *send_meta, void *ep_ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_gather_pack(const moe_shape &s, int G, const void *x, const int32_t *src_token, void *x_perm,
+                                  const WsLayout &L, void *ws, void *send_ovf, int32_t *send_meta, void *ep_ws,
+                                  int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_unpack_combine(const moe_shape &s, int G, const void *recv_back_ovf, const void *y,
                                      const int32_t *dest_row, const float *topk_w, void *out, void *ep_ws,
                                      cudaStream_t stream);
@@ -548,6 +551,23 @@ moe_status moe_ep_pack(const moe_shape *s, int32_t G, const void *x_perm, const 
     cudaError_t e = launch_ep_pack(*s, G, x_perm, L, const_cast<void *>(ws), send_ovf, send_meta, ep_ws, sms,
                                    (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_pack");
+}
+
+moe_status moe_ep_gather_pack(const moe_shape *s, int32_t G, const void *x, const int32_t *src_token, void *x_perm,
+                              void *ws, void *send_ovf, int32_t *send_meta, void *ep_ws, void *stream) {
+    moe_status st = check_ep(s, G);
+    if (st != MOE_OK) return st;
+    const bool no_ovf = ep_overflow_rows(*s, G) == 0;
+    if (!aligned(x, 16) || !aligned(src_token, 4) || !aligned_or_empty(x_perm, 16, s->C == 0) ||
+        !aligned_or_empty(send_ovf, 16, no_ovf) || !aligned(send_meta, 4) || !aligned(ep_ws, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    int sms = 0;
+    if ((st = device_info(&sms)) != MOE_OK) return st;
+    const WsLayout L = layout_of(s);
+    cudaError_t e = launch_ep_gather_pack(*s, G, x, src_token, x_perm, L, ws, send_ovf, send_meta, ep_ws, sms,
+                                          (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_gather_pack");
 }
 
 moe_status moe_ep_local_dispatch(const moe_shape *s, int32_t G, const int32_t *recv_meta, const void *recv_cap,

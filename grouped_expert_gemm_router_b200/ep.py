@@ -82,14 +82,20 @@ class CapAndSpillEP:
             moe.moe_workspace_init(L, self.ws_loc)
 
     # ---- phases -------------------------------------------------------------
-    def route_and_pack(self, x, w_router, bias, stream=None):
+    def route_and_pack(self, x, w_router, bias, stream=None, fused=True):
         """Routing and the capacity layout of this rank's tokens, then the
-        per-destination counts and overflow slots."""
+        per-destination counts and overflow slots (fused: the row copy writes
+        the overflow rows straight into the slots; else the row copy of every
+        permuted row, then the pack)."""
         s, b = self.shape, self.b
         moe.moe_route_dispatch(s, x, w_router, bias, b["logits"], b["topk_idx"], b["topk_w"], b["expert_counts"],
                                b["expert_offsets"], b["src_token"], b["dest_row"], self.ws, stream)
-        moe.moe_gather(s, x, b["src_token"], b["x_perm"], self.ws, stream)
-        moe.moe_ep_pack(s, self.G, b["x_perm"], self.ws, self.send_ovf, self.send_meta, self.ep_ws, stream)
+        if fused:
+            moe.moe_ep_gather_pack(s, self.G, x, b["src_token"], b["x_perm"], self.ws, self.send_ovf, self.send_meta,
+                                   self.ep_ws, stream)
+        else:
+            moe.moe_gather(s, x, b["src_token"], b["x_perm"], self.ws, stream)
+            moe.moe_ep_pack(s, self.G, b["x_perm"], self.ws, self.send_ovf, self.send_meta, self.ep_ws, stream)
 
     def exchange_in(self, all_to_all):
         """Pass 1 (capacity rows and counts), pass 2 (overflow slots)."""

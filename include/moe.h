@@ -470,6 +470,19 @@ MOE_API moe_status moe_ep_local_shape(const moe_shape *shape, int32_t G, moe_sha
 MOE_API moe_status moe_ep_pack(const moe_shape *shape, int32_t G, const void *x_perm, const void *ws,
                                void *send_ovf, int32_t *send_meta, void *ep_ws, void *stream);
 
+/* The row copy of step 1 and step 2 in one launch: x_perm's capacity slots
+ * filled from x by src_token (zero rows for unfilled slots), each overflow
+ * row copied from x straight into its destination's slot of send_ovf (so
+ * x_perm's overflow region is not written and may be as short as E*C rows),
+ * send_meta and the destination starts as moe_ep_pack writes them.  Replaces
+ * moe_gather + moe_ep_pack after moe_route_dispatch; x: device bf16 [T,H],
+ * src_token: from moe_route_dispatch; ws: the routing workspace (read: the
+ * capacity and overflow counts; its status word gets MOE_DEV_BAD_ROW for a
+ * row that does not fit a slot). */
+MOE_API moe_status moe_ep_gather_pack(const moe_shape *shape, int32_t G, const void *x, const int32_t *src_token,
+                                      void *x_perm, void *ws, void *send_ovf, int32_t *send_meta, void *ep_ws,
+                                      void *stream);
+
 /* Step 4.  ws_loc: a workspace of the local shape, initialised once
  * (moe_workspace_init with the local shape). */
 MOE_API moe_status moe_ep_local_dispatch(const moe_shape *shape, int32_t G, const int32_t *recv_meta,

@@ -185,16 +185,17 @@ def oracle_layer(orc, L, cfg, logits_gpu):
     return dict(idx=idx, w=w, d=d, x_perm=x_perm, h=h, y=y, out=out)
 
 
-def run_cap_and_spill_ep(dl, shape, G, fused_finish=True):
+def run_cap_and_spill_ep(dl, shape, G, fused_finish=True, fused_pack=True):
     """The two-pass expert-parallel layer on G ranks held by this process;
     rank r holds tokens [r T, (r+1) T) of the layer dl (fused_finish: the
-    unpack folded into the combine)."""
+    unpack folded into the combine; fused_pack: the row copy writing the
+    overflow rows straight into the send slots)."""
     from grouped_expert_gemm_router_b200.ep import CapAndSpillEP, exchange_in_process
     T, Eg = shape.T, shape.E // G
     ranks = [CapAndSpillEP(shape, G) for _ in range(G)]
     xs = [dl.x[r * T:(r + 1) * T] for r in range(G)]
     for r, ep in enumerate(ranks):
-        ep.route_and_pack(xs[r], dl.w_router, dl.bias)
+        ep.route_and_pack(xs[r], dl.w_router, dl.bias, fused=fused_pack)
     exchange_in_process(ranks, "exchange_in")
     for r, ep in enumerate(ranks):
         sl = slice(r * Eg, (r + 1) * Eg)

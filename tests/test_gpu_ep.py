@@ -132,6 +132,30 @@ def test_ep_unpack_combine_equals_unpack_then_combine(name, G):
         assert torch.equal(ep.b["out"], fused[r]), "rank %d" % r
 
 
+@pytest.mark.parametrize("name,G", [("decode_E64_k6_C16", 8), ("C0_all_overflow", 2), ("C_ge_T_no_overflow", 2)],
+                         ids=lambda v: str(v))
+def test_ep_gather_pack_equals_gather_then_pack(name, G):
+    """The row copy that writes overflow rows straight into the send slots
+    leaves the capacity rows, the slots and the counts sent ahead exactly as
+    the row copy followed by the pack does."""
+    from grouped_expert_gemm_router_b200.ep import CapAndSpillEP
+    cfg, _ = CASES[name]
+    L = synth.make_layer(cfg.with_(T=cfg.T * G))
+    dl = DeviceLayer(L)
+    shape = _shape(cfg)
+    for r in range(G):
+        x = dl.x[r * cfg.T:(r + 1) * cfg.T]
+        got, ref = CapAndSpillEP(shape, G), CapAndSpillEP(shape, G)
+        for ep, fused in ((got, True), (ref, False)):
+            ep.send_ovf.zero_()
+            ep.route_and_pack(x, dl.w_router, dl.bias, fused=fused)
+        torch.cuda.synchronize()
+        assert moe.moe_read_status(got.ws) == 0
+        assert torch.equal(got.send_meta, ref.send_meta), r
+        assert torch.equal(got.send_ovf, ref.send_ovf), r
+        assert torch.equal(got.b["x_perm"][:got.cap_rows], ref.b["x_perm"][:ref.cap_rows]), r
+
+
 def test_ep_rejects_uncapped_layout():
     cfg = CASES["E16_k4_C24_F384"][0]
     with pytest.raises(moe.MoeError):

@@ -81,7 +81,8 @@ def test_random_expert_parallel_matches_single_gpu(cfg, G):
     dl = DeviceLayer(L)
     if cfg.C > 0:
         shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k, C=cfg.C, capacity=True)
-        ranks, xs = run_cap_and_spill_ep(dl, shape, G, fused_finish=bool(cfg.seed % 2))
+        ranks, xs = run_cap_and_spill_ep(dl, shape, G, fused_finish=bool(cfg.seed % 2),
+                                              fused_pack=bool(cfg.T % 2))
     else:
         shape = moe.make_shape(cfg.T, cfg.H, cfg.F, cfg.E, cfg.k)
         ranks, xs = run_direct_ep(dl, shape, G, fused_return=bool(cfg.seed % 2), fused_plan=bool(cfg.T % 2))
