@@ -84,6 +84,10 @@ constexpr uint32_t kCtrlBytes = 3072;
 constexpr uint32_t kSmemBytes = 226 * 1024;
 constexpr uint32_t kEpiStageBytes = 512;      // per epilogue warp: one 8-row x 32-feature bf16 block
 constexpr uint32_t kRingBytes = (kSmemBytes - 1024 - kCtrlBytes - 16 * kEpiStageBytes) & ~1023u;
+// The largest token stages still leave room for a weight stage of both
+// accumulators, so the ring geometry below never runs out of space (its
+// unsigned arithmetic relies on it).
+static_assert((uint32_t)kMaxBStages * kTileRows * kBRowBytes + 2u * kATile <= kRingBytes, "ring too small");
 static_assert(3 * 2 * kATile + 3 * kTileRows * kBRowBytes <= kRingBytes,
               "three weight stages and three token stages of 256 rows must fit");
 constexpr int kEpiWarp0 = 3;                   // warps 0-2 load and issue, 3-10 drain tensor memory
