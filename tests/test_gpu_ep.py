@@ -34,6 +34,8 @@ CASES = {
     "C_ge_T_no_overflow": (synth.LayerConfig("ep", 64, 128, 128, 8, 2, C=64, seed=44), (2, 8)),
     # local experts of several row tiles with ragged tails
     "several_tiles_E4_k2": (synth.LayerConfig("ep", 700, 256, 256, 4, 2, C=200, alpha=0.3, seed=45), (2,)),
+    # the most experts a layer may have: 256, 128 or 32 per rank
+    "E256_k8_C2": (synth.LayerConfig("ep", 48, 128, 128, 256, 8, C=2, alpha=0.8, seed=46), (1, 2, 8)),
 }
 
 

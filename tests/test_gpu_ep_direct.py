@@ -27,6 +27,8 @@ CASES = {
     "E8_k2_skew": (synth.LayerConfig("epd", 96, 128, 256, 8, 2, alpha=3.0, seed=53), (2, 8)),
     "k_equals_E": (synth.LayerConfig("epd", 40, 128, 128, 4, 4, seed=54), (2, 4)),
     "several_tiles_E4_k2": (synth.LayerConfig("epd", 700, 256, 256, 4, 2, alpha=0.3, seed=55), (2,)),
+    # the most experts a layer may have: 256, 128 or 32 per rank
+    "E256_k8": (synth.LayerConfig("epd", 48, 128, 128, 256, 8, alpha=0.8, seed=56), (1, 2, 8)),
 }
 
 
