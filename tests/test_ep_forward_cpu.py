@@ -91,3 +91,20 @@ def test_peer_store_forward_order(monkeypatch):
     ep.forward(None, None, None, None, None, None, fused_return=False)
     assert calls == ["route", "all_gather", "plan_and_dispatch", "barrier", "experts", "send_back", "barrier",
                      "finish"]
+
+
+def test_peer_store_fp8_forward_order(monkeypatch):
+    """The fp8 layer: the rows are quantized by the dispatch launch itself (no
+    separate token quantization), then the fp8 experts with the fused return."""
+    import torch.distributed as dist
+    ep = DirectEP(moe.make_shape(40, 128, 128, 16, 3), G, 0, device="cpu", fp8=True)
+    calls = []
+    for name in ("route", "quantize_tokens", "plan_and_dispatch", "experts_fp8_and_return", "finish"):
+        monkeypatch.setattr(ep, name, (lambda n: (lambda *a, **k: calls.append(n)))(name))
+    monkeypatch.setattr(dist, "all_gather_into_tensor", lambda out, inp, group=None: calls.append("all_gather"))
+    monkeypatch.setattr(dist, "all_reduce", lambda t, group=None: calls.append("barrier"))
+    ep._flag, ep._group = torch.zeros(1, dtype=torch.int32), None
+    ep.forward_fp8(None, None, None, None, None, None, None, None, None)
+    assert calls == ["route", "all_gather", "plan_and_dispatch", "barrier", "experts_fp8_and_return", "barrier",
+                     "finish"]
+
